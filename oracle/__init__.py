@@ -1,0 +1,192 @@
+"""CPU oracle for the depthwise-convolution hot path (fp64, plain loops).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU baseline
+import this package.  The product path (the CUDA library and its Python binding) never
+imports it, and it imports nothing from the product.
+
+The arithmetic lives in ``dwconv_oracle.c`` (compiled here with gcc into
+``oracle/_build/liboracle.so``); this module only compiles it, converts numpy arrays to
+float64 and calls it.  Every function follows the definitions stated in that file, taken
+from parakeet.cpp PR #102 ("What changes": the depthwise conv as a sum over the padded
+input) and NeMo PR #16114 ("What does this PR do ?": conv0 -> ReLU -> masking -> conv_dw1,
+with pre/post masking and causal padding).
+
+Parity is pinned by ``tests/test_oracle_pins.py`` (a second formulation by im2col + matmul,
+torch's float64 CPU convolutions, hand-worked golden values and invariants).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dwconv_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lock = threading.Lock()
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I = ctypes.POINTER(ctypes.c_int32)
+_L = ctypes.c_int64
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle with gcc (-O2, strict IEEE: no fast-math, no FMA contraction) and OpenMP."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+           "-ffp-contract=off", "-o", tmp, src]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _dp(a):
+    return a.ctypes.data_as(_D) if a is not None else None
+
+
+def _ip(a):
+    return a.ctypes.data_as(_I) if a is not None else None
+
+
+def _lens(lengths, B):
+    if lengths is None:
+        return None
+    a = np.ascontiguousarray(lengths, dtype=np.int32)
+    if a.shape != (B,):
+        raise ValueError("lengths must have shape [B]")
+    return a
+
+
+def subsample_out_shape(T, F, causal):
+    """(T4, F4) of the two stride-2 stages (time pads 1|1 or 2|0, frequency pads 1|1)."""
+    def s2(n):
+        return (n + 2 - 3) // 2 + 1 if n >= 1 else 0
+    return s2(s2(T)), s2(s2(F))
+
+
+class Oracle:
+    """The oracle's functions, bound to one compiled copy of ``dwconv_oracle.c``."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_dwconv1d_fwd.argtypes = [_D, _D, _D, _I, _L, _L, _L, _L, _L, _D]
+        lib.oracle_dwconv1d_bwd_dx.argtypes = [_D, _D, _I, _L, _L, _L, _L, _L, _D]
+        lib.oracle_dwconv1d_bwd_dw.argtypes = [_D, _D, _I, _L, _L, _L, _L, _L, _D, _D]
+        lib.oracle_dw_subsample_fwd.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L,
+                                                ctypes.c_int, _D, _I]
+        for f in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_dx", "oracle_dwconv1d_bwd_dw",
+                  "oracle_dw_subsample_fwd"):
+            getattr(lib, f).restype = ctypes.c_int
+        self.lib = lib
+        self.path = lib_path
+
+    def num_threads(self) -> int:
+        """OpenMP threads the oracle runs with."""
+        return int(self.lib.oracle_num_threads())
+
+    def dwconv1d_fwd(self, x, w, bias, lengths, pad_left):
+        """y[b,t,c] = [t<len_b] (bias[c] + sum_k xpad[b,t+k,c] w[k,c]); x [B,T,C], w [K,C]."""
+        x = _f64(x); w = _f64(w)
+        B, T, C = x.shape
+        K = w.shape[0]
+        assert w.shape == (K, C)
+        b = _f64(bias) if bias is not None else None
+        ln = _lens(lengths, B)
+        y = np.empty((B, T, C), dtype=np.float64)
+        rc = self.lib.oracle_dwconv1d_fwd(_dp(x), _dp(w), _dp(b), _ip(ln),
+                                          B, T, C, K, int(pad_left), _dp(y))
+        if rc:
+            raise ValueError(f"oracle_dwconv1d_fwd rejected its arguments (rc={rc})")
+        return y
+
+    def dwconv1d_bwd_dx(self, dy, w, lengths, pad_left):
+        """Data gradient of ``dwconv1d_fwd`` (the transpose of the forward map)."""
+        dy = _f64(dy); w = _f64(w)
+        B, T, C = dy.shape
+        K = w.shape[0]
+        assert w.shape == (K, C)
+        ln = _lens(lengths, B)
+        dx = np.empty((B, T, C), dtype=np.float64)
+        rc = self.lib.oracle_dwconv1d_bwd_dx(_dp(dy), _dp(w), _ip(ln),
+                                             B, T, C, K, int(pad_left), _dp(dx))
+        if rc:
+            raise ValueError(f"oracle_dwconv1d_bwd_dx rejected its arguments (rc={rc})")
+        return dx
+
+    def dwconv1d_bwd_dw(self, x, dy, K, lengths, pad_left):
+        """Weight and bias gradients: returns (dW [K,C], dbias [C])."""
+        x = _f64(x); dy = _f64(dy)
+        B, T, C = x.shape
+        assert dy.shape == x.shape
+        ln = _lens(lengths, B)
+        dw = np.empty((int(K), C), dtype=np.float64)
+        db = np.empty((C,), dtype=np.float64)
+        rc = self.lib.oracle_dwconv1d_bwd_dw(_dp(x), _dp(dy), _ip(ln),
+                                             B, T, C, int(K), int(pad_left), _dp(dw), _dp(db))
+        if rc:
+            raise ValueError(f"oracle_dwconv1d_bwd_dw rejected its arguments (rc={rc})")
+        return dw, db
+
+    def dw_subsample_fwd(self, mel, w0, b0, w1, b1, lengths, causal):
+        """Fused subsampler front in fp64: returns (out [B,T4,F4,C], out_lengths [B])."""
+        mel = _f64(mel)
+        B, T, F = mel.shape
+        w0 = _f64(w0); w1 = _f64(w1); b0 = _f64(b0); b1 = _f64(b1)
+        C = w0.shape[-1]
+        assert w0.shape == (3, 3, C) and w1.shape == (3, 3, C)
+        assert b0.shape == (C,) and b1.shape == (C,)
+        T4, F4 = subsample_out_shape(T, F, causal)
+        ln = _lens(lengths, B)
+        out = np.empty((B, T4, F4, C), dtype=np.float64)
+        ol = np.empty((B,), dtype=np.int32)
+        rc = self.lib.oracle_dw_subsample_fwd(_dp(mel), _dp(w0), _dp(b0), _dp(w1), _dp(b1),
+                                              _ip(ln), B, T, F, C, int(bool(causal)),
+                                              _dp(out), _ip(ol))
+        if rc:
+            raise ValueError(f"oracle_dw_subsample_fwd rejected its arguments (rc={rc})")
+        return out, ol
+
+
+def default() -> Oracle:
+    """The oracle compiled from this package's source (built on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(build())
+    return _default
+
+
+_default = None
+
+
+def num_threads() -> int:
+    return default().num_threads()
+
+
+def dwconv1d_fwd(x, w, bias, lengths, pad_left):
+    return default().dwconv1d_fwd(x, w, bias, lengths, pad_left)
+
+
+def dwconv1d_bwd_dx(dy, w, lengths, pad_left):
+    return default().dwconv1d_bwd_dx(dy, w, lengths, pad_left)
+
+
+def dwconv1d_bwd_dw(x, dy, K, lengths, pad_left):
+    return default().dwconv1d_bwd_dw(x, dy, K, lengths, pad_left)
+
+
+def dw_subsample_fwd(mel, w0, b0, w1, b1, lengths, causal):
+    return default().dw_subsample_fwd(mel, w0, b0, w1, b1, lengths, causal)

@@ -1,0 +1,242 @@
+/*
+ * CPU oracle for the depthwise-convolution hot path of a conformer speech encoder.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU
+ * baseline may load this file's library.  The CUDA library never links, includes or
+ * calls it, and it shares no code with the CUDA library.
+ *
+ * Plain loops in IEEE double, no blocking, no fusion, no reordering beyond what the
+ * definitions state.  Inputs are the stored values widened to double (bf16 values are
+ * exactly representable).  OpenMP runs only over independent outputs, so every sum is
+ * taken in the same serial order whatever the thread count.
+ *
+ * Sources of the definitions:
+ *  - parakeet.cpp PR #102, "perf: faster GPU decode: one SSM_CONV for the depthwise
+ *    conv, less host work per step", section "What changes": the depthwise conv is a
+ *    sum over k of x[t + k, c] * w[k, c] over the input padded to T + K - 1 frames,
+ *    NeMo's conv for the same left padding, causal or symmetric.
+ *  - NeMo PR #16114, "Use Fused Kernels for Depthwise Striding Subsampler", section
+ *    "What does this PR do ?": mel [B,T,F,1] -> conv0 [B,T/2,F/2,256] -> ReLU -> masking
+ *    -> conv_dw1 [B,T/4,F/4,256]; the depthwise kernel fuses pre- and post-masking and
+ *    the causal padding; backward kernels exist (data and weight gradients).
+ *
+ * Readings where the pages are silent (all masks use the per-item length len_b,
+ * clamped to [0, T]):
+ *  - a frame t >= len_b of the conv input counts as zero before the conv, and output
+ *    frames t >= len_b are zero after it;
+ *  - the data gradient applies the same output mask to dy before propagating it;
+ *  - subsampler: mel frames t >= len_b count as zero; conv0 rows i >= ceil(len_b/2)
+ *    and conv_dw1 rows i >= ceil(len_b/4) are zero; time padding 1|1 (causal 2|0) and
+ *    frequency padding 1|1 for both convs; padding values are zero.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static int64_t clamp_len(const int32_t *lengths, int64_t b, int64_t T)
+{
+    if (lengths == NULL) return T;
+    int64_t L = lengths[b];
+    if (L < 0) L = 0;
+    if (L > T) L = T;
+    return L;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * xpad[b, j, c] for j in [0, T + K - 1): the input shifted right by pad_left frames,
+ * with frames outside [0, len_b) of the original sequence reading as zero.
+ */
+static double xpad_at(const double *x, int64_t b, int64_t j, int64_t c,
+                      int64_t T, int64_t C, int64_t pad_left, int64_t L)
+{
+    int64_t s = j - pad_left;          /* frame of the unpadded input */
+    if (s < 0 || s >= L) return 0.0;   /* padding, or a frame at/after len_b */
+    return x[(b * T + s) * C + c];
+}
+
+/*
+ * Forward: y[b,t,c] = [t < len_b] * (bias[c] + sum_{k<K} xpad[b,t+k,c] * w[k,c]).
+ * x, y: [B][T][C]; w: [K][C]; bias: [C] or NULL; lengths: [B] or NULL (no mask).
+ */
+int oracle_dwconv1d_fwd(const double *x, const double *w, const double *bias,
+                        const int32_t *lengths, int64_t B, int64_t T, int64_t C,
+                        int64_t K, int64_t pad_left, double *y)
+{
+    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return 1;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        #pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t c = 0; c < C; ++c) {
+                double acc = 0.0;
+                if (t < L) {
+                    acc = bias ? bias[c] : 0.0;
+                    for (int64_t k = 0; k < K; ++k)
+                        acc += xpad_at(x, b, t + k, c, T, C, pad_left, L) * w[k * C + c];
+                }
+                y[(b * T + t) * C + c] = acc;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Data gradient, as the transpose of the forward map: with dz[b,t,c] = [t < len_b] dy[b,t,c],
+ * every term xpad[b,t+k,c] * w[k,c] of y[b,t,c] that reads the real frame s = t + k - pad_left
+ * (0 <= s < len_b) sends dz[b,t,c] * w[k,c] back to dx[b,s,c].  Summation order per dx
+ * element: t ascending, then k ascending.
+ */
+int oracle_dwconv1d_bwd_dx(const double *dy, const double *w, const int32_t *lengths,
+                           int64_t B, int64_t T, int64_t C, int64_t K, int64_t pad_left,
+                           double *dx)
+{
+    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return 1;
+    const int64_t CB = 64;                         /* channels per independent task */
+    const int64_t ncb = (C + CB - 1) / CB;
+    memset(dx, 0, sizeof(double) * (size_t)(B * T * C));
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t cb = 0; cb < ncb; ++cb) {
+            const int64_t L = clamp_len(lengths, b, T);
+            const int64_t c0 = cb * CB, c1 = (c0 + CB < C) ? c0 + CB : C;
+            for (int64_t t = 0; t < L; ++t) {
+                for (int64_t k = 0; k < K; ++k) {
+                    const int64_t s = t + k - pad_left;
+                    if (s < 0 || s >= L) continue;
+                    for (int64_t c = c0; c < c1; ++c)
+                        dx[(b * T + s) * C + c] += dy[(b * T + t) * C + c] * w[k * C + c];
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Weight and bias gradients: dW[k,c] = sum_{b,t} dz[b,t,c] * xpad[b,t+k,c] and
+ * dbias[c] = sum_{b,t} dz[b,t,c], with dz[b,t,c] = [t < len_b] dy[b,t,c].
+ * Summation order per output: b ascending, then t ascending.  dbias may be NULL.
+ */
+int oracle_dwconv1d_bwd_dw(const double *x, const double *dy, const int32_t *lengths,
+                           int64_t B, int64_t T, int64_t C, int64_t K, int64_t pad_left,
+                           double *dw, double *dbias)
+{
+    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return 1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        double db = 0.0;
+        for (int64_t k = 0; k < K; ++k) dw[k * C + c] = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            const int64_t L = clamp_len(lengths, b, T);
+            for (int64_t t = 0; t < T; ++t) {
+                const double dz = (t < L) ? dy[(b * T + t) * C + c] : 0.0;
+                db += dz;
+                for (int64_t k = 0; k < K; ++k)
+                    dw[k * C + c] += dz * xpad_at(x, b, t + k, c, T, C, pad_left, L);
+            }
+        }
+        if (dbias) dbias[c] = db;
+    }
+    return 0;
+}
+
+/* Output size of a 3-tap, stride-2 convolution over n frames padded by p0|p1. */
+static int64_t s2_out(int64_t n, int64_t p0, int64_t p1)
+{
+    int64_t m = n + p0 + p1 - 3;
+    if (m < 0) return 0;
+    return m / 2 + 1;
+}
+
+static int64_t ceil_half(int64_t n) { return (n + 1) / 2; }
+
+/*
+ * Fused depthwise-striding subsampler front, computed stage by stage:
+ *   melpad  = mel (frames t >= len_b zeroed) padded by Pt|Pb in time and 1|1 in frequency
+ *   h       = ReLU(b0[c] + sum_{p,q<3} melpad[2i+p, 2j+q] * w0[p,q,c]); rows i >= ceil(len_b/2) -> 0
+ *   hpad    = h padded by Pt|Pb in time and 1|1 in frequency, zeros
+ *   out     = b1[c] + sum_{p,q<3} hpad[2i+p, 2j+q, c] * w1[p,q,c];     rows i >= ceil(len_b/4) -> 0
+ * with Pt|Pb = 1|1 (symmetric) or 2|0 (causal).
+ * mel: [B][T][F]; w0, w1: [3][3][C]; b0, b1: [C]; out: [B][T4][F4][C];
+ * out_lengths: [B] or NULL, receives ceil(ceil(len_b/2)/2).
+ */
+int oracle_dw_subsample_fwd(const double *mel, const double *w0, const double *b0,
+                            const double *w1, const double *b1, const int32_t *lengths,
+                            int64_t B, int64_t T, int64_t F, int64_t C, int causal,
+                            double *out, int32_t *out_lengths)
+{
+    if (B < 0 || T < 0 || F < 1 || C < 1) return 1;
+    const int64_t Pt = causal ? 2 : 1, Pb = causal ? 0 : 1;
+    const int64_t T2 = s2_out(T, Pt, Pb), F2 = s2_out(F, 1, 1);
+    const int64_t T4 = s2_out(T2, Pt, Pb), F4 = s2_out(F2, 1, 1);
+    const int64_t TP = T + Pt + Pb, FP = F + 2;          /* melpad extent */
+    const int64_t HT = T2 + Pt + Pb, HF = F2 + 2;        /* hpad extent */
+    double *melpad = (double *)malloc(sizeof(double) * (size_t)(TP * FP));
+    double *hpad = (double *)malloc(sizeof(double) * (size_t)(HT * HF * C));
+    if ((TP * FP > 0 && !melpad) || (HT * HF * C > 0 && !hpad)) {
+        free(melpad);
+        free(hpad);
+        return 2;
+    }
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        const int64_t L2 = ceil_half(L), L4 = ceil_half(L2);
+        if (out_lengths) out_lengths[b] = (int32_t)L4;
+
+        /* melpad: zero padding, and zero at frames t >= len_b */
+        for (int64_t r = 0; r < TP; ++r)
+            for (int64_t f = 0; f < FP; ++f) {
+                const int64_t t = r - Pt, ff = f - 1;
+                melpad[r * FP + f] = (t >= 0 && t < L && ff >= 0 && ff < F)
+                                         ? mel[(b * T + t) * F + ff] : 0.0;
+            }
+
+        /* conv0 + bias + ReLU + row mask, written into the interior of hpad */
+        memset(hpad, 0, sizeof(double) * (size_t)(HT * HF * C));
+        #pragma omp parallel for schedule(static)
+        for (int64_t i = 0; i < T2; ++i) {
+            for (int64_t j = 0; j < F2; ++j) {
+                for (int64_t c = 0; c < C; ++c) {
+                    double a = b0[c];
+                    for (int64_t p = 0; p < 3; ++p)
+                        for (int64_t q = 0; q < 3; ++q)
+                            a += melpad[(2 * i + p) * FP + (2 * j + q)] * w0[(p * 3 + q) * C + c];
+                    double hv = a > 0.0 ? a : 0.0;          /* ReLU */
+                    if (i >= L2) hv = 0.0;                  /* mask beyond ceil(len/2) */
+                    hpad[((i + Pt) * HF + (j + 1)) * C + c] = hv;
+                }
+            }
+        }
+
+        /* conv_dw1 (depthwise) + bias + row mask */
+        #pragma omp parallel for schedule(static)
+        for (int64_t i = 0; i < T4; ++i) {
+            for (int64_t j = 0; j < F4; ++j) {
+                for (int64_t c = 0; c < C; ++c) {
+                    double a = b1[c];
+                    for (int64_t p = 0; p < 3; ++p)
+                        for (int64_t q = 0; q < 3; ++q)
+                            a += hpad[((2 * i + p) * HF + (2 * j + q)) * C + c] * w1[(p * 3 + q) * C + c];
+                    if (i >= L4) a = 0.0;                   /* mask beyond ceil(len/4) */
+                    out[((b * T4 + i) * F4 + j) * C + c] = a;
+                }
+            }
+        }
+    }
+    free(melpad);
+    free(hpad);
+    return 0;
+}

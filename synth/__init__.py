@@ -1,0 +1,118 @@
+"""Seeded synthetic inputs for the depthwise-conv hot path.
+
+This module is shared by the CPU oracle's tests and by the CUDA path's tests and
+benchmark.  It only draws numbers: it holds none of the convolution arithmetic.
+
+Recipe (one ``numpy.random.default_rng(seed)`` per workload):
+
+* conv1d: draw ``x`` ~ N(0, 1), then ``w[K, C]`` ~ N(0, 1/K), then ``bias[C]``
+  ~ N(0, 0.1), then ``lengths[B]`` uniform on the inclusive integer range, then
+  (backward workloads only) ``dy`` ~ N(0, 1).  N(m, v) names the variance ``v``.
+* subsampler: draw ``mel[B, T, F]`` ~ N(0, 1), then ``w0[3, 3, C]`` ~ N(0, 1/9),
+  ``b0`` ~ N(0, 0.1), ``w1[3, 3, C]`` ~ N(0, 1/9), ``b1`` ~ N(0, 0.1), then
+  ``lengths``.  Mel frames at ``t >= lengths[b]`` are then set to zero, so a
+  reading that masks the mel before conv0 and one that does not agree.
+* bf16 workloads round every drawn value (data and weights) to the nearest
+  bf16-representable float32, ties to even, so the stored bf16 tensor and the
+  float32 weights hold exactly the values the oracle reads.
+
+All arrays are float32 (values) or int32 (lengths), C-contiguous, channels last.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "bf16_round",
+    "bf16_bits",
+    "conv1d_inputs",
+    "subsample_inputs",
+    "symmetric_pad_left",
+    "WORKLOADS",
+]
+
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bf16-representable float32 (ties to even)."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).reshape(a.shape)
+
+
+def bf16_bits(a: np.ndarray) -> np.ndarray:
+    """The upper 16 bits of bf16-representable float32 values, as uint16 (the stored bf16)."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def symmetric_pad_left(K: int) -> int:
+    """Left pad of the symmetric ('same') mode: floor((K-1)/2); the extra pad of an even K goes right."""
+    return (K - 1) // 2
+
+
+def _normal(rng, shape, var):
+    return (rng.standard_normal(shape, dtype=np.float32) * np.float32(np.sqrt(var))).astype(np.float32)
+
+
+def conv1d_inputs(B, T, C, K, *, dtype="bf16", len_range=None, seed=0, with_dy=False):
+    """Inputs of one depthwise conv1d workload.
+
+    Returns a dict with ``x[B,T,C]``, ``w[K,C]``, ``bias[C]`` (float32, rounded to
+    bf16 values when ``dtype == 'bf16'``), ``lengths[B]`` (int32, or None when
+    ``len_range`` is None: no masking) and, with ``with_dy``, ``dy[B,T,C]``.
+    """
+    rng = np.random.default_rng(seed)
+    x = _normal(rng, (B, T, C), 1.0)
+    w = _normal(rng, (K, C), 1.0 / K)
+    bias = _normal(rng, (C,), 0.1)
+    lengths = None
+    if len_range is not None:
+        lo, hi = len_range
+        lengths = rng.integers(lo, hi + 1, size=B).astype(np.int32)
+    out = {"x": x, "w": w, "bias": bias, "lengths": lengths}
+    if with_dy:
+        out["dy"] = _normal(rng, (B, T, C), 1.0)
+    if dtype == "bf16":
+        for k in ("x", "w", "bias", "dy"):
+            if k in out:
+                out[k] = bf16_round(out[k])
+    elif dtype != "f32":
+        raise ValueError(f"unknown dtype {dtype!r}")
+    return out
+
+
+def subsample_inputs(B, T, F, C, *, len_range, seed=3, zero_beyond_len=True):
+    """Inputs of one fused-subsampler workload: ``mel[B,T,F]``, ``w0,w1[3,3,C]``, ``b0,b1[C]``, ``lengths[B]``."""
+    rng = np.random.default_rng(seed)
+    mel = _normal(rng, (B, T, F), 1.0)
+    w0 = _normal(rng, (3, 3, C), 1.0 / 9.0)
+    b0 = _normal(rng, (C,), 0.1)
+    w1 = _normal(rng, (3, 3, C), 1.0 / 9.0)
+    b1 = _normal(rng, (C,), 0.1)
+    lo, hi = len_range
+    lengths = rng.integers(lo, hi + 1, size=B).astype(np.int32)
+    if zero_beyond_len:
+        for b in range(B):
+            mel[b, max(0, int(lengths[b])):, :] = 0.0
+    return {"mel": mel, "w0": w0, "b0": b0, "w1": w1, "b1": b1, "lengths": lengths}
+
+
+# The five workloads, shaped like the ones the pages run (the parakeet conformer
+# conv at K=9, a kernel-width sweep, NeMo's depthwise-striding subsampler and a
+# training-size backward).  Seed = workload index.
+WORKLOADS = {
+    "fwd_f32_small": dict(kind="conv1d", B=1, T=200, C=256, K=9, dtype="f32", len_range=None,
+                          pad="symmetric", seed=0),
+    "fwd_bf16_B16_T1500_C512_K9": dict(kind="conv1d", B=16, T=1500, C=512, K=9, dtype="bf16",
+                                       len_range=(750, 1500), pad="symmetric", seed=1),
+    "fwd_bf16_causal_sweep": dict(kind="conv1d", B=32, T=750, C=1024, Ks=(3, 4, 5, 9, 15),
+                                  dtype="bf16", len_range=(375, 750), pad="causal", seed=2,
+                                  odd_case=dict(C=520, K=7)),
+    "subsample_B16_T3000_F80_C256": dict(kind="subsample", B=16, T=3000, F=80, C=256,
+                                         len_range=(1500, 3000), seed=3),
+    "bwd_bf16_B32_T1500_C1024_K9": dict(kind="conv1d_bwd", B=32, T=1500, C=1024, K=9,
+                                        dtype="bf16", len_range=(750, 1500), pad="symmetric",
+                                        seed=4),
+}

@@ -1,0 +1,222 @@
+"""Independent formulations and invariant checks that pin the CPU oracle.
+
+Nothing here calls the oracle's C code: these are second and third ways to compute
+the same quantities (explicit im2col + matmul, a dense per-channel band matrix, and
+torch's float64 CPU convolutions with autograd), written from the definitions:
+
+* parakeet.cpp PR #102, "What changes": the depthwise conv is the sum over k of
+  x[t+k, c] * w[k, c] over the input padded to T + K - 1 frames; the old graph computed
+  the same conv as im2col + mul_mat.
+* NeMo PR #16114, "What does this PR do ?": conv0 (3x3, stride 2, 1 -> C) -> ReLU ->
+  masking -> conv_dw1 (depthwise 3x3, stride 2), with pre/post masking and causal padding.
+
+``pin_battery(o)`` runs a quick selection of every pin against an ``oracle.Oracle`` and
+returns the list of failures; the mutation test uses it to show that planted mistakes in
+the oracle are caught.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as Fnn
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def clamp_lengths(lengths, B, T):
+    if lengths is None:
+        return [T] * B
+    return [min(max(int(v), 0), T) for v in lengths]
+
+
+# ----------------------------------------------------------------------------------
+# conv1d: second formulation, explicit im2col + matmul (the old parakeet path)
+# ----------------------------------------------------------------------------------
+def im2col_fwd(x, w, bias, lengths, pad_left):
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w, np.float64)
+    B, T, C = x.shape
+    K = w.shape[0]
+    pad_right = K - 1 - pad_left
+    Ls = clamp_lengths(lengths, B, T)
+    y = np.zeros((B, T, C))
+    for b in range(B):
+        xm = x[b].copy()
+        xm[Ls[b]:] = 0.0
+        xp = np.concatenate([np.zeros((pad_left, C)), xm, np.zeros((pad_right, C))], axis=0)
+        for c in range(C):
+            cols = np.stack([xp[t:t + K, c] for t in range(T)], axis=0) if T else np.zeros((0, K))
+            y[b, :, c] = cols @ w[:, c] + (0.0 if bias is None else float(bias[c]))
+        y[b, Ls[b]:] = 0.0
+    return y
+
+
+def im2col_dw(x, dy, K, lengths, pad_left):
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    B, T, C = x.shape
+    pad_right = K - 1 - pad_left
+    Ls = clamp_lengths(lengths, B, T)
+    dw = np.zeros((K, C))
+    db = np.zeros(C)
+    for b in range(B):
+        xm = x[b].copy()
+        xm[Ls[b]:] = 0.0
+        dz = dy[b].copy()
+        dz[Ls[b]:] = 0.0
+        xp = np.concatenate([np.zeros((pad_left, C)), xm, np.zeros((pad_right, C))], axis=0)
+        for c in range(C):
+            cols = np.stack([xp[t:t + K, c] for t in range(T)], axis=0) if T else np.zeros((0, K))
+            dw[:, c] += cols.T @ dz[:, c]
+        db += dz.sum(axis=0)
+    return dw, db
+
+
+def band_matrix(wc, T, pad_left):
+    """Dense T x T matrix A with (A @ x)[t] = sum_k x[t + k - pad_left] * wc[k] (zero outside)."""
+    K = wc.shape[0]
+    A = np.zeros((T, T))
+    for t in range(T):
+        for s in range(T):
+            k = s - t + pad_left
+            if 0 <= k < K:
+                A[t, s] = wc[k]
+    return A
+
+
+def band_dx(dy, w, lengths, pad_left):
+    """dx = M A^T M dy per channel: the data gradient as the transpose of the forward matrix."""
+    dy = np.asarray(dy, np.float64)
+    w = np.asarray(w, np.float64)
+    B, T, C = dy.shape
+    Ls = clamp_lengths(lengths, B, T)
+    dx = np.zeros_like(dy)
+    for b in range(B):
+        m = (np.arange(T) < Ls[b]).astype(np.float64)
+        for c in range(C):
+            A = band_matrix(w[:, c], T, pad_left)
+            dx[b, :, c] = m * (A.T @ (m * dy[b, :, c]))
+    return dx
+
+
+# ----------------------------------------------------------------------------------
+# third formulation: torch float64 CPU convolutions + autograd (a library routine)
+# ----------------------------------------------------------------------------------
+def torch_conv1d_all(x, w, bias, dy, lengths, pad_left):
+    x = torch.tensor(np.asarray(x, np.float64), requires_grad=True)
+    w_t = torch.tensor(np.asarray(w, np.float64), requires_grad=True)
+    B, T, C = x.shape
+    K = w_t.shape[0]
+    b_t = torch.tensor(np.asarray(bias, np.float64) if bias is not None else np.zeros(C),
+                       requires_grad=True)
+    Ls = clamp_lengths(lengths, B, T)
+    mask = (torch.arange(T)[None, :] < torch.tensor(Ls)[:, None]).double()[:, :, None]
+    inp = Fnn.pad((x * mask).permute(0, 2, 1), (pad_left, K - 1 - pad_left))
+    y = Fnn.conv1d(inp, w_t.t().unsqueeze(1), b_t, groups=C).permute(0, 2, 1) * mask
+    dy_t = torch.tensor(np.asarray(dy, np.float64))
+    (y * dy_t).sum().backward()
+    return (y.detach().numpy(), x.grad.numpy(), w_t.grad.numpy(), b_t.grad.numpy())
+
+
+def torch_subsample(mel, w0, b0, w1, b1, lengths, causal):
+    mel = torch.tensor(np.asarray(mel, np.float64))
+    B, T, F = mel.shape
+    C = np.asarray(w0).shape[-1]
+    pt, pb = (2, 0) if causal else (1, 1)
+    Ls = clamp_lengths(lengths, B, T)
+    m0 = (torch.arange(T)[None, :] < torch.tensor(Ls)[:, None]).double()
+    inp = Fnn.pad((mel * m0[:, :, None])[:, None], (1, 1, pt, pb))
+    W0 = torch.tensor(np.asarray(w0, np.float64)).permute(2, 0, 1)[:, None]
+    W1 = torch.tensor(np.asarray(w1, np.float64)).permute(2, 0, 1)[:, None]
+    h = torch.relu(Fnn.conv2d(inp, W0, torch.tensor(np.asarray(b0, np.float64)), stride=2))
+    T2 = h.shape[2]
+    L2 = [(v + 1) // 2 for v in Ls]
+    m2 = (torch.arange(T2)[None, :] < torch.tensor(L2)[:, None]).double()[:, None, :, None]
+    h = h * m2
+    o = Fnn.conv2d(Fnn.pad(h, (1, 1, pt, pb)), W1, torch.tensor(np.asarray(b1, np.float64)),
+                   stride=2, groups=C)
+    T4 = o.shape[2]
+    L4 = [(v + 1) // 2 for v in L2]
+    m4 = (torch.arange(T4)[None, :] < torch.tensor(L4)[:, None]).double()[:, None, :, None]
+    o = o * m4
+    return o.permute(0, 2, 3, 1).numpy(), np.array(L4, dtype=np.int32)
+
+
+def load_golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def rel_err(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    if a.size == 0:
+        return 0.0
+    scale = max(np.max(np.abs(b)), 1e-300)
+    return float(np.max(np.abs(a - b)) / scale)
+
+
+# ----------------------------------------------------------------------------------
+# a quick battery of every kind of pin, for the mutation test
+# ----------------------------------------------------------------------------------
+def pin_battery(o):
+    """Run a fast selection of pins against oracle ``o``; returns a list of failure strings."""
+    fails = []
+    rng = np.random.default_rng(123)
+
+    # golden, hand-worked values
+    g = load_golden("dwconv1d_worked_example.json")
+    x = np.array(g["x"], float); w = np.array(g["w"], float); bias = np.array(g["bias"], float)
+    dy = np.array(g["dy"], float); L = np.array(g["lengths"], np.int32)
+    s = g["symmetric"]
+    if not np.array_equal(o.dwconv1d_fwd(x, w, bias, L, s["pad_left"]), np.array(s["y"], float)):
+        fails.append("golden fwd symmetric")
+    if not np.array_equal(o.dwconv1d_bwd_dx(dy, w, L, s["pad_left"]), np.array(s["dx"], float)):
+        fails.append("golden dx")
+    dw, db = o.dwconv1d_bwd_dw(x, dy, 3, L, s["pad_left"])
+    if not (np.array_equal(dw, np.array(s["dw"], float)) and np.array_equal(db, np.array(s["dbias"], float))):
+        fails.append("golden dw/dbias")
+    cz = g["causal_no_bias"]
+    if not np.array_equal(o.dwconv1d_fwd(x, w, None, L, cz["pad_left"]), np.array(cz["y"], float)):
+        fails.append("golden fwd causal")
+    gs = load_golden("subsample_worked_example.json")
+    for mode, causal in (("symmetric", False), ("causal", True)):
+        e = gs[mode]
+        out, ol = o.dw_subsample_fwd(np.array(gs["mel"], float), np.array(e["w0"], float),
+                                     np.array(e["b0"], float), np.array(gs["w1"], float),
+                                     np.array(gs["b1"], float), np.array(gs["lengths"], np.int32),
+                                     causal)
+        if not (np.array_equal(out, np.array(e["out"], float)) and list(ol) == e["out_lengths"]):
+            fails.append(f"golden subsample {mode}")
+
+    # second formulations (im2col, band matrix) and torch autograd on small random cases
+    for (B, T, C, K, pl) in ((3, 11, 5, 4, 1), (2, 7, 3, 9, 8), (1, 2, 2, 5, 2), (2, 16, 9, 3, 1)):
+        x = rng.standard_normal((B, T, C)); w = rng.standard_normal((K, C))
+        bias = rng.standard_normal(C); dy = rng.standard_normal((B, T, C))
+        L = rng.integers(0, T + 1, size=B).astype(np.int32)
+        y = o.dwconv1d_fwd(x, w, bias, L, pl)
+        if rel_err(y, im2col_fwd(x, w, bias, L, pl)) > 1e-12:
+            fails.append(f"im2col fwd {B, T, C, K, pl}")
+        if rel_err(o.dwconv1d_bwd_dx(dy, w, L, pl), band_dx(dy, w, L, pl)) > 1e-12:
+            fails.append(f"band dx {B, T, C, K, pl}")
+        dw, db = o.dwconv1d_bwd_dw(x, dy, K, L, pl)
+        rdw, rdb = im2col_dw(x, dy, K, L, pl)
+        if rel_err(dw, rdw) > 1e-12 or rel_err(db, rdb) > 1e-12:
+            fails.append(f"im2col dw {B, T, C, K, pl}")
+        ty, tdx, tdw, tdb = torch_conv1d_all(x, w, bias, dy, L, pl)
+        if rel_err(y, ty) > 1e-12:
+            fails.append(f"torch fwd {B, T, C, K, pl}")
+
+    for causal in (False, True):
+        B, T, F, C = 2, 13, 10, 3
+        mel = rng.standard_normal((B, T, F)); w0 = rng.standard_normal((3, 3, C))
+        w1 = rng.standard_normal((3, 3, C)); b0 = rng.standard_normal(C); b1 = rng.standard_normal(C)
+        L = np.array([13, 6], np.int32)
+        out, ol = o.dw_subsample_fwd(mel, w0, b0, w1, b1, L, causal)
+        ref, rl = torch_subsample(mel, w0, b0, w1, b1, L, causal)
+        if out.shape != ref.shape or rel_err(out, ref) > 1e-12 or not np.array_equal(ol, rl):
+            fails.append(f"torch subsample causal={causal}")
+    return fails

@@ -1,0 +1,53 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins catch each one.
+
+The mistakes are the kinds the parakeet.cpp PR's own mutation testing planted (section
+"Tests": a swapped or one-off pad, a scrambled batch axis), plus dropped masks, a dropped
+ReLU, flipped taps and transposed operands.  Each mutant is compiled from a temporary copy
+of the oracle's C source on the CPU; the committed oracle is never changed.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+from pinlib import pin_battery
+
+MUTANTS = {
+    "one-off pad": ("int64_t s = j - pad_left;", "int64_t s = j - pad_left + 1;"),
+    "pre-mask dropped": ("if (s < 0 || s >= L) return 0.0;", "if (s < 0 || s >= T) return 0.0;"),
+    "post-mask dropped": ("if (t < L) {", "if (t < T) {"),
+    "dx taps flipped": ("const int64_t s = t + k - pad_left;", "const int64_t s = t - k + pad_left;"),
+    "dx batch scrambled": ("dx[(b * T + s) * C + c] += dy[(b * T + t) * C + c]",
+                           "dx[(b * T + s) * C + c] += dy[((B - 1 - b) * T + t) * C + c]"),
+    "dw taps reversed": ("xpad_at(x, b, t + k, c, T, C, pad_left, L);\n",
+                         "xpad_at(x, b, t + K - 1 - k, c, T, C, pad_left, L);\n"),
+    "dbias unmasked": ("db += dz;", "db += dy[(b * T + t) * C + c];"),
+    "relu dropped": ("double hv = a > 0.0 ? a : 0.0;", "double hv = a;"),
+    "h mask off by one": ("if (i >= L2) hv = 0.0;", "if (i > L2) hv = 0.0;"),
+    "out mask dropped": ("if (i >= L4) a = 0.0;", "if (i > T4) a = 0.0;"),
+    "conv0 taps transposed": ("* w0[(p * 3 + q) * C + c];", "* w0[(q * 3 + p) * C + c];"),
+    "h placed with symmetric offset": ("hpad[((i + Pt) * HF + (j + 1)) * C + c] = hv;",
+                                       "hpad[((i + 1) * HF + (j + 1)) * C + c] = hv;"),
+    "conv_dw1 freq taps flipped": ("hpad[((2 * i + p) * HF + (2 * j + q)) * C + c]",
+                                   "hpad[((2 * i + p) * HF + (2 * j + 2 - q)) * C + c]"),
+    "mel not masked": ("melpad[r * FP + f] = (t >= 0 && t < L &&", "melpad[r * FP + f] = (t >= 0 && t < T &&"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(os.path.join(os.path.dirname(oracle.__file__), "dwconv_oracle.c")) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, f"mutation site for {name!r} not unique in the oracle source"
+    src = tmp_path / "mutant.c"
+    src.write_text(source.replace(old, new))
+    lib = oracle.build(force=True, src=str(src), out=str(tmp_path / "libmutant.so"))
+    fails = pin_battery(oracle.Oracle(lib))
+    assert fails, f"no pin caught the planted mistake {name!r}"
+    shutil.rmtree(tmp_path, ignore_errors=True)
