@@ -1,0 +1,474 @@
+"""Benchmark of the depthwise-convolution hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * depthwise conv1d forward, data gradient and weight/bias gradients on the conformer
+    workload x[16, 1500, 512] bf16, K = 9, symmetric padding 4|4, lengths uniform in [750, 1500];
+  * the fused depthwise-striding subsampler on mel[16, 3000, 80] fp32 -> out[16, 750, 20, 256]
+    bf16, symmetric padding, lengths uniform in [1500, 3000].
+Inputs are resident in device memory; three rotating input sets (about 237 MB each, larger
+than L2 together and alone) keep every step's reads cold in L2.  Every kernel launch is
+bracketed by CUDA events on its stream.  The value is algorithmic bytes per step (valid input
+frames read, all output frames written, parameters) divided by the step time.
+
+`--impl reference` times the CPU oracle (the only reference this path has) on a bounded
+sample of the same workload.  Multi-GPU: one process per GPU (torchrun), each rank its own
+batch, no collective on the data path (weak scaling); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("dwconv1d HBM GB/s & frames/s (B16 T1500 C512 K9 bf16); subsampler ms and % roofline")
+CONV = dict(B=16, T=1500, C=512, K=9, pad_left=4, len_range=(750, 1500), seed=1)
+SUB = dict(B=16, T=3000, F=80, C=256, causal=0, len_range=(1500, 3000), seed=3)
+N_SETS = 3
+WORKLOAD = ("conformer depthwise conv1d B16 T1500 C512 K9 bf16 sym 4|4, len U[750,1500]: fwd + dX + "
+            "dW/dbias; fused depthwise-striding subsampler B16 T3000 F80 -> B16 T750 F20 C256 bf16 sym, "
+            "len U[1500,3000]")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ algorithmic work
+def conv_work(lengths, T, C, K, esize=2):
+    """Bytes and flops of the three conv1d legs (valid input frames read, all outputs written)."""
+    B = len(lengths)
+    valid = int(np.clip(lengths, 0, T).sum())
+    params = K * C * 4 + C * 4 + B * 4
+    fwd_b = valid * C * esize + B * T * C * esize + params
+    dx_b = valid * C * esize + B * T * C * esize + K * C * 4 + B * 4
+    dw_b = 2 * valid * C * esize + (K + 1) * C * 4 + B * 4
+    fl = 2 * K * valid * C
+    return dict(fwd=(fwd_b, fl), dx=(dx_b, fl), dw=(dw_b, fl + valid * C)), valid
+
+
+def sub_work(lengths, T, F, C, esize=2):
+    s2 = lambda n: (n - 1) // 2 + 1 if n >= 1 else 0
+    T2, F2 = s2(T), s2(F)
+    T4, F4 = s2(T2), s2(F2)
+    B = len(lengths)
+    L = np.clip(lengths, 0, T).astype(np.int64)
+    L2 = np.minimum((L + 1) // 2, T2)
+    L4 = np.minimum((L2 + 1) // 2, T4)
+    by = int(L.sum()) * F * 4 + B * T4 * F4 * C * esize + 2 * (9 * C * 4 + C * 4) + B * 8
+    fl = int(L2.sum()) * F2 * C * 18 + int(L4.sum()) * F4 * C * 18
+    return by, fl, T4, F4
+
+
+# ------------------------------------------------------------------ clocks (NVML, read only)
+class ClockSampler:
+    """Samples SM clock and throttle reasons in a background thread (reads only)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        med = float(np.median(self.samples)) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "speech_encoder_depthwise_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernels have not changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        rows = [dict(kv.split("=", 1) for kv in line.split()) for line in open(path)
+                if line.strip() and not line.startswith("#")]
+    except Exception:
+        return None
+    sha = kernel_source_sha()
+    for r in rows:
+        if r.get("kernel") == kernel and r.get("sha") == sha:
+            return float(r["dram_bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------ reference arm (CPU oracle)
+def oracle_sample_step(cs, ss, frac):
+    """One bounded oracle step: item 0 of each workload, the first `frac` of its frames."""
+    import oracle
+    Tc = max(CONV["K"], int(round(frac * CONV["T"])))
+    Ts = max(8, 4 * int(round(frac * SUB["T"] / 4)))
+    x, dy = cs["x"][:1, :Tc], cs["dy"][:1, :Tc]
+    ln = np.minimum(cs["lengths"][:1], Tc).astype(np.int32)
+    oracle.dwconv1d_fwd(x, cs["w"], cs["bias"], ln, CONV["pad_left"])
+    oracle.dwconv1d_bwd_dx(dy, cs["w"], ln, CONV["pad_left"])
+    oracle.dwconv1d_bwd_dw(x, dy, CONV["K"], ln, CONV["pad_left"])
+    mel = ss["mel"][:1, :Ts]
+    sl = np.minimum(ss["lengths"][:1], Ts).astype(np.int32)
+    oracle.dw_subsample_fwd(mel, ss["w0"], ss["b0"], ss["w1"], ss["b1"], sl, SUB["causal"])
+    w, _ = conv_work(ln, Tc, CONV["C"], CONV["K"])
+    sb, _, _, _ = sub_work(sl, Ts, SUB["F"], SUB["C"])
+    return sum(v[0] for v in w.values()) + sb, f"item 0, first {Tc} of {CONV['T']} conv1d frames and " \
+        f"{Ts} of {SUB['T']} mel frames"
+
+
+def inputs():
+    from synth import conv1d_inputs, subsample_inputs
+    cs = conv1d_inputs(CONV["B"], CONV["T"], CONV["C"], CONV["K"], dtype="bf16",
+                       len_range=CONV["len_range"], seed=CONV["seed"], with_dy=True)
+    ss = subsample_inputs(SUB["B"], SUB["T"], SUB["F"], SUB["C"], len_range=SUB["len_range"], seed=SUB["seed"])
+    return cs, ss
+
+
+def cpu_rate(cs, ss, seconds, steps=None):
+    """Time the oracle on bounded samples; returns (GB/s, sample description, cores, per-step s)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle_sample_step(cs, ss, 0.02)
+    cal = max(time.perf_counter() - t0, 1e-3)
+    per_step = seconds if steps is None else seconds / max(steps, 1)
+    frac = float(min(1.0, max(0.01, 0.02 * per_step / cal)))
+    total_b, total_t, n = 0, 0.0, 0
+    desc = ""
+    while True:
+        t0 = time.perf_counter()
+        b, desc = oracle_sample_step(cs, ss, frac)
+        total_t += time.perf_counter() - t0
+        total_b += b
+        n += 1
+        if steps is not None and n >= steps:
+            break
+        if steps is None and total_t >= seconds:
+            break
+    return total_b / total_t / 1e9, desc, oracle.num_threads(), total_t / n
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return 0
+    cs, ss = inputs()
+    budget = 150.0  # seconds for warm-up + timed steps
+    per = budget / (args.steps + max(args.warmup, 0))
+    # warm-up steps (untimed)
+    if args.warmup > 0:
+        cpu_rate(cs, ss, per * args.warmup, steps=args.warmup)
+    v, desc, cores, step_s = cpu_rate(cs, ss, per * args.steps, steps=args.steps)
+    line = {"metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "parallelism": "rank 0 only (CPU)"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    import speech_encoder_depthwise_b200 as dw
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    lib = dw.lib()
+    warmup = max(args.warmup, 3)
+    steps = max(args.steps, 1)
+
+    cs, ss = inputs()
+    if rank > 0:  # each rank its own batch (weak scaling)
+        from synth import conv1d_inputs, subsample_inputs
+        cs = conv1d_inputs(CONV["B"], CONV["T"], CONV["C"], CONV["K"], dtype="bf16",
+                           len_range=CONV["len_range"], seed=100 + rank, with_dy=True)
+        ss = subsample_inputs(SUB["B"], SUB["T"], SUB["F"], SUB["C"], len_range=SUB["len_range"],
+                              seed=200 + rank)
+    B, T, C, K, pl = CONV["B"], CONV["T"], CONV["C"], CONV["K"], CONV["pad_left"]
+    SB, ST, SF, SC = SUB["B"], SUB["T"], SUB["F"], SUB["C"]
+    T4, F4 = dw.subsample_out_shape(ST, SF)
+
+    def t(a, dtype=torch.float32):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dtype)
+
+    w, bias, ln = t(cs["w"]), t(cs["bias"]), t(cs["lengths"], torch.int32)
+    w0, b0, w1, b1, sl = t(ss["w0"]), t(ss["b0"]), t(ss["w1"]), t(ss["b1"]), t(ss["lengths"], torch.int32)
+    x0, dy0, mel0 = t(cs["x"], torch.bfloat16), t(cs["dy"], torch.bfloat16), t(ss["mel"])
+    sets = []
+    for _ in range(N_SETS):
+        sets.append(dict(x=x0.clone(), dy=dy0.clone(), y=torch.empty_like(x0), dx=torch.empty_like(x0),
+                         mel=mel0.clone(), out=torch.empty(SB, T4, F4, SC, dtype=torch.bfloat16, device=dev)))
+    del x0, dy0, mel0
+    gw = torch.empty(K, C, device=dev)
+    gb = torch.empty(C, device=dev)
+    ol = torch.empty(SB, dtype=torch.int32, device=dev)
+    nws = dw.dwconv1d_bwd_dw_workspace_size(B, T, C, K)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    P = lambda tt: ctypes.c_void_p(tt.data_ptr())
+
+    # argument tuples built once: each launch is one foreign call, no tensor bookkeeping
+    calls = []
+    for s in sets:
+        calls.append([
+            ("dwconv1d_fwd", lib.dwconv1d_fwd, (P(s["x"]), P(w), P(bias), P(s["y"]), P(ln), B, T, C, K, pl,
+                                                dw.DW_BF16, ctypes.c_void_p(sp))),
+            ("dwconv1d_bwd_dx", lib.dwconv1d_bwd_dx, (P(s["dy"]), P(w), P(s["dx"]), P(ln), B, T, C, K, pl,
+                                                      dw.DW_BF16, ctypes.c_void_p(sp))),
+            ("dwconv1d_bwd_dw", lib.dwconv1d_bwd_dw, (P(s["x"]), P(s["dy"]), P(gw), P(gb), P(ln), B, T, C, K,
+                                                      pl, dw.DW_BF16, P(ws), ws.numel(), ctypes.c_void_p(sp))),
+            ("dw_subsample_fwd", lib.dw_subsample_fwd, (P(s["mel"]), P(w0), P(b0), P(w1), P(b1), P(s["out"]),
+                                                        P(sl), P(ol), SB, ST, SF, SC, SUB["causal"],
+                                                        dw.DW_BF16, ctypes.c_void_p(sp))),
+        ])
+    rows = [c[0] for c in calls[0]]
+    launches_per_row = {"dwconv1d_fwd": 1, "dwconv1d_bwd_dx": 1, "dwconv1d_bwd_dw": 2, "dw_subsample_fwd": 2}
+
+    def run_step(i, evs=None):
+        for j, (name, fn, a) in enumerate(calls[i % N_SETS]):
+            if evs is not None:
+                evs[j][0].record(stream)
+            st = fn(*a)
+            if st != 0:
+                raise RuntimeError(f"{name}: {dw.dw_status_string(st)}")
+            if evs is not None:
+                evs[j][1].record(stream)
+
+    for i in range(warmup):
+        run_step(i)
+    torch.cuda.synchronize(dev)
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    step_evs = [[(mk(), mk()) for _ in rows] for _ in range(steps)]
+    e_start, e_end = mk(), mk()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        e_start.record(stream)
+        for i in range(steps):
+            run_step(i, step_evs[i])
+        e_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = e_start.elapsed_time(e_end)
+    row_ms = {r: float(np.mean([step_evs[i][j][0].elapsed_time(step_evs[i][j][1]) for i in range(steps)]))
+              for j, r in enumerate(rows)}
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / steps
+
+    cw, valid = conv_work(cs["lengths"], T, C, K)
+    sb, sf, _, _ = sub_work(ss["lengths"], ST, SF, SC)
+    step_bytes = sum(v[0] for v in cw.values()) + sb
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---------------------------------------------------------------- e2e through the binding
+    e2e = None
+    if args.e2e_steps > 0:
+        h = dict(x=torch.from_numpy(cs["x"]).to(torch.bfloat16).pin_memory(),
+                 dy=torch.from_numpy(cs["dy"]).to(torch.bfloat16).pin_memory(),
+                 ln=torch.from_numpy(cs["lengths"]).pin_memory(),
+                 mel=torch.from_numpy(ss["mel"]).pin_memory(),
+                 sl=torch.from_numpy(ss["lengths"]).pin_memory(),
+                 w=torch.from_numpy(cs["w"]).pin_memory(), bias=torch.from_numpy(cs["bias"]).pin_memory(),
+                 w0=torch.from_numpy(ss["w0"]).pin_memory(), b0=torch.from_numpy(ss["b0"]).pin_memory(),
+                 w1=torch.from_numpy(ss["w1"]).pin_memory(), b1=torch.from_numpy(ss["b1"]).pin_memory())
+        ho = dict(y=torch.empty(B, T, C, dtype=torch.bfloat16).pin_memory(),
+                  dx=torch.empty(B, T, C, dtype=torch.bfloat16).pin_memory(),
+                  gw=torch.empty(K, C).pin_memory(), gb=torch.empty(C).pin_memory(),
+                  out=torch.empty(SB, T4, F4, SC, dtype=torch.bfloat16).pin_memory(),
+                  ol=torch.empty(SB, dtype=torch.int32).pin_memory())
+        s0 = sets[0]
+        dparams = dict(w=w, bias=bias, w0=w0, b0=b0, w1=w1, b1=b1, ln=ln, sl=sl)
+        h2d = sum(v.numel() * v.element_size() for v in h.values())
+        d2h = sum(v.numel() * v.element_size() for v in ho.values())
+
+        def e2e_step():
+            s0["x"].copy_(h["x"], non_blocking=True)
+            s0["dy"].copy_(h["dy"], non_blocking=True)
+            s0["mel"].copy_(h["mel"], non_blocking=True)
+            for k, v in dparams.items():
+                v.copy_(h[k], non_blocking=True)
+            dw.dwconv1d_fwd(s0["x"], w, bias, s0["y"], ln, pl)
+            dw.dwconv1d_bwd_dx(s0["dy"], w, s0["dx"], ln, pl)
+            dw.dwconv1d_bwd_dw(s0["x"], s0["dy"], gw, gb, ln, pl, ws)
+            dw.dw_subsample_fwd(s0["mel"], w0, b0, w1, b1, s0["out"], sl, ol, SUB["causal"])
+            ho["y"].copy_(s0["y"], non_blocking=True)
+            ho["dx"].copy_(s0["dx"], non_blocking=True)
+            ho["gw"].copy_(gw, non_blocking=True)
+            ho["gb"].copy_(gb, non_blocking=True)
+            ho["out"].copy_(s0["out"], non_blocking=True)
+            ho["ol"].copy_(ol, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        a, b_ = mk(), mk()
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = a.elapsed_time(b_) / args.e2e_steps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    # ---------------------------------------------------------------- report (rank 0)
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        hbm = float(peaks.get("hbm_gbs", 6650.0))
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        fmax = float(peaks.get("sm_max_mhz", 1965.0))
+        fp32_tflops = sms * 128 * 2 * fmax * 1e6 / 1e12
+        row = {}
+        for name, (by, fl) in cw.items():
+            key = {"fwd": "dwconv1d_fwd", "dx": "dwconv1d_bwd_dx", "dw": "dwconv1d_bwd_dw"}[name]
+            ms = row_ms[key]
+            row[key] = {"us": ms * 1e3, "GB_per_s": by / (ms * 1e-3) / 1e9,
+                        "frames_per_s": B * T / (ms * 1e-3),
+                        "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm,
+                        "hbm_frac_of_8TBps": by / (ms * 1e-3) / 1e9 / 8000.0,
+                        "alg_bytes": by, "alg_flops": fl}
+        ms = row_ms["dw_subsample_fwd"]
+        row["dw_subsample_fwd"] = {"ms": ms, "us": ms * 1e3, "TFLOP_per_s": sf / (ms * 1e-3) / 1e12,
+                                   "fp32_frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
+                                   "GB_per_s": sb / (ms * 1e-3) / 1e9,
+                                   "frames_per_s": SB * T4 / (ms * 1e-3),
+                                   "alg_bytes": sb, "alg_flops": sf}
+        # every throughput row carries its distance from the oracle (items 0-1; dW over the batch)
+        import oracle
+        f64 = lambda tt: tt.float().cpu().numpy().astype(np.float64)
+        s0 = sets[0]
+        err = lambda a, b: float(np.max(np.abs(a - b)))
+        row["dwconv1d_fwd"]["max_abs_err"] = err(f64(s0["y"][:2]), oracle.dwconv1d_fwd(
+            cs["x"][:2], cs["w"], cs["bias"], cs["lengths"][:2], pl))
+        row["dwconv1d_bwd_dx"]["max_abs_err"] = err(f64(s0["dx"][:2]), oracle.dwconv1d_bwd_dx(
+            cs["dy"][:2], cs["w"], cs["lengths"][:2], pl))
+        rdw, rdb = oracle.dwconv1d_bwd_dw(cs["x"], cs["dy"], K, cs["lengths"], pl)
+        row["dwconv1d_bwd_dw"]["max_abs_err"] = max(err(f64(gw), rdw), err(f64(gb), rdb))
+        ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
+                                        ss["lengths"][:2], SUB["causal"])
+        row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
+        cpu = None
+        if world == 1 and args.cpu_seconds > 0:
+            v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)
+            cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the pages' workloads)",
+            "config": {"workload": WORKLOAD, "global_batch": world * B, "seq_len": T,
+                       "parallelism": f"replicas x{world} (independent batches, no collective)",
+                       "l2": f"{N_SETS} rotating input sets of ~237 MB each (> L2 126 MB)"},
+            "frames_per_s": world * B * T / (row_ms["dwconv1d_fwd"] * 1e-3),
+            "subsampler_ms": row_ms["dw_subsample_fwd"],
+            "subsampler_roofline_frac": row["dw_subsample_fwd"]["fp32_frac"],
+            "rows": row,
+            "roofline": {"bound": "alu", "kernel": "dw_subsample_kernel",
+                         "achieved": sf / (ms * 1e-3) / 1e12, "peak": fp32_tflops, "unit": "TFLOP/s",
+                         "frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
+                         "peak_basis": f"{sms} SMs x 128 FP32 lanes x 2 x {fmax:.0f} MHz ({peak_kind} max clock)",
+                         "traffic": ncu_traffic("dw_subsample_kernel")},
+            "hbm_peak_gbs": hbm, "hbm_peak_kind": peak_kind,
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": steps * sum(launches_per_row.values()),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

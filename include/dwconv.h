@@ -1,0 +1,158 @@
+/*
+ * dwconv.h - C ABI of a B200 (sm_100a) library for the depthwise-convolution hot path of a
+ * conformer speech encoder: the time-axis depthwise conv1d (forward, data gradient, weight
+ * and bias gradients) and the fused depthwise-striding subsampler front.
+ *
+ * Conventions shared by every entry point
+ *  - Memory: every tensor pointer is a DEVICE pointer owned by the caller.  The library
+ *    allocates nothing, never synchronizes, and enqueues its kernels on `stream`
+ *    (a cudaStream_t; NULL means the legacy default stream).  Results are ready when the
+ *    stream reaches them.
+ *  - Layout: activations are channels-last and C-contiguous: x[B][T][C] (C fastest).
+ *    Weights and biases are float32: w[K][C], bias[C], w0/w1[3][3][C] (C fastest).  A
+ *    PyTorch depthwise weight [C][1][K] is the transpose of w.
+ *  - Lengths: `lengths` is a device int32 array [B] or NULL.  NULL means every item has
+ *    T valid frames.  Values outside [0, T] are clamped into it by the kernels.
+ *  - Masking: frame t of item b is valid when t < lengths[b].  Invalid input frames count
+ *    as zero; invalid output frames are written as +0.0.
+ *  - Errors: every call returns a dw_status_t and never aborts or traps.  Argument errors
+ *    are found on the host before any CUDA call.  A failed launch returns DW_ERR_CUDA.
+ *    B == 0 or T == 0 is a valid no-op.  Misaligned pointers, or a C that is not a
+ *    multiple of the vector width, take a narrower (slower) path and stay correct.
+ *  - Arithmetic: bf16 or float32 I/O, float32 accumulation, bf16 stores rounded to
+ *    nearest even.  No tensor cores.
+ */
+#ifndef DWCONV_B200_H
+#define DWCONV_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dw_status {
+    DW_OK = 0,
+    DW_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad padding, aliasing */
+    DW_ERR_UNSUPPORTED = 2,  /* a valid request this build cannot serve (e.g. no sm_100 device) */
+    DW_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the *_workspace_size result */
+    DW_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    DW_ERR_TIMEOUT = 5       /* reserved: no kernel of this library waits on another */
+} dw_status_t;
+
+typedef enum dw_dtype {
+    DW_F32 = 0,   /* IEEE float32 */
+    DW_BF16 = 1   /* bfloat16 (upper half of a float32) */
+} dw_dtype_t;
+
+typedef void *dw_stream_t; /* a cudaStream_t */
+
+/*
+ * dwconv1d_fwd - depthwise conv1d forward with fused pre/post masking and padding.
+ *
+ *   y[b,t,c] = [t < len_b] * (bias[c] + sum_{k<K} xpad[b,t+k,c] * w[k,c])
+ *   xpad[b,j,c] = x[b, j - pad_left, c] if 0 <= j - pad_left < len_b, else 0
+ *
+ * The sum over k of x[t+k,c] * w[k,c] over the input padded to T + K - 1 frames is the
+ * SSM_CONV form of the depthwise conv (parakeet.cpp PR #102, "faster GPU decode: one
+ * SSM_CONV for the depthwise conv", section "What changes"); masking before and after the
+ * conv and the causal padding are fused as in NeMo PR #16114 ("Use Fused Kernels for
+ * Depthwise Striding Subsampler", section "What does this PR do ?", second kernel).
+ *
+ *  x        [B][T][C] io_dtype, device, read only
+ *  w        [K][C] float32, device
+ *  bias     [C] float32, device, or NULL (no bias)
+ *  y        [B][T][C] io_dtype, device, written in full; must not overlap x
+ *  lengths  [B] int32, device, or NULL
+ *  B, T, C  sizes, B >= 0, T >= 0, C >= 1
+ *  K        kernel width, K >= 1 (any width)
+ *  pad_left 0 <= pad_left <= K-1; pad_right = K-1-pad_left.  Symmetric ('same') padding:
+ *           pad_left = (K-1)/2; causal padding: pad_left = K-1.
+ */
+dw_status_t dwconv1d_fwd(const void *x, const float *w, const float *bias, void *y,
+                         const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
+                         int pad_left, dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
+ * dwconv1d_bwd_dx - data gradient of dwconv1d_fwd (backward of NeMo PR #16114's
+ * depthwise kernel, section "What does this PR do ?").
+ *
+ *   dz[b,t,c] = [t < len_b] dy[b,t,c]
+ *   dx[b,s,c] = [s < len_b] * sum_{k<K} dz[b, s + pad_left - k, c] * w[k,c]   (dz = 0 outside [0,T))
+ *
+ * i.e. the forward correlation with the taps reversed and the pads swapped, no bias.
+ *
+ *  dy       [B][T][C] io_dtype, device          dx [B][T][C] io_dtype, device, written in full,
+ *  w        [K][C] float32, device                 must not overlap dy
+ *  other arguments as in dwconv1d_fwd (pad_left is the FORWARD pass's left pad).
+ */
+dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int32_t *lengths,
+                            int64_t B, int64_t T, int64_t C, int K, int pad_left,
+                            dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
+ * dwconv1d_bwd_dw_workspace_size - bytes of device workspace dwconv1d_bwd_dw needs for
+ * these sizes (independent of pointers, dtype and device).  Returns 0 when B*T == 0.
+ */
+size_t dwconv1d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t C, int K);
+
+/*
+ * dwconv1d_bwd_dw - weight and bias gradients of dwconv1d_fwd (NeMo PR #16114, section
+ * "What does this PR do ?", backward; deterministic like its "honor deterministic path").
+ *
+ *   dW[k,c]   = sum_{b,t} dz[b,t,c] * xpad[b,t+k,c]
+ *   dbias[c]  = sum_{b,t} dz[b,t,c],           dz[b,t,c] = [t < len_b] dy[b,t,c]
+ *
+ * float32 accumulation in a fixed order: per-block partial sums go to `workspace`, then a
+ * second kernel adds them in a fixed order.  Results are bitwise reproducible for given
+ * sizes, on any run.  No atomics.
+ *
+ *  x, dy     [B][T][C] io_dtype, device
+ *  dw        [K][C] float32, device, overwritten
+ *  dbias     [C] float32, device, overwritten, or NULL
+ *  workspace device buffer of at least dwconv1d_bwd_dw_workspace_size(B,T,C,K) bytes,
+ *            16-byte aligned; contents on entry are ignored
+ *  With B*T == 0 the gradients are written as zeros (workspace may be NULL).
+ */
+dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbias,
+                            const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
+                            int pad_left, dw_dtype_t io_dtype, void *workspace,
+                            size_t workspace_bytes, dw_stream_t stream);
+
+/*
+ * dw_subsample_fwd - fused front of the depthwise-striding subsampler (NeMo PR #16114, "Use
+ * Fused Kernels for Depthwise Striding Subsampler", section "What does this PR do ?", first
+ * kernel: mel [B,T,F,1] -> conv0 [B,T/2,F/2,C] -> ReLU -> masking -> conv_dw1 [B,T/4,F/4,C]).
+ * The conv0 output never goes to device memory.
+ *
+ *   melpad = mel with frames t >= len_b zeroed, padded Pt|Pb in time and 1|1 in frequency
+ *   h[b,i,j,c]   = [i < ceil(len_b/2)] * ReLU(b0[c] + sum_{p,q<3} melpad[2i+p, 2j+q] * w0[p,q,c])
+ *   out[b,i,j,c] = [i < ceil(len_b/4)] * (b1[c] + sum_{p,q<3} hpad[b, 2i+p, 2j+q, c] * w1[p,q,c])
+ *   hpad = h padded Pt|Pb in time and 1|1 in frequency; Pt|Pb = 1|1, or 2|0 when causal.
+ *
+ *  mel          [B][T][F] float32, device
+ *  w0, w1       [3][3][C] float32, device;  b0, b1 [C] float32, device
+ *  out          [B][T4][F4][C] out_dtype, device, written in full, where
+ *               T2 = ceil(T/2), T4 = ceil(T2/2), F2 = ceil(F/2), F4 = ceil(F2/2)
+ *  lengths      [B] int32, device, or NULL
+ *  out_lengths  [B] int32, device, or NULL; receives ceil(ceil(len_b/2)/2)
+ *  B >= 0, T >= 0, F >= 1, C >= 1; causal 0 or 1; out_dtype DW_BF16 or DW_F32
+ */
+dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
+                             const float *w1, const float *b1, void *out,
+                             const int32_t *lengths, int32_t *out_lengths, int64_t B,
+                             int64_t T, int64_t F, int64_t C, int causal,
+                             dw_dtype_t out_dtype, dw_stream_t stream);
+
+/* dw_status_string - a static, human-readable name for a status code. */
+const char *dw_status_string(dw_status_t status);
+
+/* dw_last_cuda_error - the cudaError_t behind the most recent DW_ERR_CUDA on this thread. */
+int dw_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DWCONV_B200_H */

@@ -1,0 +1,184 @@
+// The C ABI (include/dwconv.h): argument validation on the host, then dispatch to the
+// kernels.  Nothing here allocates, synchronizes or aborts.  Every argument check runs
+// before the first CUDA call, so invalid calls return without touching the device.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "dw_internal.h"
+#include "dwconv.h"
+
+namespace dwk {
+cudaError_t subsample_out_lengths_launch(const int32_t *lengths, int32_t *out_lengths, int64_t B, int64_t T,
+                                         cudaStream_t s);
+}
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+dw_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return DW_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return DW_ERR_CUDA;
+}
+
+size_t dtype_size(dw_dtype_t t) { return t == DW_BF16 ? 2 : 4; }
+
+bool valid_dtype(dw_dtype_t t) { return t == DW_F32 || t == DW_BF16; }
+
+// n = a*b*c without overflow of int64 (all >= 0)
+bool mul3(int64_t a, int64_t b, int64_t c, int64_t *n) {
+    __int128 p = static_cast<__int128>(a) * b * c;
+    if (p > static_cast<__int128>(INT64_MAX / 4)) return false;
+    *n = static_cast<int64_t>(p);
+    return true;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+bool aligned(const void *p, size_t n) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % n == 0; }
+
+// Channel-pair vector path: C even, activations aligned to one pair, parameters to float2.
+int pick_vec_width(int64_t C, size_t esize, std::initializer_list<const void *> acts,
+                   std::initializer_list<const void *> params) {
+    if (C % 2 != 0) return 1;
+    for (const void *p : acts)
+        if (!aligned(p, 2 * esize)) return 1;
+    for (const void *p : params)
+        if (!aligned(p, 8)) return 1;
+    return 2;
+}
+
+dw_status_t check_conv1d_common(const void *in, const float *w, const void *out, int64_t B, int64_t T,
+                                int64_t C, int K, int pad_left, dw_dtype_t dt, int64_t *n) {
+    if (!valid_dtype(dt)) return DW_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
+    if (!mul3(B, T, C, n)) return DW_ERR_INVALID_ARG;
+    if (*n == 0) return DW_OK;
+    if (in == nullptr || w == nullptr || out == nullptr) return DW_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(*n) * dtype_size(dt);
+    if (overlaps(in, bytes, out, bytes)) return DW_ERR_INVALID_ARG;
+    return DW_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dw_status_string(dw_status_t s) {
+    switch (s) {
+        case DW_OK: return "DW_OK";
+        case DW_ERR_INVALID_ARG: return "DW_ERR_INVALID_ARG: invalid argument";
+        case DW_ERR_UNSUPPORTED: return "DW_ERR_UNSUPPORTED: request not supported by this build";
+        case DW_ERR_WORKSPACE: return "DW_ERR_WORKSPACE: workspace missing or too small";
+        case DW_ERR_CUDA: return "DW_ERR_CUDA: a CUDA call or kernel launch failed";
+        case DW_ERR_TIMEOUT: return "DW_ERR_TIMEOUT: a device-side wait gave up";
+    }
+    return "unknown dw_status_t";
+}
+
+int dw_last_cuda_error(void) { return g_last_cuda_error; }
+
+dw_status_t dwconv1d_fwd(const void *x, const float *w, const float *bias, void *y, const int32_t *lengths,
+                         int64_t B, int64_t T, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
+                         dw_stream_t stream) {
+    int64_t n = 0;
+    dw_status_t st = check_conv1d_common(x, w, y, B, T, C, K, pad_left, io_dtype, &n);
+    if (st != DW_OK || n == 0) return st;
+    dwk::Conv1dArgs a;
+    a.x = x; a.w = w; a.bias = bias; a.y = y; a.lengths = lengths;
+    a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left; a.flip = 0;
+    a.bf16 = io_dtype == DW_BF16;
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, y}, {w, bias});
+    return cuda_status(dwk::conv1d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
+dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int32_t *lengths, int64_t B,
+                            int64_t T, int64_t C, int K, int pad_left, dw_dtype_t io_dtype, dw_stream_t stream) {
+    int64_t n = 0;
+    dw_status_t st = check_conv1d_common(dy, w, dx, B, T, C, K, pad_left, io_dtype, &n);
+    if (st != DW_OK || n == 0) return st;
+    dwk::Conv1dArgs a;
+    a.x = dy; a.w = w; a.bias = nullptr; a.y = dx; a.lengths = lengths;
+    a.B = B; a.T = T; a.C = C; a.K = K;
+    a.pad_left = K - 1 - pad_left;  // correlation with reversed taps: the pads swap
+    a.flip = 1;
+    a.bf16 = io_dtype == DW_BF16;
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {dy, dx}, {w});
+    return cuda_status(dwk::conv1d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dwconv1d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t C, int K) {
+    if (B <= 0 || T <= 0 || C < 1 || K < 1) return 0;
+    int64_t n = 0;
+    if (!mul3(B, T, C, &n)) return 0;
+    return dwk::conv1d_dw_workspace_bytes(B, T, C, K);
+}
+
+dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbias, const int32_t *lengths,
+                            int64_t B, int64_t T, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
+                            void *workspace, size_t workspace_bytes, dw_stream_t stream) {
+    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
+    int64_t n = 0;
+    if (!mul3(B, T, C, &n)) return DW_ERR_INVALID_ARG;
+    if (dw == nullptr) return DW_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(K + 1) * C > dwk::kMaxGrid * 256LL) return DW_ERR_INVALID_ARG;
+    dwk::DwArgs a;
+    a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = lengths;
+    a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left;
+    a.bf16 = io_dtype == DW_BF16;
+    a.partials = static_cast<float *>(workspace);
+    a.G = 0;
+    a.vec_width = 1;
+    if (n > 0) {
+        if (x == nullptr || dy == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t need = dwk::conv1d_dw_workspace_bytes(B, T, C, K);
+        if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return DW_ERR_WORKSPACE;
+        const size_t out_bytes = static_cast<size_t>(K) * C * sizeof(float);
+        if (overlaps(workspace, need, dw, out_bytes) ||
+            (dbias && overlaps(workspace, need, dbias, static_cast<size_t>(C) * sizeof(float))))
+            return DW_ERR_INVALID_ARG;
+        a.G = dwk::conv1d_dw_partial_rows(B, T, C, K);
+        a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, dy}, {});
+    }
+    return cuda_status(dwk::conv1d_dw_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
+dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0, const float *w1,
+                             const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
+                             int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,
+                             dw_stream_t stream) {
+    if (!valid_dtype(out_dtype)) return DW_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
+    int64_t n = 0;
+    if (!mul3(B, T, F, &n)) return DW_ERR_INVALID_ARG;
+    auto s2 = [](int64_t v) -> int64_t { return v >= 1 ? (v - 1) / 2 + 1 : 0; };
+    const int64_t T4 = s2(s2(T)), F4 = s2(s2(F));
+    int64_t nout = 0;
+    if (!mul3(B, T4 * F4, C, &nout)) return DW_ERR_INVALID_ARG;
+    if (out_lengths == nullptr && nout == 0) return DW_OK;
+    if (nout > 0) {
+        if (!mel || !w0 || !b0 || !w1 || !b1 || !out) return DW_ERR_INVALID_ARG;
+        if (overlaps(mel, static_cast<size_t>(n) * 4, out, static_cast<size_t>(nout) * dtype_size(out_dtype)))
+            return DW_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (nout > 0) {
+        dwk::SubsampleArgs a;
+        a.mel = mel; a.w0 = w0; a.b0 = b0; a.w1 = w1; a.b1 = b1; a.out = out;
+        a.lengths = lengths; a.out_lengths = out_lengths;
+        a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.bf16_out = out_dtype == DW_BF16;
+        dw_status_t st = cuda_status(dwk::subsample_launch(a, s));
+        if (st != DW_OK) return st;
+    }
+    if (out_lengths != nullptr && B > 0)
+        return cuda_status(dwk::subsample_out_lengths_launch(lengths, out_lengths, B, T, s));
+    return DW_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+// Shared device helpers: channel-vector loads/stores of bf16 or float32, bf16 <-> float32
+// conversion, packed float32x2 FMA.  sm_100a only.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dwk {
+
+typedef __nv_bfloat16 bf16;
+
+__device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
+
+// Two floats to a bf16 pair, round to nearest even; `lo` lands in the low 16 bits.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// Raw storage for V consecutive channels of element type T, loaded with one instruction.
+// Words are 32-bit; a bf16 pair sits in one word (low half = lower channel).
+template <typename T, int V> struct Vec;
+
+template <> struct Vec<bf16, 8> {
+    uint4 r;
+    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const uint4 *>(p)); }
+    __device__ __forceinline__ void zero() { r = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void to_f2(float2 (&f)[4]) const {
+        f[0] = make_float2(bf16_lo(r.x), bf16_hi(r.x)); f[1] = make_float2(bf16_lo(r.y), bf16_hi(r.y));
+        f[2] = make_float2(bf16_lo(r.z), bf16_hi(r.z)); f[3] = make_float2(bf16_lo(r.w), bf16_hi(r.w));
+    }
+    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[4]) {
+        uint4 o = make_uint4(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y),
+                             pack_bf16x2(f[2].x, f[2].y), pack_bf16x2(f[3].x, f[3].y));
+        *reinterpret_cast<uint4 *>(p) = o;
+    }
+    static __device__ __forceinline__ void store_zero(bf16 *p) {
+        *reinterpret_cast<uint4 *>(p) = make_uint4(0, 0, 0, 0);
+    }
+};
+
+template <> struct Vec<bf16, 4> {
+    uint2 r;
+    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const uint2 *>(p)); }
+    __device__ __forceinline__ void zero() { r = make_uint2(0, 0); }
+    __device__ __forceinline__ void to_f2(float2 (&f)[2]) const {
+        f[0] = make_float2(bf16_lo(r.x), bf16_hi(r.x)); f[1] = make_float2(bf16_lo(r.y), bf16_hi(r.y));
+    }
+    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[2]) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y));
+    }
+    static __device__ __forceinline__ void store_zero(bf16 *p) { *reinterpret_cast<uint2 *>(p) = make_uint2(0, 0); }
+};
+
+template <> struct Vec<bf16, 2> {
+    uint32_t r;
+    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const unsigned int *>(p)); }
+    __device__ __forceinline__ void zero() { r = 0; }
+    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const { f[0] = make_float2(bf16_lo(r), bf16_hi(r)); }
+    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[1]) {
+        *reinterpret_cast<uint32_t *>(p) = pack_bf16x2(f[0].x, f[0].y);
+    }
+    static __device__ __forceinline__ void store_zero(bf16 *p) { *reinterpret_cast<uint32_t *>(p) = 0u; }
+};
+
+template <> struct Vec<float, 4> {
+    float4 r;
+    __device__ __forceinline__ void load(const float *p) { r = __ldg(reinterpret_cast<const float4 *>(p)); }
+    __device__ __forceinline__ void zero() { r = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void to_f2(float2 (&f)[2]) const {
+        f[0] = make_float2(r.x, r.y); f[1] = make_float2(r.z, r.w);
+    }
+    static __device__ __forceinline__ void store(float *p, const float2 (&f)[2]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(f[0].x, f[0].y, f[1].x, f[1].y);
+    }
+    static __device__ __forceinline__ void store_zero(float *p) {
+        *reinterpret_cast<float4 *>(p) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+};
+
+template <> struct Vec<float, 2> {
+    float2 r;
+    __device__ __forceinline__ void load(const float *p) { r = __ldg(reinterpret_cast<const float2 *>(p)); }
+    __device__ __forceinline__ void zero() { r = make_float2(0.f, 0.f); }
+    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const { f[0] = r; }
+    static __device__ __forceinline__ void store(float *p, const float2 (&f)[1]) {
+        *reinterpret_cast<float2 *>(p) = f[0];
+    }
+    static __device__ __forceinline__ void store_zero(float *p) {
+        *reinterpret_cast<float2 *>(p) = make_float2(0.f, 0.f);
+    }
+};
+
+// One channel (any C, any alignment): the value travels as a float2 with .y = 0, so the
+// same pairwise arithmetic serves every width.  The slow, general fallback.
+template <> struct Vec<bf16, 1> {
+    unsigned short r;
+    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const unsigned short *>(p)); }
+    __device__ __forceinline__ void zero() { r = 0; }
+    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const {
+        f[0] = make_float2(__uint_as_float(static_cast<uint32_t>(r) << 16), 0.f);
+    }
+    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[1]) { *p = __float2bfloat16_rn(f[0].x); }
+    static __device__ __forceinline__ void store_zero(bf16 *p) { *reinterpret_cast<unsigned short *>(p) = 0; }
+};
+
+template <> struct Vec<float, 1> {
+    float r;
+    __device__ __forceinline__ void load(const float *p) { r = __ldg(p); }
+    __device__ __forceinline__ void zero() { r = 0.f; }
+    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const { f[0] = make_float2(r, 0.f); }
+    static __device__ __forceinline__ void store(float *p, const float2 (&f)[1]) { *p = f[0].x; }
+    static __device__ __forceinline__ void store_zero(float *p) { *p = 0.f; }
+};
+
+// Number of float2 pairs that carry V channels.
+template <int V> struct Pairs { static constexpr int n = V >= 2 ? V / 2 : 1; };
+
+// V consecutive float32 parameters (weights or biases) starting at p, as float2 pairs.
+// V >= 2 needs p 8-byte aligned; V == 1 reads one float.
+template <int V>
+__device__ __forceinline__ void load_param(const float *p, float2 (&f)[Pairs<V>::n]) {
+    if constexpr (V == 1) {
+        f[0] = make_float2(__ldg(p), 0.f);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V / 2; ++i) f[i] = __ldg(reinterpret_cast<const float2 *>(p) + i);
+    }
+}
+
+__device__ __forceinline__ int64_t clamp_len(const int32_t *lengths, int64_t b, int64_t T) {
+    if (lengths == nullptr) return T;
+    int64_t L = __ldg(lengths + b);
+    return L < 0 ? 0 : (L > T ? T : L);
+}
+
+}  // namespace dwk

@@ -1,0 +1,57 @@
+// Internal launch interface between the C ABI layer (api.cu) and the kernels.
+// Arguments arrive here already validated; launchers only pick a kernel and launch it.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "dw_common.cuh"
+
+namespace dwk {
+
+constexpr int64_t kMaxGrid = 0x7fffffffLL;
+
+struct Conv1dArgs {
+    const void *x;        // input [B][T][C] (dy for the data gradient)
+    const float *w;       // [K][C]
+    const float *bias;    // [C] or null
+    void *y;              // output [B][T][C]
+    const int32_t *lengths;
+    int64_t B, T, C;
+    int K;
+    int pad_left;         // left pad of THIS correlation (already swapped for the data gradient)
+    int flip;             // 1: use w[K-1-k] as tap k
+    int bf16;             // 1: bf16 I/O, 0: float32 I/O
+    int vec_width;        // 2: even-channel vector path allowed; 1: scalar path
+};
+
+struct DwArgs {
+    const void *x, *dy;
+    float *dw, *dbias;
+    const int32_t *lengths;
+    int64_t B, T, C;
+    int K, pad_left, bf16, vec_width;
+    float *partials;      // workspace: [G][K+1][C] float32
+    int G;                // partial rows (blocks per channel tile)
+};
+
+struct SubsampleArgs {
+    const float *mel, *w0, *b0, *w1, *b1;
+    void *out;
+    const int32_t *lengths;
+    int32_t *out_lengths;
+    int64_t B, T, F, C;
+    int causal, bf16_out;
+};
+
+cudaError_t conv1d_fwd_launch(const Conv1dArgs &a, cudaStream_t s);
+
+// dW/dbias: the number of partial rows G and the workspace bytes follow from the sizes alone.
+int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t C, int K);
+size_t conv1d_dw_workspace_bytes(int64_t B, int64_t T, int64_t C, int K);
+cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s);
+
+cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
+
+}  // namespace dwk
