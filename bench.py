@@ -300,7 +300,7 @@ def main():
                                                         dw.DW_BF16, ctypes.c_void_p(sp))),
         ])
     rows = [c[0] for c in calls[0]]
-    launches_per_row = {"dwconv1d_fwd": 1, "dwconv1d_bwd_dx": 1, "dwconv1d_bwd_dw": 2, "dw_subsample_fwd": 2}
+    launches_per_row = {"dwconv1d_fwd": 1, "dwconv1d_bwd_dx": 1, "dwconv1d_bwd_dw": 2, "dw_subsample_fwd": 1}
 
     def run_step(i, evs=None):
         for j, (name, fn, a) in enumerate(calls[i % N_SETS]):

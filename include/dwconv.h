@@ -17,6 +17,7 @@
  *    as zero; invalid output frames are written as +0.0.
  *  - Errors: every call returns a dw_status_t and never aborts or traps.  Argument errors
  *    are found on the host before any CUDA call.  A failed launch returns DW_ERR_CUDA.
+ *    C above 4,194,304 channels or K above 4096 returns DW_ERR_UNSUPPORTED.
  *    B == 0 or T == 0 is a valid no-op.  Misaligned pointers, or a C that is not a
  *    multiple of the vector width, take a narrower (slower) path and stay correct.
  *  - Arithmetic: bf16 or float32 I/O, float32 accumulation, bf16 stores rounded to
@@ -38,7 +39,7 @@ typedef enum dw_status {
     DW_ERR_UNSUPPORTED = 2,  /* a valid request this build cannot serve (e.g. no sm_100 device) */
     DW_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the *_workspace_size result */
     DW_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
-    DW_ERR_TIMEOUT = 5       /* reserved: no kernel of this library waits on another */
+    DW_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel gave up (see dw_device_error) */
 } dw_status_t;
 
 typedef enum dw_dtype {
@@ -150,6 +151,16 @@ const char *dw_status_string(dw_status_t status);
 
 /* dw_last_cuda_error - the cudaError_t behind the most recent DW_ERR_CUDA on this thread. */
 int dw_last_cuda_error(void);
+
+/*
+ * dw_device_error - reads and clears the device-side error words of the library's kernels.
+ * Pipelined kernels wait on shared-memory barriers for their own bulk copies; every such
+ * wait is bounded, and a wait that gives up records an error here instead of hanging.
+ * SYNCHRONOUS: waits for all work on the current device.  Returns DW_OK when no kernel
+ * recorded an error since the previous call, DW_ERR_TIMEOUT when one did, DW_ERR_CUDA when
+ * the query itself failed.
+ */
+dw_status_t dw_device_error(void);
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,7 @@ __all__ = [
     "DW_OK", "DW_ERR_INVALID_ARG", "DW_ERR_UNSUPPORTED", "DW_ERR_WORKSPACE", "DW_ERR_CUDA",
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
-    "dw_subsample_fwd", "dw_status_string", "subsample_out_shape",
+    "dw_subsample_fwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
 ]
 
 DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_WORKSPACE, DW_ERR_CUDA, DW_ERR_TIMEOUT = range(6)
@@ -46,6 +46,7 @@ SIGNATURES = {
                                 _int, _int, _vp]),
     "dw_status_string": (ctypes.c_char_p, [_int]),
     "dw_last_cuda_error": (_int, []),
+    "dw_device_error": (_int, []),
 }
 
 
@@ -115,6 +116,11 @@ def _stream(stream):
 
 def dw_status_string(status: int) -> str:
     return lib().dw_status_string(int(status)).decode()
+
+
+def dw_device_error() -> int:
+    """Reads and clears the kernels' device error words (synchronous); DW_OK if none was set."""
+    return int(lib().dw_device_error())
 
 
 def dwconv1d_fwd(x, w, bias, y, lengths, pad_left, stream=None):

@@ -47,8 +47,8 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def _compile(src, extra):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src, extra, objdir=BUILD):
+    obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
     cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
@@ -56,24 +56,27 @@ def _compile(src, extra):
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile the library if any source is newer than it; returns its path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB, objdir: str = BUILD) -> str:
+    """Compile the library if any source is newer than it; returns its path.
+
+    ``extra`` adds nvcc flags; ``out``/``objdir`` place a separately configured copy elsewhere.
+    """
+    if not force and out == LIB and not _stale():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    os.makedirs(objdir, exist_ok=True)
     extra = list(extra) + (["-Xptxas", "-v"] if verbose else [])
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(lambda s: _compile(s, extra), _sources()))
+        results = list(ex.map(lambda s: _compile(s, extra, objdir), _sources()))
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *[o for o, _ in results]]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

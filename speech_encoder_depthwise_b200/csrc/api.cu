@@ -42,21 +42,29 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 bool aligned(const void *p, size_t n) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % n == 0; }
 
-// Channel-pair vector path: C even, activations aligned to one pair, parameters to float2.
+// Widest channel vector (4, 2 or 1 channels) that C and every pointer allow: activations
+// aligned to the vector, float32 parameters to 8 bytes (they are read as float2).
 int pick_vec_width(int64_t C, size_t esize, std::initializer_list<const void *> acts,
                    std::initializer_list<const void *> params) {
-    if (C % 2 != 0) return 1;
-    for (const void *p : acts)
-        if (!aligned(p, 2 * esize)) return 1;
     for (const void *p : params)
         if (!aligned(p, 8)) return 1;
-    return 2;
+    for (int v : {4, 2}) {
+        if (C % v != 0) continue;
+        bool ok = true;
+        for (const void *p : acts) ok = ok && aligned(p, v * esize);
+        if (ok) return v;
+    }
+    return 1;
 }
+
+// Channel counts beyond this are rejected: frame offsets are kept in 32 bits inside a run.
+constexpr int64_t kMaxChannels = 1 << 22;
 
 dw_status_t check_conv1d_common(const void *in, const float *w, const void *out, int64_t B, int64_t T,
                                 int64_t C, int K, int pad_left, dw_dtype_t dt, int64_t *n) {
     if (!valid_dtype(dt)) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
+    if (C > kMaxChannels || K > 4096) return DW_ERR_UNSUPPORTED;
     if (!mul3(B, T, C, n)) return DW_ERR_INVALID_ARG;
     if (*n == 0) return DW_OK;
     if (in == nullptr || w == nullptr || out == nullptr) return DW_ERR_INVALID_ARG;
@@ -82,6 +90,12 @@ const char *dw_status_string(dw_status_t s) {
 }
 
 int dw_last_cuda_error(void) { return g_last_cuda_error; }
+
+dw_status_t dw_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+    const unsigned int e = dwk::conv1d_fwd_take_error() | dwk::conv1d_dw_take_error();
+    return e ? DW_ERR_TIMEOUT : DW_OK;
+}
 
 dw_status_t dwconv1d_fwd(const void *x, const float *w, const float *bias, void *y, const int32_t *lengths,
                          int64_t B, int64_t T, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
@@ -168,15 +182,14 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
             return DW_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (nout > 0) {
+    if (nout > 0) {  // the fused kernel also writes out_lengths
         dwk::SubsampleArgs a;
         a.mel = mel; a.w0 = w0; a.b0 = b0; a.w1 = w1; a.b1 = b1; a.out = out;
         a.lengths = lengths; a.out_lengths = out_lengths;
         a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.bf16_out = out_dtype == DW_BF16;
-        dw_status_t st = cuda_status(dwk::subsample_launch(a, s));
-        if (st != DW_OK) return st;
+        return cuda_status(dwk::subsample_launch(a, s));
     }
-    if (out_lengths != nullptr && B > 0)
+    if (out_lengths != nullptr && B > 0)  // no frames: only the (zero) output lengths
         return cuda_status(dwk::subsample_out_lengths_launch(lengths, out_lengths, B, T, s));
     return DW_OK;
 }

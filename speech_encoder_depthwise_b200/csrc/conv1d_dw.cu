@@ -29,12 +29,14 @@ namespace dwk {
 constexpr int kDwThreads = 256;
 constexpr int kDwCluster = 8;
 constexpr int kDwTapBlock = 8;   // taps per pass for widths without a specialisation
+constexpr int kDwMaxRows = 64;   // partial rows at most (clusters per channel tile)
+constexpr int kDwMaxRows16 = 16; // partial rows of the register-tiled kernel
 
 template <typename T, int V, int KB, int R>
-__global__ void __cluster_dims__(kDwCluster, 1, 1) __launch_bounds__(kDwThreads)
+__global__ void __cluster_dims__(kDwCluster, 1, 1) __launch_bounds__(kDwThreads, 2)
 conv1d_dw_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
                          const int32_t *__restrict__ lengths, float *__restrict__ partials,
-                         int64_t B, int64_t Tn, int64_t C, int K, int k_off, int pad_left, int TX,
+                         int64_t B, int64_t Tn, int C, int K, int k_off, int pad_left, int TX,
                          int nTC, int with_bias) {
     extern __shared__ float smem[];  // [TY][KB+1][CT]
     constexpr int NP = Pairs<V>::n;
@@ -43,8 +45,9 @@ conv1d_dw_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
     const int CT = TX * V;
     const int g = blockIdx.x, G = gridDim.x;
     const int ct = blockIdx.y;
-    const int64_t c0 = (static_cast<int64_t>(ct) * TX + tx) * V;
+    const int c0 = (ct * TX + tx) * V;
     const bool active = c0 < C;
+    const uint32_t rs = static_cast<uint32_t>(C) * sizeof(T);
 
     float2 acc[KB][NP], accb[NP];
 #pragma unroll
@@ -62,36 +65,54 @@ conv1d_dw_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
             const int64_t t0 = (u % nTC) * TU + static_cast<int64_t>(ty) * R;
             const int64_t L = clamp_len(lengths, b, Tn);
             if (t0 >= L) continue;
-            const T *xb = x + b * Tn * C + c0;
-            const T *db = dy + b * Tn * C + c0;
+            const char *xi = reinterpret_cast<const char *>(x + b * Tn * C + c0);
+            const char *di = reinterpret_cast<const char *>(dy + b * Tn * C + c0);
+            const int64_t j0 = t0 + k_off - pad_left;  // x frame paired with dz[t0] through tap k_off
             Vec<T, V> rdy[R], rx[R + KB - 1];
+            if (t0 + R <= L && j0 >= 0 && j0 + R + KB - 1 <= L) {  // every frame of the run is valid
+                const char *dp = di + t0 * rs;
+                const char *xp = xi + j0 * rs;
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                if (t0 + r < L) rdy[r].load(db + (t0 + r) * C);
-                else rdy[r].zero();
-            }
+                for (int r = 0; r < R; ++r) rdy[r].load(reinterpret_cast<const T *>(dp + static_cast<uint32_t>(r) * rs));
 #pragma unroll
-            for (int i = 0; i < R + KB - 1; ++i) {
-                const int64_t j = t0 + k_off - pad_left + i;
-                if (j >= 0 && j < L) rx[i].load(xb + j * C);
-                else rx[i].zero();
-            }
-            float2 xf[R + KB - 1][NP];
+                for (int i = 0; i < R + KB - 1; ++i)
+                    rx[i].load(reinterpret_cast<const T *>(xp + static_cast<uint32_t>(i) * rs));
+            } else {
 #pragma unroll
-            for (int i = 0; i < R + KB - 1; ++i) rx[i].to_f2(xf[i]);
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float2 dz[NP];
-                rdy[r].to_f2(dz);
-#pragma unroll
-                for (int p = 0; p < NP; ++p) {
-                    accb[p].x += dz[p].x;
-                    accb[p].y += dz[p].y;
+                for (int r = 0; r < R; ++r) {
+                    if (t0 + r < L) rdy[r].load(reinterpret_cast<const T *>(di + (t0 + r) * rs));
+                    else rdy[r].zero();
                 }
 #pragma unroll
-                for (int k = 0; k < KB; ++k)
+                for (int i = 0; i < R + KB - 1; ++i) {
+                    const int64_t j = j0 + i;
+                    if (j >= 0 && j < L) rx[i].load(reinterpret_cast<const T *>(xi + j * rs));
+                    else rx[i].zero();
+                }
+            }
+            float2 dz[R][NP];
 #pragma unroll
-                    for (int p = 0; p < NP; ++p) acc[k][p] = ffma2(dz[p], xf[r + k][p], acc[k][p]);
+            for (int r = 0; r < R; ++r) {
+                rdy[r].to_f2(dz[r]);
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    accb[p].x += dz[r][p].x;
+                    accb[p].y += dz[r][p].y;
+                }
+            }
+            // x frame i meets dz[r] through tap k = i - r
+#pragma unroll
+            for (int i = 0; i < R + KB - 1; ++i) {
+                float2 xf[NP];
+                rx[i].to_f2(xf);
+#pragma unroll
+                for (int k = 0; k < KB; ++k) {
+                    const int r = i - k;
+                    if (r >= 0 && r < R) {
+#pragma unroll
+                        for (int p = 0; p < NP; ++p) acc[k][p] = ffma2(dz[r][p], xf[p], acc[k][p]);
+                    }
+                }
             }
         }
     }
@@ -137,6 +158,185 @@ conv1d_dw_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
     cluster.sync();  // keep this block's shared memory alive until every rank has read it
 }
 
+// ---------------------------------------------------------------------------------------
+// Pipelined variant (16-byte frame rows, specialised K): grid (G, channel tiles), 2 blocks per
+// SM, clusters of 1-8 blocks along G chosen at launch.  Warp 0 streams each unit into a
+// kDwStages-deep shared-memory ring with two tensor copies (x: the TT frames plus the halo,
+// dy: the TT frames), counted in bytes on the stage's "full" mbarrier; 8 consumer warps
+// accumulate dW/dbias for their R frames in registers across all units the block is dealt,
+// then release the stage on its "empty" mbarrier.  At the end every warp (the producer adds
+// zeros) joins the block and cluster reductions of the register-tiled kernel above.
+// ---------------------------------------------------------------------------------------
+constexpr int kDwConsumers = 8;
+constexpr int kDwR = 8;
+constexpr int kDwStages = 3;
+constexpr int kDwTmaThreads = 32 * (1 + kDwConsumers);
+
+template <typename T, int V, int KB>
+struct DwTmaShape {
+    static constexpr int CT = 32 * V;
+    static constexpr int TT = kDwConsumers * kDwR;
+    static constexpr int XROWS = TT + KB - 1;
+    static constexpr int ROWB = CT * static_cast<int>(sizeof(T));
+    static constexpr int STAGE_BYTES = (XROWS + TT) * ROWB;
+    static constexpr int RED_BYTES = kDwConsumers * (KB + 1) * CT * 4;
+    static constexpr int BODY = (kDwStages * STAGE_BYTES > RED_BYTES) ? kDwStages * STAGE_BYTES : RED_BYTES;
+    static constexpr int SMEM = 128 + BODY;
+};
+
+template <typename T, int V, int KB>
+__global__ void __launch_bounds__(kDwTmaThreads, 2)
+conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
+                     const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C, int K,
+                     int k_off, int pad_left, int nT, int with_bias) {
+    using S = DwTmaShape<T, V, KB>;
+    constexpr int NP = Pairs<V>::n;
+    constexpr int R = kDwR;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw);
+    uint64_t *empty = full + kDwStages;
+    unsigned char *stages = smem_raw + 128;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int g = blockIdx.x, G = gridDim.x, ct = blockIdx.y;
+    const int c0 = ct * S::CT;
+    const int units = B * nT;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDwStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kDwConsumers);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    float2 acc[KB][NP], accb[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        accb[p] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < KB; ++k) acc[k][p] = make_float2(0.f, 0.f);
+    }
+    bool ok = true;
+
+    if (warp == 0) {  // producer warp: one elected lane, two tensor copies (x with halo, dy) per unit
+        if (lane == 0) {
+            prefetch_tmap(&xmap);
+            prefetch_tmap(&dmap);
+        }
+        int it = 0;
+        for (int u = g; u < units && ok; u += G, ++it) {
+            const int s = it % kDwStages;
+            const uint32_t ph = (it / kDwStages) & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1));
+            if (!ok) break;
+            if (lane == 0) {
+                const int b = u / nT, t0 = (u % nT) * S::TT;
+                const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+                if (t0 < L) {  // frames before 0 or past T arrive as zeros; [L, T) is masked by the consumers
+                    unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+                    tma_load_3d(st, &xmap, c0, t0 + k_off - pad_left, b, &full[s]);
+                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, t0, b, &full[s]);
+                } else {
+                    mbar_arrive(&full[s]);  // a wholly masked unit: nothing to read
+                }
+            }
+            __syncwarp();
+        }
+    } else {  // consumer warp cw computes frames [t0 + cw R, t0 + cw R + R) of every unit
+        const int cw = warp - 1;
+        const bool active = c0 + lane * V < C;
+        int it = 0;
+        for (int u = g; u < units && ok; u += G, ++it) {
+            const int s = it % kDwStages;
+            const uint32_t ph = (it / kDwStages) & 1;
+            const int b = u / nT, t0 = (u % nT) * S::TT;
+            const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+            ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph));
+            if (!ok) break;
+            const int tg = t0 + cw * R;
+            if (active && tg < L) {
+                const unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES + lane * V * sizeof(T);
+                const unsigned char *dp = st + (S::XROWS + cw * R) * S::ROWB;
+                const unsigned char *xp = st + (cw * R) * S::ROWB;
+                const int jb = tg + k_off - pad_left;  // frame of this thread's first x row
+                const bool all_valid = tg + R <= L && jb >= 0 && jb + R + KB - 1 <= L;
+                float2 dz[R][NP];
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    Vec<T, V> v;
+                    v.r = *reinterpret_cast<const decltype(v.r) *>(dp + r * S::ROWB);
+                    if (!all_valid && tg + r >= L) v.zero();
+                    v.to_f2(dz[r]);
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) {
+                        accb[p].x += dz[r][p].x;
+                        accb[p].y += dz[r][p].y;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < R + KB - 1; ++i) {
+                    Vec<T, V> v;
+                    v.r = *reinterpret_cast<const decltype(v.r) *>(xp + i * S::ROWB);
+                    if (!all_valid && (jb + i < 0 || jb + i >= L)) v.zero();
+                    float2 xf[NP];
+                    v.to_f2(xf);
+#pragma unroll
+                    for (int k = 0; k < KB; ++k) {
+                        const int r = i - k;
+                        if (r >= 0 && r < R) {
+#pragma unroll
+                            for (int p = 0; p < NP; ++p) acc[k][p] = ffma2(dz[r][p], xf[p], acc[k][p]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+    }
+    // every warp has left the pipeline; the stage memory now holds the block reduction
+    __syncthreads();
+    const int E = (KB + 1) * S::CT;
+    float *red = reinterpret_cast<float *>(stages);
+    if (warp > 0) {
+        float *mine = red + static_cast<size_t>(warp - 1) * E;
+#pragma unroll
+        for (int k = 0; k <= KB; ++k) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                const float2 v = (k < KB) ? acc[k][p] : accb[p];
+                if (2 * p < V) mine[k * S::CT + lane * V + 2 * p] = v.x;
+                if (2 * p + 1 < V) mine[k * S::CT + lane * V + 2 * p + 1] = v.y;
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float sum = red[e];
+        for (int r = 1; r < kDwConsumers; ++r) sum += red[static_cast<size_t>(r) * E + e];
+        red[e] = sum;
+    }
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int nrank = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int chunk = (E + nrank - 1) / nrank;
+    const int64_t prow = g / nrank;
+    for (int e = rank * chunk + threadIdx.x; e < min(E, (rank + 1) * chunk); e += blockDim.x) {
+        float sum = 0.f;
+        for (int q = 0; q < nrank; ++q) sum += cluster.map_shared_rank(red, q)[e];
+        const int kk = e / S::CT;
+        const int64_t c = static_cast<int64_t>(c0) + (e % S::CT);
+        if (c >= C) continue;
+        if (kk == KB) {
+            if (with_bias) partials[(prow * (K + 1) + K) * C + c] = sum;
+        } else if (k_off + kk < K) {
+            partials[(prow * (K + 1) + k_off + kk) * C + c] = sum;
+        }
+    }
+    cluster.sync();
+}
+
 __global__ void __launch_bounds__(256)
 conv1d_dw_finalize_kernel(const float *__restrict__ partials, float *__restrict__ dw,
                           float *__restrict__ dbias, int Gp, int K, int64_t C) {
@@ -155,12 +355,14 @@ __global__ void conv1d_dw_zero_kernel(float *__restrict__ dw, float *__restrict_
     if (dbias && e < C) dbias[e] = 0.f;
 }
 
+// Upper bound on the partial rows (one per cluster of blocks per channel tile); the workspace
+// is sized for it, so it depends on the sizes alone.
 int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t /*C*/, int /*K*/) {
     const int64_t frames = B * T;
     if (frames <= 0) return 0;
-    int64_t gp = (frames + 2047) / 2048;
+    int64_t gp = (frames + 255) / 256;
     if (gp < 1) gp = 1;
-    if (gp > 16) gp = 16;
+    if (gp > kDwMaxRows) gp = kDwMaxRows;
     return static_cast<int>(gp);
 }
 
@@ -177,50 +379,165 @@ int pow2_at_most(int64_t v, int cap) {
     return p;
 }
 
+// Partial rows actually used: enough clusters to fill every SM once (two blocks per SM), at most
+// the workspace's row count.  Fixed for given sizes on a given GPU, so results are reproducible.
+int used_rows(int max_rows, int nCT, int blocks_per_sm) {
+    const int64_t slots = static_cast<int64_t>(sm_count()) * blocks_per_sm;
+    int64_t gp = slots / (static_cast<int64_t>(kDwCluster) * nCT);
+    if (gp < 1) gp = 1;
+    if (gp > max_rows) gp = max_rows;
+    return static_cast<int>(gp);
+}
+
 template <typename T, int V, int KB>
-cudaError_t launch_pass(const DwArgs &a, int k_off, int with_bias, cudaStream_t s) {
-    constexpr int R = (KB <= 9) ? 16 : 8;
+cudaError_t launch_pass(const DwArgs &a, int gp, int k_off, int with_bias, cudaStream_t s) {
+    constexpr int R = (V >= 4 || KB > 9) ? 8 : 16;
     const int64_t Cv = (a.C + V - 1) / V;
     const int TX = pow2_at_most(Cv, 32);
     const int TY = kDwThreads / TX;
     const int nCT = static_cast<int>((Cv + TX - 1) / TX);
     const int nTC = static_cast<int>((a.T + static_cast<int64_t>(TY) * R - 1) / (static_cast<int64_t>(TY) * R));
-    const int G = a.G * kDwCluster;
     if (nCT > 65535) return cudaErrorInvalidConfiguration;
     const size_t smem = static_cast<size_t>(TY) * (KB + 1) * TX * V * sizeof(float);
-    conv1d_dw_partial_kernel<T, V, KB, R><<<dim3(G, nCT), kDwThreads, smem, s>>>(
+    conv1d_dw_partial_kernel<T, V, KB, R><<<dim3(gp * kDwCluster, nCT), kDwThreads, smem, s>>>(
         static_cast<const T *>(a.x), static_cast<const T *>(a.dy), a.lengths, a.partials, a.B, a.T,
-        a.C, a.K, k_off, a.pad_left, TX, nTC, with_bias);
+        static_cast<int>(a.C), a.K, k_off, a.pad_left, TX, nTC, with_bias);
     return cudaGetLastError();
 }
 
-template <typename T, int V>
-cudaError_t launch_partials(const DwArgs &a, cudaStream_t s) {
-    switch (a.K) {
-        case 1: return launch_pass<T, V, 1>(a, 0, 1, s);
-        case 2: return launch_pass<T, V, 2>(a, 0, 1, s);
-        case 3: return launch_pass<T, V, 3>(a, 0, 1, s);
-        case 4: return launch_pass<T, V, 4>(a, 0, 1, s);
-        case 5: return launch_pass<T, V, 5>(a, 0, 1, s);
-        case 7: return launch_pass<T, V, 7>(a, 0, 1, s);
-        case 9: return launch_pass<T, V, 9>(a, 0, 1, s);
-        case 15: return launch_pass<T, V, 15>(a, 0, 1, s);
-        default:
-            for (int k_off = 0; k_off < a.K; k_off += kDwTapBlock) {
-                cudaError_t e = launch_pass<T, V, kDwTapBlock>(a, k_off, k_off == 0, s);
-                if (e != cudaSuccess) return e;
-            }
-            return cudaSuccess;
+// Grid rows G and cluster size for the pipelined kernel: as many blocks per channel tile as
+// fit on the device at once, in clusters as large as that allows (fewer partial rows).
+template <typename T, int V, int KB>
+cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s) {
+    using S = DwTmaShape<T, V, KB>;
+    auto kern = conv1d_dw_tma_kernel<T, V, KB>;
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::SMEM);
+    if (attr != cudaSuccess) return attr;
+    const int nCT = static_cast<int>((a.C + S::CT - 1) / S::CT);
+    const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
+    const int64_t units = a.B * nT;
+    if (nCT > 65535 || units >= (1LL << 31)) return cudaErrorInvalidConfiguration;
+    int best_g = 0, best_c = 1;
+    for (int c : {8, 4, 2, 1}) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(c, nCT);
+        q.blockDim = dim3(kDwTmaThreads);
+        q.dynamicSmemBytes = S::SMEM;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = c;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        q.attrs = at;
+        q.numAttrs = 1;
+        int nclu = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclu, kern, &q) != cudaSuccess || nclu < 1) {
+            (void)cudaGetLastError();
+            continue;
+        }
+        int64_t gg = (static_cast<int64_t>(nclu) * c / nCT) / c * c;  // blocks per channel tile
+        const int64_t ucap = (units + c - 1) / c * c;                  // no more blocks than units
+        if (gg > ucap) gg = ucap;
+        if (gg / c > a.G) gg = static_cast<int64_t>(a.G) * c;          // workspace rows
+        if (gg > best_g) {
+            best_g = static_cast<int>(gg);
+            best_c = c;
+        }
     }
+    if (best_g < 1) return cudaErrorInvalidConfiguration;
+    *gp_out = best_g / best_c;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(best_g, nCT);
+    cfg.blockDim = dim3(kDwTmaThreads);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = best_c;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    CUtensorMap xmap, dmap;
+    cudaError_t me = make_act_map(&xmap, a.x, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::XROWS);
+    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::TT);
+    if (me != cudaSuccess) return me;
+    return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, a.lengths, a.partials, static_cast<int>(a.B),
+                              static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias);
 }
 
 template <typename T>
-cudaError_t launch_dtype(const DwArgs &a, cudaStream_t s) {
-    if (a.vec_width >= 2) return launch_partials<T, 2>(a, s);
-    return launch_partials<T, 1>(a, s);
+bool dw_tma_ok(const DwArgs &a) {
+    return (a.C * static_cast<int64_t>(sizeof(T))) % 16 == 0 && reinterpret_cast<uintptr_t>(a.x) % 16 == 0 &&
+           reinterpret_cast<uintptr_t>(a.dy) % 16 == 0 && a.T < (1LL << 30) && a.B < (1LL << 30) &&
+           a.B * a.T < (1LL << 31);
+}
+
+template <typename T, int V>
+int channel_tiles(int64_t C) {
+    const int64_t Cv = (C + V - 1) / V;
+    const int TX = pow2_at_most(Cv, 32);
+    return static_cast<int>((Cv + TX - 1) / TX);
+}
+
+template <typename T, int V>
+cudaError_t launch_partials(const DwArgs &a, int *gp_out, cudaStream_t s) {
+    if constexpr (V >= 2) {
+        if (dw_tma_ok<T>(a)) {
+            switch (a.K) {
+                case 1: return launch_tma_pass<T, V, 1>(a, 0, 1, gp_out, s);
+                case 2: return launch_tma_pass<T, V, 2>(a, 0, 1, gp_out, s);
+                case 3: return launch_tma_pass<T, V, 3>(a, 0, 1, gp_out, s);
+                case 4: return launch_tma_pass<T, V, 4>(a, 0, 1, gp_out, s);
+                case 5: return launch_tma_pass<T, V, 5>(a, 0, 1, gp_out, s);
+                case 7: return launch_tma_pass<T, V, 7>(a, 0, 1, gp_out, s);
+                case 9: return launch_tma_pass<T, V, 9>(a, 0, 1, gp_out, s);
+                default: break;
+            }
+            if constexpr (V == 2) {
+                if (a.K == 15) return launch_tma_pass<T, V, 15>(a, 0, 1, gp_out, s);
+            }
+        }
+    }
+    const int gp = used_rows(a.G < kDwMaxRows16 ? a.G : kDwMaxRows16, channel_tiles<T, V>(a.C), 2);
+    *gp_out = gp;
+    switch (a.K) {
+        case 1: return launch_pass<T, V, 1>(a, gp, 0, 1, s);
+        case 2: return launch_pass<T, V, 2>(a, gp, 0, 1, s);
+        case 3: return launch_pass<T, V, 3>(a, gp, 0, 1, s);
+        case 4: return launch_pass<T, V, 4>(a, gp, 0, 1, s);
+        case 5: return launch_pass<T, V, 5>(a, gp, 0, 1, s);
+        case 7: return launch_pass<T, V, 7>(a, gp, 0, 1, s);
+        case 9: return launch_pass<T, V, 9>(a, gp, 0, 1, s);
+        default: break;
+    }
+    if constexpr (V <= 2) {
+        if (a.K == 15) return launch_pass<T, V, 15>(a, gp, 0, 1, s);
+    }
+    for (int k_off = 0; k_off < a.K; k_off += kDwTapBlock) {
+        cudaError_t e = launch_pass<T, (V > 2 ? 2 : V), kDwTapBlock>(a, gp, k_off, k_off == 0, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t launch_dtype(const DwArgs &a, int *gp, cudaStream_t s) {
+    if constexpr (sizeof(T) == 2) {
+        if (a.vec_width >= 4 && a.K <= 9) return launch_partials<T, 4>(a, gp, s);
+    }
+    if (a.vec_width >= 2) return launch_partials<T, 2>(a, gp, s);
+    return launch_partials<T, 1>(a, gp, s);
 }
 
 }  // namespace
+
+unsigned int conv1d_dw_take_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, dw_device_error_flag, sizeof(v)) != cudaSuccess) return 0;
+    if (v) cudaMemcpyToSymbol(dw_device_error_flag, &zero, sizeof(zero));
+    return v;
+}
 
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
     const int64_t n = static_cast<int64_t>(a.K + 1) * a.C;
@@ -228,10 +545,11 @@ cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
         conv1d_dw_zero_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(a.dw, a.dbias, a.K, a.C);
         return cudaGetLastError();
     }
-    cudaError_t e = a.bf16 ? launch_dtype<bf16>(a, s) : launch_dtype<float>(a, s);
+    int gp = 0;
+    cudaError_t e = a.bf16 ? launch_dtype<bf16>(a, &gp, s) : launch_dtype<float>(a, &gp, s);
     if (e != cudaSuccess) return e;
     conv1d_dw_finalize_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(a.partials, a.dw, a.dbias,
-                                                                                   a.G, a.K, a.C);
+                                                                                   gp, a.K, a.C);
     return cudaGetLastError();
 }
 

@@ -28,81 +28,246 @@
 namespace dwk {
 
 template <typename T, int V, int K, int R>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 conv1d_fwd_vec_kernel(const T *__restrict__ x, const float *__restrict__ w,
                       const float *__restrict__ bias, T *__restrict__ y,
-                      const int32_t *__restrict__ lengths, int64_t Tn, int64_t C, int pad_left,
-                      int flip, int TX, int nT, int nC) {
+                      const int32_t *__restrict__ lengths, int64_t Tn, int C, int pad_left,
+                      int flip, int TX, int nT, int nC, int64_t units) {
     constexpr int NP = Pairs<V>::n;
     const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;
     const int TY = blockDim.x / TX;
-    int64_t lin = blockIdx.x;
-    const int ct = static_cast<int>(lin % nC);
-    lin /= nC;
-    const int tt = static_cast<int>(lin % nT);
-    const int64_t b = lin / nT;
-    const int64_t c0 = (static_cast<int64_t>(ct) * TX + tx) * V;
+    // The grid is a multiple of nC and units run channel-tile fastest, so a block keeps one
+    // channel tile (and its weights in registers) for every unit it is dealt.
+    const int ct = static_cast<int>(blockIdx.x % nC);
+    const int c0 = (ct * TX + tx) * V;
     if (c0 >= C) return;
-    const int64_t t0 = (static_cast<int64_t>(tt) * TY + ty) * R;
-    if (t0 >= Tn) return;
-    const int64_t L = clamp_len(lengths, b, Tn);
-    const T *xb = x + b * Tn * C + c0;
-    T *yb = y + b * Tn * C + c0;
+    const uint32_t rs = static_cast<uint32_t>(C) * sizeof(T);  // bytes between frames
 
-    if (t0 >= L) {  // the whole run is masked: zeros only, nothing read
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-            if (t0 + r < Tn) Vec<T, V>::store_zero(yb + (t0 + r) * C);
-        return;
-    }
-
-    Vec<T, V> raw[R + K - 1];
-#pragma unroll
-    for (int i = 0; i < R + K - 1; ++i) {
-        const int64_t j = t0 - pad_left + i;
-        if (j >= 0 && j < L) raw[i].load(xb + j * C);
-        else raw[i].zero();
-    }
-
-    float2 wv[K][NP];
+    float2 wv[K][NP], bv[NP];
 #pragma unroll
     for (int k = 0; k < K; ++k) load_param<V>(w + static_cast<int64_t>(flip ? K - 1 - k : k) * C + c0, wv[k]);
-    float2 acc[R][NP];
-    {
-        float2 bv[NP];
-        if (bias) load_param<V>(bias + c0, bv);
-        else {
+    if (bias) load_param<V>(bias + c0, bv);
+    else {
 #pragma unroll
-            for (int p = 0; p < NP; ++p) bv[p] = make_float2(0.f, 0.f);
+        for (int p = 0; p < NP; ++p) bv[p] = make_float2(0.f, 0.f);
+    }
+
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+        const int64_t bt = u / nC;
+        const int64_t b = bt / nT;
+        const int64_t t0 = ((bt % nT) * TY + ty) * R;
+        if (t0 >= Tn) continue;
+        const int64_t L = clamp_len(lengths, b, Tn);
+        const char *xi = reinterpret_cast<const char *>(x + b * Tn * C + c0);  // frame 0 of item b
+        char *yt = reinterpret_cast<char *>(y + (b * Tn + t0) * C + c0);      // frame t0 of item b
+        if (t0 >= L) {  // the whole run is masked: zeros only, nothing read
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (t0 + r < Tn) Vec<T, V>::store_zero(reinterpret_cast<T *>(yt + static_cast<uint32_t>(r) * rs));
+            continue;
         }
+        const int64_t j0 = t0 - pad_left;
+        Vec<T, V> raw[R + K - 1];
+        if (j0 >= 0 && j0 + R + K - 1 <= L) {  // every input frame of the run is valid
+            const char *xj = xi + j0 * rs;
+#pragma unroll
+            for (int i = 0; i < R + K - 1; ++i)
+                raw[i].load(reinterpret_cast<const T *>(xj + static_cast<uint32_t>(i) * rs));
+        } else {
+#pragma unroll
+            for (int i = 0; i < R + K - 1; ++i) {
+                const int64_t j = j0 + i;
+                if (j >= 0 && j < L) raw[i].load(reinterpret_cast<const T *>(xi + j * rs));
+                else raw[i].zero();
+            }
+        }
+        const bool full = t0 + R <= L;  // every output of the run is valid
+        float2 acc[R][NP];
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
             for (int p = 0; p < NP; ++p) acc[r][p] = bv[p];
+        // input frame i feeds output r = i - k through tap k; output r is complete after i = r + K - 1
+#pragma unroll
+        for (int i = 0; i < R + K - 1; ++i) {
+            float2 xf[NP];
+            raw[i].to_f2(xf);
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int r = i - k;
+                if (r >= 0 && r < R) {
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) acc[r][p] = ffma2(xf[p], wv[k][p], acc[r][p]);
+                }
+            }
+            const int rd = i - (K - 1);
+            if (rd >= 0) {
+                T *dst = reinterpret_cast<T *>(yt + static_cast<uint32_t>(rd) * rs);
+                if (full || t0 + rd < L) Vec<T, V>::store(dst, acc[rd]);
+                else if (t0 + rd < Tn) Vec<T, V>::store_zero(dst);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Pipelined variant for the common case (16-byte frame rows, specialised K): a persistent
+// block per SM, one producer warp and kTmaConsumers consumer warps.  For each tile the
+// producer issues ONE tensor copy (cp.async.bulk.tensor: CT channels x (TT + K - 1) frames,
+// starting K-1 halo frames early) into a kTmaStages-deep shared-memory ring; completion is
+// counted in bytes on the stage's "full" mbarrier.  Frames before 0 or past T arrive as zeros
+// (the padding).  Consumers read their R + K - 1 rows from shared memory with the same
+// register window as above, mask frames in [len_b, T), store straight to global memory and
+// release the stage on its "empty" mbarrier.  HBM never waits on compute: up to kTmaStages
+// tiles are in flight per SM while the consumers work on one.  Wholly masked tiles are not
+// read at all.
+// ---------------------------------------------------------------------------------------
+// Tuned on B200 (sweeps over consumer warps, frames per thread, ring depth and blocks per
+// SM): 3 blocks of 4 consumer warps per SM, 3 stages, 12 frames per thread (16 for K > 9).
+#ifndef DW_FWD_CONSUMERS
+#define DW_FWD_CONSUMERS 4
+#endif
+#ifndef DW_FWD_R
+#define DW_FWD_R 12
+#endif
+#ifndef DW_FWD_R_WIDE
+#define DW_FWD_R_WIDE 16
+#endif
+#ifndef DW_FWD_STAGES
+#define DW_FWD_STAGES 3
+#endif
+#ifndef DW_FWD_BLOCKS
+#define DW_FWD_BLOCKS 3
+#endif
+constexpr int kTmaConsumers = DW_FWD_CONSUMERS;  // consumer warps per block
+constexpr int kTmaR = DW_FWD_R;                  // frames per consumer thread, K <= 9
+constexpr int kTmaRWide = DW_FWD_R_WIDE;         // frames per consumer thread, K > 9
+constexpr int kTmaStages = DW_FWD_STAGES;        // shared-memory ring depth
+constexpr int kTmaBlocks = DW_FWD_BLOCKS;        // resident blocks per SM
+constexpr int kTmaThreads = 32 * (1 + kTmaConsumers);
+
+template <typename T, int V, int K>
+struct TmaShape {
+    static constexpr int R = (K > 9) ? kTmaRWide : kTmaR;
+    static constexpr int CT = 32 * V;                 // channels per tile (one warp row)
+    static constexpr int TT = kTmaConsumers * R;      // output frames per tile
+    static constexpr int ROWS = TT + K - 1;           // input rows per tile
+    static constexpr int ROWB = CT * static_cast<int>(sizeof(T));
+    static constexpr int STAGE_BYTES = ROWS * ROWB;
+    static constexpr int SMEM = 128 + kTmaStages * STAGE_BYTES;
+};
+
+template <typename T, int V, int K>
+__global__ void __launch_bounds__(kTmaThreads, kTmaBlocks)
+conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restrict__ w,
+                      const float *__restrict__ bias, T *__restrict__ y, const int32_t *__restrict__ lengths,
+                      int Tn, int C, int pad_left, int flip, int nT, int nC, int ntiles) {
+    using S = TmaShape<T, V, K>;
+    constexpr int NP = Pairs<V>::n;
+    constexpr int R = S::R;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw);
+    uint64_t *empty = full + kTmaStages;
+    unsigned char *stages = smem_raw + 128;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTmaStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kTmaConsumers);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (warp == 0) {  // producer warp: one elected lane, one tensor copy per tile
+        if (lane == 0) prefetch_tmap(&xmap);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int s = it % kTmaStages;
+            const uint32_t ph = (it / kTmaStages) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) return;
+            if (lane == 0) {
+                const int ct = tile % nC, bt = tile / nC;
+                const int t0 = (bt % nT) * S::TT, b = bt / nT;
+                const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+                if (t0 < L) {  // rows before frame 0 or past T arrive as zeros; rows in [L, T) are masked by the consumers
+                    mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+                    tma_load_3d(stages + static_cast<size_t>(s) * S::STAGE_BYTES, &xmap, ct * S::CT, t0 - pad_left, b,
+                                &full[s]);
+                } else {
+                    mbar_arrive(&full[s]);  // a wholly masked tile: nothing to read
+                }
+            }
+            __syncwarp();
+        }
+        return;
     }
 
-    // input frame i feeds output r = i - k through tap k
+    // consumer warps: warp g+1 computes frames [t0 + g R, t0 + g R + R) of each tile
+    const int g = warp - 1;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int s = it % kTmaStages;
+        const uint32_t ph = (it / kTmaStages) & 1;
+        const int ct = tile % nC, bt = tile / nC;
+        const int t0 = (bt % nT) * S::TT, b = bt / nT;
+        const int cv = ct * S::CT + lane * V;
+        const bool active = cv < C;
+        const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+        const int tg = t0 + g * R;
+        float2 wv[K][NP], acc[R][NP];
+        if (active && tg < L) {  // issue the parameter loads before waiting for the tile
 #pragma unroll
-    for (int i = 0; i < R + K - 1; ++i) {
-        float2 xf[NP];
-        raw[i].to_f2(xf);
+            for (int k = 0; k < K; ++k) load_param<V>(w + static_cast<int64_t>(flip ? K - 1 - k : k) * C + cv, wv[k]);
+            float2 bv[NP];
+            if (bias) load_param<V>(bias + cv, bv);
+            else {
 #pragma unroll
-        for (int k = 0; k < K; ++k) {
-            const int r = i - k;
-            if (r >= 0 && r < R) {
+                for (int p = 0; p < NP; ++p) bv[p] = make_float2(0.f, 0.f);
+            }
 #pragma unroll
-                for (int p = 0; p < NP; ++p) acc[r][p] = ffma2(xf[p], wv[k][p], acc[r][p]);
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int p = 0; p < NP; ++p) acc[r][p] = bv[p];
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) return;
+        if (active && tg < Tn) {
+            T *yp = y + (static_cast<int64_t>(b) * Tn + tg) * C + cv;
+            if (tg >= L) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    if (tg + r < Tn) Vec<T, V>::store_zero(yp + static_cast<int64_t>(r) * C);
+            } else {
+                const unsigned char *sp = stages + static_cast<size_t>(s) * S::STAGE_BYTES +
+                                          (g * R) * S::ROWB + lane * V * static_cast<int>(sizeof(T));
+                const int jb = tg - pad_left;  // frame of this thread's first row
+                const bool rows_valid = jb >= 0 && jb + R + K - 1 <= L;
+                const bool outs_valid = tg + R <= L;
+#pragma unroll
+                for (int i = 0; i < R + K - 1; ++i) {
+                    Vec<T, V> v;
+                    v.r = *reinterpret_cast<const decltype(v.r) *>(sp + i * S::ROWB);
+                    if (!rows_valid && (jb + i < 0 || jb + i >= L)) v.zero();
+                    float2 xf[NP];
+                    v.to_f2(xf);
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        const int r = i - k;
+                        if (r >= 0 && r < R) {
+#pragma unroll
+                            for (int p = 0; p < NP; ++p) acc[r][p] = ffma2(xf[p], wv[k][p], acc[r][p]);
+                        }
+                    }
+                    const int rd = i - (K - 1);
+                    if (rd >= 0) {
+                        T *dst = yp + static_cast<int64_t>(rd) * C;
+                        if (outs_valid || tg + rd < L) Vec<T, V>::store(dst, acc[rd]);
+                        else if (tg + rd < Tn) Vec<T, V>::store_zero(dst);
+                    }
+                }
             }
         }
-        // output r = i - (K-1) has received its last term
-        const int rd = i - (K - 1);
-        if (rd >= 0) {
-            const int64_t t = t0 + rd;
-            if (t < Tn) {
-                if (t < L) Vec<T, V>::store(yb + t * C, acc[rd]);
-                else Vec<T, V>::store_zero(yb + t * C);
-            }
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
     }
 }
 
@@ -184,6 +349,14 @@ int pow2_at_most(int64_t v, int cap) {
     return p;
 }
 
+// Blocks resident per SM for a kernel at 256 threads, and the SM count of the current device.
+template <typename Kern>
+int resident_blocks(Kern kern) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, 0) != cudaSuccess || n < 1) n = 1;
+    return n;
+}
+
 template <typename T, int V, int K>
 cudaError_t launch_vec_k(const Conv1dArgs &a, cudaStream_t s) {
     constexpr int R = (K <= 9) ? 16 : 8;
@@ -192,11 +365,17 @@ cudaError_t launch_vec_k(const Conv1dArgs &a, cudaStream_t s) {
     const int TY = kThreads / TX;
     const int nC = static_cast<int>((Cv + TX - 1) / TX);
     const int nT = static_cast<int>((a.T + static_cast<int64_t>(TY) * R - 1) / (static_cast<int64_t>(TY) * R));
-    const int64_t grid = a.B * nT * static_cast<int64_t>(nC);
+    const int64_t units = a.B * nT * static_cast<int64_t>(nC);
+    auto kern = conv1d_fwd_vec_kernel<T, V, K, R>;
+    static const int occ = resident_blocks(kern);
+    int64_t grid = static_cast<int64_t>(sm_count()) * occ;
+    grid = (grid / nC) * nC;
+    if (grid < nC) grid = nC;
+    if (grid > units) grid = units;          // units is a multiple of nC
     if (grid > kMaxGrid) return cudaErrorInvalidConfiguration;
-    conv1d_fwd_vec_kernel<T, V, K, R><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
-        static_cast<const T *>(a.x), a.w, a.bias, static_cast<T *>(a.y), a.lengths, a.T, a.C,
-        a.pad_left, a.flip, TX, nT, nC);
+    kern<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+        static_cast<const T *>(a.x), a.w, a.bias, static_cast<T *>(a.y), a.lengths, a.T, static_cast<int>(a.C),
+        a.pad_left, a.flip, TX, nT, nC, units);
     return cudaGetLastError();
 }
 
@@ -216,8 +395,54 @@ cudaError_t launch_vec_anyk(const Conv1dArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <typename T, int V, int K>
+cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
+    using S = TmaShape<T, V, K>;
+    auto kern = conv1d_fwd_tma_kernel<T, V, K>;
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::SMEM);
+    if (attr != cudaSuccess) return attr;
+    const int nC = static_cast<int>((a.C + S::CT - 1) / S::CT);
+    const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
+    const int64_t ntiles = a.B * static_cast<int64_t>(nT) * nC;
+    if (ntiles > kMaxGrid) return cudaErrorInvalidConfiguration;
+    CUtensorMap xmap;
+    const cudaError_t me = make_act_map(&xmap, a.x, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::ROWS);
+    if (me != cudaSuccess) return me;
+    int64_t grid = static_cast<int64_t>(sm_count()) * kTmaBlocks;
+    if (grid > ntiles) grid = ntiles;
+    kern<<<static_cast<unsigned>(grid), kTmaThreads, S::SMEM, s>>>(
+        xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.T), static_cast<int>(a.C),
+        a.pad_left, a.flip, nT, nC, static_cast<int>(ntiles));
+    return cudaGetLastError();
+}
+
+// The pipelined kernel copies whole frame rows in 16-byte units: C * sizeof(T) a multiple of
+// 16 and x 16-byte aligned.  Frame and item indices are 32-bit there.
+template <typename T>
+bool tma_ok(const Conv1dArgs &a) {
+    return (a.C * static_cast<int64_t>(sizeof(T))) % 16 == 0 && reinterpret_cast<uintptr_t>(a.x) % 16 == 0 &&
+           a.T < (1LL << 30) && a.B < (1LL << 30);
+}
+
 template <typename T, int V>
 cudaError_t dispatch_k(const Conv1dArgs &a, cudaStream_t s) {
+    if constexpr (V >= 2) {
+        if (tma_ok<T>(a)) {
+            switch (a.K) {
+                case 1: return launch_tma<T, V, 1>(a, s);
+                case 2: return launch_tma<T, V, 2>(a, s);
+                case 3: return launch_tma<T, V, 3>(a, s);
+                case 4: return launch_tma<T, V, 4>(a, s);
+                case 5: return launch_tma<T, V, 5>(a, s);
+                case 7: return launch_tma<T, V, 7>(a, s);
+                case 9: return launch_tma<T, V, 9>(a, s);
+                default: break;
+            }
+            if constexpr (V == 2) {
+                if (a.K == 15) return launch_tma<T, V, 15>(a, s);
+            }
+        }
+    }
     switch (a.K) {
         case 1: return launch_vec_k<T, V, 1>(a, s);
         case 2: return launch_vec_k<T, V, 2>(a, s);
@@ -226,19 +451,36 @@ cudaError_t dispatch_k(const Conv1dArgs &a, cudaStream_t s) {
         case 5: return launch_vec_k<T, V, 5>(a, s);
         case 7: return launch_vec_k<T, V, 7>(a, s);
         case 9: return launch_vec_k<T, V, 9>(a, s);
-        case 15: return launch_vec_k<T, V, 15>(a, s);
-        case 31: return launch_vec_k<T, V, 31>(a, s);
-        default: return launch_vec_anyk<T, V>(a, s);
+        default: break;
     }
+    if constexpr (V <= 2) {
+        if (a.K == 15) return launch_vec_k<T, V, 15>(a, s);
+    }
+    return launch_vec_anyk<T, (V > 2 ? 2 : V)>(a, s);
 }
 
 template <typename T>
 cudaError_t dispatch_dtype(const Conv1dArgs &a, cudaStream_t s) {
+    // 4 bf16 channels (8 bytes) per thread up to K = 9; pairs for wider kernels and for
+    // float32 (8 bytes), which keeps the register window under 128 registers.
+    if constexpr (sizeof(T) == 2) {
+#ifdef DW_FWD_V8
+        if (a.vec_width >= 8 && a.K <= 9) return dispatch_k<T, 8>(a, s);
+#endif
+        if (a.vec_width >= 4 && a.K <= 9) return dispatch_k<T, 4>(a, s);
+    }
     if (a.vec_width >= 2) return dispatch_k<T, 2>(a, s);
     return dispatch_k<T, 1>(a, s);
 }
 
 }  // namespace
+
+unsigned int conv1d_fwd_take_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, dw_device_error_flag, sizeof(v)) != cudaSuccess) return 0;
+    if (v) cudaMemcpyToSymbol(dw_device_error_flag, &zero, sizeof(zero));
+    return v;
+}
 
 cudaError_t conv1d_fwd_launch(const Conv1dArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;

@@ -19,7 +19,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+#ifdef DW_SCALAR_FMA
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+}
+#else
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+#endif
 
 // Raw storage for V consecutive channels of element type T, loaded with one instruction.
 // Words are 32-bit; a bf16 pair sits in one word (low half = lower channel).
@@ -136,6 +142,94 @@ __device__ __forceinline__ int64_t clamp_len(const int32_t *lengths, int64_t b, 
     if (lengths == nullptr) return T;
     int64_t L = __ldg(lengths + b);
     return L < 0 ? 0 : (L > T ? T : L);
+}
+
+}  // namespace dwk
+
+// ---------------------------------------------------------------------------------------
+// Bulk asynchronous copies (global -> shared, completion counted on an mbarrier) and
+// mbarrier helpers, in hand-written PTX for sm_90+/sm_100a.  Every wait is bounded: after
+// kSpinLimit failed polls the waiter records an error in dw_device_error_flag (read and
+// cleared by the host through dw_device_error()) and gives up, so a kernel never hangs.
+// ---------------------------------------------------------------------------------------
+namespace dwk {
+
+// One error word per translation unit (each .cu file reads and clears its own copy).
+static __device__ unsigned int dw_device_error_flag = 0;
+constexpr unsigned int kErrWaitTimeout = 1u;
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make initialised barriers visible to the asynchronous (bulk copy) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false (and the error flag set) if
+// it does not within kSpinLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicOr(&dw_device_error_flag, kErrWaitTimeout);
+    return false;
+}
+
+// size bytes from global src to shared dst (both 16-byte aligned, size a multiple of 16),
+// completion reported to bar as transaction bytes.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t size, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(size), "r"(smem_addr(bar))
+        : "memory");
+}
+
+}  // namespace dwk
+
+namespace dwk {
+
+// One box of a 3-D tensor map (coordinates innermost first: channel, frame, item) into shared
+// memory, completion counted on bar.  The channel coordinate must be a multiple of 16 bytes;
+// frame coordinates may be negative or past the end (those rows arrive as zeros).
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int c, int t, int b, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c), "r"(t), "r"(b), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
 }  // namespace dwk

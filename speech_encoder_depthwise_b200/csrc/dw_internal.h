@@ -2,6 +2,7 @@
 // Arguments arrive here already validated; launchers only pick a kernel and launch it.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -45,12 +46,33 @@ struct SubsampleArgs {
     int causal, bf16_out;
 };
 
+// Raise a kernel's dynamic shared memory limit to `bytes`, once per (kernel, device).
+cudaError_t ensure_smem_attr(const void *kern, int bytes);
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link
+// against the driver library); null if unavailable.
+typedef CUresult (*TensorMapEncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                           const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                           const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                           CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncodeTiledFn tensor_map_encoder();
+
+// Tensor map over a channels-last [B][T][C] activation (dims innermost first: C, T, B) with
+// a box of box_c channels x box_t frames x 1 item; out-of-range elements read as zero.
+cudaError_t make_act_map(CUtensorMap *map, const void *base, bool bf16, int64_t B, int64_t T, int64_t C,
+                         int box_c, int box_t);
+
+int sm_count();
+
 cudaError_t conv1d_fwd_launch(const Conv1dArgs &a, cudaStream_t s);
+// Reads and clears the device error word of the conv1d forward kernels (synchronous).
+unsigned int conv1d_fwd_take_error();
 
 // dW/dbias: the number of partial rows G and the workspace bytes follow from the sizes alone.
 int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t C, int K);
 size_t conv1d_dw_workspace_bytes(int64_t B, int64_t T, int64_t C, int K);
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s);
+unsigned int conv1d_dw_take_error();
 
 cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
 

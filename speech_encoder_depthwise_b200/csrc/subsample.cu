@@ -25,9 +25,19 @@
 
 namespace dwk {
 
-constexpr int kSubJ = 5;          // output columns per thread
-constexpr int kSubRI = 16;        // output rows per block
-constexpr int kSubWarpsMax = 4;   // channel tiles (64 channels each) per block
+#ifndef DW_SUB_J
+#define DW_SUB_J 4
+#endif
+#ifndef DW_SUB_RI
+#define DW_SUB_RI 16
+#endif
+#ifndef DW_SUB_MINB
+#define DW_SUB_MINB 5
+#endif
+constexpr int kSubJ = DW_SUB_J;          // output columns per thread
+constexpr int kSubRI = DW_SUB_RI;        // output rows per block
+constexpr int kSubWarpsMax = 4;          // channel tiles (64 channels each) per block
+constexpr int kSubMinBlocks = DW_SUB_MINB;  // resident blocks per SM the register budget aims at
 
 template <typename TO, bool VEC_STORE>
 __device__ __forceinline__ void store_pair(TO *p, float2 v, bool has_y);
@@ -53,62 +63,65 @@ __device__ __forceinline__ void store_pair<float, false>(float *p, float2 v, boo
 
 __device__ __forceinline__ float2 relu2(float2 a) { return make_float2(fmaxf(a.x, 0.f), fmaxf(a.y, 0.f)); }
 
-template <typename TO, bool VEC_STORE>
-__global__ void __launch_bounds__(kSubWarpsMax * 32)
+template <typename TO, bool VEC_STORE, int J, int RI>
+__global__ void __launch_bounds__(kSubWarpsMax * 32, kSubMinBlocks)
 dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
                     const float *__restrict__ b0, const float *__restrict__ w1,
                     const float *__restrict__ b1, TO *__restrict__ out,
-                    const int32_t *__restrict__ lengths, int64_t Tn, int64_t F, int64_t C,
-                    int64_t T2, int64_t F2, int64_t T4, int64_t F4, int Pt, int nCG, int nJB,
-                    int nRC) {
-    constexpr int J = kSubJ, RI = kSubRI;
+                    const int32_t *__restrict__ lengths, int32_t *__restrict__ out_lengths,
+                    int B, int Tn, int F, int C, int T2, int F2, int T4, int F4, int Pt, int nCG,
+                    int nJB, int nRC) {
     constexpr int NMR = 4 * RI + 3;   // mel rows a block reads
     constexpr int W = 4 * J + 8;      // staged mel columns: [4 j0 - 4, 4 j0 + 4 J + 4)
     __shared__ __align__(16) float2 sm[NMR][W];
 
     const int warps = blockDim.x / 32;
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-    int64_t lin = blockIdx.x;
-    const int cg = static_cast<int>(lin % nCG);
+    int lin = blockIdx.x;
+    const int cg = lin % nCG;
     lin /= nCG;
-    const int jb = static_cast<int>(lin % nJB);
+    const int jb = lin % nJB;
     lin /= nJB;
-    const int rc = static_cast<int>(lin % nRC);
-    const int64_t b = lin / nRC;
+    const int rc = lin % nRC;
+    const int b = lin / nRC;
 
-    const int64_t L = clamp_len(lengths, b, Tn);
-    const int64_t L2 = (L + 1) / 2, L4 = (L2 + 1) / 2;
-    const int64_t hrows = L2 < T2 ? L2 : T2;   // h rows that are neither padding nor masked
-    const int64_t i0 = static_cast<int64_t>(rc) * RI;
-    const int64_t j0 = static_cast<int64_t>(jb) * J;
-    const int64_t mrow0 = 4 * i0 - 3 * Pt;     // first mel row staged
-    const int64_t mcol0 = 4 * j0 - 4;          // first mel column staged
-
-    const int64_t c = (static_cast<int64_t>(cg) * warps + warp) * 64 + 2 * lane;
+    if (blockIdx.x == 0 && out_lengths != nullptr) {
+        for (int q = threadIdx.x; q < B; q += blockDim.x) {
+            const int Lq = static_cast<int>(clamp_len(lengths, q, Tn));
+            out_lengths[q] = ((Lq + 1) / 2 + 1) / 2;
+        }
+    }
+    const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+    const int L2 = (L + 1) / 2, L4 = (L2 + 1) / 2;
+    const int hrows = L2 < T2 ? L2 : T2;   // h rows that are neither padding nor masked
+    const int i0 = rc * RI;
+    const int j0 = jb * J;
+    const int mrow0 = 4 * i0 - 3 * Pt;     // first mel row staged
+    const int mcol0 = 4 * j0 - 4;          // first mel column staged
+    const int c = (cg * warps + warp) * 64 + 2 * lane;
     const bool has_x = c < C, has_y = c + 1 < C;
+    const bool any_valid = i0 < L4;        // some output row of this block is unmasked
 
-    // rows of this block that are valid outputs
-    const bool any_valid = i0 < L4;
     if (any_valid) {
-        const int64_t mlim = L;  // mel frames >= len_b read as zero
+        const float *melb = mel + static_cast<int64_t>(b) * Tn * F;
         for (int e = threadIdx.x; e < NMR * W; e += blockDim.x) {
             const int rr = e / W, cc = e % W;
-            const int64_t mr = mrow0 + rr, mc = mcol0 + cc;
+            const int mr = mrow0 + rr, mc = mcol0 + cc;
             float v = 0.f;
-            if (mr >= 0 && mr < mlim && mc >= 0 && mc < F) v = __ldg(mel + (b * Tn + mr) * F + mc);
+            if (mr >= 0 && mr < L && mc >= 0 && mc < F) v = __ldg(melb + mr * F + mc);  // frames >= len read as 0
             sm[rr][cc] = make_float2(v, v);
         }
     }
     __syncthreads();
-
-    TO *ob = out + b * T4 * F4 * C;
-    const int jn = static_cast<int>((F4 - j0) < J ? (F4 - j0) : J);  // columns of this block
     if (!has_x) return;
 
+    TO *ob = out + static_cast<int64_t>(b) * T4 * F4 * C + c;
+    const int jn = (F4 - j0) < J ? (F4 - j0) : J;  // columns of this block
+    const int iend = (i0 + RI) < T4 ? (i0 + RI) : T4;
     if (!any_valid) {  // every row of this block is masked: zeros only
-        for (int ii = 0; ii < RI && i0 + ii < T4; ++ii)
+        for (int i = i0; i < iend; ++i)
             for (int jj = 0; jj < jn; ++jj)
-                store_pair<TO, VEC_STORE>(ob + ((i0 + ii) * F4 + j0 + jj) * C + c, make_float2(0.f, 0.f), has_y);
+                store_pair<TO, VEC_STORE>(ob + (i * F4 + j0 + jj) * C, make_float2(0.f, 0.f), has_y);
         return;
     }
 
@@ -121,86 +134,98 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
     b0r = make_float2(__ldg(b0 + c), has_y ? __ldg(b0 + c + 1) : 0.f);
     b1r = make_float2(__ldg(b1 + c), has_y ? __ldg(b1 + c + 1) : 0.f);
 
-    // h at (row r, column hc) from the staged mel, any column (used for the block-edge columns)
-    auto h_at = [&](int64_t r, int64_t hc) -> float2 {
-        if (r < 0 || r >= hrows || hc < 0 || hc >= F2) return make_float2(0.f, 0.f);
-        const int rr = static_cast<int>(2 * r - Pt - mrow0);
-        const int cc = static_cast<int>(2 * hc - 1 - mcol0);
-        float2 a = b0r;
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-#pragma unroll
-            for (int q = 0; q < 3; ++q) a = ffma2(sm[rr + p][cc + q], w0r[p * 3 + q], a);
-        return relu2(a);
-    };
-
     // carry[n] = h(first h row of the current output row, column 2 j0 - 1 + n)
     float2 carry[2 * J + 1];
     {
-        const int64_t r = 2 * i0 - Pt;
+        const int r = 2 * i0 - Pt;               // staged row 0 is its first mel row
+        const bool rv = r >= 0 && r < hrows;
 #pragma unroll
-        for (int n = 0; n < 2 * J + 1; ++n) carry[n] = h_at(r, 2 * j0 - 1 + n);
+        for (int n = 0; n < 2 * J + 1; ++n) {
+            const int hc = 2 * j0 - 1 + n;
+            float2 a = b0r;
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int q = 0; q < 3; ++q) a = ffma2(sm[p][2 * n + 1 + q], w0r[p * 3 + q], a);
+            carry[n] = (rv && hc >= 0 && hc < F2) ? relu2(a) : make_float2(0.f, 0.f);
+        }
     }
 
-    for (int ii = 0; ii < RI; ++ii) {
-        const int64_t i = i0 + ii;
-        if (i >= T4) break;
-        TO *orow = ob + (i * F4 + j0) * C + c;
+    for (int i = i0; i < iend; ++i) {
+        TO *orow = ob + (i * F4 + j0) * C;
         if (i >= L4) {  // this and every later row of the item are masked
             for (int jj = 0; jj < jn; ++jj) store_pair<TO, VEC_STORE>(orow + jj * C, make_float2(0.f, 0.f), has_y);
             continue;
         }
-        const int64_t r1 = 2 * i - Pt + 1, r2 = r1 + 1;
+        const int r1 = 2 * i - Pt + 1, r2 = r1 + 1;   // the two new h rows
         const bool v1 = r1 >= 0 && r1 < hrows, v2 = r2 >= 0 && r2 < hrows;
-        const int rr = static_cast<int>(2 * r1 - Pt - mrow0);  // staged row of mel row 2 r1 - Pt
-        float2 prev1 = h_at(r1, 2 * j0 - 1), prev2 = h_at(r2, 2 * j0 - 1);
-        // m[p][0] = staged column 3 + 4 jj (mel column 4 j - 1), carried between columns
-        float2 m0[5];
+        const int rr = 2 * r1 - Pt - mrow0;            // staged row of mel row 2 r1 - Pt
+        // h column 2 j0 - 1 of rows r1, r2 (staged mel columns 1..3); column 3 then carries over
+        float2 prev1 = b0r, prev2 = b0r, m0[5];
 #pragma unroll
-        for (int p = 0; p < 5; ++p) m0[p] = sm[rr + p][3];
+        for (int p = 0; p < 5; ++p) {
+            const float2 m1 = sm[rr + p][1];
+            const float4 m23 = *reinterpret_cast<const float4 *>(&sm[rr + p][2]);
+            const float2 m[3] = {m1, make_float2(m23.x, m23.y), make_float2(m23.z, m23.w)};
+            m0[p] = m[2];
+            if (p <= 2) {
+#pragma unroll
+                for (int q = 0; q < 3; ++q) prev1 = ffma2(m[q], w0r[p * 3 + q], prev1);
+            }
+            if (p >= 2) {
+#pragma unroll
+                for (int q = 0; q < 3; ++q) prev2 = ffma2(m[q], w0r[(p - 2) * 3 + q], prev2);
+            }
+        }
+        prev1 = (v1 && j0 > 0) ? relu2(prev1) : make_float2(0.f, 0.f);
+        prev2 = (v2 && j0 > 0) ? relu2(prev2) : make_float2(0.f, 0.f);
 #pragma unroll
         for (int jj = 0; jj < J; ++jj) {
-            const int64_t j = j0 + jj;
-            // mel columns 4j .. 4j+3 (staged 4 + 4jj .. 7 + 4jj), two 16-byte loads per row
-            float2 m[5][5];
+            const int j = j0 + jj;
+            const bool cv1 = 2 * j < F2, cv2 = 2 * j + 1 < F2;
+            // mel columns 4j-1 .. 4j+3 are staged columns 3+4jj .. 7+4jj (column 3+4jj carries
+            // over from the previous column).  Window row p feeds h row r1 through tap row p
+            // (p <= 2) and h row r2 through tap row p-2 (p >= 2); each row is used as it arrives.
+            float2 a1 = b0r, a2 = b0r, c1 = b0r, c2 = b0r;
 #pragma unroll
             for (int p = 0; p < 5; ++p) {
                 const float4 lo = *reinterpret_cast<const float4 *>(&sm[rr + p][4 + 4 * jj]);
                 const float4 hi = *reinterpret_cast<const float4 *>(&sm[rr + p][6 + 4 * jj]);
-                m[p][0] = m0[p];
-                m[p][1] = make_float2(lo.x, lo.y);
-                m[p][2] = make_float2(lo.z, lo.w);
-                m[p][3] = make_float2(hi.x, hi.y);
-                m[p][4] = make_float2(hi.z, hi.w);
-                m0[p] = m[p][4];
-            }
-            float2 a1 = b0r, a2 = b0r, c1 = b0r, c2 = b0r;
+                const float2 m[5] = {m0[p], make_float2(lo.x, lo.y), make_float2(lo.z, lo.w),
+                                     make_float2(hi.x, hi.y), make_float2(hi.z, hi.w)};
+                m0[p] = m[4];
+                if (p <= 2) {
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
-#pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const float2 wt = w0r[p * 3 + q];
-                    a1 = ffma2(m[p][q], wt, a1);
-                    a2 = ffma2(m[p][q + 2], wt, a2);
-                    c1 = ffma2(m[p + 2][q], wt, c1);
-                    c2 = ffma2(m[p + 2][q + 2], wt, c2);
+                    for (int q = 0; q < 3; ++q) {
+                        a1 = ffma2(m[q], w0r[p * 3 + q], a1);
+                        a2 = ffma2(m[q + 2], w0r[p * 3 + q], a2);
+                    }
                 }
-            const bool cv1 = 2 * j < F2, cv2 = 2 * j + 1 < F2;
+                if (p >= 2) {
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        c1 = ffma2(m[q], w0r[(p - 2) * 3 + q], c1);
+                        c2 = ffma2(m[q + 2], w0r[(p - 2) * 3 + q], c2);
+                    }
+                }
+            }
             a1 = (v1 && cv1) ? relu2(a1) : make_float2(0.f, 0.f);
             a2 = (v1 && cv2) ? relu2(a2) : make_float2(0.f, 0.f);
             c1 = (v2 && cv1) ? relu2(c1) : make_float2(0.f, 0.f);
             c2 = (v2 && cv2) ? relu2(c2) : make_float2(0.f, 0.f);
 
-            float2 o = b1r;
-            o = ffma2(carry[2 * jj], w1r[0], o);
-            o = ffma2(carry[2 * jj + 1], w1r[1], o);
-            o = ffma2(carry[2 * jj + 2], w1r[2], o);
-            o = ffma2(prev1, w1r[3], o);
-            o = ffma2(a1, w1r[4], o);
-            o = ffma2(a2, w1r[5], o);
-            o = ffma2(prev2, w1r[6], o);
-            o = ffma2(c1, w1r[7], o);
-            o = ffma2(c2, w1r[8], o);
+            // conv_dw1 as three independent row sums, added at the end
+            float2 o0 = b1r, o1 = make_float2(0.f, 0.f), o2 = make_float2(0.f, 0.f);
+            o0 = ffma2(carry[2 * jj], w1r[0], o0);
+            o1 = ffma2(prev1, w1r[3], o1);
+            o2 = ffma2(prev2, w1r[6], o2);
+            o0 = ffma2(carry[2 * jj + 1], w1r[1], o0);
+            o1 = ffma2(a1, w1r[4], o1);
+            o2 = ffma2(c1, w1r[7], o2);
+            o0 = ffma2(carry[2 * jj + 2], w1r[2], o0);
+            o1 = ffma2(a2, w1r[5], o1);
+            o2 = ffma2(c2, w1r[8], o2);
+            const float2 o = make_float2(o0.x + o1.x + o2.x, o0.y + o1.y + o2.y);
             if (jj < jn) store_pair<TO, VEC_STORE>(orow + jj * C, o, has_y);
 
             carry[2 * jj] = prev2;
@@ -223,15 +248,18 @@ cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s) {
     const int64_t nJB = (F4 + kSubJ - 1) / kSubJ;
     const int64_t nRC = (T4 + kSubRI - 1) / kSubRI;
     const int64_t grid = a.B * nRC * nJB * nCG;
-    if (grid > kMaxGrid || nCG > 0x7fffffff || nJB > 0x7fffffff || nRC > 0x7fffffff)
+    // indices inside the kernel are 32-bit: an item's output and mel planes must fit
+    if (grid > kMaxGrid || T4 * F4 * a.C >= (1LL << 31) || a.T * a.F >= (1LL << 31) || 9 * a.C >= (1LL << 31))
         return cudaErrorInvalidConfiguration;
     const bool even = (a.C % 2) == 0;
     const bool aligned = (reinterpret_cast<uintptr_t>(a.out) % (a.bf16_out ? 4 : 8)) == 0;
     const bool vec = even && aligned;
-#define DW_SUB_LAUNCH(TO, VS)                                                                          \
-    dw_subsample_kernel<TO, VS><<<static_cast<unsigned>(grid), warps * 32, 0, s>>>(                      \
-        a.mel, a.w0, a.b0, a.w1, a.b1, static_cast<TO *>(a.out), a.lengths, a.T, a.F, a.C, T2, F2, T4, F4, \
-        Pt, static_cast<int>(nCG), static_cast<int>(nJB), static_cast<int>(nRC))
+#define DW_SUB_LAUNCH(TO, VS)                                                                           \
+    dw_subsample_kernel<TO, VS, kSubJ, kSubRI><<<static_cast<unsigned>(grid), warps * 32, 0, s>>>(          \
+        a.mel, a.w0, a.b0, a.w1, a.b1, static_cast<TO *>(a.out), a.lengths, a.out_lengths,                   \
+        static_cast<int>(a.B), static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C),           \
+        static_cast<int>(T2), static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt,          \
+        static_cast<int>(nCG), static_cast<int>(nJB), static_cast<int>(nRC))
     if (a.bf16_out) {
         if (vec) DW_SUB_LAUNCH(bf16, true);
         else DW_SUB_LAUNCH(bf16, false);

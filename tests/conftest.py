@@ -19,3 +19,16 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device on this host")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True)
+def _no_device_error(request):
+    """After every GPU test: no kernel recorded a timed-out wait."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import speech_encoder_depthwise_b200 as dw
+    assert dw.dw_device_error() == dw.DW_OK, "a kernel's bounded wait gave up (DW_ERR_TIMEOUT)"

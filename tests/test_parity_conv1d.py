@@ -226,3 +226,35 @@ def test_causal_output_ignores_future_frames():
     x2[:, 61:] = 3.0
     d2["x"] = x2
     np.testing.assert_array_equal(gpu_fwd(d2, "bf16", 8)[:, :61], base[:, :61])
+
+
+@pytest.mark.parametrize("K", [3, 9, 15])
+def test_pipelined_and_register_paths_agree(K):
+    """16-byte-aligned rows take the bulk-copy pipeline; an input 4 bytes off alignment takes
+    the register-tiled kernel.  Both sum the taps in the same order: identical bits."""
+    d = conv1d_inputs(3, 300, 256, K, dtype="bf16", len_range=(100, 300), seed=20 + K, with_dy=True)
+    x = dev(d["x"], torch.bfloat16)
+    raw = torch.empty(x.numel() + 8, dtype=torch.bfloat16, device="cuda")
+    xo = raw[2:2 + x.numel()].view(x.shape)
+    xo.copy_(x)
+    w, bias, ln = dev(d["w"]), dev(d["bias"]), dev(d["lengths"])
+    for fn, args in ((dw.dwconv1d_fwd, (w, bias)), (dw.dwconv1d_bwd_dx, (w,))):
+        ya, yb = torch.empty_like(x), torch.empty_like(x)
+        fn(x, *args, ya, ln, K - 1)
+        fn(xo, *args, yb, ln, K - 1)
+        torch.cuda.synchronize()
+        assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+    # dW: the two paths add partial sums in different orders; both must meet the bar
+    ref = oracle.dwconv1d_bwd_dw(d["x"], d["dy"], K, d["lengths"], K - 1)
+    g = dev(d["dy"], torch.bfloat16)
+    go = raw.clone()[2:2 + x.numel()].view(x.shape)
+    go.copy_(g)
+    for xx, gg in ((x, g), (xo, go)):
+        gw = torch.empty(K, 256, device="cuda")
+        gb = torch.empty(256, device="cuda")
+        ws = torch.empty(dw.dwconv1d_bwd_dw_workspace_size(3, 300, 256, K), dtype=torch.uint8, device="cuda")
+        dw.dwconv1d_bwd_dw(xx, gg, gw, gb, ln, K - 1, ws)
+        torch.cuda.synchronize()
+        for got, r in ((gw.cpu().numpy(), ref[0]), (gb.cpu().numpy(), ref[1])):
+            e = max_abs(got, r)
+            assert e <= 1e-5 * rms(r), (e, rms(r))
