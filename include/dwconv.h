@@ -122,6 +122,30 @@ dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
                             size_t workspace_bytes, dw_stream_t stream);
 
 /*
+ * dwconv1d_bwd_dw_noalloc - dwconv1d_bwd_dw without a caller-provided workspace: it allocates
+ * nothing and uses a scratch array that the library keeps in device memory.  The papers have
+ * no counterpart to this entry point; it exists for callers that cannot allocate device
+ * memory: code embedded in a host that owns all device memory through its own allocator and
+ * hands plug-ins no allocation handle, and streaming loops that must not call cudaMalloc after
+ * start-up because an allocation can block on the whole device.
+ *
+ *  Scratch: 2 MiB (2,097,152 bytes) of device memory per GPU that loads the library, held
+ *  until the process exits.  One partial row of (K+1)*C float32 must fit in it: larger
+ *  (K+1)*C returns DW_ERR_UNSUPPORTED without touching the device.  Within that limit the
+ *  results equal dwconv1d_bwd_dw's up to float32 summation order (the same order whenever
+ *  the scratch holds as many partial rows as dwconv1d_bwd_dw_workspace_size would provide).
+ *  The first call on a device looks up the scratch's device address (cudaGetSymbolAddress),
+ *  so that first call should come before any stream capture.  All calls share the scratch and
+ *  it keeps the last call's contents; calls that overlap on the GPU race on it, so the caller
+ *  must serialise them.  Every partial sum read is written by the same call first.  A failed
+ *  launch returns DW_ERR_CUDA (dw_last_cuda_error is not updated by this entry point).
+ *  Other arguments, results and errors: as dwconv1d_bwd_dw.
+ */
+dw_status_t dwconv1d_bwd_dw_noalloc(const void *x, const void *dy, float *dw, float *dbias,
+                                    const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
+                                    int pad_left, dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
  * dw_subsample_fwd - fused front of the depthwise-striding subsampler (NeMo PR #16114, "Use
  * Fused Kernels for Depthwise Striding Subsampler", section "What does this PR do ?", first
  * kernel: mel [B,T,F,1] -> conv0 [B,T/2,F/2,C] -> ReLU -> masking -> conv_dw1 [B,T/4,F/4,C]).

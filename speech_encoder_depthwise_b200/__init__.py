@@ -20,6 +20,7 @@ __all__ = [
     "DW_OK", "DW_ERR_INVALID_ARG", "DW_ERR_UNSUPPORTED", "DW_ERR_WORKSPACE", "DW_ERR_CUDA",
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
+    "dwconv1d_bwd_dw_noalloc",
     "dw_subsample_fwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
 ]
 
@@ -42,6 +43,7 @@ SIGNATURES = {
     "dwconv1d_bwd_dw_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _int]),
     "dwconv1d_bwd_dw": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp,
                                ctypes.c_size_t, _vp]),
+    "dwconv1d_bwd_dw_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
     "dw_status_string": (ctypes.c_char_p, [_int]),
@@ -162,6 +164,21 @@ def dwconv1d_bwd_dw(x, dy, dw, dbias, lengths, pad_left, workspace, stream=None)
                                _dev(lengths, "lengths", torch.int32, (B,)), B, T, C, K, int(pad_left),
                                _dtype_code(x), ws_ptr, ws_bytes, _stream(stream))
     _check("dwconv1d_bwd_dw", st)
+
+
+def dwconv1d_bwd_dw_noalloc(x, dy, dw, dbias, lengths, pad_left, stream=None):
+    """dwconv1d_bwd_dw without a workspace, for callers that cannot allocate device memory: the
+    library's own 2 MiB device scratch holds the partial sums (shared by all calls; calls that
+    overlap on the GPU race on it)."""
+    import torch
+    B, T, C = x.shape
+    K = dw.shape[0]
+    st = lib().dwconv1d_bwd_dw_noalloc(_dev(x, "x"), _dev(dy, "dy", x.dtype, x.shape),
+                                       _dev(dw, "dw", torch.float32, (K, C)),
+                                       _dev(dbias, "dbias", torch.float32, (C,)),
+                                       _dev(lengths, "lengths", torch.int32, (B,)), B, T, C, K, int(pad_left),
+                                       _dtype_code(x), _stream(stream))
+    _check("dwconv1d_bwd_dw_noalloc", st)
 
 
 def subsample_out_shape(T, F):
