@@ -77,6 +77,23 @@ def sub_work(lengths, T, F, C, esize=2):
     return by, fl, T4, F4
 
 
+# ------------------------------------------------------------------ multi-rank aggregation
+def max_over_ranks(value, world, device="cpu"):
+    """The largest value over all ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(step_bytes_per_rank, ms_per_step, world):
+    """Whole-job GB/s: every rank processes its own batch (weak scaling) in the slowest rank's time."""
+    return world * step_bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ clocks (NVML, read only)
 class ClockSampler:
     """Samples SM clock and throttle reasons in a background thread (reads only)."""
@@ -333,16 +350,13 @@ def main():
     elapsed_ms = e_start.elapsed_time(e_end)
     row_ms = {r: float(np.mean([step_evs[i][j][0].elapsed_time(step_evs[i][j][1]) for i in range(steps)]))
               for j, r in enumerate(rows)}
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = elapsed_ms / steps
 
     cw, valid = conv_work(cs["lengths"], T, C, K)
     sb, sf, _, _ = sub_work(ss["lengths"], ST, SF, SC)
     step_bytes = sum(v[0] for v in cw.values()) + sb
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(step_bytes, ms_per_step, world)
 
     # ---------------------------------------------------------------- e2e through the binding
     e2e = None
@@ -393,12 +407,8 @@ def main():
             e2e_step()
         b_.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = a.elapsed_time(b_) / args.e2e_steps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms = max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, world, dev)
+        e2e = {"value": job_throughput(step_bytes, e2e_ms, world), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     # ---------------------------------------------------------------- report (rank 0)

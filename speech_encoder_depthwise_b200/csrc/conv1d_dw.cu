@@ -167,9 +167,22 @@ conv1d_dw_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
 // then release the stage on its "empty" mbarrier.  At the end every warp (the producer adds
 // zeros) joins the block and cluster reductions of the register-tiled kernel above.
 // ---------------------------------------------------------------------------------------
-constexpr int kDwConsumers = 8;
-constexpr int kDwR = 8;
-constexpr int kDwStages = 3;
+#ifndef DW_DW_CONSUMERS
+#define DW_DW_CONSUMERS 8
+#endif
+#ifndef DW_DW_R
+#define DW_DW_R 8
+#endif
+#ifndef DW_DW_STAGES
+#define DW_DW_STAGES 3
+#endif
+#ifndef DW_DW_BLOCKS
+#define DW_DW_BLOCKS 2
+#endif
+constexpr int kDwConsumers = DW_DW_CONSUMERS;  // consumer warps per block
+constexpr int kDwR = DW_DW_R;                  // frames per consumer thread per unit
+constexpr int kDwStages = DW_DW_STAGES;        // shared-memory ring depth
+constexpr int kDwBlocks = DW_DW_BLOCKS;        // resident blocks per SM
 constexpr int kDwTmaThreads = 32 * (1 + kDwConsumers);
 
 template <typename T, int V, int KB>
@@ -185,7 +198,7 @@ struct DwTmaShape {
 };
 
 template <typename T, int V, int KB>
-__global__ void __launch_bounds__(kDwTmaThreads, 2)
+__global__ void __launch_bounds__(kDwTmaThreads, kDwBlocks)
 conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
                      const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C, int K,
                      int k_off, int pad_left, int nT, int with_bias) {
