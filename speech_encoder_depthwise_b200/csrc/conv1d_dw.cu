@@ -194,14 +194,14 @@ struct DwTmaShape {
     static constexpr int STAGE_BYTES = (XROWS + TT) * ROWB;
     static constexpr int RED_BYTES = kDwConsumers * (KB + 1) * CT * 4;
     static constexpr int BODY = (kDwStages * STAGE_BYTES > RED_BYTES) ? kDwStages * STAGE_BYTES : RED_BYTES;
-    static constexpr int SMEM = 128 + BODY;
+    static constexpr int SMEM = 128 + BODY;  // plus the tile-order tables, sized at launch
 };
 
 template <typename T, int V, int KB>
 __global__ void __launch_bounds__(kDwTmaThreads, kDwBlocks)
 conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
                      const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C, int K,
-                     int k_off, int pad_left, int nT, int with_bias) {
+                     int k_off, int pad_left, int nT, int with_bias, int ordered) {
     using S = DwTmaShape<T, V, KB>;
     constexpr int NP = Pairs<V>::n;
     constexpr int R = kDwR;
@@ -212,7 +212,11 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int g = blockIdx.x, G = gridDim.x, ct = blockIdx.y;
     const int c0 = ct * S::CT;
-    const int units = B * nT;
+    // the frame-runs to walk: only the valid ones (first frame < len_b), in balanced order, or
+    // every (item, run) pair when B is too large for the order's shared-memory tables
+    int *ord_mem = reinterpret_cast<int *>(stages + S::BODY);
+    TileOrder order{ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), B, nT, 1, 0};
+    if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDwStages; ++i) {
             mbar_init(&full[i], 1);
@@ -221,6 +225,19 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
         fence_barrier_init();
     }
     __syncthreads();
+    if (ordered) order.V = order.pv[B];
+    const int units = ordered ? order.V : B * nT;
+    auto unit_at = [&](int u, int &b, int &t0, int &L) {
+        if (ordered) {
+            int tt, ctd;
+            order.map(u, b, tt, ctd, L);
+            t0 = tt * S::TT;
+        } else {
+            b = u / nT;
+            t0 = (u % nT) * S::TT;
+            L = static_cast<int>(clamp_len(lengths, b, Tn));
+        }
+    };
     float2 acc[KB][NP], accb[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
@@ -242,8 +259,8 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
             ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1));
             if (!ok) break;
             if (lane == 0) {
-                const int b = u / nT, t0 = (u % nT) * S::TT;
-                const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+                int b, t0, L;
+                unit_at(u, b, t0, L);
                 if (t0 < L) {  // frames before 0 or past T arrive as zeros; [L, T) is masked by the consumers
                     unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
@@ -262,8 +279,8 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
         for (int u = g; u < units && ok; u += G, ++it) {
             const int s = it % kDwStages;
             const uint32_t ph = (it / kDwStages) & 1;
-            const int b = u / nT, t0 = (u % nT) * S::TT;
-            const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+            int b, t0, L;
+            unit_at(u, b, t0, L);
             ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph));
             if (!ok) break;
             const int tg = t0 + cw * R;
@@ -424,7 +441,10 @@ template <typename T, int V, int KB>
 cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s) {
     using S = DwTmaShape<T, V, KB>;
     auto kern = conv1d_dw_tma_kernel<T, V, KB>;
-    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::SMEM);
+    const int ordered = a.B <= kOrderMaxItems ? 1 : 0;
+    const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
+                                              S::SMEM + static_cast<int>(3 * (kOrderMaxItems + 1) * sizeof(int)) + 16);
     if (attr != cudaSuccess) return attr;
     const int nCT = static_cast<int>((a.C + S::CT - 1) / S::CT);
     const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
@@ -435,7 +455,7 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(c, nCT);
         q.blockDim = dim3(kDwTmaThreads);
-        q.dynamicSmemBytes = S::SMEM;
+        q.dynamicSmemBytes = smem;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = c;
@@ -462,7 +482,7 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(best_g, nCT);
     cfg.blockDim = dim3(kDwTmaThreads);
-    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -476,7 +496,8 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::TT);
     if (me != cudaSuccess) return me;
     return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, a.lengths, a.partials, static_cast<int>(a.B),
-                              static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias);
+                              static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias,
+                              ordered);
 }
 
 template <typename T>

@@ -161,7 +161,7 @@ template <typename T, int V, int K>
 __global__ void __launch_bounds__(kTmaThreads, kTmaBlocks)
 conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restrict__ w,
                       const float *__restrict__ bias, T *__restrict__ y, const int32_t *__restrict__ lengths,
-                      int Tn, int C, int pad_left, int flip, int nT, int nC, int ntiles) {
+                      int B, int Tn, int C, int pad_left, int flip, int nT, int nC, int ntiles, int ordered) {
     using S = TmaShape<T, V, K>;
     constexpr int NP = Pairs<V>::n;
     constexpr int R = S::R;
@@ -170,6 +170,9 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     uint64_t *empty = full + kTmaStages;
     unsigned char *stages = smem_raw + 128;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    int *ord_mem = reinterpret_cast<int *>(stages + static_cast<size_t>(kTmaStages) * S::STAGE_BYTES);
+    TileOrder order{ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), B, nT, nC, 0};
+    if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTmaStages; ++i) {
             mbar_init(&full[i], 1);
@@ -178,6 +181,21 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
         fence_barrier_init();
     }
     __syncthreads();
+    if (ordered) order.V = order.pv[B];
+    // position g of this block's walk -> tile (b, t0, ct) and the item's length
+    auto tile_at = [&](int g, int &b, int &t0, int &ct, int &L) {
+        if (ordered) {
+            int tt;
+            order.map(g, b, tt, ct, L);
+            t0 = tt * S::TT;
+        } else {
+            ct = g % nC;
+            const int bt = g / nC;
+            t0 = (bt % nT) * S::TT;
+            b = bt / nT;
+            L = static_cast<int>(clamp_len(lengths, b, Tn));
+        }
+    };
     if (warp == 0) {  // producer warp: one elected lane, one tensor copy per tile
         if (lane == 0) prefetch_tmap(&xmap);
         int it = 0;
@@ -186,9 +204,8 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
             const uint32_t ph = (it / kTmaStages) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) return;
             if (lane == 0) {
-                const int ct = tile % nC, bt = tile / nC;
-                const int t0 = (bt % nT) * S::TT, b = bt / nT;
-                const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+                int b, t0, ct, L;
+                tile_at(tile, b, t0, ct, L);
                 if (t0 < L) {  // rows before frame 0 or past T arrive as zeros; rows in [L, T) are masked by the consumers
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
                     tma_load_3d(stages + static_cast<size_t>(s) * S::STAGE_BYTES, &xmap, ct * S::CT, t0 - pad_left, b,
@@ -208,11 +225,10 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int s = it % kTmaStages;
         const uint32_t ph = (it / kTmaStages) & 1;
-        const int ct = tile % nC, bt = tile / nC;
-        const int t0 = (bt % nT) * S::TT, b = bt / nT;
+        int b, t0, ct, L;
+        tile_at(tile, b, t0, ct, L);
         const int cv = ct * S::CT + lane * V;
         const bool active = cv < C;
-        const int L = static_cast<int>(clamp_len(lengths, b, Tn));
         const int tg = t0 + g * R;
         float2 wv[K][NP], acc[R][NP];
         if (active && tg < L) {  // issue the parameter loads before waiting for the tile
@@ -399,7 +415,8 @@ template <typename T, int V, int K>
 cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     using S = TmaShape<T, V, K>;
     auto kern = conv1d_fwd_tma_kernel<T, V, K>;
-    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::SMEM);
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
+                                              S::SMEM + static_cast<int>(3 * (kOrderMaxItems + 1) * sizeof(int)) + 16);
     if (attr != cudaSuccess) return attr;
     const int nC = static_cast<int>((a.C + S::CT - 1) / S::CT);
     const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
@@ -410,9 +427,11 @@ cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     if (me != cudaSuccess) return me;
     int64_t grid = static_cast<int64_t>(sm_count()) * kTmaBlocks;
     if (grid > ntiles) grid = ntiles;
-    kern<<<static_cast<unsigned>(grid), kTmaThreads, S::SMEM, s>>>(
-        xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.T), static_cast<int>(a.C),
-        a.pad_left, a.flip, nT, nC, static_cast<int>(ntiles));
+    const int ordered = a.B <= kOrderMaxItems ? 1 : 0;
+    const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
+    kern<<<static_cast<unsigned>(grid), kTmaThreads, smem, s>>>(
+        xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.B), static_cast<int>(a.T),
+        static_cast<int>(a.C), a.pad_left, a.flip, nT, nC, static_cast<int>(ntiles), ordered);
     return cudaGetLastError();
 }
 

@@ -233,3 +233,87 @@ __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
 }
 
 }  // namespace dwk
+
+namespace dwk {
+
+// Balanced tile order.  Tiles whose first frame is at or beyond len_b only store zeros, so a
+// plain round robin deals some blocks far more real work than others.  Instead every block
+// builds, in shared memory, the per-item prefix counts of valid tiles (first frame < len_b)
+// and of masked tiles, and deals tiles in the order: all valid tiles, then all masked tiles,
+// each run channel-tile fastest.  Block i takes positions i, i + G, i + 2G, ...: every block
+// gets the same number of valid tiles to within one.  Used when B <= kOrderMaxItems.
+// (With nC = 1 and only positions below V it deals the valid frame-runs of one channel tile.)
+constexpr int kOrderMaxItems = 1024;
+
+struct TileOrder {
+    const int *pv;   // [B+1] valid tiles before item b (times nC)
+    const int *pm;   // [B+1] masked tiles before item b (times nC)
+    const int *len;  // [B] clamped lengths
+    int B, nT, nC, V;
+
+    // Builds the three arrays with warp 0 of the calling block (all threads must call it, then sync).
+    __device__ void build(int *spv, int *spm, int *slen, const int32_t *lengths, int Tn, int TT) {
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            int run_v = 0, run_m = 0;
+            if (lane == 0) {
+                spv[0] = 0;
+                spm[0] = 0;
+            }
+            for (int base = 0; base < B; base += 32) {
+                const int bb = base + lane;
+                int nv = 0, nm = 0;
+                if (bb < B) {
+                    const int L = static_cast<int>(clamp_len(lengths, bb, Tn));
+                    slen[bb] = L;
+                    nv = (L + TT - 1) / TT;
+                    nm = nT - nv;
+                }
+                int iv = nv * nC, im = nm * nC;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int tv = __shfl_up_sync(0xffffffffu, iv, o), tm = __shfl_up_sync(0xffffffffu, im, o);
+                    if (lane >= o) {
+                        iv += tv;
+                        im += tm;
+                    }
+                }
+                if (bb < B) {
+                    spv[bb + 1] = run_v + iv;
+                    spm[bb + 1] = run_m + im;
+                }
+                run_v += __shfl_sync(0xffffffffu, iv, 31);
+                run_m += __shfl_sync(0xffffffffu, im, 31);
+            }
+        }
+    }
+
+    // Last item b with a[b] <= g (a non-decreasing, a[0] = 0 <= g).
+    static __device__ __forceinline__ int find(const int *a, int n, int g) {
+        int lo = 0, hi = n;  // invariant: a[lo] <= g, answer in [lo, hi)
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (a[mid] <= g) lo = mid;
+            else hi = mid;
+        }
+        return lo;
+    }
+
+    __device__ __forceinline__ void map(int g, int &b, int &tt, int &ct, int &L) const {
+        if (g < V) {
+            b = find(pv, B, g);
+            const int local = g - pv[b];
+            tt = local / nC;
+            ct = local % nC;
+        } else {
+            const int m = g - V;
+            b = find(pm, B, m);
+            const int local = m - pm[b];
+            tt = (pv[b + 1] - pv[b]) / nC + local / nC;
+            ct = local % nC;
+        }
+        L = len[b];
+    }
+};
+
+}  // namespace dwk

@@ -21,6 +21,8 @@
 //    h column per column block;
 //  - h rows that are masked or padding are skipped (zero), output rows at or beyond
 //    ceil(len/4) only store zeros.
+#include <type_traits>
+
 #include "dw_internal.h"
 
 namespace dwk {
@@ -34,10 +36,14 @@ namespace dwk {
 #ifndef DW_SUB_MINB
 #define DW_SUB_MINB 5
 #endif
+#ifndef DW_SUB_NPR
+#define DW_SUB_NPR 1
+#endif
 constexpr int kSubJ = DW_SUB_J;          // output columns per thread
 constexpr int kSubRI = DW_SUB_RI;        // output rows per block
 constexpr int kSubWarpsMax = 4;          // channel tiles (64 channels each) per block
 constexpr int kSubMinBlocks = DW_SUB_MINB;  // resident blocks per SM the register budget aims at
+constexpr int kSubNPR = DW_SUB_NPR;         // channel pairs per thread
 
 template <typename TO, bool VEC_STORE>
 __device__ __forceinline__ void store_pair(TO *p, float2 v, bool has_y);
@@ -63,7 +69,26 @@ __device__ __forceinline__ void store_pair<float, false>(float *p, float2 v, boo
 
 __device__ __forceinline__ float2 relu2(float2 a) { return make_float2(fmaxf(a.x, 0.f), fmaxf(a.y, 0.f)); }
 
-template <typename TO, bool VEC_STORE, int J, int RI>
+// Stores NPR channel pairs (2*NPR consecutive channels) of one output pixel.
+template <typename TO, bool VEC_STORE, int NPR>
+__device__ __forceinline__ void store_pairs(TO *p, const float2 (&v)[NPR], int nvalid) {
+    if constexpr (VEC_STORE) {
+        if constexpr (NPR == 1) {
+            store_pair<TO, true>(p, v[0], true);
+        } else if constexpr (sizeof(TO) == 2) {
+            *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y));
+        } else {
+            *reinterpret_cast<float4 *>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            if (2 * q < nvalid) store_pair<TO, false>(p + 2 * q, v[q], 2 * q + 1 < nvalid);
+        }
+    }
+}
+
+template <typename TO, bool VEC_STORE, int J, int RI, int NPR>
 __global__ void __launch_bounds__(kSubWarpsMax * 32, kSubMinBlocks)
 dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
                     const float *__restrict__ b0, const float *__restrict__ w1,
@@ -73,6 +98,7 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
                     int nJB, int nRC) {
     constexpr int NMR = 4 * RI + 3;   // mel rows a block reads
     constexpr int W = 4 * J + 8;      // staged mel columns: [4 j0 - 4, 4 j0 + 4 J + 4)
+    constexpr int CW = 64 * NPR;      // channels per warp
     __shared__ __align__(16) float2 sm[NMR][W];
 
     const int warps = blockDim.x / 32;
@@ -98,8 +124,8 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
     const int j0 = jb * J;
     const int mrow0 = 4 * i0 - 3 * Pt;     // first mel row staged
     const int mcol0 = 4 * j0 - 4;          // first mel column staged
-    const int c = (cg * warps + warp) * 64 + 2 * lane;
-    const bool has_x = c < C, has_y = c + 1 < C;
+    const int c = (cg * warps + warp) * CW + 2 * NPR * lane;  // first channel of this thread
+    const int nvalid = C - c;                                  // channels of this thread inside C
     const bool any_valid = i0 < L4;        // some output row of this block is unmasked
 
     if (any_valid) {
@@ -113,127 +139,171 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
         }
     }
     __syncthreads();
-    if (!has_x) return;
+    if (nvalid <= 0) return;
 
     TO *ob = out + static_cast<int64_t>(b) * T4 * F4 * C + c;
     const int jn = (F4 - j0) < J ? (F4 - j0) : J;  // columns of this block
     const int iend = (i0 + RI) < T4 ? (i0 + RI) : T4;
+    float2 zero2[NPR];
+#pragma unroll
+    for (int q = 0; q < NPR; ++q) zero2[q] = make_float2(0.f, 0.f);
     if (!any_valid) {  // every row of this block is masked: zeros only
         for (int i = i0; i < iend; ++i)
-            for (int jj = 0; jj < jn; ++jj)
-                store_pair<TO, VEC_STORE>(ob + (i * F4 + j0 + jj) * C, make_float2(0.f, 0.f), has_y);
+            for (int jj = 0; jj < jn; ++jj) store_pairs<TO, VEC_STORE, NPR>(ob + (i * F4 + j0 + jj) * C, zero2, nvalid);
         return;
     }
 
-    float2 w0r[9], w1r[9], b0r, b1r;
+    float2 w0r[9][NPR], w1r[9][NPR], b0r[NPR], b1r[NPR];
+    {
+        auto ld = [&](const float *p, int k) { return k < nvalid ? __ldg(p + k) : 0.f; };
 #pragma unroll
-    for (int t = 0; t < 9; ++t) {
-        w0r[t] = make_float2(__ldg(w0 + t * C + c), has_y ? __ldg(w0 + t * C + c + 1) : 0.f);
-        w1r[t] = make_float2(__ldg(w1 + t * C + c), has_y ? __ldg(w1 + t * C + c + 1) : 0.f);
+        for (int q = 0; q < NPR; ++q) {
+#pragma unroll
+            for (int t = 0; t < 9; ++t) {
+                w0r[t][q] = make_float2(ld(w0 + t * C + c, 2 * q), ld(w0 + t * C + c, 2 * q + 1));
+                w1r[t][q] = make_float2(ld(w1 + t * C + c, 2 * q), ld(w1 + t * C + c, 2 * q + 1));
+            }
+            b0r[q] = make_float2(ld(b0 + c, 2 * q), ld(b0 + c, 2 * q + 1));
+            b1r[q] = make_float2(ld(b1 + c, 2 * q), ld(b1 + c, 2 * q + 1));
+        }
     }
-    b0r = make_float2(__ldg(b0 + c), has_y ? __ldg(b0 + c + 1) : 0.f);
-    b1r = make_float2(__ldg(b1 + c), has_y ? __ldg(b1 + c + 1) : 0.f);
 
     // carry[n] = h(first h row of the current output row, column 2 j0 - 1 + n)
-    float2 carry[2 * J + 1];
+    float2 carry[2 * J + 1][NPR];
     {
         const int r = 2 * i0 - Pt;               // staged row 0 is its first mel row
         const bool rv = r >= 0 && r < hrows;
 #pragma unroll
         for (int n = 0; n < 2 * J + 1; ++n) {
             const int hc = 2 * j0 - 1 + n;
-            float2 a = b0r;
+            const bool ok = rv && hc >= 0 && hc < F2;
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
+            for (int q = 0; q < NPR; ++q) {
+                float2 a = b0r[q];
 #pragma unroll
-                for (int q = 0; q < 3; ++q) a = ffma2(sm[p][2 * n + 1 + q], w0r[p * 3 + q], a);
-            carry[n] = (rv && hc >= 0 && hc < F2) ? relu2(a) : make_float2(0.f, 0.f);
+                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                    for (int qq = 0; qq < 3; ++qq) a = ffma2(sm[p][2 * n + 1 + qq], w0r[p * 3 + qq][q], a);
+                carry[n][q] = ok ? relu2(a) : make_float2(0.f, 0.f);
+            }
         }
     }
+    // every h column of this block is inside [0, F2) except possibly column 2 j0 - 1 (j0 == 0)
+    const bool cols_all = 2 * (j0 + J) <= F2;
 
     for (int i = i0; i < iend; ++i) {
         TO *orow = ob + (i * F4 + j0) * C;
         if (i >= L4) {  // this and every later row of the item are masked
-            for (int jj = 0; jj < jn; ++jj) store_pair<TO, VEC_STORE>(orow + jj * C, make_float2(0.f, 0.f), has_y);
+            for (int jj = 0; jj < jn; ++jj) store_pairs<TO, VEC_STORE, NPR>(orow + jj * C, zero2, nvalid);
             continue;
         }
         const int r1 = 2 * i - Pt + 1, r2 = r1 + 1;   // the two new h rows
         const bool v1 = r1 >= 0 && r1 < hrows, v2 = r2 >= 0 && r2 < hrows;
         const int rr = 2 * r1 - Pt - mrow0;            // staged row of mel row 2 r1 - Pt
         // h column 2 j0 - 1 of rows r1, r2 (staged mel columns 1..3); column 3 then carries over
-        float2 prev1 = b0r, prev2 = b0r, m0[5];
+        float2 prev1[NPR], prev2[NPR], m0[5];
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) prev1[q] = prev2[q] = b0r[q];
 #pragma unroll
         for (int p = 0; p < 5; ++p) {
             const float2 m1 = sm[rr + p][1];
             const float4 m23 = *reinterpret_cast<const float4 *>(&sm[rr + p][2]);
             const float2 m[3] = {m1, make_float2(m23.x, m23.y), make_float2(m23.z, m23.w)};
             m0[p] = m[2];
-            if (p <= 2) {
 #pragma unroll
-                for (int q = 0; q < 3; ++q) prev1 = ffma2(m[q], w0r[p * 3 + q], prev1);
-            }
-            if (p >= 2) {
-#pragma unroll
-                for (int q = 0; q < 3; ++q) prev2 = ffma2(m[q], w0r[(p - 2) * 3 + q], prev2);
-            }
-        }
-        prev1 = (v1 && j0 > 0) ? relu2(prev1) : make_float2(0.f, 0.f);
-        prev2 = (v2 && j0 > 0) ? relu2(prev2) : make_float2(0.f, 0.f);
-#pragma unroll
-        for (int jj = 0; jj < J; ++jj) {
-            const int j = j0 + jj;
-            const bool cv1 = 2 * j < F2, cv2 = 2 * j + 1 < F2;
-            // mel columns 4j-1 .. 4j+3 are staged columns 3+4jj .. 7+4jj (column 3+4jj carries
-            // over from the previous column).  Window row p feeds h row r1 through tap row p
-            // (p <= 2) and h row r2 through tap row p-2 (p >= 2); each row is used as it arrives.
-            float2 a1 = b0r, a2 = b0r, c1 = b0r, c2 = b0r;
-#pragma unroll
-            for (int p = 0; p < 5; ++p) {
-                const float4 lo = *reinterpret_cast<const float4 *>(&sm[rr + p][4 + 4 * jj]);
-                const float4 hi = *reinterpret_cast<const float4 *>(&sm[rr + p][6 + 4 * jj]);
-                const float2 m[5] = {m0[p], make_float2(lo.x, lo.y), make_float2(lo.z, lo.w),
-                                     make_float2(hi.x, hi.y), make_float2(hi.z, hi.w)};
-                m0[p] = m[4];
+            for (int q = 0; q < NPR; ++q) {
                 if (p <= 2) {
 #pragma unroll
-                    for (int q = 0; q < 3; ++q) {
-                        a1 = ffma2(m[q], w0r[p * 3 + q], a1);
-                        a2 = ffma2(m[q + 2], w0r[p * 3 + q], a2);
-                    }
+                    for (int qq = 0; qq < 3; ++qq) prev1[q] = ffma2(m[qq], w0r[p * 3 + qq][q], prev1[q]);
                 }
                 if (p >= 2) {
 #pragma unroll
-                    for (int q = 0; q < 3; ++q) {
-                        c1 = ffma2(m[q], w0r[(p - 2) * 3 + q], c1);
-                        c2 = ffma2(m[q + 2], w0r[(p - 2) * 3 + q], c2);
-                    }
+                    for (int qq = 0; qq < 3; ++qq) prev2[q] = ffma2(m[qq], w0r[(p - 2) * 3 + qq][q], prev2[q]);
                 }
             }
-            a1 = (v1 && cv1) ? relu2(a1) : make_float2(0.f, 0.f);
-            a2 = (v1 && cv2) ? relu2(a2) : make_float2(0.f, 0.f);
-            c1 = (v2 && cv1) ? relu2(c1) : make_float2(0.f, 0.f);
-            c2 = (v2 && cv2) ? relu2(c2) : make_float2(0.f, 0.f);
-
-            // conv_dw1 as three independent row sums, added at the end
-            float2 o0 = b1r, o1 = make_float2(0.f, 0.f), o2 = make_float2(0.f, 0.f);
-            o0 = ffma2(carry[2 * jj], w1r[0], o0);
-            o1 = ffma2(prev1, w1r[3], o1);
-            o2 = ffma2(prev2, w1r[6], o2);
-            o0 = ffma2(carry[2 * jj + 1], w1r[1], o0);
-            o1 = ffma2(a1, w1r[4], o1);
-            o2 = ffma2(c1, w1r[7], o2);
-            o0 = ffma2(carry[2 * jj + 2], w1r[2], o0);
-            o1 = ffma2(a2, w1r[5], o1);
-            o2 = ffma2(c2, w1r[8], o2);
-            const float2 o = make_float2(o0.x + o1.x + o2.x, o0.y + o1.y + o2.y);
-            if (jj < jn) store_pair<TO, VEC_STORE>(orow + jj * C, o, has_y);
-
-            carry[2 * jj] = prev2;
-            carry[2 * jj + 1] = c1;
-            prev1 = a2;
-            prev2 = c2;
         }
-        carry[2 * J] = prev2;
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            prev1[q] = (v1 && j0 > 0) ? relu2(prev1[q]) : make_float2(0.f, 0.f);
+            prev2[q] = (v2 && j0 > 0) ? relu2(prev2[q]) : make_float2(0.f, 0.f);
+        }
+
+        // one output row; CHECK adds the per-column and per-row validity selects
+        auto row = [&](auto check) {
+            constexpr bool CHECK = decltype(check)::value;
+#pragma unroll
+            for (int jj = 0; jj < J; ++jj) {
+                const int j = j0 + jj;
+                const bool cv1 = 2 * j < F2, cv2 = 2 * j + 1 < F2;
+                // mel columns 4j-1 .. 4j+3 are staged columns 3+4jj .. 7+4jj (column 3+4jj carries
+                // over from the previous column).  Window row p feeds h row r1 through tap row p
+                // (p <= 2) and h row r2 through tap row p-2 (p >= 2); each row is used as it arrives.
+                float2 a1[NPR], a2[NPR], c1[NPR], c2[NPR];
+#pragma unroll
+                for (int q = 0; q < NPR; ++q) a1[q] = a2[q] = c1[q] = c2[q] = b0r[q];
+#pragma unroll
+                for (int p = 0; p < 5; ++p) {
+                    const float4 lo = *reinterpret_cast<const float4 *>(&sm[rr + p][4 + 4 * jj]);
+                    const float4 hi = *reinterpret_cast<const float4 *>(&sm[rr + p][6 + 4 * jj]);
+                    const float2 m[5] = {m0[p], make_float2(lo.x, lo.y), make_float2(lo.z, lo.w),
+                                         make_float2(hi.x, hi.y), make_float2(hi.z, hi.w)};
+                    m0[p] = m[4];
+#pragma unroll
+                    for (int q = 0; q < NPR; ++q) {
+                        if (p <= 2) {
+#pragma unroll
+                            for (int qq = 0; qq < 3; ++qq) {
+                                a1[q] = ffma2(m[qq], w0r[p * 3 + qq][q], a1[q]);
+                                a2[q] = ffma2(m[qq + 2], w0r[p * 3 + qq][q], a2[q]);
+                            }
+                        }
+                        if (p >= 2) {
+#pragma unroll
+                            for (int qq = 0; qq < 3; ++qq) {
+                                c1[q] = ffma2(m[qq], w0r[(p - 2) * 3 + qq][q], c1[q]);
+                                c2[q] = ffma2(m[qq + 2], w0r[(p - 2) * 3 + qq][q], c2[q]);
+                            }
+                        }
+                    }
+                }
+                float2 o[NPR];
+#pragma unroll
+                for (int q = 0; q < NPR; ++q) {
+                    if constexpr (CHECK) {
+                        a1[q] = (v1 && cv1) ? relu2(a1[q]) : make_float2(0.f, 0.f);
+                        a2[q] = (v1 && cv2) ? relu2(a2[q]) : make_float2(0.f, 0.f);
+                        c1[q] = (v2 && cv1) ? relu2(c1[q]) : make_float2(0.f, 0.f);
+                        c2[q] = (v2 && cv2) ? relu2(c2[q]) : make_float2(0.f, 0.f);
+                    } else {
+                        a1[q] = relu2(a1[q]);
+                        a2[q] = relu2(a2[q]);
+                        c1[q] = relu2(c1[q]);
+                        c2[q] = relu2(c2[q]);
+                    }
+                    // conv_dw1 as two independent sums, added at the end
+                    float2 oa = b1r[q], ob2 = make_float2(0.f, 0.f);
+                    oa = ffma2(carry[2 * jj][q], w1r[0][q], oa);
+                    ob2 = ffma2(prev1[q], w1r[3][q], ob2);
+                    oa = ffma2(carry[2 * jj + 1][q], w1r[1][q], oa);
+                    ob2 = ffma2(a1[q], w1r[4][q], ob2);
+                    oa = ffma2(carry[2 * jj + 2][q], w1r[2][q], oa);
+                    ob2 = ffma2(a2[q], w1r[5][q], ob2);
+                    oa = ffma2(prev2[q], w1r[6][q], oa);
+                    ob2 = ffma2(c1[q], w1r[7][q], ob2);
+                    oa = ffma2(c2[q], w1r[8][q], oa);
+                    o[q] = make_float2(oa.x + ob2.x, oa.y + ob2.y);
+                    carry[2 * jj][q] = prev2[q];
+                    carry[2 * jj + 1][q] = c1[q];
+                    prev1[q] = a2[q];
+                    prev2[q] = c2[q];
+                }
+                if (jj < jn) store_pairs<TO, VEC_STORE, NPR>(orow + jj * C, o, nvalid);
+            }
+        };
+        if (v1 && v2 && cols_all) row(std::false_type{});
+        else row(std::true_type{});
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) carry[2 * J][q] = prev2[q];
     }
 }
 
@@ -242,7 +312,7 @@ cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s) {
     auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
     const int64_t T2 = s2(a.T), F2 = s2(a.F), T4 = s2(T2), F4 = s2(F2);
     if (a.B == 0 || T4 == 0) return cudaSuccess;
-    const int64_t nCT = (a.C + 63) / 64;
+    const int64_t nCT = (a.C + 64 * kSubNPR - 1) / (64 * kSubNPR);
     const int warps = static_cast<int>(nCT < kSubWarpsMax ? nCT : kSubWarpsMax);
     const int64_t nCG = (nCT + warps - 1) / warps;
     const int64_t nJB = (F4 + kSubJ - 1) / kSubJ;
@@ -251,11 +321,12 @@ cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s) {
     // indices inside the kernel are 32-bit: an item's output and mel planes must fit
     if (grid > kMaxGrid || T4 * F4 * a.C >= (1LL << 31) || a.T * a.F >= (1LL << 31) || 9 * a.C >= (1LL << 31))
         return cudaErrorInvalidConfiguration;
-    const bool even = (a.C % 2) == 0;
-    const bool aligned = (reinterpret_cast<uintptr_t>(a.out) % (a.bf16_out ? 4 : 8)) == 0;
-    const bool vec = even && aligned;
+    // vector stores of 2*kSubNPR channels need C a multiple of that and an aligned output
+    const int vch = 2 * kSubNPR;
+    const bool vec = (a.C % vch) == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.out) % (static_cast<uintptr_t>(vch) * (a.bf16_out ? 2 : 4))) == 0;
 #define DW_SUB_LAUNCH(TO, VS)                                                                           \
-    dw_subsample_kernel<TO, VS, kSubJ, kSubRI><<<static_cast<unsigned>(grid), warps * 32, 0, s>>>(          \
+    dw_subsample_kernel<TO, VS, kSubJ, kSubRI, kSubNPR><<<static_cast<unsigned>(grid), warps * 32, 0, s>>>(          \
         a.mel, a.w0, a.b0, a.w1, a.b1, static_cast<TO *>(a.out), a.lengths, a.out_lengths,                   \
         static_cast<int>(a.B), static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C),           \
         static_cast<int>(T2), static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt,          \
