@@ -19,6 +19,7 @@
 //  2. finalize kernel: dW[k][c] and dbias[c] = the partial rows added in row order.
 // Widths without a specialisation run in passes of 8 taps over the same data.
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "dw_internal.h"
 
@@ -179,6 +180,9 @@ conv1d_dw_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
 #ifndef DW_DW_BLOCKS
 #define DW_DW_BLOCKS 2
 #endif
+#ifndef DW_DW_ORDERED
+#define DW_DW_ORDERED 1
+#endif
 constexpr int kDwConsumers = DW_DW_CONSUMERS;  // consumer warps per block
 constexpr int kDwR = DW_DW_R;                  // frames per consumer thread per unit
 constexpr int kDwStages = DW_DW_STAGES;        // shared-memory ring depth
@@ -205,6 +209,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     using S = DwTmaShape<T, V, KB>;
     constexpr int NP = Pairs<V>::n;
     constexpr int R = kDwR;
+    launch_dependents();  // the finalize may be scheduled now; it waits for this grid to finish
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw);
     uint64_t *empty = full + kDwStages;
@@ -260,7 +265,13 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
             if (!ok) break;
             if (lane == 0) {
                 int b, t0, L;
-                unit_at(u, b, t0, L);
+                if (ordered || it >= kDwStages) {
+                    unit_at(u, b, t0, L);
+                } else {  // the first ring-full is issued before any length is read
+                    b = u / nT;
+                    t0 = (u % nT) * S::TT;
+                    L = Tn;
+                }
                 if (t0 < L) {  // frames before 0 or past T arrive as zeros; [L, T) is masked by the consumers
                     unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
@@ -289,36 +300,45 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
                 const unsigned char *dp = st + (S::XROWS + cw * R) * S::ROWB;
                 const unsigned char *xp = st + (cw * R) * S::ROWB;
                 const int jb = tg + k_off - pad_left;  // frame of this thread's first x row
-                const bool all_valid = tg + R <= L && jb >= 0 && jb + R + KB - 1 <= L;
-                float2 dz[R][NP];
+                // CHECK = false: every dy and x row of the run is inside [0, len_b)
+                auto run = [&](auto check) {
+                    constexpr bool CHECK = decltype(check)::value;
+                    float2 dz[R][NP];
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    Vec<T, V> v;
-                    v.r = *reinterpret_cast<const decltype(v.r) *>(dp + r * S::ROWB);
-                    if (!all_valid && tg + r >= L) v.zero();
-                    v.to_f2(dz[r]);
+                    for (int r = 0; r < R; ++r) {
+                        Vec<T, V> v;
+                        v.r = *reinterpret_cast<const decltype(v.r) *>(dp + r * S::ROWB);
+                        if constexpr (CHECK) {
+                            if (tg + r >= L) v.zero();
+                        }
+                        v.to_f2(dz[r]);
 #pragma unroll
-                    for (int p = 0; p < NP; ++p) {
-                        accb[p].x += dz[r][p].x;
-                        accb[p].y += dz[r][p].y;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < R + KB - 1; ++i) {
-                    Vec<T, V> v;
-                    v.r = *reinterpret_cast<const decltype(v.r) *>(xp + i * S::ROWB);
-                    if (!all_valid && (jb + i < 0 || jb + i >= L)) v.zero();
-                    float2 xf[NP];
-                    v.to_f2(xf);
-#pragma unroll
-                    for (int k = 0; k < KB; ++k) {
-                        const int r = i - k;
-                        if (r >= 0 && r < R) {
-#pragma unroll
-                            for (int p = 0; p < NP; ++p) acc[k][p] = ffma2(dz[r][p], xf[p], acc[k][p]);
+                        for (int p = 0; p < NP; ++p) {
+                            accb[p].x += dz[r][p].x;
+                            accb[p].y += dz[r][p].y;
                         }
                     }
-                }
+#pragma unroll
+                    for (int i = 0; i < R + KB - 1; ++i) {
+                        Vec<T, V> v;
+                        v.r = *reinterpret_cast<const decltype(v.r) *>(xp + i * S::ROWB);
+                        if constexpr (CHECK) {
+                            if (jb + i < 0 || jb + i >= L) v.zero();
+                        }
+                        float2 xf[NP];
+                        v.to_f2(xf);
+#pragma unroll
+                        for (int k = 0; k < KB; ++k) {
+                            const int r = i - k;
+                            if (r >= 0 && r < R) {
+#pragma unroll
+                                for (int p = 0; p < NP; ++p) acc[k][p] = ffma2(dz[r][p], xf[p], acc[k][p]);
+                            }
+                        }
+                    }
+                };
+                if (tg + R <= L && jb >= 0 && jb + R + KB - 1 <= L) run(std::false_type{});
+                else run(std::true_type{});
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -367,16 +387,31 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     cluster.sync();
 }
 
+// dW[k][c] / dbias[c] = sum over the partial rows.  A block covers 32 consecutive (k, c) entries
+// with 8 row groups: group r adds rows r, r+8, r+16, ... in order, then the 8 group sums are
+// added in a fixed tree.  The order depends only on the row count, so results are reproducible.
 __global__ void __launch_bounds__(256)
 conv1d_dw_finalize_kernel(const float *__restrict__ partials, float *__restrict__ dw,
                           float *__restrict__ dbias, int Gp, int K, int64_t C) {
-    const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (e >= static_cast<int64_t>(K + 1) * C) return;
-    const int64_t k = e / C, c = e % C;
+    __shared__ float red[8][33];
+    grid_dependency_wait();  // launched programmatically after the partial kernel
+    const int col = threadIdx.x % 32, rg = threadIdx.x / 32;
+    const int64_t E = static_cast<int64_t>(K + 1) * C;
+    const int64_t e = static_cast<int64_t>(blockIdx.x) * 32 + col;
     float s = 0.f;
-    for (int g = 0; g < Gp; ++g) s += partials[(static_cast<int64_t>(g) * (K + 1) + k) * C + c];
-    if (k < K) dw[k * C + c] = s;
-    else if (dbias) dbias[c] = s;
+    if (e < E) {
+#pragma unroll 4
+        for (int g = rg; g < Gp; g += 8) s += __ldg(partials + static_cast<int64_t>(g) * E + e);
+    }
+    red[rg][col] = s;
+    __syncthreads();
+    if (rg == 0 && e < E) {
+        const float t = ((red[0][col] + red[1][col]) + (red[2][col] + red[3][col])) +
+                        ((red[4][col] + red[5][col]) + (red[6][col] + red[7][col]));
+        const int64_t k = e / C, c = e % C;
+        if (k < K) dw[k * C + c] = t;
+        else if (dbias) dbias[c] = t;
+    }
 }
 
 __global__ void conv1d_dw_zero_kernel(float *__restrict__ dw, float *__restrict__ dbias, int K, int64_t C) {
@@ -441,7 +476,7 @@ template <typename T, int V, int KB>
 cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s) {
     using S = DwTmaShape<T, V, KB>;
     auto kern = conv1d_dw_tma_kernel<T, V, KB>;
-    const int ordered = a.B <= kOrderMaxItems ? 1 : 0;
+    const int ordered = (DW_DW_ORDERED && a.B <= kOrderMaxItems) ? 1 : 0;
     const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
     const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
                                               S::SMEM + static_cast<int>(3 * (kOrderMaxItems + 1) * sizeof(int)) + 16);
@@ -472,7 +507,8 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
         const int64_t ucap = (units + c - 1) / c * c;                  // no more blocks than units
         if (gg > ucap) gg = ucap;
         if (gg / c > a.G) gg = static_cast<int64_t>(a.G) * c;          // workspace rows
-        if (gg > best_g) {
+        // a smaller cluster must fill clearly more of the GPU to be worth its extra partial rows
+        if (gg > best_g + best_g / 32) {
             best_g = static_cast<int>(gg);
             best_c = c;
         }
@@ -582,9 +618,17 @@ cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
     int gp = 0;
     cudaError_t e = a.bf16 ? launch_dtype<bf16>(a, &gp, s) : launch_dtype<float>(a, &gp, s);
     if (e != cudaSuccess) return e;
-    conv1d_dw_finalize_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(a.partials, a.dw, a.dbias,
-                                                                                   gp, a.K, a.C);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((n + 31) / 32));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, conv1d_dw_finalize_kernel, static_cast<const float *>(a.partials), a.dw, a.dbias,
+                              gp, a.K, static_cast<int64_t>(a.C));
 }
 
 }  // namespace dwk

@@ -23,6 +23,8 @@
 //    neighbour warp and hit L1/L2, so DRAM sees each input frame about once;
 //  - input frames at or beyond len_b are never loaded (predicated off), and a run that lies
 //    wholly beyond len_b only stores zeros.
+#include <type_traits>
+
 #include "dw_internal.h"
 
 namespace dwk {
@@ -116,14 +118,16 @@ conv1d_fwd_vec_kernel(const T *__restrict__ x, const float *__restrict__ w,
 // producer issues ONE tensor copy (cp.async.bulk.tensor: CT channels x (TT + K - 1) frames,
 // starting K-1 halo frames early) into a kTmaStages-deep shared-memory ring; completion is
 // counted in bytes on the stage's "full" mbarrier.  Frames before 0 or past T arrive as zeros
-// (the padding).  Consumers read their R + K - 1 rows from shared memory with the same
+// (the padding).  Each block keeps one channel tile, so its weights stay in registers, and its
+// first ring-full of copies goes out before any length is known.  Consumers read their R + K - 1 rows from shared memory with the same
 // register window as above, mask frames in [len_b, T), store straight to global memory and
 // release the stage on its "empty" mbarrier.  HBM never waits on compute: up to kTmaStages
 // tiles are in flight per SM while the consumers work on one.  Wholly masked tiles are not
 // read at all.
 // ---------------------------------------------------------------------------------------
-// Tuned on B200 (sweeps over consumer warps, frames per thread, ring depth and blocks per
-// SM): 3 blocks of 4 consumer warps per SM, 3 stages, 12 frames per thread (16 for K > 9).
+// Tuned on B200 (sweeps over consumer warps, frames per thread, ring depth, blocks per SM and
+// tile width): 3 blocks of 4 consumer warps per SM, 3 stages, 12 frames per thread (16 for
+// K > 9), tiles 128 channels wide (256-byte bf16 rows; narrower rows cost DRAM efficiency).
 #ifndef DW_FWD_CONSUMERS
 #define DW_FWD_CONSUMERS 4
 #endif
@@ -139,18 +143,21 @@ conv1d_fwd_vec_kernel(const T *__restrict__ x, const float *__restrict__ w,
 #ifndef DW_FWD_BLOCKS
 #define DW_FWD_BLOCKS 3
 #endif
+
 constexpr int kTmaConsumers = DW_FWD_CONSUMERS;  // consumer warps per block
 constexpr int kTmaR = DW_FWD_R;                  // frames per consumer thread, K <= 9
 constexpr int kTmaRWide = DW_FWD_R_WIDE;         // frames per consumer thread, K > 9
 constexpr int kTmaStages = DW_FWD_STAGES;        // shared-memory ring depth
 constexpr int kTmaBlocks = DW_FWD_BLOCKS;        // resident blocks per SM
+
 constexpr int kTmaThreads = 32 * (1 + kTmaConsumers);
 
 template <typename T, int V, int K>
 struct TmaShape {
     static constexpr int R = (K > 9) ? kTmaRWide : kTmaR;
-    static constexpr int CT = 32 * V;                 // channels per tile (one warp row)
-    static constexpr int TT = kTmaConsumers * R;      // output frames per tile
+    static constexpr int WPR = (V >= 4) ? 1 : 2;      // consumer warps side by side: 128-channel tiles
+    static constexpr int CT = 32 * V * WPR;           // channels per tile
+    static constexpr int TT = (kTmaConsumers / WPR) * R;  // output frames per tile
     static constexpr int ROWS = TT + K - 1;           // input rows per tile
     static constexpr int ROWB = CT * static_cast<int>(sizeof(T));
     static constexpr int STAGE_BYTES = ROWS * ROWB;
@@ -161,7 +168,7 @@ template <typename T, int V, int K>
 __global__ void __launch_bounds__(kTmaThreads, kTmaBlocks)
 conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restrict__ w,
                       const float *__restrict__ bias, T *__restrict__ y, const int32_t *__restrict__ lengths,
-                      int B, int Tn, int C, int pad_left, int flip, int nT, int nC, int ntiles, int ordered) {
+                      int B, int Tn, int C, int pad_left, int flip, int nT, int nC, int ntiles) {
     using S = TmaShape<T, V, K>;
     constexpr int NP = Pairs<V>::n;
     constexpr int R = S::R;
@@ -170,9 +177,11 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     uint64_t *empty = full + kTmaStages;
     unsigned char *stages = smem_raw + 128;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    int *ord_mem = reinterpret_cast<int *>(stages + static_cast<size_t>(kTmaStages) * S::STAGE_BYTES);
-    TileOrder order{ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), B, nT, nC, 0};
-    if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
+    // Each block keeps one channel tile (the grid is a multiple of nC), so its weights stay in
+    // registers, and walks that tile's (item, frame-run) positions q0, q0 + qstride, ...
+    const int my_ct = static_cast<int>(blockIdx.x % nC);
+    const int q0 = static_cast<int>(blockIdx.x / nC), qstride = static_cast<int>(gridDim.x / nC);
+    const int nq = ntiles / nC;  // positions per channel tile
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTmaStages; ++i) {
             mbar_init(&full[i], 1);
@@ -181,35 +190,22 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
         fence_barrier_init();
     }
     __syncthreads();
-    if (ordered) order.V = order.pv[B];
-    // position g of this block's walk -> tile (b, t0, ct) and the item's length
-    auto tile_at = [&](int g, int &b, int &t0, int &ct, int &L) {
-        if (ordered) {
-            int tt;
-            order.map(g, b, tt, ct, L);
-            t0 = tt * S::TT;
-        } else {
-            ct = g % nC;
-            const int bt = g / nC;
-            t0 = (bt % nT) * S::TT;
-            b = bt / nT;
-            L = static_cast<int>(clamp_len(lengths, b, Tn));
-        }
-    };
     if (warp == 0) {  // producer warp: one elected lane, one tensor copy per tile
         if (lane == 0) prefetch_tmap(&xmap);
         int it = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        for (int q = q0; q < nq; q += qstride, ++it) {
             const int s = it % kTmaStages;
             const uint32_t ph = (it / kTmaStages) & 1;
+            const int b = q / nT, t0 = (q % nT) * S::TT;
+            // the first ring-full of tiles is issued without waiting for the item's length (a
+            // wholly masked one is read needlessly); later tiles skip the read when t0 >= len
+            const int L = (it >= kTmaStages && lane == 0) ? static_cast<int>(clamp_len(lengths, b, Tn)) : Tn;
             if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) return;
             if (lane == 0) {
-                int b, t0, ct, L;
-                tile_at(tile, b, t0, ct, L);
                 if (t0 < L) {  // rows before frame 0 or past T arrive as zeros; rows in [L, T) are masked by the consumers
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                    tma_load_3d(stages + static_cast<size_t>(s) * S::STAGE_BYTES, &xmap, ct * S::CT, t0 - pad_left, b,
-                                &full[s]);
+                    tma_load_3d(stages + static_cast<size_t>(s) * S::STAGE_BYTES, &xmap, my_ct * S::CT, t0 - pad_left,
+                                b, &full[s]);
                 } else {
                     mbar_arrive(&full[s]);  // a wholly masked tile: nothing to read
                 }
@@ -220,26 +216,29 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     }
 
     // consumer warps: warp g+1 computes frames [t0 + g R, t0 + g R + R) of each tile
-    const int g = warp - 1;
+    const int g = (warp - 1) / S::WPR;                  // row group
+    const int wc = ((warp - 1) % S::WPR) * 32 * V;      // first channel of this warp within the tile
+    const int cv = my_ct * S::CT + wc + lane * V;
+    const bool active = cv < C;
+    float2 wv[K][NP], bv[NP];
+    if (active) {  // the block's channel tile never changes: weights stay in registers
+#pragma unroll
+        for (int k = 0; k < K; ++k) load_param<V>(w + static_cast<int64_t>(flip ? K - 1 - k : k) * C + cv, wv[k]);
+        if (bias) load_param<V>(bias + cv, bv);
+        else {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) bv[p] = make_float2(0.f, 0.f);
+        }
+    }
     int it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    for (int q = q0; q < nq; q += qstride, ++it) {
         const int s = it % kTmaStages;
         const uint32_t ph = (it / kTmaStages) & 1;
-        int b, t0, ct, L;
-        tile_at(tile, b, t0, ct, L);
-        const int cv = ct * S::CT + lane * V;
-        const bool active = cv < C;
+        const int b = q / nT, t0 = (q % nT) * S::TT;
+        const int L = static_cast<int>(clamp_len(lengths, b, Tn));  // issued before the wait below
         const int tg = t0 + g * R;
-        float2 wv[K][NP], acc[R][NP];
-        if (active && tg < L) {  // issue the parameter loads before waiting for the tile
-#pragma unroll
-            for (int k = 0; k < K; ++k) load_param<V>(w + static_cast<int64_t>(flip ? K - 1 - k : k) * C + cv, wv[k]);
-            float2 bv[NP];
-            if (bias) load_param<V>(bias + cv, bv);
-            else {
-#pragma unroll
-                for (int p = 0; p < NP; ++p) bv[p] = make_float2(0.f, 0.f);
-            }
+        float2 acc[R][NP];
+        if (active && tg < L) {
 #pragma unroll
             for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -254,32 +253,43 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
                     if (tg + r < Tn) Vec<T, V>::store_zero(yp + static_cast<int64_t>(r) * C);
             } else {
                 const unsigned char *sp = stages + static_cast<size_t>(s) * S::STAGE_BYTES +
-                                          (g * R) * S::ROWB + lane * V * static_cast<int>(sizeof(T));
+                                          (g * R) * S::ROWB + (wc + lane * V) * static_cast<int>(sizeof(T));
                 const int jb = tg - pad_left;  // frame of this thread's first row
-                const bool rows_valid = jb >= 0 && jb + R + K - 1 <= L;
-                const bool outs_valid = tg + R <= L;
+                // CHECK = false: every row and every output of the run is inside [0, len_b)
+                auto run = [&](auto check) {
+                    constexpr bool CHECK = decltype(check)::value;
+                    T *dst = yp;
 #pragma unroll
-                for (int i = 0; i < R + K - 1; ++i) {
-                    Vec<T, V> v;
-                    v.r = *reinterpret_cast<const decltype(v.r) *>(sp + i * S::ROWB);
-                    if (!rows_valid && (jb + i < 0 || jb + i >= L)) v.zero();
-                    float2 xf[NP];
-                    v.to_f2(xf);
+                    for (int i = 0; i < R + K - 1; ++i) {
+                        Vec<T, V> v;
+                        v.r = *reinterpret_cast<const decltype(v.r) *>(sp + i * S::ROWB);
+                        if constexpr (CHECK) {
+                            if (jb + i < 0 || jb + i >= L) v.zero();
+                        }
+                        float2 xf[NP];
+                        v.to_f2(xf);
 #pragma unroll
-                    for (int k = 0; k < K; ++k) {
-                        const int r = i - k;
-                        if (r >= 0 && r < R) {
+                        for (int k = 0; k < K; ++k) {
+                            const int r = i - k;
+                            if (r >= 0 && r < R) {
 #pragma unroll
-                            for (int p = 0; p < NP; ++p) acc[r][p] = ffma2(xf[p], wv[k][p], acc[r][p]);
+                                for (int p = 0; p < NP; ++p) acc[r][p] = ffma2(xf[p], wv[k][p], acc[r][p]);
+                            }
+                        }
+                        const int rd = i - (K - 1);
+                        if (rd >= 0) {
+                            if constexpr (CHECK) {
+                                if (tg + rd < L) Vec<T, V>::store(dst, acc[rd]);
+                                else if (tg + rd < Tn) Vec<T, V>::store_zero(dst);
+                            } else {
+                                Vec<T, V>::store(dst, acc[rd]);
+                            }
+                            dst += C;
                         }
                     }
-                    const int rd = i - (K - 1);
-                    if (rd >= 0) {
-                        T *dst = yp + static_cast<int64_t>(rd) * C;
-                        if (outs_valid || tg + rd < L) Vec<T, V>::store(dst, acc[rd]);
-                        else if (tg + rd < Tn) Vec<T, V>::store_zero(dst);
-                    }
-                }
+                };
+                if (jb >= 0 && jb + R + K - 1 <= L) run(std::false_type{});  // implies tg + R <= L
+                else run(std::true_type{});
             }
         }
         __syncwarp();
@@ -415,8 +425,7 @@ template <typename T, int V, int K>
 cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     using S = TmaShape<T, V, K>;
     auto kern = conv1d_fwd_tma_kernel<T, V, K>;
-    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
-                                              S::SMEM + static_cast<int>(3 * (kOrderMaxItems + 1) * sizeof(int)) + 16);
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::SMEM);
     if (attr != cudaSuccess) return attr;
     const int nC = static_cast<int>((a.C + S::CT - 1) / S::CT);
     const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
@@ -427,11 +436,11 @@ cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     if (me != cudaSuccess) return me;
     int64_t grid = static_cast<int64_t>(sm_count()) * kTmaBlocks;
     if (grid > ntiles) grid = ntiles;
-    const int ordered = a.B <= kOrderMaxItems ? 1 : 0;
-    const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
-    kern<<<static_cast<unsigned>(grid), kTmaThreads, smem, s>>>(
+    grid = grid / nC * nC;  // whole channel tiles per block walk
+    if (grid < nC) grid = nC;
+    kern<<<static_cast<unsigned>(grid), kTmaThreads, S::SMEM, s>>>(
         xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.B), static_cast<int>(a.T),
-        static_cast<int>(a.C), a.pad_left, a.flip, nT, nC, static_cast<int>(ntiles), ordered);
+        static_cast<int>(a.C), a.pad_left, a.flip, nT, nC, static_cast<int>(ntiles));
     return cudaGetLastError();
 }
 

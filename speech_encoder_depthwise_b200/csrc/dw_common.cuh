@@ -317,3 +317,14 @@ struct TileOrder {
 };
 
 }  // namespace dwk
+
+namespace dwk {
+
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the previous kernel in the stream drains; it must wait (grid_dependency_wait)
+// before touching memory the previous kernel writes.  A kernel lets its dependents launch
+// early with launch_dependents (they still wait for its completion before reading).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace dwk

@@ -44,6 +44,33 @@ constexpr int kSubRI = DW_SUB_RI;        // output rows per block
 constexpr int kSubWarpsMax = 4;          // channel tiles (64 channels each) per block
 constexpr int kSubMinBlocks = DW_SUB_MINB;  // resident blocks per SM the register budget aims at
 constexpr int kSubNPR = DW_SUB_NPR;         // channel pairs per thread
+#ifndef DW_SUB_SCALAR
+#define DW_SUB_SCALAR 0
+#endif
+// 1: mel staged as plain floats and conv0 as scalar FMAs with the mel value as a direct operand
+// (one 16-byte shared load gives four mel columns); 0: mel staged as {m, m} pairs and conv0 as
+// packed FMAs (one 16-byte load gives two columns).
+constexpr bool kSubScalar = DW_SUB_SCALAR != 0;
+
+// acc += m * w for a channel pair: packed FMA with a {m, m} pair, or two scalar FMAs.
+__device__ __forceinline__ float2 mel_fma(float2 m, float2 w, float2 acc) { return ffma2(m, w, acc); }
+__device__ __forceinline__ float2 mel_fma(float m, float2 w, float2 acc) {
+    return make_float2(fmaf(m, w.x, acc.x), fmaf(m, w.y, acc.y));
+}
+__device__ __forceinline__ void stage_mel(float2 &dst, float v) { dst = make_float2(v, v); }
+__device__ __forceinline__ void stage_mel(float &dst, float v) { dst = v; }
+
+// Staged mel columns c .. c+3 of one row (c a multiple of 4): one 16-byte shared load of plain
+// floats, or two of {m, m} pairs.
+__device__ __forceinline__ void load4(const float *row, int c, float (&m)[4]) {
+    const float4 v = *reinterpret_cast<const float4 *>(row + c);
+    m[0] = v.x; m[1] = v.y; m[2] = v.z; m[3] = v.w;
+}
+__device__ __forceinline__ void load4(const float2 *row, int c, float2 (&m)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(row + c), b = *reinterpret_cast<const float4 *>(row + c + 2);
+    m[0] = make_float2(a.x, a.y); m[1] = make_float2(a.z, a.w);
+    m[2] = make_float2(b.x, b.y); m[3] = make_float2(b.z, b.w);
+}
 
 template <typename TO, bool VEC_STORE>
 __device__ __forceinline__ void store_pair(TO *p, float2 v, bool has_y);
@@ -99,7 +126,8 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
     constexpr int NMR = 4 * RI + 3;   // mel rows a block reads
     constexpr int W = 4 * J + 8;      // staged mel columns: [4 j0 - 4, 4 j0 + 4 J + 4)
     constexpr int CW = 64 * NPR;      // channels per warp
-    __shared__ __align__(16) float2 sm[NMR][W];
+    using MelT = typename std::conditional<kSubScalar, float, float2>::type;
+    __shared__ __align__(16) MelT sm[NMR][W];
 
     const int warps = blockDim.x / 32;
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
@@ -135,7 +163,7 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
             const int mr = mrow0 + rr, mc = mcol0 + cc;
             float v = 0.f;
             if (mr >= 0 && mr < L && mc >= 0 && mc < F) v = __ldg(melb + mr * F + mc);  // frames >= len read as 0
-            sm[rr][cc] = make_float2(v, v);
+            stage_mel(sm[rr][cc], v);
         }
     }
     __syncthreads();
@@ -183,7 +211,7 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
 #pragma unroll
                 for (int p = 0; p < 3; ++p)
 #pragma unroll
-                    for (int qq = 0; qq < 3; ++qq) a = ffma2(sm[p][2 * n + 1 + qq], w0r[p * 3 + qq][q], a);
+                    for (int qq = 0; qq < 3; ++qq) a = mel_fma(sm[p][2 * n + 1 + qq], w0r[p * 3 + qq][q], a);
                 carry[n][q] = ok ? relu2(a) : make_float2(0.f, 0.f);
             }
         }
@@ -201,24 +229,25 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
         const bool v1 = r1 >= 0 && r1 < hrows, v2 = r2 >= 0 && r2 < hrows;
         const int rr = 2 * r1 - Pt - mrow0;            // staged row of mel row 2 r1 - Pt
         // h column 2 j0 - 1 of rows r1, r2 (staged mel columns 1..3); column 3 then carries over
-        float2 prev1[NPR], prev2[NPR], m0[5];
+        float2 prev1[NPR], prev2[NPR];
+        MelT m0[5];
 #pragma unroll
         for (int q = 0; q < NPR; ++q) prev1[q] = prev2[q] = b0r[q];
 #pragma unroll
         for (int p = 0; p < 5; ++p) {
-            const float2 m1 = sm[rr + p][1];
-            const float4 m23 = *reinterpret_cast<const float4 *>(&sm[rr + p][2]);
-            const float2 m[3] = {m1, make_float2(m23.x, m23.y), make_float2(m23.z, m23.w)};
+            MelT m4[4];
+            load4(sm[rr + p], 0, m4);   // staged columns 0..3; columns 1..3 are mel 4 j0 - 3 .. 4 j0 - 1
+            const MelT m[3] = {m4[1], m4[2], m4[3]};
             m0[p] = m[2];
 #pragma unroll
             for (int q = 0; q < NPR; ++q) {
                 if (p <= 2) {
 #pragma unroll
-                    for (int qq = 0; qq < 3; ++qq) prev1[q] = ffma2(m[qq], w0r[p * 3 + qq][q], prev1[q]);
+                    for (int qq = 0; qq < 3; ++qq) prev1[q] = mel_fma(m[qq], w0r[p * 3 + qq][q], prev1[q]);
                 }
                 if (p >= 2) {
 #pragma unroll
-                    for (int qq = 0; qq < 3; ++qq) prev2[q] = ffma2(m[qq], w0r[(p - 2) * 3 + qq][q], prev2[q]);
+                    for (int qq = 0; qq < 3; ++qq) prev2[q] = mel_fma(m[qq], w0r[(p - 2) * 3 + qq][q], prev2[q]);
                 }
             }
         }
@@ -243,25 +272,24 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
                 for (int q = 0; q < NPR; ++q) a1[q] = a2[q] = c1[q] = c2[q] = b0r[q];
 #pragma unroll
                 for (int p = 0; p < 5; ++p) {
-                    const float4 lo = *reinterpret_cast<const float4 *>(&sm[rr + p][4 + 4 * jj]);
-                    const float4 hi = *reinterpret_cast<const float4 *>(&sm[rr + p][6 + 4 * jj]);
-                    const float2 m[5] = {m0[p], make_float2(lo.x, lo.y), make_float2(lo.z, lo.w),
-                                         make_float2(hi.x, hi.y), make_float2(hi.z, hi.w)};
+                    MelT m4[4];
+                    load4(sm[rr + p], 4 + 4 * jj, m4);
+                    const MelT m[5] = {m0[p], m4[0], m4[1], m4[2], m4[3]};
                     m0[p] = m[4];
 #pragma unroll
                     for (int q = 0; q < NPR; ++q) {
                         if (p <= 2) {
 #pragma unroll
                             for (int qq = 0; qq < 3; ++qq) {
-                                a1[q] = ffma2(m[qq], w0r[p * 3 + qq][q], a1[q]);
-                                a2[q] = ffma2(m[qq + 2], w0r[p * 3 + qq][q], a2[q]);
+                                a1[q] = mel_fma(m[qq], w0r[p * 3 + qq][q], a1[q]);
+                                a2[q] = mel_fma(m[qq + 2], w0r[p * 3 + qq][q], a2[q]);
                             }
                         }
                         if (p >= 2) {
 #pragma unroll
                             for (int qq = 0; qq < 3; ++qq) {
-                                c1[q] = ffma2(m[qq], w0r[(p - 2) * 3 + qq][q], c1[q]);
-                                c2[q] = ffma2(m[qq + 2], w0r[(p - 2) * 3 + qq][q], c2[q]);
+                                c1[q] = mel_fma(m[qq], w0r[(p - 2) * 3 + qq][q], c1[q]);
+                                c2[q] = mel_fma(m[qq + 2], w0r[(p - 2) * 3 + qq][q], c2[q]);
                             }
                         }
                     }
