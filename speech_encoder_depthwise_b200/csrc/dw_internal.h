@@ -75,5 +75,10 @@ cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s);
 unsigned int conv1d_dw_take_error();
 
 cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
+// Tensor-core subsampler: usable when the output rows are 16-byte aligned (C * element size a
+// multiple of 16, aligned base); the SIMT kernel serves every other case.
+bool subsample_tc_eligible(const SubsampleArgs &a);
+cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s);
+unsigned int subsample_tc_take_error();
 
 }  // namespace dwk

@@ -340,6 +340,10 @@ cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s) {
     auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
     const int64_t T2 = s2(a.T), F2 = s2(a.F), T4 = s2(T2), F4 = s2(F2);
     if (a.B == 0 || T4 == 0) return cudaSuccess;
+    if (subsample_tc_eligible(a)) {
+        const cudaError_t e = subsample_tc_launch(a, s);
+        if (e != cudaErrorNotSupported) return e;
+    }
     const int64_t nCT = (a.C + 64 * kSubNPR - 1) / (64 * kSubNPR);
     const int warps = static_cast<int>(nCT < kSubWarpsMax ? nCT : kSubWarpsMax);
     const int64_t nCG = (nCT + warps - 1) / warps;

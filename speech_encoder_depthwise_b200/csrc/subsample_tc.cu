@@ -1,0 +1,677 @@
+// Fused depthwise-striding subsampler front with conv0 on the 5th-generation tensor cores
+// (NeMo PR #16114, "Use Fused Kernels for Depthwise Striding Subsampler", section "What does
+// this PR do ?", first kernel: mel [B,T,F,1] -> conv0 -> ReLU -> masking -> conv_dw1).
+//
+// conv0 maps one input channel to C channels with a 3x3 stride-2 window, so for a block of
+// h pixels it is a dense contraction: h[c, pixel] = sum over 9 taps of w0[tap, c] *
+// patch[pixel, tap] + b0[c].  It runs as tcgen05 MMAs with the channels as M (128 per tile)
+// and the h pixels of a unit as N, so the accumulator in tensor memory holds, in lane m,
+// every h pixel of channel m.  Each epilogue thread owns one channel: it reads its lane,
+// applies ReLU, and computes the depthwise conv_dw1 (3x3, stride 2) in float32 registers.
+// The conv0 output never leaves the SM.
+//
+// Precision.  The MMA reads its operands as TF32 (10 explicit mantissa bits), so every
+// float32 operand is split into x = hi + lo, hi = x with the low 13 mantissa bits cleared
+// and lo = x - hi (exact), and the contraction sums w_hi*m_hi + w_lo*m_hi + w_hi*m_lo with
+// float32 accumulation; the dropped w_lo*m_lo term and the truncation of lo are below 2^-20
+// of each product.  This is the three-product emulation of float32 products on TF32 units.
+// The bias b0 rides along as two more K columns (b0_hi, b0_lo against a 0/1 column that is 1
+// exactly for unmasked h pixels, whose other columns are then zero too).
+//
+// Work unit: item b, output rows [i0, i0+2), output columns [j0, j0+20).  It needs h rows
+// 2 i0 - Pt + [0, 5) and h columns 2 j0 - 1 + [0, 41): N = 5 x 41 = 205 pixels (208 with
+// the pad to a multiple of 16), K = 32 TF32 words per pixel.  Padding pixels, masked h rows
+// (at or beyond ceil(len/2)) and pixels outside the h plane get an all-zero patch, so their
+// h is exactly zero.
+//
+// Roles (416 threads, one block per SM, persistent):
+//   warps 0-7   epilogue: warp w reads TMEM lanes 32 (w % 4) + [0, 32) (its channel quarter)
+//               and output columns 10 (w / 4) + [0, 10) of the unit; results are staged in
+//               shared memory and written with one bulk tensor store per channel tile
+//   warps 8-11  patch builders: stage the unit's 11 x 83 mel window (frames at or beyond
+//               len read as zero), build the split patch rows in the 128-byte-swizzled
+//               K-major layout the MMA reads
+//   warp 12     allocates tensor memory; one thread issues the MMAs (4 K-steps of 8)
+// Pipelines: 2 patch stages (builders -> MMA), 2 accumulator buffers of 256 TMEM columns
+// (MMA -> epilogue), 2 output staging buffers (epilogue -> bulk store).  Every mbarrier wait
+// is bounded; a wait that gives up records an error (dw_device_error) and the block drains.
+#include "dw_internal.h"
+
+namespace dwk {
+namespace {
+
+constexpr int kRO = 2;                       // output rows per unit
+constexpr int kJO = 20;                      // output columns per unit
+constexpr int kHR = 2 * kRO + 1;             // h rows per unit
+constexpr int kHC = 2 * kJO + 1;             // h columns per unit
+constexpr int kNUsed = kHR * kHC;            // h pixels per unit
+constexpr int kN = (kNUsed + 15) / 16 * 16;  // MMA N
+constexpr int kMR = 2 * kHR + 1;             // mel rows per unit
+constexpr int kMC = 2 * kHC + 1;             // mel columns per unit
+constexpr int kMCP = kMC + 1;                // staged mel row stride (floats)
+constexpr int kMelElems = kMR * kMC;
+constexpr int kEpiWarps = 8, kPatchWarps = 4;
+constexpr int kEpiThreads = kEpiWarps * 32, kPatchThreads = kPatchWarps * 32;
+constexpr int kMmaWarp = kEpiWarps + kPatchWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kMelLoads = (kMelElems + kPatchThreads - 1) / kPatchThreads;
+constexpr int kRowBytes = 128;               // one K row: 32 TF32 words
+constexpr int kTileA = 128 * kRowBytes;
+constexpr int kTileB = kN * kRowBytes;
+constexpr int kTmemCols = 512, kTmemBuf = 256;
+constexpr int kHalfCols = kJO / 2;           // output columns per epilogue warp
+constexpr int kChunk = 5;                    // output columns per tensor-memory read
+constexpr int kBarEpi = 1, kBarPatch = 2;    // named barrier ids
+
+static_assert(kN <= 256 && kN % 16 == 0, "MMA N");
+static_assert(kTileB % 1024 == 0 && kTileA % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+static_assert(kHalfCols % kChunk == 0 && 2 * kChunk * kHR == 50 && kHC == 41, "epilogue chunking");
+
+template <typename TO, int CTG>
+struct TcLayout {
+    static constexpr int a_off = 0;
+    static constexpr int b_off = CTG * kTileA;
+    static constexpr int mel_bytes = (kMR * kMCP * 4 + 127) / 128 * 128;
+    static constexpr int mel_off = b_off + 2 * kTileB;
+    static constexpr int st_bytes = kRO * kJO * 128 * static_cast<int>(sizeof(TO));
+    static constexpr int st_off = mel_off + 2 * mel_bytes;   // staging 0, 1, then the zero tile
+    static constexpr int wt_off = st_off + 3 * st_bytes;      // conv_dw1 weight table
+    static constexpr int bar_off = wt_off + CTG * 10 * 128 * 4;
+    static constexpr int bytes = bar_off + 128;
+    // room to align the base to 1024; at least 120 KiB so that one block holds an SM (and all
+    // of its tensor memory)
+    static constexpr int alloc = bytes + 1024 > 120 * 1024 ? bytes + 1024 : 120 * 1024;
+};
+
+// ---------------------------------------------------------------- PTX wrappers (sm_100a)
+__device__ __forceinline__ void named_bar(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Named barrier that also ANDs a flag over the participating threads, so that a group of
+// warps takes a give-up decision together (a warp that left alone would strand the others at
+// their next barrier).
+__device__ __forceinline__ bool named_bar_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major, TF32 in, float32 accumulate.
+__device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on bar when every MMA this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 bytes in groups of
+// 8 rows (1024 bytes apart).  The leading-byte offset is unused in this mode.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = static_cast<uint64_t>((saddr & 0x3ffffu) >> 4);
+    d |= static_cast<uint64_t>(1) << 16;              // leading byte offset (16 B, ignored)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;      // stride byte offset: next 8-row group
+    d |= static_cast<uint64_t>(1) << 46;              // descriptor version for sm_100
+    d |= static_cast<uint64_t>(2) << 61;              // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: D float32, A and B TF32, both K-major, M = 128, N = kN.
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(kN >> 3) << 17) |
+                            (static_cast<uint32_t>(128 >> 4) << 24);
+
+// Accumulator column of h pixel (cc, rr) of a unit.  The 50 values an epilogue chunk reads
+// (h columns 10k+1 .. 10k+10, 5 rows each) sit at columns 48k + [0, 48) and 192 + 2k + [0, 2),
+// h column 0 at 200 + rr, so that every tensor-memory load starts at a multiple of its width.
+__host__ __device__ constexpr int acc_col(int cc, int rr) {
+    return cc == 0 ? 200 + rr
+                   : (((cc - 1) % 10) * kHR + rr < 48 ? 48 * ((cc - 1) / 10) + ((cc - 1) % 10) * kHR + rr
+                                                      : 192 + 2 * ((cc - 1) / 10) + ((cc - 1) % 10) * kHR + rr - 48);
+}
+
+// The 50 accumulator values of chunk k (h columns 10k+1 .. 10k+10) of this thread's lane, in
+// (column, row) order, waited for.
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t tacc, int k, float (&v)[50]) {
+    uint32_t r[50];
+    const uint32_t a = tacc + 48 * k, t = tacc + 192 + 2 * k;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15}, [%50];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%51];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, "
+        "%44, %45, %46, %47}, [%52];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%48, %49}, [%53];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
+          "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49])
+        : "r"(a), "r"(a + 16), "r"(a + 32), "r"(t)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 50; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// The 5 accumulator values (rows 0..4) of h column cc, one single-column load each, waited for.
+__device__ __forceinline__ void tmem_ld_column(uint32_t tacc, int cc, float (&v)[5]) {
+    uint32_t r[5];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%5];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%1}, [%6];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%2}, [%7];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%3}, [%8];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%4}, [%9];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4])
+        : "r"(tacc + acc_col(cc, 0)), "r"(tacc + acc_col(cc, 1)), "r"(tacc + acc_col(cc, 2)),
+          "r"(tacc + acc_col(cc, 3)), "r"(tacc + acc_col(cc, 4))
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 5; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Bulk tensor store of one staged box (coordinates innermost first: channel, column, row, item).
+__device__ __forceinline__ void tma_store_4d(const void *tmap, const void *src, int c, int j, int i, int b) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(smem_addr(src)), "r"(c), "r"(j), "r"(i), "r"(b)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// ---------------------------------------------------------------- operand rows
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
+
+// Row `row` of a K-major 128-byte-swizzled tile: 16-byte chunk k lands at chunk k ^ (row % 8).
+__device__ __forceinline__ void store_k_row(unsigned char *tile, int row, const float (&w)[32]) {
+    unsigned char *base = tile + row * kRowBytes;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<float4 *>(base + ((k ^ (row & 7)) << 4)) =
+            make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+}
+
+template <typename TO> __device__ __forceinline__ void stage_out(TO *p, float v);
+template <> __device__ __forceinline__ void stage_out<float>(float *p, float v) { *p = v; }
+template <> __device__ __forceinline__ void stage_out<bf16>(bf16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// The units q0, q0 + qs, q0 + 2 qs, ... of one block, in order, with the item and the place
+// inside it tracked incrementally (no division per unit); the length is read once per item.
+struct UnitWalk {
+    const int32_t *lengths;
+    int qs, per_item, nJB, nUnits, Tn;
+    int q, b, rem;     // unit, its item, its index inside the item
+    int i0, j0;        // first output row and column of the unit
+    int L, L2, L4;     // clamped length, ceil(L / 2), ceil(L2 / 2)
+
+    __device__ __forceinline__ void load_len() {
+        L = static_cast<int>(clamp_len(lengths, b, Tn));
+        L2 = (L + 1) / 2;
+        L4 = (L2 + 1) / 2;
+    }
+    __device__ __forceinline__ void place() {
+        const int ip = nJB == 1 ? rem : rem / nJB;
+        i0 = ip * kRO;
+        j0 = (rem - ip * nJB) * kJO;
+    }
+    __device__ __forceinline__ void init(int q0) {
+        q = q0;
+        b = q0 / per_item;
+        rem = q0 - b * per_item;
+        if (q < nUnits) {
+            load_len();
+            place();
+        }
+    }
+    __device__ __forceinline__ void next() {
+        q += qs;
+        if (q >= nUnits) return;
+        rem += qs;
+        bool new_item = false;
+        while (rem >= per_item) {
+            rem -= per_item;
+            ++b;
+            new_item = true;
+        }
+        if (new_item) load_len();
+        place();
+    }
+    __device__ __forceinline__ bool done() const { return q >= nUnits; }
+    // some output row of the unit is unmasked (otherwise it only stores zeros)
+    __device__ __forceinline__ bool active() const { return i0 < L4; }
+    __device__ __forceinline__ void next_active() {
+        do next();
+        while (!done() && !active());
+    }
+};
+
+// ReLU of two accumulator values as a pair.  The doubled form x + |x| = 2 ReLU(x) runs on the
+// FMA pipe instead of the (half-rate) ALU pipe; its weights are halved, so products are equal.
+__device__ __forceinline__ float2 relu_pair(float a, float b) { return make_float2(fmaxf(a, 0.f), fmaxf(b, 0.f)); }
+__device__ __forceinline__ float2 relu2x_pair(float a, float b) { return make_float2(a + fabsf(a), b + fabsf(b)); }
+
+}  // namespace
+
+template <typename TO, int CTG>
+__global__ void __launch_bounds__(kThreads, 1)
+dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ w0, const float *__restrict__ b0,
+                       const float *__restrict__ w1, const float *__restrict__ b1,
+                       const int32_t *__restrict__ lengths, int32_t *__restrict__ out_lengths,
+                       const __grid_constant__ CUtensorMap out_map, int B, int Tn, int F, int C, int T2, int F2,
+                       int Pt, int nIP, int nJB, int nG) {
+    using Lay = TcLayout<TO, CTG>;
+    extern __shared__ unsigned char smem_raw[];
+    // 1024-byte aligned base (the swizzled operand tiles need it), kept as a shared pointer
+    unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    unsigned char *tileA = smem + Lay::a_off;
+    unsigned char *tileB = smem + Lay::b_off;
+    float *mel_s = reinterpret_cast<float *>(smem + Lay::mel_off);
+    TO *stage = reinterpret_cast<TO *>(smem + Lay::st_off);
+    float *wtab = reinterpret_cast<float *>(smem + Lay::wt_off);  // [CTG][10][128]: w1 taps, b1
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::bar_off);
+    uint64_t *patch_full = bars, *patch_empty = bars + 2, *acc_full = bars + 4, *acc_empty = bars + 6,
+             *mma_done = bars + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int g = blockIdx.x % nG;                 // channel group of this block
+    const int q0 = blockIdx.x / nG;
+    constexpr int kStElems = kRO * kJO * 128;
+    UnitWalk u;
+    u.lengths = lengths;
+    u.qs = gridDim.x / nG;
+    u.per_item = nIP * nJB;
+    u.nJB = nJB;
+    u.nUnits = B * nIP * nJB;
+    u.Tn = Tn;
+    u.init(q0);
+
+    // ------------------------------------------------------------ set-up
+    if (threadIdx.x == 0) {
+        mbar_init(&patch_full[0], kPatchThreads);
+        mbar_init(&patch_full[1], kPatchThreads);
+        mbar_init(&patch_empty[0], 1);
+        mbar_init(&patch_empty[1], 1);
+        mbar_init(&acc_full[0], 1);
+        mbar_init(&acc_full[1], 1);
+        mbar_init(&acc_empty[0], kEpiWarps);
+        mbar_init(&acc_empty[1], kEpiWarps);
+        mbar_init(mma_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    if (warp >= kEpiWarps && warp < kMmaWarp) {
+        // A operand: split conv0 weights and bias of this block's channel tiles
+        const int pt = threadIdx.x - kEpiThreads;
+        for (int r = pt; r < CTG * 128; r += kPatchThreads) {
+            const int c = (g * CTG + r / 128) * 128 + r % 128;
+            float w[32];
+#pragma unroll
+            for (int t = 0; t < 9; ++t) {
+                const float x = c < C ? __ldg(w0 + t * C + c) : 0.f;
+                const float hi = tf32_hi(x);
+                w[t] = hi;
+                w[9 + t] = x - hi;
+                w[18 + t] = hi;
+            }
+            const float bx = c < C ? __ldg(b0 + c) : 0.f;
+            w[27] = tf32_hi(bx);
+            w[28] = bx - w[27];
+            w[29] = w[30] = w[31] = 0.f;
+            store_k_row(tileA + (r / 128) * kTileA, r % 128, w);
+        }
+        fence_async_smem();
+    }
+    if (warp < kEpiWarps) {
+        TO *z = stage + 2 * kStElems;  // the zero tile stored for fully masked units
+        for (int e = threadIdx.x; e < kStElems; e += kEpiThreads) stage_out<TO>(z + e, 0.f);
+        fence_async_smem();
+        for (int e = threadIdx.x; e < CTG * 10 * 128; e += kEpiThreads) {  // conv_dw1 weights and bias
+            const int ct = e / 1280, t = (e / 128) % 10, c = (g * CTG + ct) * 128 + e % 128;
+            wtab[e] = c < C ? __ldg(t < 9 ? w1 + t * C + c : b1 + c) : 0.f;
+        }
+        if (blockIdx.x == 0 && out_lengths != nullptr)
+            for (int q = threadIdx.x; q < B; q += kEpiThreads) {
+                const int Lq = static_cast<int>(clamp_len(lengths, q, Tn));
+                out_lengths[q] = ((Lq + 1) / 2 + 1) / 2;
+            }
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp < kEpiWarps) {
+        // ------------------------------------------------------------ epilogue
+        const int qw = warp & 3, half = warp >> 2;
+        const int m = qw * 32 + lane;                     // channel within the tile = TMEM lane
+        const uint32_t tlane = tmem_base + (static_cast<uint32_t>(qw * 32) << 16);
+        int job = 0;
+        bool ok = true;
+        for (; !u.done() && ok; u.next()) {
+            for (int ct = 0; ct < CTG; ++ct) {
+                const int c0 = (g * CTG + ct) * 128;
+                if (!u.active()) {  // every row masked: store the zero tile
+                    if (threadIdx.x == 0 && c0 < C)
+                        tma_store_4d(&out_map, stage + 2 * kStElems, c0, u.j0, u.i0, u.b);
+                    continue;
+                }
+                // conv_dw1 taps as pairs; odd h columns arrive doubled (x + |x|), so W[p][1] is halved
+                float2 W[3][3], bias;
+                {
+                    const float *wt = wtab + ct * 1280 + m;
+#pragma unroll
+                    for (int t = 0; t < 9; ++t) {
+                        const float x = wt[t * 128] * (t % 3 == 1 ? 0.5f : 1.f);
+                        W[t / 3][t % 3] = make_float2(x, x);
+                    }
+                    bias = make_float2(wt[9 * 128], wt[9 * 128]);
+                }
+                const int buf = job & 1;
+                ok = named_bar_and(kBarEpi, kEpiThreads, mbar_wait(&acc_full[buf], (job >> 1) & 1));
+                if (!ok) break;
+                tc_fence_after();
+                const bool row1 = u.i0 + 1 < u.L4;        // the second output row is unmasked
+                TO *st = stage + (job & 1) * kStElems;
+                const uint32_t tacc = tlane + buf * kTmemBuf;
+                // P[k][p]: h rows (p, p+2) of h column cc0 + k; P[0] carries over between chunks
+                float2 P[2 * kChunk + 1][3];
+                {
+                    float v[5];
+                    tmem_ld_column(tacc, 2 * kHalfCols * half, v);
+                    P[0][0] = relu_pair(v[0], v[2]);
+                    P[0][1] = relu_pair(v[1], v[3]);
+                    P[0][2] = relu_pair(v[2], v[4]);
+                }
+#pragma unroll 1
+                for (int ch = 0; ch < kHalfCols / kChunk; ++ch) {
+                    const int jl0 = half * kHalfCols + ch * kChunk;   // first output column (unit-local)
+                    float v[50];
+                    tmem_ld_chunk(tacc, jl0 / kChunk, v);           // h columns 2 jl0 + 1 .. 2 jl0 + 10
+#pragma unroll
+                    for (int k = 1; k <= 2 * kChunk; ++k) {
+                        const float *x = v + (k - 1) * kHR;
+                        if (k & 1) {  // odd h column: doubled ReLU on the FMA pipe
+                            P[k][0] = relu2x_pair(x[0], x[2]);
+                            P[k][1] = relu2x_pair(x[1], x[3]);
+                            P[k][2] = relu2x_pair(x[2], x[4]);
+                        } else {
+                            P[k][0] = relu_pair(x[0], x[2]);
+                            P[k][1] = relu_pair(x[1], x[3]);
+                            P[k][2] = relu_pair(x[2], x[4]);
+                        }
+                    }
+                    float2 acc[kChunk];
+#pragma unroll
+                    for (int jj = 0; jj < kChunk; ++jj) acc[jj] = bias;
+#pragma unroll
+                    for (int q = 0; q < 3; ++q)
+#pragma unroll
+                        for (int p = 0; p < 3; ++p)
+#pragma unroll
+                            for (int jj = 0; jj < kChunk; ++jj) acc[jj] = ffma2(P[2 * jj + q][p], W[p][q], acc[jj]);
+#pragma unroll
+                    for (int jj = 0; jj < kChunk; ++jj) {
+                        stage_out<TO>(st + (jl0 + jj) * 128 + m, acc[jj].x);
+                        stage_out<TO>(st + (kJO + jl0 + jj) * 128 + m, row1 ? acc[jj].y : 0.f);
+                    }
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) P[0][p] = P[2 * kChunk][p];
+                }
+                // accumulator buffer free for the next MMA
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                // staged tile complete -> one bulk store
+                fence_async_smem();
+                if (threadIdx.x == 0) bulk_wait_read_all();  // the store issued two jobs ago has read its buffer
+                named_bar(kBarEpi, kEpiThreads);
+                if (threadIdx.x == 0 && c0 < C) tma_store_4d(&out_map, st, c0, u.j0, u.i0, u.b);
+                ++job;
+            }
+        }
+        if (threadIdx.x == 0) bulk_wait_all();
+    } else if (warp < kMmaWarp) {
+        // ------------------------------------------------------------ patch builders
+        const int pt = threadIdx.x - kEpiThreads;
+        // this thread's mel window elements (row << 8 | column, or -1) and patch rows: the same
+        // for every unit
+        int mel_rs[kMelLoads];
+#pragma unroll
+        for (int k = 0; k < kMelLoads; ++k) {
+            const int e = pt + k * kPatchThreads;
+            mel_rs[k] = e < kMelElems ? ((e / kMC) << 8) | (e % kMC) : -1;
+        }
+        constexpr int kRowsPer = (kN + kPatchThreads - 1) / kPatchThreads;
+        int row_cc[kRowsPer], row_rr[kRowsPer];
+#pragma unroll
+        for (int i = 0; i < kRowsPer; ++i) {  // the h pixel whose accumulator column is n (inverse of acc_col)
+            const int n = pt + i * kPatchThreads;
+            if (n < 192) {
+                const int v = n % 48;
+                row_cc[i] = 10 * (n / 48) + 1 + v / kHR;
+                row_rr[i] = v % kHR;
+            } else if (n < 200) {
+                const int v = 48 + (n - 192) % 2;
+                row_cc[i] = 10 * ((n - 192) / 2) + 1 + v / kHR;
+                row_rr[i] = v % kHR;
+            } else {
+                row_cc[i] = 0;
+                row_rr[i] = n - 200;
+            }
+        }
+        float mv[kMelLoads];
+        auto load_mel = [&](const UnitWalk &w) {
+            const float *melb = mel + static_cast<int64_t>(w.b) * Tn * F;
+            const int mr0 = 4 * w.i0 - 3 * Pt, mc0 = 4 * w.j0 - 3;
+#pragma unroll
+            for (int k = 0; k < kMelLoads; ++k) {
+                const int mr = mr0 + (mel_rs[k] >> 8), mc = mc0 + (mel_rs[k] & 255);
+                float x = 0.f;
+                if (mel_rs[k] >= 0 && mr >= 0 && mr < w.L && mc >= 0 && mc < F) x = __ldg(melb + mr * F + mc);
+                mv[k] = x;
+            }
+        };
+        if (!u.done() && !u.active()) u.next_active();
+        if (!u.done()) load_mel(u);
+        bool ok = true;
+        for (int pu = 0; !u.done() && ok; ++pu) {
+            float *S = mel_s + (pu & 1) * (Lay::mel_bytes / 4);
+#pragma unroll
+            for (int k = 0; k < kMelLoads; ++k)
+                if (mel_rs[k] >= 0) S[(mel_rs[k] >> 8) * kMCP + (mel_rs[k] & 255)] = mv[k];
+            named_bar(kBarPatch, kPatchThreads);
+            UnitWalk nx = u;
+            nx.next_active();
+            if (!nx.done()) load_mel(nx);  // in flight while this unit's patches are built
+            const int stage_i = pu & 1;
+            ok = named_bar_and(kBarPatch, kPatchThreads, mbar_wait(&patch_empty[stage_i], ((pu >> 1) & 1) ^ 1));
+            if (!ok) break;
+            unsigned char *tb = tileB + stage_i * kTileB;
+#pragma unroll
+            for (int i = 0; i < kRowsPer; ++i) {
+                const int n = pt + i * kPatchThreads;
+                if (n >= kN) break;
+                const int cc = row_cc[i], rr = row_rr[i];
+                const int hr = 2 * u.i0 - Pt + rr, hc = 2 * u.j0 - 1 + cc;
+                const bool valid = n < kNUsed && hr >= 0 && hr < u.L2 && hc >= 0 && hc < F2;
+                float w[32];
+                if (valid) {
+                    const float *sp = S + (2 * rr) * kMCP + 2 * cc;
+#pragma unroll
+                    for (int p = 0; p < 3; ++p)
+#pragma unroll
+                        for (int qq = 0; qq < 3; ++qq) {
+                            const float x = sp[p * kMCP + qq];
+                            const float hi = tf32_hi(x);
+                            w[3 * p + qq] = hi;
+                            w[9 + 3 * p + qq] = hi;
+                            w[18 + 3 * p + qq] = x - hi;
+                        }
+                    w[27] = w[28] = 1.f;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 29; ++k) w[k] = 0.f;
+                }
+                w[29] = w[30] = w[31] = 0.f;
+                store_k_row(tb, n, w);
+            }
+            fence_async_smem();
+            mbar_arrive(&patch_full[stage_i]);
+            u = nx;
+        }
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t a_base = smem_addr(tileA), b_base = smem_addr(tileB);
+        int job = 0, pu = 0;
+        bool ok = true;
+        if (!u.done() && !u.active()) u.next_active();
+        for (; !u.done() && ok; u.next_active()) {
+            const int stage_i = pu & 1;
+            ok = mbar_wait(&patch_full[stage_i], (pu >> 1) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t bdesc = sw128_desc(b_base + stage_i * kTileB);
+            for (int ct = 0; ct < CTG; ++ct) {
+                const int buf = job & 1;
+                ok = mbar_wait(&acc_empty[buf], ((job >> 1) & 1) ^ 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t adesc = sw128_desc(a_base + ct * kTileA);
+                const uint32_t d = tmem_base + buf * kTmemBuf;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // K = 32 TF32 words = 4 steps of 8 (32 bytes)
+                    mma_tf32(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+                mma_commit(&acc_full[buf]);
+                ++job;
+            }
+            mma_commit(&patch_empty[stage_i]);
+            ++pu;
+        }
+        // every issued MMA has finished before tensor memory is released
+        mma_commit(mma_done);
+        mbar_wait(mma_done, 0);
+    }
+    __syncwarp();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+unsigned int subsample_tc_take_error() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, dw_device_error_flag, sizeof(v)) != cudaSuccess) return 0;
+    if (v != 0) cudaMemcpyToSymbol(dw_device_error_flag, &zero, sizeof(zero));
+    return v;
+}
+
+// Tensor map over the output [B][T4][F4][C] (dims innermost first), box 128 x kJO x kRO x 1.
+static cudaError_t make_out_map(CUtensorMap *map, void *out, bool bf16_out, int64_t B, int64_t T4, int64_t F4,
+                                int64_t C) {
+    TensorMapEncodeTiledFn enc = tensor_map_encoder();
+    if (enc == nullptr) return cudaErrorNotSupported;
+    const int64_t es = bf16_out ? 2 : 4;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(F4),
+                                static_cast<cuuint64_t>(T4), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(C * es), static_cast<cuuint64_t>(F4 * C * es),
+                                   static_cast<cuuint64_t>(T4 * F4 * C * es)};
+    const cuuint32_t box[4] = {128u, static_cast<cuuint32_t>(kJO), static_cast<cuuint32_t>(kRO), 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult r = enc(map, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                           out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+bool subsample_tc_eligible(const SubsampleArgs &a) {
+    const int64_t es = a.bf16_out ? 2 : 4;
+    auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
+    const int64_t T4 = s2(s2(a.T)), F4 = s2(s2(a.F));
+    const int64_t nIP = (T4 + kRO - 1) / kRO, nJB = (F4 + kJO - 1) / kJO;
+    return tensor_map_encoder() != nullptr && (a.C * es) % 16 == 0 &&
+           reinterpret_cast<uintptr_t>(a.out) % 16 == 0 && a.T * a.F < (1LL << 31) &&
+           9 * a.C < (1LL << 31) && a.B * nIP * nJB < (1LL << 31) && T4 > 0;
+}
+
+cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
+    auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
+    const int64_t T2 = s2(a.T), F2 = s2(a.F), T4 = s2(T2), F4 = s2(F2);
+    const int64_t nIP = (T4 + kRO - 1) / kRO, nJB = (F4 + kJO - 1) / kJO;
+    const int64_t nCT = (a.C + 127) / 128;
+    const int ctg = nCT >= 2 ? 2 : 1;
+    const int64_t nG = (nCT + ctg - 1) / ctg;
+    const int64_t units = a.B * nIP * nJB;
+    CUtensorMap map;
+    cudaError_t e = make_out_map(&map, a.out, a.bf16_out != 0, a.B, T4, F4, a.C);
+    if (e != cudaSuccess) return cudaErrorNotSupported;  // the caller takes the SIMT kernel
+    int64_t grid = (sm_count() / nG) * nG;
+    if (grid < nG) grid = nG;
+    if (grid > units * nG) grid = units * nG;
+    if (grid > kMaxGrid) return cudaErrorInvalidConfiguration;
+    const int Pt = a.causal ? 2 : 1;
+#define DW_TC_LAUNCH(TO, CTG)                                                                                  \
+    do {                                                                                                       \
+        auto kern = dw_subsample_tc_kernel<TO, CTG>;                                                           \
+        const int bytes = TcLayout<TO, CTG>::alloc;                                                            \
+        e = ensure_smem_attr(reinterpret_cast<const void *>(kern), bytes);                                    \
+        if (e != cudaSuccess) return e;                                                                        \
+        kern<<<static_cast<unsigned>(grid), kThreads, bytes, s>>>(                                             \
+            a.mel, a.w0, a.b0, a.w1, a.b1, a.lengths, a.out_lengths, map, static_cast<int>(a.B),               \
+            static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(T2),         \
+            static_cast<int>(F2), Pt, static_cast<int>(nIP), static_cast<int>(nJB), static_cast<int>(nG));     \
+    } while (0)
+    if (a.bf16_out) {
+        if (ctg == 2) DW_TC_LAUNCH(bf16, 2);
+        else DW_TC_LAUNCH(bf16, 1);
+    } else {
+        if (ctg == 2) DW_TC_LAUNCH(float, 2);
+        else DW_TC_LAUNCH(float, 1);
+    }
+#undef DW_TC_LAUNCH
+    return cudaGetLastError();
+}
+
+}  // namespace dwk

@@ -4,6 +4,7 @@ element by element, through the C ABI.
 Full size: mel [16, 3000, 80] -> out [16, 750, 20, 256] bf16, lengths uniform in
 [1500, 3000], symmetric and causal (time pad 2|0): the configuration the benchmark times.
 Small cases: T and F from 1 up (odd and even), C not a multiple of 64 (1, 3, 100, 300),
+C up to 512 (several channel tiles), F up to 200 (several 20-column blocks),
 float32 output, len 0 and len T, unaligned output (narrow store path), guard bands.
 
 Bars: bf16 output max|err| <= 2e-2 absolute; float32 output max|err| <= 1e-5 * RMS(oracle);
@@ -60,7 +61,10 @@ def test_subsampler_full_workload(causal):
 
 
 SMALL = [(1, 1, 1, 1), (2, 2, 3, 3), (2, 5, 7, 64), (3, 9, 80, 100), (2, 64, 80, 256), (2, 37, 81, 300),
-         (1, 130, 16, 128), (2, 33, 9, 1), (1, 4, 4, 2)]
+         (1, 130, 16, 128), (2, 33, 9, 1), (1, 4, 4, 2),
+         # tensor-core path: several column blocks, an odd number of channel tiles, two channel
+         # groups, a single output column
+         (2, 45, 200, 384), (1, 70, 80, 512), (2, 23, 3, 32)]
 
 
 @pytest.mark.parametrize("causal", [False, True])
