@@ -16,7 +16,14 @@
 // float32 accumulation; the dropped w_lo*m_lo term and the truncation of lo are below 2^-20
 // of each product.  This is the three-product emulation of float32 products on TF32 units.
 // The bias b0 rides along as two more K columns (b0_hi, b0_lo against a 0/1 column that is 1
-// exactly for unmasked h pixels, whose other columns are then zero too).
+// exactly for unmasked h pixels, whose other columns are then zero too).  K layout, in 16-byte
+// chunks of 4 words (patch | weights), taps t = 3 p + q:
+//   0: m_hi[0..3] | w_hi[0..3]     1: m_hi[4..7] | w_hi[4..7]
+//   2: m_hi[0..3] | w_lo[0..3]     3: m_hi[4..7] | w_lo[4..7]
+//   4: m_lo[0..3] | w_hi[0..3]     5: m_lo[4..7] | w_hi[4..7]
+//   6: m_hi[8], m_hi[8], m_lo[8], v | w_hi[8], w_lo[8], w_hi[8], b0_hi
+//   7: v, 0, 0, 0 | b0_lo, 0, 0, 0
+// so a patch row is six distinct register quads, two of them stored twice.
 //
 // Work unit: item b, output rows [i0, i0+2), output columns [j0, j0+20).  It needs h rows
 // 2 i0 - Pt + [0, 5) and h columns 2 j0 - 1 + [0, 41): N = 5 x 41 = 205 pixels (208 with
@@ -24,16 +31,20 @@
 // (at or beyond ceil(len/2)) and pixels outside the h plane get an all-zero patch, so their
 // h is exactly zero.
 //
-// Roles (416 threads, one block per SM, persistent):
-//   warps 0-7   epilogue: warp w reads TMEM lanes 32 (w % 4) + [0, 32) (its channel quarter)
-//               and output columns 10 (w / 4) + [0, 10) of the unit; results are staged in
-//               shared memory and written with one bulk tensor store per channel tile
+// Roles (448 threads, one block per SM, persistent):
+//   warps 0-7   epilogue, two groups of four: warp w reads TMEM lanes 32 (w % 4) + [0, 32)
+//               (its channel quarter); group w / 4 takes every other job (unit x channel
+//               tile); results are staged in shared memory and written with one bulk tensor
+//               store per job
 //   warps 8-11  patch builders: stage the unit's 11 x 83 mel window (frames at or beyond
 //               len read as zero), build the split patch rows in the 128-byte-swizzled
 //               K-major layout the MMA reads
-//   warp 12     allocates tensor memory; one thread issues the MMAs (4 K-steps of 8)
+//   warp 12     allocates tensor memory and lists the block's units; one thread issues the
+//               MMAs (4 K-steps of 8)
+//   warp 13     one thread issues every bulk tensor store (staged tiles, zero tiles)
 // Pipelines: 2 patch stages (builders -> MMA), 2 accumulator buffers of 256 TMEM columns
-// (MMA -> epilogue), 2 output staging buffers (epilogue -> bulk store).  Every mbarrier wait
+// (MMA -> epilogue group; released as soon as the last column is read), one output staging
+// tile per group (epilogue group -> store thread -> back).  Every mbarrier wait
 // is bounded; a wait that gives up records an error (dw_device_error) and the block drains.
 #include "dw_internal.h"
 
@@ -52,8 +63,8 @@ constexpr int kMCP = kMC + 1;                // staged mel row stride (floats)
 constexpr int kMelElems = kMR * kMC;
 constexpr int kEpiWarps = 8, kPatchWarps = 4;
 constexpr int kEpiThreads = kEpiWarps * 32, kPatchThreads = kPatchWarps * 32;
-constexpr int kMmaWarp = kEpiWarps + kPatchWarps;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kMmaWarp = kEpiWarps + kPatchWarps;  // then one warp whose lane 0 issues the bulk stores
+constexpr int kThreads = (kMmaWarp + 2) * 32;
 constexpr int kMelLoads = (kMelElems + kPatchThreads - 1) / kPatchThreads;
 constexpr int kRowBytes = 128;               // one K row: 32 TF32 words
 constexpr int kTileA = 128 * kRowBytes;
@@ -61,7 +72,10 @@ constexpr int kTileB = kN * kRowBytes;
 constexpr int kTmemCols = 512, kTmemBuf = 256;
 constexpr int kHalfCols = kJO / 2;           // output columns per epilogue warp
 constexpr int kChunk = 5;                    // output columns per tensor-memory read
-constexpr int kBarEpi = 1, kBarPatch = 2;    // named barrier ids
+constexpr int kRowsPer = (kN + kPatchThreads - 1) / kPatchThreads;  // patch rows per builder thread
+constexpr int kBarPatch = 1;                // named barrier id of the patch builders
+constexpr int kGroupThreads = 128;          // one epilogue group: 4 warps, one per lane quarter
+constexpr int kListCap = 1024;              // units per block (the list lives in shared memory)
 
 static_assert(kN <= 256 && kN % 16 == 0, "MMA N");
 static_assert(kTileB % 1024 == 0 && kTileA % 1024 == 0, "swizzle atoms are 1024-byte aligned");
@@ -76,8 +90,9 @@ struct TcLayout {
     static constexpr int st_bytes = kRO * kJO * 128 * static_cast<int>(sizeof(TO));
     static constexpr int st_off = mel_off + 2 * mel_bytes;   // staging 0, 1, then the zero tile
     static constexpr int wt_off = st_off + 3 * st_bytes;      // conv_dw1 weight table
-    static constexpr int bar_off = wt_off + CTG * 10 * 128 * 4;
-    static constexpr int bytes = bar_off + 128;
+    static constexpr int list_off = wt_off + CTG * 10 * 128 * 4;  // unit list
+    static constexpr int bar_off = list_off + kListCap * 16;
+    static constexpr int bytes = bar_off + 256;
     // room to align the base to 1024; at least 120 KiB so that one block holds an SM (and all
     // of its tensor memory)
     static constexpr int alloc = bytes + 1024 > 120 * 1024 ? bytes + 1024 : 120 * 1024;
@@ -221,67 +236,15 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
 
 // Row `row` of a K-major 128-byte-swizzled tile: 16-byte chunk k lands at chunk k ^ (row % 8).
-__device__ __forceinline__ void store_k_row(unsigned char *tile, int row, const float (&w)[32]) {
+__device__ __forceinline__ void store_k_row(unsigned char *tile, int row, const float4 (&w)[8]) {
     unsigned char *base = tile + row * kRowBytes;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-        *reinterpret_cast<float4 *>(base + ((k ^ (row & 7)) << 4)) =
-            make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<float4 *>(base + ((k ^ (row & 7)) << 4)) = w[k];
 }
 
 template <typename TO> __device__ __forceinline__ void stage_out(TO *p, float v);
 template <> __device__ __forceinline__ void stage_out<float>(float *p, float v) { *p = v; }
 template <> __device__ __forceinline__ void stage_out<bf16>(bf16 *p, float v) { *p = __float2bfloat16_rn(v); }
-
-// The units q0, q0 + qs, q0 + 2 qs, ... of one block, in order, with the item and the place
-// inside it tracked incrementally (no division per unit); the length is read once per item.
-struct UnitWalk {
-    const int32_t *lengths;
-    int qs, per_item, nJB, nUnits, Tn;
-    int q, b, rem;     // unit, its item, its index inside the item
-    int i0, j0;        // first output row and column of the unit
-    int L, L2, L4;     // clamped length, ceil(L / 2), ceil(L2 / 2)
-
-    __device__ __forceinline__ void load_len() {
-        L = static_cast<int>(clamp_len(lengths, b, Tn));
-        L2 = (L + 1) / 2;
-        L4 = (L2 + 1) / 2;
-    }
-    __device__ __forceinline__ void place() {
-        const int ip = nJB == 1 ? rem : rem / nJB;
-        i0 = ip * kRO;
-        j0 = (rem - ip * nJB) * kJO;
-    }
-    __device__ __forceinline__ void init(int q0) {
-        q = q0;
-        b = q0 / per_item;
-        rem = q0 - b * per_item;
-        if (q < nUnits) {
-            load_len();
-            place();
-        }
-    }
-    __device__ __forceinline__ void next() {
-        q += qs;
-        if (q >= nUnits) return;
-        rem += qs;
-        bool new_item = false;
-        while (rem >= per_item) {
-            rem -= per_item;
-            ++b;
-            new_item = true;
-        }
-        if (new_item) load_len();
-        place();
-    }
-    __device__ __forceinline__ bool done() const { return q >= nUnits; }
-    // some output row of the unit is unmasked (otherwise it only stores zeros)
-    __device__ __forceinline__ bool active() const { return i0 < L4; }
-    __device__ __forceinline__ void next_active() {
-        do next();
-        while (!done() && !active());
-    }
-};
 
 // ReLU of two accumulator values as a pair.  The doubled form x + |x| = 2 ReLU(x) runs on the
 // FMA pipe instead of the (half-rate) ALU pipe; its weights are halved, so products are equal.
@@ -295,45 +258,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ w0, const float *__restrict__ b0,
                        const float *__restrict__ w1, const float *__restrict__ b1,
                        const int32_t *__restrict__ lengths, int32_t *__restrict__ out_lengths,
-                       const __grid_constant__ CUtensorMap out_map, int B, int Tn, int F, int C, int T2, int F2,
-                       int Pt, int nIP, int nJB, int nG) {
+                       const __grid_constant__ CUtensorMap out_map, int B, int Tn, int F, int C, int F2, int Pt,
+                       int nIP, int nJB, int nG) {
     using Lay = TcLayout<TO, CTG>;
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte aligned base (the swizzled operand tiles need it), kept as a shared pointer
     unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     unsigned char *tileA = smem + Lay::a_off;
     unsigned char *tileB = smem + Lay::b_off;
-    float *mel_s = reinterpret_cast<float *>(smem + Lay::mel_off);
-    TO *stage = reinterpret_cast<TO *>(smem + Lay::st_off);
+    float *mel_s_tile = reinterpret_cast<float *>(smem + Lay::mel_off);
+    TO *stage = reinterpret_cast<TO *>(smem + Lay::st_off);       // group 0, group 1, zero tile
     float *wtab = reinterpret_cast<float *>(smem + Lay::wt_off);  // [CTG][10][128]: w1 taps, b1
+    int4 *ulist = reinterpret_cast<int4 *>(smem + Lay::list_off); // units {b, i0, j0, len}
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::bar_off);
     uint64_t *patch_full = bars, *patch_empty = bars + 2, *acc_full = bars + 4, *acc_empty = bars + 6,
-             *mma_done = bars + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+             *staged = bars + 8, *stage_free = bars + 10, *mma_done = bars + 12;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    int *counts = reinterpret_cast<int *>(bars + 14);             // active units, masked units
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int g = blockIdx.x % nG;                 // channel group of this block
-    const int q0 = blockIdx.x / nG;
+    const int q0 = blockIdx.x / nG, qs = gridDim.x / nG;
+    const int nUnits = B * nIP * nJB;
     constexpr int kStElems = kRO * kJO * 128;
-    UnitWalk u;
-    u.lengths = lengths;
-    u.qs = gridDim.x / nG;
-    u.per_item = nIP * nJB;
-    u.nJB = nJB;
-    u.nUnits = B * nIP * nJB;
-    u.Tn = Tn;
-    u.init(q0);
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
-        mbar_init(&patch_full[0], kPatchThreads);
-        mbar_init(&patch_full[1], kPatchThreads);
-        mbar_init(&patch_empty[0], 1);
-        mbar_init(&patch_empty[1], 1);
-        mbar_init(&acc_full[0], 1);
-        mbar_init(&acc_full[1], 1);
-        mbar_init(&acc_empty[0], kEpiWarps);
-        mbar_init(&acc_empty[1], kEpiWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&patch_full[i], kPatchThreads);
+            mbar_init(&patch_empty[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], kGroupThreads / 32);  // one arrival per warp of the group
+            mbar_init(&staged[i], kGroupThreads);
+            mbar_init(&stage_free[i], 1);
+        }
         mbar_init(mma_done, 1);
         fence_barrier_init();
     }
@@ -341,26 +299,58 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
         tc_fence_before();
+        // this block's units q0, q0 + qs, ...: the active ones from the front of the list, the
+        // fully masked ones (zeros only) from the back, each in increasing order
+        const int per_item = nIP * nJB;
+        const int mine = q0 < nUnits ? (nUnits - q0 + qs - 1) / qs : 0;
+        int nA = 0, nZ = 0;
+        for (int base = 0; base < mine; base += 32) {
+            const int k = base + lane;
+            const bool have = k < mine;
+            int4 e = make_int4(0, 0, 0, 0);
+            bool act = false;
+            if (have) {
+                const int q = q0 + k * qs;
+                const int b = q / per_item, rem = q - b * per_item, ip = rem / nJB;
+                e = make_int4(b, ip * kRO, (rem - ip * nJB) * kJO, static_cast<int>(clamp_len(lengths, b, Tn)));
+                act = e.y < ((e.w + 1) / 2 + 1) / 2;
+            }
+            const unsigned ma = __ballot_sync(0xffffffffu, have && act), mz = __ballot_sync(0xffffffffu, have && !act);
+            const unsigned below = (1u << lane) - 1u;
+            if (have && act) ulist[nA + __popc(ma & below)] = e;
+            if (have && !act) ulist[kListCap - 1 - (nZ + __popc(mz & below))] = e;
+            nA += __popc(ma);
+            nZ += __popc(mz);
+        }
+        if (lane == 0) {
+            counts[0] = nA;
+            counts[1] = nZ;
+        }
     }
     if (warp >= kEpiWarps && warp < kMmaWarp) {
-        // A operand: split conv0 weights and bias of this block's channel tiles
+        // A operand: split conv0 weights and bias of this block's channel tiles (K layout above)
         const int pt = threadIdx.x - kEpiThreads;
         for (int r = pt; r < CTG * 128; r += kPatchThreads) {
             const int c = (g * CTG + r / 128) * 128 + r % 128;
-            float w[32];
+            float hi[9], lo[9];
 #pragma unroll
             for (int t = 0; t < 9; ++t) {
                 const float x = c < C ? __ldg(w0 + t * C + c) : 0.f;
-                const float hi = tf32_hi(x);
-                w[t] = hi;
-                w[9 + t] = x - hi;
-                w[18 + t] = hi;
+                hi[t] = tf32_hi(x);
+                lo[t] = x - hi[t];
             }
             const float bx = c < C ? __ldg(b0 + c) : 0.f;
-            w[27] = tf32_hi(bx);
-            w[28] = bx - w[27];
-            w[29] = w[30] = w[31] = 0.f;
-            store_k_row(tileA + (r / 128) * kTileA, r % 128, w);
+            const float bhi = tf32_hi(bx);
+            float4 q[8];
+            q[0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            q[1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+            q[2] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+            q[3] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+            q[4] = q[0];
+            q[5] = q[1];
+            q[6] = make_float4(hi[8], lo[8], hi[8], bhi);
+            q[7] = make_float4(bx - bhi, 0.f, 0.f, 0.f);
+            store_k_row(tileA + (r / 128) * kTileA, r % 128, q);
         }
         fence_async_smem();
     }
@@ -381,109 +371,107 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const int nA = counts[0], nZ = counts[1];
 
     if (warp < kEpiWarps) {
         // ------------------------------------------------------------ epilogue
-        const int qw = warp & 3, half = warp >> 2;
+        // Two groups of four warps (one per TMEM lane quarter) take the jobs (unit x channel
+        // tile) in turn: group 0 the even ones in accumulator buffer 0, group 1 the odd ones in
+        // buffer 1.  A group's jobs all have the same channel tile, so its conv_dw1 taps stay in
+        // registers.  No named barriers: the group hands its staged tile to the store thread and
+        // gets it back through mbarriers.
+        const int grp = warp >> 2, qw = warp & 3;
         const int m = qw * 32 + lane;                     // channel within the tile = TMEM lane
-        const uint32_t tlane = tmem_base + (static_cast<uint32_t>(qw * 32) << 16);
-        int job = 0;
-        bool ok = true;
-        for (; !u.done() && ok; u.next()) {
-            for (int ct = 0; ct < CTG; ++ct) {
-                const int c0 = (g * CTG + ct) * 128;
-                if (!u.active()) {  // every row masked: store the zero tile
-                    if (threadIdx.x == 0 && c0 < C)
-                        tma_store_4d(&out_map, stage + 2 * kStElems, c0, u.j0, u.i0, u.b);
-                    continue;
-                }
-                // conv_dw1 taps as pairs; odd h columns arrive doubled (x + |x|), so W[p][1] is halved
-                float2 W[3][3], bias;
-                {
-                    const float *wt = wtab + ct * 1280 + m;
+        const int ct = CTG == 2 ? grp : 0;
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + grp * kTmemBuf;
+        TO *st = stage + grp * kStElems;
+        // conv_dw1 taps as pairs; odd h columns arrive doubled (x + |x|), so W[p][1] is halved
+        float2 W[3][3], bias;
+        {
+            const float *wt = wtab + ct * 1280 + m;
 #pragma unroll
-                    for (int t = 0; t < 9; ++t) {
-                        const float x = wt[t * 128] * (t % 3 == 1 ? 0.5f : 1.f);
-                        W[t / 3][t % 3] = make_float2(x, x);
-                    }
-                    bias = make_float2(wt[9 * 128], wt[9 * 128]);
-                }
-                const int buf = job & 1;
-                ok = named_bar_and(kBarEpi, kEpiThreads, mbar_wait(&acc_full[buf], (job >> 1) & 1));
-                if (!ok) break;
-                tc_fence_after();
-                const bool row1 = u.i0 + 1 < u.L4;        // the second output row is unmasked
-                TO *st = stage + (job & 1) * kStElems;
-                const uint32_t tacc = tlane + buf * kTmemBuf;
-                // P[k][p]: h rows (p, p+2) of h column cc0 + k; P[0] carries over between chunks
-                float2 P[2 * kChunk + 1][3];
-                {
-                    float v[5];
-                    tmem_ld_column(tacc, 2 * kHalfCols * half, v);
-                    P[0][0] = relu_pair(v[0], v[2]);
-                    P[0][1] = relu_pair(v[1], v[3]);
-                    P[0][2] = relu_pair(v[2], v[4]);
-                }
-#pragma unroll 1
-                for (int ch = 0; ch < kHalfCols / kChunk; ++ch) {
-                    const int jl0 = half * kHalfCols + ch * kChunk;   // first output column (unit-local)
-                    float v[50];
-                    tmem_ld_chunk(tacc, jl0 / kChunk, v);           // h columns 2 jl0 + 1 .. 2 jl0 + 10
-#pragma unroll
-                    for (int k = 1; k <= 2 * kChunk; ++k) {
-                        const float *x = v + (k - 1) * kHR;
-                        if (k & 1) {  // odd h column: doubled ReLU on the FMA pipe
-                            P[k][0] = relu2x_pair(x[0], x[2]);
-                            P[k][1] = relu2x_pair(x[1], x[3]);
-                            P[k][2] = relu2x_pair(x[2], x[4]);
-                        } else {
-                            P[k][0] = relu_pair(x[0], x[2]);
-                            P[k][1] = relu_pair(x[1], x[3]);
-                            P[k][2] = relu_pair(x[2], x[4]);
-                        }
-                    }
-                    float2 acc[kChunk];
-#pragma unroll
-                    for (int jj = 0; jj < kChunk; ++jj) acc[jj] = bias;
-#pragma unroll
-                    for (int q = 0; q < 3; ++q)
-#pragma unroll
-                        for (int p = 0; p < 3; ++p)
-#pragma unroll
-                            for (int jj = 0; jj < kChunk; ++jj) acc[jj] = ffma2(P[2 * jj + q][p], W[p][q], acc[jj]);
-#pragma unroll
-                    for (int jj = 0; jj < kChunk; ++jj) {
-                        stage_out<TO>(st + (jl0 + jj) * 128 + m, acc[jj].x);
-                        stage_out<TO>(st + (kJO + jl0 + jj) * 128 + m, row1 ? acc[jj].y : 0.f);
-                    }
-#pragma unroll
-                    for (int p = 0; p < 3; ++p) P[0][p] = P[2 * kChunk][p];
-                }
-                // accumulator buffer free for the next MMA
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
-                // staged tile complete -> one bulk store
-                fence_async_smem();
-                if (threadIdx.x == 0) bulk_wait_read_all();  // the store issued two jobs ago has read its buffer
-                named_bar(kBarEpi, kEpiThreads);
-                if (threadIdx.x == 0 && c0 < C) tma_store_4d(&out_map, st, c0, u.j0, u.i0, u.b);
-                ++job;
+            for (int t = 0; t < 9; ++t) {
+                const float x = wt[t * 128] * (t % 3 == 1 ? 0.5f : 1.f);
+                W[t / 3][t % 3] = make_float2(x, x);
             }
+            bias = make_float2(wt[9 * 128], wt[9 * 128]);
         }
-        if (threadIdx.x == 0) bulk_wait_all();
+        const int first = CTG == 1 ? grp : 0, step = CTG == 1 ? 2 : 1;
+        bool ok = true;
+        for (int idx = first, n = 0; idx < nA && ok; idx += step, ++n) {
+            const int4 e = ulist[idx];
+            const bool row1 = e.y + 1 < ((e.w + 1) / 2 + 1) / 2;  // the second output row is unmasked
+            ok = mbar_wait(&acc_full[grp], n & 1);
+            if (!ok) break;
+            tc_fence_after();
+            // E[i][p]: h rows (p, p+2) of the even h column 2 jl0 + 2i; E[0] carries over
+            float2 E[kChunk + 1][3];
+            {
+                float v[5];
+                tmem_ld_column(tacc, 0, v);
+                E[0][0] = relu_pair(v[0], v[2]);
+                E[0][1] = relu_pair(v[1], v[3]);
+                E[0][2] = relu_pair(v[2], v[4]);
+            }
+#pragma unroll 1
+            for (int ch = 0; ch < kJO / kChunk && ok; ++ch) {
+                const int jl0 = ch * kChunk;                     // first output column (unit-local)
+                float v[50];
+                tmem_ld_chunk(tacc, ch, v);                      // h columns 2 jl0 + 1 .. 2 jl0 + 10
+                if (ch == kJO / kChunk - 1) {  // accumulator read out: the next MMA may start
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[grp]);
+                }
+                if (ch == 0 && n > 0) ok = mbar_wait(&stage_free[grp], (n - 1) & 1);  // previous store has read it
+#pragma unroll
+                for (int i = 1; i <= kChunk; ++i) {
+                    const float *x = v + (2 * i - 1) * kHR;
+                    E[i][0] = relu_pair(x[0], x[2]);
+                    E[i][1] = relu_pair(x[1], x[3]);
+                    E[i][2] = relu_pair(x[2], x[4]);
+                }
+                float2 acc[kChunk];
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                    for (int jj = 0; jj < kChunk; ++jj)
+                        acc[jj] = ffma2(E[jj][p], W[p][0], p == 0 ? bias : acc[jj]);
+#pragma unroll
+                for (int jj = 0; jj < kChunk; ++jj) {  // odd h column 2 jj + 1: doubled ReLU on the FMA pipe
+                    const float *x = v + (2 * jj) * kHR;
+                    acc[jj] = ffma2(relu2x_pair(x[0], x[2]), W[0][1], acc[jj]);
+                    acc[jj] = ffma2(relu2x_pair(x[1], x[3]), W[1][1], acc[jj]);
+                    acc[jj] = ffma2(relu2x_pair(x[2], x[4]), W[2][1], acc[jj]);
+                }
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                    for (int jj = 0; jj < kChunk; ++jj) acc[jj] = ffma2(E[jj + 1][p], W[p][2], acc[jj]);
+#pragma unroll
+                for (int jj = 0; jj < kChunk; ++jj) {
+                    stage_out<TO>(st + (jl0 + jj) * 128 + m, acc[jj].x);
+                    stage_out<TO>(st + (kJO + jl0 + jj) * 128 + m, row1 ? acc[jj].y : 0.f);
+                }
+#pragma unroll
+                for (int p = 0; p < 3; ++p) E[0][p] = E[kChunk][p];
+            }
+            // staged tile complete: hand it to the store thread
+            fence_async_smem();
+            mbar_arrive(&staged[grp]);
+        }
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ patch builders
         const int pt = threadIdx.x - kEpiThreads;
-        // this thread's mel window elements (row << 8 | column, or -1) and patch rows: the same
-        // for every unit
+        // This thread's mel window elements and patch rows are the same for every unit:
+        // element k sits at window row rs >> 8, column rs & 255 (rs = -1 past the window); rows
+        // n = pt + i * kPatchThreads all share n % 8 (one swizzle pattern).
         int mel_rs[kMelLoads];
 #pragma unroll
         for (int k = 0; k < kMelLoads; ++k) {
             const int e = pt + k * kPatchThreads;
             mel_rs[k] = e < kMelElems ? ((e / kMC) << 8) | (e % kMC) : -1;
         }
-        constexpr int kRowsPer = (kN + kPatchThreads - 1) / kPatchThreads;
         int row_cc[kRowsPer], row_rr[kRowsPer];
 #pragma unroll
         for (int i = 0; i < kRowsPer; ++i) {  // the h pixel whose accumulator column is n (inverse of acc_col)
@@ -502,31 +490,32 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
             }
         }
         float mv[kMelLoads];
-        auto load_mel = [&](const UnitWalk &w) {
-            const float *melb = mel + static_cast<int64_t>(w.b) * Tn * F;
-            const int mr0 = 4 * w.i0 - 3 * Pt, mc0 = 4 * w.j0 - 3;
+        auto load_mel = [&](const int4 &e) {  // e = {b, i0, j0, len}
+            const int mr0 = 4 * e.y - 3 * Pt, mc0 = 4 * e.z - 3;
+            const float *base = mel + static_cast<int64_t>(e.x) * Tn * F;
+            const bool rows_in = mr0 >= 0 && mr0 + kMR <= e.w;  // every window row is a valid frame
 #pragma unroll
             for (int k = 0; k < kMelLoads; ++k) {
                 const int mr = mr0 + (mel_rs[k] >> 8), mc = mc0 + (mel_rs[k] & 255);
+                const bool in = mel_rs[k] >= 0 && (rows_in || (mr >= 0 && mr < e.w)) && mc >= 0 && mc < F;
                 float x = 0.f;
-                if (mel_rs[k] >= 0 && mr >= 0 && mr < w.L && mc >= 0 && mc < F) x = __ldg(melb + mr * F + mc);
+                if (in) x = __ldg(base + mr * F + mc);
                 mv[k] = x;
             }
         };
-        if (!u.done() && !u.active()) u.next_active();
-        if (!u.done()) load_mel(u);
+        if (nA > 0) load_mel(ulist[0]);
         bool ok = true;
-        for (int pu = 0; !u.done() && ok; ++pu) {
-            float *S = mel_s + (pu & 1) * (Lay::mel_bytes / 4);
+        for (int idx = 0; idx < nA && ok; ++idx) {
+            const int4 e = ulist[idx];
+            const int L2 = (e.w + 1) / 2;
+            float *S = mel_s_tile + (idx & 1) * (Lay::mel_bytes / 4);
 #pragma unroll
             for (int k = 0; k < kMelLoads; ++k)
                 if (mel_rs[k] >= 0) S[(mel_rs[k] >> 8) * kMCP + (mel_rs[k] & 255)] = mv[k];
             named_bar(kBarPatch, kPatchThreads);
-            UnitWalk nx = u;
-            nx.next_active();
-            if (!nx.done()) load_mel(nx);  // in flight while this unit's patches are built
-            const int stage_i = pu & 1;
-            ok = named_bar_and(kBarPatch, kPatchThreads, mbar_wait(&patch_empty[stage_i], ((pu >> 1) & 1) ^ 1));
+            if (idx + 1 < nA) load_mel(ulist[idx + 1]);  // in flight while this unit's patches are built
+            const int stage_i = idx & 1;
+            ok = named_bar_and(kBarPatch, kPatchThreads, mbar_wait(&patch_empty[stage_i], ((idx >> 1) & 1) ^ 1));
             if (!ok) break;
             unsigned char *tb = tileB + stage_i * kTileB;
 #pragma unroll
@@ -534,64 +523,90 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
                 const int n = pt + i * kPatchThreads;
                 if (n >= kN) break;
                 const int cc = row_cc[i], rr = row_rr[i];
-                const int hr = 2 * u.i0 - Pt + rr, hc = 2 * u.j0 - 1 + cc;
-                const bool valid = n < kNUsed && hr >= 0 && hr < u.L2 && hc >= 0 && hc < F2;
-                float w[32];
+                const int hr = 2 * e.y - Pt + rr, hc = 2 * e.z - 1 + cc;
+                const bool valid = n < kNUsed && hr >= 0 && hr < L2 && hc >= 0 && hc < F2;
+                float4 q[8];
                 if (valid) {
                     const float *sp = S + (2 * rr) * kMCP + 2 * cc;
+                    float hi[9], lo[9];
 #pragma unroll
-                    for (int p = 0; p < 3; ++p)
-#pragma unroll
-                        for (int qq = 0; qq < 3; ++qq) {
-                            const float x = sp[p * kMCP + qq];
-                            const float hi = tf32_hi(x);
-                            w[3 * p + qq] = hi;
-                            w[9 + 3 * p + qq] = hi;
-                            w[18 + 3 * p + qq] = x - hi;
-                        }
-                    w[27] = w[28] = 1.f;
+                    for (int t = 0; t < 9; ++t) {
+                        const float x = sp[(t / 3) * kMCP + t % 3];
+                        hi[t] = tf32_hi(x);
+                        lo[t] = x - hi[t];
+                    }
+                    q[0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+                    q[1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+                    q[2] = q[0];
+                    q[3] = q[1];
+                    q[4] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+                    q[5] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+                    q[6] = make_float4(hi[8], hi[8], lo[8], 1.f);
+                    q[7] = make_float4(1.f, 0.f, 0.f, 0.f);
                 } else {
 #pragma unroll
-                    for (int k = 0; k < 29; ++k) w[k] = 0.f;
+                    for (int k = 0; k < 8; ++k) q[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                w[29] = w[30] = w[31] = 0.f;
-                store_k_row(tb, n, w);
+                store_k_row(tb, n, q);
             }
             fence_async_smem();
             mbar_arrive(&patch_full[stage_i]);
-            u = nx;
         }
-    } else if (lane == 0) {
-        // ------------------------------------------------------------ MMA issuer
-        const uint32_t a_base = smem_addr(tileA), b_base = smem_addr(tileB);
-        int job = 0, pu = 0;
-        bool ok = true;
-        if (!u.done() && !u.active()) u.next_active();
-        for (; !u.done() && ok; u.next_active()) {
-            const int stage_i = pu & 1;
-            ok = mbar_wait(&patch_full[stage_i], (pu >> 1) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            const uint64_t bdesc = sw128_desc(b_base + stage_i * kTileB);
-            for (int ct = 0; ct < CTG; ++ct) {
-                const int buf = job & 1;
-                ok = mbar_wait(&acc_empty[buf], ((job >> 1) & 1) ^ 1);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ MMA issuer
+            const uint32_t a_base = smem_addr(tileA), b_base = smem_addr(tileB);
+            bool ok = true;
+            for (int idx = 0; idx < nA && ok; ++idx) {
+                const int stage_i = idx & 1;
+                ok = mbar_wait(&patch_full[stage_i], (idx >> 1) & 1);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t adesc = sw128_desc(a_base + ct * kTileA);
-                const uint32_t d = tmem_base + buf * kTmemBuf;
+                const uint64_t bdesc = sw128_desc(b_base + stage_i * kTileB);
+                for (int ct = 0; ct < CTG; ++ct) {
+                    const int job = idx * CTG + ct, buf = job & 1;
+                    ok = mbar_wait(&acc_empty[buf], ((job >> 1) & 1) ^ 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t adesc = sw128_desc(a_base + ct * kTileA);
+                    const uint32_t d = tmem_base + buf * kTmemBuf;
 #pragma unroll
-                for (int k = 0; k < 4; ++k)  // K = 32 TF32 words = 4 steps of 8 (32 bytes)
-                    mma_tf32(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
-                mma_commit(&acc_full[buf]);
-                ++job;
+                    for (int k = 0; k < 4; ++k)  // K = 32 TF32 words = 4 steps of 8 (32 bytes)
+                        mma_tf32(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+                    mma_commit(&acc_full[buf]);
+                }
+                mma_commit(&patch_empty[stage_i]);
             }
-            mma_commit(&patch_empty[stage_i]);
-            ++pu;
+            // every issued MMA has finished before tensor memory is released
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0);
         }
-        // every issued MMA has finished before tensor memory is released
-        mma_commit(mma_done);
-        mbar_wait(mma_done, 0);
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ bulk stores
+        // Staged tiles of the two epilogue groups in job order, and the zero tile for every
+        // fully masked unit (one masked unit between staged jobs, so neither kind waits long).
+        const TO *zero = stage + 2 * kStElems;
+        int z = 0;
+        auto store_zero_unit = [&]() {
+            const int4 e = ulist[kListCap - 1 - z];
+            for (int ct = 0; ct < CTG; ++ct) {
+                const int c0 = (g * CTG + ct) * 128;
+                if (c0 < C) tma_store_4d(&out_map, zero, c0, e.z, e.y, e.x);
+            }
+            ++z;
+        };
+        for (int job = 0; job < nA * CTG; ++job) {
+            if (z < nZ) store_zero_unit();
+            const int grp = job & 1;
+            if (!mbar_wait(&staged[grp], (job >> 1) & 1)) break;
+            const int4 e = ulist[job / CTG];
+            const int c0 = (g * CTG + job % CTG) * 128;
+            if (c0 < C) tma_store_4d(&out_map, stage + grp * kStElems, c0, e.z, e.y, e.x);
+            bulk_wait_read_all();           // the tile has been read: the group may overwrite it
+            mbar_arrive(&stage_free[grp]);
+        }
+        while (z < nZ) store_zero_unit();
+        bulk_wait_all();
     }
     __syncwarp();
     __syncthreads();
@@ -638,7 +653,7 @@ bool subsample_tc_eligible(const SubsampleArgs &a) {
 
 cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
     auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
-    const int64_t T2 = s2(a.T), F2 = s2(a.F), T4 = s2(T2), F4 = s2(F2);
+    const int64_t F2 = s2(a.F), T4 = s2(s2(a.T)), F4 = s2(F2);
     const int64_t nIP = (T4 + kRO - 1) / kRO, nJB = (F4 + kJO - 1) / kJO;
     const int64_t nCT = (a.C + 127) / 128;
     const int ctg = nCT >= 2 ? 2 : 1;
@@ -651,6 +666,8 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
     if (grid < nG) grid = nG;
     if (grid > units * nG) grid = units * nG;
     if (grid > kMaxGrid) return cudaErrorInvalidConfiguration;
+    // every block keeps its unit list in shared memory; larger problems take the SIMT kernel
+    if ((units + grid / nG - 1) / (grid / nG) > kListCap) return cudaErrorNotSupported;
     const int Pt = a.causal ? 2 : 1;
 #define DW_TC_LAUNCH(TO, CTG)                                                                                  \
     do {                                                                                                       \
@@ -660,8 +677,8 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
         if (e != cudaSuccess) return e;                                                                        \
         kern<<<static_cast<unsigned>(grid), kThreads, bytes, s>>>(                                             \
             a.mel, a.w0, a.b0, a.w1, a.b1, a.lengths, a.out_lengths, map, static_cast<int>(a.B),               \
-            static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(T2),         \
-            static_cast<int>(F2), Pt, static_cast<int>(nIP), static_cast<int>(nJB), static_cast<int>(nG));     \
+            static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(F2), Pt,     \
+            static_cast<int>(nIP), static_cast<int>(nJB), static_cast<int>(nG));                               \
     } while (0)
     if (a.bf16_out) {
         if (ctg == 2) DW_TC_LAUNCH(bf16, 2);
