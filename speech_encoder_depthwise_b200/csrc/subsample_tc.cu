@@ -43,8 +43,8 @@
 //               MMAs (4 K-steps of 8)
 //   warp 13     one thread issues every bulk tensor store (staged tiles, zero tiles)
 // Pipelines: 2 patch stages (builders -> MMA), 2 accumulator buffers of 256 TMEM columns
-// (MMA -> epilogue group; released as soon as the last column is read), one output staging
-// tile per group (epilogue group -> store thread -> back).  Every mbarrier wait
+// (MMA -> epilogue group; released as soon as the last column is read), two output staging
+// tiles per group (epilogue group -> store thread -> back).  Every mbarrier wait
 // is bounded; a wait that gives up records an error (dw_device_error) and the block drains.
 #include "dw_internal.h"
 
@@ -88,8 +88,8 @@ struct TcLayout {
     static constexpr int mel_bytes = (kMR * kMCP * 4 + 127) / 128 * 128;
     static constexpr int mel_off = b_off + 2 * kTileB;
     static constexpr int st_bytes = kRO * kJO * 128 * static_cast<int>(sizeof(TO));
-    static constexpr int st_off = mel_off + 2 * mel_bytes;   // staging 0, 1, then the zero tile
-    static constexpr int wt_off = st_off + 3 * st_bytes;      // conv_dw1 weight table
+    static constexpr int st_off = mel_off + 2 * mel_bytes;   // 2 staging tiles per group, zero tile
+    static constexpr int wt_off = st_off + 5 * st_bytes;      // conv_dw1 weight table
     static constexpr int list_off = wt_off + CTG * 10 * 128 * 4;  // unit list
     static constexpr int bar_off = list_off + kListCap * 16;
     static constexpr int bytes = bar_off + 256;
@@ -220,16 +220,20 @@ __device__ __forceinline__ void tmem_ld_column(uint32_t tacc, int cc, float (&v)
     for (int i = 0; i < 5; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Bulk tensor store of one staged box (coordinates innermost first: channel, column, row, item).
+// Bulk tensor store of one staged box (coordinates innermost first: channel, column, row, item);
+// the caller commits the bulk group.
 __device__ __forceinline__ void tma_store_4d(const void *tmap, const void *src, int c, int j, int i, int b) {
     asm volatile(
         "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
             reinterpret_cast<uint64_t>(tmap)),
         "r"(smem_addr(src)), "r"(c), "r"(j), "r"(i), "r"(b)
         : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups of this thread still read shared memory.
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- operand rows
@@ -267,14 +271,14 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
     unsigned char *tileA = smem + Lay::a_off;
     unsigned char *tileB = smem + Lay::b_off;
     float *mel_s_tile = reinterpret_cast<float *>(smem + Lay::mel_off);
-    TO *stage = reinterpret_cast<TO *>(smem + Lay::st_off);       // group 0, group 1, zero tile
+    TO *stage = reinterpret_cast<TO *>(smem + Lay::st_off);       // [group][slot] tiles, zero tile
     float *wtab = reinterpret_cast<float *>(smem + Lay::wt_off);  // [CTG][10][128]: w1 taps, b1
     int4 *ulist = reinterpret_cast<int4 *>(smem + Lay::list_off); // units {b, i0, j0, len}
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::bar_off);
     uint64_t *patch_full = bars, *patch_empty = bars + 2, *acc_full = bars + 4, *acc_empty = bars + 6,
-             *staged = bars + 8, *stage_free = bars + 10, *mma_done = bars + 12;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
-    int *counts = reinterpret_cast<int *>(bars + 14);             // active units, masked units
+             *staged = bars + 8, *stage_free = bars + 10 /* [group][slot] */, *mma_done = bars + 14;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
+    int *counts = reinterpret_cast<int *>(bars + 16);             // active units, masked units
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int g = blockIdx.x % nG;                 // channel group of this block
@@ -290,7 +294,8 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], kGroupThreads / 32);  // one arrival per warp of the group
             mbar_init(&staged[i], kGroupThreads);
-            mbar_init(&stage_free[i], 1);
+            mbar_init(&stage_free[2 * i], 1);
+            mbar_init(&stage_free[2 * i + 1], 1);
         }
         mbar_init(mma_done, 1);
         fence_barrier_init();
@@ -355,7 +360,7 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         fence_async_smem();
     }
     if (warp < kEpiWarps) {
-        TO *z = stage + 2 * kStElems;  // the zero tile stored for fully masked units
+        TO *z = stage + 4 * kStElems;  // the zero tile stored for fully masked units
         for (int e = threadIdx.x; e < kStElems; e += kEpiThreads) stage_out<TO>(z + e, 0.f);
         fence_async_smem();
         for (int e = threadIdx.x; e < CTG * 10 * 128; e += kEpiThreads) {  // conv_dw1 weights and bias
@@ -384,7 +389,6 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         const int m = qw * 32 + lane;                     // channel within the tile = TMEM lane
         const int ct = CTG == 2 ? grp : 0;
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + grp * kTmemBuf;
-        TO *st = stage + grp * kStElems;
         // conv_dw1 taps as pairs; odd h columns arrive doubled (x + |x|), so W[p][1] is halved
         float2 W[3][3], bias;
         {
@@ -404,6 +408,7 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
             ok = mbar_wait(&acc_full[grp], n & 1);
             if (!ok) break;
             tc_fence_after();
+            TO *st = stage + (2 * grp + (n & 1)) * kStElems;
             // E[i][p]: h rows (p, p+2) of the even h column 2 jl0 + 2i; E[0] carries over
             float2 E[kChunk + 1][3];
             {
@@ -423,7 +428,8 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_empty[grp]);
                 }
-                if (ch == 0 && n > 0) ok = mbar_wait(&stage_free[grp], (n - 1) & 1);  // previous store has read it
+                // this slot's previous tile (two jobs back) has been read by its store
+                if (ch == 0 && n > 1) ok = mbar_wait(&stage_free[2 * grp + (n & 1)], ((n >> 1) - 1) & 1);
 #pragma unroll
                 for (int i = 1; i <= kChunk; ++i) {
                     const float *x = v + (2 * i - 1) * kHR;
@@ -584,8 +590,11 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
     } else if (lane == 0) {
         // ------------------------------------------------------------ bulk stores
         // Staged tiles of the two epilogue groups in job order, and the zero tile for every
-        // fully masked unit (one masked unit between staged jobs, so neither kind waits long).
-        const TO *zero = stage + 2 * kStElems;
+        // fully masked unit (one masked unit per staged job, so neither kind waits long).  Each
+        // iteration commits exactly two bulk groups (masked unit, staged tile; either may be
+        // empty), so when at most four groups are pending the staged tile of two jobs back has
+        // been read and its slot goes back to its epilogue group.
+        const TO *zero = stage + 4 * kStElems;
         int z = 0;
         auto store_zero_unit = [&]() {
             const int4 e = ulist[kListCap - 1 - z];
@@ -597,15 +606,21 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         };
         for (int job = 0; job < nA * CTG; ++job) {
             if (z < nZ) store_zero_unit();
-            const int grp = job & 1;
-            if (!mbar_wait(&staged[grp], (job >> 1) & 1)) break;
+            bulk_commit();
+            const int grp = job & 1, n = job >> 1;
+            if (!mbar_wait(&staged[grp], n & 1)) break;
             const int4 e = ulist[job / CTG];
             const int c0 = (g * CTG + job % CTG) * 128;
-            if (c0 < C) tma_store_4d(&out_map, stage + grp * kStElems, c0, e.z, e.y, e.x);
-            bulk_wait_read_all();           // the tile has been read: the group may overwrite it
-            mbar_arrive(&stage_free[grp]);
+            if (c0 < C) tma_store_4d(&out_map, stage + (2 * grp + (n & 1)) * kStElems, c0, e.z, e.y, e.x);
+            bulk_commit();
+            if (job >= 2) {
+                bulk_wait_read<4>();
+                const int np = (job - 2) >> 1;  // the same group's previous job
+                mbar_arrive(&stage_free[2 * grp + (np & 1)]);
+            }
         }
         while (z < nZ) store_zero_unit();
+        bulk_commit();
         bulk_wait_all();
     }
     __syncwarp();
