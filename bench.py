@@ -463,11 +463,15 @@ def main():
             "subsampler_ms": row_ms["dw_subsample_fwd"],
             "subsampler_roofline_frac": row["dw_subsample_fwd"]["fp32_frac"],
             "rows": row,
-            "roofline": {"bound": "alu", "kernel": "dw_subsample_kernel",
+            "roofline": {"bound": "alu", "kernel": "dw_subsample_tc_kernel",
                          "achieved": sf / (ms * 1e-3) / 1e12, "peak": fp32_tflops, "unit": "TFLOP/s",
                          "frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
                          "peak_basis": f"{sms} SMs x 128 FP32 lanes x 2 x {fmax:.0f} MHz ({peak_kind} max clock)",
-                         "traffic": ncu_traffic("dw_subsample_kernel")},
+                         "traffic": ncu_traffic("dw_subsample_tc_kernel"),
+                         "note": "roofline time = max(alg bytes / HBM, alg FLOPs / FP32 peak), the FP32 term "
+                                 "binding; conv0's 9-tap contraction runs on tcgen05 (TF32 with a 3-product "
+                                 "float32 split), ReLU and conv_dw1 on the FP32 pipes",
+                         "hbm_frac_of_measured": sb / (ms * 1e-3) / 1e9 / hbm},
             "hbm_peak_gbs": hbm, "hbm_peak_kind": peak_kind,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * sum(launches_per_row.values()),

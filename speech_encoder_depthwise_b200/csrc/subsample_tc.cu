@@ -76,9 +76,11 @@ constexpr int kRowsPer = (kN + kPatchThreads - 1) / kPatchThreads;  // patch row
 constexpr int kBarPatch = 1;                // named barrier id of the patch builders
 constexpr int kGroupThreads = 128;          // one epilogue group: 4 warps, one per lane quarter
 constexpr int kListCap = 1024;              // units per block (the list lives in shared memory)
+constexpr int kOrderItems = 4096;           // items up to which the unit deal is balanced
 
 static_assert(kN <= 256 && kN % 16 == 0, "MMA N");
 static_assert(kTileB % 1024 == 0 && kTileA % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+static_assert(3 * (kOrderItems + 1) * 4 <= 2 * kTileB, "unit-deal tables fit the patch tiles");
 static_assert(kHalfCols % kChunk == 0 && 2 * kChunk * kHR == 50 && kHC == 41, "epilogue chunking");
 
 template <typename TO, int CTG>
@@ -304,28 +306,89 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
         tc_fence_before();
-        // this block's units q0, q0 + qs, ...: the active ones from the front of the list, the
-        // fully masked ones (zeros only) from the back, each in increasing order
+        // This block's units: the active ones from the front of the list, the fully masked ones
+        // (zeros only) from the back, each in the order all blocks agree on.
         const int per_item = nIP * nJB;
-        const int mine = q0 < nUnits ? (nUnits - q0 + qs - 1) / qs : 0;
+        const unsigned below = (1u << lane) - 1u;
         int nA = 0, nZ = 0;
-        for (int base = 0; base < mine; base += 32) {
-            const int k = base + lane;
-            const bool have = k < mine;
-            int4 e = make_int4(0, 0, 0, 0);
-            bool act = false;
-            if (have) {
-                const int q = q0 + k * qs;
-                const int b = q / per_item, rem = q - b * per_item, ip = rem / nJB;
-                e = make_int4(b, ip * kRO, (rem - ip * nJB) * kJO, static_cast<int>(clamp_len(lengths, b, Tn)));
-                act = e.y < ((e.w + 1) / 2 + 1) / 2;
-            }
+        auto push = [&](bool have, bool act, const int4 &e) {
             const unsigned ma = __ballot_sync(0xffffffffu, have && act), mz = __ballot_sync(0xffffffffu, have && !act);
-            const unsigned below = (1u << lane) - 1u;
             if (have && act) ulist[nA + __popc(ma & below)] = e;
             if (have && !act) ulist[kListCap - 1 - (nZ + __popc(mz & below))] = e;
             nA += __popc(ma);
             nZ += __popc(mz);
+        };
+        if (B <= kOrderItems) {
+            // Balanced deal: number all active units item-major (then row pair, then column
+            // block) and all masked units likewise; block k takes every qs-th of each, so the
+            // blocks' active work differs by at most one unit.  The prefix tables live in the
+            // patch-operand tile, which nobody touches before the main loops.
+            int *pa = reinterpret_cast<int *>(tileB), *pz = pa + (B + 1), *pl = pz + (B + 1);
+            int run_a = 0, run_z = 0;
+            if (lane == 0) pa[0] = pz[0] = 0;
+            for (int base = 0; base < B; base += 32) {
+                const int b = base + lane;
+                int ia = 0, iz = 0;
+                if (b < B) {
+                    const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+                    const int rows = (((L + 1) / 2 + 1) / 2 + kRO - 1) / kRO;  // row pairs with an unmasked row
+                    ia = rows * nJB;
+                    iz = (nIP - rows) * nJB;
+                    pl[b] = L;
+                }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int ta = __shfl_up_sync(0xffffffffu, ia, o), tz = __shfl_up_sync(0xffffffffu, iz, o);
+                    if (lane >= o) {
+                        ia += ta;
+                        iz += tz;
+                    }
+                }
+                if (b < B) {
+                    pa[b + 1] = run_a + ia;
+                    pz[b + 1] = run_z + iz;
+                }
+                run_a += __shfl_sync(0xffffffffu, ia, 31);
+                run_z += __shfl_sync(0xffffffffu, iz, 31);
+            }
+            __syncwarp();
+            for (int k0 = 0;; k0 += 32) {  // active units q0 + k qs
+                const int a = q0 + (k0 + lane) * qs;
+                const bool have = a < run_a;
+                if (!__any_sync(0xffffffffu, have)) break;
+                int4 e = make_int4(0, 0, 0, 0);
+                if (have) {
+                    const int b = TileOrder::find(pa, B, a), local = a - pa[b], ip = local / nJB;
+                    e = make_int4(b, ip * kRO, (local - ip * nJB) * kJO, pl[b]);
+                }
+                push(have, true, e);
+            }
+            for (int k0 = 0;; k0 += 32) {  // masked units q0 + k qs
+                const int z = q0 + (k0 + lane) * qs;
+                const bool have = z < run_z;
+                if (!__any_sync(0xffffffffu, have)) break;
+                int4 e = make_int4(0, 0, 0, 0);
+                if (have) {
+                    const int b = TileOrder::find(pz, B, z), local = z - pz[b], ip = local / nJB;
+                    e = make_int4(b, ((pa[b + 1] - pa[b]) / nJB + ip) * kRO, (local - ip * nJB) * kJO, pl[b]);
+                }
+                push(have, false, e);
+            }
+        } else {  // many items: plain round robin over all units
+            const int mine = q0 < nUnits ? (nUnits - q0 + qs - 1) / qs : 0;
+            for (int base = 0; base < mine; base += 32) {
+                const int k = base + lane;
+                const bool have = k < mine;
+                int4 e = make_int4(0, 0, 0, 0);
+                bool act = false;
+                if (have) {
+                    const int q = q0 + k * qs;
+                    const int b = q / per_item, rem = q - b * per_item, ip = rem / nJB;
+                    e = make_int4(b, ip * kRO, (rem - ip * nJB) * kJO, static_cast<int>(clamp_len(lengths, b, Tn)));
+                    act = e.y < ((e.w + 1) / 2 + 1) / 2;
+                }
+                push(have, act, e);
+            }
         }
         if (lane == 0) {
             counts[0] = nA;
@@ -682,7 +745,7 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
     if (grid > units * nG) grid = units * nG;
     if (grid > kMaxGrid) return cudaErrorInvalidConfiguration;
     // every block keeps its unit list in shared memory; larger problems take the SIMT kernel
-    if ((units + grid / nG - 1) / (grid / nG) > kListCap) return cudaErrorNotSupported;
+    if ((units + grid / nG - 1) / (grid / nG) + 1 > kListCap) return cudaErrorNotSupported;
     const int Pt = a.causal ? 2 : 1;
 #define DW_TC_LAUNCH(TO, CTG)                                                                                  \
     do {                                                                                                       \
