@@ -87,8 +87,9 @@ class Oracle:
         lib.oracle_dwconv1d_bwd_dw.argtypes = [_D, _D, _I, _L, _L, _L, _L, _L, _D, _D]
         lib.oracle_dw_subsample_fwd.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L,
                                                 ctypes.c_int, _D, _I]
+        lib.oracle_dwconv1d_stream_fwd.argtypes = [_D, _D, _D, _D, _I, _L, _L, _L, _L, _D, _D]
         for f in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_dx", "oracle_dwconv1d_bwd_dw",
-                  "oracle_dw_subsample_fwd"):
+                  "oracle_dw_subsample_fwd", "oracle_dwconv1d_stream_fwd"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -111,6 +112,27 @@ class Oracle:
         if rc:
             raise ValueError(f"oracle_dwconv1d_fwd rejected its arguments (rc={rc})")
         return y
+
+    def dwconv1d_stream_fwd(self, x, w, bias, cache, lengths):
+        """One chunk of the streaming causal conv: returns (y [B,T,C], new cache [B,K-1,C]).
+
+        cache [B,K-1,C] holds each stream's K-1 most recent frames; the chunk appends the first
+        lengths[b] frames of x[b] (all T when lengths is None)."""
+        x = _f64(x); w = _f64(w)
+        B, T, C = x.shape
+        K = w.shape[0]
+        assert w.shape == (K, C)
+        cin = _f64(cache) if K > 1 else np.zeros((B, 0, C))
+        assert cin.shape == (B, K - 1, C)
+        b = _f64(bias) if bias is not None else None
+        ln = _lens(lengths, B)
+        y = np.empty((B, T, C), dtype=np.float64)
+        cout = np.empty((B, K - 1, C), dtype=np.float64)
+        rc = self.lib.oracle_dwconv1d_stream_fwd(_dp(x), _dp(w), _dp(b), _dp(cin) if K > 1 else None,
+                                                 _ip(ln), B, T, C, K, _dp(y), _dp(cout) if K > 1 else None)
+        if rc:
+            raise ValueError(f"oracle_dwconv1d_stream_fwd rejected its arguments (rc={rc})")
+        return y, cout
 
     def dwconv1d_bwd_dx(self, dy, w, lengths, pad_left):
         """Data gradient of ``dwconv1d_fwd`` (the transpose of the forward map)."""
@@ -178,6 +200,10 @@ def num_threads() -> int:
 
 def dwconv1d_fwd(x, w, bias, lengths, pad_left):
     return default().dwconv1d_fwd(x, w, bias, lengths, pad_left)
+
+
+def dwconv1d_stream_fwd(x, w, bias, cache, lengths):
+    return default().dwconv1d_stream_fwd(x, w, bias, cache, lengths)
 
 
 def dwconv1d_bwd_dx(dy, w, lengths, pad_left):

@@ -240,3 +240,47 @@ int oracle_dw_subsample_fwd(const double *mel, const double *w0, const double *b
     free(hpad);
     return 0;
 }
+
+/*
+ * Streaming causal forward, one chunk (parakeet.cpp PR #102, "What changes": the streaming
+ * encoder keeps its own depthwise conv with a cache).  For stream b the sequence seen so far
+ * ends with the K-1 cached frames, and this chunk appends its first len_b frames:
+ *   xcat_b      = [cache_b frames 0..K-2 ; x_b frames 0..len_b-1]
+ *   y[b,t,c]    = [t < len_b] * (bias[c] + sum_{k<K} xcat_b[t+k,c] * w[k,c])
+ *   cache_out_b = xcat_b frames len_b .. len_b+K-2   (the K-1 most recent frames)
+ * which is the causal conv (pad_left = K-1) of the whole stream, chunk by chunk, when the
+ * cache starts at zero.  x, y: [B][T][C]; cache_in, cache_out: [B][K-1][C] (NULL if K == 1).
+ */
+int oracle_dwconv1d_stream_fwd(const double *x, const double *w, const double *bias,
+                               const double *cache_in, const int32_t *lengths, int64_t B,
+                               int64_t T, int64_t C, int64_t K, double *y, double *cache_out)
+{
+    if (B < 0 || T < 0 || C < 1 || K < 1) return 1;
+    if (K > 1 && (cache_in == NULL || cache_out == NULL)) return 1;
+    const int64_t H = K - 1;                       /* cached frames */
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        /* H + T frames: the frames after the chunk's valid ones stay zero and are never summed */
+        double *xcat = (double *)calloc((size_t)((H + T) * C + 1), sizeof(double));
+        if (!xcat) return 2;
+        for (int64_t j = 0; j < H; ++j)
+            for (int64_t c = 0; c < C; ++c) xcat[j * C + c] = cache_in[(b * H + j) * C + c];
+        for (int64_t s = 0; s < L; ++s)
+            for (int64_t c = 0; c < C; ++c) xcat[(H + s) * C + c] = x[(b * T + s) * C + c];
+        #pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t c = 0; c < C; ++c) {
+                double acc = 0.0;
+                if (L > t) {   /* frame t of the chunk is part of the stream */
+                    acc = bias ? bias[c] : 0.0;
+                    for (int64_t k = 0; k < K; ++k) acc += xcat[(t + k) * C + c] * w[k * C + c];
+                }
+                y[(b * T + t) * C + c] = acc;
+            }
+        }
+        for (int64_t j = 0; j < H; ++j)
+            for (int64_t c = 0; c < C; ++c) cache_out[(b * H + j) * C + c] = xcat[(L + j) * C + c];
+        free(xcat);
+    }
+    return 0;
+}

@@ -162,6 +162,55 @@ def rel_err(a, b):
 # ----------------------------------------------------------------------------------
 # a quick battery of every kind of pin, for the mutation test
 # ----------------------------------------------------------------------------------
+def np_stream_fwd(x, w, bias, cache, L):
+    """One chunk of the streaming causal conv written out directly in numpy: the chunk's valid
+    frames appended to the K-1 cached ones, the K-tap sum, the output mask, the new cache."""
+    B, T, C = x.shape
+    K = w.shape[0]
+    y = np.zeros((B, T, C))
+    cout = np.zeros((B, K - 1, C))
+    for b in range(B):
+        n = T if L is None else int(min(max(L[b], 0), T))
+        xcat = np.concatenate([cache[b], x[b, :n]], axis=0)  # [K-1+n, C]
+        for t in range(n):
+            y[b, t] = (0.0 if bias is None else bias) + (xcat[t:t + K] * w).sum(axis=0)
+        cout[b] = xcat[n:n + K - 1]
+    return y, cout
+
+
+def stream_chunked_vs_whole(o, rng, B, C, K, T, n_chunks, bias=True):
+    """Feed random chunks (valid lengths 0..T, some below K-1) through ``o.dwconv1d_stream_fwd``
+    from a zero cache; compare every valid output with the causal conv (im2col formulation) of
+    each stream's concatenated valid frames, masked outputs with exact zeros, and the final
+    cache with the stream's last K-1 frames.  Returns a list of failure strings."""
+    fails = []
+    w = rng.standard_normal((K, C)); b = rng.standard_normal(C) if bias else None
+    cache = np.zeros((B, K - 1, C))
+    seen = [np.zeros((0, C)) for _ in range(B)]
+    outs = [[] for _ in range(B)]
+    for _ in range(n_chunks):
+        x = rng.standard_normal((B, T, C))
+        L = rng.integers(0, T + 1, size=B).astype(np.int32)
+        y, cache = o.dwconv1d_stream_fwd(x, w, b, cache, L)
+        for i in range(B):
+            if np.any(y[i, L[i]:] != 0.0):
+                fails.append(f"stream masked frames not zero {B, C, K, T}")
+            seen[i] = np.concatenate([seen[i], x[i, :L[i]]])
+            outs[i].append(y[i, :L[i]])
+    for i in range(B):
+        n = seen[i].shape[0]
+        if n == 0:
+            continue
+        whole = im2col_fwd(seen[i][None], w, b, None, K - 1)[0]
+        got = np.concatenate(outs[i])
+        if rel_err(got, whole) > 1e-12:
+            fails.append(f"stream chunked != whole {B, C, K, T}")
+        last = np.concatenate([np.zeros((K - 1, C)), seen[i]])[-(K - 1):] if K > 1 else np.zeros((0, C))
+        if not np.array_equal(cache[i], last):
+            fails.append(f"stream cache != last frames {B, C, K, T}")
+    return fails
+
+
 def pin_battery(o):
     """Run a fast selection of pins against oracle ``o``; returns a list of failure strings."""
     fails = []
@@ -219,4 +268,14 @@ def pin_battery(o):
         ref, rl = torch_subsample(mel, w0, b0, w1, b1, L, causal)
         if out.shape != ref.shape or rel_err(out, ref) > 1e-12 or not np.array_equal(ol, rl):
             fails.append(f"torch subsample causal={causal}")
+
+    # streaming chunks: the whole-stream causal conv, and the direct numpy statement
+    for (B, C, K, T, n) in ((3, 4, 4, 5, 6), (2, 3, 9, 3, 8), (2, 2, 1, 4, 3)):
+        fails += stream_chunked_vs_whole(o, rng, B, C, K, T, n)
+    x = rng.standard_normal((3, 6, 5)); w = rng.standard_normal((3, 5)); bias = rng.standard_normal(5)
+    cache = rng.standard_normal((3, 2, 5)); L = np.array([6, 0, 1], np.int32)
+    y, c = o.dwconv1d_stream_fwd(x, w, bias, cache, L)
+    ry, rc = np_stream_fwd(x, w, bias, cache, L)
+    if rel_err(y, ry) > 1e-12 or not np.array_equal(c, rc):
+        fails.append("numpy stream")
     return fails

@@ -32,6 +32,11 @@ MUTANTS = {
     "conv_dw1 freq taps flipped": ("hpad[((2 * i + p) * HF + (2 * j + q)) * C + c]",
                                    "hpad[((2 * i + p) * HF + (2 * j + 2 - q)) * C + c]"),
     "mel not masked": ("melpad[r * FP + f] = (t >= 0 && t < L &&", "melpad[r * FP + f] = (t >= 0 && t < T &&"),
+    "stream cache not shifted": ("cache_out[(b * H + j) * C + c] = xcat[(L + j) * C + c];",
+                                 "cache_out[(b * H + j) * C + c] = xcat[j * C + c];"),
+    "stream output mask dropped": ("if (L > t) {", "if (T > t) {"),
+    "stream taps reversed": ("acc += xcat[(t + k) * C + c] * w[k * C + c];",
+                             "acc += xcat[(t + k) * C + c] * w[(K - 1 - k) * C + c];"),
 }
 
 
