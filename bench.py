@@ -145,6 +145,58 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ helpers
+STREAM = dict(B=64, C=512, K=9, chunks=(1, 16), seed=21)
+
+
+def measure_stream(dw, dev, hbm):
+    """Streaming causal conv with a cache (a NEXT row, outside the step): 64 streams, C=512,
+    K=9, bf16, chunks of 1 and 16 frames; 8 chunks captured in a graph, replayed.  Reports µs
+    per chunk, GB/s (chunk in, output, cache in and out), frames/s and the max error of one chunk
+    against the oracle."""
+    import torch
+    import oracle
+    from synth import bf16_round
+    B, C, K = STREAM["B"], STREAM["C"], STREAM["K"]
+    rng = np.random.default_rng(STREAM["seed"])
+    w = bf16_round(rng.standard_normal((K, C)) / np.sqrt(K))
+    b = bf16_round(rng.standard_normal(C) * np.sqrt(0.1))
+    gw = torch.from_numpy(w).to(dev)
+    gb = torch.from_numpy(b).to(dev)
+    res = {}
+    for T in STREAM["chunks"]:
+        xs = [bf16_round(rng.standard_normal((B, T, C))) for _ in range(8)]
+        gx = [torch.from_numpy(x).to(dev, torch.bfloat16) for x in xs]
+        gy = [torch.empty_like(x) for x in gx]
+        cache = torch.zeros(B, K - 1, C, dtype=torch.bfloat16, device=dev)
+        s = torch.cuda.Stream(dev)
+        with torch.cuda.stream(s):
+            dw.dwconv1d_stream_fwd(gx[0], gw, gb, gy[0], cache, None)
+            torch.cuda.synchronize(dev)
+            y0 = gy[0].float().cpu().numpy()
+            ry, _ = oracle.dwconv1d_stream_fwd(xs[0], w, b, np.zeros((B, K - 1, C)), None)
+            err = float(np.max(np.abs(y0 - ry)))
+            g = torch.cuda.CUDAGraph()
+            g.capture_begin()
+            for i in range(8):
+                dw.dwconv1d_stream_fwd(gx[i], gw, gb, gy[i], cache, None)
+            g.capture_end()
+            for _ in range(5):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(50):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) / 400 * 1e3
+        by = (2 * B * T * C + 2 * B * (K - 1) * C) * 2
+        res[f"chunk{T}"] = {"us": us, "GB_per_s": by / us / 1e3, "hbm_frac_of_measured": by / us / 1e3 / hbm,
+                            "frames_per_s": B * T / (us * 1e-6), "alg_bytes": by, "max_abs_err": err}
+        del g
+    return {"workload": f"streaming causal dwconv1d with a [K-1,C] cache: {B} streams, C={C}, K={K}, bf16, "
+                        "chunks of 1 and 16 frames (8 chunks per CUDA graph)", **res}
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -470,6 +522,7 @@ def main():
         ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
+        next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm)}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
             v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)
@@ -497,6 +550,7 @@ def main():
                          "hbm_frac_of_measured": sb / (ms * 1e-3) / 1e9 / hbm},
             "hbm_peak_gbs": hbm, "hbm_peak_kind": peak_kind,
             "cpu_baseline": cpu, "e2e": e2e,
+            "next_rows": next_rows,
             "gpu_launches": steps * sum(launches_per_row.values()),
             "clocks": clocks,
         }

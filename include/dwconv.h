@@ -93,6 +93,32 @@ dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int3
                             dw_dtype_t io_dtype, dw_stream_t stream);
 
 /*
+ * dwconv1d_stream_fwd - one chunk of a streaming causal depthwise conv1d with a cache of each
+ * stream's K-1 most recent input frames (parakeet.cpp PR #102, section "What changes": the
+ * streaming encoder keeps its own depthwise conv with a cache).
+ *
+ *   xcat_b      = [cache_b (K-1 frames) ; x_b frames 0 .. len_b-1]
+ *   y[b,t,c]    = [t < len_b] (bias[c] + sum_{k<K} xcat_b[t+k,c] w[k,c])
+ *   cache_b    <- xcat_b frames len_b .. len_b+K-2   (rewritten in place)
+ *
+ * Feeding a stream chunk by chunk from a zero cache gives exactly the frames of dwconv1d_fwd
+ * with causal padding (pad_left = K-1) over the whole stream.
+ *
+ *  x        [B][T][C] io_dtype, device: this chunk; frames t >= len_b are not part of the
+ *           stream (they are neither used nor cached)
+ *  w, bias  as dwconv1d_fwd
+ *  y        [B][T][C] io_dtype, device, written in full (zeros at t >= len_b); must not
+ *           overlap x or cache
+ *  cache    [B][K-1][C] io_dtype, device, read and rewritten; may be NULL when K == 1;
+ *           must not overlap x or y.  A new stream starts from a zeroed cache.
+ *  lengths  [B] int32, device, or NULL (all T frames valid): valid frames of this chunk
+ *  B >= 0, T >= 0 (T == 0 leaves the cache unchanged), C >= 1, K >= 1
+ */
+dw_status_t dwconv1d_stream_fwd(const void *x, const float *w, const float *bias, void *y,
+                                void *cache, const int32_t *lengths, int64_t B, int64_t T,
+                                int64_t C, int K, dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
  * dwconv1d_bwd_dw_workspace_size - bytes of device workspace dwconv1d_bwd_dw needs for
  * these sizes (independent of pointers, dtype and device).  Returns 0 when B*T == 0.
  */

@@ -20,7 +20,7 @@ __all__ = [
     "DW_OK", "DW_ERR_INVALID_ARG", "DW_ERR_UNSUPPORTED", "DW_ERR_WORKSPACE", "DW_ERR_CUDA",
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
-    "dwconv1d_bwd_dw_noalloc",
+    "dwconv1d_bwd_dw_noalloc", "dwconv1d_stream_fwd",
     "dw_subsample_fwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
 ]
 
@@ -44,6 +44,7 @@ SIGNATURES = {
     "dwconv1d_bwd_dw": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp,
                                ctypes.c_size_t, _vp]),
     "dwconv1d_bwd_dw_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
+    "dwconv1d_stream_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
     "dw_status_string": (ctypes.c_char_p, [_int]),
@@ -135,6 +136,20 @@ def dwconv1d_fwd(x, w, bias, y, lengths, pad_left, stream=None):
                             _dev(lengths, "lengths", torch.int32, (B,)), B, T, C, K, int(pad_left),
                             _dtype_code(x), _stream(stream))
     _check("dwconv1d_fwd", st)
+
+
+def dwconv1d_stream_fwd(x, w, bias, y, cache, lengths, stream=None):
+    """One chunk of the streaming causal conv: ``y`` from the chunk ``x`` [B,T,C] and each
+    stream's K-1 cached frames; ``cache`` [B,K-1,C] is rewritten with the K-1 newest frames."""
+    import torch
+    B, T, C = x.shape
+    K = w.shape[0]
+    cache_ptr = _dev(cache, "cache", x.dtype, (B, K - 1, C)) if K > 1 else _dev(cache, "cache")
+    st = lib().dwconv1d_stream_fwd(_dev(x, "x"), _dev(w, "w", torch.float32, (K, C)),
+                                   _dev(bias, "bias", torch.float32, (C,)), _dev(y, "y", x.dtype, x.shape),
+                                   cache_ptr, _dev(lengths, "lengths", torch.int32, (B,)), B, T, C, K,
+                                   _dtype_code(x), _stream(stream))
+    _check("dwconv1d_stream_fwd", st)
 
 
 def dwconv1d_bwd_dx(dy, w, dx, lengths, pad_left, stream=None):

@@ -126,6 +126,30 @@ dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int3
     return cuda_status(dwk::conv1d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
 }
 
+dw_status_t dwconv1d_stream_fwd(const void *x, const float *w, const float *bias, void *y, void *cache,
+                                const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
+                                dw_dtype_t io_dtype, dw_stream_t stream) {
+    int64_t n = 0;
+    dw_status_t st = check_conv1d_common(x, w, y, B, T, C, K, K - 1, io_dtype, &n);
+    if (st != DW_OK || n == 0) return st;
+    const size_t es = dtype_size(io_dtype);
+    const size_t cache_bytes = static_cast<size_t>(B) * static_cast<size_t>(K - 1) * static_cast<size_t>(C) * es;
+    if (K > 1) {
+        if (cache == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t bytes = static_cast<size_t>(n) * es;
+        if (overlaps(cache, cache_bytes, x, bytes) || overlaps(cache, cache_bytes, y, bytes)) return DW_ERR_INVALID_ARG;
+    }
+    dwk::StreamArgs a;
+    a.x = x; a.w = w; a.bias = bias; a.y = y; a.cache = cache; a.lengths = lengths;
+    a.B = B; a.T = T; a.C = C; a.K = K;
+    a.bf16 = io_dtype == DW_BF16;
+    a.vec_width = pick_vec_width(C, es, {x, y, cache}, {w, bias});
+    // bf16 rows of 8 channels move as one 16-byte word when everything lines up
+    if (a.bf16 && a.vec_width == 4 && C % 8 == 0 && aligned(x, 16) && aligned(y, 16) && aligned(cache, 16))
+        a.vec_width = 8;
+    return cuda_status(dwk::conv1d_stream_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t dwconv1d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t C, int K) {
     if (B <= 0 || T <= 0 || C < 1 || K < 1) return 0;
     int64_t n = 0;

@@ -37,6 +37,17 @@ struct DwArgs {
     int G;                // partial rows (blocks per channel tile)
 };
 
+struct StreamArgs {
+    const void *x;        // chunk [B][T][C]
+    const float *w;       // [K][C]
+    const float *bias;    // [C] or null
+    void *y;              // [B][T][C]
+    void *cache;          // [B][K-1][C], read and rewritten
+    const int32_t *lengths;
+    int64_t B, T, C;
+    int K, bf16, vec_width;  // vec_width: 8 (bf16 only), 4, 2 or 1 channels per thread
+};
+
 struct SubsampleArgs {
     const float *mel, *w0, *b0, *w1, *b1;
     void *out;
@@ -73,6 +84,8 @@ int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t C, int K);
 size_t conv1d_dw_workspace_bytes(int64_t B, int64_t T, int64_t C, int K);
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s);
 unsigned int conv1d_dw_take_error();
+
+cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s);
 
 cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
 // Tensor-core subsampler: usable when the output rows are 16-byte aligned (C * element size a

@@ -71,6 +71,29 @@ def test_dx_rejects_invalid_arguments(lib):
     assert f(FAKE_X, FAKE_W, FAKE_Y, None, 2, 10, 8, 3, 5, dw.DW_F32, None) == dw.DW_ERR_INVALID_ARG
 
 
+def test_stream_rejects_invalid_arguments(lib):
+    f = lib.dwconv1d_stream_fwd
+    FAKE_C = 0x50000000
+    ok = (FAKE_X, FAKE_W, None, FAKE_Y, FAKE_C, None, 4, 16, 512, 9, dw.DW_BF16, None)
+
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[["x", "w", "bias", "y", "cache", "ln", "B", "T", "C", "K", "dt", "s"].index(k)] = v
+        return f(*a)
+    assert call(cache=None) == dw.DW_ERR_INVALID_ARG             # K > 1 needs a cache
+    assert call(cache=FAKE_Y + 64) == dw.DW_ERR_INVALID_ARG      # cache overlaps y
+    assert call(cache=FAKE_X) == dw.DW_ERR_INVALID_ARG           # cache overlaps x
+    assert call(y=FAKE_X + 2) == dw.DW_ERR_INVALID_ARG           # y overlaps x
+    assert call(K=0) == dw.DW_ERR_INVALID_ARG
+    assert call(C=0) == dw.DW_ERR_INVALID_ARG
+    assert call(B=-1) == dw.DW_ERR_INVALID_ARG
+    assert call(dt=3) == dw.DW_ERR_INVALID_ARG
+    assert call(K=5000) == dw.DW_ERR_UNSUPPORTED
+    assert call(T=0, x=None, y=None) == dw.DW_OK                 # no frames: nothing to do
+    assert call(B=0) == dw.DW_OK
+
+
 def test_empty_inputs_are_noops_without_a_device(lib):
     assert fwd(lib, B=0) == dw.DW_OK
     assert fwd(lib, T=0) == dw.DW_OK
