@@ -197,6 +197,65 @@ def measure_stream(dw, dev, hbm):
                         "chunks of 1 and 16 frames (8 chunks per CUDA graph)", **res}
 
 
+BWD = dict(B=32, T=1500, C=1024, K=9, pad_left=4, len_range=(750, 1500), seed=4)
+
+
+def measure_bwd(dw, dev, hbm):
+    """One-pass backward (a NEXT row, outside the step) on the training-size backward workload,
+    32x1500x1024 bf16, K=9: dwconv1d_bwd against dwconv1d_bwd_dx + dwconv1d_bwd_dw, each over 3
+    rotating input sets captured in a CUDA graph.  Algorithmic bytes: x and dy at valid frames,
+    dx written in full."""
+    import torch
+    import oracle
+    from synth import conv1d_inputs
+    B, T, C, K, pl = BWD["B"], BWD["T"], BWD["C"], BWD["K"], BWD["pad_left"]
+    d = conv1d_inputs(B, T, C, K, dtype="bf16", len_range=BWD["len_range"], seed=BWD["seed"], with_dy=True)
+    x0 = torch.from_numpy(d["x"]).to(dev, torch.bfloat16)
+    g0 = torch.from_numpy(d["dy"]).to(dev, torch.bfloat16)
+    xs, gs = [x0] + [x0.clone() for _ in range(2)], [g0] + [g0.clone() for _ in range(2)]
+    dxs = [torch.empty_like(x0) for _ in range(3)]
+    w = torch.from_numpy(d["w"]).to(dev)
+    ln = torch.from_numpy(d["lengths"]).to(dev)
+    gw, gb = torch.empty(K, C, device=dev), torch.empty(C, device=dev)
+    ws = torch.empty(dw.dwconv1d_bwd_dw_workspace_size(B, T, C, K), dtype=torch.uint8, device=dev)
+    valid = int(np.clip(d["lengths"], 0, T).sum()) * C
+    by = (2 * valid + B * T * C) * 2
+    s = torch.cuda.Stream(dev)
+
+    def timed(fn):
+        with torch.cuda.stream(s):
+            for i in range(3):
+                fn(i)
+            g = torch.cuda.CUDAGraph()
+            g.capture_begin()
+            for i in range(3):
+                fn(i)
+            g.capture_end()
+            for _ in range(3):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(20):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize(dev)
+        del g
+        return e0.elapsed_time(e1) / 60 * 1e3
+
+    fused = timed(lambda i: dw.dwconv1d_bwd(xs[i], gs[i], w, dxs[i], gw, gb, ln, pl, ws))
+    sep = timed(lambda i: (dw.dwconv1d_bwd_dx(gs[i], w, dxs[i], ln, pl),
+                           dw.dwconv1d_bwd_dw(xs[i], gs[i], gw, gb, ln, pl, ws)))
+    with torch.cuda.stream(s):
+        dw.dwconv1d_bwd(xs[0], gs[0], w, dxs[0], gw, gb, ln, pl, ws)
+    torch.cuda.synchronize(dev)
+    ref = oracle.dwconv1d_bwd_dx(d["dy"][:1], d["w"], d["lengths"][:1], pl)
+    err = float(np.max(np.abs(dxs[0][:1].float().cpu().numpy() - ref)))
+    return {"workload": f"one-pass dX + dW/dbias, {B}x{T}x{C} bf16, K={K}, sym 4|4, len U[750,1500] "
+                        "(3 rotating input sets in a CUDA graph)",
+            "us": fused, "GB_per_s": by / fused / 1e3, "hbm_frac_of_measured": by / fused / 1e3 / hbm,
+            "alg_bytes": by, "separate_dx_plus_dw_us": sep, "dx_max_abs_err_item0": err}
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -522,7 +581,7 @@ def main():
         ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
-        next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm)}
+        next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm), "dwconv1d_bwd": measure_bwd(dw, dev, hbm)}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
             v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)

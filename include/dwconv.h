@@ -148,6 +148,23 @@ dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
                             size_t workspace_bytes, dw_stream_t stream);
 
 /*
+ * dwconv1d_bwd - the data gradient and the weight/bias gradients of dwconv1d_fwd in one pass
+ * that reads dy once (NeMo PR #16114, section "What does this PR do ?", the depthwise kernel's
+ * backward).  Results equal dwconv1d_bwd_dx followed by dwconv1d_bwd_dw: dx up to float32
+ * summation order, dW/dbias bitwise reproducible for given sizes like dwconv1d_bwd_dw.
+ *
+ *  x, dy, dx  [B][T][C] io_dtype, device; dx is written in full and must not overlap x or dy
+ *  w          [K][C] float32 (the forward taps)
+ *  dw, dbias, workspace, workspace_bytes: as dwconv1d_bwd_dw
+ *  other arguments as dwconv1d_fwd (pad_left is the forward pass's).
+ * Sizes without a fused instance run the two gradients one after the other (same results).
+ */
+dw_status_t dwconv1d_bwd(const void *x, const void *dy, const float *w, void *dx, float *dw,
+                         float *dbias, const int32_t *lengths, int64_t B, int64_t T, int64_t C,
+                         int K, int pad_left, dw_dtype_t io_dtype, void *workspace,
+                         size_t workspace_bytes, dw_stream_t stream);
+
+/*
  * dwconv1d_bwd_dw_noalloc - dwconv1d_bwd_dw without a caller-provided workspace: it allocates
  * nothing and uses a scratch array that the library keeps in device memory.  The papers have
  * no counterpart to this entry point; it exists for callers that cannot allocate device

@@ -20,7 +20,7 @@ __all__ = [
     "DW_OK", "DW_ERR_INVALID_ARG", "DW_ERR_UNSUPPORTED", "DW_ERR_WORKSPACE", "DW_ERR_CUDA",
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
-    "dwconv1d_bwd_dw_noalloc", "dwconv1d_stream_fwd",
+    "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd",
     "dw_subsample_fwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
 ]
 
@@ -44,6 +44,8 @@ SIGNATURES = {
     "dwconv1d_bwd_dw": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp,
                                ctypes.c_size_t, _vp]),
     "dwconv1d_bwd_dw_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
+    "dwconv1d_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp,
+                            ctypes.c_size_t, _vp]),
     "dwconv1d_stream_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
@@ -136,6 +138,20 @@ def dwconv1d_fwd(x, w, bias, y, lengths, pad_left, stream=None):
                             _dev(lengths, "lengths", torch.int32, (B,)), B, T, C, K, int(pad_left),
                             _dtype_code(x), _stream(stream))
     _check("dwconv1d_fwd", st)
+
+
+def dwconv1d_bwd(x, dy, w, dx, gw, gb, lengths, pad_left, workspace, stream=None):
+    """dx and dW/dbias of dwconv1d_fwd in one pass over dy (dbias ``gb`` may be None)."""
+    import torch
+    B, T, C = x.shape
+    K = w.shape[0]
+    st = lib().dwconv1d_bwd(_dev(x, "x"), _dev(dy, "dy", x.dtype, x.shape), _dev(w, "w", torch.float32, (K, C)),
+                            _dev(dx, "dx", x.dtype, x.shape), _dev(gw, "dw", torch.float32, (K, C)),
+                            _dev(gb, "dbias", torch.float32, (C,)), _dev(lengths, "lengths", torch.int32, (B,)),
+                            B, T, C, K, int(pad_left), _dtype_code(x), _dev(workspace, "workspace"),
+                            workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                            _stream(stream))
+    _check("dwconv1d_bwd", st)
 
 
 def dwconv1d_stream_fwd(x, w, bias, y, cache, lengths, stream=None):

@@ -126,6 +126,46 @@ dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int3
     return cuda_status(dwk::conv1d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
 }
 
+dw_status_t dwconv1d_bwd(const void *x, const void *dy, const float *w, void *dx, float *dw, float *dbias,
+                         const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K, int pad_left,
+                         dw_dtype_t io_dtype, void *workspace, size_t workspace_bytes, dw_stream_t stream) {
+    int64_t n = 0;
+    dw_status_t st = check_conv1d_common(dy, w, dx, B, T, C, K, pad_left, io_dtype, &n);
+    if (st != DW_OK) return st;
+    if (n > 0) {
+        if (x == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t bytes = static_cast<size_t>(n) * dtype_size(io_dtype);
+        if (overlaps(dx, bytes, x, bytes)) return DW_ERR_INVALID_ARG;
+    }
+    // the weight-gradient entry validates the rest and serves the degenerate sizes
+    if (n == 0)
+        return dwconv1d_bwd_dw(x, dy, dw, dbias, lengths, B, T, C, K, pad_left, io_dtype, workspace,
+                               workspace_bytes, stream);
+    if (dw == nullptr) return DW_ERR_INVALID_ARG;
+    const size_t need = dwk::conv1d_dw_workspace_bytes(B, T, C, K);
+    if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return DW_ERR_WORKSPACE;
+    const size_t out_bytes = static_cast<size_t>(K) * C * sizeof(float);
+    if (overlaps(workspace, need, dw, out_bytes) ||
+        (dbias && overlaps(workspace, need, dbias, static_cast<size_t>(C) * sizeof(float))))
+        return DW_ERR_INVALID_ARG;
+    dwk::DwArgs a;
+    a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = lengths;
+    a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left;
+    a.bf16 = io_dtype == DW_BF16;
+    a.partials = static_cast<float *>(workspace);
+    a.G = dwk::conv1d_dw_partial_rows(B, T, C, K);
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, dy, dx}, {w});
+    a.w = w;
+    a.dx = dx;
+    const cudaError_t e = dwk::conv1d_bwd_fused_launch(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+    // no fused instance for these sizes: the two gradients, one after the other
+    st = dwconv1d_bwd_dx(dy, w, dx, lengths, B, T, C, K, pad_left, io_dtype, stream);
+    if (st != DW_OK) return st;
+    return dwconv1d_bwd_dw(x, dy, dw, dbias, lengths, B, T, C, K, pad_left, io_dtype, workspace, workspace_bytes,
+                           stream);
+}
+
 dw_status_t dwconv1d_stream_fwd(const void *x, const float *w, const float *bias, void *y, void *cache,
                                 const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
                                 dw_dtype_t io_dtype, dw_stream_t stream) {

@@ -189,26 +189,35 @@ constexpr int kDwStages = DW_DW_STAGES;        // shared-memory ring depth
 constexpr int kDwBlocks = DW_DW_BLOCKS;        // resident blocks per SM
 constexpr int kDwTmaThreads = 32 * (1 + kDwConsumers);
 
-template <typename T, int V, int KB>
+// FUSED: the same pass also computes the data gradient, so the dy tile carries K-1 halo rows
+// (the dx correlation reads dy frames s + pad_left - k).  Its threads hold two sets of
+// accumulators, so it runs one block per SM (more registers per thread).
+template <typename T, int V, int KB, bool FUSED = false>
 struct DwTmaShape {
+    static constexpr int CONS = kDwConsumers;  // consumer warps
+    static constexpr int R = kDwR;             // frames per consumer thread per unit
+    static constexpr int THREADS = 32 * (1 + CONS);
     static constexpr int CT = 32 * V;
-    static constexpr int TT = kDwConsumers * kDwR;
+    static constexpr int TT = CONS * R;
     static constexpr int XROWS = TT + KB - 1;
+    static constexpr int DROWS = FUSED ? TT + KB - 1 : TT;
     static constexpr int ROWB = CT * static_cast<int>(sizeof(T));
-    static constexpr int STAGE_BYTES = (XROWS + TT) * ROWB;
-    static constexpr int RED_BYTES = kDwConsumers * (KB + 1) * CT * 4;
+    static constexpr int STAGE_BYTES = (XROWS + DROWS) * ROWB;
+    static constexpr int RED_BYTES = CONS * (KB + 1) * CT * 4;
     static constexpr int BODY = (kDwStages * STAGE_BYTES > RED_BYTES) ? kDwStages * STAGE_BYTES : RED_BYTES;
     static constexpr int SMEM = 128 + BODY;  // plus the tile-order tables, sized at launch
 };
 
-template <typename T, int V, int KB>
-__global__ void __launch_bounds__(kDwTmaThreads, kDwBlocks)
+template <typename T, int V, int KB, bool FUSED = false>
+__global__ void __launch_bounds__(DwTmaShape<T, V, KB, FUSED>::THREADS, FUSED ? 1 : kDwBlocks)
 conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
                      const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C, int K,
-                     int k_off, int pad_left, int nT, int with_bias, int ordered) {
-    using S = DwTmaShape<T, V, KB>;
+                     int k_off, int pad_left, int nT, int with_bias, int ordered, const float *__restrict__ wgt,
+                     T *__restrict__ dx) {
+    using S = DwTmaShape<T, V, KB, FUSED>;
+    const int padR = K - 1 - pad_left;  // the data gradient's left pad
     constexpr int NP = Pairs<V>::n;
-    constexpr int R = kDwR;
+    constexpr int R = S::R;
     launch_dependents();  // the finalize may be scheduled now; it waits for this grid to finish
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw);
@@ -225,13 +234,14 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDwStages; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kDwConsumers);
+            mbar_init(&empty[i], S::CONS);
         }
         fence_barrier_init();
     }
     __syncthreads();
     if (ordered) order.V = order.pv[B];
-    const int units = ordered ? order.V : B * nT;
+    // the fused pass also walks the wholly masked units: their dx frames are written as zeros
+    const int units = (ordered && !FUSED) ? order.V : B * nT;
     auto unit_at = [&](int u, int &b, int &t0, int &L) {
         if (ordered) {
             int tt, ctd;
@@ -276,7 +286,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
                     unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
                     tma_load_3d(st, &xmap, c0, t0 + k_off - pad_left, b, &full[s]);
-                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, t0, b, &full[s]);
+                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, FUSED ? t0 - padR : t0, b, &full[s]);
                 } else {
                     mbar_arrive(&full[s]);  // a wholly masked unit: nothing to read
                 }
@@ -286,6 +296,13 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     } else {  // consumer warp cw computes frames [t0 + cw R, t0 + cw R + R) of every unit
         const int cw = warp - 1;
         const bool active = c0 + lane * V < C;
+        float2 wv[FUSED ? KB : 1][NP];  // the data gradient's taps, this thread's channels
+        if constexpr (FUSED) {
+            if (active) {
+#pragma unroll
+                for (int k = 0; k < KB; ++k) load_param<V>(wgt + static_cast<int64_t>(k) * C + c0 + lane * V, wv[k]);
+            }
+        }
         int it = 0;
         for (int u = g; u < units && ok; u += G, ++it) {
             const int s = it % kDwStages;
@@ -295,9 +312,59 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
             ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph));
             if (!ok) break;
             const int tg = t0 + cw * R;
+            if constexpr (FUSED) {
+                // data gradient: dx[s] = [s < len_b] sum_k dz[s + pad_left - k] w[k] for this thread's
+                // R frames; tile row i holds dy frame tg - padR + i
+                if (active && tg < Tn) {
+                    T *dxp = dx + (static_cast<int64_t>(b) * Tn + tg) * C + c0 + lane * V;
+                    const int nr = Tn - tg < R ? Tn - tg : R;
+                    if (tg < L) {
+                        const unsigned char *zp = stages + static_cast<size_t>(s) * S::STAGE_BYTES +
+                                                  lane * V * sizeof(T) + (S::XROWS + cw * R) * S::ROWB;
+                        const int f0 = tg - padR;
+                        auto dxrun = [&](auto check) {
+                            constexpr bool CHECK = decltype(check)::value;
+                            float2 da[R][NP];
+#pragma unroll
+                            for (int r = 0; r < R; ++r)
+#pragma unroll
+                                for (int p = 0; p < NP; ++p) da[r][p] = make_float2(0.f, 0.f);
+#pragma unroll
+                            for (int i = 0; i < R + KB - 1; ++i) {
+                                Vec<T, V> v;
+                                v.r = *reinterpret_cast<const decltype(v.r) *>(zp + i * S::ROWB);
+                                if constexpr (CHECK) {
+                                    if (f0 + i < 0 || f0 + i >= L) v.zero();
+                                }
+                                float2 z[NP];
+                                v.to_f2(z);
+#pragma unroll
+                                for (int k = 0; k < KB; ++k) {
+                                    const int r = i - (KB - 1) + k;
+                                    if (r >= 0 && r < R) {
+#pragma unroll
+                                        for (int p = 0; p < NP; ++p) da[r][p] = ffma2(z[p], wv[k][p], da[r][p]);
+                                    }
+                                }
+                            }
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                if (r < nr) {
+                                    if (CHECK && tg + r >= L) Vec<T, V>::store_zero(dxp + static_cast<int64_t>(r) * C);
+                                    else Vec<T, V>::store(dxp + static_cast<int64_t>(r) * C, da[r]);
+                                }
+                            }
+                        };
+                        if (f0 >= 0 && f0 + R + KB - 1 <= L && nr == R) dxrun(std::false_type{});
+                        else dxrun(std::true_type{});
+                    } else {
+                        for (int r = 0; r < nr; ++r) Vec<T, V>::store_zero(dxp + static_cast<int64_t>(r) * C);
+                    }
+                }
+            }
             if (active && tg < L) {
                 const unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES + lane * V * sizeof(T);
-                const unsigned char *dp = st + (S::XROWS + cw * R) * S::ROWB;
+                const unsigned char *dp = st + (S::XROWS + (FUSED ? padR : 0) + cw * R) * S::ROWB;
                 const unsigned char *xp = st + (cw * R) * S::ROWB;
                 const int jb = tg + k_off - pad_left;  // frame of this thread's first x row
                 // CHECK = false: every dy and x row of the run is inside [0, len_b)
@@ -363,7 +430,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         float sum = red[e];
-        for (int r = 1; r < kDwConsumers; ++r) sum += red[static_cast<size_t>(r) * E + e];
+        for (int r = 1; r < S::CONS; ++r) sum += red[static_cast<size_t>(r) * E + e];
         red[e] = sum;
     }
     cg::cluster_group cluster = cg::this_cluster();
@@ -472,10 +539,10 @@ cudaError_t launch_pass(const DwArgs &a, int gp, int k_off, int with_bias, cudaS
 
 // Grid rows G and cluster size for the pipelined kernel: as many blocks per channel tile as
 // fit on the device at once, in clusters as large as that allows (fewer partial rows).
-template <typename T, int V, int KB>
+template <typename T, int V, int KB, bool FUSED = false>
 cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s) {
-    using S = DwTmaShape<T, V, KB>;
-    auto kern = conv1d_dw_tma_kernel<T, V, KB>;
+    using S = DwTmaShape<T, V, KB, FUSED>;
+    auto kern = conv1d_dw_tma_kernel<T, V, KB, FUSED>;
     const int ordered = (DW_DW_ORDERED && a.B <= kOrderMaxItems) ? 1 : 0;
     const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
     const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
@@ -489,7 +556,7 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     for (int c : {8, 4, 2, 1}) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(c, nCT);
-        q.blockDim = dim3(kDwTmaThreads);
+        q.blockDim = dim3(S::THREADS);
         q.dynamicSmemBytes = smem;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeClusterDimension;
@@ -517,7 +584,7 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     *gp_out = best_g / best_c;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(best_g, nCT);
-    cfg.blockDim = dim3(kDwTmaThreads);
+    cfg.blockDim = dim3(S::THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
@@ -529,11 +596,11 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     cfg.numAttrs = 1;
     CUtensorMap xmap, dmap;
     cudaError_t me = make_act_map(&xmap, a.x, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::XROWS);
-    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::TT);
+    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::DROWS);
     if (me != cudaSuccess) return me;
     return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, a.lengths, a.partials, static_cast<int>(a.B),
                               static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias,
-                              ordered);
+                              ordered, a.w, static_cast<T *>(a.dx));
 }
 
 template <typename T>
@@ -600,7 +667,62 @@ cudaError_t launch_dtype(const DwArgs &a, int *gp, cudaStream_t s) {
     return launch_partials<T, 1>(a, gp, s);
 }
 
+// The fused data + weight gradient pass; cudaErrorNotSupported when the pipelined kernel has no
+// instance for these sizes (the caller then runs the two gradients separately).
+template <typename T>
+cudaError_t launch_fused_partials(const DwArgs &a, int *gp, cudaStream_t s) {
+    if (!dw_tma_ok<T>(a) || a.vec_width < 2) return cudaErrorNotSupported;
+    if constexpr (sizeof(T) == 2) {
+        if (a.vec_width >= 4) {
+            switch (a.K) {
+                case 1: return launch_tma_pass<T, 4, 1, true>(a, 0, 1, gp, s);
+                case 2: return launch_tma_pass<T, 4, 2, true>(a, 0, 1, gp, s);
+                case 3: return launch_tma_pass<T, 4, 3, true>(a, 0, 1, gp, s);
+                case 4: return launch_tma_pass<T, 4, 4, true>(a, 0, 1, gp, s);
+                case 5: return launch_tma_pass<T, 4, 5, true>(a, 0, 1, gp, s);
+                case 7: return launch_tma_pass<T, 4, 7, true>(a, 0, 1, gp, s);
+                case 9: return launch_tma_pass<T, 4, 9, true>(a, 0, 1, gp, s);
+                default: break;
+            }
+        }
+    }
+    switch (a.K) {
+        case 1: return launch_tma_pass<T, 2, 1, true>(a, 0, 1, gp, s);
+        case 2: return launch_tma_pass<T, 2, 2, true>(a, 0, 1, gp, s);
+        case 3: return launch_tma_pass<T, 2, 3, true>(a, 0, 1, gp, s);
+        case 4: return launch_tma_pass<T, 2, 4, true>(a, 0, 1, gp, s);
+        case 5: return launch_tma_pass<T, 2, 5, true>(a, 0, 1, gp, s);
+        case 7: return launch_tma_pass<T, 2, 7, true>(a, 0, 1, gp, s);
+        case 9: return launch_tma_pass<T, 2, 9, true>(a, 0, 1, gp, s);
+        case 15: return launch_tma_pass<T, 2, 15, true>(a, 0, 1, gp, s);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t launch_finalize(const DwArgs &a, int gp, cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(a.K + 1) * a.C;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((n + 31) / 32));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, conv1d_dw_finalize_kernel, static_cast<const float *>(a.partials), a.dw, a.dbias,
+                              gp, a.K, static_cast<int64_t>(a.C));
+}
+
 }  // namespace
+
+cudaError_t conv1d_bwd_fused_launch(const DwArgs &a, cudaStream_t s) {
+    if (a.B == 0 || a.T == 0) return cudaErrorNotSupported;  // nothing to fuse
+    int gp = 0;
+    const cudaError_t e = a.bf16 ? launch_fused_partials<bf16>(a, &gp, s) : launch_fused_partials<float>(a, &gp, s);
+    if (e != cudaSuccess) return e;
+    return launch_finalize(a, gp, s);
+}
 
 unsigned int conv1d_dw_take_error() {
     unsigned int v = 0, zero = 0;
@@ -618,17 +740,7 @@ cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
     int gp = 0;
     cudaError_t e = a.bf16 ? launch_dtype<bf16>(a, &gp, s) : launch_dtype<float>(a, &gp, s);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((n + 31) / 32));
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, conv1d_dw_finalize_kernel, static_cast<const float *>(a.partials), a.dw, a.dbias,
-                              gp, a.K, static_cast<int64_t>(a.C));
+    return launch_finalize(a, gp, s);
 }
 
 }  // namespace dwk

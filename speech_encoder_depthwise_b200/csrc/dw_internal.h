@@ -35,6 +35,8 @@ struct DwArgs {
     int K, pad_left, bf16, vec_width;
     float *partials;      // workspace: [G][K+1][C] float32
     int G;                // partial rows (blocks per channel tile)
+    const float *w = nullptr;  // [K][C]: taps of the data gradient (fused backward only)
+    void *dx = nullptr;        // [B][T][C]: data gradient (fused backward only)
 };
 
 struct StreamArgs {
@@ -83,6 +85,8 @@ unsigned int conv1d_fwd_take_error();
 int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t C, int K);
 size_t conv1d_dw_workspace_bytes(int64_t B, int64_t T, int64_t C, int K);
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s);
+// dx and dW/dbias in one pass over dy; cudaErrorNotSupported when no fused instance fits.
+cudaError_t conv1d_bwd_fused_launch(const DwArgs &a, cudaStream_t s);
 unsigned int conv1d_dw_take_error();
 
 cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s);
