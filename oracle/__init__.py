@@ -88,8 +88,10 @@ class Oracle:
         lib.oracle_dw_subsample_fwd.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L,
                                                 ctypes.c_int, _D, _I]
         lib.oracle_dwconv1d_stream_fwd.argtypes = [_D, _D, _D, _D, _I, _L, _L, _L, _L, _D, _D]
+        lib.oracle_dw_subsample_bwd.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L, ctypes.c_int,
+                                                _D, _D, _D, _D]
         for f in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_dx", "oracle_dwconv1d_bwd_dw",
-                  "oracle_dw_subsample_fwd", "oracle_dwconv1d_stream_fwd"):
+                  "oracle_dw_subsample_fwd", "oracle_dwconv1d_stream_fwd", "oracle_dw_subsample_bwd"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -181,6 +183,23 @@ class Oracle:
             raise ValueError(f"oracle_dw_subsample_fwd rejected its arguments (rc={rc})")
         return out, ol
 
+    def dw_subsample_bwd(self, mel, w0, b0, w1, dout, lengths, causal):
+        """Gradients of sum(out * dout) of the fused subsampler with respect to w0, b0, w1 and b1:
+        returns (dw0 [3,3,C], db0 [C], dw1 [3,3,C], db1 [C])."""
+        mel = _f64(mel); w0 = _f64(w0); b0 = _f64(b0); w1 = _f64(w1); dout = _f64(dout)
+        B, T, F = mel.shape
+        C = w0.shape[-1]
+        T4, F4 = subsample_out_shape(T, F, causal)
+        assert dout.shape == (B, T4, F4, C)
+        ln = _lens(lengths, B)
+        dw0 = np.empty((3, 3, C)); db0 = np.empty(C); dw1 = np.empty((3, 3, C)); db1 = np.empty(C)
+        rc = self.lib.oracle_dw_subsample_bwd(_dp(mel), _dp(w0), _dp(b0), _dp(w1), _dp(dout), _ip(ln),
+                                              B, T, F, C, int(bool(causal)), _dp(dw0), _dp(db0),
+                                              _dp(dw1), _dp(db1))
+        if rc:
+            raise ValueError(f"oracle_dw_subsample_bwd rejected its arguments (rc={rc})")
+        return dw0, db0, dw1, db1
+
 
 def default() -> Oracle:
     """The oracle compiled from this package's source (built on first use)."""
@@ -204,6 +223,10 @@ def dwconv1d_fwd(x, w, bias, lengths, pad_left):
 
 def dwconv1d_stream_fwd(x, w, bias, cache, lengths):
     return default().dwconv1d_stream_fwd(x, w, bias, cache, lengths)
+
+
+def dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal):
+    return default().dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal)
 
 
 def dwconv1d_bwd_dx(dy, w, lengths, pad_left):

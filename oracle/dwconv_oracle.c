@@ -284,3 +284,94 @@ int oracle_dwconv1d_stream_fwd(const double *x, const double *w, const double *b
     }
     return 0;
 }
+
+/*
+ * Backward of the fused subsampler front (NeMo PR #16114, "What does this PR do ?": the fused
+ * kernels come with backward passes for training): given dout [B][T4][F4][C], the gradients of
+ * sum(out * dout) with respect to w0, b0, w1 and b1, the forward's stages taken backward:
+ *   doutm[i,j,c]         = [i < ceil(len/4)] dout[i,j,c]
+ *   db1[c]              += sum_{i,j} doutm[i,j,c]
+ *   dw1[p,q,c]          += sum_{i,j} doutm[i,j,c] hpad[2i+p, 2j+q, c]
+ *   dhpad[2i+p,2j+q,c]  += doutm[i,j,c] w1[p,q,c]              (transpose of conv_dw1)
+ *   dz[r,s,c]            = [r < ceil(len/2)] [z[r,s,c] > 0] dhpad[r+Pt, s+1, c]
+ *   db0[c]              += sum_{r,s} dz[r,s,c]
+ *   dw0[p,q,c]          += sum_{r,s} dz[r,s,c] melpad[2r+p, 2s+q]
+ * with z = b0 + conv0(melpad) the pre-activation (ReLU' = [z > 0]) and melpad, hpad as in the
+ * forward.  The mel input has no gradient (it is the network's input).  Every sum runs over
+ * items, then rows, then columns, in order.  Outputs [3][3][C], [C], [3][3][C], [C].
+ */
+int oracle_dw_subsample_bwd(const double *mel, const double *w0, const double *b0,
+                            const double *w1, const double *dout, const int32_t *lengths,
+                            int64_t B, int64_t T, int64_t F, int64_t C, int causal,
+                            double *dw0, double *db0, double *dw1, double *db1)
+{
+    if (B < 0 || T < 0 || F < 1 || C < 1) return 1;
+    const int64_t Pt = causal ? 2 : 1, Pb = causal ? 0 : 1;
+    const int64_t T2 = s2_out(T, Pt, Pb), F2 = s2_out(F, 1, 1);
+    const int64_t T4 = s2_out(T2, Pt, Pb), F4 = s2_out(F2, 1, 1);
+    const int64_t TP = T + Pt + Pb, FP = F + 2;
+    const int64_t HT = T2 + Pt + Pb, HF = F2 + 2;
+    memset(dw0, 0, sizeof(double) * (size_t)(9 * C));
+    memset(dw1, 0, sizeof(double) * (size_t)(9 * C));
+    memset(db0, 0, sizeof(double) * (size_t)C);
+    memset(db1, 0, sizeof(double) * (size_t)C);
+    double *melpad = (double *)malloc(sizeof(double) * (size_t)(TP * FP + 1));
+    double *z = (double *)malloc(sizeof(double) * (size_t)(T2 * F2 * C + 1));
+    double *hpad = (double *)malloc(sizeof(double) * (size_t)(HT * HF * C + 1));
+    double *dhpad = (double *)malloc(sizeof(double) * (size_t)(HT * HF * C + 1));
+    if (!melpad || !z || !hpad || !dhpad) {
+        free(melpad); free(z); free(hpad); free(dhpad);
+        return 2;
+    }
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        const int64_t L2 = ceil_half(L), L4 = ceil_half(L2);
+        for (int64_t r = 0; r < TP; ++r)
+            for (int64_t f = 0; f < FP; ++f) {
+                const int64_t t = r - Pt, ff = f - 1;
+                melpad[r * FP + f] = (ff >= 0 && ff < F && t >= 0 && t < L)
+                                         ? mel[(b * T + t) * F + ff] : 0.0;
+            }
+        memset(hpad, 0, sizeof(double) * (size_t)(HT * HF * C));
+        memset(dhpad, 0, sizeof(double) * (size_t)(HT * HF * C));
+        #pragma omp parallel for schedule(static)
+        for (int64_t c = 0; c < C; ++c) {
+            /* forward again: pre-activation z and the masked, ReLU'd h in hpad */
+            for (int64_t r = 0; r < T2; ++r)
+                for (int64_t s = 0; s < F2; ++s) {
+                    double a = b0[c];
+                    for (int64_t p = 0; p < 3; ++p)
+                        for (int64_t q = 0; q < 3; ++q) {
+                            const double tap = w0[(p * 3 + q) * C + c];
+                            a += melpad[(2 * r + p) * FP + (2 * s + q)] * tap;
+                        }
+                    z[(r * F2 + s) * C + c] = a;
+                    hpad[((r + Pt) * HF + (s + 1)) * C + c] = (r < L2 && a > 0.0) ? a : 0.0;
+                }
+            /* conv_dw1 backward: its weight and bias gradients, and dhpad */
+            for (int64_t i = 0; i < T4; ++i)
+                for (int64_t j = 0; j < F4; ++j) {
+                    const double dm = (i < L4) ? dout[((b * T4 + i) * F4 + j) * C + c] : 0.0;
+                    db1[c] += dm;
+                    for (int64_t p = 0; p < 3; ++p)
+                        for (int64_t q = 0; q < 3; ++q) {
+                            const int64_t at = ((2 * i + p) * HF + (2 * j + q)) * C + c;
+                            dw1[(p * 3 + q) * C + c] += dm * hpad[at];
+                            dhpad[at] += dm * w1[(p * 3 + q) * C + c];
+                        }
+                }
+            /* row mask and ReLU backward, then conv0's weight and bias gradients */
+            for (int64_t r = 0; r < T2; ++r)
+                for (int64_t s = 0; s < F2; ++s) {
+                    const double dzv = (r < L2 && z[(r * F2 + s) * C + c] > 0.0)
+                                           ? dhpad[((r + Pt) * HF + (s + 1)) * C + c] : 0.0;
+                    db0[c] += dzv;
+                    for (int64_t p = 0; p < 3; ++p)
+                        for (int64_t q = 0; q < 3; ++q)
+                            dw0[(p * 3 + q) * C + c] += dzv * melpad[(2 * r + p) * FP + (2 * s + q)];
+                }
+        }
+    }
+    free(melpad); free(z); free(hpad); free(dhpad);
+    return 0;
+}

@@ -145,6 +145,60 @@ def torch_subsample(mel, w0, b0, w1, b1, lengths, causal):
     return o.permute(0, 2, 3, 1).numpy(), np.array(L4, dtype=np.int32)
 
 
+def torch_subsample_grads(mel, w0, b0, w1, b1, dout, lengths, causal):
+    """Gradients of sum(out * dout) with respect to (w0, b0, w1, b1) by float64 autograd through
+    the torch formulation above (conv2d, relu, masks); returns numpy arrays in [3,3,C] / [C]."""
+    mel = torch.tensor(np.asarray(mel, np.float64))
+    B, T, F = mel.shape
+    C = np.asarray(w0).shape[-1]
+    pt, pb = (2, 0) if causal else (1, 1)
+    Ls = clamp_lengths(lengths, B, T)
+    W0 = torch.tensor(np.asarray(w0, np.float64)).permute(2, 0, 1)[:, None].clone().requires_grad_(True)
+    W1 = torch.tensor(np.asarray(w1, np.float64)).permute(2, 0, 1)[:, None].clone().requires_grad_(True)
+    B0 = torch.tensor(np.asarray(b0, np.float64)).requires_grad_(True)
+    B1 = torch.tensor(np.asarray(b1, np.float64)).requires_grad_(True)
+    m0 = (torch.arange(T)[None, :] < torch.tensor(Ls)[:, None]).double()
+    inp = Fnn.pad((mel * m0[:, :, None])[:, None], (1, 1, pt, pb))
+    h = torch.relu(Fnn.conv2d(inp, W0, B0, stride=2))
+    L2 = [(v + 1) // 2 for v in Ls]
+    h = h * (torch.arange(h.shape[2])[None, :] < torch.tensor(L2)[:, None]).double()[:, None, :, None]
+    o = Fnn.conv2d(Fnn.pad(h, (1, 1, pt, pb)), W1, B1, stride=2, groups=C)
+    L4 = [(v + 1) // 2 for v in L2]
+    o = o * (torch.arange(o.shape[2])[None, :] < torch.tensor(L4)[:, None]).double()[:, None, :, None]
+    loss = (o * torch.tensor(np.asarray(dout, np.float64)).permute(0, 3, 1, 2)).sum()
+    loss.backward()
+    g = lambda W: W.grad[:, 0].permute(1, 2, 0).numpy()
+    return g(W0), B0.grad.numpy(), g(W1), B1.grad.numpy()
+
+
+def subsample_bwd_checks(o, rng, B, T, F, C, causal):
+    """The oracle's subsampler backward against float64 autograd, and dw1 / db1 against exact
+    finite differences of <dout, out> (out is linear in w1 and b1).  Returns failure strings."""
+    fails = []
+    mel = rng.standard_normal((B, T, F)); w0 = rng.standard_normal((3, 3, C)) / 3
+    b0 = rng.standard_normal(C) * 0.3; w1 = rng.standard_normal((3, 3, C)) / 3; b1 = rng.standard_normal(C)
+    L = rng.integers(0, T + 1, size=B).astype(np.int32)
+    L[0] = T
+    out, _ = o.dw_subsample_fwd(mel, w0, b0, w1, b1, L, causal)
+    dout = rng.standard_normal(out.shape)
+    got = o.dw_subsample_bwd(mel, w0, b0, w1, dout, L, causal)
+    ref = torch_subsample_grads(mel, w0, b0, w1, b1, dout, L, causal)
+    for name, gv, rv in zip(("dw0", "db0", "dw1", "db1"), got, ref):
+        if gv.shape != rv.shape or rel_err(gv, rv) > 1e-11:
+            fails.append(f"autograd subsample bwd {name} {B, T, F, C, causal}")
+    base = float((out * dout).sum())
+    for (p, q, c) in ((0, 0, 0), (2, 1, C - 1), (1, 2, C // 2)):
+        w1e = w1.copy(); w1e[p, q, c] += 1.0
+        oe, _ = o.dw_subsample_fwd(mel, w0, b0, w1e, b1, L, causal)
+        if abs(float((oe * dout).sum()) - base - got[2][p, q, c]) > 1e-9 * max(1.0, abs(base)):
+            fails.append(f"finite difference dw1 {p, q, c}")
+    b1e = b1.copy(); b1e[0] += 1.0
+    oe, _ = o.dw_subsample_fwd(mel, w0, b0, w1, b1e, L, causal)
+    if abs(float((oe * dout).sum()) - base - got[3][0]) > 1e-9 * max(1.0, abs(base)):
+        fails.append("finite difference db1")
+    return fails
+
+
 def load_golden(name):
     with open(os.path.join(GOLDEN, name)) as f:
         return json.load(f)
@@ -278,4 +332,8 @@ def pin_battery(o):
     ry, rc = np_stream_fwd(x, w, bias, cache, L)
     if rel_err(y, ry) > 1e-12 or not np.array_equal(c, rc):
         fails.append("numpy stream")
+
+    # subsampler backward: autograd and exact finite differences
+    for causal in (False, True):
+        fails += subsample_bwd_checks(o, rng, 2, 13, 10, 3, causal)
     return fails

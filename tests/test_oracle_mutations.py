@@ -37,6 +37,17 @@ MUTANTS = {
     "stream output mask dropped": ("if (L > t) {", "if (T > t) {"),
     "stream taps reversed": ("acc += xcat[(t + k) * C + c] * w[k * C + c];",
                              "acc += xcat[(t + k) * C + c] * w[(K - 1 - k) * C + c];"),
+    "subsample bwd relu derivative dropped": ("(r < L2 && z[(r * F2 + s) * C + c] > 0.0)", "(r < L2)"),
+    "subsample bwd h mask dropped": ("(r < L2 && z[(r * F2 + s) * C + c] > 0.0)",
+                                     "(z[(r * F2 + s) * C + c] > 0.0)"),
+    "subsample bwd dout mask dropped": ("const double dm = (i < L4) ?", "const double dm = (i < T4) ?"),
+    "subsample bwd dw1 taps transposed": ("dw1[(p * 3 + q) * C + c] += dm * hpad[at];",
+                                          "dw1[(q * 3 + p) * C + c] += dm * hpad[at];"),
+    "subsample bwd recomputed conv0 taps transposed": ("const double tap = w0[(p * 3 + q) * C + c];",
+                                                       "const double tap = w0[(q * 3 + p) * C + c];"),
+    "subsample bwd mel not masked": ("(ff >= 0 && ff < F && t >= 0 && t < L)", "(ff >= 0 && ff < F && t >= 0 && t < T)"),
+    "subsample bwd dh taps flipped": ("dhpad[at] += dm * w1[(p * 3 + q) * C + c];",
+                                      "dhpad[at] += dm * w1[((2 - p) * 3 + q) * C + c];"),
 }
 
 
