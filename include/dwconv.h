@@ -213,6 +213,38 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
                              int64_t T, int64_t F, int64_t C, int causal,
                              dw_dtype_t out_dtype, dw_stream_t stream);
 
+/*
+ * dw_subsample_bwd_workspace_size - bytes of device workspace dw_subsample_bwd needs for these
+ * sizes (independent of pointers, dtype and device).
+ */
+size_t dw_subsample_bwd_workspace_size(int64_t B, int64_t T, int64_t F, int64_t C);
+
+/*
+ * dw_subsample_bwd - backward of dw_subsample_fwd (NeMo PR #16114, "Use Fused Kernels for
+ * Depthwise Striding Subsampler", section "What does this PR do ?": the fused kernels come with
+ * backward passes): the gradients of sum(out * dout) with respect to the weights and biases.
+ *
+ *   doutm[i,j,c] = [i < ceil(len_b/4)] dout[i,j,c];  z = b0 + conv0(melpad) (recomputed)
+ *   db1 = sum doutm;   dw1[p,q,c] = sum doutm[i,j,c] hpad[2i+p, 2j+q, c]
+ *   dh  = conv_dw1 transposed applied to doutm (taps w1);  dz = [r < ceil(len_b/2)] [z > 0] dh
+ *   db0 = sum dz;      dw0[p,q,c] = sum dz[r,s,c] melpad[2r+p, 2s+q]
+ * The mel input takes no gradient.  float32 accumulation; the per-block partial sums go to
+ * `workspace` and a second kernel adds them in a fixed order (reproducible for given sizes on a
+ * given GPU model).  No atomics.
+ *
+ *  mel, w0, b0, w1, lengths, B, T, F, C, causal: as dw_subsample_fwd (b1 is not needed)
+ *  dout         [B][T4][F4][C] dout_dtype (DW_BF16 or DW_F32), device
+ *  dw0, dw1     [3][3][C] float32, device, overwritten;  db0, db1 [C] float32, overwritten
+ *  workspace    device buffer of at least dw_subsample_bwd_workspace_size(B,T,F,C) bytes,
+ *               16-byte aligned; contents on entry are ignored
+ *  With no output frames the gradients are written as zeros (workspace may be NULL).
+ */
+dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0,
+                             const float *w1, const void *dout, const int32_t *lengths,
+                             float *dw0, float *db0, float *dw1, float *db1, int64_t B,
+                             int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t dout_dtype,
+                             void *workspace, size_t workspace_bytes, dw_stream_t stream);
+
 /* dw_status_string - a static, human-readable name for a status code. */
 const char *dw_status_string(dw_status_t status);
 

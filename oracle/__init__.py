@@ -90,8 +90,11 @@ class Oracle:
         lib.oracle_dwconv1d_stream_fwd.argtypes = [_D, _D, _D, _D, _I, _L, _L, _L, _L, _D, _D]
         lib.oracle_dw_subsample_bwd.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L, ctypes.c_int,
                                                 _D, _D, _D, _D]
+        lib.oracle_dw_subsample_bwd_kinks.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L, ctypes.c_int,
+                                                      ctypes.c_double, _D, _D]
         for f in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_dx", "oracle_dwconv1d_bwd_dw",
-                  "oracle_dw_subsample_fwd", "oracle_dwconv1d_stream_fwd", "oracle_dw_subsample_bwd"):
+                  "oracle_dw_subsample_fwd", "oracle_dwconv1d_stream_fwd", "oracle_dw_subsample_bwd",
+                  "oracle_dw_subsample_bwd_kinks"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -200,6 +203,21 @@ class Oracle:
             raise ValueError(f"oracle_dw_subsample_bwd rejected its arguments (rc={rc})")
         return dw0, db0, dw1, db1
 
+    def dw_subsample_bwd_kinks(self, mel, w0, b0, w1, dout, lengths, causal, delta):
+        """Bounds on how much dw0 / db0 can move when the ReLU decision flips at h pixels with
+        |z| <= delta: returns (kdw0 [3,3,C], kdb0 [C])."""
+        mel = _f64(mel); w0 = _f64(w0); b0 = _f64(b0); w1 = _f64(w1); dout = _f64(dout)
+        B, T, F = mel.shape
+        C = w0.shape[-1]
+        ln = _lens(lengths, B)
+        kdw0 = np.empty((3, 3, C)); kdb0 = np.empty(C)
+        rc = self.lib.oracle_dw_subsample_bwd_kinks(_dp(mel), _dp(w0), _dp(b0), _dp(w1), _dp(dout), _ip(ln),
+                                                    B, T, F, C, int(bool(causal)), float(delta),
+                                                    _dp(kdw0), _dp(kdb0))
+        if rc:
+            raise ValueError(f"oracle_dw_subsample_bwd_kinks rejected its arguments (rc={rc})")
+        return kdw0, kdb0
+
 
 def default() -> Oracle:
     """The oracle compiled from this package's source (built on first use)."""
@@ -227,6 +245,10 @@ def dwconv1d_stream_fwd(x, w, bias, cache, lengths):
 
 def dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal):
     return default().dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal)
+
+
+def dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, lengths, causal, delta):
+    return default().dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, lengths, causal, delta)
 
 
 def dwconv1d_bwd_dx(dy, w, lengths, pad_left):

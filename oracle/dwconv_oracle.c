@@ -29,6 +29,7 @@
  *    and conv_dw1 rows i >= ceil(len_b/4) are zero; time padding 1|1 (causal 2|0) and
  *    frequency padding 1|1 for both convs; padding values are zero.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -373,5 +374,60 @@ int oracle_dw_subsample_bwd(const double *mel, const double *w0, const double *b
         }
     }
     free(melpad); free(z); free(hpad); free(dhpad);
+    return 0;
+}
+
+/*
+ * Tolerance term for the subsampler backward at the ReLU kink.  The derivative [z > 0] is a
+ * decision taken on a floating-point z: where |z| is within rounding of 0, a float32 evaluation
+ * and this float64 one may decide differently, and each such h pixel moves dw0 by at most
+ * |dz| |melpad tap| and db0 by at most |dz|.  This returns those bounds summed over the h pixels
+ * with |z| <= delta (unmasked rows only), per tap and channel: kdw0 [3][3][C], kdb0 [C].
+ */
+int oracle_dw_subsample_bwd_kinks(const double *mel, const double *w0, const double *b0,
+                                  const double *w1, const double *dout, const int32_t *lengths,
+                                  int64_t B, int64_t T, int64_t F, int64_t C, int causal,
+                                  double delta, double *kdw0, double *kdb0)
+{
+    if (B < 0 || T < 0 || F < 1 || C < 1) return 1;
+    const int64_t Pt = causal ? 2 : 1, Pb = causal ? 0 : 1;
+    const int64_t T2 = s2_out(T, Pt, Pb), F2 = s2_out(F, 1, 1);
+    const int64_t T4 = s2_out(T2, Pt, Pb), F4 = s2_out(F2, 1, 1);
+    const int64_t TP = T + Pt + Pb, FP = F + 2;
+    memset(kdw0, 0, sizeof(double) * (size_t)(9 * C));
+    memset(kdb0, 0, sizeof(double) * (size_t)C);
+    double *melpad = (double *)malloc(sizeof(double) * (size_t)(TP * FP + 1));
+    if (!melpad) return 2;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        const int64_t L2 = ceil_half(L), L4 = ceil_half(L2);
+        for (int64_t r = 0; r < TP; ++r)
+            for (int64_t f = 0; f < FP; ++f) {
+                const int64_t t = r - Pt, ff = f - 1;
+                melpad[r * FP + f] = (t >= 0 && t < L && ff >= 0 && ff < F) ? mel[(b * T + t) * F + ff] : 0.0;
+            }
+        #pragma omp parallel for schedule(static)
+        for (int64_t c = 0; c < C; ++c) {
+            for (int64_t r = 0; r < T2 && r < L2; ++r)
+                for (int64_t s = 0; s < F2; ++s) {
+                    double zv = b0[c];
+                    for (int64_t t = 0; t < 9; ++t) zv += melpad[(2 * r + t / 3) * FP + (2 * s + t % 3)] * w0[t * C + c];
+                    if (fabs(zv) > delta) continue;
+                    double dh = 0.0;   /* the transposed conv_dw1 at (r, s) */
+                    for (int64_t p = 0; p < 3; ++p)
+                        for (int64_t q = 0; q < 3; ++q) {
+                            const int64_t ii = r + Pt - p, jj = s + 1 - q;
+                            if (ii < 0 || jj < 0 || ii % 2 || jj % 2) continue;
+                            const int64_t i = ii / 2, j = jj / 2;
+                            if (i >= T4 || i >= L4 || j >= F4) continue;
+                            dh += dout[((b * T4 + i) * F4 + j) * C + c] * w1[(p * 3 + q) * C + c];
+                        }
+                    kdb0[c] += fabs(dh);
+                    for (int64_t t = 0; t < 9; ++t)
+                        kdw0[t * C + c] += fabs(dh) * fabs(melpad[(2 * r + t / 3) * FP + (2 * s + t % 3)]);
+                }
+        }
+    }
+    free(melpad);
     return 0;
 }

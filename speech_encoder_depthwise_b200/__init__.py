@@ -21,7 +21,7 @@ __all__ = [
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
     "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd",
-    "dw_subsample_fwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
+    "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
 ]
 
 DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_WORKSPACE, DW_ERR_CUDA, DW_ERR_TIMEOUT = range(6)
@@ -49,6 +49,9 @@ SIGNATURES = {
     "dwconv1d_stream_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
+    "dw_subsample_bwd_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
+    "dw_subsample_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int,
+                                _int, _vp, ctypes.c_size_t, _vp]),
     "dw_status_string": (ctypes.c_char_p, [_int]),
     "dw_last_cuda_error": (_int, []),
     "dw_device_error": (_int, []),
@@ -232,3 +235,25 @@ def dw_subsample_fwd(mel, w0, b0, w1, b1, out, lengths, out_lengths, causal, str
                                 _dev(out_lengths, "out_lengths", torch.int32, (B,)), B, T, F, C,
                                 int(bool(causal)), _dtype_code(out), _stream(stream))
     _check("dw_subsample_fwd", st)
+
+
+def dw_subsample_bwd_workspace_size(B, T, F, C):
+    """Bytes of workspace ``dw_subsample_bwd`` needs for these sizes."""
+    return int(lib().dw_subsample_bwd_workspace_size(B, T, F, C))
+
+
+def dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, dw0, db0, dw1, db1, causal, workspace, stream=None):
+    """Gradients of sum(out * dout) of the fused subsampler into dw0/db0/dw1/db1 (float32)."""
+    import torch
+    B, T, F = mel.shape
+    C = w0.shape[-1]
+    T4, F4 = subsample_out_shape(T, F)
+    st = lib().dw_subsample_bwd(_dev(mel, "mel", torch.float32), _dev(w0, "w0", torch.float32, (3, 3, C)),
+                                _dev(b0, "b0", torch.float32, (C,)), _dev(w1, "w1", torch.float32, (3, 3, C)),
+                                _dev(dout, "dout", None, (B, T4, F4, C)), _dev(lengths, "lengths", torch.int32, (B,)),
+                                _dev(dw0, "dw0", torch.float32, (3, 3, C)), _dev(db0, "db0", torch.float32, (C,)),
+                                _dev(dw1, "dw1", torch.float32, (3, 3, C)), _dev(db1, "db1", torch.float32, (C,)),
+                                B, T, F, C, int(bool(causal)), _dtype_code(dout), _dev(workspace, "workspace"),
+                                workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                _stream(stream))
+    _check("dw_subsample_bwd", st)

@@ -227,6 +227,44 @@ dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
     return cuda_status(dwk::conv1d_dw_launch(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t dw_subsample_bwd_workspace_size(int64_t B, int64_t T, int64_t F, int64_t C) {
+    if (B < 0 || T < 0 || F < 1 || C < 1) return 0;
+    int64_t n = 0;
+    if (!mul3(B, T, F, &n) || !mul3(B, T, C, &n)) return 0;
+    return dwk::subsample_bwd_workspace_bytes(B, T, F, C);
+}
+
+dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0, const float *w1,
+                             const void *dout, const int32_t *lengths, float *dw0, float *db0, float *dw1,
+                             float *db1, int64_t B, int64_t T, int64_t F, int64_t C, int causal,
+                             dw_dtype_t dout_dtype, void *workspace, size_t workspace_bytes, dw_stream_t stream) {
+    if (!valid_dtype(dout_dtype)) return DW_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
+    if (C > kMaxChannels) return DW_ERR_UNSUPPORTED;
+    int64_t n = 0;
+    if (!mul3(B, T, F, &n)) return DW_ERR_INVALID_ARG;
+    if (!dw0 || !db0 || !dw1 || !db1) return DW_ERR_INVALID_ARG;
+    auto s2 = [](int64_t v) -> int64_t { return v >= 1 ? (v - 1) / 2 + 1 : 0; };
+    const int64_t T4 = s2(s2(T)), F4 = s2(s2(F));
+    int64_t nout = 0;
+    if (!mul3(B, T4 * F4, C, &nout)) return DW_ERR_INVALID_ARG;
+    dwk::SubsampleBwdArgs a;
+    a.mel = mel; a.w0 = w0; a.b0 = b0; a.w1 = w1; a.dout = dout; a.lengths = lengths;
+    a.dw0 = dw0; a.db0 = db0; a.dw1 = dw1; a.db1 = db1;
+    a.partials = static_cast<float *>(workspace);
+    a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.bf16_dout = dout_dtype == DW_BF16;
+    if (nout > 0) {
+        if (!mel || !w0 || !b0 || !w1 || !dout) return DW_ERR_INVALID_ARG;
+        const size_t need = dwk::subsample_bwd_workspace_bytes(B, T, F, C);
+        if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return DW_ERR_WORKSPACE;
+        const size_t g = static_cast<size_t>(9) * C * sizeof(float), gb = static_cast<size_t>(C) * sizeof(float);
+        if (overlaps(workspace, need, dw0, g) || overlaps(workspace, need, dw1, g) ||
+            overlaps(workspace, need, db0, gb) || overlaps(workspace, need, db1, gb))
+            return DW_ERR_INVALID_ARG;
+    }
+    return cuda_status(dwk::subsample_bwd_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
 dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0, const float *w1,
                              const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
                              int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,

@@ -92,6 +92,19 @@ unsigned int conv1d_dw_take_error();
 cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s);
 
 cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
+
+struct SubsampleBwdArgs {
+    const float *mel, *w0, *b0, *w1;
+    const void *dout;             // [B][T4][F4][C] bf16 or float32
+    const int32_t *lengths;
+    float *dw0, *db0, *dw1, *db1;  // [3][3][C], [C], [3][3][C], [C]
+    float *partials;              // workspace: [rows][20][C]
+    int64_t B, T, F, C;
+    int causal, bf16_dout;
+};
+int subsample_bwd_partial_rows(int64_t B, int64_t T, int64_t F);
+size_t subsample_bwd_workspace_bytes(int64_t B, int64_t T, int64_t F, int64_t C);
+cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s);
 // Tensor-core subsampler: usable when the output rows are 16-byte aligned (C * element size a
 // multiple of 16, aligned base); the SIMT kernel serves every other case.
 bool subsample_tc_eligible(const SubsampleArgs &a);

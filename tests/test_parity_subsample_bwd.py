@@ -1,0 +1,105 @@
+"""GPU parity of the subsampler backward (dw_subsample_bwd: the gradients of sum(out * dout) with
+respect to w0, b0, w1, b1) against the fp64 CPU oracle, through the C ABI.
+
+Bars: dw1 and db1 within 1e-5 * RMS(oracle) (float32 accumulation).  dw0 and db0 within
+1e-5 * RMS(oracle) plus the oracle's kink budget: the ReLU derivative [z > 0] is decided on a
+recomputed float32 z, so at h pixels where |z| is within rounding of 0 (|z| <= 1e-5 here) the GPU
+and the float64 oracle may decide differently; each such pixel can move dw0[p,q,c] by at most
+|dz| |mel tap| and db0[c] by |dz|, and the budget is that sum per element.
+
+Workloads: the benchmark's subsampler shape (mel 16x3000x80, C=256, lengths in [1500, 3000]) with
+bf16 dout, symmetric and causal; small cases with T and F from 1, odd C, C past one channel
+group, float32 dout, misaligned dout, len 0, no lengths; bitwise reproducibility.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speech_encoder_depthwise_b200 as dw
+from gpuhelp import Guarded, dev, max_abs, rms
+from synth import bf16_round, subsample_inputs
+
+pytestmark = pytest.mark.gpu
+KINK = 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    from speech_encoder_depthwise_b200 import build
+    build.build()
+    dw.lib()
+
+
+def gpu_bwd(d, dout, causal, dtype=torch.bfloat16, offset=0, with_lengths=True):
+    B, T, F = d["mel"].shape
+    C = d["w0"].shape[-1]
+    g = Guarded(dout.shape, dtype, offset=offset)
+    g.t.copy_(torch.from_numpy(np.ascontiguousarray(dout)).to(dtype))
+    outs = [Guarded((3, 3, C), torch.float32), Guarded((C,), torch.float32),
+            Guarded((3, 3, C), torch.float32), Guarded((C,), torch.float32)]
+    n = dw.dw_subsample_bwd_workspace_size(B, T, F, C)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    dw.dw_subsample_bwd(dev(d["mel"]), dev(d["w0"]), dev(d["b0"]), dev(d["w1"]), g.t,
+                        dev(d["lengths"]) if with_lengths else None, *[o.t for o in outs], causal, ws)
+    torch.cuda.synchronize()
+    for o in outs + [g]:
+        o.check_slack()
+    return [o.numpy() for o in outs]
+
+
+def check(d, dout, causal, got, with_lengths=True):
+    L = d["lengths"] if with_lengths else None
+    ref = oracle.dw_subsample_bwd(d["mel"], d["w0"], d["b0"], d["w1"], dout, L, causal)
+    kdw0, kdb0 = oracle.dw_subsample_bwd_kinks(d["mel"], d["w0"], d["b0"], d["w1"], dout, L, causal, KINK)
+    for name, g, r, k in zip(("dw0", "db0", "dw1", "db1"), got, ref, (kdw0, kdb0, 0.0, 0.0)):
+        bound = 1e-5 * max(rms(r), 1e-6) + k
+        err = np.abs(g - r)
+        assert np.all(err <= bound), f"{name}: max error {err.max():.3g}, bound {np.min(bound):.3g}..."
+
+
+def rounded_dout(d, causal, seed, dtype="bf16"):
+    B, T, F = d["mel"].shape
+    C = d["w0"].shape[-1]
+    T4, F4 = oracle.subsample_out_shape(T, F, causal)
+    g = np.random.default_rng(seed).standard_normal((B, T4, F4, C)).astype(np.float32)
+    return bf16_round(g) if dtype == "bf16" else g
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_workload(causal):
+    d = subsample_inputs(16, 3000, 80, 256, len_range=(1500, 3000), seed=3)
+    dout = rounded_dout(d, causal, 30 + causal)
+    check(d, dout, causal, gpu_bwd(d, dout, causal))
+
+
+SMALL = [(1, 1, 1, 1), (2, 5, 7, 3), (3, 9, 80, 100), (2, 37, 81, 300), (1, 130, 16, 128), (2, 33, 9, 1),
+         (2, 64, 80, 257)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,T,F,C", SMALL)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_small_cases(B, T, F, C, causal, dtype):
+    d = subsample_inputs(B, T, F, C, len_range=(0, T), seed=T * 100 + F + C)
+    d["lengths"][0] = T
+    if B > 2:
+        d["lengths"][1] = 0
+    dout = rounded_dout(d, causal, T + C, dtype)
+    got = gpu_bwd(d, dout, causal, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
+    check(d, dout, causal, got)
+
+
+def test_misaligned_dout_and_no_lengths():
+    d = subsample_inputs(2, 50, 20, 64, len_range=(50, 50), seed=5)
+    dout = rounded_dout(d, False, 6)
+    check(d, dout, False, gpu_bwd(d, dout, False, offset=1, with_lengths=False), with_lengths=False)
+
+
+def test_results_are_bitwise_reproducible():
+    d = subsample_inputs(4, 400, 80, 256, len_range=(200, 400), seed=8)
+    dout = rounded_dout(d, False, 9)
+    a = gpu_bwd(d, dout, False)
+    b = gpu_bwd(d, dout, False)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
