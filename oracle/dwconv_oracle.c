@@ -404,7 +404,7 @@ int oracle_dw_subsample_bwd_kinks(const double *mel, const double *w0, const dou
         for (int64_t r = 0; r < TP; ++r)
             for (int64_t f = 0; f < FP; ++f) {
                 const int64_t t = r - Pt, ff = f - 1;
-                melpad[r * FP + f] = (t >= 0 && t < L && ff >= 0 && ff < F) ? mel[(b * T + t) * F + ff] : 0.0;
+                melpad[r * FP + f] = (t < L && t >= 0 && ff < F && ff >= 0) ? mel[(b * T + t) * F + ff] : 0.0;
             }
         #pragma omp parallel for schedule(static)
         for (int64_t c = 0; c < C; ++c) {
