@@ -256,6 +256,46 @@ def measure_bwd(dw, dev, hbm):
             "alg_bytes": by, "separate_dx_plus_dw_us": sep, "dx_max_abs_err_item0": err}
 
 
+def measure_sub_bwd(dw, dev, hbm, fp32_tflops):
+    """Subsampler backward (a NEXT row, outside the step) on the benchmark's subsampler shape,
+    mel 16x3000x80, C=256, bf16 dout, symmetric: µs, and the roofline of its algorithmic work:
+    mel at valid frames + dout read, 18 flop per valid h element (conv0 recomputed, dw0) and
+    18 per valid output element (dh, dw1)."""
+    import torch
+    from synth import subsample_inputs
+    B, T, F, C = SUB["B"], SUB["T"], SUB["F"], SUB["C"]
+    ss = subsample_inputs(B, T, F, C, len_range=SUB["len_range"], seed=SUB["seed"])
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    mel, w0, b0, w1, ln = t(ss["mel"]), t(ss["w0"]), t(ss["b0"]), t(ss["w1"]), t(ss["lengths"], torch.int32)
+    T4, F4 = dw.subsample_out_shape(T, F)
+    gen = torch.Generator(device=dev).manual_seed(31)
+    douts = [torch.randn(B, T4, F4, C, device=dev, generator=gen).to(torch.bfloat16) for _ in range(3)]
+    g = [torch.empty(3, 3, C, device=dev), torch.empty(C, device=dev), torch.empty(3, 3, C, device=dev),
+         torch.empty(C, device=dev)]
+    ws = torch.empty(dw.dw_subsample_bwd_workspace_size(B, T, F, C), dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        for i in range(3):
+            dw.dw_subsample_bwd(mel, w0, b0, w1, douts[i], ln, *g, SUB["causal"], ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for i in range(20):
+            dw.dw_subsample_bwd(mel, w0, b0, w1, douts[i % 3], ln, *g, SUB["causal"], ws)
+        e1.record(s)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) / 20 * 1e3
+    L = np.clip(ss["lengths"], 0, T)
+    L2 = (L + 1) // 2
+    L4 = (L2 + 1) // 2
+    F2 = (F + 1) // 2
+    by = int(L.sum()) * F * 4 + B * T4 * F4 * C * 2
+    fl = int(L2.sum()) * F2 * C * 36 + int(L4.sum()) * F4 * C * 36
+    t_roof = max(by / (hbm * 1e9), fl / (fp32_tflops * 1e12))
+    return {"workload": "subsampler backward, mel 16x3000x80 -> C256, bf16 dout, sym, len U[1500,3000]",
+            "us": us, "TFLOP_per_s": fl / (us * 1e-6) / 1e12, "roofline_frac": t_roof / (us * 1e-6),
+            "alg_bytes": by, "alg_flops": fl}
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -581,7 +621,8 @@ def main():
         ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
-        next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm), "dwconv1d_bwd": measure_bwd(dw, dev, hbm)}
+        next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm), "dwconv1d_bwd": measure_bwd(dw, dev, hbm),
+                     "dw_subsample_bwd": measure_sub_bwd(dw, dev, hbm, fp32_tflops)}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
             v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)

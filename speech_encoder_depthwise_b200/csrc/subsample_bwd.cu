@@ -13,9 +13,10 @@
 // and db1 += doutm[r/2, s/2] at even (r, s) (each output pixel exactly once).  Rows at or past
 // ceil(len/2) contribute nothing: their h and dz are zero and the outputs they feed are masked.
 //
-// A persistent grid walks spatial tiles (item, 8 h rows, up to 40 h columns); a thread owns a
+// A persistent grid walks spatial tiles (item, 8 h rows, up to 20 h columns); a thread owns a
 // channel pair and keeps all twenty gradient pairs in registers for its whole share of the
-// tiles; the tile's mel window is staged once in shared memory as {m, m} pairs.  Block b of a
+// tiles.  Per tile the mel window is staged once in shared memory as {m, m} pairs, and every
+// thread stages its own window of dout values (requested together, so their latency overlaps).  Block b of a
 // channel group writes one partial row; a finalize kernel adds the rows in a fixed order, so the
 // results are reproducible for given sizes on a given GPU model.
 #include "dw_internal.h"
@@ -25,11 +26,21 @@ namespace {
 
 constexpr int kSbThreads = 128;                      // one thread per channel pair
 constexpr int kSbRT = 8;                             // h rows per spatial tile
-constexpr int kSbST = 40;                            // h columns per spatial tile
+constexpr int kSbST = 20;                            // h columns per spatial tile
 constexpr int kSbMR = 2 * kSbRT + 1;                 // staged mel rows
 constexpr int kSbMC = 2 * kSbST + 1;                 // staged mel columns
 constexpr int kSbSlots = 20;                         // dw0[9], db0, dw1[9], db1
 constexpr int kSbMaxRows = 592;                      // partial rows per channel group (at most)
+constexpr int kSbNRW = kSbRT / 2 + 2;                // output rows a tile's h rows read
+constexpr int kSbNCW = kSbST / 2 + 3;                // output columns a tile's h columns read
+
+// A thread's staged dout value: a bf16 pair as one word, or a float pair.
+template <typename TD> struct DWord { using type = float2; };
+template <> struct DWord<bf16> { using type = uint32_t; };
+__device__ __forceinline__ float2 to_pair(float2 v) { return v; }
+__device__ __forceinline__ float2 to_pair(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
+__device__ __forceinline__ void from_pair(float2 v, float2 &w) { w = v; }
+__device__ __forceinline__ void from_pair(float2 v, uint32_t &w) { w = pack_bf16x2(v.x, v.y); }
 
 template <typename TD, bool VEC>
 __device__ __forceinline__ float2 load_dout(const TD *p, bool two) {
@@ -57,20 +68,19 @@ __device__ __forceinline__ float2 relu_mask(float2 z, float2 v) {  // [z > 0] v,
 // (tap q = 0), 2k (q = 1) and 2k+1 (q = 2), so each dout value is loaded once and the next
 // column's values are loaded one step ahead.  EVEN: r + Pt even, so output rows iA = (r+Pt)/2
 // (tap p = 0) and iB = iA - 1 (p = 2) feed the row; otherwise only iA = (r+Pt-1)/2 (p = 1).
-template <typename TD, bool VEC, bool EVEN>
-__device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt, int F4, int i4, bool two,
-                                         const TD *db, int C, const float2 (*sm)[kSbMC], const float2 (&W0)[9],
-                                         const float2 (&W1)[9], float2 bias0, float2 (&gw0)[9], float2 (&gw1)[9],
-                                         float2 &gb0, float2 &gb1) {
+template <typename W, bool EVEN>
+__device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt, const W *win, int iLo, int kLo,
+                                         const float2 (*sm)[kSbMC], const float2 (&W0)[9], const float2 (&W1)[9],
+                                         float2 bias0, float2 (&gw0)[9], float2 (&gw1)[9], float2 &gb0,
+                                         float2 &gb1) {
     constexpr int pA = EVEN ? 0 : 1;
     const int iA = EVEN ? (r + Pt) >> 1 : (r + Pt - 1) >> 1, iB = iA - 1;
-    const bool okA = iA >= 0 && iA < i4, okB = EVEN && iB >= 0 && iB < i4;
-    const TD *rowA = db + static_cast<int64_t>(iA) * F4 * C, *rowB = db + static_cast<int64_t>(iB) * F4 * C;
+    // this thread's staged window: [output row - iLo][output column - kLo], kSbThreads apart
+    const W *rowA = win + (iA - iLo) * kSbNCW * kSbThreads, *rowB = win + (iB - iLo) * kSbNCW * kSbThreads;
     const float2 zero = make_float2(0.f, 0.f);
     auto load = [&](int k, float2 &a, float2 &bb) {
-        const bool in = k >= 0 && k < F4;
-        a = (in && okA) ? load_dout<TD, VEC>(rowA + static_cast<int64_t>(k) * C, two) : zero;
-        bb = (in && okB) ? load_dout<TD, VEC>(rowB + static_cast<int64_t>(k) * C, two) : zero;
+        a = to_pair(rowA[(k - kLo) * kSbThreads]);
+        bb = EVEN ? to_pair(rowB[(k - kLo) * kSbThreads]) : zero;
     };
     // one h pixel (r, s) given its dh taps: recompute z, then every gradient term it owns
     auto pixel = [&](int s, float2 dh, const float2 (&d)[4], const int (&tap)[4], int nt, float2 db1v, bool own_b1) {
@@ -97,7 +107,8 @@ __device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt
 #pragma unroll
         for (int t = 0; t < 9; ++t) gw0[t] = ffma2(dz, mv[t], gw0[t]);
     };
-    const int k0 = S0 >> 1, k1 = send >> 1;  // h columns [S0, send) lie in output columns k0 .. k1
+    const int k0 = S0 >> 1, k1 = send >> 1;  // h columns [S0, send) lie in output columns k0 .. k1;
+                                             // the window holds columns k0 - 1 .. k1 + 1
     float2 pa, pb, ca, cb, na, nb;          // output column k-1, k and k+1 of rows iA, iB
     load(k0 - 1, pa, pb);
     load(k0, ca, cb);
@@ -130,7 +141,10 @@ dw_subsample_bwd_kernel(const float *__restrict__ mel, const float *__restrict__
                         const float *__restrict__ w1, const TD *__restrict__ dout,
                         const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int F,
                         int C, int T2, int F2, int T4, int F4, int Pt, int nRT, int nST, int nCG) {
+    using W = typename DWord<TD>::type;
     __shared__ __align__(16) float2 sm[kSbMR][kSbMC];
+    extern __shared__ __align__(16) unsigned char dyn_smem[];
+    W *win = reinterpret_cast<W *>(dyn_smem) + threadIdx.x;  // this thread's dout window
     const int cg = blockIdx.x % nCG, g = blockIdx.x / nCG, G = gridDim.x / nCG;
     const int c = (cg * kSbThreads + threadIdx.x) * 2;  // this thread's first channel
     const bool act = c < C, two = c + 1 < C;
@@ -167,15 +181,28 @@ dw_subsample_bwd_kernel(const float *__restrict__ mel, const float *__restrict__
         }
         __syncthreads();
         if (!act) continue;
+        // this thread's dout values for the tile, all requested at once: output rows
+        // iLo .. iLo + kSbNRW - 1 and columns kLo .. kLo + kSbNCW - 1, zero where masked or outside
         const TD *db = dout + static_cast<int64_t>(b) * T4 * F4 * C + c;
         const int i4 = L4 < T4 ? L4 : T4;  // output rows below this are unmasked
+        const int iLo = (R0 + Pt - 2) >> 1, kLo = (S0 >> 1) - 1;
+#pragma unroll 2
+        for (int rr = 0; rr < kSbNRW; ++rr) {
+            const int i = iLo + rr;
+#pragma unroll
+            for (int cc = 0; cc < kSbNCW; ++cc) {
+                const int k = kLo + cc;
+                float2 v = make_float2(0.f, 0.f);
+                if (i >= 0 && i < i4 && k >= 0 && k < F4) v = load_dout<TD, VEC>(db + (static_cast<int64_t>(i) * F4 + k) * C, two);
+                from_pair(v, win[(rr * kSbNCW + cc) * kSbThreads]);
+            }
+        }
         for (int r = R0; r < rend; ++r) {
             // h row r receives taps p with r + Pt - p even: rows iA (p = 0 or 1) and, for p = 0,
             // also iB = iA - 1 with p = 2
-            if (((r + Pt) & 1) == 0) row_pass<TD, VEC, true>(r, R0, S0, send, Pt, F4, i4, two, db, C, sm, W0, W1, bias0,
-                                                              gw0, gw1, gb0, gb1);
-            else row_pass<TD, VEC, false>(r, R0, S0, send, Pt, F4, i4, two, db, C, sm, W0, W1, bias0, gw0, gw1,
-                                          gb0, gb1);
+            if (((r + Pt) & 1) == 0) row_pass<W, true>(r, R0, S0, send, Pt, win, iLo, kLo, sm, W0, W1, bias0, gw0, gw1,
+                                                        gb0, gb1);
+            else row_pass<W, false>(r, R0, S0, send, Pt, win, iLo, kLo, sm, W0, W1, bias0, gw0, gw1, gb0, gb1);
         }
     }
     if (!act) return;
@@ -257,18 +284,39 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
     const int nRT = static_cast<int>((T2 + kSbRT - 1) / kSbRT), nST = static_cast<int>((F2 + kSbST - 1) / kSbST);
     const int64_t nCG = (a.C + 2 * kSbThreads - 1) / (2 * kSbThreads);
     int G = subsample_bwd_partial_rows(a.B, a.T, a.F);
-    // one wave of blocks over the device (4 per SM), never more than the workspace holds
-    const int64_t per_group = (static_cast<int64_t>(sm_count()) * 4) / nCG;
+    // one wave of resident blocks over the device, never more than the workspace holds
+    const size_t dsmem = kSbNRW * kSbNCW * kSbThreads * (a.bf16_dout ? sizeof(uint32_t) : sizeof(float2));
+    int per_sm = 0;
+    {
+        const cudaError_t ea = ensure_smem_attr(a.bf16_dout ? reinterpret_cast<const void *>(dw_subsample_bwd_kernel<bf16, true>)
+                                                            : reinterpret_cast<const void *>(dw_subsample_bwd_kernel<float, true>),
+                                                static_cast<int>(dsmem));
+        if (ea != cudaSuccess) return ea;
+    }
+    const void *kern = a.bf16_dout ? reinterpret_cast<const void *>(dw_subsample_bwd_kernel<bf16, true>)
+                                   : reinterpret_cast<const void *>(dw_subsample_bwd_kernel<float, true>);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSbThreads, dsmem) != cudaSuccess || per_sm < 1) {
+        (void)cudaGetLastError();
+        per_sm = 2;
+    }
+    const int64_t per_group = (static_cast<int64_t>(sm_count()) * per_sm) / nCG;
     if (per_group >= 1 && per_group < G) G = static_cast<int>(per_group);
     const int64_t grid = static_cast<int64_t>(G) * nCG;
     if (grid > kMaxGrid || T4 * F4 * a.C >= (1LL << 31) || a.T * a.F >= (1LL << 31)) return cudaErrorInvalidConfiguration;
     const size_t es = a.bf16_dout ? 2 : 4;
+    cudaError_t e = cudaSuccess;
     const bool vec = (a.C % 2) == 0 && (reinterpret_cast<uintptr_t>(a.dout) % (2 * es)) == 0;
 #define DW_SB_LAUNCH(TD, VV)                                                                                 \
-    dw_subsample_bwd_kernel<TD, VV><<<static_cast<unsigned>(grid), kSbThreads, 0, s>>>(                     \
+    do {                                                                                                     \
+    e = ensure_smem_attr(reinterpret_cast<const void *>(dw_subsample_bwd_kernel<TD, VV>),                    \
+                         static_cast<int>(kSbNRW * kSbNCW * kSbThreads * sizeof(typename DWord<TD>::type)));   \
+    if (e != cudaSuccess) return e;                                                                          \
+    dw_subsample_bwd_kernel<TD, VV><<<static_cast<unsigned>(grid), kSbThreads,                              \
+                                      kSbNRW * kSbNCW * kSbThreads * sizeof(typename DWord<TD>::type), s>>>(  \
         a.mel, a.w0, a.b0, a.w1, static_cast<const TD *>(a.dout), a.lengths, a.partials, static_cast<int>(a.B), \
         static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(T2),          \
-        static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt, nRT, nST, static_cast<int>(nCG))
+        static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt, nRT, nST, static_cast<int>(nCG)); \
+    } while (0)
     if (a.bf16_dout) {
         if (vec) DW_SB_LAUNCH(bf16, true);
         else DW_SB_LAUNCH(bf16, false);
@@ -277,7 +325,7 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
         else DW_SB_LAUNCH(float, false);
     }
 #undef DW_SB_LAUNCH
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t E = static_cast<int64_t>(kSbSlots) * a.C;
     dw_subsample_bwd_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(
