@@ -230,6 +230,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     // every (item, run) pair when B is too large for the order's shared-memory tables
     int *ord_mem = reinterpret_cast<int *>(stages + S::BODY);
     TileOrder order{ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), B, nT, 1, 0};
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDwStages; ++i) {
@@ -592,8 +593,11 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     at[0].val.clusterDim.x = best_c;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cudaLaunchAttribute at2[2] = {at[0], {}};
+    at2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at2[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at2;
+    cfg.numAttrs = 2;
     CUtensorMap xmap, dmap;
     cudaError_t me = make_act_map(&xmap, a.x, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::XROWS);
     if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::DROWS);

@@ -182,6 +182,7 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     const int my_ct = static_cast<int>(blockIdx.x % nC);
     const int q0 = static_cast<int>(blockIdx.x / nC), qstride = static_cast<int>(gridDim.x / nC);
     const int nq = ntiles / nC;  // positions per channel tile
+    launch_dependents();  // the next kernel in the stream may start its own set-up
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTmaStages; ++i) {
             mbar_init(&full[i], 1);
@@ -190,6 +191,7 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
         fence_barrier_init();
     }
     __syncthreads();
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     if (warp == 0) {  // producer warp: one elected lane, one tensor copy per tile
         if (lane == 0) prefetch_tmap(&xmap);
         int it = 0;
@@ -438,10 +440,21 @@ cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     if (grid > ntiles) grid = ntiles;
     grid = grid / nC * nC;  // whole channel tiles per block walk
     if (grid < nC) grid = nC;
-    kern<<<static_cast<unsigned>(grid), kTmaThreads, S::SMEM, s>>>(
-        xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.B), static_cast<int>(a.T),
-        static_cast<int>(a.C), a.pad_left, a.flip, nT, nC, static_cast<int>(ntiles));
-    return cudaGetLastError();
+    // programmatic dependent launch: the blocks come up while the previous kernel drains and
+    // wait for it (grid_dependency_wait) before touching memory
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kTmaThreads);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.B),
+                              static_cast<int>(a.T), static_cast<int>(a.C), a.pad_left, a.flip, nT, nC,
+                              static_cast<int>(ntiles));
 }
 
 // The pipelined kernel copies whole frame rows in 16-byte units: C * sizeof(T) a multiple of

@@ -289,6 +289,8 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
     constexpr int kStElems = kRO * kJO * 128;
 
     // ------------------------------------------------------------ set-up
+    launch_dependents();     // the next kernel in the stream may start its own set-up
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&patch_full[i], kPatchThreads);
@@ -753,7 +755,17 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
         const int bytes = TcLayout<TO, CTG>::alloc;                                                            \
         e = ensure_smem_attr(reinterpret_cast<const void *>(kern), bytes);                                    \
         if (e != cudaSuccess) return e;                                                                        \
-        kern<<<static_cast<unsigned>(grid), kThreads, bytes, s>>>(                                             \
+        cudaLaunchConfig_t cfg = {};                                                                           \
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));                                                       \
+        cfg.blockDim = dim3(kThreads);                                                                         \
+        cfg.dynamicSmemBytes = bytes;                                                                          \
+        cfg.stream = s;                                                                                        \
+        cudaLaunchAttribute at[1];                                                                             \
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;                                        \
+        at[0].val.programmaticStreamSerializationAllowed = 1;                                                 \
+        cfg.attrs = at;                                                                                        \
+        cfg.numAttrs = 1;                                                                                      \
+        e = cudaLaunchKernelEx(&cfg, kern,                                                                     \
             a.mel, a.w0, a.b0, a.w1, a.b1, a.lengths, a.out_lengths, map, static_cast<int>(a.B),               \
             static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(F2), Pt,     \
             static_cast<int>(nIP), static_cast<int>(nJB), static_cast<int>(nG));                               \
@@ -766,6 +778,7 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
         else DW_TC_LAUNCH(float, 1);
     }
 #undef DW_TC_LAUNCH
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
