@@ -92,9 +92,13 @@ class Oracle:
                                                 _D, _D, _D, _D]
         lib.oracle_dw_subsample_bwd_kinks.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L, ctypes.c_int,
                                                       ctypes.c_double, _D, _D]
+        lib.oracle_dwconv2d_fwd.argtypes = [_D, _D, _D, _I] + [_L] * 11 + [_D, _I]
+        lib.oracle_dwconv2d_bwd_dx.argtypes = [_D, _D, _I] + [_L] * 11 + [_D]
+        lib.oracle_dwconv2d_bwd_dw.argtypes = [_D, _D, _I] + [_L] * 11 + [_D, _D]
         for f in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_dx", "oracle_dwconv1d_bwd_dw",
                   "oracle_dw_subsample_fwd", "oracle_dwconv1d_stream_fwd", "oracle_dw_subsample_bwd",
-                  "oracle_dw_subsample_bwd_kinks"):
+                  "oracle_dw_subsample_bwd_kinks", "oracle_dwconv2d_fwd", "oracle_dwconv2d_bwd_dx",
+                  "oracle_dwconv2d_bwd_dw"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -218,6 +222,60 @@ class Oracle:
             raise ValueError(f"oracle_dw_subsample_bwd_kinks rejected its arguments (rc={rc})")
         return kdw0, kdb0
 
+    def dwconv2d_fwd(self, x, w, bias, lengths, stride, pads):
+        """Depthwise conv2d, channels-last x [B,T,F,C], w [KT,KF,C]; stride (st, sf), pads (pt, pb, pf).
+        Returns (y [B,To,Fo,C], out_lengths [B])."""
+        x = _f64(x); w = _f64(w)
+        B, T, F, C = x.shape
+        KT, KF = w.shape[:2]
+        (st, sf), (pt, pb, pf) = stride, pads
+        To, Fo = conv2d_out_shape(T, F, KT, KF, stride, pads)
+        b = _f64(bias) if bias is not None else None
+        ln = _lens(lengths, B)
+        y = np.empty((B, To, Fo, C)); ol = np.empty(B, dtype=np.int32)
+        rc = self.lib.oracle_dwconv2d_fwd(_dp(x), _dp(w), _dp(b), _ip(ln), B, T, F, C, KT, KF, st, sf, pt, pb, pf,
+                                          _dp(y), _ip(ol))
+        if rc:
+            raise ValueError(f"oracle_dwconv2d_fwd rejected its arguments (rc={rc})")
+        return y, ol
+
+    def dwconv2d_bwd_dx(self, dy, w, lengths, T, F, stride, pads):
+        """Data gradient of dwconv2d_fwd: dx [B,T,F,C] from dy [B,To,Fo,C]."""
+        dy = _f64(dy); w = _f64(w)
+        B, To, Fo, C = dy.shape
+        KT, KF = w.shape[:2]
+        (st, sf), (pt, pb, pf) = stride, pads
+        assert (To, Fo) == conv2d_out_shape(T, F, KT, KF, stride, pads)
+        ln = _lens(lengths, B)
+        dx = np.empty((B, T, F, C))
+        rc = self.lib.oracle_dwconv2d_bwd_dx(_dp(dy), _dp(w), _ip(ln), B, T, F, C, KT, KF, st, sf, pt, pb, pf, _dp(dx))
+        if rc:
+            raise ValueError(f"oracle_dwconv2d_bwd_dx rejected its arguments (rc={rc})")
+        return dx
+
+    def dwconv2d_bwd_dw(self, x, dy, KT, KF, lengths, stride, pads):
+        """Weight and bias gradients of dwconv2d_fwd: returns (dW [KT,KF,C], dbias [C])."""
+        x = _f64(x); dy = _f64(dy)
+        B, T, F, C = x.shape
+        (st, sf), (pt, pb, pf) = stride, pads
+        assert dy.shape[1:3] == conv2d_out_shape(T, F, KT, KF, stride, pads)
+        ln = _lens(lengths, B)
+        dw = np.empty((KT, KF, C)); db = np.empty(C)
+        rc = self.lib.oracle_dwconv2d_bwd_dw(_dp(x), _dp(dy), _ip(ln), B, T, F, C, KT, KF, st, sf, pt, pb, pf,
+                                             _dp(dw), _dp(db))
+        if rc:
+            raise ValueError(f"oracle_dwconv2d_bwd_dw rejected its arguments (rc={rc})")
+        return dw, db
+
+
+def conv2d_out_shape(T, F, KT, KF, stride, pads):
+    """(To, Fo) of dwconv2d_fwd: (n + pads - k) // s + 1 per axis, 0 when the window does not fit."""
+    (st, sf), (pt, pb, pf) = stride, pads
+    def o(n, p0, p1, k, s):
+        m = n + p0 + p1 - k
+        return 0 if m < 0 else m // s + 1
+    return o(T, pt, pb, KT, st), o(F, pf, pf, KF, sf)
+
 
 def default() -> Oracle:
     """The oracle compiled from this package's source (built on first use)."""
@@ -261,3 +319,15 @@ def dwconv1d_bwd_dw(x, dy, K, lengths, pad_left):
 
 def dw_subsample_fwd(mel, w0, b0, w1, b1, lengths, causal):
     return default().dw_subsample_fwd(mel, w0, b0, w1, b1, lengths, causal)
+
+
+def dwconv2d_fwd(x, w, bias, lengths, stride, pads):
+    return default().dwconv2d_fwd(x, w, bias, lengths, stride, pads)
+
+
+def dwconv2d_bwd_dx(dy, w, lengths, T, F, stride, pads):
+    return default().dwconv2d_bwd_dx(dy, w, lengths, T, F, stride, pads)
+
+
+def dwconv2d_bwd_dw(x, dy, KT, KF, lengths, stride, pads):
+    return default().dwconv2d_bwd_dw(x, dy, KT, KF, lengths, stride, pads)

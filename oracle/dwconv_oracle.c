@@ -431,3 +431,120 @@ int oracle_dw_subsample_bwd_kinks(const double *mel, const double *w0, const dou
     free(melpad);
     return 0;
 }
+
+/*
+ * General depthwise conv2d with fused length masking (NeMo PR #16114, "What does this PR do ?",
+ * the second kernel: a depthwise conv with fused pre/post masking and causal padding, for the
+ * subsampler's later stages).  Channels-last x [B][T][F][C], taps w [KT][KF][C]:
+ *   xpad[b,r,s,c] = x[b, r-pt, s-pf, c] if 0 <= r-pt < len_b and 0 <= s-pf < F, else 0
+ *   To = (T + pt + pb - KT) / st + 1, Fo = (F + 2 pf - KF) / sf + 1 (0 when negative inside)
+ *   Lo_b = min(To, (len_b + pt + pb - KT) / st + 1), the usual conv length rule
+ *   y[b,i,j,c] = [i < Lo_b] (bias[c] + sum_{p<KT,q<KF} xpad[b, st i + p, sf j + q, c] w[p,q,c])
+ * The data gradient is the transpose (scatter) of this map with dy masked to rows i < Lo_b; the
+ * weight and bias gradients sum dy_masked * xpad and dy_masked over (b, i, j).
+ */
+static int64_t conv_out(int64_t n, int64_t p0, int64_t p1, int64_t k, int64_t s)
+{
+    const int64_t m = n + p0 + p1 - k;
+    if (m < 0) return 0;
+    return m / s + 1;
+}
+
+static double xpad2(const double *x, int64_t b, int64_t r, int64_t s, int64_t c, int64_t T, int64_t F,
+                    int64_t C, int64_t pt, int64_t pf, int64_t L)
+{
+    const int64_t t = r - pt, f = s - pf;
+    if (t < 0 || t >= L || f < 0 || f >= F) return 0.0;   /* padding, or a frame at/after len_b */
+    return x[((b * T + t) * F + f) * C + c];
+}
+
+static int conv2d_args_ok(int64_t B, int64_t T, int64_t F, int64_t C, int64_t KT, int64_t KF, int64_t st,
+                          int64_t sf, int64_t pt, int64_t pb, int64_t pf)
+{
+    return B >= 0 && T >= 0 && F >= 1 && C >= 1 && KT >= 1 && KF >= 1 && st >= 1 && sf >= 1 &&
+           pt >= 0 && pb >= 0 && pf >= 0;
+}
+
+int oracle_dwconv2d_fwd(const double *x, const double *w, const double *bias, const int32_t *lengths,
+                        int64_t B, int64_t T, int64_t F, int64_t C, int64_t KT, int64_t KF, int64_t st,
+                        int64_t sf, int64_t pt, int64_t pb, int64_t pf, double *y, int32_t *out_lengths)
+{
+    if (!conv2d_args_ok(B, T, F, C, KT, KF, st, sf, pt, pb, pf)) return 1;
+    const int64_t To = conv_out(T, pt, pb, KT, st), Fo = conv_out(F, pf, pf, KF, sf);
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        int64_t Lo = conv_out(L, pt, pb, KT, st);
+        if (Lo > To) Lo = To;
+        if (out_lengths) out_lengths[b] = (int32_t)Lo;
+        #pragma omp parallel for schedule(static)
+        for (int64_t i = 0; i < To; ++i)
+            for (int64_t j = 0; j < Fo; ++j)
+                for (int64_t c = 0; c < C; ++c) {
+                    double acc = 0.0;
+                    if (i < Lo) {
+                        acc = bias ? bias[c] : 0.0;
+                        for (int64_t p = 0; p < KT; ++p)
+                            for (int64_t q = 0; q < KF; ++q)
+                                acc += xpad2(x, b, st * i + p, sf * j + q, c, T, F, C, pt, pf, L) *
+                                       w[(p * KF + q) * C + c];
+                    }
+                    y[((b * To + i) * Fo + j) * C + c] = acc;
+                }
+    }
+    return 0;
+}
+
+int oracle_dwconv2d_bwd_dx(const double *dy, const double *w, const int32_t *lengths, int64_t B, int64_t T,
+                           int64_t F, int64_t C, int64_t KT, int64_t KF, int64_t st, int64_t sf, int64_t pt,
+                           int64_t pb, int64_t pf, double *dx)
+{
+    if (!conv2d_args_ok(B, T, F, C, KT, KF, st, sf, pt, pb, pf)) return 1;
+    const int64_t To = conv_out(T, pt, pb, KT, st), Fo = conv_out(F, pf, pf, KF, sf);
+    memset(dx, 0, sizeof(double) * (size_t)(B * T * F * C));
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = clamp_len(lengths, b, T);
+        int64_t Lo = conv_out(L, pt, pb, KT, st);
+        if (Lo > To) Lo = To;
+        #pragma omp parallel for schedule(static)
+        for (int64_t c = 0; c < C; ++c)       /* scatter of every unmasked output, per channel */
+            for (int64_t i = 0; i < Lo; ++i)
+                for (int64_t j = 0; j < Fo; ++j) {
+                    const double g = dy[((b * To + i) * Fo + j) * C + c];
+                    for (int64_t p = 0; p < KT; ++p)
+                        for (int64_t q = 0; q < KF; ++q) {
+                            const int64_t t = st * i + p - pt, f = sf * j + q - pf;
+                            if (t < 0 || t >= L || f < 0 || f >= F) continue;
+                            dx[((b * T + t) * F + f) * C + c] += g * w[(p * KF + q) * C + c];
+                        }
+                }
+    }
+    return 0;
+}
+
+int oracle_dwconv2d_bwd_dw(const double *x, const double *dy, const int32_t *lengths, int64_t B, int64_t T,
+                           int64_t F, int64_t C, int64_t KT, int64_t KF, int64_t st, int64_t sf, int64_t pt,
+                           int64_t pb, int64_t pf, double *dw, double *dbias)
+{
+    if (!conv2d_args_ok(B, T, F, C, KT, KF, st, sf, pt, pb, pf)) return 1;
+    const int64_t To = conv_out(T, pt, pb, KT, st), Fo = conv_out(F, pf, pf, KF, sf);
+    #pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        double gb = 0.0;
+        for (int64_t pq = 0; pq < KT * KF; ++pq) dw[pq * C + c] = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            const int64_t L = clamp_len(lengths, b, T);
+            int64_t Lo = conv_out(L, pt, pb, KT, st);
+            if (Lo > To) Lo = To;
+            for (int64_t i = 0; i < Lo; ++i)
+                for (int64_t j = 0; j < Fo; ++j) {
+                    const double g = dy[((b * To + i) * Fo + j) * C + c];
+                    gb += g;
+                    for (int64_t p = 0; p < KT; ++p)
+                        for (int64_t q = 0; q < KF; ++q)
+                            dw[(p * KF + q) * C + c] += g * xpad2(x, b, st * i + p, sf * j + q, c, T, F, C, pt, pf, L);
+                }
+        }
+        if (dbias) dbias[c] = gb;
+    }
+    return 0;
+}

@@ -199,6 +199,55 @@ def subsample_bwd_checks(o, rng, B, T, F, C, causal):
     return fails
 
 
+def torch_dwconv2d_all(x, w, bias, dy, lengths, stride, pads):
+    """Depthwise conv2d with input and output length masks through torch float64 (conv2d with
+    groups=C) and autograd: returns (y, dx, dW [KT,KF,C], dbias) for loss = sum(y * dy)."""
+    (st, sf), (pt, pb, pf) = stride, pads
+    x = torch.tensor(np.asarray(x, np.float64), requires_grad=True)
+    B, T, F, C = x.shape
+    KT, KF = np.asarray(w).shape[:2]
+    W = torch.tensor(np.asarray(w, np.float64)).permute(2, 0, 1)[:, None].clone().requires_grad_(True)
+    bb = torch.tensor(np.asarray(bias, np.float64) if bias is not None else np.zeros(C)).requires_grad_(True)
+    Ls = clamp_lengths(lengths, B, T)
+    m = (torch.arange(T)[None, :] < torch.tensor(Ls)[:, None]).double()[:, :, None, None]
+    xin = Fnn.pad((x * m).permute(0, 3, 1, 2), (pf, pf, pt, pb))
+    y = Fnn.conv2d(xin, W, bb, stride=(st, sf), groups=C)
+    To = y.shape[2]
+    Lo = [min(To, max(0, (L + pt + pb - KT) // st + 1) if L + pt + pb - KT >= 0 else 0) for L in Ls]
+    y = y * (torch.arange(To)[None, :] < torch.tensor(Lo)[:, None]).double()[:, None, :, None]
+    y = y.permute(0, 2, 3, 1)
+    (y * torch.tensor(np.asarray(dy, np.float64))).sum().backward()
+    return y.detach().numpy(), x.grad.numpy(), W.grad[:, 0].permute(1, 2, 0).numpy(), bb.grad.numpy()
+
+
+def conv2d_checks(o, rng, B, T, F, C, KT, KF, stride, pads):
+    """The oracle's depthwise conv2d forward and gradients against torch autograd; returns
+    failure strings."""
+    import oracle as _oracle_mod  # only for the shape rule
+    fails = []
+    To, Fo = _oracle_mod.conv2d_out_shape(T, F, KT, KF, stride, pads)
+    x = rng.standard_normal((B, T, F, C)); w = rng.standard_normal((KT, KF, C)); b = rng.standard_normal(C)
+    dy = rng.standard_normal((B, To, Fo, C))
+    L = rng.integers(0, T + 1, size=B).astype(np.int32)
+    L[0] = T
+    y, ol = o.dwconv2d_fwd(x, w, b, L, stride, pads)
+    dx = o.dwconv2d_bwd_dx(dy, w, L, T, F, stride, pads)
+    gw, gb = o.dwconv2d_bwd_dw(x, dy, KT, KF, L, stride, pads)
+    tag = (B, T, F, C, KT, KF, stride, pads)
+    if To == 0 or Fo == 0:  # the window does not fit the padded input: no output, zero gradients
+        if y.size or np.any(dx != 0.0) or np.any(gw != 0.0) or np.any(gb != 0.0) or np.any(ol != 0):
+            fails.append(f"conv2d empty output {tag}")
+        return fails
+    ry, rdx, rgw, rgb = torch_dwconv2d_all(x, w, b, dy, L, stride, pads)
+    if y.shape != ry.shape or rel_err(y, ry) > 1e-12:
+        fails.append(f"torch conv2d fwd {tag}")
+    if rel_err(dx, rdx) > 1e-12:
+        fails.append(f"torch conv2d dx {tag}")
+    if rel_err(gw, rgw) > 1e-12 or rel_err(gb, rgb) > 1e-12:
+        fails.append(f"torch conv2d dw {tag}")
+    return fails
+
+
 def load_golden(name):
     with open(os.path.join(GOLDEN, name)) as f:
         return json.load(f)
@@ -336,4 +385,8 @@ def pin_battery(o):
     # subsampler backward: autograd and exact finite differences
     for causal in (False, True):
         fails += subsample_bwd_checks(o, rng, 2, 13, 10, 3, causal)
+
+    # general depthwise conv2d: torch autograd, symmetric and causal, strides 1 and 2
+    for (KT, KF, stride, pads) in ((3, 3, (2, 2), (1, 1, 1)), (3, 2, (1, 2), (2, 0, 1)), (2, 3, (2, 1), (0, 1, 0))):
+        fails += conv2d_checks(o, rng, 2, 11, 9, 3, KT, KF, stride, pads)
     return fails

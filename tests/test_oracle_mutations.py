@@ -46,6 +46,13 @@ MUTANTS = {
     "subsample bwd recomputed conv0 taps transposed": ("const double tap = w0[(p * 3 + q) * C + c];",
                                                        "const double tap = w0[(q * 3 + p) * C + c];"),
     "subsample bwd mel not masked": ("(ff >= 0 && ff < F && t >= 0 && t < L)", "(ff >= 0 && ff < F && t >= 0 && t < T)"),
+    "conv2d taps transposed": ("w[(p * KF + q) * C + c];\n                    }\n                    y[", "w[(q * KT + p) * C + c];\n                    }\n                    y["),
+    "conv2d dx stride dropped": ("const int64_t t = st * i + p - pt, f = sf * j + q - pf;",
+                                 "const int64_t t = i + p - pt, f = sf * j + q - pf;"),
+    "conv2d output mask dropped": ("                    if (i < Lo) {\n                        acc = bias ? bias[c] : 0.0;",
+                                   "                    if (i < To) {\n                        acc = bias ? bias[c] : 0.0;"),
+    "conv2d dbias unmasked rows": ("            for (int64_t i = 0; i < Lo; ++i)\n                for (int64_t j = 0; j < Fo; ++j) {\n                    const double g = dy[((b * To + i) * Fo + j) * C + c];\n                    gb += g;",
+                                   "            for (int64_t i = 0; i < To; ++i)\n                for (int64_t j = 0; j < Fo; ++j) {\n                    const double g = dy[((b * To + i) * Fo + j) * C + c];\n                    gb += g;"),
     "subsample bwd dh taps flipped": ("dhpad[at] += dm * w1[(p * 3 + q) * C + c];",
                                       "dhpad[at] += dm * w1[((2 - p) * 3 + q) * C + c];"),
 }
