@@ -296,6 +296,82 @@ def measure_sub_bwd(dw, dev, hbm, fp32_tflops):
             "alg_bytes": by, "alg_flops": fl}
 
 
+CONV2D = dict(B=16, T=750, F=20, C=256, KT=3, KF=3, stride=(2, 2), pads=(1, 1, 1), len_range=(375, 750), seed=5)
+
+
+def measure_conv2d(dw, dev, hbm):
+    """General depthwise conv2d (a NEXT row, outside the step) on the subsampler's later-stage
+    shape, [16, 750, 20, 256] bf16 -> [16, 375, 10, 256] with a 3x3 stride-2 window: forward, data
+    gradient and weight/bias gradients, each over 3 rotating input sets in a CUDA graph.
+    Algorithmic bytes: forward = x at valid frames + y in full; dx = dy at valid rows + dx in full;
+    dW = x at valid frames + dy at valid rows."""
+    import torch
+    import oracle
+    from synth import conv2d_inputs
+    c = CONV2D
+    B, T, F, C, KT, KF = c["B"], c["T"], c["F"], c["C"], c["KT"], c["KF"]
+    stride, pads = c["stride"], c["pads"]
+    To, Fo = dw.conv2d_out_shape(T, F, KT, KF, stride, pads)
+    d = conv2d_inputs(B, T, F, C, KT, KF, dtype="bf16", len_range=c["len_range"], seed=c["seed"],
+                      dy_shape=(B, To, Fo, C))
+    x0 = torch.from_numpy(d["x"]).to(dev, torch.bfloat16)
+    g0 = torch.from_numpy(d["dy"]).to(dev, torch.bfloat16)
+    xs, gs = [x0] + [x0.clone() for _ in range(2)], [g0] + [g0.clone() for _ in range(2)]
+    ys = [torch.empty(B, To, Fo, C, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    dxs = [torch.empty_like(x0) for _ in range(3)]
+    w = torch.from_numpy(d["w"]).to(dev)
+    bias = torch.from_numpy(d["bias"]).to(dev)
+    ln = torch.from_numpy(d["lengths"]).to(dev)
+    ol = torch.empty(B, dtype=torch.int32, device=dev)
+    gw, gb = torch.empty(KT, KF, C, device=dev), torch.empty(C, device=dev)
+    ws = torch.empty(dw.dwconv2d_bwd_dw_workspace_size(B, T, F, C, KT, KF, stride, pads), dtype=torch.uint8,
+                     device=dev)
+    s = torch.cuda.Stream(dev)
+
+    def timed(fn):
+        with torch.cuda.stream(s):
+            for i in range(3):
+                fn(i)
+            g = torch.cuda.CUDAGraph()
+            g.capture_begin()
+            for i in range(3):
+                fn(i)
+            g.capture_end()
+            for _ in range(3):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(20):
+                g.replay()
+            e1.record(s)
+        torch.cuda.synchronize(dev)
+        del g
+        return e0.elapsed_time(e1) / 60 * 1e3
+
+    t_fwd = timed(lambda i: dw.dwconv2d_fwd(xs[i], w, bias, ys[i], ln, ol, stride, pads))
+    t_dx = timed(lambda i: dw.dwconv2d_bwd_dx(gs[i], w, dxs[i], ln, stride, pads))
+    t_dw = timed(lambda i: dw.dwconv2d_bwd_dw(xs[i], gs[i], gw, gb, ln, stride, pads, ws))
+    L = np.clip(d["lengths"], 0, T)
+    Lo = ol.cpu().numpy()  # output lengths as the forward reported them (checked against the oracle in tests)
+    x_valid = int(L.sum()) * F * C * 2
+    dy_valid = int(Lo.sum()) * Fo * C * 2
+    by_fwd = x_valid + B * To * Fo * C * 2
+    by_dx = dy_valid + B * T * F * C * 2
+    by_dw = x_valid + dy_valid
+    with torch.cuda.stream(s):
+        dw.dwconv2d_fwd(xs[0], w, bias, ys[0], ln, ol, stride, pads)
+    torch.cuda.synchronize(dev)
+    ry, _ = oracle.dwconv2d_fwd(d["x"][:1], d["w"], d["bias"], d["lengths"][:1], stride, pads)
+    err = float(np.max(np.abs(ys[0][:1].float().cpu().numpy() - ry)))
+
+    def row(us, by):
+        return {"us": us, "GB_per_s": by / us / 1e3, "hbm_frac_of_measured": by / us / 1e3 / hbm, "alg_bytes": by}
+    return {"workload": f"depthwise conv2d {B}x{T}x{F}x{C} bf16 -> {B}x{To}x{Fo}x{C}, {KT}x{KF} stride 2, "
+                        "pads 1|1|1, len U[375,750] (3 rotating input sets in a CUDA graph)",
+            "fwd": row(t_fwd, by_fwd), "bwd_dx": row(t_dx, by_dx), "bwd_dw": row(t_dw, by_dw),
+            "fwd_max_abs_err_item0": err}
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -622,6 +698,7 @@ def main():
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
         next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm), "dwconv1d_bwd": measure_bwd(dw, dev, hbm),
+                     "dwconv2d": measure_conv2d(dw, dev, hbm),
                      "dw_subsample_bwd": measure_sub_bwd(dw, dev, hbm, fp32_tflops)}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:

@@ -245,6 +245,76 @@ dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0,
                              int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t dout_dtype,
                              void *workspace, size_t workspace_bytes, dw_stream_t stream);
 
+/*
+ * dwconv2d_fwd - general depthwise conv2d over channels-last [B][T][F][C] with fused length
+ * masking and causal padding (NeMo PR #16114, "Use Fused Kernels for Depthwise Striding
+ * Subsampler", section "What does this PR do ?", second kernel: a depthwise conv with fused
+ * masking and causal padding, used by the subsampler's later depthwise stages).
+ *
+ *   xpad[b,r,s,c] = x[b, r-pad_t, s-pad_f, c] if 0 <= r-pad_t < len_b and 0 <= s-pad_f < F, else 0
+ *   To = (T + pad_t + pad_b - KT) / stride_t + 1,  Fo = (F + 2 pad_f - KF) / stride_f + 1
+ *        (0 when the window does not fit)
+ *   Lo_b = min(To, (len_b + pad_t + pad_b - KT) / stride_t + 1)   (0 when it does not fit)
+ *   y[b,i,j,c] = [i < Lo_b] (bias[c] + sum_{p<KT, q<KF} xpad[b, stride_t i + p, stride_f j + q, c] w[p,q,c])
+ *
+ * Frames t >= len_b count as padding (the pre-mask); output rows i >= Lo_b are written as +0.0
+ * (the post-mask).  Causal time padding is pad_t = KT-1, pad_b = 0; symmetric is pad_t = pad_b.
+ * float32 accumulation, one rounding to io_dtype.
+ *
+ *  x            [B][T][F][C] io_dtype, device
+ *  w            [KT][KF][C] float32, device;  bias [C] float32, device, or NULL
+ *  y            [B][To][Fo][C] io_dtype, device, written in full; must not overlap x
+ *  lengths      [B] int32, device, or NULL (all T frames valid); values are clamped to [0, T]
+ *  out_lengths  [B] int32, device, or NULL; receives Lo_b
+ *  B >= 0, T >= 0, F >= 1, C >= 1, KT, KF >= 1, strides >= 1, pads >= 0; each of T, F, C, To,
+ *  Fo below 2^31.  Invalid arguments return DW_ERR_INVALID_ARG before any device work.
+ */
+dw_status_t dwconv2d_fwd(const void *x, const float *w, const float *bias, void *y,
+                         const int32_t *lengths, int32_t *out_lengths, int64_t B, int64_t T,
+                         int64_t F, int64_t C, int KT, int KF, int stride_t, int stride_f,
+                         int pad_t, int pad_b, int pad_f, dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
+ * dwconv2d_bwd_dx - data gradient of dwconv2d_fwd: the transpose of the masked map,
+ *   dx[b,t,f,c] = [t < len_b] sum over (i, j, p, q) with stride_t i + p - pad_t = t,
+ *                 stride_f j + q - pad_f = f and i < Lo_b of dy[b,i,j,c] w[p,q,c]
+ * computed as a gather (each dx element is written once, no atomics).
+ *
+ *  dy  [B][To][Fo][C] io_dtype, device;  dx [B][T][F][C] io_dtype, device, written in full
+ *      (+0.0 at t >= len_b); must not overlap dy
+ *  other arguments as dwconv2d_fwd.
+ */
+dw_status_t dwconv2d_bwd_dx(const void *dy, const float *w, void *dx, const int32_t *lengths,
+                            int64_t B, int64_t T, int64_t F, int64_t C, int KT, int KF,
+                            int stride_t, int stride_f, int pad_t, int pad_b, int pad_f,
+                            dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
+ * dwconv2d_bwd_dw_workspace_size - bytes of device workspace dwconv2d_bwd_dw needs for these
+ * sizes (independent of pointers, dtype and device); 0 for invalid sizes.
+ */
+size_t dwconv2d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t F, int64_t C, int KT, int KF,
+                                      int stride_t, int stride_f, int pad_t, int pad_b, int pad_f);
+
+/*
+ * dwconv2d_bwd_dw - weight and bias gradients of dwconv2d_fwd:
+ *   dW[p,q,c] = sum_{b, i < Lo_b, j} dy[b,i,j,c] xpad[b, stride_t i + p, stride_f j + q, c]
+ *   dbias[c]  = sum_{b, i < Lo_b, j} dy[b,i,j,c]
+ * float32 accumulation; per-block partial sums go to `workspace` and a second kernel adds them
+ * in a fixed order: bitwise reproducible for given sizes on a given GPU model.  No atomics.
+ *
+ *  x, dy        as dwconv2d_fwd / dwconv2d_bwd_dx
+ *  dw           [KT][KF][C] float32, device, overwritten;  dbias [C] float32, or NULL
+ *  workspace    device buffer of at least dwconv2d_bwd_dw_workspace_size(...) bytes, 16-byte
+ *               aligned; contents on entry are ignored
+ *  With no output elements the gradients are written as zeros (workspace may be NULL).
+ */
+dw_status_t dwconv2d_bwd_dw(const void *x, const void *dy, float *dw, float *dbias,
+                            const int32_t *lengths, int64_t B, int64_t T, int64_t F, int64_t C,
+                            int KT, int KF, int stride_t, int stride_f, int pad_t, int pad_b,
+                            int pad_f, dw_dtype_t io_dtype, void *workspace,
+                            size_t workspace_bytes, dw_stream_t stream);
+
 /* dw_status_string - a static, human-readable name for a status code. */
 const char *dw_status_string(dw_status_t status);
 

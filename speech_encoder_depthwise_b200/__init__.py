@@ -22,6 +22,7 @@ __all__ = [
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
     "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd",
     "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
+    "dwconv2d_fwd", "dwconv2d_bwd_dx", "dwconv2d_bwd_dw_workspace_size", "dwconv2d_bwd_dw", "conv2d_out_shape",
 ]
 
 DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_WORKSPACE, DW_ERR_CUDA, DW_ERR_TIMEOUT = range(6)
@@ -52,6 +53,14 @@ SIGNATURES = {
     "dw_subsample_bwd_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
     "dw_subsample_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int,
                                 _int, _vp, ctypes.c_size_t, _vp]),
+    "dwconv2d_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _int, _int, _int, _int,
+                            _int, _int, _int, _vp]),
+    "dwconv2d_bwd_dx": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _int, _int, _int, _int, _int,
+                               _int, _int, _vp]),
+    "dwconv2d_bwd_dw_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64, _int, _int, _int, _int, _int, _int,
+                                                         _int]),
+    "dwconv2d_bwd_dw": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _int, _int, _int, _int, _int,
+                               _int, _int, _vp, ctypes.c_size_t, _vp]),
     "dw_status_string": (ctypes.c_char_p, [_int]),
     "dw_last_cuda_error": (_int, []),
     "dw_device_error": (_int, []),
@@ -257,3 +266,65 @@ def dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, dw0, db0, dw1, db1, causal,
                                 workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                 _stream(stream))
     _check("dw_subsample_bwd", st)
+
+
+def conv2d_out_shape(T, F, KT, KF, stride, pads):
+    """(To, Fo) of ``dwconv2d_fwd``: (n + pads - k) // s + 1 per axis, 0 when the window does not fit."""
+    (st, sf), (pt, pb, pf) = stride, pads
+
+    def o(n, p0, p1, k, s):
+        m = n + p0 + p1 - k
+        return 0 if m < 0 else m // s + 1
+    return o(T, pt, pb, KT, st), o(F, pf, pf, KF, sf)
+
+
+def _c2_geom(stride, pads):
+    (st, sf), (pt, pb, pf) = stride, pads
+    return int(st), int(sf), int(pt), int(pb), int(pf)
+
+
+def dwconv2d_fwd(x, w, bias, y, lengths, out_lengths, stride, pads, stream=None):
+    """Depthwise conv2d of channels-last x [B,T,F,C] with taps w [KT,KF,C] (float32) into
+    y [B,To,Fo,C]; ``stride`` = (st, sf), ``pads`` = (pad_t, pad_b, pad_f)."""
+    import torch
+    B, T, F, C = x.shape
+    KT, KF = w.shape[:2]
+    To, Fo = conv2d_out_shape(T, F, KT, KF, stride, pads)
+    st = lib().dwconv2d_fwd(_dev(x, "x"), _dev(w, "w", torch.float32, (KT, KF, C)),
+                            _dev(bias, "bias", torch.float32, (C,)), _dev(y, "y", x.dtype, (B, To, Fo, C)),
+                            _dev(lengths, "lengths", torch.int32, (B,)),
+                            _dev(out_lengths, "out_lengths", torch.int32, (B,)), B, T, F, C, KT, KF,
+                            *_c2_geom(stride, pads), _dtype_code(x), _stream(stream))
+    _check("dwconv2d_fwd", st)
+
+
+def dwconv2d_bwd_dx(dy, w, dx, lengths, stride, pads, stream=None):
+    """Data gradient of ``dwconv2d_fwd`` into dx [B,T,F,C] from dy [B,To,Fo,C]."""
+    import torch
+    B, T, F, C = dx.shape
+    KT, KF = w.shape[:2]
+    To, Fo = conv2d_out_shape(T, F, KT, KF, stride, pads)
+    st = lib().dwconv2d_bwd_dx(_dev(dy, "dy", dx.dtype, (B, To, Fo, C)), _dev(w, "w", torch.float32, (KT, KF, C)),
+                               _dev(dx, "dx"), _dev(lengths, "lengths", torch.int32, (B,)), B, T, F, C, KT, KF,
+                               *_c2_geom(stride, pads), _dtype_code(dx), _stream(stream))
+    _check("dwconv2d_bwd_dx", st)
+
+
+def dwconv2d_bwd_dw_workspace_size(B, T, F, C, KT, KF, stride, pads) -> int:
+    """Bytes of workspace ``dwconv2d_bwd_dw`` needs for these sizes."""
+    return int(lib().dwconv2d_bwd_dw_workspace_size(B, T, F, C, KT, KF, *_c2_geom(stride, pads)))
+
+
+def dwconv2d_bwd_dw(x, dy, dw, dbias, lengths, stride, pads, workspace, stream=None):
+    """Weight and bias gradients of ``dwconv2d_fwd`` into dw [KT,KF,C] and dbias [C] (float32)."""
+    import torch
+    B, T, F, C = x.shape
+    KT, KF = dw.shape[:2]
+    To, Fo = conv2d_out_shape(T, F, KT, KF, stride, pads)
+    st = lib().dwconv2d_bwd_dw(_dev(x, "x"), _dev(dy, "dy", x.dtype, (B, To, Fo, C)),
+                               _dev(dw, "dw", torch.float32, (KT, KF, C)), _dev(dbias, "dbias", torch.float32, (C,)),
+                               _dev(lengths, "lengths", torch.int32, (B,)), B, T, F, C, KT, KF,
+                               *_c2_geom(stride, pads), _dtype_code(x), _dev(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                               _stream(stream))
+    _check("dwconv2d_bwd_dw", st)

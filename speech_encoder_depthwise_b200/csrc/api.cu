@@ -73,6 +73,39 @@ dw_status_t check_conv1d_common(const void *in, const float *w, const void *out,
     return DW_OK;
 }
 
+// Geometry of a depthwise conv2d: every size in range and the output sizes (To, Fo).  Bounds
+// keep every frame index inside the kernels (stride i + tap - pad and the like) in 32 bits.
+dw_status_t conv2d_geometry(int64_t B, int64_t T, int64_t F, int64_t C, int KT, int KF, int st, int sf, int pt,
+                            int pb, int pf, int64_t *To, int64_t *Fo) {
+    if (B < 0 || T < 0 || F < 1 || C < 1 || KT < 1 || KF < 1 || st < 1 || sf < 1 || pt < 0 || pb < 0 || pf < 0)
+        return DW_ERR_INVALID_ARG;
+    constexpr int64_t kLim = (int64_t(1) << 30);
+    if (B >= kLim || T + pt + pb >= kLim || F + 2 * static_cast<int64_t>(pf) >= kLim || KT >= kLim ||
+        KF >= kLim)
+        return DW_ERR_INVALID_ARG;
+    if (C > kMaxChannels) return DW_ERR_UNSUPPORTED;
+    auto out = [](int64_t n, int64_t p0, int64_t p1, int64_t k, int64_t s) -> int64_t {
+        const int64_t m = n + p0 + p1 - k;
+        return m < 0 ? 0 : m / s + 1;
+    };
+    *To = out(T, pt, pb, KT, st);
+    *Fo = out(F, pf, pf, KF, sf);
+    int64_t n = 0;
+    if (!mul3(B, T, F * C, &n) || !mul3(B, *To, *Fo * C, &n)) return DW_ERR_INVALID_ARG;
+    return DW_OK;
+}
+
+dwk::Conv2dArgs conv2d_args(int64_t B, int64_t T, int64_t F, int64_t C, int64_t To, int64_t Fo, int KT, int KF,
+                            int st, int sf, int pt, int pb, int pf, dw_dtype_t dt) {
+    dwk::Conv2dArgs a;
+    a.x = nullptr; a.w = nullptr; a.bias = nullptr; a.y = nullptr; a.lengths = nullptr; a.out_lengths = nullptr;
+    a.B = B; a.T = T; a.F = F; a.C = C; a.To = To; a.Fo = Fo;
+    a.KT = KT; a.KF = KF; a.st = st; a.sf = sf; a.pt = pt; a.pb = pb; a.pf = pf;
+    a.bf16 = dt == DW_BF16;
+    a.vec_width = 1;
+    return a;
+}
+
 }  // namespace
 
 extern "C" {
@@ -263,6 +296,85 @@ dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0,
             return DW_ERR_INVALID_ARG;
     }
     return cuda_status(dwk::subsample_bwd_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
+dw_status_t dwconv2d_fwd(const void *x, const float *w, const float *bias, void *y, const int32_t *lengths,
+                         int32_t *out_lengths, int64_t B, int64_t T, int64_t F, int64_t C, int KT, int KF,
+                         int stride_t, int stride_f, int pad_t, int pad_b, int pad_f, dw_dtype_t io_dtype,
+                         dw_stream_t stream) {
+    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
+    int64_t To = 0, Fo = 0;
+    dw_status_t st = conv2d_geometry(B, T, F, C, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, &To, &Fo);
+    if (st != DW_OK) return st;
+    const int64_t nin = B * T * F * C, nout = B * To * Fo * C;
+    if (nout == 0 && out_lengths == nullptr) return DW_OK;
+    if (nout > 0) {
+        if (x == nullptr || w == nullptr || y == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t es = dtype_size(io_dtype);
+        if (overlaps(x, static_cast<size_t>(nin) * es, y, static_cast<size_t>(nout) * es)) return DW_ERR_INVALID_ARG;
+    }
+    if (B == 0) return DW_OK;
+    dwk::Conv2dArgs a = conv2d_args(B, T, F, C, To, Fo, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, io_dtype);
+    a.x = x; a.w = w; a.bias = bias; a.y = y; a.lengths = lengths; a.out_lengths = out_lengths;
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, y}, {w, bias});
+    return cuda_status(dwk::conv2d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
+dw_status_t dwconv2d_bwd_dx(const void *dy, const float *w, void *dx, const int32_t *lengths, int64_t B,
+                            int64_t T, int64_t F, int64_t C, int KT, int KF, int stride_t, int stride_f, int pad_t,
+                            int pad_b, int pad_f, dw_dtype_t io_dtype, dw_stream_t stream) {
+    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
+    int64_t To = 0, Fo = 0;
+    dw_status_t st = conv2d_geometry(B, T, F, C, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, &To, &Fo);
+    if (st != DW_OK) return st;
+    const int64_t nin = B * T * F * C, nout = B * To * Fo * C;
+    if (nin == 0) return DW_OK;
+    if (dx == nullptr || w == nullptr) return DW_ERR_INVALID_ARG;
+    if (nout > 0) {
+        if (dy == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t es = dtype_size(io_dtype);
+        if (overlaps(dy, static_cast<size_t>(nout) * es, dx, static_cast<size_t>(nin) * es)) return DW_ERR_INVALID_ARG;
+    }
+    dwk::Conv2dArgs a = conv2d_args(B, T, F, C, To, Fo, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, io_dtype);
+    a.x = dy; a.w = w; a.y = dx; a.lengths = lengths;
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {dy, dx}, {w});
+    return cuda_status(dwk::conv2d_dx_launch(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dwconv2d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t F, int64_t C, int KT, int KF, int stride_t,
+                                      int stride_f, int pad_t, int pad_b, int pad_f) {
+    int64_t To = 0, Fo = 0;
+    if (conv2d_geometry(B, T, F, C, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, &To, &Fo) != DW_OK) return 0;
+    return dwk::conv2d_dw_workspace_bytes(B, To, C, KT, KF);
+}
+
+dw_status_t dwconv2d_bwd_dw(const void *x, const void *dy, float *dw, float *dbias, const int32_t *lengths,
+                            int64_t B, int64_t T, int64_t F, int64_t C, int KT, int KF, int stride_t, int stride_f,
+                            int pad_t, int pad_b, int pad_f, dw_dtype_t io_dtype, void *workspace,
+                            size_t workspace_bytes, dw_stream_t stream) {
+    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
+    int64_t To = 0, Fo = 0;
+    dw_status_t st = conv2d_geometry(B, T, F, C, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, &To, &Fo);
+    if (st != DW_OK) return st;
+    if (dw == nullptr) return DW_ERR_INVALID_ARG;
+    const int64_t ntap = static_cast<int64_t>(KT) * KF;
+    if ((ntap + 1) * C > dwk::kMaxGrid * 32LL) return DW_ERR_INVALID_ARG;
+    const size_t out_bytes = static_cast<size_t>(ntap) * C * sizeof(float), gb = static_cast<size_t>(C) * sizeof(float);
+    if (dbias != nullptr && overlaps(dw, out_bytes, dbias, gb)) return DW_ERR_INVALID_ARG;
+    dwk::Conv2dArgs a = conv2d_args(B, T, F, C, To, Fo, KT, KF, stride_t, stride_f, pad_t, pad_b, pad_f, io_dtype);
+    a.x = x; a.y = const_cast<void *>(dy); a.lengths = lengths;
+    float *partials = nullptr;
+    if (B * To * Fo > 0) {
+        if (x == nullptr || dy == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t need = dwk::conv2d_dw_workspace_bytes(B, To, C, KT, KF);
+        if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return DW_ERR_WORKSPACE;
+        if (overlaps(workspace, need, dw, out_bytes) || (dbias && overlaps(workspace, need, dbias, gb)))
+            return DW_ERR_INVALID_ARG;
+        partials = static_cast<float *>(workspace);
+        const size_t es = dtype_size(io_dtype);
+        a.vec_width = (C % 2 == 0 && aligned(x, 2 * es) && aligned(dy, 2 * es)) ? 2 : 1;
+    }
+    return cuda_status(dwk::conv2d_dw_launch(a, dw, dbias, partials, static_cast<cudaStream_t>(stream)));
 }
 
 dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0, const float *w1,

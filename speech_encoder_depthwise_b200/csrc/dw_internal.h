@@ -59,6 +59,20 @@ struct SubsampleArgs {
     int causal, bf16_out;
 };
 
+// General depthwise conv2d, channels-last [B][T][F][C], taps [KT][KF][C].  The data gradient
+// takes dy as x and writes dx through y; the weight gradient takes x and dy (as y).
+struct Conv2dArgs {
+    const void *x;
+    const float *w;           // [KT][KF][C] (forward and data gradient)
+    const float *bias;        // [C] or null (forward)
+    void *y;
+    const int32_t *lengths;
+    int32_t *out_lengths;     // [B] or null (forward)
+    int64_t B, T, F, C, To, Fo;
+    int KT, KF, st, sf, pt, pb, pf;
+    int bf16, vec_width;      // vec_width: 4, 2 or 1 channels per thread
+};
+
 // Raise a kernel's dynamic shared memory limit to `bytes`, once per (kernel, device).
 cudaError_t ensure_smem_attr(const void *kern, int bytes);
 
@@ -92,6 +106,12 @@ unsigned int conv1d_dw_take_error();
 cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s);
 
 cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
+
+cudaError_t conv2d_fwd_launch(const Conv2dArgs &a, cudaStream_t s);
+cudaError_t conv2d_dx_launch(const Conv2dArgs &a, cudaStream_t s);
+int conv2d_dw_partial_rows(int64_t B, int64_t To);
+size_t conv2d_dw_workspace_bytes(int64_t B, int64_t To, int64_t C, int KT, int KF);
+cudaError_t conv2d_dw_launch(const Conv2dArgs &a, float *dw, float *dbias, float *partials, cudaStream_t s);
 
 struct SubsampleBwdArgs {
     const float *mel, *w0, *b0, *w1;

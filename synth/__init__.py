@@ -12,6 +12,9 @@ Recipe (one ``numpy.random.default_rng(seed)`` per workload):
   ``b0`` ~ N(0, 0.1), ``w1[3, 3, C]`` ~ N(0, 1/9), ``b1`` ~ N(0, 0.1), then
   ``lengths``.  Mel frames at ``t >= lengths[b]`` are then set to zero, so a
   reading that masks the mel before conv0 and one that does not agree.
+* conv2d: draw ``x[B, T, F, C]`` ~ N(0, 1), then ``w[KT, KF, C]`` ~ N(0, 1/(KT KF)),
+  ``bias[C]`` ~ N(0, 0.1), then ``lengths``, then (when the caller gives the output
+  shape) ``dy`` ~ N(0, 1) of that shape.
 * bf16 workloads round every drawn value (data and weights) to the nearest
   bf16-representable float32, ties to even, so the stored bf16 tensor and the
   float32 weights hold exactly the values the oracle reads.
@@ -27,6 +30,7 @@ __all__ = [
     "bf16_bits",
     "conv1d_inputs",
     "subsample_inputs",
+    "conv2d_inputs",
     "symmetric_pad_left",
     "WORKLOADS",
 ]
@@ -97,6 +101,26 @@ def subsample_inputs(B, T, F, C, *, len_range, seed=3, zero_beyond_len=True):
         for b in range(B):
             mel[b, max(0, int(lengths[b])):, :] = 0.0
     return {"mel": mel, "w0": w0, "b0": b0, "w1": w1, "b1": b1, "lengths": lengths}
+
+
+def conv2d_inputs(B, T, F, C, KT, KF, *, dtype="bf16", len_range=None, seed=0, dy_shape=None):
+    """Inputs of one depthwise conv2d workload: ``x[B,T,F,C]``, ``w[KT,KF,C]``, ``bias[C]``,
+    ``lengths[B]`` (None without ``len_range``) and, given ``dy_shape``, ``dy``."""
+    rng = np.random.default_rng(seed)
+    out = {"x": _normal(rng, (B, T, F, C), 1.0), "w": _normal(rng, (KT, KF, C), 1.0 / (KT * KF)),
+           "bias": _normal(rng, (C,), 0.1), "lengths": None}
+    if len_range is not None:
+        lo, hi = len_range
+        out["lengths"] = rng.integers(lo, hi + 1, size=B).astype(np.int32)
+    if dy_shape is not None:
+        out["dy"] = _normal(rng, tuple(dy_shape), 1.0)
+    if dtype == "bf16":
+        for k in ("x", "w", "bias", "dy"):
+            if k in out:
+                out[k] = bf16_round(out[k])
+    elif dtype != "f32":
+        raise ValueError(f"unknown dtype {dtype!r}")
+    return out
 
 
 # The five workloads, shaped like the ones the pages run (the parakeet conformer

@@ -144,6 +144,61 @@ def test_subsample_rejects_invalid_arguments(lib):
     assert call(T=0) == dw.DW_OK
 
 
+def test_conv2d_rejects_invalid_arguments(lib):
+    f = lib.dwconv2d_fwd
+    names = ["x", "w", "bias", "y", "ln", "oln", "B", "T", "F", "C", "KT", "KF", "st", "sf", "pt", "pb", "pf",
+             "dt", "s"]
+    ok = [FAKE_X, FAKE_W, None, FAKE_Y, None, None, 2, 40, 20, 8, 3, 3, 2, 2, 1, 1, 1, dw.DW_BF16, None]
+
+    def call(fn=f, base=ok, keys=names, **kw):
+        a = list(base)
+        for k, v in kw.items():
+            a[keys.index(k)] = v
+        return fn(*a)
+
+    for kw in (dict(x=None), dict(w=None), dict(y=None), dict(KT=0), dict(KF=-1), dict(st=0), dict(sf=-2),
+               dict(pt=-1), dict(pb=-1), dict(pf=-1), dict(B=-1), dict(T=-1), dict(F=0), dict(C=0), dict(dt=4),
+               dict(y=FAKE_X + 64), dict(T=1 << 31), dict(pt=1 << 30)):
+        assert call(**kw) == dw.DW_ERR_INVALID_ARG, kw
+    assert call(C=1 << 23) == dw.DW_ERR_UNSUPPORTED
+    assert call(B=0) == dw.DW_OK                                  # nothing to do
+    assert call(T=0, x=None, y=None) == dw.DW_OK                  # no output rows, no lengths asked
+    assert call(KF=30, x=None, y=None) == dw.DW_OK                # the window does not fit F
+    # data gradient: dy and dx must not overlap; an empty input is a no-op
+    g = lib.dwconv2d_bwd_dx
+    gn = ["dy", "w", "dx", "ln", "B", "T", "F", "C", "KT", "KF", "st", "sf", "pt", "pb", "pf", "dt", "s"]
+    gok = [FAKE_Y, FAKE_W, FAKE_X, None, 2, 40, 20, 8, 3, 3, 2, 2, 1, 1, 1, dw.DW_BF16, None]
+    assert call(g, gok, gn, dy=None) == dw.DW_ERR_INVALID_ARG
+    assert call(g, gok, gn, dx=None) == dw.DW_ERR_INVALID_ARG
+    assert call(g, gok, gn, w=None) == dw.DW_ERR_INVALID_ARG
+    assert call(g, gok, gn, dx=FAKE_Y + 32) == dw.DW_ERR_INVALID_ARG
+    assert call(g, gok, gn, st=0) == dw.DW_ERR_INVALID_ARG
+    assert call(g, gok, gn, B=0, dy=None, dx=None) == dw.DW_OK
+    assert call(g, gok, gn, T=0, dy=None, dx=None) == dw.DW_OK
+
+
+def test_conv2d_dw_workspace_rules(lib):
+    geom = (2, 2, 1, 1, 1)
+    n = lib.dwconv2d_bwd_dw_workspace_size(16, 750, 20, 256, 3, 3, *geom)
+    assert n > 0 and n % 16 == 0
+    assert lib.dwconv2d_bwd_dw_workspace_size(16, 750, 20, 256, 5, 5, *geom) > n
+    assert lib.dwconv2d_bwd_dw_workspace_size(16, 750, 20, 512, 3, 3, *geom) > n
+    assert lib.dwconv2d_bwd_dw_workspace_size(16, 750, 0, 256, 3, 3, *geom) == 0      # invalid F
+    assert lib.dwconv2d_bwd_dw_workspace_size(16, 750, 20, 256, 3, 3, 0, 2, 1, 1, 1) == 0
+    f = lib.dwconv2d_bwd_dw
+    head = (FAKE_X, FAKE_Y, FAKE_W, None, None, 16, 750, 20, 256, 3, 3, *geom, dw.DW_BF16)
+    assert f(*head, None, n, None) == dw.DW_ERR_WORKSPACE
+    assert f(*head, FAKE_WS, n - 16, None) == dw.DW_ERR_WORKSPACE
+    assert f(*head, FAKE_WS + 8, n, None) == dw.DW_ERR_WORKSPACE
+    assert f(*head, FAKE_W - 64, n, None) == dw.DW_ERR_INVALID_ARG             # workspace overlaps dW
+    assert f(FAKE_X, FAKE_Y, None, None, None, 16, 750, 20, 256, 3, 3, *geom, dw.DW_BF16, FAKE_WS, n, None) \
+        == dw.DW_ERR_INVALID_ARG
+    assert f(FAKE_X, FAKE_Y, FAKE_W, FAKE_W + 64, None, 16, 750, 20, 256, 3, 3, *geom, dw.DW_BF16, FAKE_WS, n,
+             None) == dw.DW_ERR_INVALID_ARG                                   # dbias overlaps dW
+    assert f(None, FAKE_Y, FAKE_W, None, None, 16, 750, 20, 256, 3, 3, *geom, dw.DW_BF16, FAKE_WS, n, None) \
+        == dw.DW_ERR_INVALID_ARG
+
+
 def test_binding_rejects_host_tensors(lib):
     import torch
     x = torch.zeros(1, 4, 2, dtype=torch.bfloat16)
