@@ -126,7 +126,8 @@ int dw_last_cuda_error(void) { return g_last_cuda_error; }
 
 dw_status_t dw_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
-    const unsigned int e = dwk::conv1d_fwd_take_error() | dwk::conv1d_dw_take_error() | dwk::subsample_tc_take_error();
+    const unsigned int e = dwk::conv1d_fwd_take_error() | dwk::conv1d_dw_take_error() | dwk::subsample_tc_take_error() |
+                           dwk::conv2d_tma_take_error();
     return e ? DW_ERR_TIMEOUT : DW_OK;
 }
 

@@ -321,11 +321,15 @@ cudaError_t conv2d_fwd_launch(const Conv2dArgs &a, cudaStream_t s) {
             static_cast<int>(a.To));
         return cudaGetLastError();
     }
+    const cudaError_t e = conv2d_fwd_tma_launch(a, s);
+    if (e != cudaErrorNotSupported) return e;
     return a.bf16 ? dispatch_vec<bf16>(a, s, false) : dispatch_vec<float>(a, s, false);
 }
 
 cudaError_t conv2d_dx_launch(const Conv2dArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
+    const cudaError_t e = conv2d_dx_tma_launch(a, s);
+    if (e != cudaErrorNotSupported) return e;
     return a.bf16 ? dispatch_vec<bf16>(a, s, true) : dispatch_vec<float>(a, s, true);
 }
 
@@ -345,6 +349,17 @@ cudaError_t conv2d_dw_launch(const Conv2dArgs &a, float *dw, float *dbias, float
         dwconv2d_dw_zero_kernel<<<static_cast<unsigned>((static_cast<int64_t>(ntap) * a.C + 255) / 256), 256, 0, s>>>(
             dw, dbias, ntap, static_cast<int>(a.C));
         return cudaGetLastError();
+    }
+    const int64_t E = static_cast<int64_t>(ntap + 1) * a.C;
+    {
+        int Gt = 0;
+        const cudaError_t e = conv2d_dw_tma_partials(a, partials, conv2d_dw_partial_rows(a.B, a.To), &Gt, s);
+        if (e != cudaErrorNotSupported) {
+            if (e != cudaSuccess) return e;
+            dwconv2d_dw_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(
+                partials, Gt, ntap, static_cast<int>(a.C), dw, dbias);
+            return cudaGetLastError();
+        }
     }
     const int64_t nCG = (a.C + 2 * kC2Threads - 1) / (2 * kC2Threads);
     int G = conv2d_dw_partial_rows(a.B, a.To);
@@ -371,7 +386,6 @@ cudaError_t conv2d_dw_launch(const Conv2dArgs &a, float *dw, float *dbias, float
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    const int64_t E = static_cast<int64_t>(ntap + 1) * a.C;
     dwconv2d_dw_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(partials, G, ntap,
                                                                                       static_cast<int>(a.C), dw, dbias);
     return cudaGetLastError();

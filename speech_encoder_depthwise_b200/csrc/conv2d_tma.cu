@@ -1,0 +1,640 @@
+// Depthwise conv2d with a 3x3 window (any strides and pads): shared-memory tiled kernels fed by
+// TMA tensor copies (NeMo PR #16114, "Use Fused Kernels for Depthwise Striding Subsampler",
+// section "What does this PR do ?", the depthwise conv with fused masking and causal padding).
+// The same map as the general kernels in conv2d.cu:
+//
+//   xpad[b,r,s,c] = x[b, r-pt, s-pf, c] if 0 <= r-pt < len_b and 0 <= s-pf < F, else 0
+//   y[b,i,j,c]    = [i < Lo_b] (bias[c] + sum_{p,q<3} xpad[b, st i + p, sf j + q, c] w[p,q,c])
+//
+// Each CTA is persistent and walks tiles (item, block of rows, block of columns, channel slab).
+// One thread issues a single 4-D TMA copy per tile (box = channel slab x columns x rows x 1) into
+// one of two shared-memory stages while the block computes on the other, so every input
+// element crosses HBM once (plus a small row halo).  Padding outside the tensor arrives as TMA
+// zero fill; frames at or after len_b are real data and are skipped at compute time.  Tiles
+// whose rows are all masked only store zeros and issue no copy.
+#include "dw_internal.h"
+
+namespace dwk {
+namespace {
+
+constexpr int kC2V = 4;             // channels per thread (8 bytes bf16, 16 bytes float32)
+constexpr int kC2StageMax = 49152;  // bytes of one stage
+constexpr int kC2DwGroups = 8;      // position groups of the weight-gradient CTA
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c, int f, int t, int b, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c), "r"(f), "r"(t), "r"(b), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ int out_len(const int32_t *lengths, int b, int Tn, int pt, int pb, int st, int To) {
+    const int L = static_cast<int>(clamp_len(lengths, b, Tn));
+    const int m = L + pt + pb - 3;
+    const int Lo = m < 0 ? 0 : m / st + 1;
+    return Lo < To ? Lo : To;
+}
+
+// Geometry and tiling, passed by value.
+struct C2Geo {
+    int B, T, F, C, To, Fo, st, sf, pt, pb, pf;
+    int TI, TJ, CS;      // tile: rows, columns (of the map's output), channels
+    int BR, BF;          // box rows, box columns of the staged tensor
+    int nI, nJ, nCS;     // tiles per axis
+    int stage_bytes;     // bytes of one stage (all staged boxes, each 128-byte aligned)
+    int tx_bytes;        // bytes the copies of one stage deliver
+};
+
+template <typename T>
+__device__ __forceinline__ void lds_vec(const T *p, float2 (&f)[2]) {
+    if constexpr (sizeof(T) == 2) {
+        const uint2 r = *reinterpret_cast<const uint2 *>(p);
+        f[0] = make_float2(bf16_lo(r.x), bf16_hi(r.x));
+        f[1] = make_float2(bf16_lo(r.y), bf16_hi(r.y));
+    } else {
+        const float4 r = *reinterpret_cast<const float4 *>(p);
+        f[0] = make_float2(r.x, r.y);
+        f[1] = make_float2(r.z, r.w);
+    }
+}
+
+// Decode tile index -> (b, row block, column block, channel slab), channel slab fastest.
+__device__ __forceinline__ void decode(const C2Geo &g, int tile, int &b, int &it, int &jt, int &cs) {
+    cs = tile % g.nCS;
+    int r = tile / g.nCS;
+    jt = r % g.nJ;
+    r /= g.nJ;
+    it = r % g.nI;
+    b = r / g.nI;
+}
+
+// Shared memory: two mbarriers in the first 128 bytes, then [2 stages][stage_bytes], then (the
+// data gradient only) the per-tile row table.
+constexpr int kC2Head = 128;
+struct C2Smem {
+    unsigned char *stage[2];
+    uint64_t *full;
+};
+__device__ __forceinline__ C2Smem c2_smem(unsigned char *raw, int stage_bytes) {
+    C2Smem s;
+    s.full = reinterpret_cast<uint64_t *>(raw);
+    s.stage[0] = raw + kC2Head;
+    s.stage[1] = raw + kC2Head + stage_bytes;
+    return s;
+}
+
+// ------------------------------------------------------------------------------ forward
+// Tile = TI output rows x TJ output columns x CS channels of one item; the box covers input rows
+// st*i0 - pt .. + BR and columns sf*j0 - pf .. + BF.  Thread = (column j, channel vector cv) and
+// walks the TI rows; blockDim = TJ * CS/4 rounded up to a warp.
+template <typename T>
+__global__ void __launch_bounds__(512)
+c2_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restrict__ w,
+                  const float *__restrict__ bias, T *__restrict__ y, const int32_t *__restrict__ lengths,
+                  int32_t *__restrict__ out_lengths, C2Geo g) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const C2Smem sm = c2_smem(smem_raw, g.stage_bytes);
+    const int tid = threadIdx.x;
+    const int CSV = g.CS / kC2V;
+    const int cv = tid % CSV, jl = tid / CSV;
+    const bool active = jl < g.TJ;
+    const int ntiles = g.B * g.nI * g.nJ * g.nCS;
+    if (tid == 0) {
+        prefetch_tmap(&xmap);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+    }
+    if (blockIdx.x == 0 && out_lengths != nullptr)
+        for (int b = tid; b < g.B; b += blockDim.x) out_lengths[b] = out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
+    __syncthreads();
+
+    auto valid = [&](int tile) {
+        int b, it, jt, cs;
+        decode(g, tile, b, it, jt, cs);
+        return it * g.TI < out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
+    };
+    int cursor = blockIdx.x, issued = 0;  // producer state (thread 0)
+    auto issue_next = [&]() {
+        while (cursor < ntiles && !valid(cursor)) cursor += gridDim.x;
+        if (cursor >= ntiles) return;
+        int b, it, jt, cs;
+        decode(g, cursor, b, it, jt, cs);
+        const int s = issued & 1;
+        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(g.tx_bytes));
+        tma_load_4d(sm.stage[s], &xmap, cs * g.CS, jt * g.TJ * g.sf - g.pf, it * g.TI * g.st - g.pt, b, &sm.full[s]);
+        ++issued;
+        cursor += gridDim.x;
+    };
+    if (tid == 0) issue_next();
+
+    int n = 0;  // valid tiles consumed
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        int b, it, jt, cs;
+        decode(g, tile, b, it, jt, cs);
+        const int L = static_cast<int>(clamp_len(lengths, b, g.T));
+        const int Lo = out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
+        const int i0 = it * g.TI, j = jt * g.TJ + jl, c = cs * g.CS + cv * kC2V;
+        const bool col_ok = active && j < g.Fo && c < g.C;
+        T *yb = y + ((static_cast<int64_t>(b) * g.To) * g.Fo + j) * g.C + c;
+        const int64_t row_stride = static_cast<int64_t>(g.Fo) * g.C;
+        if (i0 >= Lo) {  // every row masked: zeros, no copy
+            if (col_ok)
+                for (int i = i0; i < i0 + g.TI && i < g.To; ++i) Vec<T, kC2V>::store_zero(yb + i * row_stride);
+            continue;
+        }
+        if (tid == 0) issue_next();  // the next valid tile into the other stage
+        const int s = n & 1;
+        const bool ok = mbar_wait(&sm.full[s], (n >> 1) & 1);
+        if (__syncthreads_or(!ok)) {  // a copy never arrived (error word set): drain and leave
+            if (tid == 0 && issued > n + 1) mbar_wait(&sm.full[s ^ 1], ((n + 1) >> 1) & 1);
+            return;
+        }
+        if (col_ok) {
+            float2 wr[9][2], bv[2];
+#pragma unroll
+            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
+            if (bias != nullptr) {
+                load_param<kC2V>(bias + c, bv);
+            } else {
+                bv[0] = bv[1] = make_float2(0.f, 0.f);
+            }
+            const T *tileb = reinterpret_cast<const T *>(sm.stage[s]) + cv * kC2V;
+            for (int il = 0; il < g.TI; ++il) {
+                const int i = i0 + il;
+                if (i >= g.To) break;
+                if (i >= Lo) {
+                    Vec<T, kC2V>::store_zero(yb + i * row_stride);
+                    continue;
+                }
+                float2 acc[2] = {bv[0], bv[1]};
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const int rl = il * g.st + p;           // box row
+                    const int r = i * g.st + p - g.pt;      // input frame
+                    if (r >= L) continue;                  // frames at/after len_b are padding
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        float2 xv[2];
+                        lds_vec<T>(tileb + (static_cast<int64_t>(rl) * g.BF + jl * g.sf + q) * g.CS, xv);
+                        acc[0] = ffma2(xv[0], wr[p * 3 + q][0], acc[0]);
+                        acc[1] = ffma2(xv[1], wr[p * 3 + q][1], acc[1]);
+                    }
+                }
+                Vec<T, kC2V>::store(yb + i * row_stride, acc);
+            }
+        }
+        __syncthreads();  // stage s is free for the copy issued at the next valid tile
+        ++n;
+    }
+}
+
+
+// ------------------------------------------------------------------------------ data gradient
+// dx[b,t,f,c] = [t < len_b] sum over taps (p, q) with (t + pt - p) = st i, (f + pf - q) = sf j,
+// 0 <= i < Lo_b, 0 <= j < Fo of dy[b,i,j,c] w[p,q,c]  (the transpose of the forward map, as a gather).
+// Tile = TI rows x TJ columns of dx x CS channels; the box covers dy rows floor((t0+pt-2)/st) ..
+// + BR and columns floor((f0+pf-2)/sf) .. + BF.  Per tile, a table gives for each (dx row, p)
+// the box row of its dy term or -1; each thread's column gives the same for q.
+template <typename T>
+__global__ void __launch_bounds__(512)
+c2_dx_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restrict__ w, T *__restrict__ dx,
+                 const int32_t *__restrict__ lengths, C2Geo g) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const C2Smem sm = c2_smem(smem_raw, g.stage_bytes);
+    int *rowtab = reinterpret_cast<int *>(sm.stage[1] + g.stage_bytes);  // [TI][3]
+    const int tid = threadIdx.x;
+    const int CSV = g.CS / kC2V;
+    const int cv = tid % CSV, jl = tid / CSV;
+    const bool active = jl < g.TJ;
+    const int ntiles = g.B * g.nI * g.nJ * g.nCS;
+    if (tid == 0) {
+        prefetch_tmap(&gmap);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto floordiv = [](int a, int d) { return a >= 0 ? a / d : -((-a + d - 1) / d); };
+    auto valid = [&](int tile) {
+        int b, it, jt, cs;
+        decode(g, tile, b, it, jt, cs);
+        return it * g.TI < static_cast<int>(clamp_len(lengths, b, g.T));
+    };
+    int cursor = blockIdx.x, issued = 0;
+    auto issue_next = [&]() {
+        while (cursor < ntiles && !valid(cursor)) cursor += gridDim.x;
+        if (cursor >= ntiles) return;
+        int b, it, jt, cs;
+        decode(g, cursor, b, it, jt, cs);
+        const int s = issued & 1;
+        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(g.tx_bytes));
+        tma_load_4d(sm.stage[s], &gmap, cs * g.CS, floordiv(jt * g.TJ + g.pf - 2, g.sf),
+                    floordiv(it * g.TI + g.pt - 2, g.st), b, &sm.full[s]);
+        ++issued;
+        cursor += gridDim.x;
+    };
+    if (tid == 0) issue_next();
+
+    int n = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        int b, it, jt, cs;
+        decode(g, tile, b, it, jt, cs);
+        const int L = static_cast<int>(clamp_len(lengths, b, g.T));
+        const int t0 = it * g.TI, f = jt * g.TJ + jl, c = cs * g.CS + cv * kC2V;
+        const bool col_ok = active && f < g.F && c < g.C;
+        T *xb = dx + ((static_cast<int64_t>(b) * g.T) * g.F + f) * g.C + c;
+        const int64_t row_stride = static_cast<int64_t>(g.F) * g.C;
+        if (t0 >= L) {
+            if (col_ok)
+                for (int t = t0; t < t0 + g.TI && t < g.T; ++t) Vec<T, kC2V>::store_zero(xb + t * row_stride);
+            continue;
+        }
+        if (tid == 0) issue_next();
+        const int Lo = out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
+        const int ia = floordiv(t0 + g.pt - 2, g.st);
+        for (int e = tid; e < g.TI * 3; e += blockDim.x) {  // (row, p) -> box row or -1
+            const int u = t0 + e / 3 + g.pt - e % 3;
+            int rb = -1;
+            if (u >= 0 && u % g.st == 0 && u / g.st < Lo) rb = u / g.st - ia;
+            rowtab[e] = rb;
+        }
+        int cb[3];
+        {
+            const int ja = floordiv(jt * g.TJ + g.pf - 2, g.sf);
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const int v = f + g.pf - q;
+                cb[q] = (v >= 0 && v % g.sf == 0 && v / g.sf < g.Fo) ? v / g.sf - ja : -1;
+            }
+        }
+        const int s = n & 1;
+        const bool ok = mbar_wait(&sm.full[s], (n >> 1) & 1);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0 && issued > n + 1) mbar_wait(&sm.full[s ^ 1], ((n + 1) >> 1) & 1);
+            return;
+        }
+        if (col_ok) {
+            float2 wr[9][2];
+#pragma unroll
+            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
+            const T *tileb = reinterpret_cast<const T *>(sm.stage[s]) + cv * kC2V;
+            for (int tl = 0; tl < g.TI; ++tl) {
+                const int t = t0 + tl;
+                if (t >= g.T) break;
+                if (t >= L) {
+                    Vec<T, kC2V>::store_zero(xb + t * row_stride);
+                    continue;
+                }
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const int rb = rowtab[tl * 3 + p];
+                    if (rb < 0) continue;
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        if (cb[q] < 0) continue;
+                        float2 gv[2];
+                        lds_vec<T>(tileb + (static_cast<int64_t>(rb) * g.BF + cb[q]) * g.CS, gv);
+                        acc[0] = ffma2(gv[0], wr[p * 3 + q][0], acc[0]);
+                        acc[1] = ffma2(gv[1], wr[p * 3 + q][1], acc[1]);
+                    }
+                }
+                Vec<T, kC2V>::store(xb + t * row_stride, acc);
+            }
+        }
+        __syncthreads();
+        ++n;
+    }
+}
+
+// ------------------------------------------------------------------------------ weight gradient
+// dW[p,q,c] = sum_{b, i < Lo_b, j} dy[b,i,j,c] xpad[b, st i + p, sf j + q, c];  dbias = sum dy.
+// CTA (slab cs, index gi) walks tiles gi, gi + G, ... of its channel slab; per tile it stages the
+// x box of the forward tile and the dy box (TI rows x TJ columns).  Thread = (channel vector cv,
+// position group pg) keeps 9 + 1 accumulator vectors over every position (i, j) of its group;
+// at the end the groups are added in a fixed order through shared memory and the CTA writes
+// partial row gi: partials[gi][slot][c], slots 0..8 the taps and 9 the bias.
+template <typename T>
+__global__ void __launch_bounds__(128)
+c2_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap gmap,
+                 const int32_t *__restrict__ lengths, float *__restrict__ partials, C2Geo g, int G, int xbytes) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const C2Smem sm = c2_smem(smem_raw, g.stage_bytes);
+    const int tid = threadIdx.x;
+    const int CSV = g.CS / kC2V;
+    const int cv = tid % CSV, pg = tid / CSV, NPG = blockDim.x / CSV;
+    const int cs = blockIdx.x % g.nCS, gi = blockIdx.x / g.nCS;
+    const int c = cs * g.CS + cv * kC2V;
+    const int ntiles = g.B * g.nI * g.nJ;  // tiles of one slab
+    if (tid == 0) {
+        prefetch_tmap(&xmap);
+        prefetch_tmap(&gmap);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto dec = [&](int tile, int &b, int &it, int &jt) {
+        jt = tile % g.nJ;
+        const int r = tile / g.nJ;
+        it = r % g.nI;
+        b = r / g.nI;
+    };
+    auto valid = [&](int tile) {
+        int b, it, jt;
+        dec(tile, b, it, jt);
+        return it * g.TI < out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
+    };
+    int cursor = gi, issued = 0;
+    auto issue_next = [&]() {
+        while (cursor < ntiles && !valid(cursor)) cursor += G;
+        if (cursor >= ntiles) return;
+        int b, it, jt;
+        dec(cursor, b, it, jt);
+        const int s = issued & 1;
+        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(g.tx_bytes));
+        tma_load_4d(sm.stage[s], &xmap, cs * g.CS, jt * g.TJ * g.sf - g.pf, it * g.TI * g.st - g.pt, b, &sm.full[s]);
+        tma_load_4d(sm.stage[s] + xbytes, &gmap, cs * g.CS, jt * g.TJ, it * g.TI, b, &sm.full[s]);
+        ++issued;
+        cursor += G;
+    };
+    if (tid == 0) issue_next();
+
+    float2 acc[10][2];
+#pragma unroll
+    for (int k = 0; k < 10; ++k) acc[k][0] = acc[k][1] = make_float2(0.f, 0.f);
+    const int npos = g.TI * g.TJ;
+    int n = 0;
+    for (int tile = gi; tile < ntiles; tile += G) {
+        int b, it, jt;
+        dec(tile, b, it, jt);
+        const int Lo = out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
+        const int i0 = it * g.TI, j0 = jt * g.TJ;
+        if (i0 >= Lo) continue;  // no unmasked output row: nothing to add
+        if (tid == 0) issue_next();
+        const int L = static_cast<int>(clamp_len(lengths, b, g.T));
+        const int s = n & 1;
+        const bool ok = mbar_wait(&sm.full[s], (n >> 1) & 1);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0 && issued > n + 1) mbar_wait(&sm.full[s ^ 1], ((n + 1) >> 1) & 1);
+            return;
+        }
+        if (c < g.C) {
+            const T *xs = reinterpret_cast<const T *>(sm.stage[s]) + cv * kC2V;
+            const T *gs = reinterpret_cast<const T *>(sm.stage[s] + xbytes) + cv * kC2V;
+            for (int pos = pg; pos < npos; pos += NPG) {
+                const int il = pos / g.TJ, jl = pos % g.TJ;
+                const int i = i0 + il;
+                if (i >= Lo || j0 + jl >= g.Fo) continue;
+                float2 gv[2];
+                lds_vec<T>(gs + static_cast<int64_t>(pos) * g.CS, gv);
+                acc[9][0].x += gv[0].x;
+                acc[9][0].y += gv[0].y;
+                acc[9][1].x += gv[1].x;
+                acc[9][1].y += gv[1].y;
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const int r = i * g.st + p - g.pt;
+                    if (r < 0 || r >= L) continue;  // padding, or a frame at/after len_b
+                    const T *xr = xs + static_cast<int64_t>(il * g.st + p) * g.BF * g.CS;
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        float2 xv[2];
+                        lds_vec<T>(xr + static_cast<int64_t>(jl * g.sf + q) * g.CS, xv);
+                        acc[p * 3 + q][0] = ffma2(gv[0], xv[0], acc[p * 3 + q][0]);
+                        acc[p * 3 + q][1] = ffma2(gv[1], xv[1], acc[p * 3 + q][1]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        ++n;
+    }
+    // fixed-order sum over the position groups (the stages are free: the last copy was consumed)
+    float *red = reinterpret_cast<float *>(sm.stage[0]);  // [NPG][10][CS]
+#pragma unroll
+    for (int k = 0; k < 10; ++k) {
+        float *d = red + (static_cast<int64_t>(pg) * 10 + k) * g.CS + cv * kC2V;
+        d[0] = acc[k][0].x;
+        d[1] = acc[k][0].y;
+        d[2] = acc[k][1].x;
+        d[3] = acc[k][1].y;
+    }
+    __syncthreads();
+    for (int e = tid; e < 10 * g.CS; e += blockDim.x) {
+        const int k = e / g.CS, ch = e % g.CS;
+        if (cs * g.CS + ch >= g.C) continue;
+        float sum = 0.f;
+        for (int q = 0; q < NPG; ++q) sum += red[(static_cast<int64_t>(q) * 10 + k) * g.CS + ch];
+        partials[(static_cast<int64_t>(gi) * 10 + k) * g.C + cs * g.CS + ch] = sum;
+    }
+}
+
+// ------------------------------------------------------------------------------ host side
+cudaError_t make_map_4d(CUtensorMap *map, const void *base, bool bf16, int64_t B, int64_t T, int64_t F, int64_t C,
+                        int box_c, int box_f, int box_t) {
+    TensorMapEncodeTiledFn enc = tensor_map_encoder();
+    if (enc == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t es = bf16 ? 2 : 4;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(T),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * es, static_cast<cuuint64_t>(F * C) * es,
+                                   static_cast<cuuint64_t>(T * F * C) * es};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_c), static_cast<cuuint32_t>(box_f),
+                               static_cast<cuuint32_t>(box_t), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                           const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorNotSupported;
+}
+
+bool aligned16(const void *p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+bool aligned8(const void *p) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % 8 == 0; }
+
+// 3x3 window; channels-last rows 16-byte aligned; every count of the tensor map in range.
+bool c2_eligible(const Conv2dArgs &a, const void *act0, const void *act1) {
+    const int es = a.bf16 ? 2 : 4;
+    if (a.KT != 3 || a.KF != 3) return false;
+    if ((a.C * es) % 16 != 0 || !aligned16(act0) || !aligned16(act1)) return false;
+    if (!aligned8(a.w) || !aligned8(a.bias)) return false;
+    if (a.B * a.T >= (int64_t(1) << 31) || a.B * a.To >= (int64_t(1) << 31)) return false;
+    return true;
+}
+
+// Smallest power-of-two channel slab >= C, between 32 and cs_max (C is a multiple of 4 here).
+int pick_cs(int64_t C, int cs_max) {
+    int cs = 32;
+    while (cs < cs_max && cs < C) cs *= 2;
+    return cs;
+}
+
+int blocks_per_sm(const void *kern, int threads, size_t smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess || n < 1) n = 1;
+    return n;
+}
+
+template <typename T>
+cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
+    const int es = sizeof(T);
+    C2Geo g{};
+    g.B = static_cast<int>(a.B); g.T = static_cast<int>(a.T); g.F = static_cast<int>(a.F); g.C = static_cast<int>(a.C);
+    g.To = static_cast<int>(a.To); g.Fo = static_cast<int>(a.Fo);
+    g.st = a.st; g.sf = a.sf; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
+    g.CS = pick_cs(a.C, 64);
+    g.TJ = static_cast<int>(a.Fo < 16 ? a.Fo : 16);
+    g.BF = a.sf * (g.TJ - 1) + 3;
+    if (g.BF > 256) return cudaErrorNotSupported;
+    const int pix = g.BF * g.CS * es;
+    g.TI = 0;
+    for (int ti : {8, 4, 2, 1}) {
+        const int br = a.st * (ti - 1) + 3;
+        if (br <= 256 && br * pix <= kC2StageMax) {
+            g.TI = ti;
+            break;
+        }
+    }
+    if (g.TI == 0) return cudaErrorNotSupported;
+    g.BR = a.st * (g.TI - 1) + 3;
+    g.nI = static_cast<int>((a.To + g.TI - 1) / g.TI);
+    g.nJ = static_cast<int>((a.Fo + g.TJ - 1) / g.TJ);
+    g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
+    g.stage_bytes = g.tx_bytes = g.BR * pix;
+    CUtensorMap map;
+    cudaError_t e = make_map_4d(&map, a.x, sizeof(T) == 2, a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
+    if (e != cudaSuccess) return e;
+    const int threads = ((g.TJ * (g.CS / kC2V) + 31) / 32) * 32;
+    const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes);
+    auto kern = c2_fwd_tma_kernel<T>;
+    if ((e = ensure_smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(smem))) != cudaSuccess) return e;
+    const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
+    if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;  // tile indices stay far from int overflow
+    const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem);
+    const int grid = static_cast<int>(ntiles < cap ? ntiles : cap);
+    kern<<<grid, threads, smem, s>>>(map, a.w, a.bias, static_cast<T *>(a.y), a.lengths, a.out_lengths, g);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dx_tma(const Conv2dArgs &a, cudaStream_t s) {
+    const int es = sizeof(T);
+    C2Geo g{};
+    g.B = static_cast<int>(a.B); g.T = static_cast<int>(a.T); g.F = static_cast<int>(a.F); g.C = static_cast<int>(a.C);
+    g.To = static_cast<int>(a.To); g.Fo = static_cast<int>(a.Fo);
+    g.st = a.st; g.sf = a.sf; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
+    g.CS = pick_cs(a.C, 128);
+    const int csv = g.CS / kC2V;
+    g.TJ = static_cast<int>(a.F < 512 / csv ? a.F : 512 / csv);
+    g.BF = (g.TJ + a.sf) / a.sf + 1;
+    const int pix = g.BF * g.CS * es;
+    g.TI = 0;
+    for (int ti : {32, 16, 8, 4, 2, 1}) {
+        const int br = (ti + a.st) / a.st + 1;
+        if (br <= 256 && br * pix <= kC2StageMax) {
+            g.TI = ti;
+            break;
+        }
+    }
+    if (g.TI == 0 || g.BF > 256) return cudaErrorNotSupported;
+    g.BR = (g.TI + a.st) / a.st + 1;
+    g.nI = static_cast<int>((a.T + g.TI - 1) / g.TI);
+    g.nJ = static_cast<int>((a.F + g.TJ - 1) / g.TJ);
+    g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
+    g.stage_bytes = g.tx_bytes = g.BR * pix;
+    CUtensorMap map;
+    cudaError_t e = make_map_4d(&map, a.x, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.BF, g.BR);
+    if (e != cudaSuccess) return e;
+    const int threads = ((g.TJ * csv + 31) / 32) * 32;
+    const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes) + static_cast<size_t>(g.TI) * 3 * sizeof(int);
+    auto kern = c2_dx_tma_kernel<T>;
+    if ((e = ensure_smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(smem))) != cudaSuccess) return e;
+    const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
+    if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;  // tile indices stay far from int overflow
+    const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem);
+    const int grid = static_cast<int>(ntiles < cap ? ntiles : cap);
+    kern<<<grid, threads, smem, s>>>(map, a.w, static_cast<T *>(a.y), a.lengths, g);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dw_tma(const Conv2dArgs &a, float *partials, int max_rows, int *G_out, cudaStream_t s) {
+    const int es = sizeof(T);
+    C2Geo g{};
+    g.B = static_cast<int>(a.B); g.T = static_cast<int>(a.T); g.F = static_cast<int>(a.F); g.C = static_cast<int>(a.C);
+    g.To = static_cast<int>(a.To); g.Fo = static_cast<int>(a.Fo);
+    g.st = a.st; g.sf = a.sf; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
+    g.CS = pick_cs(a.C, 64);
+    g.TJ = static_cast<int>(a.Fo < 16 ? a.Fo : 16);
+    g.BF = a.sf * (g.TJ - 1) + 3;
+    if (g.BF > 256) return cudaErrorNotSupported;
+    const int pix = g.BF * g.CS * es;
+    g.TI = 0;
+    for (int ti : {4, 2, 1}) {
+        const int br = a.st * (ti - 1) + 3;
+        const int xb = ((br * pix + 127) / 128) * 128;
+        if (br <= 256 && xb + ti * g.TJ * g.CS * es <= kC2StageMax) {
+            g.TI = ti;
+            break;
+        }
+    }
+    if (g.TI == 0) return cudaErrorNotSupported;
+    g.BR = a.st * (g.TI - 1) + 3;
+    g.nI = static_cast<int>((a.To + g.TI - 1) / g.TI);
+    g.nJ = static_cast<int>((a.Fo + g.TJ - 1) / g.TJ);
+    g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
+    const int xbytes = ((g.BR * pix + 127) / 128) * 128;
+    g.stage_bytes = xbytes + g.TI * g.TJ * g.CS * es;
+    g.tx_bytes = g.BR * pix + g.TI * g.TJ * g.CS * es;
+    CUtensorMap xm, gm;
+    cudaError_t e = make_map_4d(&xm, a.x, sizeof(T) == 2, a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
+    if (e != cudaSuccess) return e;
+    if ((e = make_map_4d(&gm, a.y, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.TJ, g.TI)) != cudaSuccess) return e;
+    const int threads = (g.CS / kC2V) * kC2DwGroups;
+    // the final reduction [groups][10][CS] float32 reuses the stages
+    const size_t red = static_cast<size_t>(kC2DwGroups) * 10 * g.CS * sizeof(float);
+    const size_t stages = 2 * static_cast<size_t>(g.stage_bytes);
+    const size_t smem = kC2Head + (red > stages ? red : stages);
+    auto kern = c2_dw_tma_kernel<T>;
+    if ((e = ensure_smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(smem))) != cudaSuccess) return e;
+    const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ;
+    if (ntiles * g.nCS >= (int64_t(1) << 30)) return cudaErrorNotSupported;
+    int64_t G = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem) /
+                g.nCS;
+    if (G > ntiles) G = ntiles;
+    if (G > max_rows) G = max_rows;
+    if (G < 1) G = 1;
+    kern<<<static_cast<unsigned>(G * g.nCS), threads, smem, s>>>(xm, gm, a.lengths, partials, g, static_cast<int>(G),
+                                                                 xbytes);
+    *G_out = static_cast<int>(G);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t conv2d_fwd_tma_launch(const Conv2dArgs &a, cudaStream_t s) {
+    if (a.B == 0 || a.To == 0 || a.Fo == 0 || !c2_eligible(a, a.x, a.y)) return cudaErrorNotSupported;
+    return a.bf16 ? fwd_tma<bf16>(a, s) : fwd_tma<float>(a, s);
+}
+
+cudaError_t conv2d_dx_tma_launch(const Conv2dArgs &a, cudaStream_t s) {
+    if (a.B == 0 || a.T == 0 || a.To == 0 || a.Fo == 0 || !c2_eligible(a, a.x, a.y)) return cudaErrorNotSupported;
+    return a.bf16 ? dx_tma<bf16>(a, s) : dx_tma<float>(a, s);
+}
+
+cudaError_t conv2d_dw_tma_partials(const Conv2dArgs &a, float *partials, int max_rows, int *G, cudaStream_t s) {
+    if (a.B == 0 || a.To == 0 || a.Fo == 0 || !c2_eligible(a, a.x, a.y)) return cudaErrorNotSupported;
+    return a.bf16 ? dw_tma<bf16>(a, partials, max_rows, G, s) : dw_tma<float>(a, partials, max_rows, G, s);
+}
+
+unsigned int conv2d_tma_take_error() {
+    unsigned int h = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&h, dw_device_error_flag, sizeof(h)) != cudaSuccess) return 0;
+    if (h) cudaMemcpyToSymbol(dw_device_error_flag, &zero, sizeof(zero));
+    return h;
+}
+
+}  // namespace dwk

@@ -112,6 +112,12 @@ cudaError_t conv2d_dx_launch(const Conv2dArgs &a, cudaStream_t s);
 int conv2d_dw_partial_rows(int64_t B, int64_t To);
 size_t conv2d_dw_workspace_bytes(int64_t B, int64_t To, int64_t C, int KT, int KF);
 cudaError_t conv2d_dw_launch(const Conv2dArgs &a, float *dw, float *dbias, float *partials, cudaStream_t s);
+// TMA-staged kernels for the 3x3 window (16-byte aligned rows); cudaErrorNotSupported otherwise.
+cudaError_t conv2d_fwd_tma_launch(const Conv2dArgs &a, cudaStream_t s);
+cudaError_t conv2d_dx_tma_launch(const Conv2dArgs &a, cudaStream_t s);
+// Writes partial rows [G][10][C] (G <= max_rows) for the fixed-order finalize.
+cudaError_t conv2d_dw_tma_partials(const Conv2dArgs &a, float *partials, int max_rows, int *G, cudaStream_t s);
+unsigned int conv2d_tma_take_error();
 
 struct SubsampleBwdArgs {
     const float *mel, *w0, *b0, *w1;

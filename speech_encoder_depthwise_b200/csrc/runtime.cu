@@ -13,19 +13,27 @@ int sm_count() {
     return n;
 }
 
+// The limit only ever grows, and never below the 48 KiB default: a kernel launched with
+// different amounts of shared memory keeps working for every size requested so far.
 cudaError_t ensure_smem_attr(const void *kern, int bytes) {
     static std::mutex mu;
-    static struct Entry { const void *k; int dev; } done[256];
+    static struct Entry { const void *k; int dev; int bytes; } done[256];
     static int n_done = 0;
+    constexpr int kDefault = 48 * 1024;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const int want = bytes > kDefault ? bytes : kDefault;
     std::lock_guard<std::mutex> lock(mu);
+    Entry *hit = nullptr;
     for (int i = 0; i < n_done; ++i)
-        if (done[i].k == kern && done[i].dev == dev) return cudaSuccess;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && n_done < 256) done[n_done++] = {kern, dev};
-    return e;
+        if (done[i].k == kern && done[i].dev == dev) hit = &done[i];
+    if (hit != nullptr && hit->bytes >= want) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+    if (e != cudaSuccess) return e;
+    if (hit != nullptr) hit->bytes = want;
+    else if (n_done < 256) done[n_done++] = {kern, dev, want};
+    return cudaSuccess;
 }
 
 TensorMapEncodeTiledFn tensor_map_encoder() {
