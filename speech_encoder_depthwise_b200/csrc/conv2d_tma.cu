@@ -19,7 +19,6 @@ namespace {
 
 constexpr int kC2V = 4;             // channels per thread (8 bytes bf16, 16 bytes float32)
 constexpr int kC2StageMax = 49152;  // bytes of one stage
-constexpr int kC2DwGroups = 8;      // position groups of the weight-gradient CTA
 
 __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c, int f, int t, int b, uint64_t *bar) {
     asm volatile(
@@ -88,7 +87,7 @@ __device__ __forceinline__ C2Smem c2_smem(unsigned char *raw, int stage_bytes) {
 // Tile = TI output rows x TJ output columns x CS channels of one item; the box covers input rows
 // st*i0 - pt .. + BR and columns sf*j0 - pf .. + BF.  Thread = (column j, channel vector cv) and
 // walks the TI rows; blockDim = TJ * CS/4 rounded up to a warp.
-template <typename T>
+template <typename T, int ST>
 __global__ void __launch_bounds__(512)
 c2_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restrict__ w,
                   const float *__restrict__ bias, T *__restrict__ y, const int32_t *__restrict__ lengths,
@@ -160,29 +159,68 @@ c2_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restr
             } else {
                 bv[0] = bv[1] = make_float2(0.f, 0.f);
             }
-            const T *tileb = reinterpret_cast<const T *>(sm.stage[s]) + cv * kC2V;
-            for (int il = 0; il < g.TI; ++il) {
-                const int i = i0 + il;
-                if (i >= g.To) break;
-                if (i >= Lo) {
-                    Vec<T, kC2V>::store_zero(yb + i * row_stride);
-                    continue;
-                }
-                float2 acc[2] = {bv[0], bv[1]};
-#pragma unroll
-                for (int p = 0; p < 3; ++p) {
-                    const int rl = il * g.st + p;           // box row
-                    const int r = i * g.st + p - g.pt;      // input frame
-                    if (r >= L) continue;                  // frames at/after len_b are padding
-#pragma unroll
-                    for (int q = 0; q < 3; ++q) {
-                        float2 xv[2];
-                        lds_vec<T>(tileb + (static_cast<int64_t>(rl) * g.BF + jl * g.sf + q) * g.CS, xv);
-                        acc[0] = ffma2(xv[0], wr[p * 3 + q][0], acc[0]);
-                        acc[1] = ffma2(xv[1], wr[p * 3 + q][1], acc[1]);
+            // this thread's column of the box; 32-bit element offsets inside the stage
+            const T *tb = reinterpret_cast<const T *>(sm.stage[s]) + (jl * g.sf * g.CS + cv * kC2V);
+            const int RS = g.BF * g.CS;  // box row stride
+            auto put = [&](int i, const float2 (&acc)[2]) {
+                if (i >= g.To) return;
+                if (i < Lo) Vec<T, kC2V>::store(yb + i * row_stride, acc);
+                else Vec<T, kC2V>::store_zero(yb + i * row_stride);
+            };
+            if constexpr (ST > 0) {
+                // two output rows per step: input rows i*ST + pp - pt, pp < ST + 3, feed row i
+                // through tap pp and row i+1 through tap pp - ST (two independent chains)
+                for (int il = 0; il < g.TI; il += 2) {
+                    const int i = i0 + il;
+                    if (i >= g.To || i >= Lo) {
+                        put(i, bv);
+                        put(i + 1, bv);
+                        continue;
                     }
+                    float2 a0[2] = {bv[0], bv[1]}, a1[2] = {bv[0], bv[1]};
+#pragma unroll
+                    for (int pp = 0; pp < ST + 3; ++pp) {
+                        if (i * ST + pp - g.pt >= L) break;  // this and later frames are padding
+                        const T *row = tb + (il * ST + pp) * RS;
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            float2 xv[2];
+                            lds_vec<T>(row + q * g.CS, xv);
+                            if (pp < 3) {
+                                a0[0] = ffma2(xv[0], wr[pp * 3 + q][0], a0[0]);
+                                a0[1] = ffma2(xv[1], wr[pp * 3 + q][1], a0[1]);
+                            }
+                            if (pp >= ST && pp - ST < 3) {
+                                a1[0] = ffma2(xv[0], wr[(pp - ST) * 3 + q][0], a1[0]);
+                                a1[1] = ffma2(xv[1], wr[(pp - ST) * 3 + q][1], a1[1]);
+                            }
+                        }
+                    }
+                    put(i, a0);
+                    put(i + 1, a1);
                 }
-                Vec<T, kC2V>::store(yb + i * row_stride, acc);
+            } else {
+                for (int il = 0; il < g.TI; ++il) {
+                    const int i = i0 + il;
+                    if (i >= g.To || i >= Lo) {
+                        put(i, bv);
+                        continue;
+                    }
+                    float2 acc[2] = {bv[0], bv[1]};
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        if (i * g.st + p - g.pt >= L) break;  // frames at/after len_b are padding
+                        const T *row = tb + (il * g.st + p) * RS;
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            float2 xv[2];
+                            lds_vec<T>(row + q * g.CS, xv);
+                            acc[0] = ffma2(xv[0], wr[p * 3 + q][0], acc[0]);
+                            acc[1] = ffma2(xv[1], wr[p * 3 + q][1], acc[1]);
+                        }
+                    }
+                    put(i, acc);
+                }
             }
         }
         __syncthreads();  // stage s is free for the copy issued at the next valid tile
@@ -309,15 +347,158 @@ c2_dx_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restri
     }
 }
 
+// Stride 2 in both axes: dx row pairs (t, t+1) and column pairs (f, f+1) with t, f even draw
+// on a 2x2 block of dy: rows ilo = floor((t + pt - 1)/2) and ilo+1, columns likewise.  Which
+// taps link them depends only on the parity of pt (rows) and of pf (columns), the same for the
+// whole launch (RODD, CODD).  For one axis, with "lo"/"hi" the first/second dy row of the pair:
+//   pad even: out0 = hi*tap0 + lo*tap2,  out1 = hi*tap1
+//   pad odd:  out0 = lo*tap1,            out1 = hi*tap0 + lo*tap2
+// Thread = (column pair m, channel vector cv) walking the row pairs of the tile, keeping the
+// "hi" dy row of one step as the "lo" row of the next: two shared-memory loads per 4 outputs.
+__host__ __device__ constexpr int ph_n(bool odd, int r) { return (odd ? r == 1 : r == 0) ? 2 : 1; }
+__host__ __device__ constexpr int ph_sel(bool odd, int r, int e) {
+    return ph_n(odd, r) == 2 ? (e == 0 ? 1 : 0) : (odd ? 0 : 1);
+}
+__host__ __device__ constexpr int ph_tap(bool odd, int r, int e) { return ph_n(odd, r) == 2 ? (e == 0 ? 0 : 2) : 1; }
+
+template <typename T, bool RODD, bool CODD>
+__global__ void __launch_bounds__(512)
+c2_dx2_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restrict__ w, T *__restrict__ dx,
+                  const int32_t *__restrict__ lengths, C2Geo g) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const C2Smem sm = c2_smem(smem_raw, g.stage_bytes);
+    const int tid = threadIdx.x;
+    const int CSV = g.CS / kC2V;
+    const int cv = tid % CSV, m = tid / CSV;
+    const bool active = m < g.TJ / 2;
+    const int ntiles = g.B * g.nI * g.nJ * g.nCS;
+    if (tid == 0) {
+        prefetch_tmap(&gmap);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto floordiv = [](int a, int d) { return a >= 0 ? a / d : -((-a + d - 1) / d); };
+    auto valid = [&](int tile) {
+        int b, it, jt, cs;
+        decode(g, tile, b, it, jt, cs);
+        return it * g.TI < static_cast<int>(clamp_len(lengths, b, g.T));
+    };
+    int cursor = blockIdx.x, issued = 0;
+    auto issue_next = [&]() {
+        while (cursor < ntiles && !valid(cursor)) cursor += gridDim.x;
+        if (cursor >= ntiles) return;
+        int b, it, jt, cs;
+        decode(g, cursor, b, it, jt, cs);
+        const int s = issued & 1;
+        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(g.tx_bytes));
+        tma_load_4d(sm.stage[s], &gmap, cs * g.CS, floordiv(jt * g.TJ + g.pf - 1, 2),
+                    floordiv(it * g.TI + g.pt - 1, 2), b, &sm.full[s]);
+        ++issued;
+        cursor += gridDim.x;
+    };
+    if (tid == 0) issue_next();
+
+    int n = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        int b, it, jt, cs;
+        decode(g, tile, b, it, jt, cs);
+        const int L = static_cast<int>(clamp_len(lengths, b, g.T));
+        const int t0 = it * g.TI, f = jt * g.TJ + 2 * m, c = cs * g.CS + cv * kC2V;
+        const bool col_ok = active && f < g.F && c < g.C;
+        const bool col1_ok = f + 1 < g.F;
+        T *xb = dx + ((static_cast<int64_t>(b) * g.T) * g.F + f) * g.C + c;
+        const int64_t row_stride = static_cast<int64_t>(g.F) * g.C;
+        auto put = [&](int t, int e, const float2 (&v)[2]) {  // dx[t, f + e]
+            if (t >= g.T || (e == 1 && !col1_ok)) return;
+            if (t < L) Vec<T, kC2V>::store(xb + t * row_stride + e * g.C, v);
+            else Vec<T, kC2V>::store_zero(xb + t * row_stride + e * g.C);
+        };
+        if (t0 >= L) {
+            if (col_ok) {
+                const float2 z[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                for (int t = t0; t < t0 + g.TI; ++t) {
+                    put(t, 0, z);
+                    put(t, 1, z);
+                }
+            }
+            continue;
+        }
+        if (tid == 0) issue_next();
+        const int Lo = out_len(lengths, b, g.T, g.pt, g.pb, 2, g.To);
+        const int ia = floordiv(t0 + g.pt - 1, 2);
+        const int s = n & 1;
+        const bool ok = mbar_wait(&sm.full[s], (n >> 1) & 1);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0 && issued > n + 1) mbar_wait(&sm.full[s ^ 1], ((n + 1) >> 1) & 1);
+            return;
+        }
+        if (col_ok) {
+            float2 wr[9][2];
+#pragma unroll
+            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
+            const T *tb = reinterpret_cast<const T *>(sm.stage[s]) + (m * g.CS + cv * kC2V);
+            const int RS = g.BF * g.CS;
+            float2 d[2][2][2];  // [lo/hi row][lo/hi column][pair]
+            auto load_row = [&](int k, float2 (&r)[2][2]) {  // box row k = dy row ia + k
+                const int i = ia + k;
+                if (i >= 0 && i < Lo) {
+                    lds_vec<T>(tb + k * RS, r[0]);
+                    lds_vec<T>(tb + k * RS + g.CS, r[1]);
+                } else {
+                    r[0][0] = r[0][1] = r[1][0] = r[1][1] = make_float2(0.f, 0.f);
+                }
+            };
+            load_row(0, d[0]);
+            for (int k = 0; 2 * k < g.TI; ++k) {
+                const int t = t0 + 2 * k;
+                if (t >= g.T) break;
+                load_row(k + 1, d[1]);
+                float2 out[2][2][2];
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                        for (int e = 0; e < ph_n(RODD, r); ++e)
+#pragma unroll
+                            for (int h = 0; h < ph_n(CODD, cc); ++h) {
+                                const int rs = ph_sel(RODD, r, e), cs2 = ph_sel(CODD, cc, h);
+                                const int tap = ph_tap(RODD, r, e) * 3 + ph_tap(CODD, cc, h);
+                                acc[0] = ffma2(d[rs][cs2][0], wr[tap][0], acc[0]);
+                                acc[1] = ffma2(d[rs][cs2][1], wr[tap][1], acc[1]);
+                            }
+                        out[r][cc][0] = acc[0];
+                        out[r][cc][1] = acc[1];
+                    }
+                put(t, 0, out[0][0]);
+                put(t, 1, out[0][1]);
+                put(t + 1, 0, out[1][0]);
+                put(t + 1, 1, out[1][1]);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    d[0][cc][0] = d[1][cc][0];
+                    d[0][cc][1] = d[1][cc][1];
+                }
+            }
+        }
+        __syncthreads();
+        ++n;
+    }
+}
+
 // ------------------------------------------------------------------------------ weight gradient
 // dW[p,q,c] = sum_{b, i < Lo_b, j} dy[b,i,j,c] xpad[b, st i + p, sf j + q, c];  dbias = sum dy.
 // CTA (slab cs, index gi) walks tiles gi, gi + G, ... of its channel slab; per tile it stages the
 // x box of the forward tile and the dy box (TI rows x TJ columns).  Thread = (channel vector cv,
-// position group pg) keeps 9 + 1 accumulator vectors over every position (i, j) of its group;
-// at the end the groups are added in a fixed order through shared memory and the CTA writes
-// partial row gi: partials[gi][slot][c], slots 0..8 the taps and 9 the bias.
-template <typename T>
-__global__ void __launch_bounds__(128)
+// tile column pg) keeps 9 + 1 accumulator vectors over the rows of its column (two rows per step,
+// sharing their common input row); at the end the columns are added in a fixed order through
+// shared memory and the CTA writes partial row gi: partials[gi][slot][c], slots 0..8 the taps
+// and 9 the bias.
+template <typename T, int ST>
+__global__ void __launch_bounds__(512)
 c2_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap gmap,
                  const int32_t *__restrict__ lengths, float *__restrict__ partials, C2Geo g, int G, int xbytes) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -365,7 +546,6 @@ c2_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     float2 acc[10][2];
 #pragma unroll
     for (int k = 0; k < 10; ++k) acc[k][0] = acc[k][1] = make_float2(0.f, 0.f);
-    const int npos = g.TI * g.TJ;
     int n = 0;
     for (int tile = gi; tile < ntiles; tile += G) {
         int b, it, jt;
@@ -381,30 +561,73 @@ c2_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
             if (tid == 0 && issued > n + 1) mbar_wait(&sm.full[s ^ 1], ((n + 1) >> 1) & 1);
             return;
         }
-        if (c < g.C) {
-            const T *xs = reinterpret_cast<const T *>(sm.stage[s]) + cv * kC2V;
-            const T *gs = reinterpret_cast<const T *>(sm.stage[s] + xbytes) + cv * kC2V;
-            for (int pos = pg; pos < npos; pos += NPG) {
-                const int il = pos / g.TJ, jl = pos % g.TJ;
-                const int i = i0 + il;
-                if (i >= Lo || j0 + jl >= g.Fo) continue;
-                float2 gv[2];
-                lds_vec<T>(gs + static_cast<int64_t>(pos) * g.CS, gv);
+        const int jl = pg;  // this thread's column of the tile
+        if (c < g.C && jl < g.TJ && j0 + jl < g.Fo) {
+            const T *xs = reinterpret_cast<const T *>(sm.stage[s]) + (jl * g.sf * g.CS + cv * kC2V);
+            const T *gs = reinterpret_cast<const T *>(sm.stage[s] + xbytes) + (jl * g.CS + cv * kC2V);
+            const int RS = g.BF * g.CS, GS = g.TJ * g.CS;  // box row strides (x, dy)
+            auto add_bias = [&](const float2 (&gv)[2]) {
                 acc[9][0].x += gv[0].x;
                 acc[9][0].y += gv[0].y;
                 acc[9][1].x += gv[1].x;
                 acc[9][1].y += gv[1].y;
+            };
+            if constexpr (ST > 0) {
+                // two output rows per step; input row i*ST + pp - pt meets row i through tap pp
+                // and row i+1 through tap pp - ST
+                for (int il = 0; il < g.TI; il += 2) {
+                    const int i = i0 + il;
+                    if (i >= Lo) break;  // later rows are masked too
+                    float2 g0[2], g1[2];
+                    lds_vec<T>(gs + il * GS, g0);
+                    if (i + 1 < Lo) {
+                        lds_vec<T>(gs + (il + 1) * GS, g1);
+                    } else {
+                        g1[0] = g1[1] = make_float2(0.f, 0.f);
+                    }
+                    add_bias(g0);
+                    add_bias(g1);
 #pragma unroll
-                for (int p = 0; p < 3; ++p) {
-                    const int r = i * g.st + p - g.pt;
-                    if (r < 0 || r >= L) continue;  // padding, or a frame at/after len_b
-                    const T *xr = xs + static_cast<int64_t>(il * g.st + p) * g.BF * g.CS;
+                    for (int pp = 0; pp < ST + 3; ++pp) {
+                        const int r = i * ST + pp - g.pt;
+                        if (r >= L) break;     // this and later frames are padding
+                        if (r < 0) continue;   // zero fill
+                        const T *xr = xs + (il * ST + pp) * RS;
 #pragma unroll
-                    for (int q = 0; q < 3; ++q) {
-                        float2 xv[2];
-                        lds_vec<T>(xr + static_cast<int64_t>(jl * g.sf + q) * g.CS, xv);
-                        acc[p * 3 + q][0] = ffma2(gv[0], xv[0], acc[p * 3 + q][0]);
-                        acc[p * 3 + q][1] = ffma2(gv[1], xv[1], acc[p * 3 + q][1]);
+                        for (int q = 0; q < 3; ++q) {
+                            float2 xv[2];
+                            lds_vec<T>(xr + q * g.CS, xv);
+                            if (pp < 3) {
+                                acc[pp * 3 + q][0] = ffma2(g0[0], xv[0], acc[pp * 3 + q][0]);
+                                acc[pp * 3 + q][1] = ffma2(g0[1], xv[1], acc[pp * 3 + q][1]);
+                            }
+                            if (pp >= ST && pp - ST < 3) {
+                                acc[(pp - ST) * 3 + q][0] = ffma2(g1[0], xv[0], acc[(pp - ST) * 3 + q][0]);
+                                acc[(pp - ST) * 3 + q][1] = ffma2(g1[1], xv[1], acc[(pp - ST) * 3 + q][1]);
+                            }
+                        }
+                    }
+                }
+            } else {
+                for (int il = 0; il < g.TI; ++il) {
+                    const int i = i0 + il;
+                    if (i >= Lo) break;
+                    float2 gv[2];
+                    lds_vec<T>(gs + il * GS, gv);
+                    add_bias(gv);
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        const int r = i * g.st + p - g.pt;
+                        if (r >= L) break;
+                        if (r < 0) continue;
+                        const T *xr = xs + (il * g.st + p) * RS;
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            float2 xv[2];
+                            lds_vec<T>(xr + q * g.CS, xv);
+                            acc[p * 3 + q][0] = ffma2(gv[0], xv[0], acc[p * 3 + q][0]);
+                            acc[p * 3 + q][1] = ffma2(gv[1], xv[1], acc[p * 3 + q][1]);
+                        }
                     }
                 }
             }
@@ -486,14 +709,14 @@ cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
     g.To = static_cast<int>(a.To); g.Fo = static_cast<int>(a.Fo);
     g.st = a.st; g.sf = a.sf; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
     g.CS = pick_cs(a.C, 64);
-    g.TJ = static_cast<int>(a.Fo < 16 ? a.Fo : 16);
+    g.TJ = static_cast<int>((a.Fo + (a.Fo + 15) / 16 - 1) / ((a.Fo + 15) / 16));  // <= 16, even split
     g.BF = a.sf * (g.TJ - 1) + 3;
     if (g.BF > 256) return cudaErrorNotSupported;
     const int pix = g.BF * g.CS * es;
     g.TI = 0;
-    for (int ti : {8, 4, 2, 1}) {
+    for (int ti : {4, 2, 1}) {
         const int br = a.st * (ti - 1) + 3;
-        if (br <= 256 && br * pix <= kC2StageMax) {
+        if (br <= 256 && br * pix <= kC2StageMax / 2) {
             g.TI = ti;
             break;
         }
@@ -509,7 +732,9 @@ cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int threads = ((g.TJ * (g.CS / kC2V) + 31) / 32) * 32;
     const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes);
-    auto kern = c2_fwd_tma_kernel<T>;
+    // the row-pair path needs an even row count per tile and a compiled stride
+    auto kern = (g.TI % 2 == 0 && a.st == 2) ? c2_fwd_tma_kernel<T, 2>
+                : (g.TI % 2 == 0 && a.st == 1) ? c2_fwd_tma_kernel<T, 1> : c2_fwd_tma_kernel<T, 0>;
     if ((e = ensure_smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(smem))) != cudaSuccess) return e;
     const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
     if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;  // tile indices stay far from int overflow
@@ -519,8 +744,56 @@ cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Stride 2 x 2: the 2x2-block kernel.  Tiles of TI (even) dx rows x TJ (even) columns; the box
+// holds dy rows ia .. ia + TI/2 and columns ja .. ja + TJ/2.
+template <typename T>
+cudaError_t dx2_tma(const Conv2dArgs &a, cudaStream_t s) {
+    const int es = sizeof(T);
+    C2Geo g{};
+    g.B = static_cast<int>(a.B); g.T = static_cast<int>(a.T); g.F = static_cast<int>(a.F); g.C = static_cast<int>(a.C);
+    g.To = static_cast<int>(a.To); g.Fo = static_cast<int>(a.Fo);
+    g.st = 2; g.sf = 2; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
+    g.CS = pick_cs(a.C, 64);
+    const int csv = g.CS / kC2V;
+    {  // column pairs per tile: at most 512 threads, the F columns split evenly over the tiles
+        const int64_t maxp = 512 / csv, pairs = (a.F + 1) / 2, nj = (pairs + maxp - 1) / maxp;
+        g.TJ = static_cast<int>(2 * ((pairs + nj - 1) / nj));
+    }
+    g.BF = g.TJ / 2 + 1;
+    const int pix = g.BF * g.CS * es;
+    g.TI = 0;
+    for (int ti : {16, 8, 4, 2}) {
+        if ((ti / 2 + 1) * pix <= kC2StageMax / 2) {
+            g.TI = ti;
+            break;
+        }
+    }
+    if (g.TI == 0 || g.BF > 256) return cudaErrorNotSupported;
+    g.BR = g.TI / 2 + 1;
+    g.nI = static_cast<int>((a.T + g.TI - 1) / g.TI);
+    g.nJ = static_cast<int>((a.F + g.TJ - 1) / g.TJ);
+    g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
+    g.stage_bytes = g.tx_bytes = g.BR * pix;
+    CUtensorMap map;
+    cudaError_t e = make_map_4d(&map, a.x, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.BF, g.BR);
+    if (e != cudaSuccess) return e;
+    const int threads = ((g.TJ / 2 * csv + 31) / 32) * 32;
+    const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes);
+    const bool ro = (a.pt & 1) != 0, co = (a.pf & 1) != 0;
+    auto kern = ro ? (co ? c2_dx2_tma_kernel<T, true, true> : c2_dx2_tma_kernel<T, true, false>)
+                   : (co ? c2_dx2_tma_kernel<T, false, true> : c2_dx2_tma_kernel<T, false, false>);
+    if ((e = ensure_smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(smem))) != cudaSuccess) return e;
+    const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
+    if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem);
+    const int grid = static_cast<int>(ntiles < cap ? ntiles : cap);
+    kern<<<grid, threads, smem, s>>>(map, a.w, static_cast<T *>(a.y), a.lengths, g);
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t dx_tma(const Conv2dArgs &a, cudaStream_t s) {
+    if (a.st == 2 && a.sf == 2) return dx2_tma<T>(a, s);
     const int es = sizeof(T);
     C2Geo g{};
     g.B = static_cast<int>(a.B); g.T = static_cast<int>(a.T); g.F = static_cast<int>(a.F); g.C = static_cast<int>(a.C);
@@ -528,7 +801,10 @@ cudaError_t dx_tma(const Conv2dArgs &a, cudaStream_t s) {
     g.st = a.st; g.sf = a.sf; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
     g.CS = pick_cs(a.C, 128);
     const int csv = g.CS / kC2V;
-    g.TJ = static_cast<int>(a.F < 512 / csv ? a.F : 512 / csv);
+    {  // columns per tile: at most 512 threads, the F columns split evenly over the tiles
+        const int64_t maxj = 512 / csv, nj = (a.F + maxj - 1) / maxj;
+        g.TJ = static_cast<int>((a.F + nj - 1) / nj);
+    }
     g.BF = (g.TJ + a.sf) / a.sf + 1;
     const int pix = g.BF * g.CS * es;
     g.TI = 0;
@@ -568,7 +844,7 @@ cudaError_t dw_tma(const Conv2dArgs &a, float *partials, int max_rows, int *G_ou
     g.To = static_cast<int>(a.To); g.Fo = static_cast<int>(a.Fo);
     g.st = a.st; g.sf = a.sf; g.pt = a.pt; g.pb = a.pb; g.pf = a.pf;
     g.CS = pick_cs(a.C, 64);
-    g.TJ = static_cast<int>(a.Fo < 16 ? a.Fo : 16);
+    g.TJ = static_cast<int>((a.Fo + (a.Fo + 15) / 16 - 1) / ((a.Fo + 15) / 16));  // <= 16, even split
     g.BF = a.sf * (g.TJ - 1) + 3;
     if (g.BF > 256) return cudaErrorNotSupported;
     const int pix = g.BF * g.CS * es;
@@ -593,12 +869,13 @@ cudaError_t dw_tma(const Conv2dArgs &a, float *partials, int max_rows, int *G_ou
     cudaError_t e = make_map_4d(&xm, a.x, sizeof(T) == 2, a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
     if (e != cudaSuccess) return e;
     if ((e = make_map_4d(&gm, a.y, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.TJ, g.TI)) != cudaSuccess) return e;
-    const int threads = (g.CS / kC2V) * kC2DwGroups;
+    const int threads = ((g.TJ * (g.CS / kC2V) + 31) / 32) * 32;
     // the final reduction [groups][10][CS] float32 reuses the stages
-    const size_t red = static_cast<size_t>(kC2DwGroups) * 10 * g.CS * sizeof(float);
+    const size_t red = static_cast<size_t>(threads / (g.CS / kC2V)) * 10 * g.CS * sizeof(float);
     const size_t stages = 2 * static_cast<size_t>(g.stage_bytes);
     const size_t smem = kC2Head + (red > stages ? red : stages);
-    auto kern = c2_dw_tma_kernel<T>;
+    auto kern = (g.TI % 2 == 0 && a.st == 2) ? c2_dw_tma_kernel<T, 2>
+                : (g.TI % 2 == 0 && a.st == 1) ? c2_dw_tma_kernel<T, 1> : c2_dw_tma_kernel<T, 0>;
     if ((e = ensure_smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(smem))) != cudaSuccess) return e;
     const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ;
     if (ntiles * g.nCS >= (int64_t(1) << 30)) return cudaErrorNotSupported;
