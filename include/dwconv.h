@@ -20,8 +20,9 @@
  *    C above 4,194,304 channels or K above 4096 returns DW_ERR_UNSUPPORTED.
  *    B == 0 or T == 0 is a valid no-op.  Misaligned pointers, or a C that is not a
  *    multiple of the vector width, take a narrower (slower) path and stay correct.
- *  - Arithmetic: bf16 or float32 I/O, float32 accumulation, bf16 stores rounded to
- *    nearest even.  No tensor cores.
+ *  - Arithmetic: bf16, fp16 or float32 I/O, float32 accumulation, 16-bit stores rounded to
+ *    nearest even.  The subsampler's conv0 runs on the tensor cores (float32-accurate split);
+ *    everything else on the FP32 pipes.
  */
 #ifndef DWCONV_B200_H
 #define DWCONV_B200_H
@@ -42,9 +43,17 @@ typedef enum dw_status {
     DW_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel gave up (see dw_device_error) */
 } dw_status_t;
 
+/*
+ * Element type of the activations (x, y, dy, dx, the stream cache).  Weights, biases and
+ * gradients of weights are always float32, and so is the arithmetic.  DW_F16 (IEEE binary16;
+ * "GPU inference for speech", section "Precision": inference usually runs in FP16 or BF16) is
+ * accepted by every conv1d and conv2d entry point; the subsampler entry points take DW_F32 or
+ * DW_BF16.
+ */
 typedef enum dw_dtype {
     DW_F32 = 0,   /* IEEE float32 */
-    DW_BF16 = 1   /* bfloat16 (upper half of a float32) */
+    DW_BF16 = 1,  /* bfloat16 (upper half of a float32) */
+    DW_F16 = 2    /* IEEE float16 */
 } dw_dtype_t;
 
 typedef void *dw_stream_t; /* a cudaStream_t */

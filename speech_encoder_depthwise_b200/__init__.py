@@ -7,7 +7,7 @@ runs in the library's CUDA kernels; there is no other code path.  If the library
 every call raises: build it with ``python -m speech_encoder_depthwise_b200.build``.
 
 Tensors are torch CUDA tensors, contiguous, channels last:
-x, y, dy, dx ``[B, T, C]`` (bfloat16 or float32); w ``[K, C]`` float32; bias ``[C]`` float32;
+x, y, dy, dx ``[B, T, C]`` (bfloat16, float16 or float32); w ``[K, C]`` float32; bias ``[C]`` float32;
 lengths ``[B]`` int32 (or None); mel ``[B, T, F]`` float32; w0, w1 ``[3, 3, C]`` float32.
 """
 from __future__ import annotations
@@ -18,7 +18,7 @@ import threading
 
 __all__ = [
     "DW_OK", "DW_ERR_INVALID_ARG", "DW_ERR_UNSUPPORTED", "DW_ERR_WORKSPACE", "DW_ERR_CUDA",
-    "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DwError", "lib", "library_path",
+    "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DW_F16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
     "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd",
     "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
@@ -26,7 +26,7 @@ __all__ = [
 ]
 
 DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_WORKSPACE, DW_ERR_CUDA, DW_ERR_TIMEOUT = range(6)
-DW_F32, DW_BF16 = 0, 1
+DW_F32, DW_BF16, DW_F16 = 0, 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libdwconv_b200.so")
@@ -106,7 +106,9 @@ def _dtype_code(t):
         return DW_BF16
     if t.dtype == torch.float32:
         return DW_F32
-    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32")
+    if t.dtype == torch.float16:
+        return DW_F16
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16, float16 or float32")
 
 
 def _dev(t, name, dtype=None, shape=None):

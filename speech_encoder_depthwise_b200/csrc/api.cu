@@ -23,9 +23,11 @@ dw_status_t cuda_status(cudaError_t e) {
     return DW_ERR_CUDA;
 }
 
-size_t dtype_size(dw_dtype_t t) { return t == DW_BF16 ? 2 : 4; }
+size_t dtype_size(dw_dtype_t t) { return t == DW_F32 ? 4 : 2; }
 
-bool valid_dtype(dw_dtype_t t) { return t == DW_F32 || t == DW_BF16; }
+bool valid_dtype(dw_dtype_t t) { return t == DW_F32 || t == DW_BF16 || t == DW_F16; }
+// The subsampler kernels take float32 or bf16 activations (no fp16 instance).
+bool valid_sub_dtype(dw_dtype_t t) { return t == DW_F32 || t == DW_BF16; }
 
 // n = a*b*c without overflow of int64 (all >= 0)
 bool mul3(int64_t a, int64_t b, int64_t c, int64_t *n) {
@@ -101,7 +103,7 @@ dwk::Conv2dArgs conv2d_args(int64_t B, int64_t T, int64_t F, int64_t C, int64_t 
     a.x = nullptr; a.w = nullptr; a.bias = nullptr; a.y = nullptr; a.lengths = nullptr; a.out_lengths = nullptr;
     a.B = B; a.T = T; a.F = F; a.C = C; a.To = To; a.Fo = Fo;
     a.KT = KT; a.KF = KF; a.st = st; a.sf = sf; a.pt = pt; a.pb = pb; a.pf = pf;
-    a.bf16 = dt == DW_BF16;
+    a.dtype = static_cast<int>(dt);
     a.vec_width = 1;
     return a;
 }
@@ -140,7 +142,7 @@ dw_status_t dwconv1d_fwd(const void *x, const float *w, const float *bias, void 
     dwk::Conv1dArgs a;
     a.x = x; a.w = w; a.bias = bias; a.y = y; a.lengths = lengths;
     a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left; a.flip = 0;
-    a.bf16 = io_dtype == DW_BF16;
+    a.dtype = static_cast<int>(io_dtype);
     a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, y}, {w, bias});
     return cuda_status(dwk::conv1d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
 }
@@ -155,7 +157,7 @@ dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int3
     a.B = B; a.T = T; a.C = C; a.K = K;
     a.pad_left = K - 1 - pad_left;  // correlation with reversed taps: the pads swap
     a.flip = 1;
-    a.bf16 = io_dtype == DW_BF16;
+    a.dtype = static_cast<int>(io_dtype);
     a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {dy, dx}, {w});
     return cuda_status(dwk::conv1d_fwd_launch(a, static_cast<cudaStream_t>(stream)));
 }
@@ -185,7 +187,7 @@ dw_status_t dwconv1d_bwd(const void *x, const void *dy, const float *w, void *dx
     dwk::DwArgs a;
     a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = lengths;
     a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left;
-    a.bf16 = io_dtype == DW_BF16;
+    a.dtype = static_cast<int>(io_dtype);
     a.partials = static_cast<float *>(workspace);
     a.G = dwk::conv1d_dw_partial_rows(B, T, C, K);
     a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, dy, dx}, {w});
@@ -216,10 +218,10 @@ dw_status_t dwconv1d_stream_fwd(const void *x, const float *w, const float *bias
     dwk::StreamArgs a;
     a.x = x; a.w = w; a.bias = bias; a.y = y; a.cache = cache; a.lengths = lengths;
     a.B = B; a.T = T; a.C = C; a.K = K;
-    a.bf16 = io_dtype == DW_BF16;
+    a.dtype = static_cast<int>(io_dtype);
     a.vec_width = pick_vec_width(C, es, {x, y, cache}, {w, bias});
     // bf16 rows of 8 channels move as one 16-byte word when everything lines up
-    if (a.bf16 && a.vec_width == 4 && C % 8 == 0 && aligned(x, 16) && aligned(y, 16) && aligned(cache, 16))
+    if (a.dtype != 0 && a.vec_width == 4 && C % 8 == 0 && aligned(x, 16) && aligned(y, 16) && aligned(cache, 16))
         a.vec_width = 8;
     return cuda_status(dwk::conv1d_stream_launch(a, static_cast<cudaStream_t>(stream)));
 }
@@ -243,7 +245,7 @@ dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
     dwk::DwArgs a;
     a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = lengths;
     a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left;
-    a.bf16 = io_dtype == DW_BF16;
+    a.dtype = static_cast<int>(io_dtype);
     a.partials = static_cast<float *>(workspace);
     a.G = 0;
     a.vec_width = 1;
@@ -272,7 +274,7 @@ dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0,
                              const void *dout, const int32_t *lengths, float *dw0, float *db0, float *dw1,
                              float *db1, int64_t B, int64_t T, int64_t F, int64_t C, int causal,
                              dw_dtype_t dout_dtype, void *workspace, size_t workspace_bytes, dw_stream_t stream) {
-    if (!valid_dtype(dout_dtype)) return DW_ERR_INVALID_ARG;
+    if (!valid_sub_dtype(dout_dtype)) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
     if (C > kMaxChannels) return DW_ERR_UNSUPPORTED;
     int64_t n = 0;
@@ -382,7 +384,7 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
                              const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
                              int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,
                              dw_stream_t stream) {
-    if (!valid_dtype(out_dtype)) return DW_ERR_INVALID_ARG;
+    if (!valid_sub_dtype(out_dtype)) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
     int64_t n = 0;
     if (!mul3(B, T, F, &n)) return DW_ERR_INVALID_ARG;

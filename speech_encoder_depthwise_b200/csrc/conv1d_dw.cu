@@ -599,8 +599,8 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     cfg.attrs = at2;
     cfg.numAttrs = 2;
     CUtensorMap xmap, dmap;
-    cudaError_t me = make_act_map(&xmap, a.x, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::XROWS);
-    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::DROWS);
+    cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::XROWS);
+    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::DROWS);
     if (me != cudaSuccess) return me;
     return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, a.lengths, a.partials, static_cast<int>(a.B),
                               static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias,
@@ -723,7 +723,7 @@ cudaError_t launch_finalize(const DwArgs &a, int gp, cudaStream_t s) {
 cudaError_t conv1d_bwd_fused_launch(const DwArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaErrorNotSupported;  // nothing to fuse
     int gp = 0;
-    const cudaError_t e = a.bf16 ? launch_fused_partials<bf16>(a, &gp, s) : launch_fused_partials<float>(a, &gp, s);
+    const cudaError_t e = with_dtype(a.dtype, [&](auto tag) { return launch_fused_partials<decltype(tag)>(a, &gp, s); });
     if (e != cudaSuccess) return e;
     return launch_finalize(a, gp, s);
 }
@@ -742,7 +742,7 @@ cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
         return cudaGetLastError();
     }
     int gp = 0;
-    cudaError_t e = a.bf16 ? launch_dtype<bf16>(a, &gp, s) : launch_dtype<float>(a, &gp, s);
+    cudaError_t e = with_dtype(a.dtype, [&](auto tag) { return launch_dtype<decltype(tag)>(a, &gp, s); });
     if (e != cudaSuccess) return e;
     return launch_finalize(a, gp, s);
 }

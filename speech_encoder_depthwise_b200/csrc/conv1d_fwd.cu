@@ -434,7 +434,7 @@ cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     const int64_t ntiles = a.B * static_cast<int64_t>(nT) * nC;
     if (ntiles > kMaxGrid) return cudaErrorInvalidConfiguration;
     CUtensorMap xmap;
-    const cudaError_t me = make_act_map(&xmap, a.x, sizeof(T) == 2, a.B, a.T, a.C, S::CT, S::ROWS);
+    const cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::ROWS);
     if (me != cudaSuccess) return me;
     int64_t grid = static_cast<int64_t>(sm_count()) * kTmaBlocks;
     if (grid > ntiles) grid = ntiles;
@@ -525,8 +525,7 @@ unsigned int conv1d_fwd_take_error() {
 
 cudaError_t conv1d_fwd_launch(const Conv1dArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
-    if (a.bf16) return dispatch_dtype<bf16>(a, s);
-    return dispatch_dtype<float>(a, s);
+    return with_dtype(a.dtype, [&](auto tag) { return dispatch_dtype<decltype(tag)>(a, s); });
 }
 
 }  // namespace dwk

@@ -216,19 +216,23 @@ cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s) {
     int v = a.vec_width;
     const int64_t segs = a.T <= 8 ? 1 : (a.T + 7) / 8;
     while (v > 2 && a.B * (a.C / v) * segs < (int64_t(1) << 16)) v /= 2;
-    if (a.bf16) {
-        switch (v) {
-            case 8: return launch_stream<bf16, 8>(a, s);
-            case 4: return launch_stream<bf16, 4>(a, s);
-            case 2: return launch_stream<bf16, 2>(a, s);
-            default: return launch_stream<bf16, 1>(a, s);
+    return with_dtype(a.dtype, [&](auto tag) {
+        using T = decltype(tag);
+        if constexpr (sizeof(T) == 2) {
+            switch (v) {
+                case 8: return launch_stream<T, 8>(a, s);
+                case 4: return launch_stream<T, 4>(a, s);
+                case 2: return launch_stream<T, 2>(a, s);
+                default: return launch_stream<T, 1>(a, s);
+            }
+        } else {
+            switch (v) {
+                case 4: return launch_stream<T, 4>(a, s);
+                case 2: return launch_stream<T, 2>(a, s);
+                default: return launch_stream<T, 1>(a, s);
+            }
         }
-    }
-    switch (v) {
-        case 4: return launch_stream<float, 4>(a, s);
-        case 2: return launch_stream<float, 2>(a, s);
-        default: return launch_stream<float, 1>(a, s);
-    }
+    });
 }
 
 }  // namespace dwk

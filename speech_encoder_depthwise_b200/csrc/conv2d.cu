@@ -323,14 +323,14 @@ cudaError_t conv2d_fwd_launch(const Conv2dArgs &a, cudaStream_t s) {
     }
     const cudaError_t e = conv2d_fwd_tma_launch(a, s);
     if (e != cudaErrorNotSupported) return e;
-    return a.bf16 ? dispatch_vec<bf16>(a, s, false) : dispatch_vec<float>(a, s, false);
+    return with_dtype(a.dtype, [&](auto tag) { return dispatch_vec<decltype(tag)>(a, s, false); });
 }
 
 cudaError_t conv2d_dx_launch(const Conv2dArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
     const cudaError_t e = conv2d_dx_tma_launch(a, s);
     if (e != cudaErrorNotSupported) return e;
-    return a.bf16 ? dispatch_vec<bf16>(a, s, true) : dispatch_vec<float>(a, s, true);
+    return with_dtype(a.dtype, [&](auto tag) { return dispatch_vec<decltype(tag)>(a, s, true); });
 }
 
 int conv2d_dw_partial_rows(int64_t B, int64_t To) {
@@ -375,13 +375,12 @@ cudaError_t conv2d_dw_launch(const Conv2dArgs &a, float *dw, float *dbias, float
         static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), a.KT, a.KF, a.st, a.sf, a.pt, a.pb, \
         a.pf, static_cast<int>(a.To), static_cast<int>(a.Fo), static_cast<int>(nCG), tap0, wb)
         const bool v2 = a.vec_width >= 2;
-        if (a.bf16) {
-            if (v2) DW_C2_DW(bf16, true);
-            else DW_C2_DW(bf16, false);
-        } else {
-            if (v2) DW_C2_DW(float, true);
-            else DW_C2_DW(float, false);
-        }
+        with_dtype(a.dtype, [&](auto tag) {
+            using TT = decltype(tag);
+            if (v2) DW_C2_DW(TT, true);
+            else DW_C2_DW(TT, false);
+            return 0;
+        });
 #undef DW_C2_DW
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

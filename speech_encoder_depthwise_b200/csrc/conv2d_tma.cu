@@ -49,8 +49,8 @@ template <typename T>
 __device__ __forceinline__ void lds_vec(const T *p, float2 (&f)[2]) {
     if constexpr (sizeof(T) == 2) {
         const uint2 r = *reinterpret_cast<const uint2 *>(p);
-        f[0] = make_float2(bf16_lo(r.x), bf16_hi(r.x));
-        f[1] = make_float2(bf16_lo(r.y), bf16_hi(r.y));
+        f[0] = Half16<T>::unpack(r.x);
+        f[1] = Half16<T>::unpack(r.y);
     } else {
         const float4 r = *reinterpret_cast<const float4 *>(p);
         f[0] = make_float2(r.x, r.y);
@@ -656,11 +656,11 @@ c2_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
 }
 
 // ------------------------------------------------------------------------------ host side
-cudaError_t make_map_4d(CUtensorMap *map, const void *base, bool bf16, int64_t B, int64_t T, int64_t F, int64_t C,
+cudaError_t make_map_4d(CUtensorMap *map, const void *base, int dtype, int64_t B, int64_t T, int64_t F, int64_t C,
                         int box_c, int box_f, int box_t) {
     TensorMapEncodeTiledFn enc = tensor_map_encoder();
     if (enc == nullptr) return cudaErrorNotSupported;
-    const cuuint64_t es = bf16 ? 2 : 4;
+    const cuuint64_t es = static_cast<cuuint64_t>(dtype_bytes(dtype));
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(T),
                                 static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * es, static_cast<cuuint64_t>(F * C) * es,
@@ -668,7 +668,7 @@ cudaError_t make_map_4d(CUtensorMap *map, const void *base, bool bf16, int64_t B
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_c), static_cast<cuuint32_t>(box_f),
                                static_cast<cuuint32_t>(box_t), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+    const CUresult r = enc(map, tma_dtype(dtype), 4,
                            const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -680,7 +680,7 @@ bool aligned8(const void *p) { return p == nullptr || reinterpret_cast<uintptr_t
 
 // 3x3 window; channels-last rows 16-byte aligned; every count of the tensor map in range.
 bool c2_eligible(const Conv2dArgs &a, const void *act0, const void *act1) {
-    const int es = a.bf16 ? 2 : 4;
+    const int es = dtype_bytes(a.dtype);
     if (a.KT != 3 || a.KF != 3) return false;
     if ((a.C * es) % 16 != 0 || !aligned16(act0) || !aligned16(act1)) return false;
     if (!aligned8(a.w) || !aligned8(a.bias)) return false;
@@ -728,7 +728,7 @@ cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
     g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
     g.stage_bytes = g.tx_bytes = g.BR * pix;
     CUtensorMap map;
-    cudaError_t e = make_map_4d(&map, a.x, sizeof(T) == 2, a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
+    cudaError_t e = make_map_4d(&map, a.x, dtype_code<T>(), a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
     if (e != cudaSuccess) return e;
     const int threads = ((g.TJ * (g.CS / kC2V) + 31) / 32) * 32;
     const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes);
@@ -775,7 +775,7 @@ cudaError_t dx2_tma(const Conv2dArgs &a, cudaStream_t s) {
     g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
     g.stage_bytes = g.tx_bytes = g.BR * pix;
     CUtensorMap map;
-    cudaError_t e = make_map_4d(&map, a.x, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.BF, g.BR);
+    cudaError_t e = make_map_4d(&map, a.x, dtype_code<T>(), a.B, a.To, a.Fo, a.C, g.CS, g.BF, g.BR);
     if (e != cudaSuccess) return e;
     const int threads = ((g.TJ / 2 * csv + 31) / 32) * 32;
     const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes);
@@ -822,7 +822,7 @@ cudaError_t dx_tma(const Conv2dArgs &a, cudaStream_t s) {
     g.nCS = static_cast<int>((a.C + g.CS - 1) / g.CS);
     g.stage_bytes = g.tx_bytes = g.BR * pix;
     CUtensorMap map;
-    cudaError_t e = make_map_4d(&map, a.x, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.BF, g.BR);
+    cudaError_t e = make_map_4d(&map, a.x, dtype_code<T>(), a.B, a.To, a.Fo, a.C, g.CS, g.BF, g.BR);
     if (e != cudaSuccess) return e;
     const int threads = ((g.TJ * csv + 31) / 32) * 32;
     const size_t smem = kC2Head + 2 * static_cast<size_t>(g.stage_bytes) + static_cast<size_t>(g.TI) * 3 * sizeof(int);
@@ -866,9 +866,9 @@ cudaError_t dw_tma(const Conv2dArgs &a, float *partials, int max_rows, int *G_ou
     g.stage_bytes = xbytes + g.TI * g.TJ * g.CS * es;
     g.tx_bytes = g.BR * pix + g.TI * g.TJ * g.CS * es;
     CUtensorMap xm, gm;
-    cudaError_t e = make_map_4d(&xm, a.x, sizeof(T) == 2, a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
+    cudaError_t e = make_map_4d(&xm, a.x, dtype_code<T>(), a.B, a.T, a.F, a.C, g.CS, g.BF, g.BR);
     if (e != cudaSuccess) return e;
-    if ((e = make_map_4d(&gm, a.y, sizeof(T) == 2, a.B, a.To, a.Fo, a.C, g.CS, g.TJ, g.TI)) != cudaSuccess) return e;
+    if ((e = make_map_4d(&gm, a.y, dtype_code<T>(), a.B, a.To, a.Fo, a.C, g.CS, g.TJ, g.TI)) != cudaSuccess) return e;
     const int threads = ((g.TJ * (g.CS / kC2V) + 31) / 32) * 32;
     // the final reduction [groups][10][CS] float32 reuses the stages
     const size_t red = static_cast<size_t>(threads / (g.CS / kC2V)) * 10 * g.CS * sizeof(float);
@@ -894,17 +894,17 @@ cudaError_t dw_tma(const Conv2dArgs &a, float *partials, int max_rows, int *G_ou
 
 cudaError_t conv2d_fwd_tma_launch(const Conv2dArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.To == 0 || a.Fo == 0 || !c2_eligible(a, a.x, a.y)) return cudaErrorNotSupported;
-    return a.bf16 ? fwd_tma<bf16>(a, s) : fwd_tma<float>(a, s);
+    return with_dtype(a.dtype, [&](auto tag) { return fwd_tma<decltype(tag)>(a, s); });
 }
 
 cudaError_t conv2d_dx_tma_launch(const Conv2dArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0 || a.To == 0 || a.Fo == 0 || !c2_eligible(a, a.x, a.y)) return cudaErrorNotSupported;
-    return a.bf16 ? dx_tma<bf16>(a, s) : dx_tma<float>(a, s);
+    return with_dtype(a.dtype, [&](auto tag) { return dx_tma<decltype(tag)>(a, s); });
 }
 
 cudaError_t conv2d_dw_tma_partials(const Conv2dArgs &a, float *partials, int max_rows, int *G, cudaStream_t s) {
     if (a.B == 0 || a.To == 0 || a.Fo == 0 || !c2_eligible(a, a.x, a.y)) return cudaErrorNotSupported;
-    return a.bf16 ? dw_tma<bf16>(a, partials, max_rows, G, s) : dw_tma<float>(a, partials, max_rows, G, s);
+    return with_dtype(a.dtype, [&](auto tag) { return dw_tma<decltype(tag)>(a, partials, max_rows, G, s); });
 }
 
 unsigned int conv2d_tma_take_error() {

@@ -1,14 +1,16 @@
-// Shared device helpers: channel-vector loads/stores of bf16 or float32, bf16 <-> float32
-// conversion, packed float32x2 FMA.  sm_100a only.
+// Shared device helpers: channel-vector loads/stores of bf16, fp16 or float32, 16-bit <->
+// float32 conversion, packed float32x2 FMA.  sm_100a only.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace dwk {
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
@@ -28,50 +30,94 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return _
 #endif
 
 // Raw storage for V consecutive channels of element type T, loaded with one instruction.
-// Words are 32-bit; a bf16 pair sits in one word (low half = lower channel).
+// Words are 32-bit; a 16-bit pair (bf16 or fp16) sits in one word (low half = lower channel).
 template <typename T, int V> struct Vec;
 
-template <> struct Vec<bf16, 8> {
+// The two 16-bit element types: unpacking a pair word to float32 and packing two float32 values
+// (round to nearest even) into one.
+__device__ __forceinline__ float2 f16_pair(uint32_t p) {
+    __half2 h;
+    *reinterpret_cast<uint32_t *>(&h) = p;
+    return __half22float2(h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+template <typename T> struct Half16;
+template <> struct Half16<bf16> {
+    static __device__ __forceinline__ float2 unpack(uint32_t p) { return make_float2(bf16_lo(p), bf16_hi(p)); }
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_bf16x2(lo, hi); }
+    static __device__ __forceinline__ float one(unsigned short r) { return __uint_as_float(static_cast<uint32_t>(r) << 16); }
+    static __device__ __forceinline__ bf16 cvt(float v) { return __float2bfloat16_rn(v); }
+};
+template <> struct Half16<f16> {
+    static __device__ __forceinline__ float2 unpack(uint32_t p) { return f16_pair(p); }
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) { return pack_f16x2(lo, hi); }
+    static __device__ __forceinline__ float one(unsigned short r) { return __half2float(__ushort_as_half(r)); }
+    static __device__ __forceinline__ f16 cvt(float v) { return __float2half_rn(v); }
+};
+
+template <typename T> struct Vec16x8 {
+    using H = Half16<T>;
     uint4 r;
-    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const uint4 *>(p)); }
+    __device__ __forceinline__ void load(const T *p) { r = __ldg(reinterpret_cast<const uint4 *>(p)); }
     __device__ __forceinline__ void zero() { r = make_uint4(0, 0, 0, 0); }
     __device__ __forceinline__ void to_f2(float2 (&f)[4]) const {
-        f[0] = make_float2(bf16_lo(r.x), bf16_hi(r.x)); f[1] = make_float2(bf16_lo(r.y), bf16_hi(r.y));
-        f[2] = make_float2(bf16_lo(r.z), bf16_hi(r.z)); f[3] = make_float2(bf16_lo(r.w), bf16_hi(r.w));
+        f[0] = H::unpack(r.x); f[1] = H::unpack(r.y); f[2] = H::unpack(r.z); f[3] = H::unpack(r.w);
     }
-    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[4]) {
-        uint4 o = make_uint4(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y),
-                             pack_bf16x2(f[2].x, f[2].y), pack_bf16x2(f[3].x, f[3].y));
+    static __device__ __forceinline__ void store(T *p, const float2 (&f)[4]) {
+        uint4 o = make_uint4(H::pack(f[0].x, f[0].y), H::pack(f[1].x, f[1].y), H::pack(f[2].x, f[2].y),
+                             H::pack(f[3].x, f[3].y));
         *reinterpret_cast<uint4 *>(p) = o;
     }
-    static __device__ __forceinline__ void store_zero(bf16 *p) {
-        *reinterpret_cast<uint4 *>(p) = make_uint4(0, 0, 0, 0);
-    }
+    static __device__ __forceinline__ void store_zero(T *p) { *reinterpret_cast<uint4 *>(p) = make_uint4(0, 0, 0, 0); }
 };
 
-template <> struct Vec<bf16, 4> {
+template <typename T> struct Vec16x4 {
+    using H = Half16<T>;
     uint2 r;
-    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const uint2 *>(p)); }
+    __device__ __forceinline__ void load(const T *p) { r = __ldg(reinterpret_cast<const uint2 *>(p)); }
     __device__ __forceinline__ void zero() { r = make_uint2(0, 0); }
-    __device__ __forceinline__ void to_f2(float2 (&f)[2]) const {
-        f[0] = make_float2(bf16_lo(r.x), bf16_hi(r.x)); f[1] = make_float2(bf16_lo(r.y), bf16_hi(r.y));
+    __device__ __forceinline__ void to_f2(float2 (&f)[2]) const { f[0] = H::unpack(r.x); f[1] = H::unpack(r.y); }
+    static __device__ __forceinline__ void store(T *p, const float2 (&f)[2]) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(H::pack(f[0].x, f[0].y), H::pack(f[1].x, f[1].y));
     }
-    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[2]) {
-        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y));
-    }
-    static __device__ __forceinline__ void store_zero(bf16 *p) { *reinterpret_cast<uint2 *>(p) = make_uint2(0, 0); }
+    static __device__ __forceinline__ void store_zero(T *p) { *reinterpret_cast<uint2 *>(p) = make_uint2(0, 0); }
 };
 
-template <> struct Vec<bf16, 2> {
+template <typename T> struct Vec16x2 {
+    using H = Half16<T>;
     uint32_t r;
-    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const unsigned int *>(p)); }
+    __device__ __forceinline__ void load(const T *p) { r = __ldg(reinterpret_cast<const unsigned int *>(p)); }
     __device__ __forceinline__ void zero() { r = 0; }
-    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const { f[0] = make_float2(bf16_lo(r), bf16_hi(r)); }
-    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[1]) {
-        *reinterpret_cast<uint32_t *>(p) = pack_bf16x2(f[0].x, f[0].y);
+    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const { f[0] = H::unpack(r); }
+    static __device__ __forceinline__ void store(T *p, const float2 (&f)[1]) {
+        *reinterpret_cast<uint32_t *>(p) = H::pack(f[0].x, f[0].y);
     }
-    static __device__ __forceinline__ void store_zero(bf16 *p) { *reinterpret_cast<uint32_t *>(p) = 0u; }
+    static __device__ __forceinline__ void store_zero(T *p) { *reinterpret_cast<uint32_t *>(p) = 0u; }
 };
+
+// One channel (any C, any alignment): the value travels as a float2 with .y = 0, so the
+// same pairwise arithmetic serves every width.  The slow, general fallback.
+template <typename T> struct Vec16x1 {
+    using H = Half16<T>;
+    unsigned short r;
+    __device__ __forceinline__ void load(const T *p) { r = __ldg(reinterpret_cast<const unsigned short *>(p)); }
+    __device__ __forceinline__ void zero() { r = 0; }
+    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const { f[0] = make_float2(H::one(r), 0.f); }
+    static __device__ __forceinline__ void store(T *p, const float2 (&f)[1]) { *p = H::cvt(f[0].x); }
+    static __device__ __forceinline__ void store_zero(T *p) { *reinterpret_cast<unsigned short *>(p) = 0; }
+};
+
+template <> struct Vec<bf16, 8> : Vec16x8<bf16> {};
+template <> struct Vec<bf16, 4> : Vec16x4<bf16> {};
+template <> struct Vec<bf16, 2> : Vec16x2<bf16> {};
+template <> struct Vec<bf16, 1> : Vec16x1<bf16> {};
+template <> struct Vec<f16, 8> : Vec16x8<f16> {};
+template <> struct Vec<f16, 4> : Vec16x4<f16> {};
+template <> struct Vec<f16, 2> : Vec16x2<f16> {};
+template <> struct Vec<f16, 1> : Vec16x1<f16> {};
 
 template <> struct Vec<float, 4> {
     float4 r;
@@ -101,19 +147,6 @@ template <> struct Vec<float, 2> {
     }
 };
 
-// One channel (any C, any alignment): the value travels as a float2 with .y = 0, so the
-// same pairwise arithmetic serves every width.  The slow, general fallback.
-template <> struct Vec<bf16, 1> {
-    unsigned short r;
-    __device__ __forceinline__ void load(const bf16 *p) { r = __ldg(reinterpret_cast<const unsigned short *>(p)); }
-    __device__ __forceinline__ void zero() { r = 0; }
-    __device__ __forceinline__ void to_f2(float2 (&f)[1]) const {
-        f[0] = make_float2(__uint_as_float(static_cast<uint32_t>(r) << 16), 0.f);
-    }
-    static __device__ __forceinline__ void store(bf16 *p, const float2 (&f)[1]) { *p = __float2bfloat16_rn(f[0].x); }
-    static __device__ __forceinline__ void store_zero(bf16 *p) { *reinterpret_cast<unsigned short *>(p) = 0; }
-};
-
 template <> struct Vec<float, 1> {
     float r;
     __device__ __forceinline__ void load(const float *p) { r = __ldg(p); }
@@ -125,6 +158,16 @@ template <> struct Vec<float, 1> {
 
 // Number of float2 pairs that carry V channels.
 template <int V> struct Pairs { static constexpr int n = V >= 2 ? V / 2 : 1; };
+
+// Element type of a dtype code (0 float32, 1 bf16, 2 fp16): `f` is called with a value of it.
+template <typename Fn>
+inline auto with_dtype(int dtype, Fn &&fn) -> decltype(fn(float{})) {
+    switch (dtype) {
+        case 1: return fn(bf16{});
+        case 2: return fn(f16{});
+        default: return fn(float{});
+    }
+}
 
 // V consecutive float32 parameters (weights or biases) starting at p, as float2 pairs.
 // V >= 2 needs p 8-byte aligned; V == 1 reads one float.

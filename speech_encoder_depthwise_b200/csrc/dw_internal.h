@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "dw_common.cuh"
 
 namespace dwk {
@@ -23,7 +25,7 @@ struct Conv1dArgs {
     int K;
     int pad_left;         // left pad of THIS correlation (already swapped for the data gradient)
     int flip;             // 1: use w[K-1-k] as tap k
-    int bf16;             // 1: bf16 I/O, 0: float32 I/O
+    int dtype;            // I/O element type: 0 float32, 1 bf16, 2 fp16
     int vec_width;        // 2: even-channel vector path allowed; 1: scalar path
 };
 
@@ -32,7 +34,7 @@ struct DwArgs {
     float *dw, *dbias;
     const int32_t *lengths;
     int64_t B, T, C;
-    int K, pad_left, bf16, vec_width;
+    int K, pad_left, dtype, vec_width;  // dtype: 0 float32, 1 bf16, 2 fp16
     float *partials;      // workspace: [G][K+1][C] float32
     int G;                // partial rows (blocks per channel tile)
     const float *w = nullptr;  // [K][C]: taps of the data gradient (fused backward only)
@@ -47,7 +49,7 @@ struct StreamArgs {
     void *cache;          // [B][K-1][C], read and rewritten
     const int32_t *lengths;
     int64_t B, T, C;
-    int K, bf16, vec_width;  // vec_width: 8 (bf16 only), 4, 2 or 1 channels per thread
+    int K, dtype, vec_width;  // dtype: 0 float32, 1 bf16, 2 fp16; vec_width: 8 (16-bit types only), 4, 2 or 1
 };
 
 struct SubsampleArgs {
@@ -70,7 +72,7 @@ struct Conv2dArgs {
     int32_t *out_lengths;     // [B] or null (forward)
     int64_t B, T, F, C, To, Fo;
     int KT, KF, st, sf, pt, pb, pf;
-    int bf16, vec_width;      // vec_width: 4, 2 or 1 channels per thread
+    int dtype, vec_width;     // dtype: 0 float32, 1 bf16, 2 fp16; vec_width: 4, 2 or 1 channels per thread
 };
 
 // Raise a kernel's dynamic shared memory limit to `bytes`, once per (kernel, device).
@@ -84,9 +86,17 @@ typedef CUresult (*TensorMapEncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, c
                                            CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 TensorMapEncodeTiledFn tensor_map_encoder();
 
+// dtype code of an element type (0 float32, 1 bf16, 2 fp16) and the matching tensor-map type.
+template <typename T> constexpr int dtype_code() { return sizeof(T) == 4 ? 0 : (std::is_same<T, bf16>::value ? 1 : 2); }
+inline CUtensorMapDataType tma_dtype(int dtype) {
+    return dtype == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                      : (dtype == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+}
+inline int dtype_bytes(int dtype) { return dtype == 0 ? 4 : 2; }
+
 // Tensor map over a channels-last [B][T][C] activation (dims innermost first: C, T, B) with
 // a box of box_c channels x box_t frames x 1 item; out-of-range elements read as zero.
-cudaError_t make_act_map(CUtensorMap *map, const void *base, bool bf16, int64_t B, int64_t T, int64_t C,
+cudaError_t make_act_map(CUtensorMap *map, const void *base, int dtype, int64_t B, int64_t T, int64_t C,
                          int box_c, int box_t);
 
 int sm_count();

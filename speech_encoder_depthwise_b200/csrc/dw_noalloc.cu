@@ -52,7 +52,7 @@ bool aligned_to(const void *p, size_t n) { return p == nullptr || reinterpret_ca
 extern "C" dw_status_t dwconv1d_bwd_dw_noalloc(const void *x, const void *dy, float *dw, float *dbias,
                                                const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
                                                int pad_left, dw_dtype_t io_dtype, dw_stream_t stream) {
-    if (io_dtype != DW_F32 && io_dtype != DW_BF16) return DW_ERR_INVALID_ARG;
+    if (io_dtype != DW_F32 && io_dtype != DW_BF16 && io_dtype != DW_F16) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
     if (C > (int64_t(1) << 22) || K > 4096) return DW_ERR_UNSUPPORTED;
     if (dw == nullptr) return DW_ERR_INVALID_ARG;
@@ -65,7 +65,7 @@ extern "C" dw_status_t dwconv1d_bwd_dw_noalloc(const void *x, const void *dy, fl
     dwk::DwArgs a;
     a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = lengths;
     a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left;
-    a.bf16 = io_dtype == DW_BF16;
+    a.dtype = static_cast<int>(io_dtype);
     a.partials = nullptr;
     a.G = 0;
     a.vec_width = 1;
@@ -78,7 +78,7 @@ extern "C" dw_status_t dwconv1d_bwd_dw_noalloc(const void *x, const void *dy, fl
         const int rows = dwk::conv1d_dw_partial_rows(B, T, C, K);
         a.partials = static_cast<float *>(scratch);
         a.G = rows < rows_fit ? rows : rows_fit;
-        const size_t es = a.bf16 ? 2 : 4;
+        const size_t es = io_dtype == DW_F32 ? 4 : 2;
         for (int v : {4, 2}) {
             if (C % v == 0 && aligned_to(x, v * es) && aligned_to(dy, v * es)) {
                 a.vec_width = v;

@@ -49,16 +49,16 @@ TensorMapEncodeTiledFn tensor_map_encoder() {
     return fn;
 }
 
-cudaError_t make_act_map(CUtensorMap *map, const void *base, bool bf16, int64_t B, int64_t T, int64_t C,
+cudaError_t make_act_map(CUtensorMap *map, const void *base, int dtype, int64_t B, int64_t T, int64_t C,
                          int box_c, int box_t) {
     TensorMapEncodeTiledFn enc = tensor_map_encoder();
     if (enc == nullptr) return cudaErrorNotSupported;
-    const int64_t es = bf16 ? 2 : 4;
+    const int64_t es = dtype_bytes(dtype);
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(C * es), static_cast<cuuint64_t>(T * C * es)};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_c), static_cast<cuuint32_t>(box_t), 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
-    const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+    const CUresult r = enc(map, tma_dtype(dtype), 3,
                            const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -15,9 +15,9 @@ Recipe (one ``numpy.random.default_rng(seed)`` per workload):
 * conv2d: draw ``x[B, T, F, C]`` ~ N(0, 1), then ``w[KT, KF, C]`` ~ N(0, 1/(KT KF)),
   ``bias[C]`` ~ N(0, 0.1), then ``lengths``, then (when the caller gives the output
   shape) ``dy`` ~ N(0, 1) of that shape.
-* bf16 workloads round every drawn value (data and weights) to the nearest
-  bf16-representable float32, ties to even, so the stored bf16 tensor and the
-  float32 weights hold exactly the values the oracle reads.
+* bf16 (fp16) workloads round every drawn value (data and weights) to the nearest
+  bf16- (fp16-) representable float32, ties to even, so the stored 16-bit tensor and
+  the float32 weights hold exactly the values the oracle reads.
 
 All arrays are float32 (values) or int32 (lengths), C-contiguous, channels last.
 """
@@ -27,6 +27,7 @@ import numpy as np
 
 __all__ = [
     "bf16_round",
+    "f16_round",
     "bf16_bits",
     "conv1d_inputs",
     "subsample_inputs",
@@ -43,6 +44,24 @@ def bf16_round(a: np.ndarray) -> np.ndarray:
     lsb = (u >> 16) & 1
     r = ((u + 0x7FFF + lsb) & 0xFFFF0000).astype(np.uint32)
     return r.view(np.float32).reshape(a.shape)
+
+
+def f16_round(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest IEEE float16 value (ties to even), as float32."""
+    return np.ascontiguousarray(a, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
+def _round_to(dtype, out, keys):
+    if dtype == "bf16":
+        for k in keys:
+            if k in out:
+                out[k] = bf16_round(out[k])
+    elif dtype == "f16":
+        for k in keys:
+            if k in out:
+                out[k] = f16_round(out[k])
+    elif dtype != "f32":
+        raise ValueError(f"unknown dtype {dtype!r}")
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -78,12 +97,7 @@ def conv1d_inputs(B, T, C, K, *, dtype="bf16", len_range=None, seed=0, with_dy=F
     out = {"x": x, "w": w, "bias": bias, "lengths": lengths}
     if with_dy:
         out["dy"] = _normal(rng, (B, T, C), 1.0)
-    if dtype == "bf16":
-        for k in ("x", "w", "bias", "dy"):
-            if k in out:
-                out[k] = bf16_round(out[k])
-    elif dtype != "f32":
-        raise ValueError(f"unknown dtype {dtype!r}")
+    _round_to(dtype, out, ("x", "w", "bias", "dy"))
     return out
 
 
@@ -114,12 +128,7 @@ def conv2d_inputs(B, T, F, C, KT, KF, *, dtype="bf16", len_range=None, seed=0, d
         out["lengths"] = rng.integers(lo, hi + 1, size=B).astype(np.int32)
     if dy_shape is not None:
         out["dy"] = _normal(rng, tuple(dy_shape), 1.0)
-    if dtype == "bf16":
-        for k in ("x", "w", "bias", "dy"):
-            if k in out:
-                out[k] = bf16_round(out[k])
-    elif dtype != "f32":
-        raise ValueError(f"unknown dtype {dtype!r}")
+    _round_to(dtype, out, ("x", "w", "bias", "dy"))
     return out
 
 

@@ -6,7 +6,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-SENTINEL_BITS = {torch.bfloat16: 0x7FA5, torch.float32: 0x7FC0A5A5}
+SENTINEL_BITS = {torch.bfloat16: 0x7FA5, torch.float16: 0x7DA5, torch.float32: 0x7FC0A5A5}
 SLACK = 64  # elements of guard band on each side (keeps 16-byte alignment)
 
 
@@ -25,7 +25,7 @@ class Guarded:
         self.dtype = dtype
         self.n = n
         self.offset = offset
-        idt = torch.int16 if dtype == torch.bfloat16 else torch.int32
+        idt = torch.int32 if dtype == torch.float32 else torch.int16
         bits = SENTINEL_BITS[dtype]
         if idt == torch.int16 and bits > 0x7FFF:
             bits -= 0x10000
@@ -35,7 +35,7 @@ class Guarded:
 
     def check_slack(self):
         bits = SENTINEL_BITS[self.dtype]
-        idt = torch.int16 if self.dtype == torch.bfloat16 else torch.int32
+        idt = torch.int32 if self.dtype == torch.float32 else torch.int16
         if idt == torch.int16 and bits > 0x7FFF:
             bits -= 0x10000
         head = self.raw[:SLACK + self.offset]
@@ -91,6 +91,41 @@ def assert_bf16_close(got, ref, tol=2e-2):
     unfaithful = err >= ulp + 1e-5
     assert not unfaithful.any(), f"{int(unfaithful.sum())} elements not faithfully rounded to bf16"
     return float(err.max())
+
+
+def f16_ulp(v):
+    """Spacing of IEEE float16 numbers at |v| (11 significant bits; subnormal spacing 2^-24)."""
+    v = np.abs(np.asarray(v, np.float64))
+    _, e = np.frexp(np.maximum(v, 2.0 ** -14))
+    return np.ldexp(1.0, e - 11)
+
+
+def assert_f16_close(got, ref):
+    """fp16 I/O bar (no figure is stated for fp16; this one follows from the arithmetic): float32
+    accumulation and one round-to-nearest-even store give a faithfully rounded result, so
+    |gpu - oracle| < ulp_f16(oracle) + 1e-5 element by element (the 1e-5 covers the float32
+    accumulation error of O(1) terms where cancellation makes the result tiny)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    if got.size == 0:
+        return 0.0
+    err = np.abs(got - ref)
+    bar = f16_ulp(ref) + 1e-5
+    bad = err >= bar
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bar), err.shape)
+        raise AssertionError(f"{int(bad.sum())} elements beyond the fp16 bar; worst at {i}: "
+                             f"gpu {got[i]!r} oracle {ref[i]!r} err {err[i]:.3g} bar {bar[i]:.3g}")
+    return float(err.max())
+
+
+def assert_close(dtype, got, ref):
+    """The I/O bar of `dtype` ("f32", "bf16" or "f16")."""
+    if dtype == "f32":
+        return assert_f32_close(got, ref)
+    if dtype == "f16":
+        return assert_f16_close(got, ref)
+    return assert_bf16_close(got, ref)
 
 
 def assert_f32_close(got, ref, rel=1e-5):

@@ -94,6 +94,14 @@ def test_stream_rejects_invalid_arguments(lib):
     assert call(B=0) == dw.DW_OK
 
 
+def test_fp16_is_accepted_and_unknown_dtypes_are_not(lib):
+    assert fwd(lib, B=0, dt=dw.DW_F16) == dw.DW_OK
+    assert fwd(lib, x=None, dt=dw.DW_F16) == dw.DW_ERR_INVALID_ARG
+    assert fwd(lib, dt=3) == dw.DW_ERR_INVALID_ARG
+    assert lib.dwconv2d_fwd(FAKE_X, FAKE_W, None, FAKE_Y, None, None, 0, 40, 20, 8, 3, 3, 2, 2, 1, 1, 1,
+                            dw.DW_F16, None) == dw.DW_OK
+
+
 def test_empty_inputs_are_noops_without_a_device(lib):
     assert fwd(lib, B=0) == dw.DW_OK
     assert fwd(lib, T=0) == dw.DW_OK
@@ -139,6 +147,7 @@ def test_subsample_rejects_invalid_arguments(lib):
     assert call(B=-2) == dw.DW_ERR_INVALID_ARG
     assert call(causal=2) == dw.DW_ERR_INVALID_ARG
     assert call(dt=5) == dw.DW_ERR_INVALID_ARG
+    assert call(dt=dw.DW_F16) == dw.DW_ERR_INVALID_ARG     # the subsampler has no fp16 instance
     assert call(out=FAKE_X) == dw.DW_ERR_INVALID_ARG       # output overlaps the mel input
     assert call(B=0) == dw.DW_OK
     assert call(T=0) == dw.DW_OK
