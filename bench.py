@@ -296,6 +296,65 @@ def measure_sub_bwd(dw, dev, hbm, fp32_tflops):
             "alg_bytes": by, "alg_flops": fl}
 
 
+def graph_us(dev, fns, reps=20):
+    """µs per call of fns[i] (rotating), the calls captured once in a CUDA graph and replayed."""
+    import torch
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        for f in fns:
+            f()
+        g = torch.cuda.CUDAGraph()
+        g.capture_begin()
+        for f in fns:
+            f()
+        g.capture_end()
+        for _ in range(3):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(reps):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) / (reps * len(fns)) * 1e3
+
+
+def measure_f16_packed(dw, dev, hbm):
+    """fp16 I/O and packed batches (a NEXT row, outside the step) on the conformer workload,
+    16x1500x512, K=9, lengths U[750,1500]: the forward in bf16 and in fp16 (same bytes), and the
+    same sequences as a padded batch against a packed [N, C] batch (no padding rows), each over 3
+    rotating input sets in a CUDA graph.  Algorithmic bytes: padded = x at valid frames + y in
+    full; packed = x and y over the N valid rows."""
+    import torch
+    from synth import conv1d_inputs
+    B, T, C, K, pl = 16, 1500, 512, 9, 4
+    d = conv1d_inputs(B, T, C, K, dtype="f16", len_range=(750, 1500), seed=1)
+    L = np.clip(d["lengths"], 0, T)
+    w, bias = torch.from_numpy(d["w"]).to(dev), torch.from_numpy(d["bias"]).to(dev)
+    ln = torch.from_numpy(d["lengths"]).to(dev)
+    res = {}
+    by_pad = (int(L.sum()) * C + B * T * C) * 2
+    for name, td in (("padded_bf16", torch.bfloat16), ("padded_f16", torch.float16)):
+        xs = [torch.from_numpy(d["x"]).to(dev, td) for _ in range(3)]
+        ys = [torch.empty_like(xs[0]) for _ in range(3)]
+        us = graph_us(dev, [lambda i=i: dw.dwconv1d_fwd(xs[i], w, bias, ys[i], ln, pl) for i in range(3)])
+        res[name] = {"us": us, "GB_per_s": by_pad / us / 1e3, "hbm_frac_of_measured": by_pad / us / 1e3 / hbm,
+                     "alg_bytes": by_pad}
+        del xs, ys
+    xp = np.concatenate([d["x"][b, :L[b]] for b in range(B)])
+    N = xp.shape[0]
+    offsets = torch.from_numpy(np.concatenate([[0], np.cumsum(L)]).astype(np.int32)).to(dev)
+    by_pk = 2 * N * C * 2
+    xs = [torch.from_numpy(xp).to(dev, torch.bfloat16) for _ in range(3)]
+    ys = [torch.empty_like(xs[0]) for _ in range(3)]
+    us = graph_us(dev, [lambda i=i: dw.dwconv1d_fwd_packed(xs[i], w, bias, ys[i], offsets, pl) for i in range(3)])
+    res["packed_bf16"] = {"us": us, "GB_per_s": by_pk / us / 1e3, "hbm_frac_of_measured": by_pk / us / 1e3 / hbm,
+                          "alg_bytes": by_pk, "rows": N, "padded_rows": B * T}
+    return {"workload": f"conformer dwconv1d forward {B}x{T}x{C}, K={K}, sym, len U[750,1500]: bf16 vs fp16 "
+                        "padded, and the same sequences packed (3 rotating input sets in a CUDA graph)", **res}
+
+
 CONV2D = dict(B=16, T=750, F=20, C=256, KT=3, KF=3, stride=(2, 2), pads=(1, 1, 1), len_range=(375, 750), seed=5)
 
 
@@ -699,6 +758,7 @@ def main():
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
         next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm), "dwconv1d_bwd": measure_bwd(dw, dev, hbm),
                      "dwconv2d": measure_conv2d(dw, dev, hbm),
+                     "f16_and_packed": measure_f16_packed(dw, dev, hbm),
                      "dw_subsample_bwd": measure_sub_bwd(dw, dev, hbm, fp32_tflops)}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:

@@ -102,6 +102,41 @@ dw_status_t dwconv1d_bwd_dx(const void *dy, const float *w, void *dx, const int3
                             dw_dtype_t io_dtype, dw_stream_t stream);
 
 /*
+ * dwconv1d_fwd_packed - dwconv1d_fwd over a packed batch: the B sequences lie back to back in
+ * x [N][C], sequence b on rows offsets[b] .. offsets[b+1]-1, with no padding rows ("GPU
+ * inference for speech", section "Where the time goes": padding short clips to long ones is
+ * wasted compute, fixed by length bucketing and packed sequences).  Each sequence is convolved
+ * on its own, with its own padding:
+ *
+ *   y[n,c] = bias[c] + sum_{k<K} xs[t + k - pad_left, c] * w[k,c]     for row n = offsets[b] + t
+ *   xs[j,c] = x[offsets[b] + j, c] if 0 <= j < offsets[b+1] - offsets[b], else 0
+ *
+ * which equals dwconv1d_fwd on the padded batch with lengths[b] = offsets[b+1] - offsets[b], row
+ * for row.  Work and traffic follow N, not B * max length.
+ *
+ *  x, y     [N][C] io_dtype, device; y must not overlap x.  Rows no sequence covers are left
+ *           unchanged.
+ *  offsets  [B+1] int32, device: 0 = offsets[0] <= offsets[1] <= ... <= offsets[B] <= N.  The
+ *           kernels clamp every offset into [0, N] (memory safety only; other values give
+ *           unspecified rows).
+ *  w, bias, K, pad_left, io_dtype: as dwconv1d_fwd.  B >= 0, N >= 0 (either 0: no-op);
+ *  N or B of 2^30 or more returns DW_ERR_UNSUPPORTED.
+ */
+dw_status_t dwconv1d_fwd_packed(const void *x, const float *w, const float *bias, void *y,
+                                const int32_t *offsets, int64_t B, int64_t N, int64_t C, int K,
+                                int pad_left, dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
+ * dwconv1d_bwd_dx_packed - data gradient of dwconv1d_fwd_packed (dwconv1d_bwd_dx sequence by
+ * sequence): dx[n,c] = sum_{k<K} dys[t + pad_left - k, c] * w[k,c] for row n = offsets[b] + t,
+ * dys = dy of sequence b, zero outside it.  Arguments as dwconv1d_fwd_packed (pad_left is the
+ * forward pass's).
+ */
+dw_status_t dwconv1d_bwd_dx_packed(const void *dy, const float *w, void *dx,
+                                   const int32_t *offsets, int64_t B, int64_t N, int64_t C, int K,
+                                   int pad_left, dw_dtype_t io_dtype, dw_stream_t stream);
+
+/*
  * dwconv1d_stream_fwd - one chunk of a streaming causal depthwise conv1d with a cache of each
  * stream's K-1 most recent input frames (parakeet.cpp PR #102, section "What changes": the
  * streaming encoder keeps its own depthwise conv with a cache).

@@ -301,6 +301,31 @@ def dwconv1d_stream_fwd(x, w, bias, cache, lengths):
     return default().dwconv1d_stream_fwd(x, w, bias, cache, lengths)
 
 
+def dwconv1d_fwd_packed(x, w, bias, offsets, pad_left):
+    """A packed batch ("GPU inference for speech", section "Where the time goes": packed
+    sequences instead of padding): x [N, C] holds the sequences back to back, sequence b on rows
+    offsets[b]:offsets[b+1].  Each one is convolved on its own by ``dwconv1d_fwd`` (one item, its
+    own length, no padding rows).  Rows no sequence covers come back as NaN."""
+    x = np.asarray(x, np.float64)
+    y = np.full(x.shape, np.nan)
+    for b in range(len(offsets) - 1):
+        s0, e = int(offsets[b]), int(offsets[b + 1])
+        if e > s0:
+            y[s0:e] = dwconv1d_fwd(x[None, s0:e], w, bias, None, pad_left)[0]
+    return y
+
+
+def dwconv1d_bwd_dx_packed(dy, w, offsets, pad_left):
+    """Data gradient of ``dwconv1d_fwd_packed``: ``dwconv1d_bwd_dx`` sequence by sequence."""
+    dy = np.asarray(dy, np.float64)
+    dx = np.full(dy.shape, np.nan)
+    for b in range(len(offsets) - 1):
+        s0, e = int(offsets[b]), int(offsets[b + 1])
+        if e > s0:
+            dx[s0:e] = dwconv1d_bwd_dx(dy[None, s0:e], w, None, pad_left)[0]
+    return dx
+
+
 def dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal):
     return default().dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal)
 

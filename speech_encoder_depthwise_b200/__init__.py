@@ -20,7 +20,8 @@ __all__ = [
     "DW_OK", "DW_ERR_INVALID_ARG", "DW_ERR_UNSUPPORTED", "DW_ERR_WORKSPACE", "DW_ERR_CUDA",
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DW_F16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
-    "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd",
+    "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd", "dwconv1d_fwd_packed",
+    "dwconv1d_bwd_dx_packed",
     "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
     "dwconv2d_fwd", "dwconv2d_bwd_dx", "dwconv2d_bwd_dw_workspace_size", "dwconv2d_bwd_dw", "conv2d_out_shape",
 ]
@@ -48,6 +49,8 @@ SIGNATURES = {
     "dwconv1d_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp,
                             ctypes.c_size_t, _vp]),
     "dwconv1d_stream_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp]),
+    "dwconv1d_fwd_packed": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
+    "dwconv1d_bwd_dx_packed": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
     "dw_subsample_bwd_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
@@ -180,6 +183,30 @@ def dwconv1d_stream_fwd(x, w, bias, y, cache, lengths, stream=None):
                                    cache_ptr, _dev(lengths, "lengths", torch.int32, (B,)), B, T, C, K,
                                    _dtype_code(x), _stream(stream))
     _check("dwconv1d_stream_fwd", st)
+
+
+def dwconv1d_fwd_packed(x, w, bias, y, offsets, pad_left, stream=None):
+    """Depthwise conv1d over a packed batch: x, y ``[N, C]``, sequence b on rows
+    ``offsets[b]:offsets[b+1]`` (``offsets`` int32 ``[B+1]`` on the device)."""
+    import torch
+    N, C = x.shape
+    K = w.shape[0]
+    st = lib().dwconv1d_fwd_packed(_dev(x, "x"), _dev(w, "w", torch.float32, (K, C)),
+                                   _dev(bias, "bias", torch.float32, (C,)), _dev(y, "y", x.dtype, (N, C)),
+                                   _dev(offsets, "offsets", torch.int32), offsets.numel() - 1, N, C, K, pad_left,
+                                   _dtype_code(x), _stream(stream))
+    _check("dwconv1d_fwd_packed", st)
+
+
+def dwconv1d_bwd_dx_packed(dy, w, dx, offsets, pad_left, stream=None):
+    """Data gradient of ``dwconv1d_fwd_packed``."""
+    import torch
+    N, C = dy.shape
+    K = w.shape[0]
+    st = lib().dwconv1d_bwd_dx_packed(_dev(dy, "dy"), _dev(w, "w", torch.float32, (K, C)),
+                                      _dev(dx, "dx", dy.dtype, (N, C)), _dev(offsets, "offsets", torch.int32),
+                                      offsets.numel() - 1, N, C, K, pad_left, _dtype_code(dy), _stream(stream))
+    _check("dwconv1d_bwd_dx_packed", st)
 
 
 def dwconv1d_bwd_dx(dy, w, dx, lengths, pad_left, stream=None):

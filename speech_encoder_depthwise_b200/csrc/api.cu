@@ -108,6 +108,21 @@ dwk::Conv2dArgs conv2d_args(int64_t B, int64_t T, int64_t F, int64_t C, int64_t 
     return a;
 }
 
+// Packed sequences: x/y [N][C], item b on rows offsets[b] .. offsets[b+1]-1.
+dw_status_t packed_common(const void *in, const float *w, void *out, const int32_t *offsets, int64_t B, int64_t N,
+                          int64_t C, int K, int pad_left, dw_dtype_t dt, dwk::Conv1dArgs *a) {
+    int64_t n = 0;
+    dw_status_t st = check_conv1d_common(in, w, out, 1, N, C, K, pad_left, dt, &n);
+    if (st != DW_OK) return st;
+    if (B < 0) return DW_ERR_INVALID_ARG;
+    if (N >= (int64_t(1) << 30) || B >= (int64_t(1) << 30)) return DW_ERR_UNSUPPORTED;  // 32-bit row indices
+    if (n > 0 && B > 0 && offsets == nullptr) return DW_ERR_INVALID_ARG;
+    a->B = B; a->T = N; a->C = C; a->K = K;
+    a->dtype = static_cast<int>(dt);
+    a->lengths = nullptr;
+    return DW_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -200,6 +215,30 @@ dw_status_t dwconv1d_bwd(const void *x, const void *dy, const float *w, void *dx
     if (st != DW_OK) return st;
     return dwconv1d_bwd_dw(x, dy, dw, dbias, lengths, B, T, C, K, pad_left, io_dtype, workspace, workspace_bytes,
                            stream);
+}
+
+dw_status_t dwconv1d_fwd_packed(const void *x, const float *w, const float *bias, void *y, const int32_t *offsets,
+                                int64_t B, int64_t N, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
+                                dw_stream_t stream) {
+    dwk::Conv1dArgs a;
+    dw_status_t st = packed_common(x, w, y, offsets, B, N, C, K, pad_left, io_dtype, &a);
+    if (st != DW_OK || B == 0 || N == 0) return st;
+    a.x = x; a.w = w; a.bias = bias; a.y = y; a.pad_left = pad_left; a.flip = 0;
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, y}, {w, bias});
+    return cuda_status(dwk::conv1d_fwd_packed_launch(a, offsets, static_cast<cudaStream_t>(stream)));
+}
+
+dw_status_t dwconv1d_bwd_dx_packed(const void *dy, const float *w, void *dx, const int32_t *offsets, int64_t B,
+                                   int64_t N, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
+                                   dw_stream_t stream) {
+    dwk::Conv1dArgs a;
+    dw_status_t st = packed_common(dy, w, dx, offsets, B, N, C, K, pad_left, io_dtype, &a);
+    if (st != DW_OK || B == 0 || N == 0) return st;
+    a.x = dy; a.w = w; a.bias = nullptr; a.y = dx;
+    a.pad_left = K - 1 - pad_left;  // correlation with reversed taps: the pads swap
+    a.flip = 1;
+    a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {dy, dx}, {w});
+    return cuda_status(dwk::conv1d_fwd_packed_launch(a, offsets, static_cast<cudaStream_t>(stream)));
 }
 
 dw_status_t dwconv1d_stream_fwd(const void *x, const float *w, const float *bias, void *y, void *cache,

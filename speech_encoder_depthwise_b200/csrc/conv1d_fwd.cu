@@ -164,7 +164,12 @@ struct TmaShape {
     static constexpr int SMEM = 128 + kTmaStages * STAGE_BYTES;
 };
 
-template <typename T, int V, int K>
+// PACKED: the items are sequences of a packed batch, x and y [N][C] with item b on rows
+// offsets[b] .. offsets[b+1]-1 (`lengths` then points to offsets[B+1], Tn = N).  Each item has
+// exactly its own frames (no padding rows), so only its frame-runs are dealt, in order, through a
+// prefix table of runs per item that warp 0 builds in shared memory; input rows of the
+// neighbouring items inside a tile are masked like frames past a length.
+template <typename T, int V, int K, bool PACKED = false>
 __global__ void __launch_bounds__(kTmaThreads, kTmaBlocks)
 conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restrict__ w,
                       const float *__restrict__ bias, T *__restrict__ y, const int32_t *__restrict__ lengths,
@@ -181,7 +186,10 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     // registers, and walks that tile's (item, frame-run) positions q0, q0 + qstride, ...
     const int my_ct = static_cast<int>(blockIdx.x % nC);
     const int q0 = static_cast<int>(blockIdx.x / nC), qstride = static_cast<int>(gridDim.x / nC);
-    const int nq = ntiles / nC;  // positions per channel tile
+    int nq = ntiles / nC;  // positions per channel tile
+    // packed items: runs before item b (pv[b]), its first row and its length
+    int *pv = reinterpret_cast<int *>(stages + static_cast<size_t>(kTmaStages) * S::STAGE_BYTES);
+    int *pst = pv + (B + 1), *plen = pst + B;
     launch_dependents();  // the next kernel in the stream may start its own set-up
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTmaStages; ++i) {
@@ -190,24 +198,75 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
         }
         fence_barrier_init();
     }
-    __syncthreads();
     grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
+    if constexpr (PACKED) {
+        if (warp == 0) {  // offsets are clamped into [0, N] and made non-decreasing
+            int run = 0;
+            if (lane == 0) pv[0] = 0;
+            for (int base = 0; base < B; base += 32) {
+                const int bb = base + lane;
+                int nv = 0;
+                if (bb < B) {
+                    int s0 = __ldg(lengths + bb), e = __ldg(lengths + bb + 1);
+                    s0 = s0 < 0 ? 0 : (s0 > Tn ? Tn : s0);
+                    e = e < s0 ? s0 : (e > Tn ? Tn : e);
+                    pst[bb] = s0;
+                    plen[bb] = e - s0;
+                    nv = (e - s0 + S::TT - 1) / S::TT;
+                }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, nv, o);
+                    if (lane >= o) nv += t;
+                }
+                if (bb < B) pv[bb + 1] = run + nv;
+                run += __shfl_sync(0xffffffffu, nv, 31);
+            }
+        }
+    }
+    __syncthreads();
+    if constexpr (PACKED) nq = pv[B];
+    // position q of the channel tile -> item b, first frame t0 (within the item), the item's
+    // length L, its first row r0 in x/y and its frame count TN (T, or L when packed)
+    auto unit_at = [&](int q, int &b, int &t0, int &L, int64_t &r0, int &TN) {
+        if constexpr (PACKED) {
+            b = TileOrder::find(pv, B, q);
+            t0 = (q - pv[b]) * S::TT;
+            L = plen[b];
+            r0 = pst[b];
+            TN = L;
+        } else {
+            b = q / nT;
+            t0 = (q % nT) * S::TT;
+            L = static_cast<int>(clamp_len(lengths, b, Tn));
+            r0 = static_cast<int64_t>(b) * Tn;
+            TN = Tn;
+        }
+    };
     if (warp == 0) {  // producer warp: one elected lane, one tensor copy per tile
         if (lane == 0) prefetch_tmap(&xmap);
         int it = 0;
         for (int q = q0; q < nq; q += qstride, ++it) {
             const int s = it % kTmaStages;
             const uint32_t ph = (it / kTmaStages) & 1;
-            const int b = q / nT, t0 = (q % nT) * S::TT;
-            // the first ring-full of tiles is issued without waiting for the item's length (a
-            // wholly masked one is read needlessly); later tiles skip the read when t0 >= len
-            const int L = (it >= kTmaStages && lane == 0) ? static_cast<int>(clamp_len(lengths, b, Tn)) : Tn;
+            int b, t0, L, TN;
+            int64_t r0 = 0;
+            if (PACKED || (it >= kTmaStages && lane == 0)) {
+                unit_at(q, b, t0, L, r0, TN);
+            } else {
+                // the first ring-full of tiles is issued without waiting for the item's length (a
+                // wholly masked one is read needlessly); later tiles skip the read when t0 >= len
+                b = q / nT;
+                t0 = (q % nT) * S::TT;
+                L = Tn;
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) return;
             if (lane == 0) {
                 if (t0 < L) {  // rows before frame 0 or past T arrive as zeros; rows in [L, T) are masked by the consumers
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                    tma_load_3d(stages + static_cast<size_t>(s) * S::STAGE_BYTES, &xmap, my_ct * S::CT, t0 - pad_left,
-                                b, &full[s]);
+                    // padded: item b of the [B][T][C] map; packed: rows of the [1][N][C] map
+                    tma_load_3d(stages + static_cast<size_t>(s) * S::STAGE_BYTES, &xmap, my_ct * S::CT,
+                                static_cast<int>(PACKED ? r0 : 0) + t0 - pad_left, PACKED ? 0 : b, &full[s]);
                 } else {
                     mbar_arrive(&full[s]);  // a wholly masked tile: nothing to read
                 }
@@ -236,8 +295,9 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
     for (int q = q0; q < nq; q += qstride, ++it) {
         const int s = it % kTmaStages;
         const uint32_t ph = (it / kTmaStages) & 1;
-        const int b = q / nT, t0 = (q % nT) * S::TT;
-        const int L = static_cast<int>(clamp_len(lengths, b, Tn));  // issued before the wait below
+        int b, t0, L, TN;
+        int64_t r0;
+        unit_at(q, b, t0, L, r0, TN);  // before the wait below
         const int tg = t0 + g * R;
         float2 acc[R][NP];
         if (active && tg < L) {
@@ -247,12 +307,12 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
                 for (int p = 0; p < NP; ++p) acc[r][p] = bv[p];
         }
         if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) return;
-        if (active && tg < Tn) {
-            T *yp = y + (static_cast<int64_t>(b) * Tn + tg) * C + cv;
+        if (active && tg < TN) {
+            T *yp = y + (r0 + tg) * C + cv;
             if (tg >= L) {
 #pragma unroll
                 for (int r = 0; r < R; ++r)
-                    if (tg + r < Tn) Vec<T, V>::store_zero(yp + static_cast<int64_t>(r) * C);
+                    if (tg + r < TN) Vec<T, V>::store_zero(yp + static_cast<int64_t>(r) * C);
             } else {
                 const unsigned char *sp = stages + static_cast<size_t>(s) * S::STAGE_BYTES +
                                           (g * R) * S::ROWB + (wc + lane * V) * static_cast<int>(sizeof(T));
@@ -282,7 +342,7 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
                         if (rd >= 0) {
                             if constexpr (CHECK) {
                                 if (tg + rd < L) Vec<T, V>::store(dst, acc[rd]);
-                                else if (tg + rd < Tn) Vec<T, V>::store_zero(dst);
+                                else if (tg + rd < TN) Vec<T, V>::store_zero(dst);
                             } else {
                                 Vec<T, V>::store(dst, acc[rd]);
                             }
@@ -423,6 +483,52 @@ cudaError_t launch_vec_anyk(const Conv1dArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Packed sequences, any K, any C, any alignment: thread = (row n, V channels).  The row's item
+// comes from a binary search over offsets; its inputs outside the item count as zero.  Rows
+// that no item covers are left unchanged.
+template <typename T, int V>
+__global__ void __launch_bounds__(256)
+conv1d_fwd_packed_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
+                         T *__restrict__ y, const int32_t *__restrict__ offsets, int B, int N, int C, int K,
+                         int pad_left, int flip, int nCV) {
+    constexpr int NP = Pairs<V>::n;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(N) * nCV) return;
+    const int n = static_cast<int>(idx / nCV), c = static_cast<int>(idx % nCV) * V;
+    auto off = [&](int b) {
+        const int o = __ldg(offsets + b);
+        return o < 0 ? 0 : (o > N ? N : o);
+    };
+    int lo = 0, hi = B;  // the last item b with off(b) <= n
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (off(mid) <= n) lo = mid;
+        else hi = mid;
+    }
+    const int s0 = off(lo), e = off(lo + 1);
+    if (n < s0 || n >= e) return;
+    const int t = n - s0, L = e - s0;
+    float2 acc[NP];
+    if (bias != nullptr) {
+        load_param<V>(bias + c, acc);
+    } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
+    }
+    for (int k = 0; k < K; ++k) {
+        const int j = t - pad_left + k;
+        if (j < 0 || j >= L) continue;
+        Vec<T, V> v;
+        v.load(x + (static_cast<int64_t>(s0) + j) * C + c);
+        float2 xf[NP], wf[NP];
+        v.to_f2(xf);
+        load_param<V>(w + static_cast<int64_t>(flip ? K - 1 - k : k) * C + c, wf);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) acc[p] = ffma2(xf[p], wf[p], acc[p]);
+    }
+    Vec<T, V>::store(y + static_cast<int64_t>(n) * C + c, acc);
+}
+
 template <typename T, int V, int K>
 cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     using S = TmaShape<T, V, K>;
@@ -455,6 +561,46 @@ cudaError_t launch_tma(const Conv1dArgs &a, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, kern, xmap, a.w, a.bias, static_cast<T *>(a.y), a.lengths, static_cast<int>(a.B),
                               static_cast<int>(a.T), static_cast<int>(a.C), a.pad_left, a.flip, nT, nC,
                               static_cast<int>(ntiles));
+}
+
+// Packed sequences: x and y [N][C], item b on rows offsets[b] .. offsets[b+1]-1.  The tensor
+// map views x as one item of N frames; at most kOrderMaxItems items per launch (the run table
+// lives in shared memory), so larger batches go in slices of consecutive items.
+template <typename T, int V, int K>
+cudaError_t launch_tma_packed(const Conv1dArgs &a, const int32_t *offsets, cudaStream_t s) {
+    using S = TmaShape<T, V, K>;
+    auto kern = conv1d_fwd_tma_kernel<T, V, K, true>;
+    const int smem = S::SMEM + static_cast<int>((3 * kOrderMaxItems + 1) * sizeof(int));
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern), smem);
+    if (attr != cudaSuccess) return attr;
+    const int nC = static_cast<int>((a.C + S::CT - 1) / S::CT);
+    CUtensorMap xmap;
+    const cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), 1, a.T, a.C, S::CT, S::ROWS);
+    if (me != cudaSuccess) return me;
+    // every block deals runs of its channel tile; the grid is a multiple of nC
+    int64_t grid = static_cast<int64_t>(sm_count()) * kTmaBlocks;
+    const int64_t runs_max = (a.T + S::TT - 1) / S::TT + a.B;  // at most one partial run per item
+    if (grid > runs_max * nC) grid = runs_max * nC;
+    grid = grid / nC * nC;
+    if (grid < nC) grid = nC;
+    for (int64_t b0 = 0; b0 < a.B; b0 += kOrderMaxItems) {
+        const int nb = static_cast<int>(a.B - b0 < kOrderMaxItems ? a.B - b0 : kOrderMaxItems);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(kTmaThreads);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cfg.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, xmap, a.w, a.bias, static_cast<T *>(a.y), offsets + b0,
+                                                 nb, static_cast<int>(a.T), static_cast<int>(a.C), a.pad_left, a.flip,
+                                                 0, nC, 0);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 // The pipelined kernel copies whole frame rows in 16-byte units: C * sizeof(T) a multiple of
@@ -514,7 +660,55 @@ cudaError_t dispatch_dtype(const Conv1dArgs &a, cudaStream_t s) {
     return dispatch_k<T, 1>(a, s);
 }
 
+template <typename T>
+cudaError_t dispatch_packed(const Conv1dArgs &a, const int32_t *offsets, cudaStream_t s) {
+    if (tma_ok<T>(a) && a.vec_width >= 2) {
+        if constexpr (sizeof(T) == 2) {
+            if (a.vec_width >= 4) {
+                switch (a.K) {
+                    case 1: return launch_tma_packed<T, 4, 1>(a, offsets, s);
+                    case 2: return launch_tma_packed<T, 4, 2>(a, offsets, s);
+                    case 3: return launch_tma_packed<T, 4, 3>(a, offsets, s);
+                    case 4: return launch_tma_packed<T, 4, 4>(a, offsets, s);
+                    case 5: return launch_tma_packed<T, 4, 5>(a, offsets, s);
+                    case 7: return launch_tma_packed<T, 4, 7>(a, offsets, s);
+                    case 9: return launch_tma_packed<T, 4, 9>(a, offsets, s);
+                    default: break;
+                }
+            }
+        }
+        switch (a.K) {
+            case 1: return launch_tma_packed<T, 2, 1>(a, offsets, s);
+            case 2: return launch_tma_packed<T, 2, 2>(a, offsets, s);
+            case 3: return launch_tma_packed<T, 2, 3>(a, offsets, s);
+            case 4: return launch_tma_packed<T, 2, 4>(a, offsets, s);
+            case 5: return launch_tma_packed<T, 2, 5>(a, offsets, s);
+            case 7: return launch_tma_packed<T, 2, 7>(a, offsets, s);
+            case 9: return launch_tma_packed<T, 2, 9>(a, offsets, s);
+            case 15: return launch_tma_packed<T, 2, 15>(a, offsets, s);
+            default: break;
+        }
+    }
+    const int V = a.vec_width >= 2 ? 2 : 1;
+    const int nCV = static_cast<int>(a.C / V);
+    const int64_t grid = (a.T * nCV + 255) / 256;
+    if (grid > kMaxGrid) return cudaErrorInvalidConfiguration;
+#define DW_PK(VV)                                                                                              \
+    conv1d_fwd_packed_kernel<T, VV><<<static_cast<unsigned>(grid), 256, 0, s>>>(                               \
+        static_cast<const T *>(a.x), a.w, a.bias, static_cast<T *>(a.y), offsets, static_cast<int>(a.B),       \
+        static_cast<int>(a.T), static_cast<int>(a.C), a.K, a.pad_left, a.flip, nCV)
+    if (V == 2) DW_PK(2);
+    else DW_PK(1);
+#undef DW_PK
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t conv1d_fwd_packed_launch(const Conv1dArgs &a, const int32_t *offsets, cudaStream_t s) {
+    if (a.B == 0 || a.T == 0) return cudaSuccess;
+    return with_dtype(a.dtype, [&](auto tag) { return dispatch_packed<decltype(tag)>(a, offsets, s); });
+}
 
 unsigned int conv1d_fwd_take_error() {
     unsigned int v = 0, zero = 0;

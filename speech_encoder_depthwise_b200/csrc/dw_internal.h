@@ -102,6 +102,8 @@ cudaError_t make_act_map(CUtensorMap *map, const void *base, int dtype, int64_t 
 int sm_count();
 
 cudaError_t conv1d_fwd_launch(const Conv1dArgs &a, cudaStream_t s);
+// Packed sequences: a.B items, a.T = N rows of x/y [N][C], item b on rows offsets[b] .. offsets[b+1]-1.
+cudaError_t conv1d_fwd_packed_launch(const Conv1dArgs &a, const int32_t *offsets, cudaStream_t s);
 // Reads and clears the device error word of the conv1d forward kernels (synchronous).
 unsigned int conv1d_fwd_take_error();
 

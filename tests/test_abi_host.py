@@ -102,6 +102,31 @@ def test_fp16_is_accepted_and_unknown_dtypes_are_not(lib):
                             dw.DW_F16, None) == dw.DW_OK
 
 
+def test_packed_rejects_invalid_arguments(lib):
+    f = lib.dwconv1d_fwd_packed
+    OFF = 0x60000000
+    ok = [FAKE_X, FAKE_W, None, FAKE_Y, OFF, 4, 100, 64, 9, 4, dw.DW_BF16, None]
+    names = ["x", "w", "bias", "y", "off", "B", "N", "C", "K", "pl", "dt", "s"]
+
+    def call(fn=f, **kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return fn(*a)
+    assert call(off=None) == dw.DW_ERR_INVALID_ARG
+    assert call(x=None) == dw.DW_ERR_INVALID_ARG
+    assert call(y=FAKE_X + 16) == dw.DW_ERR_INVALID_ARG      # y overlaps x
+    assert call(B=-1) == dw.DW_ERR_INVALID_ARG
+    assert call(pl=9) == dw.DW_ERR_INVALID_ARG
+    assert call(dt=7) == dw.DW_ERR_INVALID_ARG
+    assert call(N=1 << 30, y=1 << 44) == dw.DW_ERR_UNSUPPORTED
+    assert call(B=0, off=None) == dw.DW_OK
+    assert call(N=0, x=None, y=None) == dw.DW_OK
+    g = lib.dwconv1d_bwd_dx_packed
+    assert g(FAKE_X, FAKE_W, FAKE_Y, None, 4, 100, 64, 9, 4, dw.DW_BF16, None) == dw.DW_ERR_INVALID_ARG
+    assert g(FAKE_X, FAKE_W, FAKE_X, OFF, 4, 100, 64, 9, 4, dw.DW_BF16, None) == dw.DW_ERR_INVALID_ARG
+
+
 def test_empty_inputs_are_noops_without_a_device(lib):
     assert fwd(lib, B=0) == dw.DW_OK
     assert fwd(lib, T=0) == dw.DW_OK
