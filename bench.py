@@ -649,16 +649,39 @@ def main():
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = elapsed_ms / steps
 
-    # per-kernel durations: the same launches, eagerly, each bracketed by events (untimed above)
+    # per-kernel durations (untimed above): each row's launches for the N_SETS input sets
+    # captured in one CUDA graph and replayed back to back, as in the step; the eager figure
+    # (each launch bracketed by events, launch gaps included) is kept beside it
+    del graphs
+
+    def row_graph_ms(j, reps=50):
+        with torch.cuda.stream(stream):
+            g = torch.cuda.CUDAGraph()
+            g.capture_begin()
+            for i in range(N_SETS):
+                name, fn, a = calls[i][j]
+                fn(*a)
+            g.capture_end()
+            for _ in range(3):
+                g.replay()
+            e0, e1 = mk(), mk()
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del g
+        return e0.elapsed_time(e1) / (reps * N_SETS)
+
+    row_ms = {r: row_graph_ms(j) for j, r in enumerate(rows)}
     row_steps = min(steps, 200)
     step_evs = [[(mk(), mk()) for _ in rows] for _ in range(row_steps)]
     with torch.cuda.stream(stream):
         for i in range(row_steps):
             run_step(i, step_evs[i])
     torch.cuda.synchronize(dev)
-    row_ms = {r: float(np.mean([step_evs[i][j][0].elapsed_time(step_evs[i][j][1]) for i in range(row_steps)]))
-              for j, r in enumerate(rows)}
-    del graphs
+    row_eager_ms = {r: float(np.mean([step_evs[i][j][0].elapsed_time(step_evs[i][j][1]) for i in range(row_steps)]))
+                    for j, r in enumerate(rows)}
 
     cw, valid = conv_work(cs["lengths"], T, C, K)
     sb, sf, _, _ = sub_work(ss["lengths"], ST, SF, SC)
@@ -731,13 +754,14 @@ def main():
         for name, (by, fl) in cw.items():
             key = {"fwd": "dwconv1d_fwd", "dx": "dwconv1d_bwd_dx", "dw": "dwconv1d_bwd_dw"}[name]
             ms = row_ms[key]
-            row[key] = {"us": ms * 1e3, "GB_per_s": by / (ms * 1e-3) / 1e9,
+            row[key] = {"us": ms * 1e3, "eager_us": row_eager_ms[key] * 1e3, "GB_per_s": by / (ms * 1e-3) / 1e9,
                         "frames_per_s": B * T / (ms * 1e-3),
                         "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / hbm,
                         "hbm_frac_of_8TBps": by / (ms * 1e-3) / 1e9 / 8000.0,
                         "alg_bytes": by, "alg_flops": fl}
         ms = row_ms["dw_subsample_fwd"]
-        row["dw_subsample_fwd"] = {"ms": ms, "us": ms * 1e3, "TFLOP_per_s": sf / (ms * 1e-3) / 1e12,
+        row["dw_subsample_fwd"] = {"ms": ms, "us": ms * 1e3, "eager_us": row_eager_ms["dw_subsample_fwd"] * 1e3,
+                                   "TFLOP_per_s": sf / (ms * 1e-3) / 1e12,
                                    "fp32_frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
                                    "GB_per_s": sb / (ms * 1e-3) / 1e9,
                                    "frames_per_s": SB * T4 / (ms * 1e-3),
