@@ -90,9 +90,13 @@ __device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt
         for (int p = 0; p < 3; ++p)
 #pragma unroll
             for (int q = 0; q < 3; ++q) mv[3 * p + q] = m0[p * kSbMC + q];
-        float2 z = bias0;
+        // three independent chains (one per tap row), then two adds: a short dependency chain
+        float2 zr[3] = {bias0, make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int t = 0; t < 9; ++t) z = ffma2(mv[t], W0[t], z);
+        for (int q = 0; q < 3; ++q)
+#pragma unroll
+            for (int p = 0; p < 3; ++p) zr[p] = ffma2(mv[3 * p + q], W0[3 * p + q], zr[p]);
+        const float2 z = make_float2(zr[0].x + (zr[1].x + zr[2].x), zr[0].y + (zr[1].y + zr[2].y));
         const float2 h = make_float2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f));
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -135,8 +139,11 @@ __device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt
     }
 }
 
+#ifndef DW_SB_MINB
+#define DW_SB_MINB 4
+#endif
 template <typename TD, bool VEC>
-__global__ void __launch_bounds__(kSbThreads)
+__global__ void __launch_bounds__(kSbThreads, DW_SB_MINB)
 dw_subsample_bwd_kernel(const float *__restrict__ mel, const float *__restrict__ w0, const float *__restrict__ b0,
                         const float *__restrict__ w1, const TD *__restrict__ dout,
                         const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int F,
