@@ -128,6 +128,20 @@ c2_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restr
     };
     if (tid == 0) issue_next();
 
+    // the grid is a multiple of nCS, so the block's channel slab, and its taps, never change
+    float2 wr[9][2], bv[2];
+    {
+        const int c = (static_cast<int>(blockIdx.x) % g.nCS) * g.CS + cv * kC2V;
+        if (active && c < g.C) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
+            if (bias != nullptr) {
+                load_param<kC2V>(bias + c, bv);
+            } else {
+                bv[0] = bv[1] = make_float2(0.f, 0.f);
+            }
+        }
+    }
     int n = 0;  // valid tiles consumed
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         int b, it, jt, cs;
@@ -151,14 +165,6 @@ c2_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restr
             return;
         }
         if (col_ok) {
-            float2 wr[9][2], bv[2];
-#pragma unroll
-            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
-            if (bias != nullptr) {
-                load_param<kC2V>(bias + c, bv);
-            } else {
-                bv[0] = bv[1] = make_float2(0.f, 0.f);
-            }
             // this thread's column of the box; 32-bit element offsets inside the stage
             const T *tb = reinterpret_cast<const T *>(sm.stage[s]) + (jl * g.sf * g.CS + cv * kC2V);
             const int RS = g.BF * g.CS;  // box row stride
@@ -275,6 +281,15 @@ c2_dx_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restri
     };
     if (tid == 0) issue_next();
 
+    // the grid is a multiple of nCS, so the block's channel slab, and its taps, never change
+    float2 wr[9][2];
+    {
+        const int c = (static_cast<int>(blockIdx.x) % g.nCS) * g.CS + cv * kC2V;
+        if (active && c < g.C) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
+        }
+    }
     int n = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         int b, it, jt, cs;
@@ -314,9 +329,6 @@ c2_dx_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restri
             return;
         }
         if (col_ok) {
-            float2 wr[9][2];
-#pragma unroll
-            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
             const T *tileb = reinterpret_cast<const T *>(sm.stage[s]) + cv * kC2V;
             for (int tl = 0; tl < g.TI; ++tl) {
                 const int t = t0 + tl;
@@ -400,6 +412,15 @@ c2_dx2_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restr
     };
     if (tid == 0) issue_next();
 
+    // the grid is a multiple of nCS, so the block's channel slab, and its taps, never change
+    float2 wr[9][2];
+    {
+        const int c = (static_cast<int>(blockIdx.x) % g.nCS) * g.CS + cv * kC2V;
+        if (active && c < g.C) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
+        }
+    }
     int n = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         int b, it, jt, cs;
@@ -435,9 +456,6 @@ c2_dx2_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restr
             return;
         }
         if (col_ok) {
-            float2 wr[9][2];
-#pragma unroll
-            for (int k = 0; k < 9; ++k) load_param<kC2V>(w + static_cast<int64_t>(k) * g.C + c, wr[k]);
             const T *tb = reinterpret_cast<const T *>(sm.stage[s]) + (m * g.CS + cv * kC2V);
             const int RS = g.BF * g.CS;
             float2 d[2][2][2];  // [lo/hi row][lo/hi column][pair]
@@ -739,7 +757,10 @@ cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
     const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
     if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;  // tile indices stay far from int overflow
     const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem);
-    const int grid = static_cast<int>(ntiles < cap ? ntiles : cap);
+    int64_t gridl = ntiles < cap ? ntiles : cap;
+    gridl = gridl / g.nCS * g.nCS;  // whole channel slabs per block (its taps stay in registers)
+    if (gridl < g.nCS) gridl = g.nCS;
+    const int grid = static_cast<int>(gridl);
     kern<<<grid, threads, smem, s>>>(map, a.w, a.bias, static_cast<T *>(a.y), a.lengths, a.out_lengths, g);
     return cudaGetLastError();
 }
@@ -786,7 +807,10 @@ cudaError_t dx2_tma(const Conv2dArgs &a, cudaStream_t s) {
     const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
     if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;
     const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem);
-    const int grid = static_cast<int>(ntiles < cap ? ntiles : cap);
+    int64_t gridl = ntiles < cap ? ntiles : cap;
+    gridl = gridl / g.nCS * g.nCS;  // whole channel slabs per block (its taps stay in registers)
+    if (gridl < g.nCS) gridl = g.nCS;
+    const int grid = static_cast<int>(gridl);
     kern<<<grid, threads, smem, s>>>(map, a.w, static_cast<T *>(a.y), a.lengths, g);
     return cudaGetLastError();
 }
@@ -831,7 +855,10 @@ cudaError_t dx_tma(const Conv2dArgs &a, cudaStream_t s) {
     const int64_t ntiles = static_cast<int64_t>(g.B) * g.nI * g.nJ * g.nCS;
     if (ntiles >= (int64_t(1) << 30)) return cudaErrorNotSupported;  // tile indices stay far from int overflow
     const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(reinterpret_cast<const void *>(kern), threads, smem);
-    const int grid = static_cast<int>(ntiles < cap ? ntiles : cap);
+    int64_t gridl = ntiles < cap ? ntiles : cap;
+    gridl = gridl / g.nCS * g.nCS;  // whole channel slabs per block (its taps stay in registers)
+    if (gridl < g.nCS) gridl = g.nCS;
+    const int grid = static_cast<int>(gridl);
     kern<<<grid, threads, smem, s>>>(map, a.w, static_cast<T *>(a.y), a.lengths, g);
     return cudaGetLastError();
 }
