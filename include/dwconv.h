@@ -47,8 +47,7 @@ typedef enum dw_status {
  * Element type of the activations (x, y, dy, dx, the stream cache).  Weights, biases and
  * gradients of weights are always float32, and so is the arithmetic.  DW_F16 (IEEE binary16;
  * "GPU inference for speech", section "Precision": inference usually runs in FP16 or BF16) is
- * accepted by every conv1d and conv2d entry point; the subsampler entry points take DW_F32 or
- * DW_BF16.
+ * accepted wherever an io_dtype, out_dtype or dout_dtype is taken.
  */
 typedef enum dw_dtype {
     DW_F32 = 0,   /* IEEE float32 */
@@ -249,7 +248,7 @@ dw_status_t dwconv1d_bwd_dw_noalloc(const void *x, const void *dy, float *dw, fl
  *               T2 = ceil(T/2), T4 = ceil(T2/2), F2 = ceil(F/2), F4 = ceil(F2/2)
  *  lengths      [B] int32, device, or NULL
  *  out_lengths  [B] int32, device, or NULL; receives ceil(ceil(len_b/2)/2)
- *  B >= 0, T >= 0, F >= 1, C >= 1; causal 0 or 1; out_dtype DW_BF16 or DW_F32
+ *  B >= 0, T >= 0, F >= 1, C >= 1; causal 0 or 1; out_dtype DW_BF16, DW_F16 or DW_F32
  */
 dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
                              const float *w1, const float *b1, void *out,
@@ -277,7 +276,7 @@ size_t dw_subsample_bwd_workspace_size(int64_t B, int64_t T, int64_t F, int64_t 
  * given GPU model).  No atomics.
  *
  *  mel, w0, b0, w1, lengths, B, T, F, C, causal: as dw_subsample_fwd (b1 is not needed)
- *  dout         [B][T4][F4][C] dout_dtype (DW_BF16 or DW_F32), device
+ *  dout         [B][T4][F4][C] dout_dtype (DW_BF16, DW_F16 or DW_F32), device
  *  dw0, dw1     [3][3][C] float32, device, overwritten;  db0, db1 [C] float32, overwritten
  *  workspace    device buffer of at least dw_subsample_bwd_workspace_size(B,T,F,C) bytes,
  *               16-byte aligned; contents on entry are ignored

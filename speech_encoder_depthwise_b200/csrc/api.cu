@@ -26,8 +26,6 @@ dw_status_t cuda_status(cudaError_t e) {
 size_t dtype_size(dw_dtype_t t) { return t == DW_F32 ? 4 : 2; }
 
 bool valid_dtype(dw_dtype_t t) { return t == DW_F32 || t == DW_BF16 || t == DW_F16; }
-// The subsampler kernels take float32 or bf16 activations (no fp16 instance).
-bool valid_sub_dtype(dw_dtype_t t) { return t == DW_F32 || t == DW_BF16; }
 
 // n = a*b*c without overflow of int64 (all >= 0)
 bool mul3(int64_t a, int64_t b, int64_t c, int64_t *n) {
@@ -313,7 +311,7 @@ dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0,
                              const void *dout, const int32_t *lengths, float *dw0, float *db0, float *dw1,
                              float *db1, int64_t B, int64_t T, int64_t F, int64_t C, int causal,
                              dw_dtype_t dout_dtype, void *workspace, size_t workspace_bytes, dw_stream_t stream) {
-    if (!valid_sub_dtype(dout_dtype)) return DW_ERR_INVALID_ARG;
+    if (!valid_dtype(dout_dtype)) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
     if (C > kMaxChannels) return DW_ERR_UNSUPPORTED;
     int64_t n = 0;
@@ -327,7 +325,7 @@ dw_status_t dw_subsample_bwd(const float *mel, const float *w0, const float *b0,
     a.mel = mel; a.w0 = w0; a.b0 = b0; a.w1 = w1; a.dout = dout; a.lengths = lengths;
     a.dw0 = dw0; a.db0 = db0; a.dw1 = dw1; a.db1 = db1;
     a.partials = static_cast<float *>(workspace);
-    a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.bf16_dout = dout_dtype == DW_BF16;
+    a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.dout_dtype = static_cast<int>(dout_dtype);
     if (nout > 0) {
         if (!mel || !w0 || !b0 || !w1 || !dout) return DW_ERR_INVALID_ARG;
         const size_t need = dwk::subsample_bwd_workspace_bytes(B, T, F, C);
@@ -423,7 +421,7 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
                              const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
                              int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,
                              dw_stream_t stream) {
-    if (!valid_sub_dtype(out_dtype)) return DW_ERR_INVALID_ARG;
+    if (!valid_dtype(out_dtype)) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
     int64_t n = 0;
     if (!mul3(B, T, F, &n)) return DW_ERR_INVALID_ARG;
@@ -442,7 +440,7 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
         dwk::SubsampleArgs a;
         a.mel = mel; a.w0 = w0; a.b0 = b0; a.w1 = w1; a.b1 = b1; a.out = out;
         a.lengths = lengths; a.out_lengths = out_lengths;
-        a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.bf16_out = out_dtype == DW_BF16;
+        a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.out_dtype = static_cast<int>(out_dtype);
         return cuda_status(dwk::subsample_launch(a, s));
     }
     if (out_lengths != nullptr && B > 0)  // no frames: only the (zero) output lengths

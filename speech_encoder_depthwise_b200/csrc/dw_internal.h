@@ -58,7 +58,7 @@ struct SubsampleArgs {
     const int32_t *lengths;
     int32_t *out_lengths;
     int64_t B, T, F, C;
-    int causal, bf16_out;
+    int causal, out_dtype;  // out_dtype: 0 float32, 1 bf16, 2 fp16
 };
 
 // General depthwise conv2d, channels-last [B][T][F][C], taps [KT][KF][C].  The data gradient
@@ -138,7 +138,7 @@ struct SubsampleBwdArgs {
     float *dw0, *db0, *dw1, *db1;  // [3][3][C], [C], [3][3][C], [C]
     float *partials;              // workspace: [rows][20][C]
     int64_t B, T, F, C;
-    int causal, bf16_dout;
+    int causal, dout_dtype;  // 0 float32, 1 bf16, 2 fp16
 };
 int subsample_bwd_partial_rows(int64_t B, int64_t T, int64_t F);
 size_t subsample_bwd_workspace_bytes(int64_t B, int64_t T, int64_t F, int64_t C);

@@ -85,6 +85,15 @@ __device__ __forceinline__ void store_pair<bf16, false>(bf16 *p, float2 v, bool 
     if (has_y) p[1] = __float2bfloat16_rn(v.y);
 }
 template <>
+__device__ __forceinline__ void store_pair<f16, true>(f16 *p, float2 v, bool) {
+    *reinterpret_cast<uint32_t *>(p) = pack_f16x2(v.x, v.y);
+}
+template <>
+__device__ __forceinline__ void store_pair<f16, false>(f16 *p, float2 v, bool has_y) {
+    p[0] = __float2half_rn(v.x);
+    if (has_y) p[1] = __float2half_rn(v.y);
+}
+template <>
 __device__ __forceinline__ void store_pair<float, true>(float *p, float2 v, bool) {
     *reinterpret_cast<float2 *>(p) = v;
 }
@@ -103,7 +112,8 @@ __device__ __forceinline__ void store_pairs(TO *p, const float2 (&v)[NPR], int n
         if constexpr (NPR == 1) {
             store_pair<TO, true>(p, v[0], true);
         } else if constexpr (sizeof(TO) == 2) {
-            *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y));
+            *reinterpret_cast<uint2 *>(p) =
+                make_uint2(Half16<TO>::pack(v[0].x, v[0].y), Half16<TO>::pack(v[1].x, v[1].y));
         } else {
             *reinterpret_cast<float4 *>(p) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
         }
@@ -356,16 +366,19 @@ cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s) {
     // vector stores of 2*kSubNPR channels need C a multiple of that and an aligned output
     const int vch = 2 * kSubNPR;
     const bool vec = (a.C % vch) == 0 &&
-                     (reinterpret_cast<uintptr_t>(a.out) % (static_cast<uintptr_t>(vch) * (a.bf16_out ? 2 : 4))) == 0;
+                     (reinterpret_cast<uintptr_t>(a.out) % (static_cast<uintptr_t>(vch) * dtype_bytes(a.out_dtype))) == 0;
 #define DW_SUB_LAUNCH(TO, VS)                                                                           \
     dw_subsample_kernel<TO, VS, kSubJ, kSubRI, kSubNPR><<<static_cast<unsigned>(grid), warps * 32, 0, s>>>(          \
         a.mel, a.w0, a.b0, a.w1, a.b1, static_cast<TO *>(a.out), a.lengths, a.out_lengths,                   \
         static_cast<int>(a.B), static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C),           \
         static_cast<int>(T2), static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt,          \
         static_cast<int>(nCG), static_cast<int>(nJB), static_cast<int>(nRC))
-    if (a.bf16_out) {
+    if (a.out_dtype == 1) {
         if (vec) DW_SUB_LAUNCH(bf16, true);
         else DW_SUB_LAUNCH(bf16, false);
+    } else if (a.out_dtype == 2) {
+        if (vec) DW_SUB_LAUNCH(f16, true);
+        else DW_SUB_LAUNCH(f16, false);
     } else {
         if (vec) DW_SUB_LAUNCH(float, true);
         else DW_SUB_LAUNCH(float, false);

@@ -34,26 +34,32 @@ constexpr int kSbMaxRows = 592;                      // partial rows per channel
 constexpr int kSbNRW = kSbRT / 2 + 2;                // output rows a tile's h rows read
 constexpr int kSbNCW = kSbST / 2 + 3;                // output columns a tile's h columns read
 
-// A thread's staged dout value: a bf16 pair as one word, or a float pair.
-template <typename TD> struct DWord { using type = float2; };
-template <> struct DWord<bf16> { using type = uint32_t; };
-__device__ __forceinline__ float2 to_pair(float2 v) { return v; }
-__device__ __forceinline__ float2 to_pair(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
-__device__ __forceinline__ void from_pair(float2 v, float2 &w) { w = v; }
-__device__ __forceinline__ void from_pair(float2 v, uint32_t &w) { w = pack_bf16x2(v.x, v.y); }
+// A thread's staged dout value: a 16-bit pair as one word (the values are exact in it), or a
+// float pair.
+template <typename TD> struct DWord {
+    using type = float2;
+    static __device__ __forceinline__ float2 get(float2 v) { return v; }
+    static __device__ __forceinline__ void put(float2 v, float2 &w) { w = v; }
+};
+template <typename TD> struct DWord16 {
+    using type = uint32_t;
+    static __device__ __forceinline__ float2 get(uint32_t u) { return Half16<TD>::unpack(u); }
+    static __device__ __forceinline__ void put(float2 v, uint32_t &w) { w = Half16<TD>::pack(v.x, v.y); }
+};
+template <> struct DWord<bf16> : DWord16<bf16> {};
+template <> struct DWord<f16> : DWord16<f16> {};
 
 template <typename TD, bool VEC>
 __device__ __forceinline__ float2 load_dout(const TD *p, bool two) {
     if constexpr (VEC) {
         if constexpr (sizeof(TD) == 2) {
-            const uint32_t u = __ldg(reinterpret_cast<const unsigned int *>(p));
-            return make_float2(bf16_lo(u), bf16_hi(u));
+            return Half16<TD>::unpack(__ldg(reinterpret_cast<const unsigned int *>(p)));
         } else {
             return __ldg(reinterpret_cast<const float2 *>(p));
         }
     } else {
         auto f = [](const TD *q) -> float {
-            if constexpr (sizeof(TD) == 2) return __bfloat162float(*q);
+            if constexpr (sizeof(TD) == 2) return static_cast<float>(*q);
             else return __ldg(q);
         };
         return make_float2(f(p), two ? f(p + 1) : 0.f);
@@ -68,7 +74,7 @@ __device__ __forceinline__ float2 relu_mask(float2 z, float2 v) {  // [z > 0] v,
 // (tap q = 0), 2k (q = 1) and 2k+1 (q = 2), so each dout value is loaded once and the next
 // column's values are loaded one step ahead.  EVEN: r + Pt even, so output rows iA = (r+Pt)/2
 // (tap p = 0) and iB = iA - 1 (p = 2) feed the row; otherwise only iA = (r+Pt-1)/2 (p = 1).
-template <typename W, bool EVEN>
+template <typename TD, bool EVEN, typename W = typename DWord<TD>::type>
 __device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt, const W *win, int iLo, int kLo,
                                          const float2 (*sm)[kSbMC], const float2 (&W0)[9], const float2 (&W1)[9],
                                          float2 bias0, float2 (&gw0)[9], float2 (&gw1)[9], float2 &gb0,
@@ -79,8 +85,8 @@ __device__ __forceinline__ void row_pass(int r, int R0, int S0, int send, int Pt
     const W *rowA = win + (iA - iLo) * kSbNCW * kSbThreads, *rowB = win + (iB - iLo) * kSbNCW * kSbThreads;
     const float2 zero = make_float2(0.f, 0.f);
     auto load = [&](int k, float2 &a, float2 &bb) {
-        a = to_pair(rowA[(k - kLo) * kSbThreads]);
-        bb = EVEN ? to_pair(rowB[(k - kLo) * kSbThreads]) : zero;
+        a = DWord<TD>::get(rowA[(k - kLo) * kSbThreads]);
+        bb = EVEN ? DWord<TD>::get(rowB[(k - kLo) * kSbThreads]) : zero;
     };
     // one h pixel (r, s) given its dh taps: recompute z, then every gradient term it owns
     auto pixel = [&](int s, float2 dh, const float2 (&d)[4], const int (&tap)[4], int nt, float2 db1v, bool own_b1) {
@@ -201,15 +207,15 @@ dw_subsample_bwd_kernel(const float *__restrict__ mel, const float *__restrict__
                 const int k = kLo + cc;
                 float2 v = make_float2(0.f, 0.f);
                 if (i >= 0 && i < i4 && k >= 0 && k < F4) v = load_dout<TD, VEC>(db + (static_cast<int64_t>(i) * F4 + k) * C, two);
-                from_pair(v, win[(rr * kSbNCW + cc) * kSbThreads]);
+                DWord<TD>::put(v, win[(rr * kSbNCW + cc) * kSbThreads]);
             }
         }
         for (int r = R0; r < rend; ++r) {
             // h row r receives taps p with r + Pt - p even: rows iA (p = 0 or 1) and, for p = 0,
             // also iB = iA - 1 with p = 2
-            if (((r + Pt) & 1) == 0) row_pass<W, true>(r, R0, S0, send, Pt, win, iLo, kLo, sm, W0, W1, bias0, gw0, gw1,
+            if (((r + Pt) & 1) == 0) row_pass<TD, true>(r, R0, S0, send, Pt, win, iLo, kLo, sm, W0, W1, bias0, gw0, gw1,
                                                         gb0, gb1);
-            else row_pass<W, false>(r, R0, S0, send, Pt, win, iLo, kLo, sm, W0, W1, bias0, gw0, gw1, gb0, gb1);
+            else row_pass<TD, false>(r, R0, S0, send, Pt, win, iLo, kLo, sm, W0, W1, bias0, gw0, gw1, gb0, gb1);
         }
     }
     if (!act) return;
@@ -292,16 +298,16 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
     const int64_t nCG = (a.C + 2 * kSbThreads - 1) / (2 * kSbThreads);
     int G = subsample_bwd_partial_rows(a.B, a.T, a.F);
     // one wave of resident blocks over the device, never more than the workspace holds
-    const size_t dsmem = kSbNRW * kSbNCW * kSbThreads * (a.bf16_dout ? sizeof(uint32_t) : sizeof(float2));
+    const bool half = a.dout_dtype != 0;
+    const size_t dsmem = kSbNRW * kSbNCW * kSbThreads * (half ? sizeof(uint32_t) : sizeof(float2));
     int per_sm = 0;
+    // the 16-bit instances share one occupancy (same registers and shared memory)
+    const void *kern = half ? reinterpret_cast<const void *>(dw_subsample_bwd_kernel<bf16, true>)
+                            : reinterpret_cast<const void *>(dw_subsample_bwd_kernel<float, true>);
     {
-        const cudaError_t ea = ensure_smem_attr(a.bf16_dout ? reinterpret_cast<const void *>(dw_subsample_bwd_kernel<bf16, true>)
-                                                            : reinterpret_cast<const void *>(dw_subsample_bwd_kernel<float, true>),
-                                                static_cast<int>(dsmem));
+        const cudaError_t ea = ensure_smem_attr(kern, static_cast<int>(dsmem));
         if (ea != cudaSuccess) return ea;
     }
-    const void *kern = a.bf16_dout ? reinterpret_cast<const void *>(dw_subsample_bwd_kernel<bf16, true>)
-                                   : reinterpret_cast<const void *>(dw_subsample_bwd_kernel<float, true>);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSbThreads, dsmem) != cudaSuccess || per_sm < 1) {
         (void)cudaGetLastError();
         per_sm = 2;
@@ -310,7 +316,7 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
     if (per_group >= 1 && per_group < G) G = static_cast<int>(per_group);
     const int64_t grid = static_cast<int64_t>(G) * nCG;
     if (grid > kMaxGrid || T4 * F4 * a.C >= (1LL << 31) || a.T * a.F >= (1LL << 31)) return cudaErrorInvalidConfiguration;
-    const size_t es = a.bf16_dout ? 2 : 4;
+    const size_t es = half ? 2 : 4;
     cudaError_t e = cudaSuccess;
     const bool vec = (a.C % 2) == 0 && (reinterpret_cast<uintptr_t>(a.dout) % (2 * es)) == 0;
 #define DW_SB_LAUNCH(TD, VV)                                                                                 \
@@ -324,9 +330,12 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
         static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(T2),          \
         static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt, nRT, nST, static_cast<int>(nCG)); \
     } while (0)
-    if (a.bf16_dout) {
+    if (a.dout_dtype == 1) {
         if (vec) DW_SB_LAUNCH(bf16, true);
         else DW_SB_LAUNCH(bf16, false);
+    } else if (a.dout_dtype == 2) {
+        if (vec) DW_SB_LAUNCH(f16, true);
+        else DW_SB_LAUNCH(f16, false);
     } else {
         if (vec) DW_SB_LAUNCH(float, true);
         else DW_SB_LAUNCH(float, false);

@@ -251,6 +251,7 @@ __device__ __forceinline__ void store_k_row(unsigned char *tile, int row, const 
 template <typename TO> __device__ __forceinline__ void stage_out(TO *p, float v);
 template <> __device__ __forceinline__ void stage_out<float>(float *p, float v) { *p = v; }
 template <> __device__ __forceinline__ void stage_out<bf16>(bf16 *p, float v) { *p = __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ void stage_out<f16>(f16 *p, float v) { *p = __float2half_rn(v); }
 
 // ReLU of two accumulator values as a pair.  The doubled form x + |x| = 2 ReLU(x) runs on the
 // FMA pipe instead of the (half-rate) ALU pipe; its weights are halved, so products are equal.
@@ -704,25 +705,25 @@ unsigned int subsample_tc_take_error() {
 }
 
 // Tensor map over the output [B][T4][F4][C] (dims innermost first), box 128 x kJO x kRO x 1.
-static cudaError_t make_out_map(CUtensorMap *map, void *out, bool bf16_out, int64_t B, int64_t T4, int64_t F4,
+static cudaError_t make_out_map(CUtensorMap *map, void *out, int dtype, int64_t B, int64_t T4, int64_t F4,
                                 int64_t C) {
     TensorMapEncodeTiledFn enc = tensor_map_encoder();
     if (enc == nullptr) return cudaErrorNotSupported;
-    const int64_t es = bf16_out ? 2 : 4;
+    const int64_t es = dtype_bytes(dtype);
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(F4),
                                 static_cast<cuuint64_t>(T4), static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(C * es), static_cast<cuuint64_t>(F4 * C * es),
                                    static_cast<cuuint64_t>(T4 * F4 * C * es)};
     const cuuint32_t box[4] = {128u, static_cast<cuuint32_t>(kJO), static_cast<cuuint32_t>(kRO), 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-    const CUresult r = enc(map, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+    const CUresult r = enc(map, tma_dtype(dtype), 4,
                            out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 bool subsample_tc_eligible(const SubsampleArgs &a) {
-    const int64_t es = a.bf16_out ? 2 : 4;
+    const int64_t es = dtype_bytes(a.out_dtype);
     auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
     const int64_t T4 = s2(s2(a.T)), F4 = s2(s2(a.F));
     const int64_t nIP = (T4 + kRO - 1) / kRO, nJB = (F4 + kJO - 1) / kJO;
@@ -740,7 +741,7 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
     const int64_t nG = (nCT + ctg - 1) / ctg;
     const int64_t units = a.B * nIP * nJB;
     CUtensorMap map;
-    cudaError_t e = make_out_map(&map, a.out, a.bf16_out != 0, a.B, T4, F4, a.C);
+    cudaError_t e = make_out_map(&map, a.out, a.out_dtype, a.B, T4, F4, a.C);
     if (e != cudaSuccess) return cudaErrorNotSupported;  // the caller takes the SIMT kernel
     int64_t grid = (sm_count() / nG) * nG;
     if (grid < nG) grid = nG;
@@ -770,9 +771,12 @@ cudaError_t subsample_tc_launch(const SubsampleArgs &a, cudaStream_t s) {
             static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C), static_cast<int>(F2), Pt,     \
             static_cast<int>(nIP), static_cast<int>(nJB), static_cast<int>(nG));                               \
     } while (0)
-    if (a.bf16_out) {
+    if (a.out_dtype == 1) {
         if (ctg == 2) DW_TC_LAUNCH(bf16, 2);
         else DW_TC_LAUNCH(bf16, 1);
+    } else if (a.out_dtype == 2) {
+        if (ctg == 2) DW_TC_LAUNCH(f16, 2);
+        else DW_TC_LAUNCH(f16, 1);
     } else {
         if (ctg == 2) DW_TC_LAUNCH(float, 2);
         else DW_TC_LAUNCH(float, 1);

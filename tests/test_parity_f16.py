@@ -1,5 +1,5 @@
-"""GPU parity of the fp16 I/O variants (dtype DW_F16) of every conv1d and conv2d entry point
-against the fp64 CPU oracle, element by element, through the C ABI.
+"""GPU parity of the fp16 I/O variants (dtype DW_F16) of every entry point against the fp64
+CPU oracle, element by element, through the C ABI.
 
 fp16 ("GPU inference for speech", section "Precision": 16-bit inference in FP16 or BF16) keeps
 float32 weights and float32 arithmetic; only the activations are 16-bit.  Inputs are drawn as
@@ -10,7 +10,9 @@ masked frames +0.0; weight gradients (float32) <= 2e-2 absolute and <= 1e-5 * RM
 Cases: the conformer shape (16x1500x512, K=9, symmetric) for forward, dX, dW and the one-pass
 backward; a causal K=15 and a runtime K=6; C that takes 2- and 1-channel vectors; misaligned
 buffers (narrow path); the streaming conv over chunks; the conv2d subsampler-stage shape on the
-TMA path and windows/strides of the general kernels; the workspace-free dW.
+TMA path and windows/strides of the general kernels; the workspace-free dW; the subsampler with
+fp16 output (tensor-core kernel and, for an odd C, the SIMT kernel) and its backward with fp16
+dout (bars as for bf16 dout: 1e-5 * RMS plus the oracle's ReLU-kink budget).
 """
 import numpy as np
 import pytest
@@ -19,7 +21,7 @@ import torch
 import oracle
 import speech_encoder_depthwise_b200 as dw
 from gpuhelp import Guarded, assert_f16_close, assert_masked_zero, dev, max_abs, rms
-from synth import conv1d_inputs, conv2d_inputs, f16_round, symmetric_pad_left
+from synth import conv1d_inputs, conv2d_inputs, f16_round, subsample_inputs, symmetric_pad_left
 
 pytestmark = pytest.mark.gpu
 H = torch.float16
@@ -169,3 +171,39 @@ def test_conv2d_general(KT, KF, stride, pads, C):
     d = conv2d_inputs(3, T, F, C, KT, KF, dtype="f16", len_range=(0, T), seed=KT * 7 + C, dy_shape=(3, To, Fo, C))
     d["lengths"][0], d["lengths"][1] = T, 0
     run_conv2d(d, stride, pads)
+
+
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("B,T,F,C", [(16, 3000, 80, 256), (2, 37, 81, 300), (2, 23, 9, 3)])
+def test_subsampler_f16_output(B, T, F, C, causal):
+    d = subsample_inputs(B, T, F, C, len_range=(T // 2, T), seed=T + C)
+    T4, F4 = dw.subsample_out_shape(T, F)
+    out = Guarded((B, T4, F4, C), H)
+    ol = torch.empty(B, dtype=torch.int32, device="cuda")
+    dw.dw_subsample_fwd(dev(d["mel"]), dev(d["w0"]), dev(d["b0"]), dev(d["w1"]), dev(d["b1"]), out.t,
+                        dev(d["lengths"]), ol, causal)
+    torch.cuda.synchronize()
+    out.check_slack()
+    ref, rl = oracle.dw_subsample_fwd(d["mel"], d["w0"], d["b0"], d["w1"], d["b1"], d["lengths"], causal)
+    assert_f16_close(out.numpy(), ref)
+    assert np.array_equal(ol.cpu().numpy(), rl)
+
+
+@pytest.mark.parametrize("B,T,F,C", [(4, 600, 80, 256), (2, 37, 81, 300)])
+def test_subsampler_backward_f16_dout(B, T, F, C):
+    d = subsample_inputs(B, T, F, C, len_range=(T // 2, T), seed=7 + C)
+    T4, F4 = dw.subsample_out_shape(T, F)
+    dout = f16_round(np.random.default_rng(C).standard_normal((B, T4, F4, C)))
+    g = Guarded(dout.shape, H)
+    g.t.copy_(torch.from_numpy(dout).to(H))
+    outs = [Guarded((3, 3, C), torch.float32), Guarded((C,), torch.float32),
+            Guarded((3, 3, C), torch.float32), Guarded((C,), torch.float32)]
+    ws = torch.empty(max(dw.dw_subsample_bwd_workspace_size(B, T, F, C), 16), dtype=torch.uint8, device="cuda")
+    dw.dw_subsample_bwd(dev(d["mel"]), dev(d["w0"]), dev(d["b0"]), dev(d["w1"]), g.t, dev(d["lengths"]),
+                        *[o.t for o in outs], 0, ws)
+    torch.cuda.synchronize()
+    ref = oracle.dw_subsample_bwd(d["mel"], d["w0"], d["b0"], d["w1"], dout, d["lengths"], 0)
+    kdw0, kdb0 = oracle.dw_subsample_bwd_kinks(d["mel"], d["w0"], d["b0"], d["w1"], dout, d["lengths"], 0, 1e-5)
+    for name, o, r, k in zip(("dw0", "db0", "dw1", "db1"), outs, ref, (kdw0, kdb0, 0.0, 0.0)):
+        err = np.abs(o.numpy() - r)
+        assert np.all(err <= 1e-5 * max(rms(r), 1e-6) + k), (name, float(err.max()))
