@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--next-rows", default="all",
+                   help="comma list of the NEXT-row measurements after the step (stream, bwd, conv2d, "
+                        "f16_packed, sub_bwd), 'all' or 'none'")
     return p.parse_args()
 
 
@@ -351,6 +354,12 @@ def measure_f16_packed(dw, dev, hbm):
     us = graph_us(dev, [lambda i=i: dw.dwconv1d_fwd_packed(xs[i], w, bias, ys[i], offsets, pl) for i in range(3)])
     res["packed_bf16"] = {"us": us, "GB_per_s": by_pk / us / 1e3, "hbm_frac_of_measured": by_pk / us / 1e3 / hbm,
                           "alg_bytes": by_pk, "rows": N, "padded_rows": B * T}
+    # the weight gradient of the same packed batch (x and dy over the N rows read once)
+    gw, gb = torch.empty(K, C, device=dev), torch.empty(C, device=dev)
+    ws = torch.empty(dw.dwconv1d_bwd_dw_packed_workspace_size(B, N, C, K), dtype=torch.uint8, device=dev)
+    us = graph_us(dev, [lambda i=i: dw.dwconv1d_bwd_dw_packed(xs[i], ys[i], gw, gb, offsets, pl, ws) for i in range(3)])
+    res["packed_bf16_bwd_dw"] = {"us": us, "GB_per_s": by_pk / us / 1e3, "hbm_frac_of_measured": by_pk / us / 1e3 / hbm,
+                                 "alg_bytes": by_pk}
     return {"workload": f"conformer dwconv1d forward {B}x{T}x{C}, K={K}, sym, len U[750,1500]: bf16 vs fp16 "
                         "padded, and the same sequences packed (3 rotating input sets in a CUDA graph)", **res}
 
@@ -780,10 +789,14 @@ def main():
         ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
-        next_rows = {"dwconv1d_stream_fwd": measure_stream(dw, dev, hbm), "dwconv1d_bwd": measure_bwd(dw, dev, hbm),
-                     "dwconv2d": measure_conv2d(dw, dev, hbm),
-                     "f16_and_packed": measure_f16_packed(dw, dev, hbm),
-                     "dw_subsample_bwd": measure_sub_bwd(dw, dev, hbm, fp32_tflops)}
+        want = {"stream", "bwd", "conv2d", "f16_packed", "sub_bwd"} if args.next_rows == "all" else \
+            set() if args.next_rows == "none" else set(args.next_rows.split(","))
+        measures = [("stream", "dwconv1d_stream_fwd", lambda: measure_stream(dw, dev, hbm)),
+                    ("bwd", "dwconv1d_bwd", lambda: measure_bwd(dw, dev, hbm)),
+                    ("conv2d", "dwconv2d", lambda: measure_conv2d(dw, dev, hbm)),
+                    ("f16_packed", "f16_and_packed", lambda: measure_f16_packed(dw, dev, hbm)),
+                    ("sub_bwd", "dw_subsample_bwd", lambda: measure_sub_bwd(dw, dev, hbm, fp32_tflops))]
+        next_rows = {name: fn() for key, name, fn in measures if key in want}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
             v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)

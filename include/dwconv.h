@@ -136,6 +136,30 @@ dw_status_t dwconv1d_bwd_dx_packed(const void *dy, const float *w, void *dx,
                                    int pad_left, dw_dtype_t io_dtype, dw_stream_t stream);
 
 /*
+ * dwconv1d_bwd_dw_packed_workspace_size - bytes of device workspace dwconv1d_bwd_dw_packed needs
+ * (depends on N, C and K only); 0 for invalid sizes.
+ */
+size_t dwconv1d_bwd_dw_packed_workspace_size(int64_t B, int64_t N, int64_t C, int K);
+
+/*
+ * dwconv1d_bwd_dw_packed - weight and bias gradients of dwconv1d_fwd_packed:
+ *   dW[k,c] = sum over sequences b and their frames t of dy[offsets[b]+t, c] xs_b[t + k - pad_left, c]
+ *   dbias[c] = sum over the rows of every sequence of dy[n, c]
+ * with xs_b = x of sequence b, zero outside it.  float32 partial sums per block go to `workspace`
+ * and a second kernel adds them in a fixed order (bitwise reproducible for given sizes).  No
+ * atomics.  Rows no sequence covers are ignored.
+ *
+ *  x, dy      [N][C] io_dtype, device;  offsets as dwconv1d_fwd_packed
+ *  dw         [K][C] float32, device, overwritten;  dbias [C] float32, or NULL
+ *  workspace  at least dwconv1d_bwd_dw_packed_workspace_size(B, N, C, K) bytes, 16-byte aligned,
+ *             contents on entry ignored.  With B == 0 or N == 0 the gradients are zeros.
+ */
+dw_status_t dwconv1d_bwd_dw_packed(const void *x, const void *dy, float *dw, float *dbias,
+                                   const int32_t *offsets, int64_t B, int64_t N, int64_t C, int K,
+                                   int pad_left, dw_dtype_t io_dtype, void *workspace,
+                                   size_t workspace_bytes, dw_stream_t stream);
+
+/*
  * dwconv1d_stream_fwd - one chunk of a streaming causal depthwise conv1d with a cache of each
  * stream's K-1 most recent input frames (parakeet.cpp PR #102, section "What changes": the
  * streaming encoder keeps its own depthwise conv with a cache).

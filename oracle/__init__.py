@@ -315,6 +315,22 @@ def dwconv1d_fwd_packed(x, w, bias, offsets, pad_left):
     return y
 
 
+def dwconv1d_bwd_dw_packed(x, dy, K, offsets, pad_left):
+    """Weight and bias gradients of ``dwconv1d_fwd_packed``: ``dwconv1d_bwd_dw`` of every sequence,
+    summed.  Returns (dW [K, C], dbias [C])."""
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    C = x.shape[1]
+    gw, gb = np.zeros((K, C)), np.zeros(C)
+    for b in range(len(offsets) - 1):
+        s0, e = int(offsets[b]), int(offsets[b + 1])
+        if e > s0:
+            w_b, b_b = dwconv1d_bwd_dw(x[None, s0:e], dy[None, s0:e], K, None, pad_left)
+            gw += w_b
+            gb += b_b
+    return gw, gb
+
+
 def dwconv1d_bwd_dx_packed(dy, w, offsets, pad_left):
     """Data gradient of ``dwconv1d_fwd_packed``: ``dwconv1d_bwd_dx`` sequence by sequence."""
     dy = np.asarray(dy, np.float64)

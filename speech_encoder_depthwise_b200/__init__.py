@@ -21,7 +21,7 @@ __all__ = [
     "DW_ERR_TIMEOUT", "DW_F32", "DW_BF16", "DW_F16", "DwError", "lib", "library_path",
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
     "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd", "dwconv1d_fwd_packed",
-    "dwconv1d_bwd_dx_packed",
+    "dwconv1d_bwd_dx_packed", "dwconv1d_bwd_dw_packed_workspace_size", "dwconv1d_bwd_dw_packed",
     "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
     "dwconv2d_fwd", "dwconv2d_bwd_dx", "dwconv2d_bwd_dw_workspace_size", "dwconv2d_bwd_dw", "conv2d_out_shape",
 ]
@@ -51,6 +51,9 @@ SIGNATURES = {
     "dwconv1d_stream_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp]),
     "dwconv1d_fwd_packed": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
     "dwconv1d_bwd_dx_packed": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp]),
+    "dwconv1d_bwd_dw_packed_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _int]),
+    "dwconv1d_bwd_dw_packed": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _vp,
+                                      ctypes.c_size_t, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
     "dw_subsample_bwd_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
@@ -207,6 +210,25 @@ def dwconv1d_bwd_dx_packed(dy, w, dx, offsets, pad_left, stream=None):
                                       _dev(dx, "dx", dy.dtype, (N, C)), _dev(offsets, "offsets", torch.int32),
                                       offsets.numel() - 1, N, C, K, pad_left, _dtype_code(dy), _stream(stream))
     _check("dwconv1d_bwd_dx_packed", st)
+
+
+def dwconv1d_bwd_dw_packed_workspace_size(B, N, C, K) -> int:
+    """Bytes of workspace ``dwconv1d_bwd_dw_packed`` needs."""
+    return int(lib().dwconv1d_bwd_dw_packed_workspace_size(B, N, C, K))
+
+
+def dwconv1d_bwd_dw_packed(x, dy, dw_, dbias, offsets, pad_left, workspace, stream=None):
+    """Weight and bias gradients of ``dwconv1d_fwd_packed`` into dw_ [K, C] and dbias [C] (float32)."""
+    import torch
+    N, C = x.shape
+    K = dw_.shape[0]
+    st = lib().dwconv1d_bwd_dw_packed(_dev(x, "x"), _dev(dy, "dy", x.dtype, (N, C)),
+                                      _dev(dw_, "dw", torch.float32, (K, C)), _dev(dbias, "dbias", torch.float32, (C,)),
+                                      _dev(offsets, "offsets", torch.int32), offsets.numel() - 1, N, C, K, pad_left,
+                                      _dtype_code(x), _dev(workspace, "workspace"),
+                                      workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                      _stream(stream))
+    _check("dwconv1d_bwd_dw_packed", st)
 
 
 def dwconv1d_bwd_dx(dy, w, dx, lengths, pad_left, stream=None):

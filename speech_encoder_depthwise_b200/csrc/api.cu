@@ -239,6 +239,45 @@ dw_status_t dwconv1d_bwd_dx_packed(const void *dy, const float *w, void *dx, con
     return cuda_status(dwk::conv1d_fwd_packed_launch(a, offsets, static_cast<cudaStream_t>(stream)));
 }
 
+size_t dwconv1d_bwd_dw_packed_workspace_size(int64_t B, int64_t N, int64_t C, int K) {
+    if (B < 0 || N < 0 || C < 1 || K < 1) return 0;
+    int64_t n = 0;
+    if (!mul3(1, N, C, &n)) return 0;
+    return dwk::conv1d_dw_packed_workspace_bytes(N, C, K);
+}
+
+dw_status_t dwconv1d_bwd_dw_packed(const void *x, const void *dy, float *dw, float *dbias, const int32_t *offsets,
+                                   int64_t B, int64_t N, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
+                                   void *workspace, size_t workspace_bytes, dw_stream_t stream) {
+    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
+    if (B < 0 || N < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
+    if (C > kMaxChannels || K > 4096) return DW_ERR_UNSUPPORTED;
+    if (N >= (int64_t(1) << 30) || B >= (int64_t(1) << 30)) return DW_ERR_UNSUPPORTED;
+    int64_t n = 0;
+    if (!mul3(1, N, C, &n)) return DW_ERR_INVALID_ARG;
+    if (dw == nullptr) return DW_ERR_INVALID_ARG;
+    const size_t out_bytes = static_cast<size_t>(K) * C * sizeof(float), gb = static_cast<size_t>(C) * sizeof(float);
+    if (dbias != nullptr && overlaps(dw, out_bytes, dbias, gb)) return DW_ERR_INVALID_ARG;
+    dwk::DwArgs a;
+    a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = nullptr;
+    a.B = B; a.T = N; a.C = C; a.K = K; a.pad_left = pad_left;
+    a.dtype = static_cast<int>(io_dtype);
+    a.partials = static_cast<float *>(workspace);
+    a.G = 0;
+    a.vec_width = 1;
+    if (B > 0 && N > 0) {
+        if (x == nullptr || dy == nullptr || offsets == nullptr) return DW_ERR_INVALID_ARG;
+        const size_t need = dwk::conv1d_dw_packed_workspace_bytes(N, C, K);
+        if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return DW_ERR_WORKSPACE;
+        if (overlaps(workspace, need, dw, out_bytes) || (dbias && overlaps(workspace, need, dbias, gb)))
+            return DW_ERR_INVALID_ARG;
+        a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, dy}, {});
+    } else {
+        a.B = 0;  // no rows: the gradients are zeros
+    }
+    return cuda_status(dwk::conv1d_dw_packed_launch(a, offsets, static_cast<cudaStream_t>(stream)));
+}
+
 dw_status_t dwconv1d_stream_fwd(const void *x, const float *w, const float *bias, void *y, void *cache,
                                 const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
                                 dw_dtype_t io_dtype, dw_stream_t stream) {

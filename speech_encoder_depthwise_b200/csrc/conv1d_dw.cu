@@ -735,6 +735,194 @@ unsigned int conv1d_dw_take_error() {
     return v;
 }
 
+// ---------------------------------------------------------------------------------------
+// Packed batches: x and dy [N][C], item b on rows offsets[b] .. offsets[b+1]-1, each item with its
+// own padding.  Grid (G, channel tiles of 32 V channels); block g walks rows N g / G .. N (g+1) / G,
+// its 8 warps each a contiguous share, tracking the item of the current row as it goes (offsets
+// clamped into [0, N]).  A thread keeps a window of the kDwPackedTaps x frames t - pad + k_off + k
+// of the current row t (zero outside the item) and slides it one frame per row, so each row costs
+// one dy and one x load: dbias += dz, dW[k_off + k] += dz win[k].  Widths beyond kDwPackedTaps run
+// in passes.  The warps' sums are added in a fixed order in shared memory and each block writes
+// partial row g; the finalize kernel adds the rows in order (reproducible, no atomics).
+constexpr int kDwPackedTaps = 16;
+
+template <typename T, int V>
+__global__ void __launch_bounds__(256)
+conv1d_dw_packed_kernel(const T *__restrict__ x, const T *__restrict__ dy, const int32_t *__restrict__ offsets,
+                        float *__restrict__ partials, int B, int N, int C, int K, int k_off, int kb, int pad_left,
+                        int with_bias, int G) {
+    constexpr int NP = Pairs<V>::n;
+    constexpr int KT = kDwPackedTaps;
+    extern __shared__ float red[];  // [8][KT + 1][32 V]
+    const int lane = threadIdx.x % 32, wp = threadIdx.x / 32;
+    const int CT = 32 * V;
+    const int cl = lane * V, c = blockIdx.y * CT + cl;
+    const bool act = c < C;
+    auto off = [&](int b) {
+        const int o = __ldg(offsets + b);
+        return o < 0 ? 0 : (o > N ? N : o);
+    };
+    const int64_t g = blockIdx.x;
+    const int rb = static_cast<int>(static_cast<int64_t>(N) * g / G), re = static_cast<int>(static_cast<int64_t>(N) * (g + 1) / G);
+    const int n0 = rb + static_cast<int>(static_cast<int64_t>(re - rb) * wp / 8);
+    const int n1 = rb + static_cast<int>(static_cast<int64_t>(re - rb) * (wp + 1) / 8);
+    float2 acc[KT][NP], accb[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        accb[p] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < KT; ++k) acc[k][p] = make_float2(0.f, 0.f);
+    }
+    if (act && n0 < n1) {
+        int lo = 0, hi = B;  // the last item whose first row is <= n0
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (off(mid) <= n0) lo = mid;
+            else hi = mid;
+        }
+        int b = lo, s0 = off(b), e = off(b + 1);
+        if (e < s0) e = s0;
+        auto load_x = [&](int j, int L, float2 (&f)[NP]) {  // frame j of the current item, zero outside
+            if (j >= 0 && j < L) {
+                Vec<T, V> v;
+                v.load(x + (static_cast<int64_t>(s0) + j) * C + c);
+                v.to_f2(f);
+            } else {
+#pragma unroll
+                for (int p = 0; p < NP; ++p) f[p] = make_float2(0.f, 0.f);
+            }
+        };
+        // window: slot (k + r) % KT holds frame j0 + k of row r of the current group of KT rows,
+        // so every slot index is a compile-time constant; the frame that enters for row r + 1
+        // (j0 + KT) takes the slot row r's frame j0 leaves
+        float2 win[KT][NP];
+        bool fresh = true;  // the window must be (re)filled for the current row
+        for (int base = n0; base < n1; base += KT) {
+#pragma unroll
+            for (int r = 0; r < KT; ++r) {
+                const int n = base + r;
+                if (n < n1) {
+                    while (n >= e && b + 1 < B) {  // the next item
+                        ++b;
+                        s0 = off(b);
+                        e = off(b + 1);
+                        if (e < s0) e = s0;
+                        fresh = true;
+                    }
+                    if (n < s0 || n >= e) {  // a row no item covers
+                        fresh = true;
+                    } else {
+                        const int t = n - s0, L = e - s0, j0 = t - pad_left + k_off;
+                        if (fresh) {
+#pragma unroll
+                            for (int k = 0; k < KT; ++k) load_x(j0 + k, L, win[(k + r) % KT]);
+                            fresh = false;
+                        }
+                        Vec<T, V> v;
+                        v.load(dy + static_cast<int64_t>(n) * C + c);
+                        float2 dz[NP];
+                        v.to_f2(dz);
+#pragma unroll
+                        for (int p = 0; p < NP; ++p) {
+                            accb[p].x += dz[p].x;
+                            accb[p].y += dz[p].y;
+                        }
+#pragma unroll
+                        for (int k = 0; k < KT; ++k) {
+                            if (k < kb) {
+#pragma unroll
+                                for (int p = 0; p < NP; ++p)
+                                    acc[k][p] = ffma2(dz[p], win[(k + r) % KT][p], acc[k][p]);
+                            }
+                        }
+                        load_x(j0 + KT, L, win[r % KT]);  // frame j0 + KT for the next row
+                    }
+                }
+            }
+        }
+    }
+    // fixed-order sum over the 8 warps: red[warp][slot][channel of the tile]
+#pragma unroll
+    for (int kk = 0; kk <= KT; ++kk) {
+        float2 v[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) v[p] = kk < KT ? acc[kk][p] : accb[p];
+        float *d = red + (wp * (KT + 1) + kk) * CT + cl;
+        if constexpr (V == 1) {
+            d[0] = v[0].x;
+        } else {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                d[2 * p] = v[p].x;
+                d[2 * p + 1] = v[p].y;
+            }
+        }
+    }
+    __syncthreads();
+    const int E = (KT + 1) * CT;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        const int kk = i / CT, ch = blockIdx.y * CT + i % CT;
+        if (ch >= C) continue;
+        float t = 0.f;
+        {
+            float r[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) r[w] = red[w * E + i];
+            t = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+        }
+        if (kk == KT) {
+            if (with_bias) partials[(g * (K + 1) + K) * C + ch] = t;
+        } else if (kk < kb) {
+            partials[(g * (K + 1) + k_off + kk) * C + ch] = t;
+        }
+    }
+}
+
+constexpr int kDwPackedRows = 256;  // partial rows of the packed weight gradient (at most)
+
+int conv1d_dw_packed_rows(int64_t N) {
+    const int64_t g = (N + 127) / 128;
+    return static_cast<int>(g < 1 ? 1 : (g > kDwPackedRows ? kDwPackedRows : g));
+}
+
+size_t conv1d_dw_packed_workspace_bytes(int64_t N, int64_t C, int K) {
+    return static_cast<size_t>(conv1d_dw_packed_rows(N)) * static_cast<size_t>(K + 1) * static_cast<size_t>(C) *
+           sizeof(float);
+}
+
+cudaError_t conv1d_dw_packed_launch(const DwArgs &a, const int32_t *offsets, cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(a.K + 1) * a.C;
+    if (a.B == 0 || a.T == 0) {
+        conv1d_dw_zero_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(a.dw, a.dbias, a.K, a.C);
+        return cudaGetLastError();
+    }
+    const int G = conv1d_dw_packed_rows(a.T);
+    const int V = a.vec_width >= 2 ? 2 : 1;
+    const int64_t nCT = (a.C + 32 * V - 1) / (32 * V);
+    if (nCT > 65535) return cudaErrorInvalidConfiguration;
+    const size_t red_bytes = static_cast<size_t>(8) * (kDwPackedTaps + 1) * 32 * V * sizeof(float);
+    for (int k_off = 0; k_off < a.K; k_off += kDwPackedTaps) {
+        const int kb = a.K - k_off < kDwPackedTaps ? a.K - k_off : kDwPackedTaps;
+        const cudaError_t e = with_dtype(a.dtype, [&](auto tag) {
+            using T = decltype(tag);
+            const dim3 grid(static_cast<unsigned>(G), static_cast<unsigned>(nCT));
+            if (V == 2)
+                conv1d_dw_packed_kernel<T, 2><<<grid, 256, red_bytes, s>>>(
+                    static_cast<const T *>(a.x), static_cast<const T *>(a.dy), offsets, a.partials, static_cast<int>(a.B),
+                    static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, kb, a.pad_left, k_off == 0 ? 1 : 0, G);
+            else
+                conv1d_dw_packed_kernel<T, 1><<<grid, 256, red_bytes, s>>>(
+                    static_cast<const T *>(a.x), static_cast<const T *>(a.dy), offsets, a.partials, static_cast<int>(a.B),
+                    static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, kb, a.pad_left, k_off == 0 ? 1 : 0, G);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
+    }
+    conv1d_dw_finalize_kernel<<<static_cast<unsigned>((n + 31) / 32), 256, 0, s>>>(a.partials, a.dw, a.dbias, G, a.K,
+                                                                                    a.C);
+    return cudaGetLastError();
+}
+
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
     const int64_t n = static_cast<int64_t>(a.K + 1) * a.C;
     if (a.B == 0 || a.T == 0) {

@@ -111,6 +111,11 @@ unsigned int conv1d_fwd_take_error();
 int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t C, int K);
 size_t conv1d_dw_workspace_bytes(int64_t B, int64_t T, int64_t C, int K);
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s);
+// Packed batches (a.T = N rows, a.B items on rows offsets[b] .. offsets[b+1]-1): partial rows
+// [rows][K+1][C] in a.partials, then the fixed-order finalize.
+int conv1d_dw_packed_rows(int64_t N);
+size_t conv1d_dw_packed_workspace_bytes(int64_t N, int64_t C, int K);
+cudaError_t conv1d_dw_packed_launch(const DwArgs &a, const int32_t *offsets, cudaStream_t s);
 // dx and dW/dbias in one pass over dy; cudaErrorNotSupported when no fused instance fits.
 cudaError_t conv1d_bwd_fused_launch(const DwArgs &a, cudaStream_t s);
 unsigned int conv1d_dw_take_error();

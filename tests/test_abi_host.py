@@ -122,6 +122,17 @@ def test_packed_rejects_invalid_arguments(lib):
     assert call(N=1 << 30, y=1 << 44) == dw.DW_ERR_UNSUPPORTED
     assert call(B=0, off=None) == dw.DW_OK
     assert call(N=0, x=None, y=None) == dw.DW_OK
+    n = lib.dwconv1d_bwd_dw_packed_workspace_size(4, 100, 64, 9)
+    assert n > 0 and n % 16 == 0 and lib.dwconv1d_bwd_dw_packed_workspace_size(4, 100, 0, 9) == 0
+    h = lib.dwconv1d_bwd_dw_packed
+    args = (FAKE_X, FAKE_Y, FAKE_W, None, OFF, 4, 100, 64, 9, 4, dw.DW_BF16)
+    assert h(*args, None, n, None) == dw.DW_ERR_WORKSPACE
+    assert h(*args, FAKE_WS, n - 16, None) == dw.DW_ERR_WORKSPACE
+    assert h(*args, FAKE_W, n, None) == dw.DW_ERR_INVALID_ARG           # workspace overlaps dW
+    assert h(FAKE_X, FAKE_Y, FAKE_W, None, None, 4, 100, 64, 9, 4, dw.DW_BF16, FAKE_WS, n, None) \
+        == dw.DW_ERR_INVALID_ARG                                         # no offsets
+    assert h(FAKE_X, FAKE_Y, None, None, OFF, 4, 100, 64, 9, 4, dw.DW_BF16, FAKE_WS, n, None) \
+        == dw.DW_ERR_INVALID_ARG
     g = lib.dwconv1d_bwd_dx_packed
     assert g(FAKE_X, FAKE_W, FAKE_Y, None, 4, 100, 64, 9, 4, dw.DW_BF16, None) == dw.DW_ERR_INVALID_ARG
     assert g(FAKE_X, FAKE_W, FAKE_X, OFF, 4, 100, 64, 9, 4, dw.DW_BF16, None) == dw.DW_ERR_INVALID_ARG

@@ -1,4 +1,4 @@
-"""Pins of the oracle's packed-batch conv1d (forward and data gradient): sequences back to back
+"""Pins of the oracle's packed-batch conv1d (forward, data and weight gradients): sequences back to back
 in [N, C], each convolved on its own ("GPU inference for speech", section "Where the time goes":
 packed sequences instead of padding).
 
@@ -35,6 +35,16 @@ def torch_seq_dx(dy, w, pad_left):
     return x.grad[0].T.numpy()
 
 
+def torch_seq_dw(x, dy, K, pad_left):
+    L, C = x.shape
+    w = torch.zeros(C, 1, K, dtype=torch.float64, requires_grad=True)
+    b = torch.zeros(C, dtype=torch.float64, requires_grad=True)
+    xt = torch.nn.functional.pad(torch.from_numpy(np.asarray(x, np.float64).T[None]), (pad_left, K - 1 - pad_left))
+    y = torch.nn.functional.conv1d(xt, w, b, groups=C)
+    y.backward(torch.from_numpy(np.asarray(dy, np.float64).T[None]))
+    return w.grad[:, 0, :].T.numpy(), b.grad.numpy()
+
+
 CASES = [(K, mode, seed) for K in (1, 2, 4, 9, 15) for mode in ("sym", "causal") for seed in (0, 1)]
 
 
@@ -63,6 +73,16 @@ def test_packed_matches_torch_per_sequence(K, mode, seed):
         np.testing.assert_allclose(y[s0:e], torch_seq(x[s0:e], w, bias, pl), rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(dx[s0:e], torch_seq_dx(dy[s0:e], w, pl), rtol=1e-12, atol=1e-12)
     assert not np.isnan(y).any() and not np.isnan(dx).any()  # every row belongs to a sequence
+    gw, gb = oracle.dwconv1d_bwd_dw_packed(x, dy, K, offsets, pl)
+    tw, tb = np.zeros((K, C)), np.zeros(C)
+    for b in range(B):
+        s0, e = offsets[b], offsets[b + 1]
+        if e > s0:
+            w_b, b_b = torch_seq_dw(x[s0:e], dy[s0:e], K, pl)
+            tw += w_b
+            tb += b_b
+    np.testing.assert_allclose(gw, tw, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(gb, tb, rtol=1e-11, atol=1e-11)
 
 
 def test_packed_equals_padded_batch_on_valid_frames():

@@ -1,4 +1,5 @@
-"""GPU parity of the packed-batch conv1d (dwconv1d_fwd_packed, dwconv1d_bwd_dx_packed) against
+"""GPU parity of the packed-batch conv1d (dwconv1d_fwd_packed, dwconv1d_bwd_dx_packed,
+dwconv1d_bwd_dw_packed) against
 the fp64 CPU oracle, element by element, through the C ABI.
 
 Workload: the conformer batch (16 sequences, lengths U[750, 1500], C=512, K=9, symmetric)
@@ -6,7 +7,8 @@ packed back to back, in bf16, fp16 and float32.  Edge cases: empty sequences and
 shorter than the window, causal K=15, runtime K=6, C that takes 2- and 1-channel vectors,
 misaligned buffers (general kernel), more sequences than one launch's table holds (1500 short
 ones), and rows after offsets[B] (must stay untouched).  Bars as the padded kernels: bf16
-|err| <= max(2e-2, 1 ulp) and faithful, fp16 faithful, float32 <= 1e-5 * RMS.
+|err| <= max(2e-2, 1 ulp) and faithful, fp16 faithful, float32 <= 1e-5 * RMS; dW/dbias <= 2e-2
+absolute and <= 1e-5 * RMS, bitwise reproducible.
 """
 import numpy as np
 import pytest
@@ -14,7 +16,7 @@ import torch
 
 import oracle
 import speech_encoder_depthwise_b200 as dw
-from gpuhelp import Guarded, assert_close, dev
+from gpuhelp import Guarded, assert_close, dev, max_abs, rms
 from synth import conv1d_inputs, symmetric_pad_left
 
 pytestmark = pytest.mark.gpu
@@ -62,6 +64,24 @@ def run(x, dy, w, bias, offsets, pl, dtype, offset=0):
     gdx = dx.numpy()
     assert_close(dtype, gdx[:covered], oracle.dwconv1d_bwd_dx_packed(dy, w, offsets, pl)[:covered])
     assert np.all(gdx[covered:] == 7.0)
+    K = w.shape[0]
+    gw, gb = gpu_dw_packed(xg.t, gy.t, offsets, K, pl)
+    rw, rb = oracle.dwconv1d_bwd_dw_packed(x[:covered], dy[:covered], K, offsets, pl)
+    for g, r in ((gw, rw), (gb, rb)):
+        e = max_abs(g, r)
+        assert e <= 2e-2 and e <= 1e-5 * max(rms(r), 1e-6), (e, rms(r))
+
+
+def gpu_dw_packed(xt, gyt, offsets, K, pl):
+    N, C = xt.shape
+    gw, gb = Guarded((K, C), torch.float32), Guarded((C,), torch.float32)
+    n = dw.dwconv1d_bwd_dw_packed_workspace_size(len(offsets) - 1, N, C, K)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    dw.dwconv1d_bwd_dw_packed(xt, gyt, gw.t, gb.t, dev(offsets), pl, ws)
+    torch.cuda.synchronize()
+    gw.check_slack()
+    gb.check_slack()
+    return gw.numpy(), gb.numpy()
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
@@ -111,3 +131,13 @@ def test_packed_equals_padded_gpu_on_valid_frames():
     torch.cuda.synchronize()
     for b in range(B):
         assert torch.equal(y[offsets[b]:offsets[b + 1]], yp[b, :lens[b]])
+
+
+def test_packed_weight_gradient_is_reproducible():
+    rng = np.random.default_rng(21)
+    x, dy, w, bias, offsets = packed_case(rng.integers(100, 900, size=12), 512, 9, "bf16", seed=21)
+    xt, gt = dev(x, torch.bfloat16), dev(dy, torch.bfloat16)
+    a = gpu_dw_packed(xt, gt, offsets, 9, 4)
+    b = gpu_dw_packed(xt, gt, offsets, 9, 4)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
