@@ -208,7 +208,11 @@ struct DwTmaShape {
     static constexpr int SMEM = 128 + BODY;  // plus the tile-order tables, sized at launch
 };
 
-template <typename T, int V, int KB, bool FUSED = false>
+// PACKED: items are the sequences of a packed batch (x, dy [N][C], `lengths` = offsets[B+1],
+// Tn = N): only each sequence's own frame-runs are dealt, through a prefix table of runs per item
+// built like the order tables; boxes start at the sequence's first row of the [1][N][C] maps and
+// rows of the neighbouring sequences are masked like frames past a length.
+template <typename T, int V, int KB, bool FUSED = false, bool PACKED = false>
 __global__ void __launch_bounds__(DwTmaShape<T, V, KB, FUSED>::THREADS, FUSED ? 1 : kDwBlocks)
 conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
                      const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C, int K,
@@ -231,7 +235,35 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     int *ord_mem = reinterpret_cast<int *>(stages + S::BODY);
     TileOrder order{ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), B, nT, 1, 0};
     grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
-    if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
+    // packed: pv = runs before item b, pst = its first row, plen = its length
+    int *pv = ord_mem, *pst = ord_mem + (B + 1), *plen = pst + B;
+    if constexpr (PACKED) {
+        if (warp == 0) {  // offsets clamped into [0, N]
+            int run = 0;
+            if (lane == 0) pv[0] = 0;
+            for (int base = 0; base < B; base += 32) {
+                const int bb = base + lane;
+                int nv = 0;
+                if (bb < B) {
+                    int s0 = __ldg(lengths + bb), e = __ldg(lengths + bb + 1);
+                    s0 = s0 < 0 ? 0 : (s0 > Tn ? Tn : s0);
+                    e = e < s0 ? s0 : (e > Tn ? Tn : e);
+                    pst[bb] = s0;
+                    plen[bb] = e - s0;
+                    nv = (e - s0 + S::TT - 1) / S::TT;
+                }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, nv, o);
+                    if (lane >= o) nv += t;
+                }
+                if (bb < B) pv[bb + 1] = run + nv;
+                run += __shfl_sync(0xffffffffu, nv, 31);
+            }
+        }
+    } else {
+        if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDwStages; ++i) {
             mbar_init(&full[i], 1);
@@ -240,11 +272,15 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
         fence_barrier_init();
     }
     __syncthreads();
-    if (ordered) order.V = order.pv[B];
+    if (!PACKED && ordered) order.V = order.pv[B];
     // the fused pass also walks the wholly masked units: their dx frames are written as zeros
-    const int units = (ordered && !FUSED) ? order.V : B * nT;
+    const int units = PACKED ? pv[B] : ((ordered && !FUSED) ? order.V : B * nT);
     auto unit_at = [&](int u, int &b, int &t0, int &L) {
-        if (ordered) {
+        if constexpr (PACKED) {
+            b = TileOrder::find(pv, B, u);
+            t0 = (u - pv[b]) * S::TT;
+            L = plen[b];
+        } else if (ordered) {
             int tt, ctd;
             order.map(u, b, tt, ctd, L);
             t0 = tt * S::TT;
@@ -276,7 +312,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
             if (!ok) break;
             if (lane == 0) {
                 int b, t0, L;
-                if (ordered || it >= kDwStages) {
+                if (PACKED || ordered || it >= kDwStages) {
                     unit_at(u, b, t0, L);
                 } else {  // the first ring-full is issued before any length is read
                     b = u / nT;
@@ -285,9 +321,11 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
                 }
                 if (t0 < L) {  // frames before 0 or past T arrive as zeros; [L, T) is masked by the consumers
                     unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
+                    // padded: item b of the [B][T][C] maps; packed: rows of the [1][N][C] maps
+                    const int r0 = PACKED ? pst[b] : 0, bi = PACKED ? 0 : b;
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                    tma_load_3d(st, &xmap, c0, t0 + k_off - pad_left, b, &full[s]);
-                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, FUSED ? t0 - padR : t0, b, &full[s]);
+                    tma_load_3d(st, &xmap, c0, r0 + t0 + k_off - pad_left, bi, &full[s]);
+                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, r0 + (FUSED ? t0 - padR : t0), bi, &full[s]);
                 } else {
                     mbar_arrive(&full[s]);  // a wholly masked unit: nothing to read
                 }
@@ -540,18 +578,20 @@ cudaError_t launch_pass(const DwArgs &a, int gp, int k_off, int with_bias, cudaS
 
 // Grid rows G and cluster size for the pipelined kernel: as many blocks per channel tile as
 // fit on the device at once, in clusters as large as that allows (fewer partial rows).
-template <typename T, int V, int KB, bool FUSED = false>
-cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s) {
+template <typename T, int V, int KB, bool FUSED = false, bool PACKED = false>
+cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s,
+                            const int32_t *offsets = nullptr) {
     using S = DwTmaShape<T, V, KB, FUSED>;
-    auto kern = conv1d_dw_tma_kernel<T, V, KB, FUSED>;
-    const int ordered = (DW_DW_ORDERED && a.B <= kOrderMaxItems) ? 1 : 0;
+    auto kern = conv1d_dw_tma_kernel<T, V, KB, FUSED, PACKED>;
+    const int ordered = PACKED ? 1 : ((DW_DW_ORDERED && a.B <= kOrderMaxItems) ? 1 : 0);
     const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
     const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
                                               S::SMEM + static_cast<int>(3 * (kOrderMaxItems + 1) * sizeof(int)) + 16);
     if (attr != cudaSuccess) return attr;
     const int nCT = static_cast<int>((a.C + S::CT - 1) / S::CT);
     const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
-    const int64_t units = a.B * nT;
+    // packed: the runs of all sequences, at most one partial run per sequence beyond N / TT
+    const int64_t units = PACKED ? nT + a.B : a.B * nT;
     if (nCT > 65535 || units >= (1LL << 31)) return cudaErrorInvalidConfiguration;
     int best_g = 0, best_c = 1;
     for (int c : {8, 4, 2, 1}) {
@@ -599,10 +639,11 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     cfg.attrs = at2;
     cfg.numAttrs = 2;
     CUtensorMap xmap, dmap;
-    cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::XROWS);
-    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::DROWS);
+    const int64_t mB = PACKED ? 1 : a.B;
+    cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), mB, a.T, a.C, S::CT, S::XROWS);
+    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, dtype_code<T>(), mB, a.T, a.C, S::CT, S::DROWS);
     if (me != cudaSuccess) return me;
-    return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, a.lengths, a.partials, static_cast<int>(a.B),
+    return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, PACKED ? offsets : a.lengths, a.partials, static_cast<int>(a.B),
                               static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias,
                               ordered, a.w, static_cast<T *>(a.dx));
 }
@@ -895,6 +936,39 @@ cudaError_t conv1d_dw_packed_launch(const DwArgs &a, const int32_t *offsets, cud
     if (a.B == 0 || a.T == 0) {
         conv1d_dw_zero_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(a.dw, a.dbias, a.K, a.C);
         return cudaGetLastError();
+    }
+    if (a.B <= kOrderMaxItems) {  // the pipelined kernel in its packed mode
+        int gp = 0;
+        const cudaError_t et = with_dtype(a.dtype, [&](auto tag) -> cudaError_t {
+            using T = decltype(tag);
+            if (!dw_tma_ok<T>(a) || a.vec_width < 2) return cudaErrorNotSupported;
+            DwArgs b = a;
+            b.G = conv1d_dw_packed_rows(a.T);
+            if constexpr (sizeof(T) == 2) {
+                if (a.vec_width >= 4) {
+                    switch (a.K) {
+                        case 3: return launch_tma_pass<T, 4, 3, false, true>(b, 0, 1, &gp, s, offsets);
+                        case 4: return launch_tma_pass<T, 4, 4, false, true>(b, 0, 1, &gp, s, offsets);
+                        case 5: return launch_tma_pass<T, 4, 5, false, true>(b, 0, 1, &gp, s, offsets);
+                        case 7: return launch_tma_pass<T, 4, 7, false, true>(b, 0, 1, &gp, s, offsets);
+                        case 9: return launch_tma_pass<T, 4, 9, false, true>(b, 0, 1, &gp, s, offsets);
+                        default: return cudaErrorNotSupported;
+                    }
+                }
+            }
+            switch (a.K) {
+                case 3: return launch_tma_pass<T, 2, 3, false, true>(b, 0, 1, &gp, s, offsets);
+                case 9: return launch_tma_pass<T, 2, 9, false, true>(b, 0, 1, &gp, s, offsets);
+                case 15: return launch_tma_pass<T, 2, 15, false, true>(b, 0, 1, &gp, s, offsets);
+                default: return cudaErrorNotSupported;
+            }
+        });
+        if (et != cudaErrorNotSupported) {
+            if (et != cudaSuccess) return et;
+            conv1d_dw_finalize_kernel<<<static_cast<unsigned>((n + 31) / 32), 256, 0, s>>>(a.partials, a.dw, a.dbias,
+                                                                                            gp, a.K, a.C);
+            return cudaGetLastError();
+        }
     }
     const int G = conv1d_dw_packed_rows(a.T);
     const int V = a.vec_width >= 2 ? 2 : 1;
