@@ -713,40 +713,61 @@ def main():
                   gw=torch.empty(K, C).pin_memory(), gb=torch.empty(C).pin_memory(),
                   out=torch.empty(SB, T4, F4, SC, dtype=torch.bfloat16).pin_memory(),
                   ol=torch.empty(SB, dtype=torch.int32).pin_memory())
-        s0 = sets[0]
-        dparams = dict(w=w, bias=bias, w0=w0, b0=b0, w1=w1, b1=b1, ln=ln, sl=sl)
         h2d = sum(v.numel() * v.element_size() for v in h.values())
         d2h = sum(v.numel() * v.element_size() for v in ho.values())
+        # Two device sets and three streams, as a serving pipeline runs: the inputs of step i go
+        # up on s_in while step i-1 computes and step i-2's results come down on s_out (the two
+        # copy directions use separate copy engines).  Set i % 2 is reused once step i-2's
+        # results are down.  Every step still copies all of its inputs and outputs.
+        dsets = []
+        for k in range(2):
+            z = sets[k]
+            dsets.append(dict(x=z["x"], dy=z["dy"], y=z["y"], dx=z["dx"], mel=z["mel"], out=z["out"],
+                              gw=torch.empty(K, C, device=dev), gb=torch.empty(C, device=dev),
+                              ol=torch.empty(SB, dtype=torch.int32, device=dev),
+                              w=torch.empty_like(w), bias=torch.empty_like(bias), w0=torch.empty_like(w0),
+                              b0=torch.empty_like(b0), w1=torch.empty_like(w1), b1=torch.empty_like(b1),
+                              ln=torch.empty_like(ln), sl=torch.empty_like(sl)))
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            s0["x"].copy_(h["x"], non_blocking=True)
-            s0["dy"].copy_(h["dy"], non_blocking=True)
-            s0["mel"].copy_(h["mel"], non_blocking=True)
-            for k, v in dparams.items():
-                v.copy_(h[k], non_blocking=True)
-            dw.dwconv1d_fwd(s0["x"], w, bias, s0["y"], ln, pl)
-            dw.dwconv1d_bwd_dx(s0["dy"], w, s0["dx"], ln, pl)
-            dw.dwconv1d_bwd_dw(s0["x"], s0["dy"], gw, gb, ln, pl, ws)
-            dw.dw_subsample_fwd(s0["mel"], w0, b0, w1, b1, s0["out"], sl, ol, SUB["causal"])
-            ho["y"].copy_(s0["y"], non_blocking=True)
-            ho["dx"].copy_(s0["dx"], non_blocking=True)
-            ho["gw"].copy_(gw, non_blocking=True)
-            ho["gb"].copy_(gb, non_blocking=True)
-            ho["out"].copy_(s0["out"], non_blocking=True)
-            ho["ol"].copy_(ol, non_blocking=True)
+        def e2e_step(i):
+            k = i % 2
+            z = dsets[k]
+            if i >= 2:
+                s_in.wait_event(ev_out[k])
+            with torch.cuda.stream(s_in):
+                for name in ("x", "dy", "mel", "w", "bias", "w0", "b0", "w1", "b1", "ln", "sl"):
+                    z[name].copy_(h[name], non_blocking=True)
+                ev_in[k].record(s_in)
+            stream.wait_event(ev_in[k])
+            with torch.cuda.stream(stream):  # the binding launches on the current stream
+                dw.dwconv1d_fwd(z["x"], z["w"], z["bias"], z["y"], z["ln"], pl)
+                dw.dwconv1d_bwd_dx(z["dy"], z["w"], z["dx"], z["ln"], pl)
+                dw.dwconv1d_bwd_dw(z["x"], z["dy"], z["gw"], z["gb"], z["ln"], pl, ws)
+                dw.dw_subsample_fwd(z["mel"], z["w0"], z["b0"], z["w1"], z["b1"], z["out"], z["sl"], z["ol"],
+                                    SUB["causal"])
+                ev_comp[k].record(stream)
+            s_out.wait_event(ev_comp[k])
+            with torch.cuda.stream(s_out):
+                for name in ("y", "dx", "gw", "gb", "out", "ol"):
+                    ho[name].copy_(z[name], non_blocking=True)
+                ev_out[k].record(s_out)
 
-        with torch.cuda.stream(stream):  # the binding and the copies run on the current stream
-            for _ in range(2):
-                e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         a, b_ = mk(), mk()
         if world > 1:
             dist.barrier()
-        with torch.cuda.stream(stream):
-            a.record(stream)
-            for _ in range(args.e2e_steps):
-                e2e_step()
-            b_.record(stream)
+        torch.cuda.synchronize(dev)
+        a.record(s_in)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        s_in.wait_stream(s_out)
+        b_.record(s_in)  # after the last step's results are down
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, world, dev)
         e2e = {"value": job_throughput(step_bytes, e2e_ms, world), "unit": "GB/s",
