@@ -398,6 +398,15 @@ int dw_last_cuda_error(void);
  */
 dw_status_t dw_device_error(void);
 
+/*
+ * dw_selftest_wait_timeout - checks the bounded waits: launches one block that runs the kernels'
+ * bounded mbarrier wait (with a limit 256 times shorter than theirs) on an mbarrier nothing will
+ * complete.  The wait gives up after its poll limit,
+ * records the error that dw_device_error() then reports as DW_ERR_TIMEOUT, writes 2 to *done
+ * (a device int32) and returns; no fault is raised and the context stays usable.
+ */
+dw_status_t dw_selftest_wait_timeout(int *done, dw_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,7 @@ __all__ = [
     "dwconv1d_bwd_dx_packed", "dwconv1d_bwd_dw_packed_workspace_size", "dwconv1d_bwd_dw_packed",
     "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
     "dwconv2d_fwd", "dwconv2d_bwd_dx", "dwconv2d_bwd_dw_workspace_size", "dwconv2d_bwd_dw", "conv2d_out_shape",
+    "dw_selftest_wait_timeout",
 ]
 
 DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_WORKSPACE, DW_ERR_CUDA, DW_ERR_TIMEOUT = range(6)
@@ -70,6 +71,7 @@ SIGNATURES = {
     "dw_status_string": (ctypes.c_char_p, [_int]),
     "dw_last_cuda_error": (_int, []),
     "dw_device_error": (_int, []),
+    "dw_selftest_wait_timeout": (_int, [_vp, _vp]),
 }
 
 
@@ -379,3 +381,11 @@ def dwconv2d_bwd_dw(x, dy, dw, dbias, lengths, stride, pads, workspace, stream=N
                                workspace.numel() * workspace.element_size() if workspace is not None else 0,
                                _stream(stream))
     _check("dwconv2d_bwd_dw", st)
+
+
+def dw_selftest_wait_timeout(done, stream=None):
+    """Launch the bounded-wait self-test: ``done`` (int32 CUDA tensor of 1) receives 2 once the
+    wait has given up; ``dw_device_error()`` then returns DW_ERR_TIMEOUT (and clears it)."""
+    import torch
+    _check("dw_selftest_wait_timeout", lib().dw_selftest_wait_timeout(_dev(done, "done", torch.int32, (1,)),
+                                                                      _stream(stream)))

@@ -139,10 +139,15 @@ const char *dw_status_string(dw_status_t s) {
 
 int dw_last_cuda_error(void) { return g_last_cuda_error; }
 
+dw_status_t dw_selftest_wait_timeout(int *done, dw_stream_t stream) {
+    if (done == nullptr) return DW_ERR_INVALID_ARG;
+    return cuda_status(dwk::selftest_wait_timeout_launch(done, static_cast<cudaStream_t>(stream)));
+}
+
 dw_status_t dw_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
     const unsigned int e = dwk::conv1d_fwd_take_error() | dwk::conv1d_dw_take_error() | dwk::subsample_tc_take_error() |
-                           dwk::conv2d_tma_take_error();
+                           dwk::conv2d_tma_take_error() | dwk::selftest_take_error();
     return e ? DW_ERR_TIMEOUT : DW_OK;
 }
 

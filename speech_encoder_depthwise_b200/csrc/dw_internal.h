@@ -136,6 +136,11 @@ cudaError_t conv2d_dx_tma_launch(const Conv2dArgs &a, cudaStream_t s);
 cudaError_t conv2d_dw_tma_partials(const Conv2dArgs &a, float *partials, int max_rows, int *G, cudaStream_t s);
 unsigned int conv2d_tma_take_error();
 
+// A one-block kernel whose bounded mbarrier wait must run out (nothing completes the barrier);
+// writes 2 to *done when it gave up, 1 if the wait (impossibly) succeeded.
+cudaError_t selftest_wait_timeout_launch(int *done, cudaStream_t s);
+unsigned int selftest_take_error();
+
 struct SubsampleBwdArgs {
     const float *mel, *w0, *b0, *w1;
     const void *dout;             // [B][T4][F4][C] bf16 or float32
