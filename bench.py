@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--next-rows", default="all",
                    help="comma list of the NEXT-row measurements after the step (stream, bwd, conv2d, "
-                        "f16_packed, sub_bwd), 'all' or 'none'")
+                        "f16_packed, sub_bwd, batch), 'all' or 'none'")
     return p.parse_args()
 
 
@@ -364,6 +364,35 @@ def measure_f16_packed(dw, dev, hbm):
                         "padded, and the same sequences packed (3 rotating input sets in a CUDA graph)", **res}
 
 
+def measure_batch_scaling(dw, dev, hbm):
+    """The conv1d forward and dW on the conformer shape (T=1500, C=512, K=9, len U[750,1500]) at
+    B = 16, 32 and 64 (a NEXT-row measurement, outside the step): graph replay over 3 rotating
+    input sets.  Shows the fixed cost of a launch against the per-item cost."""
+    import torch
+    from synth import conv1d_inputs
+    T, C, K, pl = 1500, 512, 9, 4
+    res = {}
+    for B in (16, 32, 64):
+        d = conv1d_inputs(B, T, C, K, dtype="bf16", len_range=(750, 1500), seed=1, with_dy=True)
+        xs = [torch.from_numpy(d["x"]).to(dev, torch.bfloat16) for _ in range(3)]
+        gs = [torch.from_numpy(d["dy"]).to(dev, torch.bfloat16) for _ in range(3)]
+        ys = [torch.empty_like(xs[0]) for _ in range(3)]
+        w, bias, ln = (torch.from_numpy(d["w"]).to(dev), torch.from_numpy(d["bias"]).to(dev),
+                       torch.from_numpy(d["lengths"]).to(dev))
+        gw, gb = torch.empty(K, C, device=dev), torch.empty(C, device=dev)
+        ws = torch.empty(dw.dwconv1d_bwd_dw_workspace_size(B, T, C, K), dtype=torch.uint8, device=dev)
+        L = np.clip(d["lengths"], 0, T)
+        byf = (int(L.sum()) + B * T) * C * 2
+        byw = 2 * int(L.sum()) * C * 2
+        tf = graph_us(dev, [lambda i=i: dw.dwconv1d_fwd(xs[i], w, bias, ys[i], ln, pl) for i in range(3)])
+        tw = graph_us(dev, [lambda i=i: dw.dwconv1d_bwd_dw(xs[i], gs[i], gw, gb, ln, pl, ws) for i in range(3)])
+        res[f"B{B}"] = {"fwd_us": tf, "fwd_hbm_frac_of_measured": byf / tf / 1e3 / hbm,
+                        "dw_us": tw, "dw_hbm_frac_of_measured": byw / tw / 1e3 / hbm}
+        del xs, gs, ys
+    return {"workload": f"conformer dwconv1d {T}x{C}, K={K}, bf16, len U[750,1500], B in 16/32/64 "
+                        "(3 rotating input sets in a CUDA graph)", **res}
+
+
 CONV2D = dict(B=16, T=750, F=20, C=256, KT=3, KF=3, stride=(2, 2), pads=(1, 1, 1), len_range=(375, 750), seed=5)
 
 
@@ -521,6 +550,29 @@ def cpu_rate(cs, ss, seconds, steps=None):
         if steps is None and total_t >= seconds:
             break
     return total_b / total_t / 1e9, desc, oracle.num_threads(), total_t / n
+
+
+def cpu_single_thread_cfg1_ms():
+    """The oracle's conv1d forward on the fp32 parity workload (1x200x256, K=9, pads 4|4, no
+    mask), on one host thread: median of 5 runs, in a subprocess with OMP_NUM_THREADS=1."""
+    import subprocess
+    code = ("import sys, time; sys.path.insert(0, %r)\n"
+            "import numpy as np, oracle\n"
+            "from synth import conv1d_inputs\n"
+            "d = conv1d_inputs(1, 200, 256, 9, dtype='f32', len_range=None, seed=0)\n"
+            "oracle.dwconv1d_fwd(d['x'], d['w'], d['bias'], None, 4)\n"
+            "ts = []\n"
+            "for _ in range(5):\n"
+            "    t0 = time.perf_counter(); oracle.dwconv1d_fwd(d['x'], d['w'], d['bias'], None, 4)\n"
+            "    ts.append(time.perf_counter() - t0)\n"
+            "print(sorted(ts)[2] * 1e3, oracle.num_threads())\n") % ROOT
+    try:
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120,
+                           env=dict(os.environ, OMP_NUM_THREADS="1"))
+        ms, thr = r.stdout.split()
+        return {"ms": float(ms), "threads": int(thr), "workload": "conv1d forward 1x200x256 fp32, K=9, pads 4|4"}
+    except Exception as e:  # reported, never fatal
+        return {"unavailable": str(e)[:200]}
 
 
 def reference_arm(args, world, rank):
@@ -810,18 +862,20 @@ def main():
         ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
-        want = {"stream", "bwd", "conv2d", "f16_packed", "sub_bwd"} if args.next_rows == "all" else \
+        want = {"stream", "bwd", "conv2d", "f16_packed", "sub_bwd", "batch"} if args.next_rows == "all" else \
             set() if args.next_rows == "none" else set(args.next_rows.split(","))
         measures = [("stream", "dwconv1d_stream_fwd", lambda: measure_stream(dw, dev, hbm)),
                     ("bwd", "dwconv1d_bwd", lambda: measure_bwd(dw, dev, hbm)),
                     ("conv2d", "dwconv2d", lambda: measure_conv2d(dw, dev, hbm)),
                     ("f16_packed", "f16_and_packed", lambda: measure_f16_packed(dw, dev, hbm)),
-                    ("sub_bwd", "dw_subsample_bwd", lambda: measure_sub_bwd(dw, dev, hbm, fp32_tflops))]
+                    ("sub_bwd", "dw_subsample_bwd", lambda: measure_sub_bwd(dw, dev, hbm, fp32_tflops)),
+                    ("batch", "conv1d_batch_scaling", lambda: measure_batch_scaling(dw, dev, hbm))]
         next_rows = {name: fn() for key, name, fn in measures if key in want}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
             v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)
-            cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+            cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc,
+                   "single_thread_cfg1": cpu_single_thread_cfg1_ms()}
         clocks = clk.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
