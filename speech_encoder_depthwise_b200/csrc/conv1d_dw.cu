@@ -187,7 +187,6 @@ constexpr int kDwConsumers = DW_DW_CONSUMERS;  // consumer warps per block
 constexpr int kDwR = DW_DW_R;                  // frames per consumer thread per unit
 constexpr int kDwStages = DW_DW_STAGES;        // shared-memory ring depth
 constexpr int kDwBlocks = DW_DW_BLOCKS;        // resident blocks per SM
-constexpr int kDwTmaThreads = 32 * (1 + kDwConsumers);
 
 // FUSED: the same pass also computes the data gradient, so the dy tile carries K-1 halo rows
 // (the dx correlation reads dy frames s + pad_left - k).  Its threads hold two sets of
