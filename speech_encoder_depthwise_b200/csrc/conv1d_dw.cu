@@ -620,7 +620,10 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
             best_c = c;
         }
     }
-    if (best_g < 1) return cudaErrorInvalidConfiguration;
+    if (best_g < 1) {  // more channel tiles than resident blocks: one block per tile, in waves
+        best_g = 1;
+        best_c = 1;
+    }
     *gp_out = best_g / best_c;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(best_g, nCT);
