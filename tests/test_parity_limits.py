@@ -4,7 +4,9 @@
   gradient (32768 channel tiles: more tiles than resident blocks);
 - a long sequence (T = 2^20 frames) for the conv1d forward and weight gradient;
 - the subsampler with more items (4097) than its balanced unit deal handles (round robin);
-- the conv2d kernels with 65536 channels (1024 channel slabs).
+- the conv2d kernels with 65536 channels (1024 channel slabs);
+- the widest accepted kernel (K = 4096, longer than the sequence) and 4096 streams of the
+  streaming conv.
 Bars as in the other parity tests (bf16: <= max(2e-2, 1 ulp) and faithful; weight gradients
 <= 2e-2 absolute and <= 1e-5 * RMS).
 """
@@ -100,3 +102,28 @@ def test_conv2d_many_channel_slabs():
     assert_bf16_close(y.numpy(), oracle.dwconv2d_fwd(d["x"], d["w"], d["bias"], d["lengths"], stride, pads)[0])
     assert_bf16_close(dx.numpy(), oracle.dwconv2d_bwd_dx(d["dy"], d["w"], d["lengths"], T, F, stride, pads))
     grads_close((gw.numpy(), gb.numpy()), oracle.dwconv2d_bwd_dw(d["x"], d["dy"], 3, 3, d["lengths"], stride, pads))
+
+
+def test_widest_kernel():
+    """K = 4096 (the largest accepted width), far longer than the sequence: the runtime-width
+    kernels and the weight gradient's passes of taps."""
+    d = conv1d_inputs(2, 100, 8, 4096, dtype="bf16", len_range=(60, 100), seed=6, with_dy=True)
+    conv1d_all(d, 4096, 2048)
+
+
+def test_many_streams():
+    B, T, C, K = 4096, 1, 64, 9
+    rng = np.random.default_rng(8)
+    from synth import bf16_round
+    w = bf16_round(rng.standard_normal((K, C)) / 3.0)
+    b = bf16_round(rng.standard_normal(C) * 0.3)
+    cache = torch.zeros(B, K - 1, C, dtype=BF, device="cuda")
+    cache_o = np.zeros((B, K - 1, C))
+    for _ in range(3):
+        x = bf16_round(rng.standard_normal((B, T, C)))
+        y = torch.empty(B, T, C, dtype=BF, device="cuda")
+        dw.dwconv1d_stream_fwd(dev(x, BF), dev(w), dev(b), y, cache, None)
+        torch.cuda.synchronize()
+        ry, cache_o = oracle.dwconv1d_stream_fwd(x, w, b, cache_o, None)
+        assert_bf16_close(y.float().cpu().numpy(), ry)
+        assert np.array_equal(cache.float().cpu().numpy(), cache_o)
