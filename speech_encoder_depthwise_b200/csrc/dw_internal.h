@@ -143,7 +143,7 @@ unsigned int selftest_take_error();
 
 struct SubsampleBwdArgs {
     const float *mel, *w0, *b0, *w1;
-    const void *dout;             // [B][T4][F4][C] bf16 or float32
+    const void *dout;             // [B][T4][F4][C] bf16, fp16 or float32
     const int32_t *lengths;
     float *dw0, *db0, *dw1, *db1;  // [3][3][C], [C], [3][3][C], [C]
     float *partials;              // workspace: [rows][20][C]
@@ -153,6 +153,10 @@ struct SubsampleBwdArgs {
 int subsample_bwd_partial_rows(int64_t B, int64_t T, int64_t F);
 size_t subsample_bwd_workspace_bytes(int64_t B, int64_t T, int64_t F, int64_t C);
 cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s);
+// Tensor-core subsampler backward for 16-bit dout with C a multiple of 8 (16-byte aligned dout
+// rows): writes partial rows [rows][20][C] (rows <= max_rows) for the fixed-order finalize;
+// cudaErrorNotSupported where the SIMT kernel must serve.
+cudaError_t subsample_bwd_tc_launch(const SubsampleBwdArgs &a, int max_rows, int *rows, cudaStream_t s);
 // Tensor-core subsampler: usable when the output rows are 16-byte aligned (C * element size a
 // multiple of 16, aligned base); the SIMT kernel serves every other case.
 bool subsample_tc_eligible(const SubsampleArgs &a);

@@ -294,6 +294,17 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
             a.dw0, a.db0, a.dw1, a.db1, static_cast<int>(a.C));
         return cudaGetLastError();
     }
+    const int64_t E = static_cast<int64_t>(kSbSlots) * a.C;
+    {
+        int rows = 0;
+        const cudaError_t et = subsample_bwd_tc_launch(a, subsample_bwd_partial_rows(a.B, a.T, a.F), &rows, s);
+        if (et == cudaSuccess) {
+            dw_subsample_bwd_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(
+                a.partials, rows, static_cast<int>(a.C), a.dw0, a.db0, a.dw1, a.db1);
+            return cudaGetLastError();
+        }
+        if (et != cudaErrorNotSupported) return et;
+    }
     const int nRT = static_cast<int>((T2 + kSbRT - 1) / kSbRT), nST = static_cast<int>((F2 + kSbST - 1) / kSbST);
     const int64_t nCG = (a.C + 2 * kSbThreads - 1) / (2 * kSbThreads);
     int G = subsample_bwd_partial_rows(a.B, a.T, a.F);
@@ -343,7 +354,6 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
 #undef DW_SB_LAUNCH
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t E = static_cast<int64_t>(kSbSlots) * a.C;
     dw_subsample_bwd_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(
         a.partials, G, static_cast<int>(a.C), a.dw0, a.db0, a.dw1, a.db1);
     return cudaGetLastError();

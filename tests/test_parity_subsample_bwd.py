@@ -18,7 +18,7 @@ import torch
 import oracle
 import speech_encoder_depthwise_b200 as dw
 from gpuhelp import Guarded, dev, max_abs, rms
-from synth import bf16_round, subsample_inputs
+from synth import bf16_round, f16_round, subsample_inputs
 
 pytestmark = pytest.mark.gpu
 KINK = 1e-5
@@ -63,7 +63,7 @@ def rounded_dout(d, causal, seed, dtype="bf16"):
     C = d["w0"].shape[-1]
     T4, F4 = oracle.subsample_out_shape(T, F, causal)
     g = np.random.default_rng(seed).standard_normal((B, T4, F4, C)).astype(np.float32)
-    return bf16_round(g) if dtype == "bf16" else g
+    return {"bf16": bf16_round, "f16": f16_round}.get(dtype, lambda x: x)(g)
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -103,3 +103,25 @@ def test_results_are_bitwise_reproducible():
     b = gpu_bwd(d, dout, False)
     for u, v in zip(a, b):
         assert np.array_equal(u, v)
+
+
+# Shapes the tensor-core kernel takes (16-bit dout, C a multiple of 8): one channel tile and a
+# ragged second one, F2 past one 40-column block, T from 1, many short items, odd unit counts.
+TC = [(1, 1, 1, 8), (2, 37, 81, 136), (3, 130, 100, 256), (5, 61, 80, 64), (7, 9, 3, 16), (1, 400, 80, 384)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,T,F,C", TC)
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_tensor_core_shapes(B, T, F, C, causal, dtype):
+    d = subsample_inputs(B, T, F, C, len_range=(0, T), seed=T * 7 + F + C)
+    d["lengths"][0] = T
+    dout = rounded_dout(d, causal, T + F + C, dtype)
+    got = gpu_bwd(d, dout, causal, dtype=torch.bfloat16 if dtype == "bf16" else torch.float16)
+    check(d, dout, causal, got)
+
+
+def test_tensor_core_full_workload_f16_causal():
+    d = subsample_inputs(16, 3000, 80, 256, len_range=(1500, 3000), seed=13)
+    dout = rounded_dout(d, True, 14, "f16")
+    check(d, dout, True, gpu_bwd(d, dout, True, dtype=torch.float16))
