@@ -74,7 +74,7 @@ constexpr int kDoutElems = 128 * kDoutCols * kDoutRows;
 constexpr int kRing = 4;                    // dout chunks in flight per group
 constexpr int kWinSlots = 4;
 constexpr int kListCap = 768;
-constexpr int kBarBuild = 1, kBarGroup0 = 2, kBarAll = 4;
+constexpr int kBarBuild = 1, kBarAll = 2;
 constexpr int kTmemCols = 512;
 constexpr int kD2Col = 192;
 
@@ -87,7 +87,7 @@ constexpr int kOffDout = kOffB2 + kGroups * 2 * kTileB2;         // [group][ring
 constexpr int kOffWin = kOffDout + kGroups * kRing * kDoutElems * 2;
 constexpr int kOffList = kOffWin + kWinSlots * kWinFloats * 4;
 constexpr int kOffBar = kOffList + kListCap * 4;
-constexpr int kSmemBytes = kOffBar + 256;
+constexpr int kSmemBytes = kOffBar + 320;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 
 static_assert(kOffB1 % 1024 == 0 && kOffA2 % 1024 == 0 && kOffB2 % 1024 == 0, "swizzle atoms are 1024-byte aligned");
@@ -113,6 +113,19 @@ __device__ __forceinline__ void dout_box_load(void *dst, const void *tmap, int c
         "%5}], [%6];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c), "r"(j), "r"(i), "r"(b), "r"(smem_addr(bar))
         : "memory");
+}
+
+// Whether the phase with the given parity has completed (does not wait).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 // 32 consecutive accumulator columns of this thread's lane, waited for.
@@ -181,8 +194,9 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
              *d1_empty = bars + 4 /* [group] */, *a2_empty = bars + 6 /* [group][slot] */,
              *dfull = bars + 10 /* [group][ring] */, *win_full = bars + 18, *win_free = bars + 22,
              *mma_done = bars + 26, *d2_done = bars + 27 /* [group] */;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 29);
-    int *count = reinterpret_cast<int *>(bars + 30);
+    uint64_t *a2_full = bars + 29;  // [group][slot]: one arrival per warp of the group
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 33);
+    int *count = reinterpret_cast<int *>(bars + 34);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int g = blockIdx.x % nG;                 // channel tile of this block
@@ -198,6 +212,8 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
             mbar_init(&d1_empty[i], kGroupThreads / 32);  // one arrival per warp of the group
             mbar_init(&a2_empty[2 * i], 1);
             mbar_init(&a2_empty[2 * i + 1], 1);
+            mbar_init(&a2_full[2 * i], kGroupThreads / 32);
+            mbar_init(&a2_full[2 * i + 1], kGroupThreads / 32);
             for (int r = 0; r < kRing; ++r) mbar_init(&dfull[i * kRing + r], 1);
             mbar_init(&d2_done[i], 1);
         }
@@ -276,7 +292,6 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
         // ------------------------------------------------------------ epilogue groups
         const int grp = warp >> 2, qw = warp & 3, m = qw * 32 + lane;
         const int c = g * 128 + m;
-        const bool leader = (threadIdx.x & (kGroupThreads - 1)) == 0;
         const uint32_t tl = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + grp * 256;
         const uint32_t d1 = tl, d2 = tl + kD2Col;
         float2 W[3][3], gw1[3][3];
@@ -298,22 +313,10 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
             gb0 += r[18];
         };
         const int nU = (nA - grp + 1) / 2;            // units grp, grp + 2, ...
-        const int nPos = nU * kChunks;                 // chunks of this group
         unsigned char *a2 = tA2 + grp * (2 * 2 * kTileA2);
         unsigned char *b2 = tB2 + grp * (2 * kTileB2);
         TD *rg = ring + grp * kRing * kDoutElems;
         uint64_t *df = dfull + grp * kRing;
-        int issued = 0;                                // dout chunks requested (leader)
-        auto prefetch = [&](int p) {
-            const int ul = p / kChunks, k = p - ul * kChunks;
-            const uint32_t e = ulist[grp + 2 * ul];
-            uint64_t *bar = &df[p & (kRing - 1)];
-            mbar_arrive_expect_tx(bar, kDoutElems * static_cast<uint32_t>(sizeof(TD)));
-            dout_box_load(rg + (p & (kRing - 1)) * kDoutElems, &dout_map, g * 128, 20 * unit_cb(e) + 4 * k,
-                          2 * unit_rb(e), unit_b(e), bar);
-        };
-        if (leader)
-            for (; issued < kRing && issued < nPos; ++issued) prefetch(issued);
         // pixel pairs: rows eA, eA + 2 take the taps p = 0 and 2, rows oA, oA + 2 the tap p = 1
         constexpr int eA = PT1 ? 1 : 0, oA = PT1 ? 0 : 1;
         bool ok = true;
@@ -328,6 +331,8 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
             const float *wE = win + ws * kWinFloats, *wO = wE + kWR * kWS;
             bool wok = mbar_wait(&d1_full[grp], ul & 1);
             wok = wok && mbar_wait(&win_full[ws], (idx >> 2) & 1);
+            ok = __all_sync(0xffffffffu, wok);
+            if (!ok) break;
             tc_fence_after();
 #pragma unroll 1
             for (int k = 0; k < kChunks; ++k, ++pos) {
@@ -417,35 +422,21 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
                         *swz_word(bt, 9 + t, lane) = x - h;
                     }
                 }
+                // this warp's rows of the chunk are written: hand them to the MMA thread
                 fence_async_smem();
-                ok = named_bar_and(kBarGroup0 + grp, kGroupThreads, wok);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a2_full[2 * grp + (pos & 1)]);
+                ok = __all_sync(0xffffffffu, wok);
                 if (!ok) break;
-                if (leader) {
-                    tc_fence_after();
-                    const uint64_t bd = sw128_desc(smem_addr(bt));
-#pragma unroll
-                    for (int hl = 0; hl < 2; ++hl) {
-                        const uint64_t ad = sw128_desc(smem_addr(ah + hl * kTileA2));
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)  // 32 pixels = 4 K-steps of 8
-                            mma_tf32(d2 + 32 * (pos & 1), ad + 2 * ks, bd + 2 * ks, kIdescW, (hl | ks) != 0 ? 1u : 0u);
-                    }
-                    mma_commit(&a2_empty[2 * grp + (pos & 1)]);
-                    if (k == kChunks - 1) mbar_arrive(&win_free[ws]);  // the group is done with the window
-                    if (issued < nPos) prefetch(issued++);
-                }
                 ++done;
             }
         }
-        // dout chunks requested but never consumed (only after a give-up)
-        if (leader)
-            for (int p = pos; p < issued; ++p) mbar_wait(&df[p & (kRing - 1)], (p / kRing) & 1, kSpinLimit >> 4);
         // slots 0..8 dw0, 9 db0, 10..18 dw1, 19 db1 (the partial row layout)
         float vals[20];
 #pragma unroll
         for (int i = 0; i < 20; ++i) vals[i] = 0.f;
-        if (done > 0) {  // the last two chunks' sums
-            if (leader) mma_commit(&d2_done[grp]);
+        if (done > 0) {  // the last two chunks' sums, once the group's last MMAs have completed
             const bool dok = mbar_wait(&d2_done[grp], 0);
             tc_fence_after();
             for (int p = done >= 2 ? done - 2 : 0; p < done; ++p) take_d2(p);
@@ -545,21 +536,76 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
             mbar_arrive(b1_full);
         }
     } else if (lane == 0) {
-        // ------------------------------------------------------------ conv0 MMA issuer
+        // ------------------------------------------------------------ MMA and copy issuer
+        // Three streams, served as their inputs become ready (polled, so that no stream waits
+        // behind another): the conv0 MMAs of each unit (patch rows built, the group's z buffer
+        // free), and per group the dw0 MMAs of each chunk (all four warps' rows written), each
+        // followed by the dout copy of the group's chunk four ahead.
         const uint64_t ad = sw128_desc(smem_addr(tA1)), bd = sw128_desc(smem_addr(tB1));
-        bool ok = true;
-        for (int idx = 0; idx < nA && ok; ++idx) {
-            const int grp = idx & 1, n = idx >> 1;
-            ok = mbar_wait(b1_full, idx & 1) && mbar_wait(&d1_empty[grp], (n & 1) ^ 1);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t d = tmem_base + grp * 256;
+        const int nP[2] = {(nA + 1) / 2 * kChunks, nA / 2 * kChunks};
+        int cp[2] = {0, 0}, issued[2] = {0, 0}, zi = 0;
+        auto prefetch = [&](int grp, int p) {
+            const int ul = p / kChunks, k = p - ul * kChunks;
+            const uint32_t e = ulist[grp + 2 * ul];
+            uint64_t *bar = &dfull[grp * kRing + (p & (kRing - 1))];
+            mbar_arrive_expect_tx(bar, kDoutElems * static_cast<uint32_t>(sizeof(TD)));
+            dout_box_load(ring + (grp * kRing + (p & (kRing - 1))) * kDoutElems, &dout_map, g * 128,
+                          20 * unit_cb(e) + 4 * k, 2 * unit_rb(e), unit_b(e), bar);
+        };
+        for (int grp = 0; grp < kGroups; ++grp)
+            for (; issued[grp] < kRing && issued[grp] < nP[grp]; ++issued[grp]) prefetch(grp, issued[grp]);
+        uint32_t idle = 0;
+        while (zi < nA || cp[0] < nP[0] || cp[1] < nP[1]) {
+            bool prog = false;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // K = 32 TF32 words = 4 steps of 8
-                mma_tf32(d, ad + 2 * ks, bd + 2 * ks, kIdescZ, ks > 0 ? 1u : 0u);
-            mma_commit(&d1_full[grp]);
-            mma_commit(b1_empty);
+            for (int grp = 0; grp < kGroups; ++grp) {
+                const int p = cp[grp];
+                if (p < nP[grp] && mbar_test(&a2_full[2 * grp + (p & 1)], (p >> 1) & 1)) {
+                    tc_fence_after();
+                    unsigned char *ah = tA2 + grp * (2 * 2 * kTileA2) + (p & 1) * (2 * kTileA2);
+                    const uint64_t b2d = sw128_desc(smem_addr(tB2 + grp * (2 * kTileB2) + (p & 1) * kTileB2));
+                    const uint32_t d2 = tmem_base + grp * 256 + kD2Col + 32 * (p & 1);
+#pragma unroll
+                    for (int hl = 0; hl < 2; ++hl) {
+                        const uint64_t a2d = sw128_desc(smem_addr(ah + hl * kTileA2));
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)  // 32 pixels = 4 K-steps of 8
+                            mma_tf32(d2, a2d + 2 * ks, b2d + 2 * ks, kIdescW, (hl | ks) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&a2_empty[2 * grp + (p & 1)]);
+                    if (p % kChunks == kChunks - 1)  // the group is done with the unit's window
+                        mbar_arrive(&win_free[(grp + 2 * (p / kChunks)) & (kWinSlots - 1)]);
+                    if (issued[grp] < nP[grp]) prefetch(grp, issued[grp]++);
+                    cp[grp] = p + 1;
+                    if (cp[grp] == nP[grp]) mma_commit(&d2_done[grp]);
+                    prog = true;
+                }
+            }
+            if (zi < nA && mbar_test(b1_full, zi & 1) && mbar_test(&d1_empty[zi & 1], ((zi >> 1) & 1) ^ 1)) {
+                tc_fence_after();
+                const uint32_t d = tmem_base + (zi & 1) * 256;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // K = 32 TF32 words = 4 steps of 8
+                    mma_tf32(d, ad + 2 * ks, bd + 2 * ks, kIdescZ, ks > 0 ? 1u : 0u);
+                mma_commit(&d1_full[zi & 1]);
+                mma_commit(b1_empty);
+                ++zi;
+                prog = true;
+            }
+            if (prog) {
+                idle = 0;
+            } else {
+                if (++idle > kSpinLimit) {  // nothing became ready for a long time: give up
+                    atomicOr(&dw_device_error_flag, kErrWaitTimeout);
+                    break;
+                }
+                __nanosleep(32);
+            }
         }
+        // the copies still in flight land before shared memory is released
+        for (int grp = 0; grp < kGroups; ++grp)
+            for (int p = issued[grp] > kRing ? issued[grp] - kRing : 0; p < issued[grp]; ++p)
+                mbar_wait(&dfull[grp * kRing + (p & (kRing - 1))], (p / kRing) & 1, kSpinLimit >> 4);
         // every issued MMA has finished before tensor memory is released
         mma_commit(mma_done);
         mbar_wait(mma_done, 0);
