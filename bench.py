@@ -295,6 +295,7 @@ def measure_sub_bwd(dw, dev, hbm, fp32_tflops):
     fl = int(L2.sum()) * F2 * C * 36 + int(L4.sum()) * F4 * C * 36
     t_roof = max(by / (hbm * 1e9), fl / (fp32_tflops * 1e12))
     return {"workload": "subsampler backward, mel 16x3000x80 -> C256, bf16 dout, sym, len U[1500,3000]",
+            "kernel": "dw_subsample_bwd_tc_kernel (tcgen05: conv0 recompute and dw0/db0) + finalize",
             "us": us, "TFLOP_per_s": fl / (us * 1e-6) / 1e12, "roofline_frac": t_roof / (us * 1e-6),
             "alg_bytes": by, "alg_flops": fl}
 
