@@ -368,7 +368,9 @@ def measure_f16_packed(dw, dev, hbm):
 def measure_batch_scaling(dw, dev, hbm):
     """The conv1d forward and dW on the conformer shape (T=1500, C=512, K=9, len U[750,1500]) at
     B = 16, 32 and 64 (a NEXT-row measurement, outside the step): graph replay over 3 rotating
-    input sets.  Shows the fixed cost of a launch against the per-item cost."""
+    input sets.  Shows the fixed cost of a launch against the per-item cost, next to torch's
+    elementwise kernel moving the forward's bytes (what a generic bandwidth-bound launch gets at
+    each size)."""
     import torch
     from synth import conv1d_inputs
     T, C, K, pl = 1500, 512, 9, 4
@@ -387,9 +389,15 @@ def measure_batch_scaling(dw, dev, hbm):
         byw = 2 * int(L.sum()) * C * 2
         tf = graph_us(dev, [lambda i=i: dw.dwconv1d_fwd(xs[i], w, bias, ys[i], ln, pl) for i in range(3)])
         tw = graph_us(dev, [lambda i=i: dw.dwconv1d_bwd_dw(xs[i], gs[i], gw, gb, ln, pl, ws) for i in range(3)])
+        # the floor at this size: torch's elementwise kernel (a STREAM-style scale, dst = 1 * src)
+        # moving the forward's bytes, half read and half written, timed the same way
+        srcs = [torch.zeros(byf // 4, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        dsts = [torch.empty_like(srcs[0]) for _ in range(3)]
+        tc = graph_us(dev, [lambda i=i: torch.mul(srcs[i], 1.0, out=dsts[i]) for i in range(3)])
         res[f"B{B}"] = {"fwd_us": tf, "fwd_hbm_frac_of_measured": byf / tf / 1e3 / hbm,
-                        "dw_us": tw, "dw_hbm_frac_of_measured": byw / tw / 1e3 / hbm}
-        del xs, gs, ys
+                        "dw_us": tw, "dw_hbm_frac_of_measured": byw / tw / 1e3 / hbm,
+                        "copy_us": tc, "fwd_vs_copy": tc / tf}
+        del xs, gs, ys, srcs, dsts
     return {"workload": f"conformer dwconv1d {T}x{C}, K={K}, bf16, len U[750,1500], B in 16/32/64 "
                         "(3 rotating input sets in a CUDA graph)", **res}
 
