@@ -107,7 +107,8 @@ def test_results_are_bitwise_reproducible():
 
 # Shapes the tensor-core kernel takes (16-bit dout, C a multiple of 8): one channel tile and a
 # ragged second one, F2 past one 40-column block, T from 1, many short items, odd unit counts.
-TC = [(1, 1, 1, 8), (2, 37, 81, 136), (3, 130, 100, 256), (5, 61, 80, 64), (7, 9, 3, 16), (1, 400, 80, 384)]
+TC = [(1, 1, 1, 8), (2, 37, 81, 136), (3, 130, 100, 256), (5, 61, 80, 64), (7, 9, 3, 16), (1, 400, 80, 384),
+      (1, 9, 1270, 8), (1, 9, 1290, 8)]  # 16 column blocks (the most a unit entry holds), then 17 (SIMT)
 
 
 @pytest.mark.parametrize("causal", [False, True])
