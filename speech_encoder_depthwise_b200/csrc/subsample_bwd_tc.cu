@@ -32,14 +32,15 @@
 // Roles (384 threads, one block per SM, persistent; three warps per SM sub-partition leave
 // 168 registers a thread):
 //   warps 0-3, 4-7  two epilogue groups; group g takes the block's units g, g + 2, ...;
-//                   warp w reads TMEM lanes 32 (w % 4) + [0, 32) (its channel quarter).  A group
-//                   reads z, computes dz, dh, dw1 and writes the chunk's A2 rows and B2 rows;
-//                   its leader thread then issues the chunk's MMAs and prefetches dout chunks
-//                   four ahead
+//                   warp w reads TMEM lanes 32 (w % 4) + [0, 32) (its channel quarter).  Per
+//                   chunk a warp reads z, computes dz, dh, dw1, writes its 32 rows of A2 and its
+//                   taps' B2 rows, and arrives on the slot's mbarrier; the warps of a group never
+//                   wait for one another
 //   warps 8-10      patch builders: stage the unit's 9 x 81 mel window (even and odd columns
 //                   apart, so that pixel-wise reads are free of bank conflicts) and build B1
-//   warp 11         allocates tensor memory, lists the block's units; one thread issues the
-//                   conv0 MMAs
+//   warp 11         allocates tensor memory and lists the block's units; its lane 0 polls the
+//                   ready-streams (conv0 per unit, dw0 per chunk of either group) and issues the
+//                   MMAs and the dout copies, four chunks ahead per group
 // Tensor memory: group g has D1 at columns 256 g + [0, 160) and its two D2 slots at
 // 256 g + 192 + 32 s + [0, 32).
 // Every mbarrier wait is bounded; a wait that gives up records an error (dw_device_error) and
