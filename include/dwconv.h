@@ -21,8 +21,9 @@
  *    B == 0 or T == 0 is a valid no-op.  Misaligned pointers, or a C that is not a
  *    multiple of the vector width, take a narrower (slower) path and stay correct.
  *  - Arithmetic: bf16, fp16 or float32 I/O, float32 accumulation, 16-bit stores rounded to
- *    nearest even.  The subsampler's conv0 runs on the tensor cores (float32-accurate split);
- *    everything else on the FP32 pipes.
+ *    nearest even.  The subsampler's conv0 runs on the tensor cores (float32-accurate split),
+ *    and so do its backward's conv0 recompute and dw0/db0 reduction; everything else runs on the
+ *    FP32 pipes.
  */
 #ifndef DWCONV_B200_H
 #define DWCONV_B200_H
@@ -295,9 +296,10 @@ size_t dw_subsample_bwd_workspace_size(int64_t B, int64_t T, int64_t F, int64_t 
  *   db1 = sum doutm;   dw1[p,q,c] = sum doutm[i,j,c] hpad[2i+p, 2j+q, c]
  *   dh  = conv_dw1 transposed applied to doutm (taps w1);  dz = [r < ceil(len_b/2)] [z > 0] dh
  *   db0 = sum dz;      dw0[p,q,c] = sum dz[r,s,c] melpad[2r+p, 2s+q]
- * The mel input takes no gradient.  float32 accumulation; the per-block partial sums go to
- * `workspace` and a second kernel adds them in a fixed order (reproducible for given sizes on a
- * given GPU model).  No atomics.
+ * The mel input takes no gradient.  float32 accumulation (z and the dw0/db0 sums on the tensor
+ * cores with float32-accurate operand splits when dout rows are 16-byte aligned and 16-bit);
+ * the per-block partial sums go to `workspace` and a second kernel adds them in a fixed order
+ * (reproducible for given sizes on a given GPU model).  No atomics.
  *
  *  mel, w0, b0, w1, lengths, B, T, F, C, causal: as dw_subsample_fwd (b1 is not needed)
  *  dout         [B][T4][F4][C] dout_dtype (DW_BF16, DW_F16 or DW_F32), device
