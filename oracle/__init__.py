@@ -91,7 +91,7 @@ class Oracle:
         lib.oracle_dw_subsample_bwd.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L, ctypes.c_int,
                                                 _D, _D, _D, _D]
         lib.oracle_dw_subsample_bwd_kinks.argtypes = [_D, _D, _D, _D, _D, _I, _L, _L, _L, _L, ctypes.c_int,
-                                                      ctypes.c_double, _D, _D]
+                                                      ctypes.c_double, ctypes.c_double, _D, _D]
         lib.oracle_dwconv2d_fwd.argtypes = [_D, _D, _D, _I] + [_L] * 11 + [_D, _I]
         lib.oracle_dwconv2d_bwd_dx.argtypes = [_D, _D, _I] + [_L] * 11 + [_D]
         lib.oracle_dwconv2d_bwd_dw.argtypes = [_D, _D, _I] + [_L] * 11 + [_D, _D]
@@ -207,9 +207,10 @@ class Oracle:
             raise ValueError(f"oracle_dw_subsample_bwd rejected its arguments (rc={rc})")
         return dw0, db0, dw1, db1
 
-    def dw_subsample_bwd_kinks(self, mel, w0, b0, w1, dout, lengths, causal, delta):
+    def dw_subsample_bwd_kinks(self, mel, w0, b0, w1, dout, lengths, causal, delta, delta_rel=0.0):
         """Bounds on how much dw0 / db0 can move when the ReLU decision flips at h pixels with
-        |z| <= delta: returns (kdw0 [3,3,C], kdb0 [C])."""
+        |z| <= delta + delta_rel * S, S = |b0| + sum_t |melpad_t w0_t| (the magnitudes of z's
+        terms): returns (kdw0 [3,3,C], kdb0 [C])."""
         mel = _f64(mel); w0 = _f64(w0); b0 = _f64(b0); w1 = _f64(w1); dout = _f64(dout)
         B, T, F = mel.shape
         C = w0.shape[-1]
@@ -217,7 +218,7 @@ class Oracle:
         kdw0 = np.empty((3, 3, C)); kdb0 = np.empty(C)
         rc = self.lib.oracle_dw_subsample_bwd_kinks(_dp(mel), _dp(w0), _dp(b0), _dp(w1), _dp(dout), _ip(ln),
                                                     B, T, F, C, int(bool(causal)), float(delta),
-                                                    _dp(kdw0), _dp(kdb0))
+                                                    float(delta_rel), _dp(kdw0), _dp(kdb0))
         if rc:
             raise ValueError(f"oracle_dw_subsample_bwd_kinks rejected its arguments (rc={rc})")
         return kdw0, kdb0
@@ -346,8 +347,8 @@ def dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal):
     return default().dw_subsample_bwd(mel, w0, b0, w1, dout, lengths, causal)
 
 
-def dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, lengths, causal, delta):
-    return default().dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, lengths, causal, delta)
+def dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, lengths, causal, delta, delta_rel=0.0):
+    return default().dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, lengths, causal, delta, delta_rel)
 
 
 def dwconv1d_bwd_dx(dy, w, lengths, pad_left):

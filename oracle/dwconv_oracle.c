@@ -381,13 +381,16 @@ int oracle_dw_subsample_bwd(const double *mel, const double *w0, const double *b
  * Tolerance term for the subsampler backward at the ReLU kink.  The derivative [z > 0] is a
  * decision taken on a floating-point z: where |z| is within rounding of 0, a float32 evaluation
  * and this float64 one may decide differently, and each such h pixel moves dw0 by at most
- * |dz| |melpad tap| and db0 by at most |dz|.  This returns those bounds summed over the h pixels
- * with |z| <= delta (unmasked rows only), per tap and channel: kdw0 [3][3][C], kdb0 [C].
+ * |dz| |melpad tap| and db0 by at most |dz|.  The rounding error of any evaluation of
+ * z = b0 + sum_t melpad_t w0_t is bounded by a multiple of the sum of the magnitudes of its
+ * terms, S = |b0| + sum_t |melpad_t w0_t|, so a pixel counts when |z| <= delta + delta_rel * S
+ * (unmasked rows only).  This returns the bounds summed over those pixels, per tap and
+ * channel: kdw0 [3][3][C], kdb0 [C].
  */
 int oracle_dw_subsample_bwd_kinks(const double *mel, const double *w0, const double *b0,
                                   const double *w1, const double *dout, const int32_t *lengths,
                                   int64_t B, int64_t T, int64_t F, int64_t C, int causal,
-                                  double delta, double *kdw0, double *kdb0)
+                                  double delta, double delta_rel, double *kdw0, double *kdb0)
 {
     if (B < 0 || T < 0 || F < 1 || C < 1) return 1;
     const int64_t Pt = causal ? 2 : 1, Pb = causal ? 0 : 1;
@@ -410,9 +413,13 @@ int oracle_dw_subsample_bwd_kinks(const double *mel, const double *w0, const dou
         for (int64_t c = 0; c < C; ++c) {
             for (int64_t r = 0; r < T2 && r < L2; ++r)
                 for (int64_t s = 0; s < F2; ++s) {
-                    double zv = b0[c];
-                    for (int64_t t = 0; t < 9; ++t) zv += melpad[(2 * r + t / 3) * FP + (2 * s + t % 3)] * w0[t * C + c];
-                    if (fabs(zv) > delta) continue;
+                    double zv = b0[c], mag = fabs(b0[c]);
+                    for (int64_t t = 0; t < 9; ++t) {
+                        const double term = melpad[(2 * r + t / 3) * FP + (2 * s + t % 3)] * w0[t * C + c];
+                        zv += term;
+                        mag += fabs(term);
+                    }
+                    if (fabs(zv) > delta + delta_rel * mag) continue;
                     double dh = 0.0;   /* the transposed conv_dw1 at (r, s) */
                     for (int64_t p = 0; p < 3; ++p)
                         for (int64_t q = 0; q < 3; ++q) {

@@ -171,6 +171,64 @@ def torch_subsample_grads(mel, w0, b0, w1, b1, dout, lengths, causal):
     return g(W0), B0.grad.numpy(), g(W1), B1.grad.numpy()
 
 
+def torch_subsample_kinks(mel, w0, b0, w1, dout, lengths, causal, delta, delta_rel):
+    """Brute-force recount of the kink budget of the subsampler backward, written from its
+    definition with torch float64 tensors: z = b0 + patches @ w0 over melpad's 3x3 stride-2
+    patches (torch's unfold), S = |b0| + |patches| @ |w0|, dh = the gradient of
+    sum(mask4 * conv_dw1(pad(h)) * dout) with respect to h by autograd; a valid h pixel
+    (row < ceil(len/2)) counts when |z| <= delta + delta_rel * S, and the budget sums |dh| (db0)
+    and |dh| |patch tap| (dw0, per tap) over those pixels.  Returns (kdw0 [3,3,C], kdb0 [C])."""
+    mel = torch.tensor(np.asarray(mel, np.float64))
+    B, T, F = mel.shape
+    W0 = torch.tensor(np.asarray(w0, np.float64)).reshape(9, -1)
+    C = W0.shape[1]
+    pt, pb = (2, 0) if causal else (1, 1)
+    Ls = clamp_lengths(lengths, B, T)
+    m0 = (torch.arange(T)[None, :] < torch.tensor(Ls)[:, None]).double()
+    inp = Fnn.pad((mel * m0[:, :, None])[:, None], (1, 1, pt, pb))
+    TP, FP = inp.shape[2], inp.shape[3]
+    T2, F2 = (TP - 3) // 2 + 1, (FP - 3) // 2 + 1
+    patches = Fnn.unfold(inp, kernel_size=3, stride=2)            # [B, 9, T2*F2], tap = 3p + q
+    bb = torch.tensor(np.asarray(b0, np.float64))
+    z = torch.einsum("bkn,kc->bnc", patches, W0) + bb          # [B, T2*F2, C]
+    S = torch.einsum("bkn,kc->bnc", patches.abs(), W0.abs()) + bb.abs()
+    L2 = [(v + 1) // 2 for v in Ls]
+    rows = torch.arange(T2)[:, None].expand(T2, F2).reshape(-1)
+    valid = rows[None, :] < torch.tensor(L2)[:, None]          # [B, T2*F2]
+    hv = torch.zeros(B, C, T2, F2, dtype=torch.float64, requires_grad=True)
+    W1 = torch.tensor(np.asarray(w1, np.float64)).permute(2, 0, 1)[:, None]
+    o = Fnn.conv2d(Fnn.pad(hv, (1, 1, pt, pb)), W1, None, stride=2, groups=C)
+    L4 = [(v + 1) // 2 for v in L2]
+    o = o * (torch.arange(o.shape[2])[None, :] < torch.tensor(L4)[:, None]).double()[:, None, :, None]
+    (o * torch.tensor(np.asarray(dout, np.float64)).permute(0, 3, 1, 2)).sum().backward()
+    dh = hv.grad.permute(0, 2, 3, 1).reshape(B, T2 * F2, C).abs()
+    sel = (valid[:, :, None] & (z.abs() <= delta + delta_rel * S)).double()
+    kdb0 = (sel * dh).sum(dim=(0, 1))
+    kdw0 = torch.einsum("bkn,bnc->kc", patches.abs(), sel * dh)
+    return kdw0.reshape(3, 3, C).numpy(), kdb0.numpy()
+
+
+def subsample_kink_checks(o, rng, B, T, F, C, causal):
+    """The oracle's kink budget against the brute-force recount above, at thresholds that take
+    no pixel, about half of them, and all of them; returns failure strings."""
+    fails = []
+    mel = rng.standard_normal((B, T, F)); w0 = rng.standard_normal((3, 3, C)) / 3
+    b0 = rng.standard_normal(C) * 0.3; w1 = rng.standard_normal((3, 3, C)) / 3
+    L = rng.integers(0, T + 1, size=B).astype(np.int32)
+    L[0] = T
+    T4, F4 = (((T + 1) // 2 + 1) // 2, ((F + 1) // 2 + 1) // 2)
+    dout = rng.standard_normal((B, T4, F4, C))
+    for delta, delta_rel in ((0.0, 0.0), (0.3, 0.0), (0.05, 0.2), (1e300, 0.0)):
+        got = o.dw_subsample_bwd_kinks(mel, w0, b0, w1, dout, L, causal, delta, delta_rel)
+        ref = torch_subsample_kinks(mel, w0, b0, w1, dout, L, causal, delta, delta_rel)
+        for name, gv, rv in zip(("kdw0", "kdb0"), got, ref):
+            if gv.shape != rv.shape or rel_err(gv, rv) > 1e-12:
+                fails.append(f"kink budget {name} {B, T, F, C, causal, delta, delta_rel}")
+        if delta == 0.0 and delta_rel == 0.0 and (np.any(got[0] != 0.0) or np.any(got[1] != 0.0)):
+            fails.append(f"kink budget not exactly 0 without kinks {B, T, F, C, causal}")
+    return fails
+
+
 def subsample_bwd_checks(o, rng, B, T, F, C, causal):
     """The oracle's subsampler backward against float64 autograd, and dw1 / db1 against exact
     finite differences of <dout, out> (out is linear in w1 and b1).  Returns failure strings."""
@@ -382,9 +440,10 @@ def pin_battery(o):
     if rel_err(y, ry) > 1e-12 or not np.array_equal(c, rc):
         fails.append("numpy stream")
 
-    # subsampler backward: autograd and exact finite differences
+    # subsampler backward: autograd and exact finite differences; its kink budget: brute force
     for causal in (False, True):
         fails += subsample_bwd_checks(o, rng, 2, 13, 10, 3, causal)
+        fails += subsample_kink_checks(o, rng, 3, 14, 9, 4, causal)
 
     # general depthwise conv2d: torch autograd, symmetric and causal, strides 1 and 2
     for (KT, KF, stride, pads) in ((3, 3, (2, 2), (1, 1, 1)), (3, 2, (1, 2), (2, 0, 1)), (2, 3, (2, 1), (0, 1, 0))):

@@ -53,6 +53,14 @@ MUTANTS = {
                                    "                    if (i < To) {\n                        acc = bias ? bias[c] : 0.0;"),
     "conv2d dbias unmasked rows": ("            for (int64_t i = 0; i < Lo; ++i)\n                for (int64_t j = 0; j < Fo; ++j) {\n                    const double g = dy[((b * To + i) * Fo + j) * C + c];\n                    gb += g;",
                                    "            for (int64_t i = 0; i < To; ++i)\n                for (int64_t j = 0; j < Fo; ++j) {\n                    const double g = dy[((b * To + i) * Fo + j) * C + c];\n                    gb += g;"),
+    "kink budget sign of z ignored": ("if (fabs(zv) > delta + delta_rel * mag) continue;",
+                                      "if (zv > delta + delta_rel * mag) continue;"),
+    "kink budget row mask off by one": ("for (int64_t r = 0; r < T2 && r < L2; ++r)",
+                                        "for (int64_t r = 0; r < T2 && r <= L2; ++r)"),
+    "kink budget dout mask dropped": ("if (i >= T4 || i >= L4 || j >= F4) continue;",
+                                      "if (i >= T4 || j >= F4) continue;"),
+    "kink budget signed dh": ("kdb0[c] += fabs(dh);", "kdb0[c] += dh;"),
+    "kink budget signed term magnitudes": ("mag += fabs(term);", "mag += term;"),
     "subsample bwd dh taps flipped": ("dhpad[at] += dm * w1[(p * 3 + q) * C + c];",
                                       "dhpad[at] += dm * w1[((2 - p) * 3 + q) * C + c];"),
 }
