@@ -28,6 +28,7 @@ import numpy as np
 __all__ = [
     "bf16_round",
     "f16_round",
+    "dyadic_round",
     "bf16_bits",
     "conv1d_inputs",
     "subsample_inputs",
@@ -101,12 +102,29 @@ def conv1d_inputs(B, T, C, K, *, dtype="bf16", len_range=None, seed=0, with_dy=F
     return out
 
 
-def subsample_inputs(B, T, F, C, *, len_range, seed=3, zero_beyond_len=True):
-    """Inputs of one fused-subsampler workload: ``mel[B,T,F]``, ``w0,w1[3,3,C]``, ``b0,b1[C]``, ``lengths[B]``."""
+def dyadic_round(a: np.ndarray, frac_bits: int) -> np.ndarray:
+    """Round float32 values to the nearest multiple of 2**-frac_bits (ties to even), as float32."""
+    s = np.float32(2.0 ** frac_bits)
+    return (np.rint(np.asarray(a, np.float32) * s) / s).astype(np.float32)
+
+
+def subsample_inputs(B, T, F, C, *, len_range, seed=3, zero_beyond_len=True, dyadic=False):
+    """Inputs of one fused-subsampler workload: ``mel[B,T,F]``, ``w0,w1[3,3,C]``, ``b0,b1[C]``, ``lengths[B]``.
+
+    ``dyadic=True`` rounds the same draws onto coarse binary grids: mel to multiples of 2**-6,
+    w0 to 2**-8 and b0 to 2**-14.  Every mel value and w0 weight then has at most 11
+    significant bits and every product and partial sum of conv0 is a multiple of 2**-14 below
+    2**7 in magnitude, so conv0's output is exactly representable in float32 however its terms
+    are split, ordered or rounded.
+    """
     rng = np.random.default_rng(seed)
     mel = _normal(rng, (B, T, F), 1.0)
     w0 = _normal(rng, (3, 3, C), 1.0 / 9.0)
     b0 = _normal(rng, (C,), 0.1)
+    if dyadic:
+        mel = dyadic_round(np.clip(mel, -7.0, 7.0), 6)
+        w0 = dyadic_round(np.clip(w0, -1.9, 1.9), 8)
+        b0 = dyadic_round(b0, 14)
     w1 = _normal(rng, (3, 3, C), 1.0 / 9.0)
     b1 = _normal(rng, (C,), 0.1)
     lo, hi = len_range
