@@ -147,8 +147,9 @@ size_t dwconv1d_bwd_dw_packed_workspace_size(int64_t B, int64_t N, int64_t C, in
  *   dW[k,c] = sum over sequences b and their frames t of dy[offsets[b]+t, c] xs_b[t + k - pad_left, c]
  *   dbias[c] = sum over the rows of every sequence of dy[n, c]
  * with xs_b = x of sequence b, zero outside it.  float32 partial sums per block go to `workspace`
- * and a second kernel adds them in a fixed order (bitwise reproducible for given sizes).  No
- * atomics.  Rows no sequence covers are ignored.
+ * and a second kernel adds them in a fixed order (bitwise reproducible for given sizes on a
+ * given GPU model: the grid follows the SM count).  No atomics.  Rows no sequence covers are
+ * ignored.
  *
  *  x, dy      [N][C] io_dtype, device;  offsets as dwconv1d_fwd_packed
  *  dw         [K][C] float32, device, overwritten;  dbias [C] float32, or NULL
@@ -201,7 +202,8 @@ size_t dwconv1d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t C, int K);
  *
  * float32 accumulation in a fixed order: per-block partial sums go to `workspace`, then a
  * second kernel adds them in a fixed order.  Results are bitwise reproducible for given
- * sizes, on any run.  No atomics.
+ * sizes on a given GPU model (the grid, and so the order of the sums, follows the SM count).
+ * No atomics.
  *
  *  x, dy     [B][T][C] io_dtype, device
  *  dw        [K][C] float32, device, overwritten
@@ -219,7 +221,8 @@ dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
  * dwconv1d_bwd - the data gradient and the weight/bias gradients of dwconv1d_fwd in one pass
  * that reads dy once (NeMo PR #16114, section "What does this PR do ?", the depthwise kernel's
  * backward).  Results equal dwconv1d_bwd_dx followed by dwconv1d_bwd_dw: dx up to float32
- * summation order, dW/dbias bitwise reproducible for given sizes like dwconv1d_bwd_dw.
+ * summation order, dW/dbias bitwise reproducible for given sizes on a given GPU model, like
+ * dwconv1d_bwd_dw.
  *
  *  x, dy, dx  [B][T][C] io_dtype, device; dx is written in full and must not overlap x or dy
  *  w          [K][C] float32 (the forward taps)
@@ -246,11 +249,12 @@ dw_status_t dwconv1d_bwd(const void *x, const void *dy, const float *w, void *dx
  *  results equal dwconv1d_bwd_dw's up to float32 summation order (the same order whenever
  *  the scratch holds as many partial rows as dwconv1d_bwd_dw_workspace_size would provide).
  *  The first call on a device looks up the scratch's device address (cudaGetSymbolAddress),
- *  so that first call should come before any stream capture.  All calls share the scratch and
+ *  and so does the first call after the device's context has changed (cudaDeviceReset), so
+ *  that first call should come before any stream capture.  All calls share the scratch and
  *  it keeps the last call's contents; calls that overlap on the GPU race on it, so the caller
- *  must serialise them.  Every partial sum read is written by the same call first.  A failed
- *  launch returns DW_ERR_CUDA (dw_last_cuda_error is not updated by this entry point).
- *  Other arguments, results and errors: as dwconv1d_bwd_dw.
+ *  must serialise them.  Every partial sum read is written by the same call first.  Argument
+ *  checks, results and errors are those of dwconv1d_bwd_dw (a failed launch returns
+ *  DW_ERR_CUDA and sets dw_last_cuda_error), plus the scratch limit above.
  */
 dw_status_t dwconv1d_bwd_dw_noalloc(const void *x, const void *dy, float *dw, float *dbias,
                                     const int32_t *lengths, int64_t B, int64_t T, int64_t C, int K,
@@ -280,6 +284,21 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
                              const int32_t *lengths, int32_t *out_lengths, int64_t B,
                              int64_t T, int64_t F, int64_t C, int causal,
                              dw_dtype_t out_dtype, dw_stream_t stream);
+
+/*
+ * dw_subsample_fwd_simt - the same operation, arguments and results as dw_subsample_fwd, computed
+ * entirely on the FP32 FMA pipes: conv0, ReLU, the masks and conv_dw1 as packed float32 FMAs, no
+ * tensor cores, for every size and alignment.  The NeMo PR's kernel runs conv0 as a TF32 dot
+ * (NeMo PR #16114, "What does this PR do ?"); dw_subsample_fwd runs it on the tcgen05 tensor
+ * cores with float32-accurate operand splits whenever the output rows are 16-byte aligned.  This
+ * entry point is the all-FP32 design of the depthwise path: the kernel whose throughput is
+ * stated against the FP32 peak.  Results agree with dw_subsample_fwd within float32 rounding.
+ */
+dw_status_t dw_subsample_fwd_simt(const float *mel, const float *w0, const float *b0,
+                                  const float *w1, const float *b1, void *out,
+                                  const int32_t *lengths, int32_t *out_lengths, int64_t B,
+                                  int64_t T, int64_t F, int64_t C, int causal,
+                                  dw_dtype_t out_dtype, dw_stream_t stream);
 
 /*
  * dw_subsample_bwd_workspace_size - bytes of device workspace dw_subsample_bwd needs for these

@@ -22,7 +22,7 @@ __all__ = [
     "dwconv1d_fwd", "dwconv1d_bwd_dx", "dwconv1d_bwd_dw_workspace_size", "dwconv1d_bwd_dw",
     "dwconv1d_bwd_dw_noalloc", "dwconv1d_bwd", "dwconv1d_stream_fwd", "dwconv1d_fwd_packed",
     "dwconv1d_bwd_dx_packed", "dwconv1d_bwd_dw_packed_workspace_size", "dwconv1d_bwd_dw_packed",
-    "dw_subsample_fwd", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
+    "dw_subsample_fwd", "dw_subsample_fwd_simt", "dw_subsample_bwd_workspace_size", "dw_subsample_bwd", "dw_status_string", "dw_device_error", "subsample_out_shape",
     "dwconv2d_fwd", "dwconv2d_bwd_dx", "dwconv2d_bwd_dw_workspace_size", "dwconv2d_bwd_dw", "conv2d_out_shape",
     "dw_selftest_wait_timeout",
 ]
@@ -57,6 +57,8 @@ SIGNATURES = {
                                       ctypes.c_size_t, _vp]),
     "dw_subsample_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                 _int, _int, _vp]),
+    "dw_subsample_fwd_simt": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                     _int, _int, _vp]),
     "dw_subsample_bwd_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
     "dw_subsample_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int,
                                 _int, _vp, ctypes.c_size_t, _vp]),
@@ -286,17 +288,26 @@ def subsample_out_shape(T, F):
 
 def dw_subsample_fwd(mel, w0, b0, w1, b1, out, lengths, out_lengths, causal, stream=None):
     """Fused conv0 + bias + ReLU + mask + depthwise conv_dw1 + bias + mask into ``out [B,T4,F4,C]``."""
+    _subsample_fwd("dw_subsample_fwd", mel, w0, b0, w1, b1, out, lengths, out_lengths, causal, stream)
+
+
+def dw_subsample_fwd_simt(mel, w0, b0, w1, b1, out, lengths, out_lengths, causal, stream=None):
+    """``dw_subsample_fwd`` computed entirely on the FP32 FMA pipes (no tensor cores)."""
+    _subsample_fwd("dw_subsample_fwd_simt", mel, w0, b0, w1, b1, out, lengths, out_lengths, causal, stream)
+
+
+def _subsample_fwd(name, mel, w0, b0, w1, b1, out, lengths, out_lengths, causal, stream):
     import torch
     B, T, F = mel.shape
     C = w0.shape[-1]
     T4, F4 = subsample_out_shape(T, F)
-    st = lib().dw_subsample_fwd(_dev(mel, "mel", torch.float32), _dev(w0, "w0", torch.float32, (3, 3, C)),
-                                _dev(b0, "b0", torch.float32, (C,)), _dev(w1, "w1", torch.float32, (3, 3, C)),
-                                _dev(b1, "b1", torch.float32, (C,)), _dev(out, "out", None, (B, T4, F4, C)),
-                                _dev(lengths, "lengths", torch.int32, (B,)),
-                                _dev(out_lengths, "out_lengths", torch.int32, (B,)), B, T, F, C,
-                                int(bool(causal)), _dtype_code(out), _stream(stream))
-    _check("dw_subsample_fwd", st)
+    st = getattr(lib(), name)(
+        _dev(mel, "mel", torch.float32), _dev(w0, "w0", torch.float32, (3, 3, C)),
+        _dev(b0, "b0", torch.float32, (C,)), _dev(w1, "w1", torch.float32, (3, 3, C)),
+        _dev(b1, "b1", torch.float32, (C,)), _dev(out, "out", None, (B, T4, F4, C)),
+        _dev(lengths, "lengths", torch.int32, (B,)), _dev(out_lengths, "out_lengths", torch.int32, (B,)),
+        B, T, F, C, int(bool(causal)), _dtype_code(out), _stream(stream))
+    _check(name, st)
 
 
 def dw_subsample_bwd_workspace_size(B, T, F, C):

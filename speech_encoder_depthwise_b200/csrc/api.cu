@@ -5,8 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
-#include "dw_internal.h"
-#include "dwconv.h"
+#include "api_internal.h"
 
 namespace dwk {
 cudaError_t subsample_out_lengths_launch(const int32_t *lengths, int32_t *out_lengths, int64_t B, int64_t T,
@@ -14,14 +13,20 @@ cudaError_t subsample_out_lengths_launch(const int32_t *lengths, int32_t *out_le
 }
 
 namespace {
-
 thread_local int g_last_cuda_error = 0;
+}  // namespace
 
+namespace dwapi {
 dw_status_t cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return DW_OK;
     g_last_cuda_error = static_cast<int>(e);
     return DW_ERR_CUDA;
 }
+}  // namespace dwapi
+
+namespace {
+
+using dwapi::cuda_status;
 
 size_t dtype_size(dw_dtype_t t) { return t == DW_F32 ? 4 : 2; }
 
@@ -122,6 +127,27 @@ dw_status_t packed_common(const void *in, const float *w, void *out, const int32
 }
 
 }  // namespace
+
+namespace dwapi {
+dw_status_t bwd_dw_prepare(const void *x, const void *dy, float *dw, float *dbias, const int32_t *lengths,
+                           int64_t B, int64_t T, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
+                           dwk::DwArgs *a, int64_t *n) {
+    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
+    if (C > kMaxChannels || K > 4096) return DW_ERR_UNSUPPORTED;
+    if (!mul3(B, T, C, n)) return DW_ERR_INVALID_ARG;
+    if (dw == nullptr) return DW_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(K + 1) * C > dwk::kMaxGrid * 256LL) return DW_ERR_INVALID_ARG;
+    if (*n > 0 && (x == nullptr || dy == nullptr)) return DW_ERR_INVALID_ARG;
+    a->x = x; a->dy = dy; a->dw = dw; a->dbias = dbias; a->lengths = lengths;
+    a->B = B; a->T = T; a->C = C; a->K = K; a->pad_left = pad_left;
+    a->dtype = static_cast<int>(io_dtype);
+    a->partials = nullptr;
+    a->G = 0;
+    a->vec_width = *n > 0 ? pick_vec_width(C, dtype_size(io_dtype), {x, dy}, {}) : 1;
+    return DW_OK;
+}
+}  // namespace dwapi
 
 extern "C" {
 
@@ -314,24 +340,16 @@ size_t dwconv1d_bwd_dw_workspace_size(int64_t B, int64_t T, int64_t C, int K) {
     return dwk::conv1d_dw_workspace_bytes(B, T, C, K);
 }
 
+
 dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbias, const int32_t *lengths,
                             int64_t B, int64_t T, int64_t C, int K, int pad_left, dw_dtype_t io_dtype,
                             void *workspace, size_t workspace_bytes, dw_stream_t stream) {
-    if (!valid_dtype(io_dtype)) return DW_ERR_INVALID_ARG;
-    if (B < 0 || T < 0 || C < 1 || K < 1 || pad_left < 0 || pad_left > K - 1) return DW_ERR_INVALID_ARG;
-    int64_t n = 0;
-    if (!mul3(B, T, C, &n)) return DW_ERR_INVALID_ARG;
-    if (dw == nullptr) return DW_ERR_INVALID_ARG;
-    if (static_cast<int64_t>(K + 1) * C > dwk::kMaxGrid * 256LL) return DW_ERR_INVALID_ARG;
     dwk::DwArgs a;
-    a.x = x; a.dy = dy; a.dw = dw; a.dbias = dbias; a.lengths = lengths;
-    a.B = B; a.T = T; a.C = C; a.K = K; a.pad_left = pad_left;
-    a.dtype = static_cast<int>(io_dtype);
+    int64_t n = 0;
+    const dw_status_t st = dwapi::bwd_dw_prepare(x, dy, dw, dbias, lengths, B, T, C, K, pad_left, io_dtype, &a, &n);
+    if (st != DW_OK) return st;
     a.partials = static_cast<float *>(workspace);
-    a.G = 0;
-    a.vec_width = 1;
     if (n > 0) {
-        if (x == nullptr || dy == nullptr) return DW_ERR_INVALID_ARG;
         const size_t need = dwk::conv1d_dw_workspace_bytes(B, T, C, K);
         if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)) return DW_ERR_WORKSPACE;
         const size_t out_bytes = static_cast<size_t>(K) * C * sizeof(float);
@@ -339,7 +357,6 @@ dw_status_t dwconv1d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
             (dbias && overlaps(workspace, need, dbias, static_cast<size_t>(C) * sizeof(float))))
             return DW_ERR_INVALID_ARG;
         a.G = dwk::conv1d_dw_partial_rows(B, T, C, K);
-        a.vec_width = pick_vec_width(C, dtype_size(io_dtype), {x, dy}, {});
     }
     return cuda_status(dwk::conv1d_dw_launch(a, static_cast<cudaStream_t>(stream)));
 }
@@ -461,10 +478,11 @@ dw_status_t dwconv2d_bwd_dw(const void *x, const void *dy, float *dw, float *dbi
     return cuda_status(dwk::conv2d_dw_launch(a, dw, dbias, partials, static_cast<cudaStream_t>(stream)));
 }
 
-dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0, const float *w1,
-                             const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
-                             int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,
-                             dw_stream_t stream) {
+namespace {
+
+dw_status_t subsample_fwd(const float *mel, const float *w0, const float *b0, const float *w1, const float *b1,
+                          void *out, const int32_t *lengths, int32_t *out_lengths, int64_t B, int64_t T, int64_t F,
+                          int64_t C, int causal, dw_dtype_t out_dtype, bool tensor_cores, cudaStream_t s) {
     if (!valid_dtype(out_dtype)) return DW_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || F < 1 || C < 1 || (causal != 0 && causal != 1)) return DW_ERR_INVALID_ARG;
     int64_t n = 0;
@@ -479,17 +497,34 @@ dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0,
         if (overlaps(mel, static_cast<size_t>(n) * 4, out, static_cast<size_t>(nout) * dtype_size(out_dtype)))
             return DW_ERR_INVALID_ARG;
     }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (nout > 0) {  // the fused kernel also writes out_lengths
         dwk::SubsampleArgs a;
         a.mel = mel; a.w0 = w0; a.b0 = b0; a.w1 = w1; a.b1 = b1; a.out = out;
         a.lengths = lengths; a.out_lengths = out_lengths;
         a.B = B; a.T = T; a.F = F; a.C = C; a.causal = causal; a.out_dtype = static_cast<int>(out_dtype);
-        return cuda_status(dwk::subsample_launch(a, s));
+        return cuda_status(dwk::subsample_launch(a, tensor_cores, s));
     }
     if (out_lengths != nullptr && B > 0)  // no frames: only the (zero) output lengths
         return cuda_status(dwk::subsample_out_lengths_launch(lengths, out_lengths, B, T, s));
     return DW_OK;
+}
+
+}  // namespace
+
+dw_status_t dw_subsample_fwd(const float *mel, const float *w0, const float *b0, const float *w1,
+                             const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
+                             int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,
+                             dw_stream_t stream) {
+    return subsample_fwd(mel, w0, b0, w1, b1, out, lengths, out_lengths, B, T, F, C, causal, out_dtype, true,
+                         static_cast<cudaStream_t>(stream));
+}
+
+dw_status_t dw_subsample_fwd_simt(const float *mel, const float *w0, const float *b0, const float *w1,
+                                  const float *b1, void *out, const int32_t *lengths, int32_t *out_lengths,
+                                  int64_t B, int64_t T, int64_t F, int64_t C, int causal, dw_dtype_t out_dtype,
+                                  dw_stream_t stream) {
+    return subsample_fwd(mel, w0, b0, w1, b1, out, lengths, out_lengths, B, T, F, C, causal, out_dtype, false,
+                         static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -122,7 +122,8 @@ unsigned int conv1d_dw_take_error();
 
 cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s);
 
-cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s);
+// tensor_cores: the tcgen05 kernel where eligible; false keeps every size on the FP32 SIMT kernel.
+cudaError_t subsample_launch(const SubsampleArgs &a, bool tensor_cores, cudaStream_t s);
 
 cudaError_t conv2d_fwd_launch(const Conv2dArgs &a, cudaStream_t s);
 cudaError_t conv2d_dx_launch(const Conv2dArgs &a, cudaStream_t s);

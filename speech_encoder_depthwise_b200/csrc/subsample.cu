@@ -345,12 +345,12 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
     }
 }
 
-cudaError_t subsample_launch(const SubsampleArgs &a, cudaStream_t s) {
+cudaError_t subsample_launch(const SubsampleArgs &a, bool tensor_cores, cudaStream_t s) {
     const int Pt = a.causal ? 2 : 1;
     auto s2 = [](int64_t n) -> int64_t { return n >= 1 ? (n - 1) / 2 + 1 : 0; };
     const int64_t T2 = s2(a.T), F2 = s2(a.F), T4 = s2(T2), F4 = s2(F2);
     if (a.B == 0 || T4 == 0) return cudaSuccess;
-    if (subsample_tc_eligible(a)) {
+    if (tensor_cores && subsample_tc_eligible(a)) {
         const cudaError_t e = subsample_tc_launch(a, s);
         if (e != cudaErrorNotSupported) return e;
     }

@@ -164,8 +164,9 @@ def test_dw_workspace_rules(lib):
     assert f(*args[:9], 9, dw.DW_BF16, FAKE_WS, n, None) == dw.DW_ERR_INVALID_ARG
 
 
-def test_subsample_rejects_invalid_arguments(lib):
-    f = lib.dw_subsample_fwd
+@pytest.mark.parametrize("entry", ["dw_subsample_fwd", "dw_subsample_fwd_simt"])
+def test_subsample_rejects_invalid_arguments(lib, entry):
+    f = getattr(lib, entry)
     ok = [FAKE_X, FAKE_W, FAKE_W + 4096, FAKE_W + 8192, FAKE_W + 12288, FAKE_Y, None, None,
           2, 40, 16, 8, 0, dw.DW_BF16, None]
 

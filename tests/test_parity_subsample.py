@@ -7,6 +7,10 @@ Small cases: T and F from 1 up (odd and even), C not a multiple of 64 (1, 3, 100
 C up to 512 (several channel tiles), F up to 200 (several 20-column blocks),
 float32 output, len 0 and len T, unaligned output (narrow store path), guard bands.
 
+Both entry points are checked at full size: dw_subsample_fwd (conv0 on the tensor cores where
+the output rows are 16-byte aligned) and dw_subsample_fwd_simt (every step on the FP32 pipes);
+the small cases also run dw_subsample_fwd_simt on shapes the tensor-core kernel would take.
+
 Bars: bf16 output max|err| <= 2e-2 absolute; float32 output max|err| <= 1e-5 * RMS(oracle);
 masked rows exactly +0.0; out_lengths bit-exact.
 """
@@ -29,15 +33,16 @@ def _lib(cuda_device):
     dw.lib()
 
 
-def gpu_subsample(d, causal, out_dtype=torch.bfloat16, offset=0, with_lengths=True):
+def gpu_subsample(d, causal, out_dtype=torch.bfloat16, offset=0, with_lengths=True, simt=False):
     mel = dev(d["mel"])
     B, T, F = mel.shape
     C = d["w0"].shape[-1]
     T4, F4 = dw.subsample_out_shape(T, F)
     out = Guarded((B, T4, F4, C), out_dtype, offset=offset)
     ol = torch.full((B,), -7, dtype=torch.int32, device="cuda")
-    dw.dw_subsample_fwd(mel, dev(d["w0"]), dev(d["b0"]), dev(d["w1"]), dev(d["b1"]), out.t,
-                        dev(d["lengths"]) if with_lengths else None, ol, causal)
+    fn = dw.dw_subsample_fwd_simt if simt else dw.dw_subsample_fwd
+    fn(mel, dev(d["w0"]), dev(d["b0"]), dev(d["w1"]), dev(d["b1"]), out.t,
+       dev(d["lengths"]) if with_lengths else None, ol, causal)
     torch.cuda.synchronize()
     out.check_slack()
     return out.numpy(), ol.cpu().numpy()
@@ -49,11 +54,13 @@ def check_masked_rows(got, out_lengths):
         assert np.all(tail == 0.0) and not np.any(np.signbit(tail))
 
 
+@pytest.mark.parametrize("simt", [False, True])
 @pytest.mark.parametrize("causal", [False, True])
-def test_subsampler_full_workload(causal):
+def test_subsampler_full_workload(causal, simt):
+    """Both entry points: dw_subsample_fwd (tensor-core conv0) and dw_subsample_fwd_simt (all FP32)."""
     d = subsample_inputs(16, 3000, 80, 256, len_range=(1500, 3000), seed=3)
     ref, rl = oracle.dw_subsample_fwd(d["mel"], d["w0"], d["b0"], d["w1"], d["b1"], d["lengths"], causal)
-    got, gl = gpu_subsample(d, causal)
+    got, gl = gpu_subsample(d, causal, simt=simt)
     assert got.shape == ref.shape == (16, 750, 20, 256)
     assert_bf16_close(got, ref)
     np.testing.assert_array_equal(gl, rl)
@@ -84,6 +91,19 @@ def test_subsampler_small_cases(B, T, F, C, causal, out_dtype):
         assert_bf16_close(got, ref)
     np.testing.assert_array_equal(gl, rl)
     check_masked_rows(got, gl)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,T,F,C", [(2, 45, 200, 384), (1, 70, 80, 512), (2, 23, 3, 32), (2, 64, 80, 256)])
+def test_subsampler_simt_entry_on_aligned_shapes(B, T, F, C, causal):
+    d = subsample_inputs(B, T, F, C, len_range=(0, T), seed=T * 100 + F + C)
+    d["lengths"][0] = T
+    ref, rl = oracle.dw_subsample_fwd(d["mel"], d["w0"], d["b0"], d["w1"], d["b1"], d["lengths"], causal)
+    for td, close in ((torch.float32, assert_f32_close), (torch.bfloat16, assert_bf16_close)):
+        got, gl = gpu_subsample(d, causal, out_dtype=td, simt=True)
+        close(got, ref)
+        np.testing.assert_array_equal(gl, rl)
+        check_masked_rows(got, gl)
 
 
 def test_subsampler_unaligned_output_and_no_lengths():
