@@ -11,7 +11,7 @@
 // Channels-last, so a thread owns V consecutive channels (one 8- or 16-byte vector) of one output
 // row and walks its columns; every access of a warp is 32 consecutive vectors.  The weight
 // gradient keeps per-thread partial sums over a persistent share of the rows, writes one partial
-// row per block and adds the rows in a fixed order (reproducible for given sizes, no atomics).
+// row per block and adds the rows in a fixed order (reproducible for given sizes on a given GPU model, no atomics).
 #include "dw_internal.h"
 
 namespace dwk {
