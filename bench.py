@@ -49,8 +49,10 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--next-rows", default="all",
-                   help="comma list of the NEXT-row measurements after the step (stream, bwd, conv2d, "
-                        "f16_packed, sub_bwd, batch), 'all' or 'none'")
+                   help="comma list of the measurements after the step: the other workloads (sweep: causal "
+                        "kernel-width sweep; sub: subsampler symmetric/causal, tensor-core and FP32 kernels; bwd: "
+                        "training-size dX, dW and one-pass backward) and the NEXT rows (stream, conv2d, "
+                        "f16_packed, sub_bwd, batch); 'all' or 'none'")
     return p.parse_args()
 
 
@@ -95,6 +97,27 @@ def max_over_ranks(value, world, device="cpu"):
 def job_throughput(step_bytes_per_rank, ms_per_step, world):
     """Whole-job GB/s: every rank processes its own batch (weak scaling) in the slowest rank's time."""
     return world * step_bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
+# ------------------------------------------------------------------ errors against the parity bars
+def bf16_err_over_bar(got, ref):
+    """max over elements of |gpu - oracle| / bar with the bf16 I/O bar the parity tests apply element
+    by element: bar = max(2e-2, one bf16 ulp of the oracle value) (where |y| >= 4 the bf16 spacing
+    exceeds 2e-2, so the bar there is one unit of the output precision).  <= 1 passes."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    _, e = np.frexp(np.maximum(np.abs(ref), 2.0 ** -126))
+    bar = np.maximum(2e-2, np.ldexp(1.0, e - 8))
+    return float(np.max(np.abs(got - ref) / bar)) if ref.size else 0.0
+
+
+def dw_err_over_bar(got, ref):
+    """|gpu - oracle| / bar for float32 weight gradients from bf16 inputs: the tests hold the max error
+    to both 2e-2 absolute and 1e-5 * RMS(oracle), so bar = the smaller of the two.  <= 1 passes."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    bar = min(2e-2, 1e-5 * float(np.sqrt(np.mean(ref * ref))))
+    return float(np.max(np.abs(got - ref)) / max(bar, 1e-30))
 
 
 # ------------------------------------------------------------------ clocks (NVML, read only)
@@ -204,10 +227,11 @@ BWD = dict(B=32, T=1500, C=1024, K=9, pad_left=4, len_range=(750, 1500), seed=4)
 
 
 def measure_bwd(dw, dev, hbm):
-    """One-pass backward (a NEXT row, outside the step) on the training-size backward workload,
-    32x1500x1024 bf16, K=9: dwconv1d_bwd against dwconv1d_bwd_dx + dwconv1d_bwd_dw, each over 3
-    rotating input sets captured in a CUDA graph.  Algorithmic bytes: x and dy at valid frames,
-    dx written in full."""
+    """The training-size backward workload, 32x1500x1024 bf16, K=9, sym 4|4, len U[750,1500]:
+    the data gradient (dwconv1d_bwd_dx) and the weight/bias gradients (dwconv1d_bwd_dw) as rows of
+    their own, and the one-pass dwconv1d_bwd (a NEXT row), each over 3 rotating input sets
+    captured in a CUDA graph.  Algorithmic bytes: dX = dy at valid frames + dx in full; dW = x and
+    dy at valid frames; one pass = x and dy at valid frames + dx in full."""
     import torch
     import oracle
     from synth import conv1d_inputs
@@ -222,41 +246,37 @@ def measure_bwd(dw, dev, hbm):
     gw, gb = torch.empty(K, C, device=dev), torch.empty(C, device=dev)
     ws = torch.empty(dw.dwconv1d_bwd_dw_workspace_size(B, T, C, K), dtype=torch.uint8, device=dev)
     valid = int(np.clip(d["lengths"], 0, T).sum()) * C
-    by = (2 * valid + B * T * C) * 2
-    s = torch.cuda.Stream(dev)
-
-    def timed(fn):
-        with torch.cuda.stream(s):
-            for i in range(3):
-                fn(i)
-            g = torch.cuda.CUDAGraph()
-            g.capture_begin()
-            for i in range(3):
-                fn(i)
-            g.capture_end()
-            for _ in range(3):
-                g.replay()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(s)
-            for _ in range(20):
-                g.replay()
-            e1.record(s)
-        torch.cuda.synchronize(dev)
-        del g
-        return e0.elapsed_time(e1) / 60 * 1e3
-
-    fused = timed(lambda i: dw.dwconv1d_bwd(xs[i], gs[i], w, dxs[i], gw, gb, ln, pl, ws))
-    sep = timed(lambda i: (dw.dwconv1d_bwd_dx(gs[i], w, dxs[i], ln, pl),
-                           dw.dwconv1d_bwd_dw(xs[i], gs[i], gw, gb, ln, pl, ws)))
-    with torch.cuda.stream(s):
-        dw.dwconv1d_bwd(xs[0], gs[0], w, dxs[0], gw, gb, ln, pl, ws)
+    by_dx = (valid + B * T * C) * 2 + K * C * 4 + B * 4
+    by_dw = 2 * valid * 2 + (K + 1) * C * 4 + B * 4
+    by_one = (2 * valid + B * T * C) * 2
+    fl = 2 * K * valid
+    t_dx = graph_us(dev, [lambda i=i: dw.dwconv1d_bwd_dx(gs[i], w, dxs[i], ln, pl) for i in range(3)])
+    t_dw = graph_us(dev, [lambda i=i: dw.dwconv1d_bwd_dw(xs[i], gs[i], gw, gb, ln, pl, ws) for i in range(3)])
+    t_one = graph_us(dev, [lambda i=i: dw.dwconv1d_bwd(xs[i], gs[i], w, dxs[i], gw, gb, ln, pl, ws)
+                           for i in range(3)])
+    # errors against the oracle: dX on items 0-1, dW/dbias over the whole batch
+    dw.dwconv1d_bwd_dx(gs[0], w, dxs[0], ln, pl)
+    dw.dwconv1d_bwd_dw(xs[0], gs[0], gw, gb, ln, pl, ws)
     torch.cuda.synchronize(dev)
-    ref = oracle.dwconv1d_bwd_dx(d["dy"][:1], d["w"], d["lengths"][:1], pl)
-    err = float(np.max(np.abs(dxs[0][:1].float().cpu().numpy() - ref)))
-    return {"workload": f"one-pass dX + dW/dbias, {B}x{T}x{C} bf16, K={K}, sym 4|4, len U[750,1500] "
+    rdx = oracle.dwconv1d_bwd_dx(d["dy"][:2], d["w"], d["lengths"][:2], pl)
+    gdx = dxs[0][:2].float().cpu().numpy()
+    rdw, rdb = oracle.dwconv1d_bwd_dw(d["x"], d["dy"], K, d["lengths"], pl)
+    gdw, gdb = gw.cpu().numpy(), gb.cpu().numpy()
+
+    def row(us, by, flops):
+        return {"us": us, "GB_per_s": by / us / 1e3, "frames_per_s": B * T / (us * 1e-6),
+                "hbm_frac_of_measured": by / us / 1e3 / hbm, "hbm_frac_of_8TBps": by / us / 1e3 / 8000.0,
+                "alg_bytes": by, "alg_flops": flops}
+    rdx_row = row(t_dx, by_dx, fl)
+    rdx_row.update(max_abs_err=float(np.max(np.abs(gdx - rdx))), err_over_bar=bf16_err_over_bar(gdx, rdx))
+    rdw_row = row(t_dw, by_dw, fl + valid)
+    rdw_row.update(max_abs_err=max(float(np.max(np.abs(gdw - rdw))), float(np.max(np.abs(gdb - rdb)))),
+                   err_over_bar=max(dw_err_over_bar(gdw, rdw), dw_err_over_bar(gdb, rdb)))
+    one = row(t_one, by_one, 2 * fl + valid)
+    one["dx_plus_dw_as_two_launches_us"] = t_dx + t_dw
+    return {"workload": f"conv1d backward {B}x{T}x{C} bf16, K={K}, sym 4|4, len U[750,1500] "
                         "(3 rotating input sets in a CUDA graph)",
-            "us": fused, "GB_per_s": by / fused / 1e3, "hbm_frac_of_measured": by / fused / 1e3 / hbm,
-            "alg_bytes": by, "separate_dx_plus_dw_us": sep, "dx_max_abs_err_item0": err}
+            "dwconv1d_bwd_dx": rdx_row, "dwconv1d_bwd_dw": rdw_row, "dwconv1d_bwd_one_pass": one}
 
 
 def measure_sub_bwd(dw, dev, hbm, fp32_tflops):
@@ -400,6 +420,94 @@ def measure_batch_scaling(dw, dev, hbm):
         del xs, gs, ys, srcs, dsts
     return {"workload": f"conformer dwconv1d {T}x{C}, K={K}, bf16, len U[750,1500], B in 16/32/64 "
                         "(3 rotating input sets in a CUDA graph)", **res}
+
+
+SWEEP = dict(B=32, T=750, C=1024, Ks=(3, 4, 5, 9, 15), odd=(520, 7), len_range=(375, 750), seed=2)
+
+
+def measure_causal_sweep(dw, dev, hbm, fp32_tflops):
+    """The causal kernel-width sweep: dwconv1d_fwd on x[32, 750, 1024] bf16 with K in {3,4,5,9,15},
+    left padding K-1, lengths U[375,750], plus C=520, K=7 (channels not a multiple of 128); each over
+    3 rotating input sets in a CUDA graph.  Algorithmic bytes: x at valid frames + y in full;
+    flops 2K per valid output.  The roofline time is the larger of bytes / HBM and flops / FP32
+    peak (K=15 comes near the balance); the max error is taken on items 0-1."""
+    import torch
+    import oracle
+    from synth import conv1d_inputs
+    c = SWEEP
+    B, T = c["B"], c["T"]
+    res = {}
+    for C, K in [(c["C"], k) for k in c["Ks"]] + [c["odd"]]:
+        d = conv1d_inputs(B, T, C, K, dtype="bf16", len_range=c["len_range"], seed=c["seed"])
+        xs = [torch.from_numpy(d["x"]).to(dev, torch.bfloat16) for _ in range(3)]
+        ys = [torch.empty_like(xs[0]) for _ in range(3)]
+        w, bias, ln = (torch.from_numpy(d["w"]).to(dev), torch.from_numpy(d["bias"]).to(dev),
+                       torch.from_numpy(d["lengths"]).to(dev))
+        us = graph_us(dev, [lambda i=i: dw.dwconv1d_fwd(xs[i], w, bias, ys[i], ln, K - 1) for i in range(3)])
+        valid = int(np.clip(d["lengths"], 0, T).sum())
+        by = (valid + B * T) * C * 2 + (K + 1) * C * 4 + B * 4
+        fl = 2 * K * valid * C
+        t_roof = max(by / (hbm * 1e3), fl / (fp32_tflops * 1e6))  # µs
+        dw.dwconv1d_fwd(xs[0], w, bias, ys[0], ln, K - 1)
+        torch.cuda.synchronize(dev)
+        got = ys[0][:2].float().cpu().numpy()
+        ref = oracle.dwconv1d_fwd(d["x"][:2], d["w"], d["bias"], d["lengths"][:2], K - 1)
+        res[f"C{C}_K{K}"] = {"us": us, "GB_per_s": by / us / 1e3, "frames_per_s": B * T / (us * 1e-6),
+                             "hbm_frac_of_measured": by / us / 1e3 / hbm, "hbm_frac_of_8TBps": by / us / 1e3 / 8000.0,
+                             "alu_frac": fl / us / 1e6 / fp32_tflops, "roofline_frac": t_roof / us,
+                             "alg_bytes": by, "alg_flops": fl, "max_abs_err": float(np.max(np.abs(got - ref))),
+                             "err_over_bar": bf16_err_over_bar(got, ref)}
+        del xs, ys
+    return {"workload": f"causal dwconv1d forward {B}x{T}x1024 bf16, K in {c['Ks']}, pads (K-1)|0, "
+                        "len U[375,750]; plus C=520, K=7 (3 rotating input sets in a CUDA graph)", **res}
+
+
+def measure_subsamplers(dw, dev, hbm, fp32_tflops):
+    """The fused subsampler on mel[16, 3000, 80] -> [16, 750, 20, 256] bf16, len U[1500,3000]:
+    symmetric and causal (time pad 2|0), through dw_subsample_fwd (conv0 on the tcgen05 tensor
+    cores, the default) and dw_subsample_fwd_simt (every step on the FP32 pipes), each over 3
+    rotating mel sets in a CUDA graph.  Algorithmic bytes: mel at valid frames + out in full;
+    flops 18 per valid h element + 18 per valid output element.  fp32_frac is the roofline the
+    depthwise path is stated against (the larger of bytes / HBM and flops / FP32 peak); for the
+    tensor-core kernel, whose conv0 does not run on the FP32 pipes, the HBM fraction is the binding
+    one.  The max error is taken on items 0-1."""
+    import torch
+    import oracle
+    from synth import subsample_inputs
+    B, T, F, C = SUB["B"], SUB["T"], SUB["F"], SUB["C"]
+    ss = subsample_inputs(B, T, F, C, len_range=SUB["len_range"], seed=SUB["seed"])
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    mels = [t(ss["mel"]) for _ in range(3)]
+    w0, b0, w1, b1, ln = t(ss["w0"]), t(ss["b0"]), t(ss["w1"]), t(ss["b1"]), t(ss["lengths"], torch.int32)
+    T4, F4 = dw.subsample_out_shape(T, F)
+    outs = [torch.empty(B, T4, F4, C, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    ol = torch.empty(B, dtype=torch.int32, device=dev)
+    by, fl, _, _ = sub_work(ss["lengths"], T, F, C)
+    res = {}
+    for causal in (0, 1):
+        ref, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"], ss["lengths"][:2],
+                                         causal)
+        for name, fn in (("tc", dw.dw_subsample_fwd), ("fp32_simt", dw.dw_subsample_fwd_simt)):
+            us = graph_us(dev, [lambda i=i: fn(mels[i], w0, b0, w1, b1, outs[i], ln, ol, causal) for i in range(3)])
+            fn(mels[0], w0, b0, w1, b1, outs[0], ln, ol, causal)
+            torch.cuda.synchronize(dev)
+            got = outs[0][:2].float().cpu().numpy()
+            t_fp32 = fl / (fp32_tflops * 1e6)
+            t_hbm = by / (hbm * 1e3)
+            r = {"us": us, "ms": us * 1e-3, "TFLOP_per_s": fl / us / 1e6, "fp32_frac": max(t_fp32, t_hbm) / us,
+                 "hbm_frac_of_measured": t_hbm / us, "GB_per_s": by / us / 1e3,
+                 "frames_per_s": B * T4 / (us * 1e-6), "alg_bytes": by, "alg_flops": fl,
+                 "max_abs_err": float(np.max(np.abs(got - ref))), "err_over_bar": bf16_err_over_bar(got, ref)}
+            if name == "tc":
+                r["kernel"] = "dw_subsample_tc_kernel (conv0 on tcgen05, TF32 3-product split; ReLU, conv_dw1 on FP32)"
+                r["roofline"] = "hbm"
+            else:
+                r["kernel"] = "dw_subsample_kernel (conv0, ReLU, conv_dw1 all packed FP32 FMA)"
+                r["roofline"] = "fp32" if t_fp32 >= t_hbm else "hbm"
+            res[f"{'causal' if causal else 'sym'}_{name}"] = r
+    del mels, outs
+    return {"workload": f"fused subsampler mel {B}x{T}x{F} fp32 -> {B}x{T4}x{F4}x{C} bf16, len U[1500,3000], "
+                        "symmetric 1|1 and causal 2|0 (3 rotating mel sets in a CUDA graph)", **res}
 
 
 CONV2D = dict(B=16, T=750, F=20, C=256, KT=3, KF=3, stride=(2, 2), pads=(1, 1, 1), len_range=(375, 750), seed=5)
@@ -603,6 +711,33 @@ def reference_arm(args, world, rank):
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def summary_table(line):
+    """One compact string per kernel row (µs, roofline fraction, error / parity bar), placed last in
+    the JSON line so that a reader of its tail sees every configuration."""
+    out = {}
+
+    def put(key, r, frac_key="hbm_frac_of_measured"):
+        if r:
+            out[key] = f"{r['us']:.1f}us {frac_key.split('_of')[0].replace('_frac', '')} {r[frac_key]:.2f}" + \
+                (f" err/bar {r['err_over_bar']:.2f}" if "err_over_bar" in r else "")
+    rows = line["rows"]
+    put("cfg2_fwd", rows.get("dwconv1d_fwd"))
+    put("cfg2_dx", rows.get("dwconv1d_bwd_dx"))
+    put("cfg2_dw", rows.get("dwconv1d_bwd_dw"))
+    cf = line.get("configs", {})
+    for k, r in cf.get("causal_kernel_width_sweep", {}).items():
+        if isinstance(r, dict):
+            put(f"cfg3_{k}", r, "roofline_frac")
+    for k, r in cf.get("subsampler", {}).items():
+        if isinstance(r, dict):
+            put(f"cfg4_{k}", r, "fp32_frac" if "simt" in k else "hbm_frac_of_measured")
+    tb = cf.get("training_backward", {})
+    put("cfg5_dx", tb.get("dwconv1d_bwd_dx"))
+    put("cfg5_dw", tb.get("dwconv1d_bwd_dw"))
+    put("cfg5_one_pass", tb.get("dwconv1d_bwd_one_pass"))
+    return out
 
 
 # ------------------------------------------------------------------ our arm
@@ -851,9 +986,11 @@ def main():
                         "hbm_frac_of_8TBps": by / (ms * 1e-3) / 1e9 / 8000.0,
                         "alg_bytes": by, "alg_flops": fl}
         ms = row_ms["dw_subsample_fwd"]
-        row["dw_subsample_fwd"] = {"ms": ms, "us": ms * 1e3, "eager_us": row_eager_ms["dw_subsample_fwd"] * 1e3,
+        row["dw_subsample_fwd"] = {"kernel": "dw_subsample_tc_kernel (conv0 on tcgen05)",
+                                   "ms": ms, "us": ms * 1e3, "eager_us": row_eager_ms["dw_subsample_fwd"] * 1e3,
                                    "TFLOP_per_s": sf / (ms * 1e-3) / 1e12,
-                                   "fp32_frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
+                                   "hbm_frac_of_measured": sb / (ms * 1e-3) / 1e9 / hbm,
+                                   "fp32_term_frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
                                    "GB_per_s": sb / (ms * 1e-3) / 1e9,
                                    "frames_per_s": SB * T4 / (ms * 1e-3),
                                    "alg_bytes": sb, "alg_flops": sf}
@@ -862,30 +999,45 @@ def main():
         f64 = lambda tt: tt.float().cpu().numpy().astype(np.float64)
         s0 = sets[0]
         err = lambda a, b: float(np.max(np.abs(a - b)))
-        row["dwconv1d_fwd"]["max_abs_err"] = err(f64(s0["y"][:2]), oracle.dwconv1d_fwd(
-            cs["x"][:2], cs["w"], cs["bias"], cs["lengths"][:2], pl))
-        row["dwconv1d_bwd_dx"]["max_abs_err"] = err(f64(s0["dx"][:2]), oracle.dwconv1d_bwd_dx(
-            cs["dy"][:2], cs["w"], cs["lengths"][:2], pl))
+        ry = oracle.dwconv1d_fwd(cs["x"][:2], cs["w"], cs["bias"], cs["lengths"][:2], pl)
+        row["dwconv1d_fwd"]["max_abs_err"] = err(f64(s0["y"][:2]), ry)
+        row["dwconv1d_fwd"]["err_over_bar"] = bf16_err_over_bar(f64(s0["y"][:2]), ry)
+        rdx = oracle.dwconv1d_bwd_dx(cs["dy"][:2], cs["w"], cs["lengths"][:2], pl)
+        row["dwconv1d_bwd_dx"]["max_abs_err"] = err(f64(s0["dx"][:2]), rdx)
+        row["dwconv1d_bwd_dx"]["err_over_bar"] = bf16_err_over_bar(f64(s0["dx"][:2]), rdx)
         rdw, rdb = oracle.dwconv1d_bwd_dw(cs["x"], cs["dy"], K, cs["lengths"], pl)
         row["dwconv1d_bwd_dw"]["max_abs_err"] = max(err(f64(gw), rdw), err(f64(gb), rdb))
+        row["dwconv1d_bwd_dw"]["err_over_bar"] = max(dw_err_over_bar(f64(gw), rdw), dw_err_over_bar(f64(gb), rdb))
         ro, _ = oracle.dw_subsample_fwd(ss["mel"][:2], ss["w0"], ss["b0"], ss["w1"], ss["b1"],
                                         ss["lengths"][:2], SUB["causal"])
         row["dw_subsample_fwd"]["max_abs_err"] = err(f64(s0["out"][:2]), ro)
-        want = {"stream", "bwd", "conv2d", "f16_packed", "sub_bwd", "batch"} if args.next_rows == "all" else \
-            set() if args.next_rows == "none" else set(args.next_rows.split(","))
+        row["dw_subsample_fwd"]["err_over_bar"] = bf16_err_over_bar(f64(s0["out"][:2]), ro)
+        want = {"sweep", "sub", "bwd", "stream", "conv2d", "f16_packed", "sub_bwd", "batch"} \
+            if args.next_rows == "all" else set() if args.next_rows == "none" else set(args.next_rows.split(","))
+        cfg_measures = [("sweep", "causal_kernel_width_sweep", lambda: measure_causal_sweep(dw, dev, hbm, fp32_tflops)),
+                        ("sub", "subsampler", lambda: measure_subsamplers(dw, dev, hbm, fp32_tflops)),
+                        ("bwd", "training_backward", lambda: measure_bwd(dw, dev, hbm))]
         measures = [("stream", "dwconv1d_stream_fwd", lambda: measure_stream(dw, dev, hbm)),
-                    ("bwd", "dwconv1d_bwd", lambda: measure_bwd(dw, dev, hbm)),
                     ("conv2d", "dwconv2d", lambda: measure_conv2d(dw, dev, hbm)),
                     ("f16_packed", "f16_and_packed", lambda: measure_f16_packed(dw, dev, hbm)),
                     ("sub_bwd", "dw_subsample_bwd", lambda: measure_sub_bwd(dw, dev, hbm, fp32_tflops)),
                     ("batch", "conv1d_batch_scaling", lambda: measure_batch_scaling(dw, dev, hbm))]
-        next_rows = {name: fn() for key, name, fn in measures if key in want}
+        with ClockSampler(local) as clk_rows:
+            configs = {name: fn() for key, name, fn in cfg_measures if key in want}
+            next_rows = {name: fn() for key, name, fn in measures if key in want}
         cpu = None
         if world == 1 and args.cpu_seconds > 0:
             v, desc, cores, _ = cpu_rate(cs, ss, args.cpu_seconds)
             cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc,
                    "single_thread_cfg1": cpu_single_thread_cfg1_ms()}
         clocks = clk.summary()
+        if clk_rows.samples:  # the timed steps are ~2 ms: add the samples of the per-config replays
+            clocks = dict(clocks, window="timed steps and the per-config graph replays after them",
+                          sm_mhz=float(np.median(clk.samples + clk_rows.samples)),
+                          reasons=sorted(set(clocks["reasons"]) | clk_rows.reasons),
+                          samples=len(clk.samples) + len(clk_rows.samples))
+        simt = configs.get("subsampler", {}).get("sym_fp32_simt")
+        tc_us = ms * 1e3
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -894,24 +1046,29 @@ def main():
                        "parallelism": f"replicas x{world} (independent batches, no collective)",
                        "l2": f"{N_SETS} rotating input sets of ~237 MB each (> L2 126 MB)"},
             "frames_per_s": world * B * T / (row_ms["dwconv1d_fwd"] * 1e-3),
-            "subsampler_ms": row_ms["dw_subsample_fwd"],
-            "subsampler_roofline_frac": row["dw_subsample_fwd"]["fp32_frac"],
+            # the depthwise subsampler metric on the all-FP32 kernel (its roofline: max(bytes / HBM,
+            # flops / FP32 peak)); the tensor-core kernel the step runs is reported beside it
+            "subsampler_ms": simt["ms"] if simt else None,
+            "subsampler_roofline_frac": simt["fp32_frac"] if simt else None,
+            "subsampler_fp32_pipe_frac": simt["TFLOP_per_s"] / fp32_tflops if simt else None,
+            "subsampler_tc_ms": ms, "subsampler_tc_hbm_frac": sb / (ms * 1e-3) / 1e9 / hbm,
             "rows": row,
-            "roofline": {"bound": "alu", "kernel": "dw_subsample_tc_kernel",
-                         "achieved": sf / (ms * 1e-3) / 1e12, "peak": fp32_tflops, "unit": "TFLOP/s",
-                         "frac": sf / (ms * 1e-3) / 1e12 / fp32_tflops,
-                         "peak_basis": f"{sms} SMs x 128 FP32 lanes x 2 x {fmax:.0f} MHz ({peak_kind} max clock)",
-                         "traffic": ncu_traffic("dw_subsample_tc_kernel"),
-                         "note": "roofline time = max(alg bytes / HBM, alg FLOPs / FP32 peak), the FP32 term "
-                                 "binding; conv0's 9-tap contraction runs on tcgen05 (TF32 with a 3-product "
-                                 "float32 split), ReLU and conv_dw1 on the FP32 pipes",
-                         "hbm_frac_of_measured": sb / (ms * 1e-3) / 1e9 / hbm},
+            "configs": configs,
+            "roofline": {"bound": "hbm", "kernel": "dw_subsample_tc_kernel",
+                         "achieved": sb / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": sb / (ms * 1e-3) / 1e9 / hbm, "traffic": ncu_traffic("dw_subsample_tc_kernel"),
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "note": "the step's dominant kernel, bound by HBM on the resources it uses: conv0 runs on "
+                                 "tcgen05 (TF32 3-product split), ReLU and conv_dw1 on the FP32 pipes "
+                                 f"({sf / 1e9:.2f} GFLOP algorithmic, {sf / tc_us / 1e6 / fp32_tflops:.2f} of the "
+                                 f"FP32 peak {fp32_tflops:.1f} TFLOP/s = {sms} SMs x 128 x 2 x {fmax:.0f} MHz)"},
             "hbm_peak_gbs": hbm, "hbm_peak_kind": peak_kind,
             "cpu_baseline": cpu, "e2e": e2e,
             "next_rows": next_rows,
             "gpu_launches": steps * sum(launches_per_row.values()),
             "clocks": clocks,
         }
+        line["summary"] = summary_table(line)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
