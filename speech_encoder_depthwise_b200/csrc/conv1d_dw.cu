@@ -30,7 +30,7 @@ namespace dwk {
 constexpr int kDwThreads = 256;
 constexpr int kDwCluster = 8;
 constexpr int kDwTapBlock = 8;   // taps per pass for widths without a specialisation
-constexpr int kDwMaxRows = 64;   // partial rows at most (clusters per channel tile)
+constexpr int kDwMaxRows = 256;  // partial rows at most (blocks, or clusters, per channel tile)
 constexpr int kDwMaxRows16 = 16; // partial rows of the register-tiled kernel
 
 template <typename T, int V, int KB, int R>
@@ -207,11 +207,9 @@ struct DwTmaShape {
     static constexpr int SMEM = 128 + BODY;  // plus the tile-order tables, sized at launch
 };
 
-// PACKED: items are the sequences of a packed batch (x, dy [N][C], `lengths` = offsets[B+1],
-// Tn = N): only each sequence's own frame-runs are dealt, through a prefix table of runs per item
-// built like the order tables; boxes start at the sequence's first row of the [1][N][C] maps and
-// rows of the neighbouring sequences are masked like frames past a length.
-template <typename T, int V, int KB, bool FUSED = false, bool PACKED = false>
+// Used for the one-pass data + weight gradient (FUSED) and for batches of more than
+// kOrderMaxItems items; the span-balanced kernel below takes every other pipelined case.
+template <typename T, int V, int KB, bool FUSED = false>
 __global__ void __launch_bounds__(DwTmaShape<T, V, KB, FUSED>::THREADS, FUSED ? 1 : kDwBlocks)
 conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
                      const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C, int K,
@@ -234,35 +232,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     int *ord_mem = reinterpret_cast<int *>(stages + S::BODY);
     TileOrder order{ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), B, nT, 1, 0};
     grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
-    // packed: pv = runs before item b, pst = its first row, plen = its length
-    int *pv = ord_mem, *pst = ord_mem + (B + 1), *plen = pst + B;
-    if constexpr (PACKED) {
-        if (warp == 0) {  // offsets clamped into [0, N]
-            int run = 0;
-            if (lane == 0) pv[0] = 0;
-            for (int base = 0; base < B; base += 32) {
-                const int bb = base + lane;
-                int nv = 0;
-                if (bb < B) {
-                    int s0 = __ldg(lengths + bb), e = __ldg(lengths + bb + 1);
-                    s0 = s0 < 0 ? 0 : (s0 > Tn ? Tn : s0);
-                    e = e < s0 ? s0 : (e > Tn ? Tn : e);
-                    pst[bb] = s0;
-                    plen[bb] = e - s0;
-                    nv = (e - s0 + S::TT - 1) / S::TT;
-                }
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int t = __shfl_up_sync(0xffffffffu, nv, o);
-                    if (lane >= o) nv += t;
-                }
-                if (bb < B) pv[bb + 1] = run + nv;
-                run += __shfl_sync(0xffffffffu, nv, 31);
-            }
-        }
-    } else {
-        if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
-    }
+    if (ordered) order.build(ord_mem, ord_mem + (B + 1), ord_mem + 2 * (B + 1), lengths, Tn, S::TT);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDwStages; ++i) {
             mbar_init(&full[i], 1);
@@ -271,15 +241,11 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
         fence_barrier_init();
     }
     __syncthreads();
-    if (!PACKED && ordered) order.V = order.pv[B];
+    if (ordered) order.V = order.pv[B];
     // the fused pass also walks the wholly masked units: their dx frames are written as zeros
-    const int units = PACKED ? pv[B] : ((ordered && !FUSED) ? order.V : B * nT);
+    const int units = (ordered && !FUSED) ? order.V : B * nT;
     auto unit_at = [&](int u, int &b, int &t0, int &L) {
-        if constexpr (PACKED) {
-            b = TileOrder::find(pv, B, u);
-            t0 = (u - pv[b]) * S::TT;
-            L = plen[b];
-        } else if (ordered) {
+        if (ordered) {
             int tt, ctd;
             order.map(u, b, tt, ctd, L);
             t0 = tt * S::TT;
@@ -311,7 +277,7 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
             if (!ok) break;
             if (lane == 0) {
                 int b, t0, L;
-                if (PACKED || ordered || it >= kDwStages) {
+                if (ordered || it >= kDwStages) {
                     unit_at(u, b, t0, L);
                 } else {  // the first ring-full is issued before any length is read
                     b = u / nT;
@@ -320,11 +286,9 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
                 }
                 if (t0 < L) {  // frames before 0 or past T arrive as zeros; [L, T) is masked by the consumers
                     unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
-                    // padded: item b of the [B][T][C] maps; packed: rows of the [1][N][C] maps
-                    const int r0 = PACKED ? pst[b] : 0, bi = PACKED ? 0 : b;
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                    tma_load_3d(st, &xmap, c0, r0 + t0 + k_off - pad_left, bi, &full[s]);
-                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, r0 + (FUSED ? t0 - padR : t0), bi, &full[s]);
+                    tma_load_3d(st, &xmap, c0, t0 + k_off - pad_left, b, &full[s]);
+                    tma_load_3d(st + S::XROWS * S::ROWB, &dmap, c0, FUSED ? t0 - padR : t0, b, &full[s]);
                 } else {
                     mbar_arrive(&full[s]);  // a wholly masked unit: nothing to read
                 }
@@ -492,6 +456,251 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
     cluster.sync();
 }
 
+// ---------------------------------------------------------------------------------------
+// Span-balanced variant (the default for 16-byte rows, specialised K and up to kOrderMaxItems
+// items): grid (G, channel tiles), kDwBlocks blocks per SM, no clusters.  The valid frames of
+// all items (t < len_b; in a packed batch every row of every sequence), item after item, form
+// one sequence of V frames per channel tile: block j of the tile's G blocks takes the contiguous
+// span [V j / G, V (j+1) / G) of it, cut into tiles of at most TT frames that never cross an
+// item, so every block reads the same number of frames to within one.  The producer copies a
+// tile of n frames as ceil((n + K - 1) / SB) tensor boxes of x (halo included) and ceil(n / SB)
+// boxes of dy, SB rows each, so a short tile reads little beyond its own rows.  The consumers
+// accumulate dW/dbias for their R frames of every tile in registers, as in the kernel above.  At
+// the end the block adds its warps' sums in a fixed order through shared memory and writes one
+// partial row; the finalize kernel adds the G rows in a fixed order (no atomics, reproducible
+// for given sizes on a given GPU model).  The lengths are prefetched into L2 before the
+// dependency wait: a prefetch only warms the cache, so writes of the previous kernel are seen.
+// ---------------------------------------------------------------------------------------
+constexpr int kDwSB = 8;  // rows per tensor box
+
+template <typename T, int V, int KB>
+struct DwSpanShape {
+    static constexpr int CONS = kDwConsumers;
+    static constexpr int R = kDwR;
+    static constexpr int THREADS = 32 * (1 + CONS);
+    static constexpr int CT = 32 * V;
+    static constexpr int TT = CONS * R;
+    static constexpr int ROWB = CT * static_cast<int>(sizeof(T));
+    static constexpr int XROWS = (TT + KB - 1 + kDwSB - 1) / kDwSB * kDwSB;
+    static constexpr int DROWS = (TT + kDwSB - 1) / kDwSB * kDwSB;
+    static constexpr int BOX_BYTES = kDwSB * ROWB;
+    static constexpr int STAGE_BYTES = (XROWS + DROWS) * ROWB;
+    static constexpr int RED_BYTES = CONS * (KB + 1) * CT * 4;
+    static constexpr int BODY = (kDwStages * STAGE_BYTES > RED_BYTES) ? kDwStages * STAGE_BYTES : RED_BYTES;
+    static constexpr int SMEM = 128 + BODY;  // plus the item tables, sized at launch
+};
+
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
+}
+
+// PACKED: x and dy [N][C], `lengths` = offsets[B+1] (clamped into [0, N], non-decreasing), Tn = N.
+template <typename T, int V, int KB, bool PACKED>
+__global__ void __launch_bounds__(DwSpanShape<T, V, KB>::THREADS, kDwBlocks)
+conv1d_dw_span_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
+                      const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C,
+                      int K, int k_off, int pad_left, int with_bias) {
+    using S = DwSpanShape<T, V, KB>;
+    constexpr int NP = Pairs<V>::n;
+    constexpr int R = S::R;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw);
+    uint64_t *empty = full + kDwStages;
+    unsigned char *stages = smem_raw + 128;
+    // per item: valid frames before it (pv), its valid frames (plen) and its first row (pst)
+    int *pv = reinterpret_cast<int *>(stages + S::BODY);
+    int *plen = pv + (B + 1), *pst = plen + B;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int jj = static_cast<int>(blockIdx.x), G = static_cast<int>(gridDim.x), ct = static_cast<int>(blockIdx.y);
+    const int c0 = ct * S::CT;
+    launch_dependents();  // the finalize may be scheduled now; it waits for this grid to finish
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDwStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], S::CONS);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&xmap);
+            prefetch_tmap(&dmap);
+        }
+        if (lengths != nullptr)  // one 128-byte line per 32 entries
+            for (int i = lane * 32; i < (PACKED ? B + 1 : B); i += 32 * 32) prefetch_l2(lengths + i);
+    }
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
+    for (int bb = static_cast<int>(threadIdx.x); bb < B; bb += static_cast<int>(blockDim.x)) {
+        int s0 = 0, L;
+        if constexpr (PACKED) {
+            s0 = __ldg(lengths + bb);
+            int e = __ldg(lengths + bb + 1);
+            s0 = s0 < 0 ? 0 : (s0 > Tn ? Tn : s0);
+            e = e < s0 ? s0 : (e > Tn ? Tn : e);
+            L = e - s0;
+        } else {
+            L = static_cast<int>(clamp_len(lengths, bb, Tn));
+        }
+        plen[bb] = L;
+        pst[bb] = s0;
+    }
+    __syncthreads();
+    if (warp == 0) {  // prefix sums of the valid frames
+        int run = 0;
+        if (lane == 0) pv[0] = 0;
+        for (int base = 0; base < B; base += 32) {
+            const int bb = base + lane;
+            int v = bb < B ? plen[bb] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += t;
+            }
+            if (bb < B) pv[bb + 1] = run + v;
+            run += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    __syncthreads();
+    const int v_begin = static_cast<int>(static_cast<int64_t>(pv[B]) * jj / G);
+    const int v_end = static_cast<int>(static_cast<int64_t>(pv[B]) * (jj + 1) / G);
+    // the tile that starts at position p of the valid sequence: item b (advanced in place; items
+    // without valid frames are skipped), its first frame t0 and its frame count n
+    auto tile_at = [&](int p, int &b, int &t0, int &n) {
+        while (pv[b + 1] <= p) ++b;
+        t0 = p - pv[b];
+        const int left = plen[b] - t0, span = v_end - p;
+        n = left < span ? left : span;
+        if (n > S::TT) n = S::TT;
+    };
+    float2 acc[KB][NP], accb[NP];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+        accb[q] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < KB; ++k) acc[k][q] = make_float2(0.f, 0.f);
+    }
+
+    if (warp == 0) {  // producer warp: one elected lane issues the tile's tensor boxes
+        int b = v_begin < v_end ? TileOrder::find(pv, B, v_begin) : 0;
+        int it = 0;
+        for (int p = v_begin; p < v_end; ++it) {
+            int t0, n;
+            tile_at(p, b, t0, n);
+            const int s = it % kDwStages;
+            const uint32_t ph = (it / kDwStages) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) break;
+            if (lane == 0) {
+                const int nbx = (n + KB - 1 + kDwSB - 1) / kDwSB, nby = (n + kDwSB - 1) / kDwSB;
+                unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>((nbx + nby) * S::BOX_BYTES));
+                // padded: frames of item b of the [B][T][C] maps; packed: rows of the [1][N][C] maps
+                const int r0 = PACKED ? pst[b] : 0, bi = PACKED ? 0 : b;
+                for (int i = 0; i < nbx; ++i)
+                    tma_load_3d(st + i * S::BOX_BYTES, &xmap, c0, r0 + t0 + k_off - pad_left + i * kDwSB, bi, &full[s]);
+                for (int i = 0; i < nby; ++i)
+                    tma_load_3d(st + S::XROWS * S::ROWB + i * S::BOX_BYTES, &dmap, c0, r0 + t0 + i * kDwSB, bi,
+                                &full[s]);
+            }
+            __syncwarp();
+            p += n;
+        }
+    } else {  // consumer warp cw: frames [t0 + cw R, t0 + cw R + R) of every tile
+        const int cw = warp - 1;
+        const bool active = c0 + lane * V < C;
+        int b = v_begin < v_end ? TileOrder::find(pv, B, v_begin) : 0;
+        int it = 0;
+        for (int p = v_begin; p < v_end; ++it) {
+            int t0, n;
+            tile_at(p, b, t0, n);
+            const int s = it % kDwStages;
+            const uint32_t ph = (it / kDwStages) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) break;
+            const int tg = t0 + cw * R;   // this warp's first frame
+            const int nr = n - cw * R;    // its frame count (R at most; none when <= 0)
+            if (active && nr > 0) {
+                const int L = plen[b];
+                const unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES + lane * V * sizeof(T);
+                const unsigned char *dp = st + (S::XROWS + cw * R) * S::ROWB;
+                const unsigned char *xp = st + (cw * R) * S::ROWB;
+                const int jb = tg + k_off - pad_left;  // frame of this warp's first x row
+                // CHECK = false: all R frames are this warp's and every x row is inside [0, len_b).
+                // With CHECK, rows past this warp's frames (not loaded, or of the next warp) are
+                // zeroed as well, so that nothing stale meets a zero dz.
+                auto run = [&](auto check) {
+                    constexpr bool CHECK = decltype(check)::value;
+                    float2 dz[R][NP];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        Vec<T, V> v;
+                        v.r = *reinterpret_cast<const decltype(v.r) *>(dp + r * S::ROWB);
+                        if constexpr (CHECK) {
+                            if (r >= nr) v.zero();
+                        }
+                        v.to_f2(dz[r]);
+#pragma unroll
+                        for (int q = 0; q < NP; ++q) {
+                            accb[q].x += dz[r][q].x;
+                            accb[q].y += dz[r][q].y;
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < R + KB - 1; ++i) {
+                        Vec<T, V> v;
+                        v.r = *reinterpret_cast<const decltype(v.r) *>(xp + i * S::ROWB);
+                        if constexpr (CHECK) {
+                            if (jb + i < 0 || jb + i >= L || i >= nr + KB - 1) v.zero();
+                        }
+                        float2 xf[NP];
+                        v.to_f2(xf);
+#pragma unroll
+                        for (int k = 0; k < KB; ++k) {
+                            const int r = i - k;
+                            if (r >= 0 && r < R) {
+#pragma unroll
+                                for (int q = 0; q < NP; ++q) acc[k][q] = ffma2(dz[r][q], xf[q], acc[k][q]);
+                            }
+                        }
+                    }
+                };
+                if (nr >= R && jb >= 0 && jb + R + KB - 1 <= L) run(std::false_type{});
+                else run(std::true_type{});
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            p += n;
+        }
+    }
+    // every warp has left the pipeline; the stage memory now holds the block's sums
+    __syncthreads();
+    const int E = (KB + 1) * S::CT;
+    float *red = reinterpret_cast<float *>(stages);
+    if (warp > 0) {
+        float *mine = red + static_cast<size_t>(warp - 1) * E;
+#pragma unroll
+        for (int k = 0; k <= KB; ++k) {
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float2 v = (k < KB) ? acc[k][q] : accb[q];
+                if (2 * q < V) mine[k * S::CT + lane * V + 2 * q] = v.x;
+                if (2 * q + 1 < V) mine[k * S::CT + lane * V + 2 * q + 1] = v.y;
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = static_cast<int>(threadIdx.x); e < E; e += static_cast<int>(blockDim.x)) {
+        float sum = red[e];
+        for (int r = 1; r < S::CONS; ++r) sum += red[static_cast<size_t>(r) * E + e];
+        const int kk = e / S::CT;
+        const int64_t c = static_cast<int64_t>(c0) + (e % S::CT);
+        if (c >= C) continue;
+        if (kk == KB) {
+            if (with_bias) partials[(static_cast<int64_t>(jj) * (K + 1) + K) * C + c] = sum;
+        } else if (k_off + kk < K) {
+            partials[(static_cast<int64_t>(jj) * (K + 1) + k_off + kk) * C + c] = sum;
+        }
+    }
+}
+
 // dW[k][c] / dbias[c] = sum over the partial rows.  A block covers 32 consecutive (k, c) entries
 // with 8 row groups: group r adds rows r, r+8, r+16, ... in order, then the 8 group sums are
 // added in a fixed tree.  The order depends only on the row count, so results are reproducible.
@@ -519,20 +728,98 @@ conv1d_dw_finalize_kernel(const float *__restrict__ partials, float *__restrict_
     }
 }
 
+// The same sum for (K+1)*C a multiple of 4, with every load of a thread in flight at once: a
+// block covers 64 consecutive entries (16 lanes x float4) with 16 row groups; group r loads rows
+// r, r+16, r+32, ... (at most 16 per thread; G <= 256) and adds them in order, then the 16 group
+// sums are added in a fixed tree.  Reproducible for a given row count.
+constexpr int kFinGroups = 16;
+__global__ void __launch_bounds__(256)
+conv1d_dw_finalize4_kernel(const float *__restrict__ partials, float *__restrict__ dw,
+                           float *__restrict__ dbias, int Gp, int K, int64_t C) {
+    __shared__ float4 red[kFinGroups][16];
+    grid_dependency_wait();  // launched programmatically after the partial kernel
+    const int lane = threadIdx.x % 16, rg = threadIdx.x / 16;
+    const int64_t E4 = static_cast<int64_t>(K + 1) * C / 4;
+    const int64_t e4 = static_cast<int64_t>(blockIdx.x) * 16 + lane;
+    const float4 *p4 = reinterpret_cast<const float4 *>(partials);
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e4 < E4) {
+        float4 v[kDwMaxRows / kFinGroups];
+#pragma unroll
+        for (int i = 0; i < kDwMaxRows / kFinGroups; ++i) {
+            const int g = rg + i * kFinGroups;
+            v[i] = g < Gp ? __ldg(p4 + static_cast<int64_t>(g) * E4 + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < kDwMaxRows / kFinGroups; ++i) {
+            s.x += v[i].x;
+            s.y += v[i].y;
+            s.z += v[i].z;
+            s.w += v[i].w;
+        }
+    }
+    red[rg][lane] = s;
+    __syncthreads();
+    if (rg == 0 && e4 < E4) {
+        float4 t[kFinGroups];
+#pragma unroll
+        for (int r = 0; r < kFinGroups; ++r) t[r] = red[r][lane];
+#pragma unroll
+        for (int w = 1; w < kFinGroups; w <<= 1) {
+#pragma unroll
+            for (int r = 0; r + w < kFinGroups; r += 2 * w) {
+                t[r].x += t[r + w].x;
+                t[r].y += t[r + w].y;
+                t[r].z += t[r + w].z;
+                t[r].w += t[r + w].w;
+            }
+        }
+        const float o[4] = {t[0].x, t[0].y, t[0].z, t[0].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t e = 4 * e4 + q, k = e / C, c = e % C;
+            if (k < K) dw[k * C + c] = o[q];
+            else if (dbias) dbias[c] = o[q];
+        }
+    }
+}
+
+// dW / dbias from Gp partial rows [Gp][K+1][C] (programmatic dependent launch).
+cudaError_t launch_finalize_rows(const float *partials, float *dw, float *dbias, int Gp, int K, int64_t C,
+                                 cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(K + 1) * C;
+    const bool vec = n % 4 == 0 && reinterpret_cast<uintptr_t>(partials) % 16 == 0 && Gp <= kDwMaxRows;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(vec ? (n / 4 + 15) / 16 : (n + 31) / 32));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (vec) return cudaLaunchKernelEx(&cfg, conv1d_dw_finalize4_kernel, partials, dw, dbias, Gp, K, C);
+    return cudaLaunchKernelEx(&cfg, conv1d_dw_finalize_kernel, partials, dw, dbias, Gp, K, C);
+}
+
 __global__ void conv1d_dw_zero_kernel(float *__restrict__ dw, float *__restrict__ dbias, int K, int64_t C) {
     const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (e < static_cast<int64_t>(K) * C) dw[e] = 0.f;
     if (dbias && e < C) dbias[e] = 0.f;
 }
 
-// Upper bound on the partial rows (one per cluster of blocks per channel tile); the workspace
-// is sized for it, so it depends on the sizes alone.
-int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t /*C*/, int /*K*/) {
+// Upper bound on the partial rows (one per block, or per cluster of blocks, of a channel tile):
+// one per 64 frames, at most kDwMaxRows, and no more than keep the workspace within 64 MiB when
+// the rows are wide.  The workspace is sized for it, so it depends on the sizes alone.
+int conv1d_dw_partial_rows(int64_t B, int64_t T, int64_t C, int K) {
     const int64_t frames = B * T;
     if (frames <= 0) return 0;
-    int64_t gp = (frames + 255) / 256;
-    if (gp < 1) gp = 1;
+    int64_t gp = (frames + 63) / 64;
     if (gp > kDwMaxRows) gp = kDwMaxRows;
+    const int64_t row_bytes = static_cast<int64_t>(K + 1) * C * static_cast<int64_t>(sizeof(float));
+    const int64_t cap = (int64_t(64) << 20) / (row_bytes > 0 ? row_bytes : 1);
+    if (gp > cap) gp = cap;
+    if (gp < 1) gp = 1;
     return static_cast<int>(gp);
 }
 
@@ -577,20 +864,18 @@ cudaError_t launch_pass(const DwArgs &a, int gp, int k_off, int with_bias, cudaS
 
 // Grid rows G and cluster size for the pipelined kernel: as many blocks per channel tile as
 // fit on the device at once, in clusters as large as that allows (fewer partial rows).
-template <typename T, int V, int KB, bool FUSED = false, bool PACKED = false>
-cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s,
-                            const int32_t *offsets = nullptr) {
+template <typename T, int V, int KB, bool FUSED = false>
+cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_out, cudaStream_t s) {
     using S = DwTmaShape<T, V, KB, FUSED>;
-    auto kern = conv1d_dw_tma_kernel<T, V, KB, FUSED, PACKED>;
-    const int ordered = PACKED ? 1 : ((DW_DW_ORDERED && a.B <= kOrderMaxItems) ? 1 : 0);
+    auto kern = conv1d_dw_tma_kernel<T, V, KB, FUSED>;
+    const int ordered = (DW_DW_ORDERED && a.B <= kOrderMaxItems) ? 1 : 0;
     const int smem = S::SMEM + (ordered ? static_cast<int>((3 * (a.B + 1) * sizeof(int) + 15) / 16 * 16) : 0);
     const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
                                               S::SMEM + static_cast<int>(3 * (kOrderMaxItems + 1) * sizeof(int)) + 16);
     if (attr != cudaSuccess) return attr;
     const int nCT = static_cast<int>((a.C + S::CT - 1) / S::CT);
     const int nT = static_cast<int>((a.T + S::TT - 1) / S::TT);
-    // packed: the runs of all sequences, at most one partial run per sequence beyond N / TT
-    const int64_t units = PACKED ? nT + a.B : a.B * nT;
+    const int64_t units = a.B * nT;
     if (nCT > 65535 || units >= (1LL << 31)) return cudaErrorInvalidConfiguration;
     int best_g = 0, best_c = 1;
     for (int c : {8, 4, 2, 1}) {
@@ -641,13 +926,57 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
     cfg.attrs = at2;
     cfg.numAttrs = 2;
     CUtensorMap xmap, dmap;
-    const int64_t mB = PACKED ? 1 : a.B;
-    cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), mB, a.T, a.C, S::CT, S::XROWS);
-    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, dtype_code<T>(), mB, a.T, a.C, S::CT, S::DROWS);
+    cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::XROWS);
+    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, dtype_code<T>(), a.B, a.T, a.C, S::CT, S::DROWS);
     if (me != cudaSuccess) return me;
-    return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, PACKED ? offsets : a.lengths, a.partials, static_cast<int>(a.B),
+    return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, a.lengths, a.partials, static_cast<int>(a.B),
                               static_cast<int>(a.T), static_cast<int>(a.C), a.K, k_off, a.pad_left, nT, with_bias,
                               ordered, a.w, static_cast<T *>(a.dx));
+}
+
+// The span-balanced kernel for a padded batch (offsets == null) or a packed one: grid (G, channel
+// tiles), G = the blocks per channel tile that fit on the device at once, at most a.G (the
+// workspace's partial rows) and no more than the frames fill tiles of TT.
+template <typename T, int V, int KB>
+cudaError_t launch_span_pass(const DwArgs &a, const int32_t *offsets, int *gp_out, cudaStream_t s) {
+    using S = DwSpanShape<T, V, KB>;
+    const bool packed = offsets != nullptr;
+    auto kern = packed ? conv1d_dw_span_kernel<T, V, KB, true> : conv1d_dw_span_kernel<T, V, KB, false>;
+    const int smem = S::SMEM + static_cast<int>((3 * a.B + 1) * sizeof(int));
+    const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
+                                              S::SMEM + static_cast<int>((3 * kOrderMaxItems + 1) * sizeof(int)));
+    if (attr != cudaSuccess) return attr;
+    const int64_t nCT = (a.C + S::CT - 1) / S::CT;
+    if (nCT > 65535) return cudaErrorInvalidConfiguration;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, S::THREADS, smem) != cudaSuccess || per_sm < 1) {
+        (void)cudaGetLastError();
+        per_sm = 1;
+    }
+    const int64_t frames = packed ? a.T : a.B * a.T;  // an upper bound on the valid frames
+    int64_t G = static_cast<int64_t>(sm_count()) * per_sm / nCT;
+    const int64_t gmax = (frames + S::TT - 1) / S::TT;
+    if (G > gmax) G = gmax;
+    if (G > a.G) G = a.G;
+    if (G < 1) G = 1;  // more channel tiles than resident blocks: one block per tile, in waves
+    *gp_out = static_cast<int>(G);
+    CUtensorMap xmap, dmap;
+    const int64_t mB = packed ? 1 : a.B;
+    cudaError_t me = make_act_map(&xmap, a.x, dtype_code<T>(), mB, a.T, a.C, S::CT, kDwSB);
+    if (me == cudaSuccess) me = make_act_map(&dmap, a.dy, dtype_code<T>(), mB, a.T, a.C, S::CT, kDwSB);
+    if (me != cudaSuccess) return me;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(G), static_cast<unsigned>(nCT));
+    cfg.blockDim = dim3(S::THREADS);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, packed ? offsets : a.lengths, a.partials, static_cast<int>(a.B),
+                              static_cast<int>(a.T), static_cast<int>(a.C), a.K, 0, a.pad_left, 1);
 }
 
 template <typename T>
@@ -667,6 +996,21 @@ int channel_tiles(int64_t C) {
 template <typename T, int V>
 cudaError_t launch_partials(const DwArgs &a, int *gp_out, cudaStream_t s) {
     if constexpr (V >= 2) {
+        if (dw_tma_ok<T>(a) && a.B <= kOrderMaxItems) {
+            switch (a.K) {
+                case 1: return launch_span_pass<T, V, 1>(a, nullptr, gp_out, s);
+                case 2: return launch_span_pass<T, V, 2>(a, nullptr, gp_out, s);
+                case 3: return launch_span_pass<T, V, 3>(a, nullptr, gp_out, s);
+                case 4: return launch_span_pass<T, V, 4>(a, nullptr, gp_out, s);
+                case 5: return launch_span_pass<T, V, 5>(a, nullptr, gp_out, s);
+                case 7: return launch_span_pass<T, V, 7>(a, nullptr, gp_out, s);
+                case 9: return launch_span_pass<T, V, 9>(a, nullptr, gp_out, s);
+                default: break;
+            }
+            if constexpr (V == 2) {
+                if (a.K == 15) return launch_span_pass<T, V, 15>(a, nullptr, gp_out, s);
+            }
+        }
         if (dw_tma_ok<T>(a)) {
             switch (a.K) {
                 case 1: return launch_tma_pass<T, V, 1>(a, 0, 1, gp_out, s);
@@ -747,18 +1091,7 @@ cudaError_t launch_fused_partials(const DwArgs &a, int *gp, cudaStream_t s) {
 }
 
 cudaError_t launch_finalize(const DwArgs &a, int gp, cudaStream_t s) {
-    const int64_t n = static_cast<int64_t>(a.K + 1) * a.C;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((n + 31) / 32));
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, conv1d_dw_finalize_kernel, static_cast<const float *>(a.partials), a.dw, a.dbias,
-                              gp, a.K, static_cast<int64_t>(a.C));
+    return launch_finalize_rows(a.partials, a.dw, a.dbias, gp, a.K, a.C, s);
 }
 
 }  // namespace
@@ -949,27 +1282,32 @@ cudaError_t conv1d_dw_packed_launch(const DwArgs &a, const int32_t *offsets, cud
             if constexpr (sizeof(T) == 2) {
                 if (a.vec_width >= 4) {
                     switch (a.K) {
-                        case 3: return launch_tma_pass<T, 4, 3, false, true>(b, 0, 1, &gp, s, offsets);
-                        case 4: return launch_tma_pass<T, 4, 4, false, true>(b, 0, 1, &gp, s, offsets);
-                        case 5: return launch_tma_pass<T, 4, 5, false, true>(b, 0, 1, &gp, s, offsets);
-                        case 7: return launch_tma_pass<T, 4, 7, false, true>(b, 0, 1, &gp, s, offsets);
-                        case 9: return launch_tma_pass<T, 4, 9, false, true>(b, 0, 1, &gp, s, offsets);
+                        case 1: return launch_span_pass<T, 4, 1>(b, offsets, &gp, s);
+                        case 2: return launch_span_pass<T, 4, 2>(b, offsets, &gp, s);
+                        case 3: return launch_span_pass<T, 4, 3>(b, offsets, &gp, s);
+                        case 4: return launch_span_pass<T, 4, 4>(b, offsets, &gp, s);
+                        case 5: return launch_span_pass<T, 4, 5>(b, offsets, &gp, s);
+                        case 7: return launch_span_pass<T, 4, 7>(b, offsets, &gp, s);
+                        case 9: return launch_span_pass<T, 4, 9>(b, offsets, &gp, s);
                         default: return cudaErrorNotSupported;
                     }
                 }
             }
             switch (a.K) {
-                case 3: return launch_tma_pass<T, 2, 3, false, true>(b, 0, 1, &gp, s, offsets);
-                case 9: return launch_tma_pass<T, 2, 9, false, true>(b, 0, 1, &gp, s, offsets);
-                case 15: return launch_tma_pass<T, 2, 15, false, true>(b, 0, 1, &gp, s, offsets);
+                case 1: return launch_span_pass<T, 2, 1>(b, offsets, &gp, s);
+                case 2: return launch_span_pass<T, 2, 2>(b, offsets, &gp, s);
+                case 3: return launch_span_pass<T, 2, 3>(b, offsets, &gp, s);
+                case 4: return launch_span_pass<T, 2, 4>(b, offsets, &gp, s);
+                case 5: return launch_span_pass<T, 2, 5>(b, offsets, &gp, s);
+                case 7: return launch_span_pass<T, 2, 7>(b, offsets, &gp, s);
+                case 9: return launch_span_pass<T, 2, 9>(b, offsets, &gp, s);
+                case 15: return launch_span_pass<T, 2, 15>(b, offsets, &gp, s);
                 default: return cudaErrorNotSupported;
             }
         });
         if (et != cudaErrorNotSupported) {
             if (et != cudaSuccess) return et;
-            conv1d_dw_finalize_kernel<<<static_cast<unsigned>((n + 31) / 32), 256, 0, s>>>(a.partials, a.dw, a.dbias,
-                                                                                            gp, a.K, a.C);
-            return cudaGetLastError();
+            return launch_finalize_rows(a.partials, a.dw, a.dbias, gp, a.K, a.C, s);
         }
     }
     const int G = conv1d_dw_packed_rows(a.T);
@@ -994,9 +1332,7 @@ cudaError_t conv1d_dw_packed_launch(const DwArgs &a, const int32_t *offsets, cud
         });
         if (e != cudaSuccess) return e;
     }
-    conv1d_dw_finalize_kernel<<<static_cast<unsigned>((n + 31) / 32), 256, 0, s>>>(a.partials, a.dw, a.dbias, G, a.K,
-                                                                                    a.C);
-    return cudaGetLastError();
+    return launch_finalize_rows(a.partials, a.dw, a.dbias, G, a.K, a.C, s);
 }
 
 cudaError_t conv1d_dw_launch(const DwArgs &a, cudaStream_t s) {
