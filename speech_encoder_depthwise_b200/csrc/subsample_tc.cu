@@ -67,6 +67,7 @@ constexpr int kEpiThreads = kEpiWarps * 32, kPatchThreads = kPatchWarps * 32;
 constexpr int kMmaWarp = kEpiWarps + kPatchWarps;  // then one warp whose lane 0 issues the bulk stores
 constexpr int kThreads = (kMmaWarp + 2) * 32;
 constexpr int kMelLoads = (kMelElems + kPatchThreads - 1) / kPatchThreads;
+constexpr int kMelStages = 3;               // mel windows in shared memory: copies run two units ahead
 constexpr int kRowBytes = 128;               // one K row: 32 TF32 words
 constexpr int kTileA = 128 * kRowBytes;
 constexpr int kTileB = kN * kRowBytes;
@@ -89,9 +90,9 @@ struct TcLayout {
     static constexpr int a_off = 0;
     static constexpr int b_off = CTG * kTileA;
     static constexpr int mel_bytes = (kMR * kMCP * 4 + 127) / 128 * 128;
-    static constexpr int mel_off = b_off + 2 * kTileB;
+    static constexpr int mel_off = b_off + 2 * kTileB;        // kMelStages staged mel windows
     static constexpr int st_bytes = kRO * kJO * 128 * static_cast<int>(sizeof(TO));
-    static constexpr int st_off = mel_off + 2 * mel_bytes;   // 2 staging tiles per group, zero tile
+    static constexpr int st_off = mel_off + kMelStages * mel_bytes;  // 2 staging tiles per group, zero tile
     static constexpr int wt_off = st_off + 5 * st_bytes;      // conv_dw1 weight table
     static constexpr int list_off = wt_off + CTG * 10 * 128 * 4;  // unit list
     static constexpr int bar_off = list_off + kListCap * 16;
@@ -174,6 +175,14 @@ template <int N> __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 4-byte asynchronous copy global -> shared; src_bytes = 0 writes a zero and reads nothing.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <typename TO> __device__ __forceinline__ void stage_out(TO *p, float v);
 template <> __device__ __forceinline__ void stage_out<float>(float *p, float v) { *p = v; }
@@ -411,8 +420,8 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
                 E[0][1] = relu_pair(v[1], v[3]);
                 E[0][2] = relu_pair(v[2], v[4]);
             }
-#pragma unroll 1
-            for (int ch = 0; ch < kJO / kChunk && ok; ++ch) {
+#pragma unroll
+            for (int ch = 0; ch < kJO / kChunk; ++ch) {  // unrolled: the per-chunk branches resolve at compile time
                 const int jl0 = ch * kChunk;                     // first output column (unit-local)
                 float v[50];
                 tmem_ld_chunk(tacc, ch, v);                      // h columns 2 jl0 + 1 .. 2 jl0 + 10
@@ -422,7 +431,10 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
                     if (lane == 0) mbar_arrive(&acc_empty[grp]);
                 }
                 // this slot's previous tile (two jobs back) has been read by its store
-                if (ch == 0 && n > 1) ok = mbar_wait(&stage_free[2 * grp + (n & 1)], ((n >> 1) - 1) & 1);
+                if (ch == 0 && n > 1) {
+                    ok = mbar_wait(&stage_free[2 * grp + (n & 1)], ((n >> 1) - 1) & 1);
+                    if (!ok) break;
+                }
 #pragma unroll
                 for (int i = 1; i <= kChunk; ++i) {
                     const float *x = v + (2 * i - 1) * kHR;
@@ -461,7 +473,10 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         }
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ patch builders
-        const int pt = threadIdx.x - kEpiThreads;
+        // Builder thread pt takes rows pt, pt + 128 (< kN): the builder warps with two rows a lane
+        // are the last ones (SM sub-partitions 2 and 3), because the MMA issuer and the store
+        // thread share sub-partitions 0 and 1 with the first ones.
+        const int pt = kPatchThreads - 1 - (static_cast<int>(threadIdx.x) - kEpiThreads);
         // This thread's mel window elements and patch rows are the same for every unit:
         // element k sits at window row rs >> 8, column rs & 255 (rs = -1 past the window); rows
         // n = pt + i * kPatchThreads all share n % 8 (one swizzle pattern).
@@ -488,31 +503,36 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
                 row_rr[i] = n - 200;
             }
         }
-        float mv[kMelLoads];
-        auto load_mel = [&](const int4 &e) {  // e = {b, i0, j0, len}
+        // The unit's mel window goes straight to shared memory with 4-byte asynchronous copies
+        // (elements outside the window's valid frames and columns are written as zero without a
+        // read), two units ahead of the one being built, in kMelStages rotating windows.
+        auto load_mel = [&](int u) {
+            const int4 e = ulist[u];  // {b, i0, j0, len}
+            float *S = mel_s_tile + (u % kMelStages) * (Lay::mel_bytes / 4);
             const int mr0 = 4 * e.y - 3 * Pt, mc0 = 4 * e.z - 3;
             const float *base = mel + static_cast<int64_t>(e.x) * Tn * F;
             const bool rows_in = mr0 >= 0 && mr0 + kMR <= e.w;  // every window row is a valid frame
 #pragma unroll
             for (int k = 0; k < kMelLoads; ++k) {
+                if (mel_rs[k] < 0) continue;
                 const int mr = mr0 + (mel_rs[k] >> 8), mc = mc0 + (mel_rs[k] & 255);
-                const bool in = mel_rs[k] >= 0 && (rows_in || (mr >= 0 && mr < e.w)) && mc >= 0 && mc < F;
-                float x = 0.f;
-                if (in) x = __ldg(base + mr * F + mc);
-                mv[k] = x;
+                const bool in = (rows_in || (mr >= 0 && mr < e.w)) && mc >= 0 && mc < F;
+                cp_async4(S + (mel_rs[k] >> 8) * kMCP + (mel_rs[k] & 255), in ? base + mr * F + mc : base, in ? 4u : 0u);
             }
         };
-        if (nA > 0) load_mel(ulist[0]);
+        if (nA > 0) load_mel(0);
+        cp_async_commit();
+        if (nA > 1) load_mel(1);
+        cp_async_commit();
         bool ok = true;
         for (int idx = 0; idx < nA && ok; ++idx) {
             const int4 e = ulist[idx];
             const int L2 = (e.w + 1) / 2;
-            float *S = mel_s_tile + (idx & 1) * (Lay::mel_bytes / 4);
-#pragma unroll
-            for (int k = 0; k < kMelLoads; ++k)
-                if (mel_rs[k] >= 0) S[(mel_rs[k] >> 8) * kMCP + (mel_rs[k] & 255)] = mv[k];
-            named_bar(kBarPatch, kPatchThreads);
-            if (idx + 1 < nA) load_mel(ulist[idx + 1]);  // in flight while this unit's patches are built
+            const float *S = mel_s_tile + (idx % kMelStages) * (Lay::mel_bytes / 4);
+            cp_async_wait<1>();  // this thread's copies of unit idx have landed (idx + 1 may be in flight)
+            named_bar(kBarPatch, kPatchThreads);  // ... and every builder's; all are done with unit idx - 1
+            if (idx + 2 < nA) load_mel(idx + 2);  // into the window unit idx - 1 used
+            cp_async_commit();
             const int stage_i = idx & 1;
             ok = named_bar_and(kBarPatch, kPatchThreads, mbar_wait(&patch_empty[stage_i], ((idx >> 1) & 1) ^ 1));
             if (!ok) break;
@@ -551,6 +571,7 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
             fence_async_smem();
             mbar_arrive(&patch_full[stage_i]);
         }
+        cp_async_wait<0>();  // no copy outlives the loop (it may have ended early)
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
