@@ -473,7 +473,12 @@ conv1d_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_cons
 // ---------------------------------------------------------------------------------------
 constexpr int kDwSB = 8;  // rows per tensor box
 
-template <typename T, int V, int KB>
+// FUSED: the same pass also computes the data gradient dx[s] = [s < len_b] sum_k dz[s + pad_left
+// - k] w[k] of every valid frame, so the dy tile carries the K - 1 halo rows too; each block also
+// writes the zeros of its share of the masked frames' dx (an equal share of the sequence of
+// masked frames, len_b <= t < T), while its first tiles load.  Two sets of accumulators per
+// thread: one block per SM.
+template <typename T, int V, int KB, bool FUSED = false>
 struct DwSpanShape {
     static constexpr int CONS = kDwConsumers;
     static constexpr int R = kDwR;
@@ -482,11 +487,12 @@ struct DwSpanShape {
     static constexpr int TT = CONS * R;
     static constexpr int ROWB = CT * static_cast<int>(sizeof(T));
     static constexpr int XROWS = (TT + KB - 1 + kDwSB - 1) / kDwSB * kDwSB;
-    static constexpr int DROWS = (TT + kDwSB - 1) / kDwSB * kDwSB;
+    static constexpr int DROWS = ((FUSED ? TT + KB - 1 : TT) + kDwSB - 1) / kDwSB * kDwSB;
     static constexpr int BOX_BYTES = kDwSB * ROWB;
     static constexpr int STAGE_BYTES = (XROWS + DROWS) * ROWB;
+    static constexpr int STAGES = FUSED ? 5 : kDwStages;  // one block per SM when fused: a deeper ring
     static constexpr int RED_BYTES = CONS * (KB + 1) * CT * 4;
-    static constexpr int BODY = (kDwStages * STAGE_BYTES > RED_BYTES) ? kDwStages * STAGE_BYTES : RED_BYTES;
+    static constexpr int BODY = (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
     static constexpr int SMEM = 128 + BODY;  // plus the item tables, sized at launch
 };
 
@@ -495,27 +501,31 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
 }
 
 // PACKED: x and dy [N][C], `lengths` = offsets[B+1] (clamped into [0, N], non-decreasing), Tn = N.
-template <typename T, int V, int KB, bool PACKED>
-__global__ void __launch_bounds__(DwSpanShape<T, V, KB>::THREADS, kDwBlocks)
+template <typename T, int V, int KB, bool PACKED, bool FUSED = false>
+__global__ void __launch_bounds__(DwSpanShape<T, V, KB, FUSED>::THREADS, FUSED ? 1 : kDwBlocks)
 conv1d_dw_span_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
                       const int32_t *__restrict__ lengths, float *__restrict__ partials, int B, int Tn, int C,
-                      int K, int k_off, int pad_left, int with_bias) {
-    using S = DwSpanShape<T, V, KB>;
+                      int K, int k_off, int pad_left, int with_bias, const float *__restrict__ wgt,
+                      T *__restrict__ dx) {
+    static_assert(!(PACKED && FUSED), "the one-pass backward takes padded batches");
+    using S = DwSpanShape<T, V, KB, FUSED>;
+    const int padR = K - 1 - pad_left;  // the data gradient's left pad
     constexpr int NP = Pairs<V>::n;
     constexpr int R = S::R;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw);
-    uint64_t *empty = full + kDwStages;
+    uint64_t *empty = full + S::STAGES;
     unsigned char *stages = smem_raw + 128;
-    // per item: valid frames before it (pv), its valid frames (plen) and its first row (pst)
+    // per item: valid frames before it (pv), its valid frames (plen), its first row (pst) and
+    // (FUSED) its masked frames before it (pm)
     int *pv = reinterpret_cast<int *>(stages + S::BODY);
-    int *plen = pv + (B + 1), *pst = plen + B;
+    int *plen = pv + (B + 1), *pst = plen + B, *pm = pst + B;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int jj = static_cast<int>(blockIdx.x), G = static_cast<int>(gridDim.x), ct = static_cast<int>(blockIdx.y);
     const int c0 = ct * S::CT;
     launch_dependents();  // the finalize may be scheduled now; it waits for this grid to finish
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kDwStages; ++i) {
+        for (int i = 0; i < S::STAGES; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], S::CONS);
         }
@@ -545,19 +555,29 @@ conv1d_dw_span_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_con
         pst[bb] = s0;
     }
     __syncthreads();
-    if (warp == 0) {  // prefix sums of the valid frames
-        int run = 0;
-        if (lane == 0) pv[0] = 0;
+    if (warp == 0) {  // prefix sums of the valid (and, FUSED, of the masked) frames
+        int run = 0, run_m = 0;
+        if (lane == 0) {
+            pv[0] = 0;
+            if (FUSED) pm[0] = 0;
+        }
         for (int base = 0; base < B; base += 32) {
             const int bb = base + lane;
-            int v = bb < B ? plen[bb] : 0;
+            int v = bb < B ? plen[bb] : 0, m = bb < B ? Tn - plen[bb] : 0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += t;
+                const int t = __shfl_up_sync(0xffffffffu, v, o), tm = __shfl_up_sync(0xffffffffu, m, o);
+                if (lane >= o) {
+                    v += t;
+                    m += tm;
+                }
             }
-            if (bb < B) pv[bb + 1] = run + v;
+            if (bb < B) {
+                pv[bb + 1] = run + v;
+                if (FUSED) pm[bb + 1] = run_m + m;
+            }
             run += __shfl_sync(0xffffffffu, v, 31);
+            run_m += __shfl_sync(0xffffffffu, m, 31);
         }
     }
     __syncthreads();
@@ -586,20 +606,22 @@ conv1d_dw_span_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_con
         for (int p = v_begin; p < v_end; ++it) {
             int t0, n;
             tile_at(p, b, t0, n);
-            const int s = it % kDwStages;
-            const uint32_t ph = (it / kDwStages) & 1;
+            const int s = it % S::STAGES;
+            const uint32_t ph = (it / S::STAGES) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) break;
             if (lane == 0) {
-                const int nbx = (n + KB - 1 + kDwSB - 1) / kDwSB, nby = (n + kDwSB - 1) / kDwSB;
+                const int nbx = (n + KB - 1 + kDwSB - 1) / kDwSB;
+                const int nby = ((FUSED ? n + KB - 1 : n) + kDwSB - 1) / kDwSB;
                 unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES;
                 mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>((nbx + nby) * S::BOX_BYTES));
-                // padded: frames of item b of the [B][T][C] maps; packed: rows of the [1][N][C] maps
+                // padded: frames of item b of the [B][T][C] maps; packed: rows of the [1][N][C] maps.
+                // FUSED: the dy rows start K-1-pad_left frames early (the data gradient's halo).
                 const int r0 = PACKED ? pst[b] : 0, bi = PACKED ? 0 : b;
+                const int d0 = r0 + t0 - (FUSED ? padR : 0);
                 for (int i = 0; i < nbx; ++i)
                     tma_load_3d(st + i * S::BOX_BYTES, &xmap, c0, r0 + t0 + k_off - pad_left + i * kDwSB, bi, &full[s]);
                 for (int i = 0; i < nby; ++i)
-                    tma_load_3d(st + S::XROWS * S::ROWB + i * S::BOX_BYTES, &dmap, c0, r0 + t0 + i * kDwSB, bi,
-                                &full[s]);
+                    tma_load_3d(st + S::XROWS * S::ROWB + i * S::BOX_BYTES, &dmap, c0, d0 + i * kDwSB, bi, &full[s]);
             }
             __syncwarp();
             p += n;
@@ -607,20 +629,79 @@ conv1d_dw_span_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_con
     } else {  // consumer warp cw: frames [t0 + cw R, t0 + cw R + R) of every tile
         const int cw = warp - 1;
         const bool active = c0 + lane * V < C;
+        float2 wv[FUSED ? KB : 1][NP];  // the data gradient's taps, this thread's channels
+        if constexpr (FUSED) {
+            if (active) {
+#pragma unroll
+                for (int k = 0; k < KB; ++k) load_param<V>(wgt + static_cast<int64_t>(k) * C + c0 + lane * V, wv[k]);
+            }
+            // this block's share of the masked frames: dx zeros, issued while the first tiles load
+            const int m_begin = static_cast<int>(static_cast<int64_t>(pm[B]) * jj / G);
+            const int m_end = static_cast<int>(static_cast<int64_t>(pm[B]) * (jj + 1) / G);
+            if (active && m_begin + cw < m_end) {
+                int mb = TileOrder::find(pm, B, m_begin + cw);
+                for (int m = m_begin + cw; m < m_end; m += S::CONS) {
+                    while (pm[mb + 1] <= m) ++mb;
+                    const int t = plen[mb] + (m - pm[mb]);
+                    Vec<T, V>::store_zero(dx + (static_cast<int64_t>(mb) * Tn + t) * C + c0 + lane * V);
+                }
+            }
+        }
         int b = v_begin < v_end ? TileOrder::find(pv, B, v_begin) : 0;
         int it = 0;
         for (int p = v_begin; p < v_end; ++it) {
             int t0, n;
             tile_at(p, b, t0, n);
-            const int s = it % kDwStages;
-            const uint32_t ph = (it / kDwStages) & 1;
+            const int s = it % S::STAGES;
+            const uint32_t ph = (it / S::STAGES) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) break;
             const int tg = t0 + cw * R;   // this warp's first frame
             const int nr = n - cw * R;    // its frame count (R at most; none when <= 0)
+            if constexpr (FUSED) {
+                // data gradient of this warp's frames: dy tile row i holds frame tg - padR + i - cw R
+                if (active && nr > 0) {
+                    const int L = plen[b];
+                    T *dxp = dx + (static_cast<int64_t>(b) * Tn + tg) * C + c0 + lane * V;
+                    const unsigned char *zp = stages + static_cast<size_t>(s) * S::STAGE_BYTES + lane * V * sizeof(T) +
+                                              (S::XROWS + cw * R) * S::ROWB;
+                    const int f0 = tg - padR;  // frame of this warp's first dy row
+                    auto dxrun = [&](auto check) {
+                        constexpr bool CHECK = decltype(check)::value;
+                        float2 da[R][NP];
+#pragma unroll
+                        for (int r = 0; r < R; ++r)
+#pragma unroll
+                            for (int q = 0; q < NP; ++q) da[r][q] = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int i = 0; i < R + KB - 1; ++i) {
+                            Vec<T, V> v;
+                            v.r = *reinterpret_cast<const decltype(v.r) *>(zp + i * S::ROWB);
+                            if constexpr (CHECK) {  // frames outside [0, len_b), and rows past this warp's reach
+                                if (f0 + i < 0 || f0 + i >= L || i >= nr + KB - 1) v.zero();
+                            }
+                            float2 z[NP];
+                            v.to_f2(z);
+#pragma unroll
+                            for (int k = 0; k < KB; ++k) {
+                                const int r = i - (KB - 1) + k;
+                                if (r >= 0 && r < R) {
+#pragma unroll
+                                    for (int q = 0; q < NP; ++q) da[r][q] = ffma2(z[q], wv[k][q], da[r][q]);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < R; ++r)
+                            if (!CHECK || r < nr) Vec<T, V>::store(dxp + static_cast<int64_t>(r) * C, da[r]);
+                    };
+                    if (nr >= R && f0 >= 0 && f0 + R + KB - 1 <= L) dxrun(std::false_type{});
+                    else dxrun(std::true_type{});
+                }
+            }
             if (active && nr > 0) {
                 const int L = plen[b];
                 const unsigned char *st = stages + static_cast<size_t>(s) * S::STAGE_BYTES + lane * V * sizeof(T);
-                const unsigned char *dp = st + (S::XROWS + cw * R) * S::ROWB;
+                const unsigned char *dp = st + (S::XROWS + (FUSED ? padR : 0) + cw * R) * S::ROWB;
                 const unsigned char *xp = st + (cw * R) * S::ROWB;
                 const int jb = tg + k_off - pad_left;  // frame of this warp's first x row
                 // CHECK = false: all R frames are this warp's and every x row is inside [0, len_b).
@@ -937,14 +1018,15 @@ cudaError_t launch_tma_pass(const DwArgs &a, int k_off, int with_bias, int *gp_o
 // The span-balanced kernel for a padded batch (offsets == null) or a packed one: grid (G, channel
 // tiles), G = the blocks per channel tile that fit on the device at once, at most a.G (the
 // workspace's partial rows) and no more than the frames fill tiles of TT.
-template <typename T, int V, int KB>
+template <typename T, int V, int KB, bool FUSED = false>
 cudaError_t launch_span_pass(const DwArgs &a, const int32_t *offsets, int *gp_out, cudaStream_t s) {
-    using S = DwSpanShape<T, V, KB>;
+    using S = DwSpanShape<T, V, KB, FUSED>;
     const bool packed = offsets != nullptr;
-    auto kern = packed ? conv1d_dw_span_kernel<T, V, KB, true> : conv1d_dw_span_kernel<T, V, KB, false>;
-    const int smem = S::SMEM + static_cast<int>((3 * a.B + 1) * sizeof(int));
+    auto kern = FUSED ? conv1d_dw_span_kernel<T, V, KB, false, FUSED>
+                      : (packed ? conv1d_dw_span_kernel<T, V, KB, true> : conv1d_dw_span_kernel<T, V, KB, false>);
+    const int smem = S::SMEM + static_cast<int>((4 * a.B + 2) * sizeof(int));
     const cudaError_t attr = ensure_smem_attr(reinterpret_cast<const void *>(kern),
-                                              S::SMEM + static_cast<int>((3 * kOrderMaxItems + 1) * sizeof(int)));
+                                              S::SMEM + static_cast<int>((4 * kOrderMaxItems + 2) * sizeof(int)));
     if (attr != cudaSuccess) return attr;
     const int64_t nCT = (a.C + S::CT - 1) / S::CT;
     if (nCT > 65535) return cudaErrorInvalidConfiguration;
@@ -976,7 +1058,8 @@ cudaError_t launch_span_pass(const DwArgs &a, const int32_t *offsets, int *gp_ou
     cfg.attrs = at;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, xmap, dmap, packed ? offsets : a.lengths, a.partials, static_cast<int>(a.B),
-                              static_cast<int>(a.T), static_cast<int>(a.C), a.K, 0, a.pad_left, 1);
+                              static_cast<int>(a.T), static_cast<int>(a.C), a.K, 0, a.pad_left, 1, a.w,
+                              static_cast<T *>(a.dx));
 }
 
 template <typename T>
@@ -1063,6 +1146,33 @@ cudaError_t launch_dtype(const DwArgs &a, int *gp, cudaStream_t s) {
 template <typename T>
 cudaError_t launch_fused_partials(const DwArgs &a, int *gp, cudaStream_t s) {
     if (!dw_tma_ok<T>(a) || a.vec_width < 2) return cudaErrorNotSupported;
+    if (a.B <= kOrderMaxItems) {  // the span-balanced kernel in its one-pass form
+        if constexpr (sizeof(T) == 2) {
+            if (a.vec_width >= 4) {
+                switch (a.K) {
+                    case 1: return launch_span_pass<T, 4, 1, true>(a, nullptr, gp, s);
+                    case 2: return launch_span_pass<T, 4, 2, true>(a, nullptr, gp, s);
+                    case 3: return launch_span_pass<T, 4, 3, true>(a, nullptr, gp, s);
+                    case 4: return launch_span_pass<T, 4, 4, true>(a, nullptr, gp, s);
+                    case 5: return launch_span_pass<T, 4, 5, true>(a, nullptr, gp, s);
+                    case 7: return launch_span_pass<T, 4, 7, true>(a, nullptr, gp, s);
+                    case 9: return launch_span_pass<T, 4, 9, true>(a, nullptr, gp, s);
+                    default: break;
+                }
+            }
+        }
+        switch (a.K) {
+            case 1: return launch_span_pass<T, 2, 1, true>(a, nullptr, gp, s);
+            case 2: return launch_span_pass<T, 2, 2, true>(a, nullptr, gp, s);
+            case 3: return launch_span_pass<T, 2, 3, true>(a, nullptr, gp, s);
+            case 4: return launch_span_pass<T, 2, 4, true>(a, nullptr, gp, s);
+            case 5: return launch_span_pass<T, 2, 5, true>(a, nullptr, gp, s);
+            case 7: return launch_span_pass<T, 2, 7, true>(a, nullptr, gp, s);
+            case 9: return launch_span_pass<T, 2, 9, true>(a, nullptr, gp, s);
+            case 15: return launch_span_pass<T, 2, 15, true>(a, nullptr, gp, s);
+            default: return cudaErrorNotSupported;
+        }
+    }
     if constexpr (sizeof(T) == 2) {
         if (a.vec_width >= 4) {
             switch (a.K) {
