@@ -604,7 +604,8 @@ def kernel_source_sha():
 
 
 def ncu_traffic(kernel):
-    """DRAM bytes per launch recorded from an ncu capture, if the kernels have not changed since."""
+    """Bytes per launch recorded from an ncu capture, if the kernels have not changed since:
+    (DRAM bytes read + bytes the SMs wrote into L2, dram read, SM writes), else None."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         rows = [dict(kv.split("=", 1) for kv in line.split()) for line in open(path)
@@ -614,7 +615,8 @@ def ncu_traffic(kernel):
     sha = kernel_source_sha()
     for r in rows:
         if r.get("kernel") == kernel and r.get("sha") == sha:
-            return float(r["dram_bytes_per_launch"])
+            rd, wr = float(r["dram_read"]), float(r["sm_write"])
+            return rd + wr, rd, wr
     return None
 
 
@@ -1037,6 +1039,7 @@ def main():
                           reasons=sorted(set(clocks["reasons"]) | clk_rows.reasons),
                           samples=len(clk.samples) + len(clk_rows.samples))
         simt = configs.get("subsampler", {}).get("sym_fp32_simt")
+        tc_traffic = ncu_traffic("dw_subsample_tc_kernel")
         tc_us = ms * 1e3
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
@@ -1056,7 +1059,12 @@ def main():
             "configs": configs,
             "roofline": {"bound": "hbm", "kernel": "dw_subsample_tc_kernel",
                          "achieved": sb / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                         "frac": sb / (ms * 1e-3) / 1e9 / hbm, "traffic": ncu_traffic("dw_subsample_tc_kernel"),
+                         "frac": sb / (ms * 1e-3) / 1e9 / hbm,
+                         "traffic": tc_traffic[0] if tc_traffic else None,
+                         "traffic_split": {"dram_read": tc_traffic[1], "sm_write_to_l2": tc_traffic[2],
+                                           "method": "ncu dram__bytes_read.sum + 32 x "
+                                                     "lts__t_sectors_srcunit_tex_op_write.sum, one launch"}
+                         if tc_traffic else None,
                          "peak_kind": f"{peak_kind} HBM copy bandwidth",
                          "note": "the step's dominant kernel, bound by HBM on the resources it uses: conv0 runs on "
                                  "tcgen05 (TF32 3-product split), ReLU and conv_dw1 on the FP32 pipes "

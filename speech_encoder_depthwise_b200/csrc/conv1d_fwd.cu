@@ -126,8 +126,9 @@ conv1d_fwd_vec_kernel(const T *__restrict__ x, const float *__restrict__ w,
 // read at all.
 // ---------------------------------------------------------------------------------------
 // Tuned on B200 (sweeps over consumer warps, frames per thread, ring depth, blocks per SM and
-// tile width): 3 blocks of 4 consumer warps per SM, 3 stages, 12 frames per thread (16 for
-// K > 9), tiles 128 channels wide (256-byte bf16 rows; narrower rows cost DRAM efficiency).
+// tile width): 3 blocks of 4 consumer warps per SM, 3 stages, 12 frames per thread (K = 15: 8
+// with 4 channels a thread, 16 with 2), tiles 128 channels wide (256-byte bf16 rows; narrower
+// rows cost DRAM efficiency).
 #ifndef DW_FWD_CONSUMERS
 #define DW_FWD_CONSUMERS 4
 #endif
@@ -147,6 +148,10 @@ conv1d_fwd_vec_kernel(const T *__restrict__ x, const float *__restrict__ w,
 constexpr int kTmaConsumers = DW_FWD_CONSUMERS;  // consumer warps per block
 constexpr int kTmaR = DW_FWD_R;                  // frames per consumer thread, K <= 9
 constexpr int kTmaRWide = DW_FWD_R_WIDE;         // frames per consumer thread, K > 9
+#ifndef DW_FWD_R_WIDE4
+#define DW_FWD_R_WIDE4 8
+#endif
+constexpr int kTmaRWide4 = DW_FWD_R_WIDE4;       // frames per consumer thread, K = 15 with 4 channels
 constexpr int kTmaStages = DW_FWD_STAGES;        // shared-memory ring depth
 constexpr int kTmaBlocks = DW_FWD_BLOCKS;        // resident blocks per SM
 
@@ -154,7 +159,7 @@ constexpr int kTmaThreads = 32 * (1 + kTmaConsumers);
 
 template <typename T, int V, int K>
 struct TmaShape {
-    static constexpr int R = (K > 9) ? kTmaRWide : kTmaR;
+    static constexpr int R = (K > 9) ? (V >= 4 ? kTmaRWide4 : kTmaRWide) : kTmaR;
     static constexpr int WPR = (V >= 4) ? 1 : 2;      // consumer warps side by side: 128-channel tiles
     static constexpr int CT = 32 * V * WPR;           // channels per tile
     static constexpr int TT = (kTmaConsumers / WPR) * R;  // output frames per tile
@@ -625,7 +630,7 @@ cudaError_t dispatch_k(const Conv1dArgs &a, cudaStream_t s) {
                 case 9: return launch_tma<T, V, 9>(a, s);
                 default: break;
             }
-            if constexpr (V == 2) {
+            if constexpr (V == 2 || V == 4) {
                 if (a.K == 15) return launch_tma<T, V, 15>(a, s);
             }
         }
@@ -648,13 +653,14 @@ cudaError_t dispatch_k(const Conv1dArgs &a, cudaStream_t s) {
 
 template <typename T>
 cudaError_t dispatch_dtype(const Conv1dArgs &a, cudaStream_t s) {
-    // 4 bf16 channels (8 bytes) per thread up to K = 9; pairs for wider kernels and for
-    // float32 (8 bytes), which keeps the register window under 128 registers.
+    // 4 bf16 channels (8 bytes) per thread up to K = 9, and for K = 15 on the pipelined kernel with
+    // 8 frames per thread (26.0 against 27.9 us for pairs at 32x750x1024); pairs for other wide
+    // kernels and for float32 (8 bytes), which keeps the register window under 128 registers.
     if constexpr (sizeof(T) == 2) {
 #ifdef DW_FWD_V8
         if (a.vec_width >= 8 && a.K <= 9) return dispatch_k<T, 8>(a, s);
 #endif
-        if (a.vec_width >= 4 && a.K <= 9) return dispatch_k<T, 4>(a, s);
+        if (a.vec_width >= 4 && (a.K <= 9 || (a.K == 15 && tma_ok<T>(a)))) return dispatch_k<T, 4>(a, s);
     }
     if (a.vec_width >= 2) return dispatch_k<T, 2>(a, s);
     return dispatch_k<T, 1>(a, s);
