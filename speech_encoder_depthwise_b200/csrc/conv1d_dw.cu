@@ -496,10 +496,6 @@ struct DwSpanShape {
     static constexpr int SMEM = 128 + BODY;  // plus the item tables, sized at launch
 };
 
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
-}
-
 // PACKED: x and dy [N][C], `lengths` = offsets[B+1] (clamped into [0, N], non-decreasing), Tn = N.
 template <typename T, int V, int KB, bool PACKED, bool FUSED = false>
 __global__ void __launch_bounds__(DwSpanShape<T, V, KB, FUSED>::THREADS, FUSED ? 1 : kDwBlocks)

@@ -369,5 +369,10 @@ namespace dwk {
 // early with launch_dependents (they still wait for its completion before reading).
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Warm L2 with the line holding p.  Safe before grid_dependency_wait: a prefetch only fills the
+// cache (L2 is where the previous kernel's writes land), so later reads still see those writes.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
+}
 
 }  // namespace dwk

@@ -76,6 +76,7 @@ constexpr int kHalfCols = kJO / 2;           // output columns per epilogue warp
 constexpr int kChunk = 5;                    // output columns per tensor-memory read
 constexpr int kRowsPer = (kN + kPatchThreads - 1) / kPatchThreads;  // patch rows per builder thread
 constexpr int kBarPatch = 1;                // named barrier id of the patch builders
+constexpr int kBarList = 2;                 // named barrier id: unit list ready (list warp + builders)
 constexpr int kGroupThreads = 128;          // one epilogue group: 4 warps, one per lane quarter
 constexpr int kListCap = 1024;              // units per block (the list lives in shared memory)
 constexpr int kOrderItems = 4096;           // items up to which the unit deal is balanced
@@ -225,8 +226,72 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
     const int nUnits = B * nIP * nJB;
     constexpr int kStElems = kRO * kJO * 128;
 
+    // ------------------------------------------------------------ patch-builder constants
+    // Builder thread pt takes rows pt, pt + 128 (< kN): the builder warps with two rows a lane
+    // are the last ones (SM sub-partitions 2 and 3), because the MMA issuer and the store
+    // thread share sub-partitions 0 and 1 with the first ones.  (Meaningless for other warps.)
+    const int pt = kPatchThreads - 1 - (static_cast<int>(threadIdx.x) - kEpiThreads);
+    // This thread's mel window elements and patch rows are the same for every unit:
+    // element k sits at window row rs >> 8, column rs & 255 (rs = -1 past the window); rows
+    // n = pt + i * kPatchThreads all share n % 8 (one swizzle pattern).
+    int mel_rs[kMelLoads];
+#pragma unroll
+    for (int k = 0; k < kMelLoads; ++k) {
+        const int e = pt + k * kPatchThreads;
+        mel_rs[k] = e < kMelElems ? ((e / kMC) << 8) | (e % kMC) : -1;
+    }
+    int row_cc[kRowsPer], row_rr[kRowsPer];
+#pragma unroll
+    for (int i = 0; i < kRowsPer; ++i) {  // the h pixel whose accumulator column is n (inverse of acc_col)
+        const int n = pt + i * kPatchThreads;
+        if (n < 192) {
+            const int v = n % 48;
+            row_cc[i] = 10 * (n / 48) + 1 + v / kHR;
+            row_rr[i] = v % kHR;
+        } else if (n < 200) {
+            const int v = 48 + (n - 192) % 2;
+            row_cc[i] = 10 * ((n - 192) / 2) + 1 + v / kHR;
+            row_rr[i] = v % kHR;
+        } else {
+            row_cc[i] = 0;
+            row_rr[i] = n - 200;
+        }
+    }
+    // The unit's mel window goes straight to shared memory with 4-byte asynchronous copies
+    // (elements outside the window's valid frames and columns are written as zero without a
+    // read), two units ahead of the one being built, in kMelStages rotating windows.
+    auto load_mel = [&](int u) {
+        const int4 e = ulist[u];  // {b, i0, j0, len}
+        float *S = mel_s_tile + (u % kMelStages) * (Lay::mel_bytes / 4);
+        const int mr0 = 4 * e.y - 3 * Pt, mc0 = 4 * e.z - 3;
+        const float *base = mel + static_cast<int64_t>(e.x) * Tn * F;
+        const bool rows_in = mr0 >= 0 && mr0 + kMR <= e.w;  // every window row is a valid frame
+#pragma unroll
+        for (int k = 0; k < kMelLoads; ++k) {
+            if (mel_rs[k] < 0) continue;
+            const int mr = mr0 + (mel_rs[k] >> 8), mc = mc0 + (mel_rs[k] & 255);
+            const bool in = (rows_in || (mr >= 0 && mr < e.w)) && mc >= 0 && mc < F;
+            cp_async4(S + (mel_rs[k] >> 8) * kMCP + (mel_rs[k] & 255), in ? base + mr * F + mc : base, in ? 4u : 0u);
+        }
+    };
+
     // ------------------------------------------------------------ set-up
-    launch_dependents();     // the next kernel in the stream may start its own set-up
+    launch_dependents();  // the next kernel in the stream may start its own set-up
+    {
+        // Warm L2 with this block's parameters (w0, w1 rows and b0, b1 over its channels) and the
+        // lengths while the previous kernel drains; the loads below then hit L2.
+        constexpr int kLines = CTG * 4;  // 128-byte lines of one parameter row over CTG x 128 channels
+        const int t = threadIdx.x, c = g * CTG * 128 + (t % kLines) * 32;
+        if (t < 10 * kLines) {
+            const int row = t / kLines;  // taps 0..8, then the bias
+            if (c < C) {
+                prefetch_l2(row < 9 ? w0 + row * C + c : b0 + c);
+                prefetch_l2(row < 9 ? w1 + row * C + c : b1 + c);
+            }
+        } else if (lengths != nullptr && B <= kOrderItems) {
+            for (int i = (t - 10 * kLines) * 32; i < B; i += (kThreads - 10 * kLines) * 32) prefetch_l2(lengths + i);
+        }
+    }
     grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -333,20 +398,28 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
             counts[0] = nA;
             counts[1] = nZ;
         }
+        named_bar(kBarList, 32 + kPatchThreads);  // the list is ready for the builders' first copies
     }
     if (warp >= kEpiWarps && warp < kMmaWarp) {
-        // A operand: split conv0 weights and bias of this block's channel tiles (K layout above)
-        const int pt = threadIdx.x - kEpiThreads;
-        for (int r = pt; r < CTG * 128; r += kPatchThreads) {
-            const int c = (g * CTG + r / 128) * 128 + r % 128;
+        // A operand: split conv0 weights and bias of this block's channel tiles (K layout above);
+        // row r of tile i is channel (g CTG + i) 128 + r, every load issued before the first use
+        const int r = threadIdx.x - kEpiThreads;
+        float xw[CTG][10];
+#pragma unroll
+        for (int i = 0; i < CTG; ++i) {
+            const int c = (g * CTG + i) * 128 + r;
+#pragma unroll
+            for (int t = 0; t < 10; ++t) xw[i][t] = c < C ? __ldg(t < 9 ? w0 + t * C + c : b0 + c) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < CTG; ++i) {
             float hi[9], lo[9];
 #pragma unroll
             for (int t = 0; t < 9; ++t) {
-                const float x = c < C ? __ldg(w0 + t * C + c) : 0.f;
-                hi[t] = tf32_hi(x);
-                lo[t] = x - hi[t];
+                hi[t] = tf32_hi(xw[i][t]);
+                lo[t] = xw[i][t] - hi[t];
             }
-            const float bx = c < C ? __ldg(b0 + c) : 0.f;
+            const float bx = xw[i][9];
             const float bhi = tf32_hi(bx);
             float4 q[8];
             q[0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
@@ -357,18 +430,33 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
             q[5] = q[1];
             q[6] = make_float4(hi[8], lo[8], hi[8], bhi);
             q[7] = make_float4(bx - bhi, 0.f, 0.f, 0.f);
-            store_k_row(tileA + (r / 128) * kTileA, r % 128, q);
+            store_k_row(tileA + i * kTileA, r, q);
         }
         fence_async_smem();
+        // the first two units' mel windows start copying before the block-wide barrier
+        named_bar(kBarList, 32 + kPatchThreads);
+        const int nA0 = counts[0];
+        if (nA0 > 0) load_mel(0);
+        cp_async_commit();
+        if (nA0 > 1) load_mel(1);
+        cp_async_commit();
     }
     if (warp < kEpiWarps) {
+        // conv_dw1 weights and bias: every load issued first, the zero tile written meanwhile
+        constexpr int kWtPer = CTG * 10 * 128 / kEpiThreads;
+        static_assert(CTG * 10 * 128 % kEpiThreads == 0, "weight table split");
+        float wv[kWtPer];
+#pragma unroll
+        for (int j = 0; j < kWtPer; ++j) {
+            const int e = threadIdx.x + j * kEpiThreads;
+            const int ct = e / 1280, t = (e / 128) % 10, c = (g * CTG + ct) * 128 + e % 128;
+            wv[j] = c < C ? __ldg(t < 9 ? w1 + t * C + c : b1 + c) : 0.f;
+        }
         TO *z = stage + 4 * kStElems;  // the zero tile stored for fully masked units
         for (int e = threadIdx.x; e < kStElems; e += kEpiThreads) stage_out<TO>(z + e, 0.f);
         fence_async_smem();
-        for (int e = threadIdx.x; e < CTG * 10 * 128; e += kEpiThreads) {  // conv_dw1 weights and bias
-            const int ct = e / 1280, t = (e / 128) % 10, c = (g * CTG + ct) * 128 + e % 128;
-            wtab[e] = c < C ? __ldg(t < 9 ? w1 + t * C + c : b1 + c) : 0.f;
-        }
+#pragma unroll
+        for (int j = 0; j < kWtPer; ++j) wtab[threadIdx.x + j * kEpiThreads] = wv[j];
         if (blockIdx.x == 0 && out_lengths != nullptr)
             for (int q = threadIdx.x; q < B; q += kEpiThreads) {
                 const int Lq = static_cast<int>(clamp_len(lengths, q, Tn));
@@ -473,57 +561,7 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         }
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ patch builders
-        // Builder thread pt takes rows pt, pt + 128 (< kN): the builder warps with two rows a lane
-        // are the last ones (SM sub-partitions 2 and 3), because the MMA issuer and the store
-        // thread share sub-partitions 0 and 1 with the first ones.
-        const int pt = kPatchThreads - 1 - (static_cast<int>(threadIdx.x) - kEpiThreads);
-        // This thread's mel window elements and patch rows are the same for every unit:
-        // element k sits at window row rs >> 8, column rs & 255 (rs = -1 past the window); rows
-        // n = pt + i * kPatchThreads all share n % 8 (one swizzle pattern).
-        int mel_rs[kMelLoads];
-#pragma unroll
-        for (int k = 0; k < kMelLoads; ++k) {
-            const int e = pt + k * kPatchThreads;
-            mel_rs[k] = e < kMelElems ? ((e / kMC) << 8) | (e % kMC) : -1;
-        }
-        int row_cc[kRowsPer], row_rr[kRowsPer];
-#pragma unroll
-        for (int i = 0; i < kRowsPer; ++i) {  // the h pixel whose accumulator column is n (inverse of acc_col)
-            const int n = pt + i * kPatchThreads;
-            if (n < 192) {
-                const int v = n % 48;
-                row_cc[i] = 10 * (n / 48) + 1 + v / kHR;
-                row_rr[i] = v % kHR;
-            } else if (n < 200) {
-                const int v = 48 + (n - 192) % 2;
-                row_cc[i] = 10 * ((n - 192) / 2) + 1 + v / kHR;
-                row_rr[i] = v % kHR;
-            } else {
-                row_cc[i] = 0;
-                row_rr[i] = n - 200;
-            }
-        }
-        // The unit's mel window goes straight to shared memory with 4-byte asynchronous copies
-        // (elements outside the window's valid frames and columns are written as zero without a
-        // read), two units ahead of the one being built, in kMelStages rotating windows.
-        auto load_mel = [&](int u) {
-            const int4 e = ulist[u];  // {b, i0, j0, len}
-            float *S = mel_s_tile + (u % kMelStages) * (Lay::mel_bytes / 4);
-            const int mr0 = 4 * e.y - 3 * Pt, mc0 = 4 * e.z - 3;
-            const float *base = mel + static_cast<int64_t>(e.x) * Tn * F;
-            const bool rows_in = mr0 >= 0 && mr0 + kMR <= e.w;  // every window row is a valid frame
-#pragma unroll
-            for (int k = 0; k < kMelLoads; ++k) {
-                if (mel_rs[k] < 0) continue;
-                const int mr = mr0 + (mel_rs[k] >> 8), mc = mc0 + (mel_rs[k] & 255);
-                const bool in = (rows_in || (mr >= 0 && mr < e.w)) && mc >= 0 && mc < F;
-                cp_async4(S + (mel_rs[k] >> 8) * kMCP + (mel_rs[k] & 255), in ? base + mr * F + mc : base, in ? 4u : 0u);
-            }
-        };
-        if (nA > 0) load_mel(0);
-        cp_async_commit();
-        if (nA > 1) load_mel(1);
-        cp_async_commit();
+        // (the first two units' mel windows were requested during the set-up)
         bool ok = true;
         for (int idx = 0; idx < nA && ok; ++idx) {
             const int4 e = ulist[idx];
