@@ -203,6 +203,23 @@ conv1d_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__r
         }
         fence_barrier_init();
     }
+    if constexpr (!PACKED) {
+        // While the previous kernel drains, warm L2 with this block's first ring-full of tiles (the
+        // same boxes the producer copies after the wait), its taps and bias, and the lengths.
+        if (threadIdx.x == 0) {
+            prefetch_tmap(&xmap);
+            for (int i = 0, q = q0; i < kTmaStages && q < nq; ++i, q += qstride)
+                tma_prefetch_3d(&xmap, my_ct * S::CT, (q % nT) * S::TT - pad_left, q / nT);
+        } else if (warp == 1) {  // taps and bias over the tile's channels: (K + 1) rows of CT floats
+            constexpr int kLines = S::CT * 4 / 128;
+            for (int i = lane; i < (K + 1) * kLines; i += 32) {
+                const int row = i / kLines, c = my_ct * S::CT + (i % kLines) * 32;
+                if (c < C && (row < K || bias != nullptr)) prefetch_l2(row < K ? w + static_cast<int64_t>(row) * C + c : bias + c);
+            }
+        } else if (warp == 2 && lengths != nullptr) {
+            for (int i = lane * 32; i < B; i += 32 * 32) prefetch_l2(lengths + i);
+        }
+    }
     grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     if constexpr (PACKED) {
         if (warp == 0) {  // offsets are clamped into [0, N] and made non-decreasing

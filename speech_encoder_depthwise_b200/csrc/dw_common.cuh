@@ -271,6 +271,15 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int c, 
         : "memory");
 }
 
+// L2 prefetch of one tensor box (no shared-memory destination, no completion to wait for).  Safe
+// before grid_dependency_wait for the same reason as prefetch_l2: it only fills the cache.
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int c, int t, int b) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c), "r"(t), "r"(b)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
