@@ -785,6 +785,7 @@ __global__ void __launch_bounds__(256)
 conv1d_dw_finalize_kernel(const float *__restrict__ partials, float *__restrict__ dw,
                           float *__restrict__ dbias, int Gp, int K, int64_t C) {
     __shared__ float red[8][33];
+    launch_dependents();     // the next kernel may start its own set-up
     grid_dependency_wait();  // launched programmatically after the partial kernel
     const int col = threadIdx.x % 32, rg = threadIdx.x / 32;
     const int64_t E = static_cast<int64_t>(K + 1) * C;
@@ -814,6 +815,7 @@ __global__ void __launch_bounds__(256)
 conv1d_dw_finalize4_kernel(const float *__restrict__ partials, float *__restrict__ dw,
                            float *__restrict__ dbias, int Gp, int K, int64_t C) {
     __shared__ float4 red[kFinGroups][16];
+    launch_dependents();     // the next kernel may start its own set-up
     grid_dependency_wait();  // launched programmatically after the partial kernel
     const int lane = threadIdx.x % 16, rg = threadIdx.x / 16;
     const int64_t E4 = static_cast<int64_t>(K + 1) * C / 4;
