@@ -356,9 +356,8 @@ cudaError_t conv2d_dw_launch(const Conv2dArgs &a, float *dw, float *dbias, float
         const cudaError_t e = conv2d_dw_tma_partials(a, partials, conv2d_dw_partial_rows(a.B, a.To), &Gt, s);
         if (e != cudaErrorNotSupported) {
             if (e != cudaSuccess) return e;
-            dwconv2d_dw_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(
-                partials, Gt, ntap, static_cast<int>(a.C), dw, dbias);
-            return cudaGetLastError();
+            // the same [rows][taps + 1][C] layout as the conv1d weight gradient
+            return launch_finalize_rows(partials, dw, dbias, Gt, ntap, a.C, s);
         }
     }
     const int64_t nCG = (a.C + 2 * kC2Threads - 1) / (2 * kC2Threads);

@@ -28,6 +28,27 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c, 
         : "memory");
 }
 
+// L2 prefetch of one tensor box (no destination, nothing to wait for): safe before the dependency
+// wait, since it only fills the cache.
+__device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int c, int f, int t, int b) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c), "r"(f), "r"(t), "r"(b)
+                 : "memory");
+}
+
+// Before the dependency wait: the taps (9 rows over the slab's CS channels) and the lengths into L2.
+__device__ __forceinline__ void c2_prefetch_params(const float *w, const int32_t *lengths, int C, int c0, int CS, int B,
+                                                   int tid, int nthreads) {
+    const int lines = (CS * 4 + 127) / 128;
+    for (int i = tid; i < 9 * lines; i += nthreads) {
+        const int c = c0 + (i % lines) * 32;
+        if (w != nullptr && c < C) prefetch_l2(w + static_cast<int64_t>(i / lines) * C + c);
+    }
+    if (lengths != nullptr)
+        for (int i = tid * 32; i < B; i += nthreads * 32) prefetch_l2(lengths + i);
+}
+
 __device__ __forceinline__ int out_len(const int32_t *lengths, int b, int Tn, int pt, int pb, int st, int To) {
     const int L = static_cast<int>(clamp_len(lengths, b, Tn));
     const int m = L + pt + pb - 3;
@@ -99,12 +120,22 @@ c2_fwd_tma_kernel(const __grid_constant__ CUtensorMap xmap, const float *__restr
     const int cv = tid % CSV, jl = tid / CSV;
     const bool active = jl < g.TJ;
     const int ntiles = g.B * g.nI * g.nJ * g.nCS;
+    launch_dependents();  // the next kernel in the stream may start its own set-up
     if (tid == 0) {
         prefetch_tmap(&xmap);
         mbar_init(&sm.full[0], 1);
         mbar_init(&sm.full[1], 1);
         fence_barrier_init();
+        if (static_cast<int>(blockIdx.x) < ntiles) {  // the first tile's box, before its length is known
+            int b, it, jt, cs;
+            decode(g, blockIdx.x, b, it, jt, cs);
+            tma_prefetch_4d(&xmap, cs * g.CS, jt * g.TJ * g.sf - g.pf, it * g.TI * g.st - g.pt, b);
+        }
+    } else {
+        c2_prefetch_params(w, lengths, g.C, (static_cast<int>(blockIdx.x) % g.nCS) * g.CS, g.CS, g.B, tid - 1,
+                           static_cast<int>(blockDim.x) - 1);
     }
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     if (blockIdx.x == 0 && out_lengths != nullptr)
         for (int b = tid; b < g.B; b += blockDim.x) out_lengths[b] = out_len(lengths, b, g.T, g.pt, g.pb, g.st, g.To);
     __syncthreads();
@@ -253,14 +284,24 @@ c2_dx_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restri
     const int cv = tid % CSV, jl = tid / CSV;
     const bool active = jl < g.TJ;
     const int ntiles = g.B * g.nI * g.nJ * g.nCS;
+    auto floordiv = [](int a, int d) { return a >= 0 ? a / d : -((-a + d - 1) / d); };
+    launch_dependents();  // the next kernel in the stream may start its own set-up
     if (tid == 0) {
         prefetch_tmap(&gmap);
         mbar_init(&sm.full[0], 1);
         mbar_init(&sm.full[1], 1);
         fence_barrier_init();
+        if (static_cast<int>(blockIdx.x) < ntiles) {  // the first tile's box, before its length is known
+            int b, it, jt, cs;
+            decode(g, blockIdx.x, b, it, jt, cs);
+            tma_prefetch_4d(&gmap, cs * g.CS, floordiv(jt * g.TJ + g.pf - 2, g.sf), floordiv(it * g.TI + g.pt - 2, g.st), b);
+        }
+    } else {
+        c2_prefetch_params(w, lengths, g.C, (static_cast<int>(blockIdx.x) % g.nCS) * g.CS, g.CS, g.B, tid - 1,
+                           static_cast<int>(blockDim.x) - 1);
     }
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     __syncthreads();
-    auto floordiv = [](int a, int d) { return a >= 0 ? a / d : -((-a + d - 1) / d); };
     auto valid = [&](int tile) {
         int b, it, jt, cs;
         decode(g, tile, b, it, jt, cs);
@@ -384,14 +425,24 @@ c2_dx2_tma_kernel(const __grid_constant__ CUtensorMap gmap, const float *__restr
     const int cv = tid % CSV, m = tid / CSV;
     const bool active = m < g.TJ / 2;
     const int ntiles = g.B * g.nI * g.nJ * g.nCS;
+    auto floordiv = [](int a, int d) { return a >= 0 ? a / d : -((-a + d - 1) / d); };
+    launch_dependents();  // the next kernel in the stream may start its own set-up
     if (tid == 0) {
         prefetch_tmap(&gmap);
         mbar_init(&sm.full[0], 1);
         mbar_init(&sm.full[1], 1);
         fence_barrier_init();
+        if (static_cast<int>(blockIdx.x) < ntiles) {  // the first tile's box, before its length is known
+            int b, it, jt, cs;
+            decode(g, blockIdx.x, b, it, jt, cs);
+            tma_prefetch_4d(&gmap, cs * g.CS, floordiv(jt * g.TJ + g.pf - 1, 2), floordiv(it * g.TI + g.pt - 1, 2), b);
+        }
+    } else {
+        c2_prefetch_params(w, lengths, g.C, (static_cast<int>(blockIdx.x) % g.nCS) * g.CS, g.CS, g.B, tid - 1,
+                           static_cast<int>(blockDim.x) - 1);
     }
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
     __syncthreads();
-    auto floordiv = [](int a, int d) { return a >= 0 ? a / d : -((-a + d - 1) / d); };
     auto valid = [&](int tile) {
         int b, it, jt, cs;
         decode(g, tile, b, it, jt, cs);
@@ -527,20 +578,30 @@ c2_dw_tma_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant
     const int cs = blockIdx.x % g.nCS, gi = blockIdx.x / g.nCS;
     const int c = cs * g.CS + cv * kC2V;
     const int ntiles = g.B * g.nI * g.nJ;  // tiles of one slab
-    if (tid == 0) {
-        prefetch_tmap(&xmap);
-        prefetch_tmap(&gmap);
-        mbar_init(&sm.full[0], 1);
-        mbar_init(&sm.full[1], 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
     auto dec = [&](int tile, int &b, int &it, int &jt) {
         jt = tile % g.nJ;
         const int r = tile / g.nJ;
         it = r % g.nI;
         b = r / g.nI;
     };
+    launch_dependents();  // the finalize may be scheduled now; it waits for this grid to finish
+    if (tid == 0) {
+        prefetch_tmap(&xmap);
+        prefetch_tmap(&gmap);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
+        if (gi < ntiles) {  // the first tile's boxes, before its length is known
+            int b, it, jt;
+            dec(gi, b, it, jt);
+            tma_prefetch_4d(&xmap, cs * g.CS, jt * g.TJ * g.sf - g.pf, it * g.TI * g.st - g.pt, b);
+            tma_prefetch_4d(&gmap, cs * g.CS, jt * g.TJ, it * g.TI, b);
+        }
+    } else if (lengths != nullptr) {
+        for (int i = (tid - 1) * 32; i < g.B; i += (static_cast<int>(blockDim.x) - 1) * 32) prefetch_l2(lengths + i);
+    }
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
+    __syncthreads();
     auto valid = [&](int tile) {
         int b, it, jt;
         dec(tile, b, it, jt);
@@ -761,8 +822,8 @@ cudaError_t fwd_tma(const Conv2dArgs &a, cudaStream_t s) {
     gridl = gridl / g.nCS * g.nCS;  // whole channel slabs per block (its taps stay in registers)
     if (gridl < g.nCS) gridl = g.nCS;
     const int grid = static_cast<int>(gridl);
-    kern<<<grid, threads, smem, s>>>(map, a.w, a.bias, static_cast<T *>(a.y), a.lengths, a.out_lengths, g);
-    return cudaGetLastError();
+    return launch_programmatic(kern, dim3(grid), dim3(threads), smem, s, map, a.w, a.bias, static_cast<T *>(a.y),
+                               a.lengths, a.out_lengths, g);
 }
 
 // Stride 2 x 2: the 2x2-block kernel.  Tiles of TI (even) dx rows x TJ (even) columns; the box
@@ -811,8 +872,7 @@ cudaError_t dx2_tma(const Conv2dArgs &a, cudaStream_t s) {
     gridl = gridl / g.nCS * g.nCS;  // whole channel slabs per block (its taps stay in registers)
     if (gridl < g.nCS) gridl = g.nCS;
     const int grid = static_cast<int>(gridl);
-    kern<<<grid, threads, smem, s>>>(map, a.w, static_cast<T *>(a.y), a.lengths, g);
-    return cudaGetLastError();
+    return launch_programmatic(kern, dim3(grid), dim3(threads), smem, s, map, a.w, static_cast<T *>(a.y), a.lengths, g);
 }
 
 template <typename T>
@@ -859,8 +919,7 @@ cudaError_t dx_tma(const Conv2dArgs &a, cudaStream_t s) {
     gridl = gridl / g.nCS * g.nCS;  // whole channel slabs per block (its taps stay in registers)
     if (gridl < g.nCS) gridl = g.nCS;
     const int grid = static_cast<int>(gridl);
-    kern<<<grid, threads, smem, s>>>(map, a.w, static_cast<T *>(a.y), a.lengths, g);
-    return cudaGetLastError();
+    return launch_programmatic(kern, dim3(grid), dim3(threads), smem, s, map, a.w, static_cast<T *>(a.y), a.lengths, g);
 }
 
 template <typename T>
@@ -911,10 +970,9 @@ cudaError_t dw_tma(const Conv2dArgs &a, float *partials, int max_rows, int *G_ou
     if (G > ntiles) G = ntiles;
     if (G > max_rows) G = max_rows;
     if (G < 1) G = 1;
-    kern<<<static_cast<unsigned>(G * g.nCS), threads, smem, s>>>(xm, gm, a.lengths, partials, g, static_cast<int>(G),
-                                                                 xbytes);
     *G_out = static_cast<int>(G);
-    return cudaGetLastError();
+    return launch_programmatic(kern, dim3(static_cast<unsigned>(G * g.nCS)), dim3(threads), smem, s, xm, gm, a.lengths,
+                               partials, g, static_cast<int>(G), xbytes);
 }
 
 }  // namespace

@@ -101,6 +101,24 @@ cudaError_t make_act_map(CUtensorMap *map, const void *base, int dtype, int64_t 
 
 int sm_count();
 
+// Launch with programmatic stream serialization: the kernel may start while the previous one in
+// the stream drains, and must call grid_dependency_wait before touching memory that one writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_programmatic(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 cudaError_t conv1d_fwd_launch(const Conv1dArgs &a, cudaStream_t s);
 // Packed sequences: a.B items, a.T = N rows of x/y [N][C], item b on rows offsets[b] .. offsets[b+1]-1.
 cudaError_t conv1d_fwd_packed_launch(const Conv1dArgs &a, const int32_t *offsets, cudaStream_t s);
@@ -118,6 +136,10 @@ size_t conv1d_dw_packed_workspace_bytes(int64_t N, int64_t C, int K);
 cudaError_t conv1d_dw_packed_launch(const DwArgs &a, const int32_t *offsets, cudaStream_t s);
 // dx and dW/dbias in one pass over dy; cudaErrorNotSupported when no fused instance fits.
 cudaError_t conv1d_bwd_fused_launch(const DwArgs &a, cudaStream_t s);
+// dW / dbias = partial rows [Gp][K+1][C] (slots 0..K-1 the taps, slot K the bias) summed in a
+// fixed order; launched programmatically after the kernel that wrote them.
+cudaError_t launch_finalize_rows(const float *partials, float *dw, float *dbias, int Gp, int K, int64_t C,
+                                 cudaStream_t s);
 unsigned int conv1d_dw_take_error();
 
 cudaError_t conv1d_stream_launch(const StreamArgs &a, cudaStream_t s);
