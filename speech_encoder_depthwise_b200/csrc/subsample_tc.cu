@@ -190,10 +190,9 @@ template <> __device__ __forceinline__ void stage_out<float>(float *p, float v) 
 template <> __device__ __forceinline__ void stage_out<bf16>(bf16 *p, float v) { *p = __float2bfloat16_rn(v); }
 template <> __device__ __forceinline__ void stage_out<f16>(f16 *p, float v) { *p = __float2half_rn(v); }
 
-// ReLU of two accumulator values as a pair.  The doubled form x + |x| = 2 ReLU(x) runs on the
-// FMA pipe instead of the (half-rate) ALU pipe; its weights are halved, so products are equal.
+// ReLU of two accumulator values as a pair, as fmaxf on the ALU pipe: the FMA pipe is the busier
+// one here (conv_dw1's packed FMAs), so a ReLU there (x + |x| with halved weights) is slower.
 __device__ __forceinline__ float2 relu_pair(float a, float b) { return make_float2(fmaxf(a, 0.f), fmaxf(b, 0.f)); }
-__device__ __forceinline__ float2 relu2x_pair(float a, float b) { return make_float2(a + fabsf(a), b + fabsf(b)); }
 
 }  // namespace
 
@@ -479,13 +478,13 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
         const int m = qw * 32 + lane;                     // channel within the tile = TMEM lane
         const int ct = CTG == 2 ? grp : 0;
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + grp * kTmemBuf;
-        // conv_dw1 taps as pairs; odd h columns arrive doubled (x + |x|), so W[p][1] is halved
+        // conv_dw1 taps as pairs
         float2 W[3][3], bias;
         {
             const float *wt = wtab + ct * 1280 + m;
 #pragma unroll
             for (int t = 0; t < 9; ++t) {
-                const float x = wt[t * 128] * (t % 3 == 1 ? 0.5f : 1.f);
+                const float x = wt[t * 128];
                 W[t / 3][t % 3] = make_float2(x, x);
             }
             bias = make_float2(wt[9 * 128], wt[9 * 128]);
@@ -537,11 +536,11 @@ dw_subsample_tc_kernel(const float *__restrict__ mel, const float *__restrict__ 
                     for (int jj = 0; jj < kChunk; ++jj)
                         acc[jj] = ffma2(E[jj][p], W[p][0], p == 0 ? bias : acc[jj]);
 #pragma unroll
-                for (int jj = 0; jj < kChunk; ++jj) {  // odd h column 2 jj + 1: doubled ReLU on the FMA pipe
+                for (int jj = 0; jj < kChunk; ++jj) {  // odd h column 2 jj + 1
                     const float *x = v + (2 * jj) * kHR;
-                    acc[jj] = ffma2(relu2x_pair(x[0], x[2]), W[0][1], acc[jj]);
-                    acc[jj] = ffma2(relu2x_pair(x[1], x[3]), W[1][1], acc[jj]);
-                    acc[jj] = ffma2(relu2x_pair(x[2], x[4]), W[2][1], acc[jj]);
+                    acc[jj] = ffma2(relu_pair(x[0], x[2]), W[0][1], acc[jj]);
+                    acc[jj] = ffma2(relu_pair(x[1], x[3]), W[1][1], acc[jj]);
+                    acc[jj] = ffma2(relu_pair(x[2], x[4]), W[2][1], acc[jj]);
                 }
 #pragma unroll
                 for (int p = 0; p < 3; ++p)
