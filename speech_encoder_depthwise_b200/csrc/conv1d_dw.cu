@@ -747,34 +747,39 @@ conv1d_dw_span_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_con
             p += n;
         }
     }
-    // every warp has left the pipeline; the stage memory now holds the block's sums
+    // every warp has left the pipeline; the stage memory now holds the block's sums, as channel
+    // pairs (V is even here: 2 or 4 channels a thread)
+    static_assert(V % 2 == 0, "pairs of channels");
     __syncthreads();
-    const int E = (KB + 1) * S::CT;
-    float *red = reinterpret_cast<float *>(stages);
+    const int E2 = (KB + 1) * S::CT / 2;
+    float2 *red = reinterpret_cast<float2 *>(stages);
     if (warp > 0) {
-        float *mine = red + static_cast<size_t>(warp - 1) * E;
+        float2 *mine = red + static_cast<size_t>(warp - 1) * E2;
 #pragma unroll
         for (int k = 0; k <= KB; ++k) {
 #pragma unroll
-            for (int q = 0; q < NP; ++q) {
-                const float2 v = (k < KB) ? acc[k][q] : accb[q];
-                if (2 * q < V) mine[k * S::CT + lane * V + 2 * q] = v.x;
-                if (2 * q + 1 < V) mine[k * S::CT + lane * V + 2 * q + 1] = v.y;
-            }
+            for (int q = 0; q < NP; ++q) mine[(k * S::CT + lane * V) / 2 + q] = (k < KB) ? acc[k][q] : accb[q];
         }
     }
     __syncthreads();
-    for (int e = static_cast<int>(threadIdx.x); e < E; e += static_cast<int>(blockDim.x)) {
-        float sum = red[e];
-        for (int r = 1; r < S::CONS; ++r) sum += red[static_cast<size_t>(r) * E + e];
-        const int kk = e / S::CT;
-        const int64_t c = static_cast<int64_t>(c0) + (e % S::CT);
-        if (c >= C) continue;
-        if (kk == KB) {
-            if (with_bias) partials[(static_cast<int64_t>(jj) * (K + 1) + K) * C + c] = sum;
-        } else if (k_off + kk < K) {
-            partials[(static_cast<int64_t>(jj) * (K + 1) + k_off + kk) * C + c] = sum;
+    for (int e = static_cast<int>(threadIdx.x); e < E2; e += static_cast<int>(blockDim.x)) {
+        float2 sum = red[e];
+#pragma unroll
+        for (int r = 1; r < S::CONS; ++r) {
+            const float2 t = red[static_cast<size_t>(r) * E2 + e];
+            sum.x += t.x;
+            sum.y += t.y;
         }
+        const int kk = (2 * e) / S::CT;
+        const int64_t c = static_cast<int64_t>(c0) + (2 * e) % S::CT;  // even; C is even on this path
+        if (c >= C) continue;
+        float *row = nullptr;
+        if (kk == KB) {
+            if (with_bias) row = partials + (static_cast<int64_t>(jj) * (K + 1) + K) * C;
+        } else if (k_off + kk < K) {
+            row = partials + (static_cast<int64_t>(jj) * (K + 1) + k_off + kk) * C;
+        }
+        if (row != nullptr) *reinterpret_cast<float2 *>(row + c) = sum;
     }
 }
 

@@ -64,6 +64,8 @@ conv1d_stream_kernel(const T *__restrict__ x, const float *__restrict__ w, const
                      int nCV, int S, int nSeg) {
     constexpr int H = K - 1;
     constexpr int P = Pairs<V>::n;
+    launch_dependents();     // the next chunk's kernel may start its own set-up
+    grid_dependency_wait();  // launched programmatically: the previous chunk's cache writes are visible after this
     StreamIdx r;
     if (!stream_idx(B, Tn, nCV, V, S, nSeg, r)) return;
     const int c = r.c;
@@ -134,6 +136,8 @@ conv1d_stream_anyk_kernel(const T *__restrict__ x, const float *__restrict__ w, 
                           int K, int nCV, int S, int nSeg) {
     constexpr int P = Pairs<V>::n;
     const int H = K - 1;
+    launch_dependents();     // the next chunk's kernel may start its own set-up
+    grid_dependency_wait();  // launched programmatically: the previous chunk's cache writes are visible after this
     StreamIdx r;
     if (!stream_idx(B, Tn, nCV, V, S, nSeg, r)) return;
     const int c = r.c;
@@ -191,20 +195,19 @@ cudaError_t launch_stream(const StreamArgs &a, cudaStream_t s) {
     const T *x = static_cast<const T *>(a.x);
     T *y = static_cast<T *>(a.y), *cache = static_cast<T *>(a.cache);
     const int B = static_cast<int>(a.B), Tn = static_cast<int>(a.T), C = static_cast<int>(a.C);
+    const dim3 g3(static_cast<unsigned>(grid)), b3(kStreamThreads);
 #define DW_STREAM_K(KK)                                                                                   \
     case KK:                                                                                              \
-        conv1d_stream_kernel<T, V, KK><<<static_cast<unsigned>(grid), kStreamThreads, 0, s>>>(            \
-            x, a.w, a.bias, y, cache, a.lengths, B, Tn, C, nCV, S, nSeg);                                 \
-        break;
+        return launch_programmatic(conv1d_stream_kernel<T, V, KK>, g3, b3, 0, s, x, a.w, a.bias, y, cache, \
+                                   a.lengths, B, Tn, C, nCV, S, nSeg);
     switch (a.K) {
         DW_STREAM_K(1) DW_STREAM_K(2) DW_STREAM_K(3) DW_STREAM_K(4) DW_STREAM_K(5) DW_STREAM_K(7)
         DW_STREAM_K(9) DW_STREAM_K(15)
         default:
-            conv1d_stream_anyk_kernel<T, V><<<static_cast<unsigned>(grid), kStreamThreads, 0, s>>>(
-                x, a.w, a.bias, y, cache, a.lengths, B, Tn, C, a.K, nCV, S, nSeg);
+            return launch_programmatic(conv1d_stream_anyk_kernel<T, V>, g3, b3, 0, s, x, a.w, a.bias, y, cache,
+                                       a.lengths, B, Tn, C, a.K, nCV, S, nSeg);
     }
 #undef DW_STREAM_K
-    return cudaGetLastError();
 }
 
 }  // namespace

@@ -148,6 +148,8 @@ dw_subsample_kernel(const float *__restrict__ mel, const float *__restrict__ w0,
     lin /= nJB;
     const int rc = lin % nRC;
     const int b = lin / nRC;
+    launch_dependents();     // the next kernel in the stream may start its own set-up
+    grid_dependency_wait();  // launched programmatically: the previous kernel's writes are visible after this
 
     if (blockIdx.x == 0 && out_lengths != nullptr) {
         for (int q = threadIdx.x; q < B; q += blockDim.x) {
@@ -368,23 +370,21 @@ cudaError_t subsample_launch(const SubsampleArgs &a, bool tensor_cores, cudaStre
     const bool vec = (a.C % vch) == 0 &&
                      (reinterpret_cast<uintptr_t>(a.out) % (static_cast<uintptr_t>(vch) * dtype_bytes(a.out_dtype))) == 0;
 #define DW_SUB_LAUNCH(TO, VS)                                                                           \
-    dw_subsample_kernel<TO, VS, kSubJ, kSubRI, kSubNPR><<<static_cast<unsigned>(grid), warps * 32, 0, s>>>(          \
-        a.mel, a.w0, a.b0, a.w1, a.b1, static_cast<TO *>(a.out), a.lengths, a.out_lengths,                   \
+    return launch_programmatic(dw_subsample_kernel<TO, VS, kSubJ, kSubRI, kSubNPR>, dim3(static_cast<unsigned>(grid)), \
+        dim3(warps * 32), 0, s, a.mel, a.w0, a.b0, a.w1, a.b1, static_cast<TO *>(a.out), a.lengths, a.out_lengths, \
         static_cast<int>(a.B), static_cast<int>(a.T), static_cast<int>(a.F), static_cast<int>(a.C),           \
         static_cast<int>(T2), static_cast<int>(F2), static_cast<int>(T4), static_cast<int>(F4), Pt,          \
         static_cast<int>(nCG), static_cast<int>(nJB), static_cast<int>(nRC))
     if (a.out_dtype == 1) {
         if (vec) DW_SUB_LAUNCH(bf16, true);
-        else DW_SUB_LAUNCH(bf16, false);
+        DW_SUB_LAUNCH(bf16, false);
     } else if (a.out_dtype == 2) {
         if (vec) DW_SUB_LAUNCH(f16, true);
-        else DW_SUB_LAUNCH(f16, false);
-    } else {
-        if (vec) DW_SUB_LAUNCH(float, true);
-        else DW_SUB_LAUNCH(float, false);
+        DW_SUB_LAUNCH(f16, false);
     }
+    if (vec) DW_SUB_LAUNCH(float, true);
+    DW_SUB_LAUNCH(float, false);
 #undef DW_SUB_LAUNCH
-    return cudaGetLastError();
 }
 
 __global__ void dw_out_lengths_kernel(const int32_t *__restrict__ lengths, int32_t *__restrict__ out_lengths,

@@ -259,6 +259,66 @@ dw_subsample_bwd_finalize_kernel(const float *__restrict__ partials, int G, int 
     }
 }
 
+// The same sum for 16-byte aligned partials and at most kSbMaxRows4 rows: a block covers 64
+// consecutive entries (16 lanes x float4) with 16 row groups; group r loads rows r, r+16, ... (all
+// of its loads issued before the first add) and adds them in order, then the 16 group sums are
+// added in a fixed tree.  Launched programmatically after the partial kernel.
+constexpr int kSbFinGroups = 16, kSbMaxRows4 = 256;
+__global__ void __launch_bounds__(256)
+dw_subsample_bwd_finalize4_kernel(const float *__restrict__ partials, int G, int C, float *__restrict__ dw0,
+                                  float *__restrict__ db0, float *__restrict__ dw1, float *__restrict__ db1) {
+    __shared__ float4 red[kSbFinGroups][16];
+    launch_dependents();     // the next kernel may start its own set-up
+    grid_dependency_wait();  // the partial rows are complete and visible after this
+    const int lane = threadIdx.x % 16, rg = threadIdx.x / 16;
+    const int64_t E4 = static_cast<int64_t>(kSbSlots) * C / 4;
+    const int64_t e4 = static_cast<int64_t>(blockIdx.x) * 16 + lane;
+    const float4 *p4 = reinterpret_cast<const float4 *>(partials);
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e4 < E4) {
+        float4 v[kSbMaxRows4 / kSbFinGroups];
+#pragma unroll
+        for (int i = 0; i < kSbMaxRows4 / kSbFinGroups; ++i) {
+            const int r = rg + i * kSbFinGroups;
+            v[i] = r < G ? __ldg(p4 + static_cast<int64_t>(r) * E4 + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < kSbMaxRows4 / kSbFinGroups; ++i) {
+            s.x += v[i].x;
+            s.y += v[i].y;
+            s.z += v[i].z;
+            s.w += v[i].w;
+        }
+    }
+    red[rg][lane] = s;
+    __syncthreads();
+    if (rg == 0 && e4 < E4) {
+        float4 t[kSbFinGroups];
+#pragma unroll
+        for (int r = 0; r < kSbFinGroups; ++r) t[r] = red[r][lane];
+#pragma unroll
+        for (int w = 1; w < kSbFinGroups; w <<= 1) {
+#pragma unroll
+            for (int r = 0; r + w < kSbFinGroups; r += 2 * w) {
+                t[r].x += t[r + w].x;
+                t[r].y += t[r + w].y;
+                t[r].z += t[r + w].z;
+                t[r].w += t[r + w].w;
+            }
+        }
+        const float o[4] = {t[0].x, t[0].y, t[0].z, t[0].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t e = 4 * e4 + q;
+            const int slot = static_cast<int>(e / C), c = static_cast<int>(e % C);
+            if (slot < 9) dw0[slot * C + c] = o[q];
+            else if (slot == 9) db0[c] = o[q];
+            else if (slot < 19) dw1[(slot - 10) * C + c] = o[q];
+            else db1[c] = o[q];
+        }
+    }
+}
+
 __global__ void dw_subsample_bwd_zero_kernel(float *dw0, float *db0, float *dw1, float *db1, int C) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e < 9 * C) {
@@ -299,6 +359,10 @@ cudaError_t subsample_bwd_launch(const SubsampleBwdArgs &a, cudaStream_t s) {
         int rows = 0;
         const cudaError_t et = subsample_bwd_tc_launch(a, subsample_bwd_partial_rows(a.B, a.T, a.F), &rows, s);
         if (et == cudaSuccess) {
+            if (rows <= kSbMaxRows4 && reinterpret_cast<uintptr_t>(a.partials) % 16 == 0)
+                return launch_programmatic(dw_subsample_bwd_finalize4_kernel, dim3(static_cast<unsigned>((E / 4 + 15) / 16)),
+                                           dim3(256), 0, s, static_cast<const float *>(a.partials), rows,
+                                           static_cast<int>(a.C), a.dw0, a.db0, a.dw1, a.db1);
             dw_subsample_bwd_finalize_kernel<<<static_cast<unsigned>((E + 31) / 32), 256, 0, s>>>(
                 a.partials, rows, static_cast<int>(a.C), a.dw0, a.db0, a.dw1, a.db1);
             return cudaGetLastError();

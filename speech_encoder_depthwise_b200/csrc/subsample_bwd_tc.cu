@@ -205,6 +205,7 @@ dw_subsample_bwd_tc_kernel(const float *__restrict__ mel, const float *__restric
     const int perItem = nRB * nCB, nUnits = B * perItem;
 
     // ------------------------------------------------------------ set-up
+    launch_dependents();  // the finalize may be scheduled now; it waits for this grid to finish
     if (threadIdx.x == 0) {
         mbar_init(b1_full, kBuildThreads);
         mbar_init(b1_empty, 1);
