@@ -8,6 +8,14 @@
  *    allocates nothing, never synchronizes, and enqueues its kernels on `stream`
  *    (a cudaStream_t; NULL means the legacy default stream).  Results are ready when the
  *    stream reaches them.
+ *  - Stream order: the kernels are launched with programmatic stream serialization, so one
+ *    may start while the previous kernel in the stream drains.  Until that kernel has
+ *    completed it only initialises its own shared memory and warms L2 with prefetches, then
+ *    it waits for it (griddepcontrol.wait) before its first read: inputs written by earlier
+ *    work in the stream, lengths included, are always seen.  Each kernel also lets the next
+ *    one start early.  A caller's kernel launched normally after a call waits for the call to
+ *    complete as usual; one launched with programmatic serialization must itself wait
+ *    (cudaGridDependencySynchronize) before it reads the call's outputs.
  *  - Layout: activations are channels-last and C-contiguous: x[B][T][C] (C fastest).
  *    Weights and biases are float32: w[K][C], bias[C], w0/w1[3][3][C] (C fastest).  A
  *    PyTorch depthwise weight [C][1][K] is the transpose of w.
